@@ -1,0 +1,385 @@
+"""Benchmark of the SRU layer training step on B200.
+
+One step = one pass of the whole hot path over one batch: the projection
+U = X W_cat^T (tcgen05 GEMM), the forward recurrence, the backward recurrence
+(+ the dv/db reduction), and the projection gradients dX += dU W_cat and
+dW_cat = dU^T X.  Workload: the language-model training layer, L = 1024,
+B = 16 tokens-per-step rows, d = 2048, bf16 projection and fp32 recurrence
+(seeded synthetic inputs; no dataset).
+
+Prints ONE JSON line (rank 0).  `value` is device-timed throughput (tokens/s)
+with inputs resident in HBM; `e2e` is the same step through the same C-ABI
+calls with the per-step inputs copied from pinned host memory and the
+gradients copied back inside the timed region.
+
+--impl reference times the fp64 CPU oracle (the baseline this build is
+checked against) on the host cores, on a bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SRU fwd+bwd tokens/s and recurrence HBM GB/s (% of peak) on 1 B200"
+WORKLOAD = "lm_train"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            pk = json.load(fh)
+        return dict(hbm_gbs=float(pk["hbm_gbs"]), bf16_tflops=float(pk["bf16_tflops"]),
+                    bf16_tflops_sustained=float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def workload_config():
+    from synthetic import CONFIGS
+    cfg = CONFIGS[WORKLOAD]
+    return cfg, {"workload": f"{cfg.name}: SRU layer training step L={cfg.L} B={cfg.B} d={cfg.d} "
+                             f"unidirectional, bf16 projection, fp32 recurrence",
+                 "L": cfg.L, "B_per_gpu": cfg.B, "d": cfg.d, "tokens_per_step_per_gpu": cfg.tokens,
+                 "l2": "inputs larger than L2 (step working set ~1.3 GB vs 126 MB L2); no flush"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as fh:
+                for line in fh:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        finally:
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "", 1).isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "", 1).isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------- CPU baseline
+def cpu_baseline(cfg, budget_s: float = 10.0, seed: int = 0):
+    """Time the fp64 oracle on a bounded sample of the workload on one host core
+    and extrapolate to the full step (projection, its two gradients, forward and
+    backward recurrence over every channel).  Returns (tokens/s, description)."""
+    import oracle
+    from synthetic import f32_to_bf16_bits
+    rng = np.random.default_rng(seed)
+    L, B, d = cfg.L, cfg.B, cfg.d
+    M, N, K = L * B, cfg.N, d
+    # recurrence: every batch row of n_ch channels, all L steps
+    n_ch = 8
+    U = rng.standard_normal((L, B, 1, 3, n_ch))
+    x = rng.standard_normal((L, B, n_ch))
+    v = rng.uniform(-0.5, 0.5, (1, 2, n_ch))
+    bias = 0.1 * rng.standard_normal((1, 2, n_ch))
+    dh = rng.standard_normal((L, B, 1, n_ch))
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.forward(U, x, v, bias)
+        oracle.backward(U, x, v, bias, dh)
+        reps += 1
+        if time.perf_counter() - t0 > budget_s * 0.3:
+            break
+    t_rec = (time.perf_counter() - t0) / (reps * B * n_ch)          # s per channel (fwd + bwd)
+    # projection and gradients: entries of each product, each a K_red-long plain sum
+    Xb = f32_to_bf16_bits(rng.standard_normal((512, K)).astype(np.float32))
+    Wb = f32_to_bf16_bits(rng.standard_normal((512, K)).astype(np.float32))
+    rows = rng.integers(0, 512, 64)
+    cols = rng.integers(0, 512, 64)
+    t0 = time.perf_counter()
+    n_ent = 0
+    while True:
+        oracle.project_entries(Xb, Wb, rows, cols)
+        n_ent += rows.size
+        if time.perf_counter() - t0 > budget_s * 0.7:
+            break
+    t_mac = (time.perf_counter() - t0) / (n_ent * K)                # s per multiply-add
+    full = t_rec * B * d * cfg.n_dir + t_mac * 3 * M * N * K
+    desc = (f"fp64 oracle, 1 thread: recurrence fwd+bwd on {n_ch} channels x {B} rows x L={L} "
+            f"({reps} reps), projection plain sums {n_ent} entries x K={K}; extrapolated to the full step "
+            f"({B * d * cfg.n_dir} channels, 3 products of {M}x{N}x{K})")
+    return cfg.tokens / full, desc, full
+
+
+# ------------------------------------------------------------ GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import parallelizable_recurrence_b200 as sru
+    from synthetic import generate
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    sru.load_library()
+    peaks = load_peaks()
+    cfg, config = workload_config()
+    cfg = cfg.replace(seed=cfg.seed + 100 * rank)      # each rank its own batch (data parallel)
+    inp = generate(cfg)
+    L, B, d = cfg.L, cfg.B, cfg.d
+    M, N, K = L * B, cfg.N, d
+
+    def bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    def f32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+
+    X, W = bf16(inp["X"]), bf16(inp["W"])
+    x, v, b, c0, dh = f32(inp["x"]), f32(inp["v"]), f32(inp["bias"]), f32(inp["c0"]), f32(inp["dh"])
+    U = torch.empty(L, B, 1, 3, d, device=dev, dtype=torch.bfloat16)
+    h = torch.empty(L, B, 1, d, device=dev)
+    cT = torch.empty(B, 1, d, device=dev)
+    ws = sru.alloc_workspace(L, B, d, False, device=dev)
+    dU = torch.empty_like(U)
+    dx = torch.empty(L, B, d, device=dev)
+    dv = torch.empty(1, 2, d, device=dev)
+    db = torch.empty(1, 2, d, device=dev)
+    dc0 = torch.empty(B, 1, d, device=dev)
+    dW = torch.empty(N, K, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    grads = torch.empty(N * K + 4 * d, device=dev) if world > 1 else None
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sru.sru_project(X, W, U)
+        if ev is not None:
+            ev[1].record(stream)
+        sru.sru_forward(U, x, v, b, h, cT, c0=c0, workspace=ws)
+        if ev is not None:
+            ev[2].record(stream)
+        sru.sru_backward(U, x, v, b, dh, ws, dU, dx, dv, db, dc0, c0=c0)
+        if ev is not None:
+            ev[3].record(stream)
+        sru.sru_project_backward(dU, X, W, dX=dx, accumulate=True)
+        if ev is not None:
+            ev[4].record(stream)
+        sru.sru_project_backward(dU, X, W, dW=dW)
+        if ev is not None:
+            ev[5].record(stream)
+        if world > 1:  # data-parallel gradient sum (the pages' DDP)
+            grads[:N * K].copy_(dW.view(-1))
+            grads[N * K:N * K + 2 * d].copy_(dv.view(-1))
+            grads[N * K + 2 * d:].copy_(db.view(-1))
+            dist.all_reduce(grads)
+
+    for _ in range(args.warmup):
+        step()
+    st = sru.sru_sync_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    # ---- device-timed region
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    clocks = clk.summary()
+    st = sru.sru_sync_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} in the timed region")
+    names = ["project", "forward", "backward", "project_dX", "project_dW"]
+    phase_ms = {n: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
+                for i, n in enumerate(names)}
+    t = torch.tensor([elapsed_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t.item())
+
+    # ---- end to end: per-step inputs from pinned host memory, gradients back
+    hX = torch.from_numpy(np.ascontiguousarray(inp["X"]).view(np.int16)).pin_memory()
+    hx = torch.from_numpy(inp["x"]).pin_memory()
+    hdh = torch.from_numpy(inp["dh"]).pin_memory()
+    out_dW = torch.empty(N, K).pin_memory()
+    out_small = torch.empty(4 * d + B * d).pin_memory()
+    small = torch.empty(4 * d + B * d, device=dev)
+    Xi = X.view(torch.int16)
+
+    def e2e_step():
+        Xi.copy_(hX, non_blocking=True)
+        x.copy_(hx, non_blocking=True)
+        dh.copy_(hdh, non_blocking=True)
+        step()
+        small[:2 * d].copy_(dv.view(-1))
+        small[2 * d:4 * d].copy_(db.view(-1))
+        small[4 * d:].copy_(dc0.view(-1))
+        out_dW.copy_(dW, non_blocking=True)
+        out_small.copy_(small, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    t = torch.tensor([e2e_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.barrier()
+    e2e_ms = float(t.item())
+    h2d = hX.numel() * 2 + hx.numel() * 4 + hdh.numel() * 4
+    d2h = out_dW.numel() * 4 + out_small.numel() * 4
+
+    if rank == 0:
+        tokens = cfg.tokens * world * args.steps
+        value = tokens / (elapsed_ms / 1e3)
+        gemm_flops = 2.0 * M * N * K
+        gemm_ms = {n: phase_ms[n] for n in ("project", "project_dX", "project_dW")}
+        dom = max(gemm_ms, key=gemm_ms.get)
+        peak_tc = peaks["bf16_tflops_sustained"]
+        ach_tc = gemm_flops / (gemm_ms[dom] / 1e3) / 1e12
+        fwd_bytes = 14.0 * L * B * d
+        bwd_bytes = 24.0 * L * B * d
+        ach_f = fwd_bytes / (phase_ms["forward"] / 1e3) / 1e9
+        ach_b = bwd_bytes / (phase_ms["backward"] / 1e3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 GEMM + f32 recurrence",
+            "data": "synthetic", "config": config,
+            "roofline": {"bound": "tensor", "kernel": f"tc_gemm ({dom})", "achieved": ach_tc, "peak": peak_tc,
+                         "unit": "TFLOP/s", "frac": ach_tc / peak_tc, "traffic": None,
+                         "peak_source": f"{peaks['source']} bf16 sustained (kernel inside a long step)",
+                         "algorithmic_per_launch": f"2*M*N*K = {gemm_flops:.4g} flop"},
+            "roofline_recurrence": {
+                "bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                "forward": {"achieved": ach_f, "frac": ach_f / peaks["hbm_gbs"], "bytes": fwd_bytes,
+                            "ms": phase_ms["forward"]},
+                "backward": {"achieved": ach_b, "frac": ach_b / peaks["hbm_gbs"], "bytes": bwd_bytes,
+                             "ms": phase_ms["backward"]},
+                "frac_of_nominal_8TBs": {"forward": ach_f / 8000.0, "backward": ach_b / 8000.0}},
+            "phase_ms": phase_ms,
+            "e2e": {"value": cfg.tokens * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 6 * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1:
+            cpu_tps, desc, _ = cpu_baseline(cfg, budget_s=args.cpu_budget)
+            line["cpu_baseline"] = {"value": cpu_tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                    "sample": desc}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores, same workload/metric; rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    cfg, config = workload_config()
+    per_step = []
+    desc = ""
+    for k in range(args.warmup + args.steps):
+        tps, desc, full = cpu_baseline(cfg, budget_s=args.ref_step_budget, seed=k)
+        if k >= args.warmup:
+            per_step.append(full)
+    full_s = statistics.mean(per_step)
+    value = cfg.tokens / full_s
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": full_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-step-budget", type=float, default=2.0, help="seconds of oracle work per reference step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,152 @@
+/*
+ * sru.h -- C ABI of the B200 (sm_100a) Simple Recurrent Unit layer library (libsru.so).
+ *
+ * The layer is the SRU cell of "When Attention Meets Fast Recurrence: Training
+ * Language Models with Reduced Compute" (T. Lei), background section on SRU:
+ *
+ *   Eq. (1)      U^T = [W; W'; W''] X^T        one product over all L time steps
+ *   Eqs. (2)-(5) f[t] = sigma(U[t,f] + v_f * c[t-1] + b_f)
+ *                r[t] = sigma(U[t,r] + v_r * c[t-1] + b_r)
+ *                c[t] = f[t] * c[t-1] + (1 - f[t]) * U[t,c]
+ *                h[t] = r[t] * c[t] + (1 - r[t]) * alpha * x[t]
+ *
+ * computed independently for every hidden channel j and batch row b.  The
+ * backward pass (not printed on the page) is the reverse-mode derivative of
+ * those equations, walked in reverse time.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Layouts are time-major and row-major (last index fastest):
+ *   X, x     (L, B, d)              layer input; X in the projection's type, x fp32
+ *   W_cat    (n_dir * 3 * d, d)     rows [dir][gate][j]; gate 0 = candidate (W),
+ *                                    1 = forget (W_f), 2 = reset (W_r)
+ *   U        (L, B, n_dir, 3, d)    = (M, N) with M = L*B, N = n_dir*3*d
+ *   h, dh    (L, B, n_dir, d)       fp32
+ *   v, b     (n_dir, 2, d)          fp32; row 0 = forget gate, row 1 = reset gate
+ *   c0, c_T  (B, n_dir, d)          fp32
+ *   mask     (L, B) uint8           1 = padded position (nullable = no padding)
+ * n_dir = 2 when `bidirectional`: direction 1 walks t = L-1 ... 0 with its own
+ * gate block of U, v, b and c0; both directions read the same x.
+ * A padded position leaves the state unchanged, writes h = 0, and gets zero
+ * gradient (dU = 0, no dx contribution); the state gradient passes through it.
+ *
+ * Pointers: every data pointer is a DEVICE pointer owned by the caller, at
+ * least 16-byte aligned, to densely packed memory of the stated layout.
+ * The library allocates no device memory.  `stream` is a cudaStream_t (NULL =
+ * legacy default stream); calls are stream-ordered and asynchronous (none
+ * synchronises).  Size limits: d % 8 == 0, 1 <= d, 0 <= L, 0 <= B, L*B < 2^31.
+ *
+ * Errors: every call returns an sru_status.  Invalid arguments are rejected
+ * before anything is launched (SRU_ERR_INVALID / SRU_ERR_UNSUPPORTED).  A
+ * failed launch returns SRU_ERR_CUDA (see sru_get_last_cuda_error).  Every
+ * wait inside a kernel is bounded (2 s); if one expires the kernel records a
+ * code in a device error word and returns early, and the next
+ * sru_sync_status() on that device returns SRU_ERR_TIMEOUT.  Nothing aborts,
+ * traps or exits.
+ */
+#ifndef SRU_B200_H
+#define SRU_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SRU_OK = 0,
+    SRU_ERR_INVALID = 1,      /* bad pointer, size, alignment or dtype */
+    SRU_ERR_CUDA = 2,         /* a CUDA runtime/driver call failed */
+    SRU_ERR_TIMEOUT = 3,      /* a bounded device-side wait expired */
+    SRU_ERR_UNSUPPORTED = 4   /* valid request this build does not implement */
+} sru_status;
+
+typedef enum { SRU_F32 = 0, SRU_BF16 = 1 } sru_dtype;
+
+/* Caller asserts v == 0 (all entries): the recurrence is then linear in c and
+ * may run as a chunked associative scan over t (sru_forward / sru_backward). */
+#define SRU_FLAG_V_ZERO 0x1u
+/* With SRU_FLAG_V_ZERO: force the scan path / force the sequential path. */
+#define SRU_FLAG_FORCE_SCAN 0x2u
+#define SRU_FLAG_FORCE_SEQUENTIAL 0x4u
+
+/* Human-readable name of a status code (static string). */
+const char* sru_status_string(int status);
+
+/* The cudaError_t of the most recent SRU_ERR_CUDA on the calling thread (0 if none). */
+int sru_get_last_cuda_error(void);
+
+/* Library ABI version (major * 100 + minor). */
+int sru_version(void);
+
+/*
+ * Bytes of caller-provided device workspace that sru_forward and sru_backward
+ * need for a layer of these sizes and flags.  The workspace carries state
+ * checkpoints from sru_forward to sru_backward (pass the same buffer to both)
+ * and holds the backward's per-row partial sums.  Returns 0 on bad sizes.
+ */
+size_t sru_workspace_bytes(int64_t L, int64_t B, int64_t d, int bidirectional, unsigned flags);
+
+/*
+ * Eq. (1): U[M, N] = X[M, K] * W[N, K]^T, fp32 accumulation.
+ *   M = L*B tokens, K = d, N = n_dir*3*d.  Supported type triples (x_t, w_t, u_t):
+ *   (BF16, BF16, BF16) and (BF16, BF16, F32) on the tcgen05 tensor cores;
+ *   (F32, F32, F32) on a CUDA-core kernel.  Requires K % 8 == 0, N % 8 == 0.
+ */
+sru_status sru_project(const void* X, int x_t, const void* W, int w_t, void* U, int u_t,
+                       int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * Gradients of Eq. (1), fp32 accumulation, fp32 outputs:
+ *   dX[M, K] = dU[M, N] * W[N, K]      (accumulate != 0: dX += ..., e.g. onto the
+ *                                       highway part returned by sru_backward)
+ *   dW[N, K] = dU[M, N]^T * X[M, K]
+ * dU, X and W share one type t (BF16 on the tensor cores, F32 on CUDA cores).
+ * Either output may be NULL to skip it.  Requires K % 8 == 0, N % 8 == 0.
+ */
+sru_status sru_project_backward(const void* dU, const void* X, const void* W, int t,
+                                float* dX, int accumulate, float* dW,
+                                int64_t M, int64_t N, int64_t K, void* stream);
+
+/*
+ * Eqs. (2)-(5) over all t for every (direction, batch row, channel).
+ *   U (u_t = F32 or BF16), x, v, b as above; c0 nullable (zero state);
+ *   mask nullable.  Outputs h (L, B, n_dir, d) and c_T (B, n_dir, d), fp32.
+ *   workspace: sru_workspace_bytes(...) bytes, or NULL for inference only
+ *   (then no checkpoints are written and sru_backward cannot follow).
+ *   flags: SRU_FLAG_* above.
+ */
+sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, const float* b,
+                       const float* c0, const uint8_t* mask, int64_t L, int64_t B, int64_t d,
+                       float alpha, int bidirectional, unsigned flags,
+                       float* h, float* c_T, void* workspace, void* stream);
+
+/*
+ * Backward of sru_forward for Loss = sum(dh * h) + sum(dc_T * c_T).
+ * Inputs: the forward's U, x, v, b, c0, mask, sizes, alpha, flags and the
+ *   workspace the forward filled; dh (L, B, n_dir, d); dc_T nullable (zero).
+ * Outputs (overwritten):
+ *   dU (L, B, n_dir, 3, d) of type du_t (F32 or BF16),
+ *   dx (L, B, d) fp32: the highway part alpha * (1 - r) * dh, summed over directions
+ *      (add the projection part with sru_project_backward(..., accumulate = 1)),
+ *   dv, db (n_dir, 2, d) fp32 summed over t and b (deterministic order),
+ *   dc0 (B, n_dir, d) fp32.
+ */
+sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, const float* b,
+                        const float* c0, const uint8_t* mask, int64_t L, int64_t B, int64_t d,
+                        float alpha, int bidirectional, unsigned flags,
+                        const float* dh, const float* dc_T, void* workspace,
+                        void* dU, int du_t, float* dx, float* dv, float* db, float* dc0,
+                        void* stream);
+
+/* Synchronise `stream`, then read and clear the device error word of the
+ * current device: SRU_ERR_TIMEOUT if a bounded wait expired since the last
+ * call, SRU_ERR_CUDA if the stream reported an error, else SRU_OK. */
+sru_status sru_sync_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SRU_B200_H */

@@ -1,0 +1,427 @@
+// sru_api.cu -- the C ABI of libsru.so (declared in include/sru.h): argument
+// validation, TMA tensor-map construction and kernel dispatch.  The library is
+// built as this single translation unit so the device error word has one
+// definition; the kernels live in the included .cuh files.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/sru.h"
+#include "sru_gemm.cuh"
+#include "sru_recurrence.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+sru_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error = (int)e;
+    return SRU_ERR_CUDA;
+}
+
+#define SRU_CUDA_TRY(expr)                          \
+    do {                                            \
+        cudaError_t e_ = (expr);                    \
+        if (e_ != cudaSuccess) return cuda_fail(e_); \
+    } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------- tensor maps
+using EncodeTiledFn = decltype(&cuTensorMapEncodeTiled);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// rank-R tiled map; dims/box innermost first; strides (bytes) of dims 1..R-1
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+              const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
+                    reinterpret_cast<const cuuint64_t*>(strides), reinterpret_cast<const cuuint32_t*>(box), estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- device facts
+constexpr int kMaxDevices = 64;
+
+int sm_count() {
+    static int cache[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t ensure_smem(const void* kernel, size_t bytes) {
+    static std::mutex mu;
+    static const void* done_kernel[256];
+    static int done_dev[256];
+    static int ndone = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < ndone; ++i)
+        if (done_kernel[i] == kernel && done_dev[i] == dev) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    if (ndone < 256) {
+        done_kernel[ndone] = kernel;
+        done_dev[ndone] = dev;
+        ++ndone;
+    }
+    return cudaSuccess;
+}
+
+// ---------------------------------------------------------- workspace layout
+struct WsLayout {
+    size_t ckpt_off, ckpt_bytes, partial_off, partial_bytes, total;
+};
+
+WsLayout ws_layout(int64_t L, int64_t B, int64_t d, int n_dir) {
+    WsLayout w{};
+    const int64_t nch = (L + sru::kChunkT - 1) / sru::kChunkT;
+    w.ckpt_off = 0;
+    w.ckpt_bytes = round256((size_t)nch * B * n_dir * d * sizeof(float));
+    w.partial_off = w.ckpt_off + w.ckpt_bytes;
+    w.partial_bytes = round256((size_t)B * n_dir * 4 * d * sizeof(double));
+    w.total = w.partial_off + w.partial_bytes;
+    return w;
+}
+
+sru_status check_layer_sizes(int64_t L, int64_t B, int64_t d) {
+    if (L < 0 || B < 0 || d < 1) return SRU_ERR_INVALID;
+    if (d % 8 != 0) return SRU_ERR_UNSUPPORTED;
+    if (B > 65535 || L > (int64_t)1 << 30 || d > (int64_t)1 << 24) return SRU_ERR_UNSUPPORTED;
+    if (L * B >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
+    return SRU_OK;
+}
+
+inline unsigned blocks_for(size_t n, unsigned threads) { return (unsigned)((n + threads - 1) / threads); }
+
+// ------------------------------------------------------------- GEMM launch
+template <bool A_MN, bool B_MN, int OUT>
+sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
+                          int64_t Kr, cudaStream_t st) {
+    auto kern = sru::gemm::tc_gemm_kernel<A_MN, B_MN, OUT>;
+    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::SMEM_BYTES));
+    const int64_t tiles = ((R + sru::gemm::BM - 1) / sru::gemm::BM) * ((C + sru::gemm::BN - 1) / sru::gemm::BN);
+    const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+    kern<<<grid, sru::gemm::THREADS, sru::gemm::SMEM_BYTES, st>>>(ma, mb, out, (int)R, (int)C, (int)Kr, (int)C);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+// K-major operand (rows x K), contiguous K: box (64, box_rows)
+bool map_kmajor(CUtensorMap* m, const void* p, int64_t rows, int64_t K, uint32_t box_rows) {
+    const uint64_t dims[2] = {(uint64_t)K, (uint64_t)rows};
+    const uint64_t strides[1] = {(uint64_t)K * 2};
+    const uint32_t box[2] = {64, box_rows};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// MN-major operand: element (r, k) at p[k * ld + r], rows r contiguous: box (64, 64)
+bool map_mnmajor(CUtensorMap* m, const void* p, int64_t rows, int64_t K, int64_t ld) {
+    const uint64_t dims[2] = {(uint64_t)rows, (uint64_t)K};
+    const uint64_t strides[1] = {(uint64_t)ld * 2};
+    const uint32_t box[2] = {64, 64};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+sru_status launch_simt(const float* A, int64_t a_rs, int64_t a_ks, const float* Bm, int64_t b_rs, int64_t b_ks,
+                       float* out, int64_t R, int64_t C, int64_t K, int accumulate, cudaStream_t st) {
+    dim3 grid((unsigned)((C + sru::gemm::ST - 1) / sru::gemm::ST), (unsigned)((R + sru::gemm::ST - 1) / sru::gemm::ST));
+    if (grid.y > 65535) return SRU_ERR_UNSUPPORTED;
+    sru::gemm::simt_gemm_f32_kernel<<<grid, 256, 0, st>>>(A, a_rs, a_ks, Bm, b_rs, b_ks, out, C, (int)R, (int)C,
+                                                          (int)K, accumulate);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+sru_status zero_f32(float* p, size_t n, cudaStream_t st) {
+    if (n == 0) return SRU_OK;
+    sru::sru_fill_f32_kernel<<<blocks_for(n, 256), 256, 0, st>>>(p, n, 0.f);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+// ------------------------------------------------------- recurrence launch
+struct RecMaps {
+    CUtensorMap u, x, dh, dx;
+};
+
+bool map_u_tensor(CUtensorMap* m, const void* U, int u_t, int64_t L, int64_t B, int64_t d, int n_dir) {
+    const uint64_t es = u_t == SRU_BF16 ? 2 : 4;
+    const uint64_t dims[4] = {(uint64_t)d, 3, (uint64_t)(B * n_dir), (uint64_t)L};
+    const uint64_t strides[3] = {(uint64_t)d * es, (uint64_t)3 * d * es, (uint64_t)B * n_dir * 3 * d * es};
+    const uint32_t box[4] = {(uint32_t)sru::kRecCJ, 3, 1, (uint32_t)sru::kChunkT};
+    return make_map(m, u_t == SRU_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, U,
+                    dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+// fp32 (L, rows, d) tensor with tiles (CJ, 1, T)
+bool map_f32_rows(CUtensorMap* m, const float* p, int64_t L, int64_t rows, int64_t d) {
+    const uint64_t dims[3] = {(uint64_t)d, (uint64_t)rows, (uint64_t)L};
+    const uint64_t strides[2] = {(uint64_t)d * 4, (uint64_t)rows * d * 4};
+    const uint32_t box[3] = {(uint32_t)sru::kRecCJ, 1, (uint32_t)sru::kChunkT};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <typename UT>
+sru_status launch_fwd_seq(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
+                          float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
+                          cudaStream_t st) {
+    using Lay = sru::FwdLayout<UT>;
+    auto kern = sru::sru_fwd_seq_kernel<UT>;
+    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
+    dim3 grid((unsigned)((d + sru::kRecCJ - 1) / sru::kRecCJ), (unsigned)B, (unsigned)n_dir);
+    kern<<<grid, sru::kRecCJ, Lay::SMEM, st>>>(mp.u, mp.x, v, b, c0, mask, h, c_T, ckpt, (int)L, (int)B, (int)d,
+                                               n_dir, alpha);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+template <typename UT, typename DUT, bool ACC, int DIR>
+sru_status launch_bwd_seq_dir(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
+                              const float* ckpt, const float* dc_T, DUT* dU, float* dx, double* partial, float* dc0,
+                              int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
+    using Lay = sru::BwdLayout<UT, ACC>;
+    auto kern = sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR>;
+    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
+    dim3 grid((unsigned)((d + sru::kRecCJ - 1) / sru::kRecCJ), (unsigned)B, 1);
+    kern<<<grid, sru::kRecCJ, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.dx, v, b, mask, ckpt, dc_T, dU, dx, partial,
+                                               dc0, (int)L, (int)B, (int)d, n_dir, alpha);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+template <typename UT, typename DUT>
+sru_status launch_bwd_seq(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask, const float* ckpt,
+                          const float* dc_T, void* dU, float* dx, double* partial, float* dc0, int64_t L, int64_t B,
+                          int64_t d, int n_dir, float alpha, cudaStream_t st) {
+    DUT* du = reinterpret_cast<DUT*>(dU);
+    sru_status s = launch_bwd_seq_dir<UT, DUT, false, 0>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d,
+                                                        n_dir, alpha, st);
+    if (s != SRU_OK || n_dir == 1) return s;
+    return launch_bwd_seq_dir<UT, DUT, true, 1>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir,
+                                               alpha, st);
+}
+
+}  // namespace
+
+// =========================================================================
+extern "C" {
+
+const char* sru_status_string(int status) {
+    switch (status) {
+        case SRU_OK: return "SRU_OK";
+        case SRU_ERR_INVALID: return "SRU_ERR_INVALID: bad pointer, size, alignment or dtype";
+        case SRU_ERR_CUDA: return "SRU_ERR_CUDA: a CUDA call failed";
+        case SRU_ERR_TIMEOUT: return "SRU_ERR_TIMEOUT: a bounded device-side wait expired";
+        case SRU_ERR_UNSUPPORTED: return "SRU_ERR_UNSUPPORTED: request outside this build's limits";
+        default: return "unknown sru_status";
+    }
+}
+
+int sru_get_last_cuda_error(void) { return g_last_cuda_error; }
+
+int sru_version(void) { return 100; }
+
+size_t sru_workspace_bytes(int64_t L, int64_t B, int64_t d, int bidirectional, unsigned flags) {
+    (void)flags;
+    if (check_layer_sizes(L, B, d) != SRU_OK) return 0;
+    return ws_layout(L, B, d, bidirectional ? 2 : 1).total;
+}
+
+sru_status sru_project(const void* X, int x_t, const void* W, int w_t, void* U, int u_t, int64_t M, int64_t N,
+                       int64_t K, void* stream) {
+    if (M < 0 || N < 0 || K < 0) return SRU_ERR_INVALID;
+    if (M == 0 || N == 0) return SRU_OK;
+    if (!X || !W || !U || !aligned16(X) || !aligned16(W) || !aligned16(U)) return SRU_ERR_INVALID;
+    if (K % 8 != 0 || N % 8 != 0) return SRU_ERR_UNSUPPORTED;
+    if (M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    if (x_t == SRU_F32 && w_t == SRU_F32 && u_t == SRU_F32) {
+        if (K == 0) return zero_f32(reinterpret_cast<float*>(U), (size_t)M * N, st);
+        return launch_simt(reinterpret_cast<const float*>(X), K, 1, reinterpret_cast<const float*>(W), K, 1,
+                           reinterpret_cast<float*>(U), M, N, K, 0, st);
+    }
+    if (x_t != SRU_BF16 || w_t != SRU_BF16 || (u_t != SRU_BF16 && u_t != SRU_F32)) return SRU_ERR_INVALID;
+    if (K == 0) return SRU_ERR_UNSUPPORTED;
+    CUtensorMap ma, mb;
+    if (!map_kmajor(&ma, X, M, K, sru::gemm::BM) || !map_kmajor(&mb, W, N, K, sru::gemm::BN)) return SRU_ERR_INVALID;
+    if (u_t == SRU_BF16) return launch_tc_gemm<false, false, sru::gemm::kOutBF16>(ma, mb, U, M, N, K, st);
+    return launch_tc_gemm<false, false, sru::gemm::kOutF32>(ma, mb, U, M, N, K, st);
+}
+
+sru_status sru_project_backward(const void* dU, const void* X, const void* W, int t, float* dX, int accumulate,
+                                float* dW, int64_t M, int64_t N, int64_t K, void* stream) {
+    if (M < 0 || N < 0 || K < 0) return SRU_ERR_INVALID;
+    if (!dU || !aligned16(dU)) return SRU_ERR_INVALID;
+    if (dX && (!W || !aligned16(W) || !aligned16(dX))) return SRU_ERR_INVALID;
+    if (dW && (!X || !aligned16(X) || !aligned16(dW))) return SRU_ERR_INVALID;
+    if (K % 8 != 0 || N % 8 != 0) return SRU_ERR_UNSUPPORTED;
+    if (M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
+    if (t != SRU_F32 && t != SRU_BF16) return SRU_ERR_INVALID;
+    cudaStream_t st = as_stream(stream);
+    if (K == 0) return SRU_OK;
+    if (t == SRU_F32) {
+        const float* du = reinterpret_cast<const float*>(dU);
+        if (dX) {
+            if (N == 0) {
+                if (!accumulate) { sru_status s = zero_f32(dX, (size_t)M * K, st); if (s) return s; }
+            } else if (M > 0) {
+                sru_status s = launch_simt(du, N, 1, reinterpret_cast<const float*>(W), 1, K, dX, M, K, N, accumulate, st);
+                if (s != SRU_OK) return s;
+            }
+        }
+        if (dW && N > 0) {
+            if (M == 0) return zero_f32(dW, (size_t)N * K, st);
+            return launch_simt(du, 1, N, reinterpret_cast<const float*>(X), 1, K, dW, N, K, M, 0, st);
+        }
+        return SRU_OK;
+    }
+    // bf16 on the tensor cores
+    if (dX && M > 0) {
+        if (N == 0) {
+            if (!accumulate) { sru_status s = zero_f32(dX, (size_t)M * K, st); if (s) return s; }
+        } else {
+            CUtensorMap ma, mb;
+            // A = dU (M x N) K-major; B(c = k, red = n) = W[n][k]: MN-major with ld = K
+            if (!map_kmajor(&ma, dU, M, N, sru::gemm::BM) || !map_mnmajor(&mb, W, K, N, K)) return SRU_ERR_INVALID;
+            sru_status s = accumulate ? launch_tc_gemm<false, true, sru::gemm::kOutF32Acc>(ma, mb, dX, M, K, N, st)
+                                      : launch_tc_gemm<false, true, sru::gemm::kOutF32>(ma, mb, dX, M, K, N, st);
+            if (s != SRU_OK) return s;
+        }
+    }
+    if (dW && N > 0) {
+        if (M == 0) return zero_f32(dW, (size_t)N * K, st);
+        CUtensorMap ma, mb;
+        // A(r = n, red = m) = dU[m][n]: MN-major, ld = N; B(c = k, red = m) = X[m][k]: MN-major, ld = K
+        if (!map_mnmajor(&ma, dU, N, M, N) || !map_mnmajor(&mb, X, K, M, K)) return SRU_ERR_INVALID;
+        return launch_tc_gemm<true, true, sru::gemm::kOutF32>(ma, mb, dW, N, K, M, st);
+    }
+    return SRU_OK;
+}
+
+sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, const float* b, const float* c0,
+                       const uint8_t* mask, int64_t L, int64_t B, int64_t d, float alpha, int bidirectional,
+                       unsigned flags, float* h, float* c_T, void* workspace, void* stream) {
+    (void)flags;
+    sru_status s = check_layer_sizes(L, B, d);
+    if (s != SRU_OK) return s;
+    if (u_t != SRU_F32 && u_t != SRU_BF16) return SRU_ERR_INVALID;
+    const int n_dir = bidirectional ? 2 : 1;
+    if (B == 0) return SRU_OK;
+    if (!v || !b || !c_T) return SRU_ERR_INVALID;
+    cudaStream_t st = as_stream(stream);
+    if (L == 0) {
+        const size_t n = (size_t)B * n_dir * d;
+        sru::sru_copy_state_kernel<<<blocks_for(n, 256), 256, 0, st>>>(c0, c_T, n);
+        SRU_CUDA_TRY(cudaGetLastError());
+        return SRU_OK;
+    }
+    if (!U || !x || !h || !aligned16(U) || !aligned16(x) || !aligned16(h)) return SRU_ERR_INVALID;
+    if (workspace && !aligned16(workspace)) return SRU_ERR_INVALID;
+    RecMaps mp;
+    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir) || !map_f32_rows(&mp.x, x, L, B, d)) return SRU_ERR_INVALID;
+    float* ckpt = workspace ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ws_layout(L, B, d, n_dir).ckpt_off)
+                            : nullptr;
+    if (u_t == SRU_BF16)
+        return launch_fwd_seq<__nv_bfloat16>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+    return launch_fwd_seq<float>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+}
+
+sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, const float* b, const float* c0,
+                        const uint8_t* mask, int64_t L, int64_t B, int64_t d, float alpha, int bidirectional,
+                        unsigned flags, const float* dh, const float* dc_T, void* workspace, void* dU, int du_t,
+                        float* dx, float* dv, float* db, float* dc0, void* stream) {
+    (void)flags;
+    (void)c0;  // the forward's checkpoints already hold the state derived from c0
+    sru_status s = check_layer_sizes(L, B, d);
+    if (s != SRU_OK) return s;
+    if (u_t != SRU_F32 && u_t != SRU_BF16) return SRU_ERR_INVALID;
+    if (du_t != SRU_F32 && du_t != SRU_BF16) return SRU_ERR_INVALID;
+    const int n_dir = bidirectional ? 2 : 1;
+    if (!v || !b || !dv || !db) return SRU_ERR_INVALID;
+    cudaStream_t st = as_stream(stream);
+    if (B == 0 || L == 0) {
+        // no steps: dv = db = 0, dc0 = dc_T
+        s = zero_f32(dv, (size_t)n_dir * 2 * d, st);
+        if (s == SRU_OK) s = zero_f32(db, (size_t)n_dir * 2 * d, st);
+        if (s == SRU_OK && B > 0) {
+            if (!dc0) return SRU_ERR_INVALID;
+            const size_t n = (size_t)B * n_dir * d;
+            sru::sru_copy_state_kernel<<<blocks_for(n, 256), 256, 0, st>>>(dc_T, dc0, n);
+            SRU_CUDA_TRY(cudaGetLastError());
+        }
+        return s;
+    }
+    if (!U || !x || !dh || !workspace || !dU || !dx || !dc0) return SRU_ERR_INVALID;
+    if (!aligned16(U) || !aligned16(x) || !aligned16(dh) || !aligned16(workspace) || !aligned16(dU) || !aligned16(dx))
+        return SRU_ERR_INVALID;
+    RecMaps mp;
+    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir) || !map_f32_rows(&mp.x, x, L, B, d) ||
+        !map_f32_rows(&mp.dh, dh, L, B * n_dir, d) || !map_f32_rows(&mp.dx, dx, L, B, d))
+        return SRU_ERR_INVALID;
+    const WsLayout w = ws_layout(L, B, d, n_dir);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const float* ckpt = reinterpret_cast<const float*>(ws + w.ckpt_off);
+    double* partial = reinterpret_cast<double*>(ws + w.partial_off);
+    if (u_t == SRU_BF16) {
+        s = du_t == SRU_BF16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial,
+                                                                             dc0, L, B, d, n_dir, alpha, st)
+                             : launch_bwd_seq<__nv_bfloat16, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
+                                                                    L, B, d, n_dir, alpha, st);
+    } else {
+        s = du_t == SRU_BF16 ? launch_bwd_seq<float, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
+                                                                     L, B, d, n_dir, alpha, st)
+                             : launch_bwd_seq<float, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
+                                                            n_dir, alpha, st);
+    }
+    if (s != SRU_OK) return s;
+    const size_t nred = (size_t)n_dir * 4 * d;
+    sru::sru_reduce_dvdb_kernel<<<blocks_for(nred, 256), 256, 0, st>>>(partial, (int)B, (int)d, n_dir, dv, db);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+sru_status sru_sync_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned word = 0;
+    e = cudaMemcpyFromSymbol(&word, sru::g_error_word, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (word != 0) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(sru::g_error_word, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_fail(e);
+        return SRU_ERR_TIMEOUT;
+    }
+    return SRU_OK;
+}
+
+}  // extern "C"

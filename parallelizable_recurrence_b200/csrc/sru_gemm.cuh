@@ -1,0 +1,323 @@
+// sru_gemm.cuh -- the projection of Eq. (1) and its gradients on sm_100a.
+//
+// "When Attention Meets Fast Recurrence" (T. Lei), background section on SRU:
+// the three per-step matrix-vector products of all L steps are grouped into one
+// product U^T = [W; W'; W''] X^T, the only dense contraction of the layer.
+//
+// tc_gemm_kernel computes  out[r, c] (+)= sum_k A(r, k) * B(c, k)  on the
+// 5th-generation tensor cores: bf16 operands staged by TMA into 128-byte
+// swizzled shared memory, tcgen05.mma issued by a single thread into a fp32
+// accumulator in tensor memory (TMEM), and an epilogue that reads TMEM with
+// tcgen05.ld.  The kernel is persistent (one CTA per SM walking output tiles)
+// and warp specialised:
+//   warp 0        TMA producer (one elected lane), STAGES-deep smem ring
+//   warp 1        TMEM allocator and MMA issuer (one elected lane)
+//   warps 2..5    epilogue, one TMEM lane quarter each
+// Two 128 x 256 fp32 accumulators (512 TMEM columns) let the epilogue of tile
+// i overlap the main loop of tile i+1.
+//
+// Operand majorness (which index is contiguous in global memory):
+//   U  = X  W^T : A = X  (M x K, K-major), B = W (N x K, K-major)
+//   dX = dU W   : A = dU (M x N, K-major), B = W read as (K x N): MN-major
+//   dW = dU^T X : A = dU read as (N x M): MN-major, B = X read as (K x M): MN-major
+// A K-major tile is one TMA box of (64 K, rows); an MN-major tile is boxes of
+// (64 rows, 64 K) placed 8 KB apart.
+#pragma once
+
+#include "sru_ptx.cuh"
+
+namespace sru {
+namespace gemm {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 2 * BN;  // two fp32 accumulators
+constexpr uint32_t MN_BOX_BYTES = 64 * 64 * 2;  // one (64 x 64) MN-major box
+constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+enum OutMode : int { kOutBF16 = 0, kOutF32 = 1, kOutF32Acc = 2 };
+
+// Shared-memory matrix descriptor (tcgen05 "smem descriptor"): start address,
+// leading- and stride-dimension byte offsets (16-byte units), descriptor
+// version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= 1ull << 46;  // version for sm_100
+    d |= 2ull << 61;  // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B,
+// operand majorness, N >> 3 and M >> 4.
+__host__ __device__ constexpr uint32_t idesc_bf16(bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+template <bool A_MN, bool B_MN, int OUT>
+__global__ void __launch_bounds__(THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                   void* __restrict__ out, int M, int N, int K, int ldo) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile uint32_t* consumed = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m_tiles = (M + BM - 1) / BM, n_tiles = (N + BN - 1) / BN;
+    const int tiles = m_tiles * n_tiles;
+    const int kblocks = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        *consumed = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------------ producer
+            uint32_t issued = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x) {
+                const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, kErrTimeoutMma) || *abort_flag) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    uint8_t* a_dst = smem + stage * STAGE_BYTES;
+                    uint8_t* b_dst = a_dst + A_BYTES;
+                    const int k0 = kb * BK;
+                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                    if (!A_MN) {
+                        tma_load_2d(a_dst, &map_a, &full[stage], k0, m0);
+                    } else {
+                        tma_load_2d(a_dst, &map_a, &full[stage], m0, k0);
+                        tma_load_2d(a_dst + MN_BOX_BYTES, &map_a, &full[stage], m0 + 64, k0);
+                    }
+                    if (!B_MN) {
+                        tma_load_2d(b_dst, &map_b, &full[stage], k0, n0);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < BN / 64; ++q)
+                            tma_load_2d(b_dst + q * MN_BOX_BYTES, &map_b, &full[stage], n0 + 64 * q, k0);
+                    }
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (*abort_flag) {
+                // wait (bounded) for the loads still in flight before this CTA may exit
+                for (uint32_t q = *consumed; q < issued; ++q)
+                    mbar_wait(&full[q % STAGES], (q / STAGES) & 1u, kErrTimeoutLoad);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = idesc_bf16(A_MN, B_MN);
+            int stage = 0;
+            uint32_t phase = 0, nconsumed = 0;
+            int it = 0;
+            for (int tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, kErrTimeoutEpilogue)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                bool ok = true;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, kErrTimeoutLoad)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t adesc = A_MN ? smem_desc_sw128(a_addr + kk * 2048, MN_BOX_BYTES, 1024)
+                                                    : smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+                        const uint64_t bdesc = B_MN ? smem_desc_sw128(b_addr + kk * 2048, MN_BOX_BYTES, 1024)
+                                                    : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+                        tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty[stage]);  // frees the smem stage once these MMAs retire
+                    *consumed = ++nconsumed;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_commit(&tfull[acc]);  // accumulator ready for the epilogue
+            }
+            // every MMA this thread issued has retired before TMEM is released
+            tc_commit(drain);
+            mbar_wait(drain, 0, kErrTimeoutMma);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+        int it = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
+            const bool ok = mbar_wait(&tfull[acc], acc_phase, kErrTimeoutMma);
+            if (!__all_sync(0xffffffffu, ok) || *abort_flag) {
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const int row = m0 + quarter * 32 + lane;
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                const int col0 = n0 + ch * 32;
+                if (col0 >= N) break;  // uniform across the warp
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN + ch * 32, r);
+                tc_wait_ld();
+                if (row < M) {
+                    if (OUT == kOutBF16) {
+                        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * ldo + col0;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            if (col0 + g * 8 < N) {
+                                uint4 pk;
+                                uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    __nv_bfloat162 two = __floats2bfloat162_rn(__uint_as_float(r[g * 8 + 2 * e]),
+                                                                               __uint_as_float(r[g * 8 + 2 * e + 1]));
+                                    w[e] = *reinterpret_cast<uint32_t*>(&two);
+                                }
+                                *reinterpret_cast<uint4*>(o + g * 8) = pk;
+                            }
+                        }
+                    } else {
+                        float* o = reinterpret_cast<float*>(out) + (size_t)row * ldo + col0;
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) {
+                            if (col0 + g * 4 < N) {
+                                float4 val = make_float4(__uint_as_float(r[g * 4 + 0]), __uint_as_float(r[g * 4 + 1]),
+                                                         __uint_as_float(r[g * 4 + 2]), __uint_as_float(r[g * 4 + 3]));
+                                if (OUT == kOutF32Acc) {
+                                    const float4 old = *reinterpret_cast<const float4*>(o + g * 4);
+                                    val.x += old.x;
+                                    val.y += old.y;
+                                    val.z += old.z;
+                                    val.w += old.w;
+                                }
+                                *reinterpret_cast<float4*>(o + g * 4) = val;
+                            }
+                        }
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core fp32 product with explicit element strides (the fp32 path):
+//   out[r * ldo + c] (+)= sum_k A[r*a_rs + k*a_ks] * B[c*b_rs + k*b_ks]
+// 64 x 64 output tile per 256-thread CTA, 4 x 4 outputs per thread.
+constexpr int ST = 64, SK = 16;
+
+__global__ void __launch_bounds__(256)
+    simt_gemm_f32_kernel(const float* __restrict__ A, long long a_rs, long long a_ks, const float* __restrict__ Bm,
+                         long long b_rs, long long b_ks, float* __restrict__ out, long long ldo, int R, int C, int K,
+                         int accumulate) {
+    __shared__ float As[SK][ST + 1];
+    __shared__ float Bs[SK][ST + 1];
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    const int r0 = blockIdx.y * ST, c0 = blockIdx.x * ST;
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < K; k0 += SK) {
+        for (int e = threadIdx.x; e < SK * ST; e += 256) {
+            const int kk = e / ST, rr = e % ST;
+            const int k = k0 + kk;
+            As[kk][rr] = (r0 + rr < R && k < K) ? A[(long long)(r0 + rr) * a_rs + (long long)k * a_ks] : 0.f;
+            Bs[kk][rr] = (c0 + rr < C && k < K) ? Bm[(long long)(c0 + rr) * b_rs + (long long)k * b_ks] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < SK; ++kk) {
+            float a[4], bb[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                a[i] = As[kk][ty * 4 + i];
+                bb[i] = Bs[kk][tx * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) acc[i][jj] = fmaf(a[i], bb[jj], acc[i][jj]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const int r = r0 + ty * 4 + i, c = c0 + tx * 4 + jj;
+            if (r < R && c < C) {
+                float* o = out + (long long)r * ldo + c;
+                *o = accumulate ? *o + acc[i][jj] : acc[i][jj];
+            }
+        }
+}
+
+}  // namespace gemm
+}  // namespace sru

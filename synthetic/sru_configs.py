@@ -26,10 +26,14 @@ import numpy as np
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
-    """Round fp32 values to bf16 (nearest, ties to even); returns the 16-bit patterns."""
-    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return rounded.astype(np.uint16)
+    """Round finite fp32 values to bf16 (nearest, ties to even); returns the 16-bit patterns."""
+    flat = np.ascontiguousarray(a, dtype=np.float32).reshape(-1)
+    out = np.empty(flat.shape, dtype=np.uint16)
+    step = 1 << 24
+    for s in range(0, flat.size, step):
+        u = flat[s:s + step].view(np.uint32)
+        out[s:s + step] = ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
+    return out.reshape(np.shape(a))
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -88,7 +92,7 @@ CONFIGS: Dict[str, SRUConfig] = {
 }
 
 
-def generate(cfg: SRUConfig, with_grad: Optional[bool] = None) -> Dict[str, np.ndarray]:
+def generate(cfg: SRUConfig, with_grad: Optional[bool] = None, u_direct: bool = False) -> Dict[str, np.ndarray]:
     """Draw every input of one workload, deterministically from cfg.seed.
 
     Returns numpy arrays (host memory):
@@ -96,7 +100,10 @@ def generate(cfg: SRUConfig, with_grad: Optional[bool] = None) -> Dict[str, np.n
       mask (L,B) u8 or None; lengths (B,) or None; dh (L,B,n_dir,d) f32 (if with_grad);
       for a projected workload: X (L*B,d) and W (N,d) in the projection type
         (bf16 bit patterns as uint16, or f32), and X_f32/W_f32 (their exact fp32 values);
-      for a U-given workload: U (L,B,n_dir,3,d) as bf16 bits, U_f32 its exact values.
+      for a U-given workload, or with u_direct=True: U (L,B,n_dir,3,d) ~ N(0,1) in the
+        storage type (bf16 bits, or f32 for an fp32 workload) and U_f32 its exact values.
+        (X W^T with these distributions has N(0,1) entries, so a drawn U has the
+        distribution of a projected one.)
     """
     if with_grad is None:
         with_grad = cfg.backward
@@ -105,7 +112,7 @@ def generate(cfg: SRUConfig, with_grad: Optional[bool] = None) -> Dict[str, np.n
     out: Dict[str, Optional[np.ndarray]] = {}
     x = rng.standard_normal((L, B, d), dtype=np.float32)
     out["x"] = x
-    if cfg.proj_dtype != "none":
+    if cfg.proj_dtype != "none" and not u_direct:
         a = math.sqrt(3.0 / d)
         W = rng.uniform(-a, a, size=(nd * 3 * d, d)).astype(np.float32)
         if cfg.proj_dtype == "bf16":
@@ -117,9 +124,15 @@ def generate(cfg: SRUConfig, with_grad: Optional[bool] = None) -> Dict[str, np.n
             out["X"], out["W"] = x.reshape(L * B, d), W
             out["X_f32"], out["W_f32"] = out["X"], W
     else:
-        Ub = f32_to_bf16_bits(rng.standard_normal((L, B, nd, 3, d), dtype=np.float32))
-        out["U"] = Ub
-        out["U_f32"] = bf16_bits_to_f32(Ub)
+        Uf = rng.standard_normal((L, B, nd, 3, d), dtype=np.float32)
+        if cfg.proj_dtype == "fp32":
+            out["U"] = Uf
+            out["U_f32"] = Uf
+        else:
+            Ub = f32_to_bf16_bits(Uf)
+            del Uf
+            out["U"] = Ub
+            out["U_f32"] = None  # widen on demand with bf16_bits_to_f32 (saves host memory)
     v = rng.uniform(-0.5, 0.5, size=(nd, 2, d)).astype(np.float32)
     if cfg.v_zero:
         v = np.zeros_like(v)

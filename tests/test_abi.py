@@ -1,0 +1,90 @@
+"""The C-ABI library loads and exports every entry point include/sru.h declares,
+and its host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sru.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sru_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib_path():
+    from parallelizable_recurrence_b200 import build
+    return build.build()
+
+
+@pytest.fixture(scope="module")
+def lib(lib_path):
+    import parallelizable_recurrence_b200 as m
+    return m.load_library(lib_path)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("sru_project", "sru_project_backward", "sru_forward", "sru_backward",
+                     "sru_workspace_bytes", "sru_sync_status"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib_path, lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib_path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (sru_[a-z_0-9]+)\b", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_binding_lists_every_declared_symbol():
+    import parallelizable_recurrence_b200 as m
+    assert sorted(m.EXPORTED) == declared_functions()
+
+
+def test_status_strings_and_version(lib):
+    assert lib.sru_status_string(0) == b"SRU_OK"
+    assert b"TIMEOUT" in lib.sru_status_string(3)
+    assert lib.sru_version() >= 100
+
+
+def test_workspace_size_is_host_arithmetic(lib):
+    # checkpoints (ceil(L/16) * B * n_dir * d floats) + partial sums (B * n_dir * 4 * d doubles)
+    n = lib.sru_workspace_bytes(1024, 16, 2048, 0, 0)
+    assert n >= 64 * 16 * 2048 * 4 + 16 * 4 * 2048 * 8
+    assert lib.sru_workspace_bytes(1024, 16, 2048, 1, 0) > n
+    assert lib.sru_workspace_bytes(10, 2, 12, 0, 0) == 0      # d % 8 != 0 is unsupported
+
+
+def test_invalid_arguments_return_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)
+    # d not a multiple of 8
+    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4, 2, 12, 1.0, 0, 0, fake, fake, None, None)
+    assert st == 4
+    # negative sizes
+    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, -1, 2, 16, 1.0, 0, 0, fake, fake, None, None)
+    assert st == 1
+    # unknown U dtype
+    st = lib.sru_forward(fake, 7, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, fake, None, None)
+    assert st == 1
+    # null outputs
+    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, None, None, None, None)
+    assert st == 1
+    # misaligned pointer
+    st = lib.sru_project(vp(0x1001), 1, fake, 1, fake, 1, 64, 64, 64, None)
+    assert st == 1
+    # unsupported type combination
+    st = lib.sru_project(fake, 0, fake, 1, fake, 1, 64, 64, 64, None)
+    assert st == 1
+    # backward without a workspace
+    st = lib.sru_backward(fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, None, None,
+                          fake, 1, fake, fake, fake, fake, None)
+    assert st == 1
