@@ -113,19 +113,24 @@ sru_status sru_project_backward(const void* dU, const void* X, const void* W, in
  * Eqs. (2)-(5) over all t for every (direction, batch row, channel).
  *   U (u_t = F32 or BF16), x, v, b as above; c0 nullable (zero state);
  *   mask nullable.  Outputs h (L, B, n_dir, d) and c_T (B, n_dir, d), fp32.
- *   workspace: sru_workspace_bytes(...) bytes, or NULL for inference only
- *   (then no checkpoints are written and sru_backward cannot follow).
- *   flags: SRU_FLAG_* above.
+ *   workspace / workspace_bytes: a device buffer of at least
+ *   sru_workspace_bytes(L, B, d, bidirectional, flags) bytes (checked:
+ *   SRU_ERR_INVALID if smaller), or NULL for inference only (then no
+ *   checkpoints are written, sru_backward cannot follow, and the scan path is
+ *   not available).  flags: SRU_FLAG_* above.  With SRU_FLAG_V_ZERO the
+ *   library runs the chunked scan when the sequential kernel would leave SMs
+ *   idle (fewer than two 64-channel CTAs per SM), or when forced.
  */
 sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, const float* b,
                        const float* c0, const uint8_t* mask, int64_t L, int64_t B, int64_t d,
                        float alpha, int bidirectional, unsigned flags,
-                       float* h, float* c_T, void* workspace, void* stream);
+                       float* h, float* c_T, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Backward of sru_forward for Loss = sum(dh * h) + sum(dc_T * c_T).
  * Inputs: the forward's U, x, v, b, c0, mask, sizes, alpha, flags and the
- *   workspace the forward filled; dh (L, B, n_dir, d); dc_T nullable (zero).
+ *   workspace the forward filled (same buffer and size); dh (L, B, n_dir, d);
+ *   dc_T nullable (zero).  c0 is not read: the checkpoints carry it.
  * Outputs (overwritten):
  *   dU (L, B, n_dir, 3, d) of type du_t (F32 or BF16),
  *   dx (L, B, d) fp32: the highway part alpha * (1 - r) * dh, summed over directions
@@ -136,7 +141,7 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
 sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, const float* b,
                         const float* c0, const uint8_t* mask, int64_t L, int64_t B, int64_t d,
                         float alpha, int bidirectional, unsigned flags,
-                        const float* dh, const float* dc_T, void* workspace,
+                        const float* dh, const float* dc_T, void* workspace, size_t workspace_bytes,
                         void* dU, int du_t, float* dx, float* dv, float* db, float* dc0,
                         void* stream);
 

@@ -71,10 +71,10 @@ def load_library(path: str = LIB_PATH):
     lib.sru_project_backward.argtypes = [_vp, _vp, _vp, _int, _vp, _int, _vp, _i64, _i64, _i64, _vp]
     lib.sru_forward.restype = _int
     lib.sru_forward.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _f32, _int, _u32,
-                                _vp, _vp, _vp, _vp]
+                                _vp, _vp, _vp, ctypes.c_size_t, _vp]
     lib.sru_backward.restype = _int
     lib.sru_backward.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _f32, _int, _u32,
-                                 _vp, _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp]
+                                 _vp, _vp, _vp, ctypes.c_size_t, _vp, _int, _vp, _vp, _vp, _vp, _vp]
     lib.sru_sync_status.restype = _int
     lib.sru_sync_status.argtypes = [_vp]
     _lib = lib
@@ -99,6 +99,10 @@ def _ptr(t: Optional[torch.Tensor], dtype=None):
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"expected {dtype}, got {t.dtype}")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _nbytes(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
 
 
 def _stream(stream=None):
@@ -158,7 +162,8 @@ def sru_forward(U, x, v, b, h, c_T, c0=None, mask=None, alpha: float = 1.0, bidi
     _check(lib.sru_forward(_ptr(U), _dtype_code(U), _ptr(x, torch.float32), _ptr(v, torch.float32),
                            _ptr(b, torch.float32), _ptr(c0, torch.float32), _ptr(mask, torch.uint8),
                            L, B, d, float(alpha), int(bool(bidirectional)), flags,
-                           _ptr(h, torch.float32), _ptr(c_T, torch.float32), _ptr(workspace), _stream(stream)),
+                           _ptr(h, torch.float32), _ptr(c_T, torch.float32), _ptr(workspace),
+                           _nbytes(workspace), _stream(stream)),
            "sru_forward")
     return h, c_T
 
@@ -172,7 +177,7 @@ def sru_backward(U, x, v, b, dh, workspace, dU, dx, dv, db, dc0, c0=None, mask=N
                             _ptr(b, torch.float32), _ptr(c0, torch.float32), _ptr(mask, torch.uint8),
                             L, B, d, float(alpha), int(bool(bidirectional)), flags,
                             _ptr(dh, torch.float32), _ptr(dc_T, torch.float32), _ptr(workspace),
-                            _ptr(dU), _dtype_code(dU), _ptr(dx, torch.float32), _ptr(dv, torch.float32),
+                            _nbytes(workspace), _ptr(dU), _dtype_code(dU), _ptr(dx, torch.float32), _ptr(dv, torch.float32),
                             _ptr(db, torch.float32), _ptr(dc0, torch.float32), _stream(stream)),
            "sru_backward")
     return dU, dx, dv, db, dc0

@@ -12,6 +12,7 @@
 #include "../../include/sru.h"
 #include "sru_gemm.cuh"
 #include "sru_recurrence.cuh"
+#include "sru_scan.cuh"
 
 namespace {
 
@@ -99,19 +100,59 @@ cudaError_t ensure_smem(const void* kernel, size_t bytes) {
 }
 
 // ---------------------------------------------------------- workspace layout
+// [checkpoints | dv/db partial sums | scan flags | scan aggregates A, B, prefix]
+// The scan regions exist only when SRU_FLAG_V_ZERO is set.
 struct WsLayout {
-    size_t ckpt_off, ckpt_bytes, partial_off, partial_bytes, total;
+    size_t ckpt_off, partial_off, flags_off, agg_a_off, agg_b_off, prefix_off, total;
+    int64_t scan_items;
 };
 
-WsLayout ws_layout(int64_t L, int64_t B, int64_t d, int n_dir) {
+int64_t scan_chunks(int64_t L) { return (L + sru::kScanT - 1) / sru::kScanT; }
+
+WsLayout ws_layout(int64_t L, int64_t B, int64_t d, int n_dir, unsigned flags) {
     WsLayout w{};
     const int64_t nch = (L + sru::kChunkT - 1) / sru::kChunkT;
-    w.ckpt_off = 0;
-    w.ckpt_bytes = round256((size_t)nch * B * n_dir * d * sizeof(float));
-    w.partial_off = w.ckpt_off + w.ckpt_bytes;
-    w.partial_bytes = round256((size_t)B * n_dir * 4 * d * sizeof(double));
-    w.total = w.partial_off + w.partial_bytes;
+    const int64_t n_jt = (d + sru::kRecCJ - 1) / sru::kRecCJ;
+    const bool scan = (flags & SRU_FLAG_V_ZERO) != 0;
+    size_t off = 0;
+    w.ckpt_off = off;
+    off += round256((size_t)nch * B * n_dir * d * sizeof(float));
+    w.partial_off = off;
+    const int64_t partial_rows = scan ? scan_chunks(L) * B : B;
+    off += round256((size_t)partial_rows * n_dir * 4 * d * sizeof(double));
+    w.scan_items = scan ? scan_chunks(L) * n_jt * B * n_dir : 0;
+    w.flags_off = off;
+    if (scan) {
+        off += round256((size_t)(w.scan_items + 1) * sizeof(unsigned));
+        w.agg_a_off = off;
+        off += round256((size_t)w.scan_items * sru::kRecCJ * sizeof(float));
+        w.agg_b_off = off;
+        off += round256((size_t)w.scan_items * sru::kRecCJ * sizeof(float));
+        w.prefix_off = off;
+        off += round256((size_t)w.scan_items * sru::kRecCJ * sizeof(float));
+    }
+    w.total = off;
     return w;
+}
+
+sru::ScanState scan_state(void* workspace, const WsLayout& w) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    sru::ScanState ss;
+    ss.flags = reinterpret_cast<unsigned*>(ws + w.flags_off);
+    ss.agg_a = reinterpret_cast<float*>(ws + w.agg_a_off);
+    ss.agg_b = reinterpret_cast<float*>(ws + w.agg_b_off);
+    ss.prefix = reinterpret_cast<float*>(ws + w.prefix_off);
+    return ss;
+}
+
+// The chunked scan pays off when the sequential kernel would leave SMs idle:
+// fewer than two 64-channel CTAs per SM.  Only with SRU_FLAG_V_ZERO.
+bool use_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir) {
+    if (!(flags & SRU_FLAG_V_ZERO)) return false;
+    if (flags & SRU_FLAG_FORCE_SCAN) return true;
+    if (flags & SRU_FLAG_FORCE_SEQUENTIAL) return false;
+    const int64_t seq_ctas = ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B * n_dir;
+    return L >= 2 * sru::kScanT && seq_ctas < 2 * (int64_t)sm_count();
 }
 
 sru_status check_layer_sizes(int64_t L, int64_t B, int64_t d) {
@@ -230,6 +271,61 @@ sru_status launch_bwd_seq(const RecMaps& mp, const float* v, const float* b, con
                                                alpha, st);
 }
 
+
+sru_status reset_scan_flags(unsigned* flags, int64_t n, cudaStream_t st) {
+    sru::sru_scan_reset_kernel<<<blocks_for((size_t)n, 256), 256, 0, st>>>(flags, (int)n);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+template <typename UT>
+sru_status launch_fwd_scan(const RecMaps& mp, const float* b, const float* c0, const uint8_t* mask, float* h,
+                           float* c_T, float* ckpt, const sru::ScanState& ss, int64_t L, int64_t B, int64_t d,
+                           int n_dir, float alpha, cudaStream_t st) {
+    using Lay = sru::FwdScanLayout<UT>;
+    auto kern = sru::sru_fwd_scan_kernel<UT>;
+    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
+    const int64_t items = scan_chunks(L) * ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B * n_dir;
+    if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
+    sru_status s = reset_scan_flags(ss.flags, items + 1, st);
+    if (s != SRU_OK) return s;
+    kern<<<(unsigned)items, sru::kRecCJ, Lay::SMEM, st>>>(mp.u, mp.x, b, c0, mask, h, c_T, ckpt, ss, (int)L, (int)B,
+                                                          (int)d, n_dir, alpha);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+template <typename UT, typename DUT, bool ACC, int DIR>
+sru_status launch_bwd_scan_dir(const RecMaps& mp, const float* b, const uint8_t* mask, const float* ckpt,
+                               const float* dc_T, DUT* dU, float* dx, double* partial, float* dc0,
+                               const sru::ScanState& ss, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
+                               cudaStream_t st) {
+    using Lay = sru::BwdScanLayout<UT, ACC>;
+    auto kern = sru::sru_bwd_scan_kernel<UT, DUT, ACC, DIR>;
+    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
+    const int64_t items = scan_chunks(L) * ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B;
+    if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
+    sru_status s = reset_scan_flags(ss.flags, items + 1, st);
+    if (s != SRU_OK) return s;
+    kern<<<(unsigned)items, sru::kRecCJ, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.dx, b, mask, ckpt, dc_T, dU, dx,
+                                                          partial, dc0, ss, (int)L, (int)B, (int)d, n_dir, alpha);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+template <typename UT, typename DUT>
+sru_status launch_bwd_scan(const RecMaps& mp, const float* b, const uint8_t* mask, const float* ckpt,
+                           const float* dc_T, void* dU, float* dx, double* partial, float* dc0,
+                           const sru::ScanState& ss, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
+                           cudaStream_t st) {
+    DUT* du = reinterpret_cast<DUT*>(dU);
+    sru_status s = launch_bwd_scan_dir<UT, DUT, false, 0>(mp, b, mask, ckpt, dc_T, du, dx, partial, dc0, ss, L, B,
+                                                         d, n_dir, alpha, st);
+    if (s != SRU_OK || n_dir == 1) return s;
+    return launch_bwd_scan_dir<UT, DUT, true, 1>(mp, b, mask, ckpt, dc_T, du, dx, partial, dc0, ss, L, B, d, n_dir,
+                                                alpha, st);
+}
+
 }  // namespace
 
 // =========================================================================
@@ -251,9 +347,8 @@ int sru_get_last_cuda_error(void) { return g_last_cuda_error; }
 int sru_version(void) { return 100; }
 
 size_t sru_workspace_bytes(int64_t L, int64_t B, int64_t d, int bidirectional, unsigned flags) {
-    (void)flags;
     if (check_layer_sizes(L, B, d) != SRU_OK) return 0;
-    return ws_layout(L, B, d, bidirectional ? 2 : 1).total;
+    return ws_layout(L, B, d, bidirectional ? 2 : 1, flags).total;
 }
 
 sru_status sru_project(const void* X, int x_t, const void* W, int w_t, void* U, int u_t, int64_t M, int64_t N,
@@ -329,8 +424,8 @@ sru_status sru_project_backward(const void* dU, const void* X, const void* W, in
 
 sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, const float* b, const float* c0,
                        const uint8_t* mask, int64_t L, int64_t B, int64_t d, float alpha, int bidirectional,
-                       unsigned flags, float* h, float* c_T, void* workspace, void* stream) {
-    (void)flags;
+                       unsigned flags, float* h, float* c_T, void* workspace, size_t workspace_bytes,
+                       void* stream) {
     sru_status s = check_layer_sizes(L, B, d);
     if (s != SRU_OK) return s;
     if (u_t != SRU_F32 && u_t != SRU_BF16) return SRU_ERR_INVALID;
@@ -345,11 +440,22 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
         return SRU_OK;
     }
     if (!U || !x || !h || !aligned16(U) || !aligned16(x) || !aligned16(h)) return SRU_ERR_INVALID;
-    if (workspace && !aligned16(workspace)) return SRU_ERR_INVALID;
+    const WsLayout w = ws_layout(L, B, d, n_dir, flags);
+    const bool scan = use_scan(flags, L, B, d, n_dir);
+    if (workspace) {
+        if (!aligned16(workspace) || workspace_bytes < w.total) return SRU_ERR_INVALID;
+    } else if (scan) {
+        return SRU_ERR_INVALID;  // the scan needs its flags and aggregates
+    }
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir) || !map_f32_rows(&mp.x, x, L, B, d)) return SRU_ERR_INVALID;
-    float* ckpt = workspace ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ws_layout(L, B, d, n_dir).ckpt_off)
-                            : nullptr;
+    float* ckpt = workspace ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.ckpt_off) : nullptr;
+    if (scan) {
+        const sru::ScanState ss = scan_state(workspace, w);
+        if (u_t == SRU_BF16)
+            return launch_fwd_scan<__nv_bfloat16>(mp, b, c0, mask, h, c_T, ckpt, ss, L, B, d, n_dir, alpha, st);
+        return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, ckpt, ss, L, B, d, n_dir, alpha, st);
+    }
     if (u_t == SRU_BF16)
         return launch_fwd_seq<__nv_bfloat16>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
     return launch_fwd_seq<float>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
@@ -357,9 +463,9 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
 
 sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, const float* b, const float* c0,
                         const uint8_t* mask, int64_t L, int64_t B, int64_t d, float alpha, int bidirectional,
-                        unsigned flags, const float* dh, const float* dc_T, void* workspace, void* dU, int du_t,
-                        float* dx, float* dv, float* db, float* dc0, void* stream) {
-    (void)flags;
+                        unsigned flags, const float* dh, const float* dc_T, void* workspace,
+                        size_t workspace_bytes, void* dU, int du_t, float* dx, float* dv, float* db, float* dc0,
+                        void* stream) {
     (void)c0;  // the forward's checkpoints already hold the state derived from c0
     sru_status s = check_layer_sizes(L, B, d);
     if (s != SRU_OK) return s;
@@ -383,28 +489,45 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     if (!U || !x || !dh || !workspace || !dU || !dx || !dc0) return SRU_ERR_INVALID;
     if (!aligned16(U) || !aligned16(x) || !aligned16(dh) || !aligned16(workspace) || !aligned16(dU) || !aligned16(dx))
         return SRU_ERR_INVALID;
+    const WsLayout w = ws_layout(L, B, d, n_dir, flags);
+    if (workspace_bytes < w.total) return SRU_ERR_INVALID;
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir) || !map_f32_rows(&mp.x, x, L, B, d) ||
         !map_f32_rows(&mp.dh, dh, L, B * n_dir, d) || !map_f32_rows(&mp.dx, dx, L, B, d))
         return SRU_ERR_INVALID;
-    const WsLayout w = ws_layout(L, B, d, n_dir);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const float* ckpt = reinterpret_cast<const float*>(ws + w.ckpt_off);
     double* partial = reinterpret_cast<double*>(ws + w.partial_off);
-    if (u_t == SRU_BF16) {
-        s = du_t == SRU_BF16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial,
-                                                                             dc0, L, B, d, n_dir, alpha, st)
-                             : launch_bwd_seq<__nv_bfloat16, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
-                                                                    L, B, d, n_dir, alpha, st);
-    } else {
-        s = du_t == SRU_BF16 ? launch_bwd_seq<float, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
+    const bool scan = use_scan(flags, L, B, d, n_dir);
+    const bool ub = u_t == SRU_BF16, db16 = du_t == SRU_BF16;
+    if (scan) {
+        const sru::ScanState ss = scan_state(workspace, w);
+        if (ub)
+            s = db16 ? launch_bwd_scan<__nv_bfloat16, __nv_bfloat16>(mp, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss,
                                                                      L, B, d, n_dir, alpha, st)
-                             : launch_bwd_seq<float, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
+                     : launch_bwd_scan<__nv_bfloat16, float>(mp, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss, L, B,
+                                                             d, n_dir, alpha, st);
+        else
+            s = db16 ? launch_bwd_scan<float, __nv_bfloat16>(mp, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss, L, B,
+                                                             d, n_dir, alpha, st)
+                     : launch_bwd_scan<float, float>(mp, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss, L, B, d, n_dir,
+                                                     alpha, st);
+    } else {
+        if (ub)
+            s = db16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L,
+                                                                    B, d, n_dir, alpha, st)
+                     : launch_bwd_seq<__nv_bfloat16, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
                                                             n_dir, alpha, st);
+        else
+            s = db16 ? launch_bwd_seq<float, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
+                                                            n_dir, alpha, st)
+                     : launch_bwd_seq<float, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d, n_dir,
+                                                    alpha, st);
     }
     if (s != SRU_OK) return s;
+    const int64_t rows = scan ? scan_chunks(L) * B : B;
     const size_t nred = (size_t)n_dir * 4 * d;
-    sru::sru_reduce_dvdb_kernel<<<blocks_for(nred, 256), 256, 0, st>>>(partial, (int)B, (int)d, n_dir, dv, db);
+    sru::sru_reduce_dvdb_kernel<<<blocks_for(nred, 256), 256, 0, st>>>(partial, (int)rows, (int)d, n_dir, dv, db);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }

@@ -26,19 +26,53 @@ constexpr int kRecCJ = 64;   // channels (threads) per CTA
 constexpr int kFwdStages = 4;
 constexpr int kBwdStages = 3;
 
+// Per-channel constants of Eqs. (2)-(3), pre-scaled by -log2(e) so that one
+// FMA gives the exponent of 2 in sigma(z) = 1 / (1 + 2^(-z log2 e)):
+//   nvf = -v_f log2(e), nbf = -b_f log2(e)  (and the same for the reset gate).
 struct GateParams {
-    float vf, vr, bf, br;
+    float vf, vr, bf, br;      // as given (the backward needs v_f, v_r)
+    float nvf, nvr, nbf, nbr;  // scaled by -log2(e)
 };
+constexpr float kNegLog2e = -1.4426950408889634f;
 
-// logistic sigma(z) = 1 / (1 + e^-z), through the CUDA intrinsics (saturates to 0 / 1)
-__device__ __forceinline__ float sigmoid_f(float z) { return __frcp_rn(1.0f + __expf(-z)); }
+__device__ __forceinline__ GateParams make_gate_params(float vf, float vr, float bf, float br) {
+    GateParams p;
+    p.vf = vf;
+    p.vr = vr;
+    p.bf = bf;
+    p.br = br;
+    p.nvf = __fmul_rn(vf, kNegLog2e);
+    p.nvr = __fmul_rn(vr, kNegLog2e);
+    p.nbf = __fmul_rn(bf, kNegLog2e);
+    p.nbr = __fmul_rn(br, kNegLog2e);
+    return p;
+}
+
+// 2^x and 1/x with the single-instruction approximations of the PTX ISA
+// (ex2.approx: relative error ~2^-22; rcp.approx: within 1 ulp).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// logistic sigma(z) given e = -z log2(e): 1 / (1 + 2^e); saturates to exactly 0 and 1.
+__device__ __forceinline__ float sigmoid_nl2(float e) { return rcp_approx(__fadd_rn(1.0f, ex2_approx(e))); }
+// logistic sigma(u + b) for a gate with no peephole term (v = 0)
+__device__ __forceinline__ float sigmoid_f(float z) { return sigmoid_nl2(__fmul_rn(z, kNegLog2e)); }
 
 // One step of Eqs. (2)-(4): returns c[t] from c[t-1], and the gate values.
+// Every operation is explicitly rounded so the forward and the backward's
+// recomputation of a chunk produce bit-identical states.
 __device__ __forceinline__ float sru_cell(float c, float uc, float uf, float ur, const GateParams& p,
                                           float& f, float& r) {
-    f = sigmoid_f(fmaf(p.vf, c, uf + p.bf));
-    r = sigmoid_f(fmaf(p.vr, c, ur + p.br));
-    return fmaf(f, c - uc, uc);
+    f = sigmoid_nl2(__fmaf_rn(p.nvf, c, __fmaf_rn(uf, kNegLog2e, p.nbf)));
+    r = sigmoid_nl2(__fmaf_rn(p.nvr, c, __fmaf_rn(ur, kNegLog2e, p.nbr)));
+    return __fmaf_rn(f, __fsub_rn(c, uc), uc);
 }
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
@@ -80,19 +114,40 @@ __device__ __forceinline__ float fwd_chunk(const UT* __restrict__ us, const floa
                                            uint32_t valid, uint32_t inrange, float c, const GateParams& p,
                                            float alpha, int dir, float* __restrict__ hp, size_t h_tstride,
                                            bool jok, int tid) {
+    constexpr uint32_t kFull = (1u << kChunkT) - 1u;
+    if (valid == kFull) {  // every row present and unpadded: no per-row predicates
+        if (dir == 0) {
+#pragma unroll
+            for (int i = 0; i < kChunkT; ++i) {
+                float f, r;
+                c = sru_cell(c, to_f32(us[(i * 3 + 0) * kRecCJ + tid]), to_f32(us[(i * 3 + 1) * kRecCJ + tid]),
+                             to_f32(us[(i * 3 + 2) * kRecCJ + tid]), p, f, r);
+                const float ax = __fmul_rn(alpha, xs[i * kRecCJ + tid]);
+                if (jok) hp[(size_t)i * h_tstride] = __fmaf_rn(r, __fsub_rn(c, ax), ax);  // Eq. (5)
+            }
+        } else {
+#pragma unroll
+            for (int i = kChunkT - 1; i >= 0; --i) {
+                float f, r;
+                c = sru_cell(c, to_f32(us[(i * 3 + 0) * kRecCJ + tid]), to_f32(us[(i * 3 + 1) * kRecCJ + tid]),
+                             to_f32(us[(i * 3 + 2) * kRecCJ + tid]), p, f, r);
+                const float ax = __fmul_rn(alpha, xs[i * kRecCJ + tid]);
+                if (jok) hp[(size_t)i * h_tstride] = __fmaf_rn(r, __fsub_rn(c, ax), ax);
+            }
+        }
+        return c;
+    }
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
         const int i = dir == 0 ? q : kChunkT - 1 - q;
         if (!((inrange >> i) & 1u)) continue;
         float hv = 0.f;
         if ((valid >> i) & 1u) {
-            const float uc = to_f32(us[(i * 3 + 0) * kRecCJ + tid]);
-            const float uf = to_f32(us[(i * 3 + 1) * kRecCJ + tid]);
-            const float ur = to_f32(us[(i * 3 + 2) * kRecCJ + tid]);
-            const float ax = alpha * xs[i * kRecCJ + tid];
             float f, r;
-            c = sru_cell(c, uc, uf, ur, p, f, r);
-            hv = fmaf(r, c - ax, ax);  // Eq. (5): r*c + (1-r)*alpha*x
+            c = sru_cell(c, to_f32(us[(i * 3 + 0) * kRecCJ + tid]), to_f32(us[(i * 3 + 1) * kRecCJ + tid]),
+                         to_f32(us[(i * 3 + 2) * kRecCJ + tid]), p, f, r);
+            const float ax = __fmul_rn(alpha, xs[i * kRecCJ + tid]);
+            hv = __fmaf_rn(r, __fsub_rn(c, ax), ax);  // Eq. (5): r*c + (1-r)*alpha*x
         }
         if (jok) hp[(size_t)i * h_tstride] = hv;
     }
@@ -129,13 +184,11 @@ __global__ void __launch_bounds__(kRecCJ) sru_fwd_seq_kernel(
     const bool jok = j < d;
     const int nch = (L + kChunkT - 1) / kChunkT;
 
-    GateParams p{0.f, 0.f, 0.f, 0.f};
+    GateParams p = make_gate_params(0.f, 0.f, 0.f, 0.f);
     float c = 0.f;
     if (jok) {
-        p.vf = v[(dir * 2 + 0) * d + j];
-        p.vr = v[(dir * 2 + 1) * d + j];
-        p.bf = bias[(dir * 2 + 0) * d + j];
-        p.br = bias[(dir * 2 + 1) * d + j];
+        p = make_gate_params(v[(dir * 2 + 0) * d + j], v[(dir * 2 + 1) * d + j], bias[(dir * 2 + 0) * d + j],
+                             bias[(dir * 2 + 1) * d + j]);
         if (c0 != nullptr) c = c0[(size_t)bd * d + j];
     }
     if (tid == 0) {
@@ -204,6 +257,8 @@ __device__ __forceinline__ void bwd_chunk(const UT* __restrict__ us, const float
                                           float alpha, float& g, double (&acc)[4], DUT* __restrict__ dUp,
                                           float* __restrict__ dxp, size_t u_tstride, size_t x_tstride, int d,
                                           bool jok, int tid) {
+    constexpr uint32_t kFull = (1u << kChunkT) - 1u;
+    const bool full = valid == kFull;
     float cp[kChunkT], fs[kChunkT], rs[kChunkT];
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
@@ -211,47 +266,51 @@ __device__ __forceinline__ void bwd_chunk(const UT* __restrict__ us, const float
         cp[i] = c;
         fs[i] = 0.f;
         rs[i] = 0.f;
-        if ((valid >> i) & 1u) {
-            const float uc = to_f32(us[(i * 3 + 0) * kRecCJ + tid]);
-            const float uf = to_f32(us[(i * 3 + 1) * kRecCJ + tid]);
-            const float ur = to_f32(us[(i * 3 + 2) * kRecCJ + tid]);
-            c = sru_cell(c, uc, uf, ur, p, fs[i], rs[i]);
-        }
+        if (full || ((valid >> i) & 1u))
+            c = sru_cell(c, to_f32(us[(i * 3 + 0) * kRecCJ + tid]), to_f32(us[(i * 3 + 1) * kRecCJ + tid]),
+                         to_f32(us[(i * 3 + 2) * kRecCJ + tid]), p, fs[i], rs[i]);
     }
+    // chunk partial sums in fp32 (16 terms), folded into the double totals once per chunk
+    float s_vf = 0.f, s_vr = 0.f, s_bf = 0.f, s_br = 0.f;
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
         const int i = DIR == 0 ? kChunkT - 1 - q : q;
-        if (!((inrange >> i) & 1u)) continue;
+        if (!full && !((inrange >> i) & 1u)) continue;
         float duc = 0.f, dzf = 0.f, dzr = 0.f, dxv = 0.f;
-        if ((valid >> i) & 1u) {
+        const bool row = full || ((valid >> i) & 1u);
+        if (row) {
             const float f = fs[i], r = rs[i], cpv = cp[i];
             const float uc = to_f32(us[(i * 3 + 0) * kRecCJ + tid]);
-            const float ax = alpha * xs[i * kRecCJ + tid];
+            const float ax = __fmul_rn(alpha, xs[i * kRecCJ + tid]);
             const float dhv = dhs[i * kRecCJ + tid];
-            const float cn = fmaf(f, cpv - uc, uc);
-            const float G = fmaf(dhv, r, g);  // dLoss/dc[t]
-            const float d_r = dhv * (cn - ax);
-            dxv = dhv * (1.f - r) * alpha;
-            dzf = G * (cpv - uc) * (f * (1.f - f));
-            dzr = d_r * (r * (1.f - r));
-            duc = G * (1.f - f);
-            g = fmaf(dzr, p.vr, fmaf(dzf, p.vf, G * f));  // dLoss/dc[t-1]
-            acc[0] += (double)(dzf * cpv);
-            acc[1] += (double)(dzr * cpv);
-            acc[2] += (double)dzf;
-            acc[3] += (double)dzr;
+            const float cn = __fmaf_rn(f, __fsub_rn(cpv, uc), uc);
+            const float G = __fmaf_rn(dhv, r, g);  // dLoss/dc[t]
+            const float omr = __fsub_rn(1.f, r), omf = __fsub_rn(1.f, f);
+            dxv = __fmul_rn(__fmul_rn(dhv, omr), alpha);
+            dzf = __fmul_rn(__fmul_rn(G, __fsub_rn(cpv, uc)), __fmul_rn(f, omf));
+            dzr = __fmul_rn(__fmul_rn(dhv, __fsub_rn(cn, ax)), __fmul_rn(r, omr));
+            duc = __fmul_rn(G, omf);
+            g = __fmaf_rn(dzr, p.vr, __fmaf_rn(dzf, p.vf, __fmul_rn(G, f)));  // dLoss/dc[t-1]
+            s_vf = __fmaf_rn(dzf, cpv, s_vf);
+            s_vr = __fmaf_rn(dzr, cpv, s_vr);
+            s_bf = __fadd_rn(s_bf, dzf);
+            s_br = __fadd_rn(s_br, dzr);
         }
         if (jok) {
             dUp[(size_t)i * u_tstride] = from_f32<DUT>(duc);
             dUp[(size_t)i * u_tstride + d] = from_f32<DUT>(dzf);
             dUp[(size_t)i * u_tstride + 2 * d] = from_f32<DUT>(dzr);
             if (ACC_DX) {
-                if ((valid >> i) & 1u) dxp[(size_t)i * x_tstride] = dxin[i * kRecCJ + tid] + dxv;
+                if (row) dxp[(size_t)i * x_tstride] = __fadd_rn(dxin[i * kRecCJ + tid], dxv);
             } else {
                 dxp[(size_t)i * x_tstride] = dxv;
             }
         }
     }
+    acc[0] += (double)s_vf;
+    acc[1] += (double)s_vr;
+    acc[2] += (double)s_bf;
+    acc[3] += (double)s_br;
 }
 
 // A chunk with no valid row: zero dU (and dx unless accumulating); g passes through.
@@ -305,13 +364,11 @@ __global__ void __launch_bounds__(kRecCJ) sru_bwd_seq_kernel(
     const bool jok = j < d;
     const int nch = (L + kChunkT - 1) / kChunkT;
 
-    GateParams p{0.f, 0.f, 0.f, 0.f};
+    GateParams p = make_gate_params(0.f, 0.f, 0.f, 0.f);
     float g = 0.f;
     if (jok) {
-        p.vf = v[(dir * 2 + 0) * d + j];
-        p.vr = v[(dir * 2 + 1) * d + j];
-        p.bf = bias[(dir * 2 + 0) * d + j];
-        p.br = bias[(dir * 2 + 1) * d + j];
+        p = make_gate_params(v[(dir * 2 + 0) * d + j], v[(dir * 2 + 1) * d + j], bias[(dir * 2 + 0) * d + j],
+                             bias[(dir * 2 + 1) * d + j]);
         if (dc_T != nullptr) g = dc_T[(size_t)bd * d + j];
     }
     if (tid == 0) {

@@ -1,0 +1,394 @@
+// sru_scan.cuh -- the linear case v = 0 of the SRU recurrence as a chunked
+// associative scan over t.
+//
+// With v_f = v_r = 0 the gates of Eqs. (2)-(3) no longer read c[t-1]
+// ("When Attention Meets Fast Recurrence", background section on SRU), so
+// Eq. (4) is a first-order linear recurrence c[t] = f[t] c[t-1] + (1-f[t]) u[t]
+// and a chunk of steps acts on the state as an affine map c -> A c + Bc with
+// A = prod f.  Linear recurrent layers can be trained in parallel over time
+// ("Parallelizing Legendre Memory Unit Training", abstract); here time is cut
+// into chunks of kScanT steps so that B*d channels x L/kScanT chunks of work
+// exist even when B*d alone cannot fill the GPU.
+//
+// One CTA = one (chunk, 64-channel tile).  It stages its chunk in shared
+// memory with TMA, reduces it to (A, Bc), publishes that aggregate, and finds
+// the state entering the chunk by a decoupled look-back over its predecessors
+// (each publishes its aggregate, then its inclusive prefix).  Work items are
+// handed out by an atomic ticket in chunk-major order, so every predecessor a
+// CTA waits on was started earlier by a resident CTA: the waits always end.
+// They are bounded anyway; an expired wait publishes an abort flag that
+// releases every successor, records kErrTimeoutScan and returns.
+// The chunk is then walked again from shared memory with the carried-in state
+// (forward: h, checkpoints; backward: dU, dx, dv/db partials).
+// The backward uses the same scheme on the state gradient, which for v = 0 is
+// the linear recurrence g[t-1] = f[t] (g[t] + dh[t] r[t]).
+#pragma once
+
+#include "sru_recurrence.cuh"
+
+namespace sru {
+
+constexpr int kScanSub = 4;                 // 16-step sub-chunks per scan chunk
+constexpr int kScanT = kScanSub * kChunkT;  // steps per scan chunk
+
+enum ScanFlag : unsigned { kFlagNone = 0, kFlagAgg = 1, kFlagPrefix = 2, kFlagAbort = 3 };
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ float ld_relaxed_gpu(const float* p) {
+    float v;
+    asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+    return v;
+}
+
+struct ScanState {
+    unsigned* flags;  // n_items flags, then the ticket counter
+    float* agg_a;     // n_items * CJ
+    float* agg_b;
+    float* prefix;
+};
+
+// Whole CTA: publish this item's value(s) (already stored by every thread) under flag f.
+__device__ __forceinline__ void scan_publish(unsigned* flag, unsigned f) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        st_release_gpu(flag, f);
+    }
+}
+
+// Whole CTA: wait (bounded) until flag != 0; returns its value (kFlagAbort on timeout).
+__device__ __forceinline__ unsigned scan_wait_flag(const unsigned* flag, unsigned* s_flag) {
+    if (threadIdx.x == 0) {
+        unsigned f = ld_acquire_gpu(flag);
+        if (f == kFlagNone) {
+            const uint64_t t0 = globaltimer_ns();
+            while ((f = ld_acquire_gpu(flag)) == kFlagNone) {
+                if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                    record_error(kErrTimeoutScan);
+                    f = kFlagAbort;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        *s_flag = f;
+    }
+    __syncthreads();
+    const unsigned f = *s_flag;
+    __syncthreads();
+    return f;
+}
+
+// Decoupled look-back: the composition of the affine maps of items
+// k-1, k-2, ... (same tile) applied to the first available inclusive prefix.
+// Returns false on abort.
+__device__ __forceinline__ bool scan_lookback(const ScanState& ss, int k, int tile, int n_tiles, int tid,
+                                              unsigned* s_flag, float& carry) {
+    float a_acc = 1.f, b_acc = 0.f;
+    for (int p = k - 1; p >= 0; --p) {
+        const size_t item = (size_t)p * n_tiles + tile;
+        const unsigned f = scan_wait_flag(&ss.flags[item], s_flag);
+        if (f == kFlagAbort) return false;
+        if (f == kFlagPrefix) {
+            carry = fmaf(a_acc, ld_relaxed_gpu(&ss.prefix[item * kRecCJ + tid]), b_acc);
+            return true;
+        }
+        const float a = ld_relaxed_gpu(&ss.agg_a[item * kRecCJ + tid]);
+        const float bb = ld_relaxed_gpu(&ss.agg_b[item * kRecCJ + tid]);
+        b_acc = fmaf(a_acc, bb, b_acc);
+        a_acc *= a;
+    }
+    carry = b_acc;  // unreachable in practice: item 0 always publishes a prefix
+    return true;
+}
+
+// Zero the flags and the ticket counter before a scan launch.
+__global__ void sru_scan_reset_kernel(unsigned* __restrict__ flags, int n) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) flags[i] = 0u;
+}
+
+template <typename UT>
+struct FwdScanLayout {
+    static constexpr int STAGE = FwdLayout<UT>::STAGE;
+    static constexpr int BAR_OFF = kScanSub * STAGE;
+    static constexpr int SMEM = BAR_OFF + 64 + 128;
+};
+
+// Forward, v = 0.  1-D grid of n_items = ceil(L/kScanT) * ceil(d/CJ) * B * n_dir CTAs.
+template <typename UT>
+__global__ void __launch_bounds__(kRecCJ) sru_fwd_scan_kernel(
+    const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
+    const float* __restrict__ bias, const float* __restrict__ c0, const uint8_t* __restrict__ mask,
+    float* __restrict__ h, float* __restrict__ c_T, float* __restrict__ ckpt, ScanState ss, int L, int B, int d,
+    int n_dir, float alpha) {
+    using Lay = FwdScanLayout<UT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
+    unsigned* s_misc = reinterpret_cast<unsigned*>(bar + 1);  // [0] ticket, [1] flag
+
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int n_jt = (d + kRecCJ - 1) / kRecCJ;
+    const int n_tiles = n_jt * B * n_dir;
+    const int n_items = gridDim.x;
+    if (tid == 0) {
+        s_misc[0] = atomicAdd(&ss.flags[n_items], 1u);
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int w = (int)s_misc[0];
+    const int k = w / n_tiles, tile = w % n_tiles;
+    const int jt = tile % n_jt, bd = tile / n_jt;
+    const int b = bd / n_dir, dir = bd % n_dir;
+    const int nchs = (L + kScanT - 1) / kScanT;
+    const int tc = dir == 0 ? k : nchs - 1 - k;
+    const int t0 = tc * kScanT;
+    const int j0 = jt * kRecCJ, j = j0 + tid;
+    const bool jok = j < d;
+    const int nch16 = (L + kChunkT - 1) / kChunkT;
+
+    GateParams p = make_gate_params(0.f, 0.f, 0.f, 0.f);
+    if (jok) p = make_gate_params(0.f, 0.f, bias[(dir * 2 + 0) * d + j], bias[(dir * 2 + 1) * d + j]);
+    uint32_t valid[kScanSub], inrange[kScanSub];
+    bool any = false;
+#pragma unroll
+    for (int q = 0; q < kScanSub; ++q) {
+        const int ts = t0 + q * kChunkT;
+        valid[q] = ts < L ? chunk_valid_bits(mask, ts, L, B, b, lane) : 0u;
+        inrange[q] = ts < L ? chunk_inrange_bits(ts, L) : 0u;
+        any |= valid[q] != 0u;
+    }
+    if (tid == 0 && any) {
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int q = 0; q < kScanSub; ++q) bytes += valid[q] ? (uint32_t)Lay::STAGE : 0u;
+        mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+        for (int q = 0; q < kScanSub; ++q) {
+            if (!valid[q]) continue;
+            uint8_t* st = smem + q * Lay::STAGE;
+            tma_load_4d(st, &map_u, bar, j0, 0, bd, t0 + q * kChunkT);
+            tma_load_3d(st + FwdLayout<UT>::U_BYTES, &map_x, bar, j0, b, t0 + q * kChunkT);
+        }
+    }
+    if (any) {
+        const bool ok = mbar_wait(bar, 0, kErrTimeoutLoad);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) mbar_wait(bar, 0, kErrTimeoutLoad);
+            scan_publish(&ss.flags[w], kFlagAbort);
+            return;
+        }
+    }
+
+    // 1. the chunk as an affine map of the entering state: c_out = A c_in + Bc
+    float A = 1.f, Bc = 0.f;
+#pragma unroll
+    for (int qq = 0; qq < kScanSub; ++qq) {
+        const int q = dir == 0 ? qq : kScanSub - 1 - qq;
+        const UT* us = reinterpret_cast<const UT*>(smem + q * Lay::STAGE);
+#pragma unroll
+        for (int r = 0; r < kChunkT; ++r) {
+            const int i = dir == 0 ? r : kChunkT - 1 - r;
+            if ((valid[q] >> i) & 1u) {
+                const float uc = to_f32(us[(i * 3 + 0) * kRecCJ + tid]);
+                const float f = sigmoid_nl2(__fmaf_rn(to_f32(us[(i * 3 + 1) * kRecCJ + tid]), kNegLog2e, p.nbf));
+                A *= f;
+                Bc = fmaf(f, Bc - uc, uc);
+            }
+        }
+    }
+    // 2. state entering the chunk
+    float c_in = 0.f;
+    const size_t me = (size_t)w * kRecCJ + tid;
+    if (k == 0) {
+        c_in = (jok && c0 != nullptr) ? c0[(size_t)bd * d + j] : 0.f;
+    } else {
+        ss.agg_a[me] = A;
+        ss.agg_b[me] = Bc;
+        scan_publish(&ss.flags[w], kFlagAgg);
+        if (!scan_lookback(ss, k, tile, n_tiles, tid, s_misc + 1, c_in)) {
+            scan_publish(&ss.flags[w], kFlagAbort);
+            return;
+        }
+    }
+    ss.prefix[me] = fmaf(A, c_in, Bc);
+    scan_publish(&ss.flags[w], kFlagPrefix);
+
+    // 3. walk the chunk again from shared memory: h and the 16-step checkpoints
+    float c = c_in;
+    const size_t h_tstride = (size_t)B * n_dir * d;
+#pragma unroll
+    for (int qq = 0; qq < kScanSub; ++qq) {
+        const int q = dir == 0 ? qq : kScanSub - 1 - qq;
+        const int ts = t0 + q * kChunkT;
+        if (ts >= L) continue;
+        const int c16 = tc * kScanSub + q;
+        if (ckpt != nullptr && jok && c16 < nch16) ckpt[((size_t)c16 * B * n_dir + bd) * d + j] = c;
+        const UT* us = reinterpret_cast<const UT*>(smem + q * Lay::STAGE);
+        const float* xs = reinterpret_cast<const float*>(smem + q * Lay::STAGE + FwdLayout<UT>::U_BYTES);
+        float* hp = h + (size_t)ts * h_tstride + (size_t)bd * d + j;
+        c = fwd_chunk<UT>(us, xs, valid[q], inrange[q], c, p, alpha, dir, hp, h_tstride, jok, tid);
+    }
+    if (k == nchs - 1 && jok) c_T[(size_t)bd * d + j] = c;
+}
+
+template <typename UT, bool ACC_DX>
+struct BwdScanLayout {
+    static constexpr int STAGE = BwdLayout<UT, ACC_DX>::STAGE;
+    static constexpr int BAR_OFF = kScanSub * STAGE;
+    static constexpr int SMEM = BAR_OFF + 64 + 128;
+};
+
+// Backward of direction DIR, v = 0.  1-D grid of n_items = ceil(L/kScanT) * ceil(d/CJ) * B.
+// partial: (nchs * B, n_dir, 4, d) doubles.
+template <typename UT, typename DUT, bool ACC_DX, int DIR>
+__global__ void __launch_bounds__(kRecCJ) sru_bwd_scan_kernel(
+    const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
+    const __grid_constant__ CUtensorMap map_dh, const __grid_constant__ CUtensorMap map_dxin,
+    const float* __restrict__ bias, const uint8_t* __restrict__ mask, const float* __restrict__ ckpt,
+    const float* __restrict__ dc_T, DUT* __restrict__ dU, float* __restrict__ dx, double* __restrict__ partial,
+    float* __restrict__ dc0, ScanState ss, int L, int B, int d, int n_dir, float alpha) {
+    using Lay = BwdScanLayout<UT, ACC_DX>;
+    using SL = BwdLayout<UT, ACC_DX>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
+    unsigned* s_misc = reinterpret_cast<unsigned*>(bar + 1);
+
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int n_jt = (d + kRecCJ - 1) / kRecCJ;
+    const int n_tiles = n_jt * B;
+    const int n_items = gridDim.x;
+    if (tid == 0) {
+        s_misc[0] = atomicAdd(&ss.flags[n_items], 1u);
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int w = (int)s_misc[0];
+    const int k = w / n_tiles, tile = w % n_tiles;
+    const int jt = tile % n_jt, b = tile / n_jt;
+    const int bd = b * n_dir + DIR;
+    const int nchs = (L + kScanT - 1) / kScanT;
+    const int tc = DIR == 0 ? nchs - 1 - k : k;  // backward walks direction 0 from the end
+    const int t0 = tc * kScanT;
+    const int j0 = jt * kRecCJ, j = j0 + tid;
+    const bool jok = j < d;
+
+    GateParams p = make_gate_params(0.f, 0.f, 0.f, 0.f);
+    if (jok) p = make_gate_params(0.f, 0.f, bias[(DIR * 2 + 0) * d + j], bias[(DIR * 2 + 1) * d + j]);
+    uint32_t valid[kScanSub], inrange[kScanSub];
+    bool any = false;
+#pragma unroll
+    for (int q = 0; q < kScanSub; ++q) {
+        const int ts = t0 + q * kChunkT;
+        valid[q] = ts < L ? chunk_valid_bits(mask, ts, L, B, b, lane) : 0u;
+        inrange[q] = ts < L ? chunk_inrange_bits(ts, L) : 0u;
+        any |= valid[q] != 0u;
+    }
+    if (tid == 0 && any) {
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int q = 0; q < kScanSub; ++q) bytes += valid[q] ? (uint32_t)SL::STAGE : 0u;
+        mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+        for (int q = 0; q < kScanSub; ++q) {
+            if (!valid[q]) continue;
+            uint8_t* st = smem + q * SL::STAGE;
+            const int ts = t0 + q * kChunkT;
+            tma_load_4d(st, &map_u, bar, j0, 0, bd, ts);
+            tma_load_3d(st + SL::U_BYTES, &map_x, bar, j0, b, ts);
+            tma_load_3d(st + SL::U_BYTES + SL::V_BYTES, &map_dh, bar, j0, bd, ts);
+            if (ACC_DX) tma_load_3d(st + SL::U_BYTES + 2 * SL::V_BYTES, &map_dxin, bar, j0, b, ts);
+        }
+    }
+    if (any) {
+        const bool ok = mbar_wait(bar, 0, kErrTimeoutLoad);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) mbar_wait(bar, 0, kErrTimeoutLoad);
+            scan_publish(&ss.flags[w], kFlagAbort);
+            return;
+        }
+    }
+
+    // 1. the chunk as an affine map of the state gradient: g_out = A g_in + Bg,
+    //    g <- f (g + dh r) per valid row, in backward order
+    float A = 1.f, Bg = 0.f;
+#pragma unroll
+    for (int qq = 0; qq < kScanSub; ++qq) {
+        const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
+        const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
+        const float* dhs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES + SL::V_BYTES);
+#pragma unroll
+        for (int r = 0; r < kChunkT; ++r) {
+            const int i = DIR == 0 ? kChunkT - 1 - r : r;
+            if ((valid[q] >> i) & 1u) {
+                const float f = sigmoid_nl2(__fmaf_rn(to_f32(us[(i * 3 + 1) * kRecCJ + tid]), kNegLog2e, p.nbf));
+                const float rr = sigmoid_nl2(__fmaf_rn(to_f32(us[(i * 3 + 2) * kRecCJ + tid]), kNegLog2e, p.nbr));
+                A *= f;
+                Bg = f * fmaf(dhs[i * kRecCJ + tid], rr, Bg);
+            }
+        }
+    }
+    // 2. state gradient entering the chunk (from later times)
+    float g_in = 0.f;
+    const size_t me = (size_t)w * kRecCJ + tid;
+    if (k == 0) {
+        g_in = (jok && dc_T != nullptr) ? dc_T[(size_t)bd * d + j] : 0.f;
+    } else {
+        ss.agg_a[me] = A;
+        ss.agg_b[me] = Bg;
+        scan_publish(&ss.flags[w], kFlagAgg);
+        if (!scan_lookback(ss, k, tile, n_tiles, tid, s_misc + 1, g_in)) {
+            scan_publish(&ss.flags[w], kFlagAbort);
+            return;
+        }
+    }
+    ss.prefix[me] = fmaf(A, g_in, Bg);
+    scan_publish(&ss.flags[w], kFlagPrefix);
+
+    // 3. gradients of every row, sub-chunk by sub-chunk in backward order
+    float g = g_in;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    const size_t u_tstride = (size_t)B * n_dir * 3 * d;
+    const size_t x_tstride = (size_t)B * d;
+#pragma unroll
+    for (int qq = 0; qq < kScanSub; ++qq) {
+        const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
+        const int ts = t0 + q * kChunkT;
+        if (ts >= L) continue;
+        DUT* dUp = dU + (size_t)ts * u_tstride + (size_t)bd * 3 * d + j;
+        float* dxp = dx + (size_t)ts * x_tstride + (size_t)b * d + j;
+        if (valid[q] == 0u) {
+            bwd_chunk_padded<DUT, ACC_DX>(inrange[q], dUp, dxp, u_tstride, x_tstride, d, jok);
+            continue;
+        }
+        const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
+        const float* xs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES);
+        const float* dhs = xs + kChunkT * kRecCJ;
+        const float* dxin = dhs + kChunkT * kRecCJ;
+        const int c16 = tc * kScanSub + q;
+        const float c_start = jok ? ckpt[((size_t)c16 * B * n_dir + bd) * d + j] : 0.f;
+        bwd_chunk<UT, DUT, ACC_DX, DIR>(us, xs, dhs, dxin, valid[q], inrange[q], c_start, p, alpha, g, acc, dUp,
+                                        dxp, u_tstride, x_tstride, d, jok, tid);
+    }
+    if (jok) {
+        if (k == nchs - 1) dc0[(size_t)bd * d + j] = g;
+        double* pp = partial + (((size_t)tc * B + b) * n_dir + DIR) * 4 * d + j;
+        pp[0] = acc[0];
+        pp[(size_t)d] = acc[1];
+        pp[(size_t)2 * d] = acc[2];
+        pp[(size_t)3 * d] = acc[3];
+    }
+}
+
+}  // namespace sru

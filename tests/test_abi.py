@@ -67,16 +67,16 @@ def test_invalid_arguments_return_before_any_launch(lib):
     vp = ctypes.c_void_p
     fake = vp(0x1000)
     # d not a multiple of 8
-    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4, 2, 12, 1.0, 0, 0, fake, fake, None, None)
+    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4, 2, 12, 1.0, 0, 0, fake, fake, None, 0, None)
     assert st == 4
     # negative sizes
-    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, -1, 2, 16, 1.0, 0, 0, fake, fake, None, None)
+    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, -1, 2, 16, 1.0, 0, 0, fake, fake, None, 0, None)
     assert st == 1
     # unknown U dtype
-    st = lib.sru_forward(fake, 7, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, fake, None, None)
+    st = lib.sru_forward(fake, 7, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, fake, None, 0, None)
     assert st == 1
     # null outputs
-    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, None, None, None, None)
+    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, None, None, None, 0, None)
     assert st == 1
     # misaligned pointer
     st = lib.sru_project(vp(0x1001), 1, fake, 1, fake, 1, 64, 64, 64, None)
@@ -85,6 +85,17 @@ def test_invalid_arguments_return_before_any_launch(lib):
     st = lib.sru_project(fake, 0, fake, 1, fake, 1, 64, 64, 64, None)
     assert st == 1
     # backward without a workspace
-    st = lib.sru_backward(fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, None, None,
+    st = lib.sru_backward(fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, None, None, 0,
                           fake, 1, fake, fake, fake, fake, None)
+    assert st == 1
+    # a workspace smaller than sru_workspace_bytes reports
+    need = lib.sru_workspace_bytes(4, 2, 16, 0, 0)
+    st = lib.sru_backward(fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, None, fake, need - 1,
+                          fake, 1, fake, fake, fake, fake, None)
+    assert st == 1
+    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, fake, fake, need - 1, None)
+    assert st == 1
+    # the scan path needs a workspace sized with SRU_FLAG_V_ZERO
+    assert lib.sru_workspace_bytes(4096, 2, 64, 0, 1) > lib.sru_workspace_bytes(4096, 2, 64, 0, 0)
+    st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4096, 2, 64, 1.0, 0, 1 | 2, fake, fake, None, 0, None)
     assert st == 1

@@ -37,11 +37,14 @@ def _sample_channels(rng, d, n=N_CHANNELS):
     return np.sort(rng.choice(d, size=min(n, d), replace=False))
 
 
-@pytest.mark.parametrize("name", ["lm_fwd", "lm_train", "bidir_masked", "rec_only", "rec_only_v0"])
-def test_recurrence_full_size(sru, name):
+@pytest.mark.parametrize("name,force_scan", [("lm_fwd", False), ("lm_train", False), ("bidir_masked", False),
+                                             ("rec_only", False), ("rec_only_v0", False), ("rec_only_v0", True)])
+def test_recurrence_full_size(sru, name, force_scan):
     cfg = CONFIGS[name]
     inp = generate(cfg, u_direct=True)
     flags = sru.SRU_FLAG_V_ZERO if cfg.v_zero else 0
+    if force_scan:
+        flags |= sru.SRU_FLAG_FORCE_SCAN
     gpu = tl.run_gpu_recurrence(sru, inp, cfg.n_dir, cfg.alpha, du_dtype=torch.bfloat16, flags=flags,
                                 backward=cfg.backward)
     rng = np.random.default_rng(1000 + cfg.seed)
@@ -109,12 +112,10 @@ def test_projection_backward_full_size(sru, name):
     adU = tl.abs_operand(dUb)
     ref = oracle.project_dX_entries(dUb, inp["W"], rows, cols) + hw[rows, cols]
     absref = oracle.project_dX_entries(adU, tl.abs_operand(inp["W"]), rows, cols) + np.abs(hw[rows, cols])
-    tl.assert_close("dX sampled (bf16 class)", tl.host_f64(dX)[rows, cols], ref, tl.BF16_TOL)
     tl.assert_close_sum("dX sampled", tl.host_f64(dX)[rows, cols], ref, absref)
     rows, cols = rng.integers(0, N, N_ENTRIES), rng.integers(0, d, N_ENTRIES)
     ref = oracle.project_dW_entries(dUb, inp["X"], rows, cols)
     absref = oracle.project_dW_entries(adU, tl.abs_operand(inp["X"]), rows, cols)
-    tl.assert_close("dW sampled (bf16 class)", tl.host_f64(dW)[rows, cols], ref, tl.BF16_TOL)
     tl.assert_close_sum("dW sampled", tl.host_f64(dW)[rows, cols], ref, absref)
 
 

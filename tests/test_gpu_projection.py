@@ -14,10 +14,12 @@ from synthetic import bf16_bits_to_f32, f32_to_bf16_bits
 
 pytestmark = pytest.mark.gpu
 
-# Products with fp32 outputs are checked twice: in the bf16-projection class
-# 2e-2 * (1 + |ref|), and against a bound that scales with sum_k |a_k b_k|
-# (the size of an fp32 sum's rounding error), which a dropped or misplaced
-# k-slice exceeds by orders of magnitude.
+# Products with fp32 outputs (dX, dW, fp32 U) are long sums: their rounding
+# error grows with sum_k |a_k b_k|, not with |ref| (which cancellation can make
+# arbitrarily small), so they are checked against
+#   |gpu - ref| <= 1e-5 * (1 + |ref|) + 1e-5 * sum_k |a_k b_k|,
+# a bound that a dropped or misplaced k-slice exceeds by orders of magnitude.
+# bf16 outputs (U) are also checked within one bf16 ulp and in the 2e-2 class.
 
 
 @pytest.fixture(scope="module")
@@ -66,8 +68,6 @@ def test_project_backward_bf16(sru, M, N, K, accumulate):
     assert sru.sru_sync_status() == 0
     abs_dX = oracle.project_dX(tl.abs_operand(dUb), tl.abs_operand(Wb)) + (np.abs(base) if accumulate else 0.0)
     abs_dW = oracle.project_dW(tl.abs_operand(dUb), tl.abs_operand(Xb))
-    tl.assert_close("dX (bf16 class)", tl.host_f64(dX), ref_dX, tl.BF16_TOL)
-    tl.assert_close("dW (bf16 class)", tl.host_f64(dW), ref_dW, tl.BF16_TOL)
     tl.assert_close_sum("dX", tl.host_f64(dX), ref_dX, abs_dX)
     tl.assert_close_sum("dW", tl.host_f64(dW), ref_dW, abs_dW)
 
@@ -101,5 +101,4 @@ def test_project_large_k_sampled(sru):
     rows, cols = rng.integers(0, N, 2048), rng.integers(0, K, 2048)
     ref = oracle.project_dW_entries(dUb, Xb, rows, cols)
     absref = oracle.project_dW_entries(tl.abs_operand(dUb), tl.abs_operand(Xb), rows, cols)
-    tl.assert_close("dW sampled (bf16 class)", tl.host_f64(dW)[rows, cols], ref, tl.BF16_TOL)
     tl.assert_close_sum("dW sampled", tl.host_f64(dW)[rows, cols], ref, absref)

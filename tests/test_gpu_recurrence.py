@@ -123,3 +123,31 @@ def test_invalid_arguments_are_rejected(sru):
     with pytest.raises(sru.SRUError) as e:
         sru.sru_forward(U, x, v, v, torch.zeros(4, 2, 1, 12, device="cuda"), torch.zeros(2, 1, 12, device="cuda"))
     assert e.value.status == sru.SRU_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("n_dir,masked", [(1, False), (2, True), (1, True)])
+@pytest.mark.parametrize("L", [1, 37, 200])
+@pytest.mark.parametrize("du_dtype", [torch.float32, torch.bfloat16])
+def test_scan_path_matches_oracle(sru, n_dir, masked, L, du_dtype):
+    """v = 0 through the chunked associative scan (forced), against the oracle."""
+    cfg = _cfg(L=L, B=3, d=200, n_dir=n_dir, masked=masked, v_zero=True)
+    inp = generate(cfg, u_direct=True)
+    if masked and L > 5:
+        inp["mask"][5, 1] = 1
+    dcT = np.random.default_rng(6).standard_normal((cfg.B, n_dir, cfg.d)).astype(np.float32)
+    flags = sru.SRU_FLAG_V_ZERO | sru.SRU_FLAG_FORCE_SCAN
+    gpu = tl.run_gpu_recurrence(sru, inp, n_dir, 0.75, du_dtype=du_dtype, flags=flags, dc_T=dcT)
+    ref = tl.oracle_recurrence(inp, 0.75, dc_T=dcT)
+    tl.compare_recurrence(gpu, ref, du_bf16=du_dtype == torch.bfloat16)
+
+
+def test_scan_equals_sequential_many_chunks(sru):
+    """Scan and sequential paths agree at v = 0 over many scan chunks (L = 1000, 16 chunks)."""
+    cfg = _cfg(L=1000, B=2, d=128, n_dir=2, masked=True, v_zero=True)
+    inp = generate(cfg, u_direct=True)
+    seq = tl.run_gpu_recurrence(sru, inp, 2, 1.0, flags=sru.SRU_FLAG_V_ZERO | sru.SRU_FLAG_FORCE_SEQUENTIAL)
+    scan = tl.run_gpu_recurrence(sru, inp, 2, 1.0, flags=sru.SRU_FLAG_V_ZERO | sru.SRU_FLAG_FORCE_SCAN)
+    for k in seq:
+        tl.assert_close(k, scan[k], seq[k], tl.REC_TOL)
+    ref = tl.oracle_recurrence(inp, 1.0, bs=np.arange(2), js=np.arange(0, 128, 9))
+    tl.compare_recurrence(scan, ref, bs=np.arange(2), js=np.arange(0, 128, 9))
