@@ -145,6 +145,39 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
                         void* dU, int du_t, float* dx, float* dv, float* db, float* dc0,
                         void* stream);
 
+/*
+ * Allocation-free forward for the linear case v = 0 (the paper has no
+ * counterpart to this entry point; it is a deployment variant of sru_forward).
+ *
+ * Some callers cannot allocate device memory: an inference plugin whose host
+ * framework owns every device buffer and hands the op no scratch, or a
+ * latency-critical loop that must not call cudaMalloc (which can block and
+ * synchronise the device).  This call computes what
+ *   sru_forward(U, u_t, x, v = 0, b, c0, mask, L, B, d, alpha, bidirectional,
+ *               SRU_FLAG_V_ZERO | SRU_FLAG_FORCE_SCAN, h, c_T, NULL workspace)
+ * would (the chunked scan over t, inference only: no checkpoints, so no
+ * sru_backward can follow) without any workspace argument: its scan flags,
+ * ticket and per-chunk aggregates live in an 8 MiB static device array inside
+ * libsru.so, which every GPU that loads the library holds until the process
+ * exits.  The caller still passes all inputs and outputs (same layouts and
+ * rules as sru_forward; v is not read and is taken as 0).
+ *
+ * Limit: ceil(L/64) * ceil(d/64) * B * n_dir work items, each needing 772
+ * bytes of the scratch (about 10 800 items); a larger request returns
+ * SRU_ERR_UNSUPPORTED before anything is launched.
+ * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * call).  Its first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, once per device, with that device current); make
+ * that first call before any stream capture.  Every call zeroes the flags it
+ * uses before launching and otherwise reuses whatever the previous call left
+ * in the array, so calls that overlap on the GPU (concurrent streams, or
+ * several host threads on the same device) race on the shared scratch and
+ * must be serialised by the caller.
+ */
+sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, const float* b,
+                                    const float* c0, const uint8_t* mask, int64_t L, int64_t B, int64_t d,
+                                    float alpha, int bidirectional, float* h, float* c_T, void* stream);
+
 /* Synchronise `stream`, then read and clear the device error word of the
  * current device: SRU_ERR_TIMEOUT if a bounded wait expired since the last
  * call, SRU_ERR_CUDA if the stream reported an error, else SRU_OK. */

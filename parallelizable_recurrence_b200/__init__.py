@@ -30,7 +30,8 @@ SRU_FLAG_FORCE_SEQUENTIAL = 0x4
 
 # every symbol include/sru.h declares
 EXPORTED = ("sru_status_string", "sru_get_last_cuda_error", "sru_version", "sru_workspace_bytes",
-            "sru_project", "sru_project_backward", "sru_forward", "sru_backward", "sru_sync_status")
+            "sru_project", "sru_project_backward", "sru_forward", "sru_backward", "sru_forward_scan_noalloc",
+            "sru_sync_status")
 
 
 class SRUError(RuntimeError):
@@ -75,6 +76,9 @@ def load_library(path: str = LIB_PATH):
     lib.sru_backward.restype = _int
     lib.sru_backward.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _f32, _int, _u32,
                                  _vp, _vp, _vp, ctypes.c_size_t, _vp, _int, _vp, _vp, _vp, _vp, _vp]
+    lib.sru_forward_scan_noalloc.restype = _int
+    lib.sru_forward_scan_noalloc.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _f32, _int,
+                                             _vp, _vp, _vp]
     lib.sru_sync_status.restype = _int
     lib.sru_sync_status.argtypes = [_vp]
     _lib = lib
@@ -181,6 +185,23 @@ def sru_backward(U, x, v, b, dh, workspace, dU, dx, dv, db, dc0, c0=None, mask=N
                             _ptr(db, torch.float32), _ptr(dc0, torch.float32), _stream(stream)),
            "sru_backward")
     return dU, dx, dv, db, dc0
+
+
+def sru_forward_scan_noalloc(U, x, b, h, c_T, c0=None, mask=None, alpha: float = 1.0,
+                             bidirectional: bool = False, stream=None):
+    """Forward for v = 0 with no workspace, for callers that cannot allocate
+    device memory: the scan's scratch is an 8 MiB static array inside libsru.so
+    (shared by every call on a device, so calls must not overlap on the GPU).
+    Inference only (no checkpoints).  Outputs h and c_T are written in place;
+    a request larger than the static scratch raises SRUError (SRU_ERR_UNSUPPORTED)."""
+    lib = load_library()
+    L, B, d = x.shape
+    _check(lib.sru_forward_scan_noalloc(_ptr(U), _dtype_code(U), _ptr(x, torch.float32), _ptr(b, torch.float32),
+                                        _ptr(c0, torch.float32), _ptr(mask, torch.uint8), L, B, d, float(alpha),
+                                        int(bool(bidirectional)), _ptr(h, torch.float32),
+                                        _ptr(c_T, torch.float32), _stream(stream)),
+           "sru_forward_scan_noalloc")
+    return h, c_T
 
 
 def sru_sync_status(stream=None) -> int:

@@ -328,6 +328,49 @@ sru_status launch_bwd_scan(const RecMaps& mp, const float* b, const uint8_t* mas
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Static scratch of the allocation-free entry point sru_forward_scan_noalloc.
+// Every GPU that loads this library holds these 8 MiB until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Scan flags, ticket and aggregates of `items` work items carved from the scratch.
+size_t noalloc_scan_bytes(int64_t items, size_t* agg_a_off, size_t* agg_b_off, size_t* prefix_off) {
+    size_t off = round256((size_t)(items + 1) * sizeof(unsigned));
+    *agg_a_off = off;
+    off += round256((size_t)items * sru::kRecCJ * sizeof(float));
+    *agg_b_off = off;
+    off += round256((size_t)items * sru::kRecCJ * sizeof(float));
+    *prefix_off = off;
+    off += round256((size_t)items * sru::kRecCJ * sizeof(float));
+    return off;
+}
+
+// Device address of the scratch on the current device, looked up once per
+// device.  In host code g_noalloc_scratch names a host-side stand-in, never
+// the device array, so kernels only ever receive this looked-up address.
+cudaError_t noalloc_scratch_address(void** out) {
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
 // =========================================================================
 extern "C" {
 
@@ -530,6 +573,42 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     sru::sru_reduce_dvdb_kernel<<<blocks_for(nred, 256), 256, 0, st>>>(partial, (int)rows, (int)d, n_dir, dv, db);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
+}
+
+sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, const float* b, const float* c0,
+                                    const uint8_t* mask, int64_t L, int64_t B, int64_t d, float alpha,
+                                    int bidirectional, float* h, float* c_T, void* stream) {
+    sru_status s = check_layer_sizes(L, B, d);
+    if (s != SRU_OK) return s;
+    if (u_t != SRU_F32 && u_t != SRU_BF16) return SRU_ERR_INVALID;
+    const int n_dir = bidirectional ? 2 : 1;
+    if (B == 0) return SRU_OK;
+    if (!b || !c_T) return SRU_ERR_INVALID;
+    if (L > 0 && (!U || !x || !h || !aligned16(U) || !aligned16(x) || !aligned16(h))) return SRU_ERR_INVALID;
+    const int64_t items = scan_chunks(L) * ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B * n_dir;
+    size_t agg_a_off = 0, agg_b_off = 0, prefix_off = 0;
+    if (noalloc_scan_bytes(items, &agg_a_off, &agg_b_off, &prefix_off) > kNoAllocScratchBytes)
+        return SRU_ERR_UNSUPPORTED;  // larger than the static scratch
+    cudaStream_t st = as_stream(stream);
+    if (L == 0) {
+        const size_t n = (size_t)B * n_dir * d;
+        sru::sru_copy_state_kernel<<<blocks_for(n, 256), 256, 0, st>>>(c0, c_T, n);
+        SRU_CUDA_TRY(cudaGetLastError());
+        return SRU_OK;
+    }
+    void* scratch = nullptr;
+    SRU_CUDA_TRY(noalloc_scratch_address(&scratch));
+    uint8_t* base = static_cast<uint8_t*>(scratch);
+    sru::ScanState ss;
+    ss.flags = reinterpret_cast<unsigned*>(base);
+    ss.agg_a = reinterpret_cast<float*>(base + agg_a_off);
+    ss.agg_b = reinterpret_cast<float*>(base + agg_b_off);
+    ss.prefix = reinterpret_cast<float*>(base + prefix_off);
+    RecMaps mp;
+    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir) || !map_f32_rows(&mp.x, x, L, B, d)) return SRU_ERR_INVALID;
+    if (u_t == SRU_BF16)
+        return launch_fwd_scan<__nv_bfloat16>(mp, b, c0, mask, h, c_T, nullptr, ss, L, B, d, n_dir, alpha, st);
+    return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, nullptr, ss, L, B, d, n_dir, alpha, st);
 }
 
 sru_status sru_sync_status(void* stream) {
