@@ -222,7 +222,10 @@ def run_ours(args):
     dc0 = torch.empty(B, 1, d, device=dev)
     dW = torch.empty(N, K, device=dev)
     stream = torch.cuda.current_stream(dev)
-    grads = torch.empty(N * K + 4 * d, device=dev) if world > 1 else None
+    reducer = None
+    if world > 1:
+        from parallelizable_recurrence_b200.dist import GradReducer
+        reducer = GradReducer([dW, dv, db])  # one NCCL all-reduce of the parameter gradients
 
     def step(ev=None):
         if ev is not None:
@@ -242,11 +245,8 @@ def run_ours(args):
         sru.sru_project_backward(dU, X, W, dW=dW)
         if ev is not None:
             ev[5].record(stream)
-        if world > 1:  # data-parallel gradient sum (the pages' DDP)
-            grads[:N * K].copy_(dW.view(-1))
-            grads[N * K:N * K + 2 * d].copy_(dv.view(-1))
-            grads[N * K + 2 * d:].copy_(db.view(-1))
-            dist.all_reduce(grads)
+        if reducer is not None:  # data-parallel gradient sum over ranks (batch sharding)
+            reducer()
 
     for _ in range(args.warmup):
         step()

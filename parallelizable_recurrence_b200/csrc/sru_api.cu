@@ -50,6 +50,9 @@ EncodeTiledFn encode_fn() {
 }
 
 // rank-R tiled map; dims/box innermost first; strides (bytes) of dims 1..R-1
+#ifndef SRU_TMA_L2_PROMOTION
+#define SRU_TMA_L2_PROMOTION CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
               const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw) {
     EncodeTiledFn fn = encode_fn();
@@ -57,7 +60,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
                     reinterpret_cast<const cuuint64_t*>(strides), reinterpret_cast<const cuuint32_t*>(box), estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, SRU_TMA_L2_PROMOTION,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -166,14 +169,33 @@ sru_status check_layer_sizes(int64_t L, int64_t B, int64_t d) {
 inline unsigned blocks_for(size_t n, unsigned threads) { return (unsigned)((n + threads - 1) / threads); }
 
 // ------------------------------------------------------------- GEMM launch
+// The CTA-pair kernel (256 x 256 tiles over two SMs) is the default; the
+// single-CTA kernel (128 x 256) remains for comparison builds.
+#ifndef SRU_GEMM_USE_PAIR
+#define SRU_GEMM_USE_PAIR 1
+#endif
+constexpr bool kGemmPair = SRU_GEMM_USE_PAIR != 0;
+// rows of B staged per CTA for a K-major B operand
+constexpr uint32_t kGemmBRows = kGemmPair ? (uint32_t)sru::gemm::P_CN : (uint32_t)sru::gemm::BN;
+
 template <bool A_MN, bool B_MN, int OUT>
 sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
                           int64_t Kr, cudaStream_t st) {
-    auto kern = sru::gemm::tc_gemm_kernel<A_MN, B_MN, OUT>;
-    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::SMEM_BYTES));
-    const int64_t tiles = ((R + sru::gemm::BM - 1) / sru::gemm::BM) * ((C + sru::gemm::BN - 1) / sru::gemm::BN);
-    const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-    kern<<<grid, sru::gemm::THREADS, sru::gemm::SMEM_BYTES, st>>>(ma, mb, out, (int)R, (int)C, (int)Kr, (int)C);
+    if (kGemmPair) {
+        auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT>;
+        SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
+        const int64_t tiles =
+            ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN);
+        const int64_t pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;
+        kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(ma, mb, out, (int)R, (int)C,
+                                                                                       (int)Kr, (int)C);
+    } else {
+        auto kern = sru::gemm::tc_gemm_kernel<A_MN, B_MN, OUT>;
+        SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::SMEM_BYTES));
+        const int64_t tiles = ((R + sru::gemm::BM - 1) / sru::gemm::BM) * ((C + sru::gemm::BN - 1) / sru::gemm::BN);
+        const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+        kern<<<grid, sru::gemm::THREADS, sru::gemm::SMEM_BYTES, st>>>(ma, mb, out, (int)R, (int)C, (int)Kr, (int)C);
+    }
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
@@ -215,62 +237,99 @@ struct RecMaps {
     CUtensorMap u, x, dh, dx;
 };
 
-bool map_u_tensor(CUtensorMap* m, const void* U, int u_t, int64_t L, int64_t B, int64_t d, int n_dir) {
+bool map_u_tensor(CUtensorMap* m, const void* U, int u_t, int64_t L, int64_t B, int64_t d, int n_dir, int cj) {
     const uint64_t es = u_t == SRU_BF16 ? 2 : 4;
     const uint64_t dims[4] = {(uint64_t)d, 3, (uint64_t)(B * n_dir), (uint64_t)L};
     const uint64_t strides[3] = {(uint64_t)d * es, (uint64_t)3 * d * es, (uint64_t)B * n_dir * 3 * d * es};
-    const uint32_t box[4] = {(uint32_t)sru::kRecCJ, 3, 1, (uint32_t)sru::kChunkT};
+    const uint32_t box[4] = {(uint32_t)cj, 3, 1, (uint32_t)sru::kChunkT};
     return make_map(m, u_t == SRU_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, U,
                     dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
-// fp32 (L, rows, d) tensor with tiles (CJ, 1, T)
-bool map_f32_rows(CUtensorMap* m, const float* p, int64_t L, int64_t rows, int64_t d) {
+// fp32 (L, rows, d) tensor with tiles (cj, 1, T)
+bool map_f32_rows(CUtensorMap* m, const float* p, int64_t L, int64_t rows, int64_t d, int cj) {
     const uint64_t dims[3] = {(uint64_t)d, (uint64_t)rows, (uint64_t)L};
     const uint64_t strides[2] = {(uint64_t)d * 4, (uint64_t)rows * d * 4};
-    const uint32_t box[3] = {(uint32_t)sru::kRecCJ, 1, (uint32_t)sru::kChunkT};
+    const uint32_t box[3] = {(uint32_t)cj, 1, (uint32_t)sru::kChunkT};
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-template <typename UT>
-sru_status launch_fwd_seq(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
-                          float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
-                          cudaStream_t st) {
-    using Lay = sru::FwdLayout<UT>;
-    auto kern = sru::sru_fwd_seq_kernel<UT>;
+// Channel-tile width of the sequential kernels.  Measured on B200 for the
+// language-model training layer (L1024 B16 d2048) and the bidirectional
+// layer (L2048 B64 d1024): 64 channels per CTA beat 128 and 256 (wider rows
+// per TMA box gave 4-25% less bandwidth), so 64 is used throughout.
+int pick_seq_cj(int64_t B, int64_t d, int n_dir) {
+    (void)B;
+    (void)d;
+    (void)n_dir;
+#ifdef SRU_FORCE_CJ
+    return SRU_FORCE_CJ;
+#else
+    return 64;
+#endif
+}
+
+template <typename UT, int CJ>
+sru_status launch_fwd_seq_cj(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
+                             float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d, int n_dir,
+                             float alpha, cudaStream_t st) {
+    using Lay = sru::FwdLayout<UT, CJ>;
+    auto kern = sru::sru_fwd_seq_kernel<UT, CJ>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
-    dim3 grid((unsigned)((d + sru::kRecCJ - 1) / sru::kRecCJ), (unsigned)B, (unsigned)n_dir);
-    kern<<<grid, sru::kRecCJ, Lay::SMEM, st>>>(mp.u, mp.x, v, b, c0, mask, h, c_T, ckpt, (int)L, (int)B, (int)d,
-                                               n_dir, alpha);
+    dim3 grid((unsigned)((d + CJ - 1) / CJ), (unsigned)B, (unsigned)n_dir);
+    kern<<<grid, CJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, v, b, c0, mask, h, c_T, ckpt, (int)L, (int)B, (int)d, n_dir,
+                                          alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
 
-template <typename UT, typename DUT, bool ACC, int DIR>
+template <typename UT>
+sru_status launch_fwd_seq(int cj, const RecMaps& mp, const float* v, const float* b, const float* c0,
+                          const uint8_t* mask, float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d,
+                          int n_dir, float alpha, cudaStream_t st) {
+    if (cj == 256) return launch_fwd_seq_cj<UT, 256>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+    if (cj == 128) return launch_fwd_seq_cj<UT, 128>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+    return launch_fwd_seq_cj<UT, 64>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+}
+
+template <typename UT, typename DUT, bool ACC, int DIR, int CJ>
 sru_status launch_bwd_seq_dir(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
                               const float* ckpt, const float* dc_T, DUT* dU, float* dx, double* partial, float* dc0,
                               int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
-    using Lay = sru::BwdLayout<UT, ACC>;
-    auto kern = sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR>;
+    using Lay = sru::BwdLayout<UT, ACC, CJ>;
+    auto kern = sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR, CJ>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
-    dim3 grid((unsigned)((d + sru::kRecCJ - 1) / sru::kRecCJ), (unsigned)B, 1);
-    kern<<<grid, sru::kRecCJ, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.dx, v, b, mask, ckpt, dc_T, dU, dx, partial,
-                                               dc0, (int)L, (int)B, (int)d, n_dir, alpha);
+    dim3 grid((unsigned)((d + CJ - 1) / CJ), (unsigned)B, 1);
+    kern<<<grid, CJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.dx, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
+                                          (int)L, (int)B, (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
 
-template <typename UT, typename DUT>
-sru_status launch_bwd_seq(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask, const float* ckpt,
-                          const float* dc_T, void* dU, float* dx, double* partial, float* dc0, int64_t L, int64_t B,
-                          int64_t d, int n_dir, float alpha, cudaStream_t st) {
-    DUT* du = reinterpret_cast<DUT*>(dU);
-    sru_status s = launch_bwd_seq_dir<UT, DUT, false, 0>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d,
-                                                        n_dir, alpha, st);
+template <typename UT, typename DUT, int CJ>
+sru_status launch_bwd_seq_cj(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
+                             const float* ckpt, const float* dc_T, DUT* du, float* dx, double* partial, float* dc0,
+                             int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
+    sru_status s = launch_bwd_seq_dir<UT, DUT, false, 0, CJ>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B,
+                                                            d, n_dir, alpha, st);
     if (s != SRU_OK || n_dir == 1) return s;
-    return launch_bwd_seq_dir<UT, DUT, true, 1>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir,
-                                               alpha, st);
+    return launch_bwd_seq_dir<UT, DUT, true, 1, CJ>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d,
+                                                   n_dir, alpha, st);
 }
 
+template <typename UT, typename DUT>
+sru_status launch_bwd_seq(int cj, const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
+                          const float* ckpt, const float* dc_T, void* dU, float* dx, double* partial, float* dc0,
+                          int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
+    DUT* du = reinterpret_cast<DUT*>(dU);
+    if (cj == 256)
+        return launch_bwd_seq_cj<UT, DUT, 256>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir,
+                                               alpha, st);
+    if (cj == 128)
+        return launch_bwd_seq_cj<UT, DUT, 128>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir,
+                                               alpha, st);
+    return launch_bwd_seq_cj<UT, DUT, 64>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir, alpha,
+                                          st);
+}
 
 sru_status reset_scan_flags(unsigned* flags, int64_t n, cudaStream_t st) {
     sru::sru_scan_reset_kernel<<<blocks_for((size_t)n, 256), 256, 0, st>>>(flags, (int)n);
@@ -289,7 +348,7 @@ sru_status launch_fwd_scan(const RecMaps& mp, const float* b, const float* c0, c
     if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
     sru_status s = reset_scan_flags(ss.flags, items + 1, st);
     if (s != SRU_OK) return s;
-    kern<<<(unsigned)items, sru::kRecCJ, Lay::SMEM, st>>>(mp.u, mp.x, b, c0, mask, h, c_T, ckpt, ss, (int)L, (int)B,
+    kern<<<(unsigned)items, sru::kRecThreads, Lay::SMEM, st>>>(mp.u, mp.x, b, c0, mask, h, c_T, ckpt, ss, (int)L, (int)B,
                                                           (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
@@ -307,7 +366,7 @@ sru_status launch_bwd_scan_dir(const RecMaps& mp, const float* b, const uint8_t*
     if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
     sru_status s = reset_scan_flags(ss.flags, items + 1, st);
     if (s != SRU_OK) return s;
-    kern<<<(unsigned)items, sru::kRecCJ, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.dx, b, mask, ckpt, dc_T, dU, dx,
+    kern<<<(unsigned)items, sru::kRecThreads, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.dx, b, mask, ckpt, dc_T, dU, dx,
                                                           partial, dc0, ss, (int)L, (int)B, (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
@@ -410,7 +469,7 @@ sru_status sru_project(const void* X, int x_t, const void* W, int w_t, void* U, 
     if (x_t != SRU_BF16 || w_t != SRU_BF16 || (u_t != SRU_BF16 && u_t != SRU_F32)) return SRU_ERR_INVALID;
     if (K == 0) return SRU_ERR_UNSUPPORTED;
     CUtensorMap ma, mb;
-    if (!map_kmajor(&ma, X, M, K, sru::gemm::BM) || !map_kmajor(&mb, W, N, K, sru::gemm::BN)) return SRU_ERR_INVALID;
+    if (!map_kmajor(&ma, X, M, K, sru::gemm::BM) || !map_kmajor(&mb, W, N, K, kGemmBRows)) return SRU_ERR_INVALID;
     if (u_t == SRU_BF16) return launch_tc_gemm<false, false, sru::gemm::kOutBF16>(ma, mb, U, M, N, K, st);
     return launch_tc_gemm<false, false, sru::gemm::kOutF32>(ma, mb, U, M, N, K, st);
 }
@@ -490,8 +549,10 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
     } else if (scan) {
         return SRU_ERR_INVALID;  // the scan needs its flags and aggregates
     }
+    const int cj = scan ? sru::kRecCJ : pick_seq_cj(B, d, n_dir);
     RecMaps mp;
-    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir) || !map_f32_rows(&mp.x, x, L, B, d)) return SRU_ERR_INVALID;
+    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj))
+        return SRU_ERR_INVALID;
     float* ckpt = workspace ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.ckpt_off) : nullptr;
     if (scan) {
         const sru::ScanState ss = scan_state(workspace, w);
@@ -500,8 +561,8 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
         return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, ckpt, ss, L, B, d, n_dir, alpha, st);
     }
     if (u_t == SRU_BF16)
-        return launch_fwd_seq<__nv_bfloat16>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
-    return launch_fwd_seq<float>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+        return launch_fwd_seq<__nv_bfloat16>(cj, mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+    return launch_fwd_seq<float>(cj, mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
 }
 
 sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, const float* b, const float* c0,
@@ -534,14 +595,15 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
         return SRU_ERR_INVALID;
     const WsLayout w = ws_layout(L, B, d, n_dir, flags);
     if (workspace_bytes < w.total) return SRU_ERR_INVALID;
+    const bool scan = use_scan(flags, L, B, d, n_dir);
+    const int cj = scan ? sru::kRecCJ : pick_seq_cj(B, d, 1);
     RecMaps mp;
-    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir) || !map_f32_rows(&mp.x, x, L, B, d) ||
-        !map_f32_rows(&mp.dh, dh, L, B * n_dir, d) || !map_f32_rows(&mp.dx, dx, L, B, d))
+    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj) ||
+        !map_f32_rows(&mp.dh, dh, L, B * n_dir, d, cj) || !map_f32_rows(&mp.dx, dx, L, B, d, cj))
         return SRU_ERR_INVALID;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const float* ckpt = reinterpret_cast<const float*>(ws + w.ckpt_off);
     double* partial = reinterpret_cast<double*>(ws + w.partial_off);
-    const bool scan = use_scan(flags, L, B, d, n_dir);
     const bool ub = u_t == SRU_BF16, db16 = du_t == SRU_BF16;
     if (scan) {
         const sru::ScanState ss = scan_state(workspace, w);
@@ -557,14 +619,14 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
                                                      alpha, st);
     } else {
         if (ub)
-            s = db16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L,
+            s = db16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(cj, mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L,
                                                                     B, d, n_dir, alpha, st)
-                     : launch_bwd_seq<__nv_bfloat16, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
+                     : launch_bwd_seq<__nv_bfloat16, float>(cj, mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
                                                             n_dir, alpha, st);
         else
-            s = db16 ? launch_bwd_seq<float, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
+            s = db16 ? launch_bwd_seq<float, __nv_bfloat16>(cj, mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
                                                             n_dir, alpha, st)
-                     : launch_bwd_seq<float, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d, n_dir,
+                     : launch_bwd_seq<float, float>(cj, mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d, n_dir,
                                                     alpha, st);
     }
     if (s != SRU_OK) return s;
@@ -605,7 +667,8 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
     ss.agg_b = reinterpret_cast<float*>(base + agg_b_off);
     ss.prefix = reinterpret_cast<float*>(base + prefix_off);
     RecMaps mp;
-    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir) || !map_f32_rows(&mp.x, x, L, B, d)) return SRU_ERR_INVALID;
+    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, sru::kRecCJ) || !map_f32_rows(&mp.x, x, L, B, d, sru::kRecCJ))
+        return SRU_ERR_INVALID;
     if (u_t == SRU_BF16)
         return launch_fwd_scan<__nv_bfloat16>(mp, b, c0, mask, h, c_T, nullptr, ss, L, B, d, n_dir, alpha, st);
     return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, nullptr, ss, L, B, d, n_dir, alpha, st);

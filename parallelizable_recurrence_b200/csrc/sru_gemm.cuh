@@ -60,6 +60,47 @@ __host__ __device__ constexpr uint32_t idesc_bf16(bool a_mn, bool b_mn) {
            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
+// Store 32 consecutive accumulator columns (r[0..31]) of one output row.
+template <int OUT>
+__device__ __forceinline__ void epilogue_store_row32(void* __restrict__ out, int row, int col0, int M, int N, int ldo,
+                                                     const uint32_t (&r)[32]) {
+    if (row >= M) return;
+    if (OUT == kOutBF16) {
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * ldo + col0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            if (col0 + g * 8 < N) {
+                uint4 pk;
+                uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    __nv_bfloat162 two =
+                        __floats2bfloat162_rn(__uint_as_float(r[g * 8 + 2 * e]), __uint_as_float(r[g * 8 + 2 * e + 1]));
+                    w[e] = *reinterpret_cast<uint32_t*>(&two);
+                }
+                *reinterpret_cast<uint4*>(o + g * 8) = pk;
+            }
+        }
+    } else {
+        float* o = reinterpret_cast<float*>(out) + (size_t)row * ldo + col0;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            if (col0 + g * 4 < N) {
+                float4 val = make_float4(__uint_as_float(r[g * 4 + 0]), __uint_as_float(r[g * 4 + 1]),
+                                         __uint_as_float(r[g * 4 + 2]), __uint_as_float(r[g * 4 + 3]));
+                if (OUT == kOutF32Acc) {
+                    const float4 old = *reinterpret_cast<const float4*>(o + g * 4);
+                    val.x += old.x;
+                    val.y += old.y;
+                    val.z += old.z;
+                    val.w += old.w;
+                }
+                *reinterpret_cast<float4*>(o + g * 4) = val;
+            }
+        }
+    }
+}
+
 template <bool A_MN, bool B_MN, int OUT>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
@@ -219,42 +260,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN + ch * 32, r);
                 tc_wait_ld();
-                if (row < M) {
-                    if (OUT == kOutBF16) {
-                        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * ldo + col0;
-#pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            if (col0 + g * 8 < N) {
-                                uint4 pk;
-                                uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    __nv_bfloat162 two = __floats2bfloat162_rn(__uint_as_float(r[g * 8 + 2 * e]),
-                                                                               __uint_as_float(r[g * 8 + 2 * e + 1]));
-                                    w[e] = *reinterpret_cast<uint32_t*>(&two);
-                                }
-                                *reinterpret_cast<uint4*>(o + g * 8) = pk;
-                            }
-                        }
-                    } else {
-                        float* o = reinterpret_cast<float*>(out) + (size_t)row * ldo + col0;
-#pragma unroll
-                        for (int g = 0; g < 8; ++g) {
-                            if (col0 + g * 4 < N) {
-                                float4 val = make_float4(__uint_as_float(r[g * 4 + 0]), __uint_as_float(r[g * 4 + 1]),
-                                                         __uint_as_float(r[g * 4 + 2]), __uint_as_float(r[g * 4 + 3]));
-                                if (OUT == kOutF32Acc) {
-                                    const float4 old = *reinterpret_cast<const float4*>(o + g * 4);
-                                    val.x += old.x;
-                                    val.y += old.y;
-                                    val.z += old.z;
-                                    val.w += old.w;
-                                }
-                                *reinterpret_cast<float4*>(o + g * 4) = val;
-                            }
-                        }
-                    }
-                }
+                epilogue_store_row32<OUT>(out, row, col0, M, N, ldo, r);
             }
             tc_fence_before_sync();
             __syncwarp();
@@ -266,6 +272,209 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 1) {
         tc_fence_after_sync();
         tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant: a cluster of two CTAs (two SMs) computes one 256 x 256
+// output tile with tcgen05.mma.cta_group::2 (M = 256).  Each CTA stages its own
+// 128 rows of A and its own 128 columns of B (32 KB per k-block instead of
+// 48 KB for a 128 x 256 tile on one SM), and holds its 128 rows of the
+// accumulator in its own TMEM.  The pair leader (cluster rank 0) issues the
+// MMAs; both CTAs' TMA loads count on the leader's "full" barrier (the
+// .cta_group::2 form of the load); the leader's commits arrive on both CTAs'
+// "empty" and "accumulator full" barriers (commit with .multicast::cluster);
+// both CTAs' epilogue warps release the accumulator on the leader's barrier.
+// No TMA load uses cluster multicast.
+constexpr int P_BM = 256, P_BN = 256, P_STAGES = 6;   // per pair (BK as above)
+constexpr int P_CM = 128, P_CN = 128;                  // per CTA
+constexpr uint32_t P_A_BYTES = P_CM * BK * 2;          // 16 KB
+constexpr uint32_t P_B_BYTES = P_CN * BK * 2;          // 16 KB
+constexpr uint32_t P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+constexpr uint32_t P_TMEM_COLS = 2 * P_BN;             // two 128 x 256 fp32 accumulators per CTA
+constexpr size_t P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + 256;
+
+__host__ __device__ constexpr uint32_t idesc_bf16_pair(bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(P_BN >> 3) << 17) | ((uint32_t)(P_BM >> 4) << 24);
+}
+
+template <bool A_MN, bool B_MN, int OUT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                        void* __restrict__ out, int M, int N, int K, int ldo) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
+    uint64_t* empty = full + P_STAGES;
+    uint64_t* tfull = empty + P_STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile uint32_t* consumed = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0 = leader
+    const int pair_id = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    const int m_tiles = (M + P_BM - 1) / P_BM, n_tiles = (N + P_BN - 1) / P_BN;
+    const int tiles = m_tiles * n_tiles;
+    const int kblocks = (K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < P_STAGES; ++s) {
+            mbar_init(&full[s], 1);   // leader only: its producer's expect_tx covers both CTAs' bytes
+            mbar_init(&empty[s], 1);  // one multicast commit per phase
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);   // one multicast commit per phase
+            mbar_init(&tempty[a], 8);  // leader's: 4 epilogue warps of each CTA
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        *consumed = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, P_TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    cluster_sync_all();  // barriers of both CTAs initialised before any remote use
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
+    const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------------ producer (both CTAs)
+            uint32_t issued = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = pair_id; tile < tiles && !*abort_flag; tile += n_pairs) {
+                const int m0 = (tile / n_tiles) * P_BM + (int)rank * P_CM;
+                const int n0 = (tile % n_tiles) * P_BN + (int)rank * P_CN;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, kErrTimeoutMma) || *abort_flag) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    uint8_t* a_dst = smem + stage * P_STAGE_BYTES;
+                    uint8_t* b_dst = a_dst + P_A_BYTES;
+                    const int k0 = kb * BK;
+                    const uint32_t bar = leader_full0 + (uint32_t)stage * 8u;
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
+                    if (!A_MN) {
+                        tma_load_2d_pair(a_dst, &map_a, bar, k0, m0);
+                    } else {
+                        tma_load_2d_pair(a_dst, &map_a, bar, m0, k0);
+                        tma_load_2d_pair(a_dst + MN_BOX_BYTES, &map_a, bar, m0 + 64, k0);
+                    }
+                    if (!B_MN) {
+                        tma_load_2d_pair(b_dst, &map_b, bar, k0, n0);
+                    } else {
+                        tma_load_2d_pair(b_dst, &map_b, bar, n0, k0);
+                        tma_load_2d_pair(b_dst + MN_BOX_BYTES, &map_b, bar, n0 + 64, k0);
+                    }
+                    ++issued;
+                    if (++stage == P_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (*abort_flag && rank == 0) {
+                for (uint32_t q = *consumed; q < issued; ++q)
+                    mbar_wait(&full[q % P_STAGES], (q / P_STAGES) & 1u, kErrTimeoutLoad);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ------------------------------------------------------ MMA issuer (leader)
+            constexpr uint32_t idesc = idesc_bf16_pair(A_MN, B_MN);
+            int stage = 0;
+            uint32_t phase = 0, nconsumed = 0;
+            int it = 0;
+            for (int tile = pair_id; tile < tiles && !*abort_flag; tile += n_pairs, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, kErrTimeoutEpilogue)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + acc * P_BN;
+                bool ok = true;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, kErrTimeoutLoad)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_addr = smem_u32(smem + stage * P_STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + P_A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t adesc = A_MN ? smem_desc_sw128(a_addr + kk * 2048, MN_BOX_BYTES, 1024)
+                                                    : smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+                        const uint64_t bdesc = B_MN ? smem_desc_sw128(b_addr + kk * 2048, MN_BOX_BYTES, 1024)
+                                                    : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+                        tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    tc_commit_pair_mc(&empty[stage], 0x3);  // frees this stage in both CTAs
+                    *consumed = ++nconsumed;
+                    if (++stage == P_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) {
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_commit_pair_mc(&tfull[acc], 0x3);  // accumulator ready in both CTAs
+            }
+            tc_commit_pair_mc(drain, 0x1);
+            mbar_wait(drain, 0, kErrTimeoutMma);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue (both CTAs)
+        const int quarter = warp & 3;
+        int it = 0;
+        for (int tile = pair_id; tile < tiles; tile += n_pairs, ++it) {
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            const int m0 = (tile / n_tiles) * P_BM + (int)rank * P_CM, n0 = (tile % n_tiles) * P_BN;
+            const bool ok = mbar_wait(&tfull[acc], acc_phase, kErrTimeoutMma);
+            if (!__all_sync(0xffffffffu, ok) || *abort_flag) {
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const int row = m0 + quarter * 32 + lane;
+            for (int ch = 0; ch < P_BN / 32; ++ch) {
+                const int col0 = n0 + ch * 32;
+                if (col0 >= N) break;  // uniform across the warp
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * P_BN + ch * 32, r);
+                tc_wait_ld();
+                epilogue_store_row32<OUT>(out, row, col0, M, N, ldo, r);
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)acc * 8u);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while its peer may still signal its barriers
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc_pair(tmem_base, P_TMEM_COLS);
     }
 }
 

@@ -2,52 +2,43 @@
 //
 // Method: "When Attention Meets Fast Recurrence" (T. Lei), background section
 // on SRU, Eqs. (2)-(5).  Once U is known every (direction, batch row b,
-// channel j) stream is independent, so each thread owns one stream and walks
-// t sequentially with the state c in a register.  A CTA owns CJ consecutive
-// channels of one (b, direction); the U / x / dh tiles of T consecutive time
-// steps are brought into shared memory by TMA (cp.async.bulk.tensor) through
-// an S-stage mbarrier ring, so (S-1)*T steps of input are in flight while T
-// steps are computed.  Outputs are written with coalesced stores (a warp
-// writes 32 consecutive channels of one time step).
+// channel j) stream is independent; each is walked sequentially over t with
+// its state c in a register.
 //
-// The backward pass re-runs the forward over one chunk of T steps from the
-// state checkpoint the forward stored at the chunk start (keeping c, f and r
-// of the chunk in registers), then walks the chunk in reverse.  The partial
-// sums of dv and db are accumulated per thread in double precision and
-// reduced over the batch in a fixed order by a second kernel.
+// Layout of the work: a CTA owns CJ (64, 128 or 256) consecutive channels of
+// one (b, direction), CJ/2 threads; each thread owns two adjacent channels and
+// advances both with the packed fp32x2 instructions of sm_100 (__ffma2_rn,
+// __fadd2_rn, __fmul2_rn), so the two independent recurrences interleave and
+// most arithmetic costs one instruction per pair.  The U / x / dh tiles of
+// kChunkT consecutive steps are brought into shared memory by TMA
+// (cp.async.bulk.tensor) through an S-stage mbarrier ring, so (S-1)*kChunkT
+// steps of input are in flight while kChunkT steps are computed.  Outputs are
+// written with coalesced 8-byte (fp32 pair) / 4-byte (bf16 pair) stores.
+//
+// The backward re-runs the forward over one chunk from the state checkpoint
+// the forward stored at the chunk start (keeping c, f and r of the chunk in
+// registers), then walks it in reverse.  dv/db partial sums are fp32 within a
+// chunk, fp64 per thread, and reduced over the batch in a fixed order.
 #pragma once
 
 #include "sru_ptx.cuh"
 
 namespace sru {
 
-constexpr int kChunkT = 16;  // time steps per pipeline stage == checkpoint interval
-constexpr int kRecCJ = 64;   // channels (threads) per CTA
-constexpr int kFwdStages = 4;
-constexpr int kBwdStages = 3;
-
-// Per-channel constants of Eqs. (2)-(3), pre-scaled by -log2(e) so that one
-// FMA gives the exponent of 2 in sigma(z) = 1 / (1 + 2^(-z log2 e)):
-//   nvf = -v_f log2(e), nbf = -b_f log2(e)  (and the same for the reset gate).
-struct GateParams {
-    float vf, vr, bf, br;      // as given (the backward needs v_f, v_r)
-    float nvf, nvr, nbf, nbr;  // scaled by -log2(e)
-};
+constexpr int kChunkT = 16;          // time steps per pipeline stage == checkpoint interval
+constexpr int kRecCJ = 64;           // channels per CTA
+constexpr int kRecThreads = 32;      // one warp; thread i owns channels 2i and 2i+1 of the tile
+#ifndef SRU_FWD_STAGES
+#define SRU_FWD_STAGES 4
+#endif
+#ifndef SRU_BWD_STAGES
+#define SRU_BWD_STAGES 3
+#endif
+constexpr int kFwdStages = SRU_FWD_STAGES;  // TMA ring depth (build-time tuning knobs)
+constexpr int kBwdStages = SRU_BWD_STAGES;
 constexpr float kNegLog2e = -1.4426950408889634f;
 
-__device__ __forceinline__ GateParams make_gate_params(float vf, float vr, float bf, float br) {
-    GateParams p;
-    p.vf = vf;
-    p.vr = vr;
-    p.bf = bf;
-    p.br = br;
-    p.nvf = __fmul_rn(vf, kNegLog2e);
-    p.nvr = __fmul_rn(vr, kNegLog2e);
-    p.nbf = __fmul_rn(bf, kNegLog2e);
-    p.nbr = __fmul_rn(br, kNegLog2e);
-    return p;
-}
-
+// ------------------------------------------------------------ scalar helpers
 // 2^x and 1/x with the single-instruction approximations of the PTX ISA
 // (ex2.approx: relative error ~2^-22; rcp.approx: within 1 ulp).
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -62,27 +53,56 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 // logistic sigma(z) given e = -z log2(e): 1 / (1 + 2^e); saturates to exactly 0 and 1.
 __device__ __forceinline__ float sigmoid_nl2(float e) { return rcp_approx(__fadd_rn(1.0f, ex2_approx(e))); }
-// logistic sigma(u + b) for a gate with no peephole term (v = 0)
-__device__ __forceinline__ float sigmoid_f(float z) { return sigmoid_nl2(__fmul_rn(z, kNegLog2e)); }
 
-// One step of Eqs. (2)-(4): returns c[t] from c[t-1], and the gate values.
-// Every operation is explicitly rounded so the forward and the backward's
-// recomputation of a chunk produce bit-identical states.
-__device__ __forceinline__ float sru_cell(float c, float uc, float uf, float ur, const GateParams& p,
-                                          float& f, float& r) {
-    f = sigmoid_nl2(__fmaf_rn(p.nvf, c, __fmaf_rn(uf, kNegLog2e, p.nbf)));
-    r = sigmoid_nl2(__fmaf_rn(p.nvr, c, __fmaf_rn(ur, kNegLog2e, p.nbr)));
-    return __fmaf_rn(f, __fsub_rn(c, uc), uc);
+// -------------------------------------------------------------- pair helpers
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+// a - b, rounded once (the fma of -1*b + a is exact before its single rounding)
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, f2(-1.0f), a); }
+__device__ __forceinline__ float2 sigmoid2_nl2(float2 e) {
+    const float2 t = add2(f2(1.0f), make_float2(ex2_approx(e.x), ex2_approx(e.y)));
+    return make_float2(rcp_approx(t.x), rcp_approx(t.y));
 }
 
-__device__ __forceinline__ float to_f32(float x) { return x; }
-__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
-template <typename T>
-__device__ __forceinline__ T from_f32(float x);
-template <>
-__device__ __forceinline__ float from_f32<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+// Per-channel-pair constants of Eqs. (2)-(3), pre-scaled by -log2(e) so that
+// one FMA gives the exponent of 2 in sigma(z) = 1 / (1 + 2^(-z log2 e)).
+struct GateParams2 {
+    float2 vf, vr;              // as given (the backward needs v_f, v_r)
+    float2 nvf, nvr, nbf, nbr;  // -v log2(e), -b log2(e)
+};
+__device__ __forceinline__ GateParams2 make_gate_params2(float2 vf, float2 vr, float2 bf, float2 br) {
+    GateParams2 p;
+    p.vf = vf;
+    p.vr = vr;
+    p.nvf = mul2(vf, f2(kNegLog2e));
+    p.nvr = mul2(vr, f2(kNegLog2e));
+    p.nbf = mul2(bf, f2(kNegLog2e));
+    p.nbr = mul2(br, f2(kNegLog2e));
+    return p;
+}
+
+// One step of Eqs. (2)-(4) for two channels: returns c[t] from c[t-1] and the
+// gate values.  Every operation is explicitly rounded, so the forward and the
+// backward's recomputation of a chunk give bit-identical states.
+__device__ __forceinline__ float2 sru_cell2(float2 c, float2 uc, float2 uf, float2 ur, const GateParams2& p,
+                                            float2& f, float2& r) {
+    f = sigmoid2_nl2(fma2(p.nvf, c, fma2(uf, f2(kNegLog2e), p.nbf)));
+    r = sigmoid2_nl2(fma2(p.nvr, c, fma2(ur, f2(kNegLog2e), p.nbr)));
+    return fma2(f, sub2(c, uc), uc);
+}
+
+// Loads/stores of a channel pair (2 adjacent elements, 4- or 8-byte aligned).
+__device__ __forceinline__ float2 load_pair(const __nv_bfloat16* p) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ float2 load_pair(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ void store_pair(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
+__device__ __forceinline__ void store_pair(__nv_bfloat16* p, float2 v) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v.x, v.y);
+}
 
 // Bit i set: row t0+i of this chunk exists (t < L) and is not padded.  Whole warp calls.
 __device__ __forceinline__ uint32_t chunk_valid_bits(const uint8_t* __restrict__ mask, int t0, int L, int B,
@@ -96,7 +116,7 @@ __device__ __forceinline__ uint32_t chunk_inrange_bits(int t0, int L) {
     return n >= kChunkT ? ((1u << kChunkT) - 1u) : ((1u << n) - 1u);
 }
 
-// After a failed wait: thread 0 waits (bounded) for the loads it issued that
+// After a failed wait: lane 0 waits (bounded) for the loads it issued that
 // have not landed yet, so no copy is still writing this CTA's shared memory.
 template <int S>
 __device__ __forceinline__ void drain_pending_loads(uint64_t* full, uint32_t pending, uint32_t phase_bits) {
@@ -105,35 +125,26 @@ __device__ __forceinline__ void drain_pending_loads(uint64_t* full, uint32_t pen
         if ((pending >> s) & 1u) mbar_wait(&full[s], (phase_bits >> s) & 1u, kErrTimeoutLoad);
 }
 
+// ---------------------------------------------------------------- forward
 // Eqs. (2)-(5) over one chunk of kChunkT rows staged in shared memory
 // (us: [T][3][CJ] gate blocks, xs: [T][CJ]), walked in the direction's time
-// order from state c.  Writes h for the rows that exist (0 at padded rows) and
-// returns the state after the chunk.
-template <typename UT>
-__device__ __forceinline__ float fwd_chunk(const UT* __restrict__ us, const float* __restrict__ xs,
-                                           uint32_t valid, uint32_t inrange, float c, const GateParams& p,
-                                           float alpha, int dir, float* __restrict__ hp, size_t h_tstride,
-                                           bool jok, int tid) {
+// order from state c, for this thread's channel pair (offset cj in the tile).
+// Writes h for the rows that exist (0 at padded rows); returns the state.
+template <typename UT, int CJ = kRecCJ>
+__device__ __forceinline__ float2 fwd_chunk(const UT* __restrict__ us, const float* __restrict__ xs,
+                                            uint32_t valid, uint32_t inrange, float2 c, const GateParams2& p,
+                                            float2 alpha, int dir, float* __restrict__ hp, size_t h_tstride,
+                                            bool jok, int cj) {
     constexpr uint32_t kFull = (1u << kChunkT) - 1u;
     if (valid == kFull) {  // every row present and unpadded: no per-row predicates
-        if (dir == 0) {
 #pragma unroll
-            for (int i = 0; i < kChunkT; ++i) {
-                float f, r;
-                c = sru_cell(c, to_f32(us[(i * 3 + 0) * kRecCJ + tid]), to_f32(us[(i * 3 + 1) * kRecCJ + tid]),
-                             to_f32(us[(i * 3 + 2) * kRecCJ + tid]), p, f, r);
-                const float ax = __fmul_rn(alpha, xs[i * kRecCJ + tid]);
-                if (jok) hp[(size_t)i * h_tstride] = __fmaf_rn(r, __fsub_rn(c, ax), ax);  // Eq. (5)
-            }
-        } else {
-#pragma unroll
-            for (int i = kChunkT - 1; i >= 0; --i) {
-                float f, r;
-                c = sru_cell(c, to_f32(us[(i * 3 + 0) * kRecCJ + tid]), to_f32(us[(i * 3 + 1) * kRecCJ + tid]),
-                             to_f32(us[(i * 3 + 2) * kRecCJ + tid]), p, f, r);
-                const float ax = __fmul_rn(alpha, xs[i * kRecCJ + tid]);
-                if (jok) hp[(size_t)i * h_tstride] = __fmaf_rn(r, __fsub_rn(c, ax), ax);
-            }
+        for (int q = 0; q < kChunkT; ++q) {
+            const int i = dir == 0 ? q : kChunkT - 1 - q;
+            float2 f, r;
+            c = sru_cell2(c, load_pair(us + (i * 3 + 0) * CJ + cj), load_pair(us + (i * 3 + 1) * CJ + cj),
+                          load_pair(us + (i * 3 + 2) * CJ + cj), p, f, r);
+            const float2 ax = mul2(alpha, load_pair(xs + i * CJ + cj));
+            if (jok) store_pair(hp + (size_t)i * h_tstride, fma2(r, sub2(c, ax), ax));  // Eq. (5)
         }
         return c;
     }
@@ -141,56 +152,57 @@ __device__ __forceinline__ float fwd_chunk(const UT* __restrict__ us, const floa
     for (int q = 0; q < kChunkT; ++q) {
         const int i = dir == 0 ? q : kChunkT - 1 - q;
         if (!((inrange >> i) & 1u)) continue;
-        float hv = 0.f;
+        float2 hv = f2(0.f);
         if ((valid >> i) & 1u) {
-            float f, r;
-            c = sru_cell(c, to_f32(us[(i * 3 + 0) * kRecCJ + tid]), to_f32(us[(i * 3 + 1) * kRecCJ + tid]),
-                         to_f32(us[(i * 3 + 2) * kRecCJ + tid]), p, f, r);
-            const float ax = __fmul_rn(alpha, xs[i * kRecCJ + tid]);
-            hv = __fmaf_rn(r, __fsub_rn(c, ax), ax);  // Eq. (5): r*c + (1-r)*alpha*x
+            float2 f, r;
+            c = sru_cell2(c, load_pair(us + (i * 3 + 0) * CJ + cj), load_pair(us + (i * 3 + 1) * CJ + cj),
+                          load_pair(us + (i * 3 + 2) * CJ + cj), p, f, r);
+            const float2 ax = mul2(alpha, load_pair(xs + i * CJ + cj));
+            hv = fma2(r, sub2(c, ax), ax);  // Eq. (5): r*c + (1-r)*alpha*x
         }
-        if (jok) hp[(size_t)i * h_tstride] = hv;
+        if (jok) store_pair(hp + (size_t)i * h_tstride, hv);
     }
     return c;
 }
 
-template <typename UT>
+template <typename UT, int CJ = kRecCJ>
 struct FwdLayout {
-    static constexpr int U_BYTES = kChunkT * 3 * kRecCJ * (int)sizeof(UT);
-    static constexpr int X_BYTES = kChunkT * kRecCJ * 4;
+    static constexpr int U_BYTES = kChunkT * 3 * CJ * (int)sizeof(UT);
+    static constexpr int X_BYTES = kChunkT * CJ * 4;
     static constexpr int STAGE = U_BYTES + X_BYTES;
     static constexpr int BAR_OFF = kFwdStages * STAGE;
     static constexpr int SMEM = BAR_OFF + 64 + 128;  // barriers + alignment slack
 };
 
-// Forward.  Grid (ceil(d/CJ), B, n_dir), block CJ threads.
+// Forward.  Grid (ceil(d/CJ), B, n_dir), CJ/2 threads (CJ/64 warps) per CTA.
 //   map_u: 4-D (d, 3, B*n_dir, L) of UT, box (CJ, 3, 1, T)
 //   map_x: 3-D (d, B, L) fp32, box (CJ, 1, T)
-template <typename UT>
-__global__ void __launch_bounds__(kRecCJ) sru_fwd_seq_kernel(
+template <typename UT, int CJ>
+__global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
     const float* __restrict__ v, const float* __restrict__ bias, const float* __restrict__ c0,
     const uint8_t* __restrict__ mask, float* __restrict__ h, float* __restrict__ c_T, float* __restrict__ ckpt,
     int L, int B, int d, int n_dir, float alpha) {
-    using Lay = FwdLayout<UT>;
+    using Lay = FwdLayout<UT, CJ>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
 
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int j0 = blockIdx.x * kRecCJ, j = j0 + tid;
+    const int tid = threadIdx.x, lane = tid & 31, cj = 2 * tid;
+    const int j0 = blockIdx.x * CJ, j = j0 + cj;
     const int b = blockIdx.y, dir = blockIdx.z;
     const int bd = b * n_dir + dir;
-    const bool jok = j < d;
+    const bool jok = j < d;  // d is even, so the pair is either in or out
     const int nch = (L + kChunkT - 1) / kChunkT;
 
-    GateParams p = make_gate_params(0.f, 0.f, 0.f, 0.f);
-    float c = 0.f;
+    GateParams2 p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
+    float2 c = f2(0.f);
     if (jok) {
-        p = make_gate_params(v[(dir * 2 + 0) * d + j], v[(dir * 2 + 1) * d + j], bias[(dir * 2 + 0) * d + j],
-                             bias[(dir * 2 + 1) * d + j]);
-        if (c0 != nullptr) c = c0[(size_t)bd * d + j];
+        p = make_gate_params2(load_pair(v + (dir * 2 + 0) * d + j), load_pair(v + (dir * 2 + 1) * d + j),
+                              load_pair(bias + (dir * 2 + 0) * d + j), load_pair(bias + (dir * 2 + 1) * d + j));
+        if (c0 != nullptr) c = load_pair(c0 + (size_t)bd * d + j);
     }
+    const float2 alpha2 = f2(alpha);
     if (tid == 0) {
         for (int s = 0; s < kFwdStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
@@ -205,7 +217,7 @@ __global__ void __launch_bounds__(kRecCJ) sru_fwd_seq_kernel(
     auto issue = [&](int k) {
         const int t0 = time_chunk(k) * kChunkT;
         const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
-        if (lane == 0 && valid != 0u) {
+        if (tid == 0 && valid != 0u) {
             const int s = k % kFwdStages;
             pending |= 1u << s;
             uint8_t* st = smem + s * Lay::STAGE;
@@ -224,7 +236,7 @@ __global__ void __launch_bounds__(kRecCJ) sru_fwd_seq_kernel(
         const int tc = time_chunk(k), t0 = tc * kChunkT;
         const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
         const uint32_t inrange = chunk_inrange_bits(t0, L);
-        if (ckpt != nullptr && jok) ckpt[((size_t)tc * B * n_dir + bd) * d + j] = c;
+        if (ckpt != nullptr && jok) store_pair(ckpt + ((size_t)tc * B * n_dir + bd) * d + j, c);
         if (valid != 0u) {
             const bool ok = mbar_wait(&full[s], (phase_bits >> s) & 1u, kErrTimeoutLoad);
             if (__syncthreads_or(!ok)) {  // a load never landed: give up (error recorded)
@@ -237,80 +249,87 @@ __global__ void __launch_bounds__(kRecCJ) sru_fwd_seq_kernel(
         const UT* us = reinterpret_cast<const UT*>(smem + s * Lay::STAGE);
         const float* xs = reinterpret_cast<const float*>(smem + s * Lay::STAGE + Lay::U_BYTES);
         float* hp = h + (size_t)t0 * h_tstride + (size_t)bd * d + j;
-        c = fwd_chunk<UT>(us, xs, valid, inrange, c, p, alpha, dir, hp, h_tstride, jok, tid);
+        c = fwd_chunk<UT, CJ>(us, xs, valid, inrange, c, p, alpha2, dir, hp, h_tstride, jok, cj);
         __syncthreads();  // every thread is done with stage s
         if (tid < 32 && k + kFwdStages < nch) issue(k + kFwdStages);
     }
-    if (jok) c_T[(size_t)bd * d + j] = c;
+    if (jok) store_pair(c_T + (size_t)bd * d + j, c);
 }
 
+// ---------------------------------------------------------------- backward
 // Backward over one chunk staged in shared memory (us, xs, dhs and, with
-// ACC_DX, the other direction's dx in dxin), given the state c entering the
-// chunk in forward order and the state gradient g leaving it.  Re-runs the
-// forward over the chunk keeping c, f and r in registers, then walks it in
-// reverse: writes dU and dx for the rows that exist, accumulates the dv/db
-// partial sums in acc = {dv_f, dv_r, db_f, db_r}, and updates g.
-template <typename UT, typename DUT, bool ACC_DX, int DIR>
+// ACC_DX, the dx the other direction already wrote in dxin), given the state c
+// entering the chunk in forward order and the state gradient g leaving it.
+// Re-runs the forward over the chunk keeping c, f and r in registers, then
+// walks it in reverse: writes dU and dx for the rows that exist, accumulates
+// the dv/db partial sums in acc[q] = {dv_f, dv_r, db_f, db_r} (per channel of
+// the pair), and updates g.
+template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ = kRecCJ>
 __device__ __forceinline__ void bwd_chunk(const UT* __restrict__ us, const float* __restrict__ xs,
                                           const float* __restrict__ dhs, const float* __restrict__ dxin,
-                                          uint32_t valid, uint32_t inrange, float c, const GateParams& p,
-                                          float alpha, float& g, double (&acc)[4], DUT* __restrict__ dUp,
+                                          uint32_t valid, uint32_t inrange, float2 c, const GateParams2& p,
+                                          float2 alpha, float2& g, double (&acc)[4][2], DUT* __restrict__ dUp,
                                           float* __restrict__ dxp, size_t u_tstride, size_t x_tstride, int d,
-                                          bool jok, int tid) {
+                                          bool jok, int cj) {
     constexpr uint32_t kFull = (1u << kChunkT) - 1u;
     const bool full = valid == kFull;
-    float cp[kChunkT], fs[kChunkT], rs[kChunkT];
+    float2 cp[kChunkT], fs[kChunkT], rs[kChunkT];
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
         const int i = DIR == 0 ? q : kChunkT - 1 - q;
         cp[i] = c;
-        fs[i] = 0.f;
-        rs[i] = 0.f;
+        fs[i] = f2(0.f);
+        rs[i] = f2(0.f);
         if (full || ((valid >> i) & 1u))
-            c = sru_cell(c, to_f32(us[(i * 3 + 0) * kRecCJ + tid]), to_f32(us[(i * 3 + 1) * kRecCJ + tid]),
-                         to_f32(us[(i * 3 + 2) * kRecCJ + tid]), p, fs[i], rs[i]);
+            c = sru_cell2(c, load_pair(us + (i * 3 + 0) * CJ + cj), load_pair(us + (i * 3 + 1) * CJ + cj),
+                          load_pair(us + (i * 3 + 2) * CJ + cj), p, fs[i], rs[i]);
     }
-    // chunk partial sums in fp32 (16 terms), folded into the double totals once per chunk
-    float s_vf = 0.f, s_vr = 0.f, s_bf = 0.f, s_br = 0.f;
+    // chunk partial sums in fp32 (16 terms), folded into the fp64 totals once per chunk
+    float2 s_vf = f2(0.f), s_vr = f2(0.f), s_bf = f2(0.f), s_br = f2(0.f);
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
         const int i = DIR == 0 ? kChunkT - 1 - q : q;
         if (!full && !((inrange >> i) & 1u)) continue;
-        float duc = 0.f, dzf = 0.f, dzr = 0.f, dxv = 0.f;
+        float2 duc = f2(0.f), dzf = f2(0.f), dzr = f2(0.f), dxv = f2(0.f);
         const bool row = full || ((valid >> i) & 1u);
         if (row) {
-            const float f = fs[i], r = rs[i], cpv = cp[i];
-            const float uc = to_f32(us[(i * 3 + 0) * kRecCJ + tid]);
-            const float ax = __fmul_rn(alpha, xs[i * kRecCJ + tid]);
-            const float dhv = dhs[i * kRecCJ + tid];
-            const float cn = __fmaf_rn(f, __fsub_rn(cpv, uc), uc);
-            const float G = __fmaf_rn(dhv, r, g);  // dLoss/dc[t]
-            const float omr = __fsub_rn(1.f, r), omf = __fsub_rn(1.f, f);
-            dxv = __fmul_rn(__fmul_rn(dhv, omr), alpha);
-            dzf = __fmul_rn(__fmul_rn(G, __fsub_rn(cpv, uc)), __fmul_rn(f, omf));
-            dzr = __fmul_rn(__fmul_rn(dhv, __fsub_rn(cn, ax)), __fmul_rn(r, omr));
-            duc = __fmul_rn(G, omf);
-            g = __fmaf_rn(dzr, p.vr, __fmaf_rn(dzf, p.vf, __fmul_rn(G, f)));  // dLoss/dc[t-1]
-            s_vf = __fmaf_rn(dzf, cpv, s_vf);
-            s_vr = __fmaf_rn(dzr, cpv, s_vr);
-            s_bf = __fadd_rn(s_bf, dzf);
-            s_br = __fadd_rn(s_br, dzr);
+            const float2 f = fs[i], r = rs[i], cpv = cp[i];
+            const float2 uc = load_pair(us + (i * 3 + 0) * CJ + cj);
+            const float2 ax = mul2(alpha, load_pair(xs + i * CJ + cj));
+            const float2 dhv = load_pair(dhs + i * CJ + cj);
+            const float2 cmu = sub2(cpv, uc);
+            const float2 cn = fma2(f, cmu, uc);
+            const float2 G = fma2(dhv, r, g);  // dLoss/dc[t]
+            const float2 omr = sub2(f2(1.f), r), omf = sub2(f2(1.f), f);
+            dxv = mul2(mul2(dhv, omr), alpha);
+            dzf = mul2(mul2(G, cmu), mul2(f, omf));
+            dzr = mul2(mul2(dhv, sub2(cn, ax)), mul2(r, omr));
+            duc = mul2(G, omf);
+            g = fma2(dzr, p.vr, fma2(dzf, p.vf, mul2(G, f)));  // dLoss/dc[t-1]
+            s_vf = fma2(dzf, cpv, s_vf);
+            s_vr = fma2(dzr, cpv, s_vr);
+            s_bf = add2(s_bf, dzf);
+            s_br = add2(s_br, dzr);
         }
         if (jok) {
-            dUp[(size_t)i * u_tstride] = from_f32<DUT>(duc);
-            dUp[(size_t)i * u_tstride + d] = from_f32<DUT>(dzf);
-            dUp[(size_t)i * u_tstride + 2 * d] = from_f32<DUT>(dzr);
+            store_pair(dUp + (size_t)i * u_tstride, duc);
+            store_pair(dUp + (size_t)i * u_tstride + d, dzf);
+            store_pair(dUp + (size_t)i * u_tstride + 2 * d, dzr);
             if (ACC_DX) {
-                if (row) dxp[(size_t)i * x_tstride] = __fadd_rn(dxin[i * kRecCJ + tid], dxv);
+                if (row) store_pair(dxp + (size_t)i * x_tstride, add2(load_pair(dxin + i * CJ + cj), dxv));
             } else {
-                dxp[(size_t)i * x_tstride] = dxv;
+                store_pair(dxp + (size_t)i * x_tstride, dxv);
             }
         }
     }
-    acc[0] += (double)s_vf;
-    acc[1] += (double)s_vr;
-    acc[2] += (double)s_bf;
-    acc[3] += (double)s_br;
+    acc[0][0] += (double)s_vf.x;
+    acc[0][1] += (double)s_vf.y;
+    acc[1][0] += (double)s_vr.x;
+    acc[1][1] += (double)s_vr.y;
+    acc[2][0] += (double)s_bf.x;
+    acc[2][1] += (double)s_bf.y;
+    acc[3][0] += (double)s_br.x;
+    acc[3][1] += (double)s_br.y;
 }
 
 // A chunk with no valid row: zero dU (and dx unless accumulating); g passes through.
@@ -321,56 +340,63 @@ __device__ __forceinline__ void bwd_chunk_padded(uint32_t inrange, DUT* __restri
 #pragma unroll
     for (int i = 0; i < kChunkT; ++i) {
         if (!((inrange >> i) & 1u)) continue;
-        dUp[(size_t)i * u_tstride] = from_f32<DUT>(0.f);
-        dUp[(size_t)i * u_tstride + d] = from_f32<DUT>(0.f);
-        dUp[(size_t)i * u_tstride + 2 * d] = from_f32<DUT>(0.f);
-        if (!ACC_DX) dxp[(size_t)i * x_tstride] = 0.f;
+        store_pair(dUp + (size_t)i * u_tstride, f2(0.f));
+        store_pair(dUp + (size_t)i * u_tstride + d, f2(0.f));
+        store_pair(dUp + (size_t)i * u_tstride + 2 * d, f2(0.f));
+        if (!ACC_DX) store_pair(dxp + (size_t)i * x_tstride, f2(0.f));
     }
 }
 
-template <typename UT, bool ACC_DX>
+// Per-thread dv/db totals of a channel pair -> partial[row][q][j .. j+1]
+__device__ __forceinline__ void store_partials(double* __restrict__ pp, const double (&acc)[4][2], int d) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) *reinterpret_cast<double2*>(pp + (size_t)q * d) = make_double2(acc[q][0], acc[q][1]);
+}
+
+template <typename UT, bool ACC_DX, int CJ = kRecCJ>
 struct BwdLayout {
-    static constexpr int U_BYTES = kChunkT * 3 * kRecCJ * (int)sizeof(UT);
-    static constexpr int V_BYTES = kChunkT * kRecCJ * 4;  // one fp32 (T, CJ) tile
+    static constexpr int U_BYTES = kChunkT * 3 * CJ * (int)sizeof(UT);
+    static constexpr int V_BYTES = kChunkT * CJ * 4;  // one fp32 (T, CJ) tile
     static constexpr int STAGE = U_BYTES + V_BYTES * (ACC_DX ? 3 : 2);
     static constexpr int BAR_OFF = kBwdStages * STAGE;
     static constexpr int SMEM = BAR_OFF + 64 + 128;
 };
 
-// Backward of direction DIR.  Grid (ceil(d/CJ), B), block CJ threads.
+// Backward of direction DIR.  Grid (ceil(d/CJ), B), CJ/2 threads (CJ/64 warps) per CTA.
 // ACC_DX: dx += this direction's highway gradient (dx already holds the other
 // direction's, written by an earlier launch on the same stream), else dx = it.
 //   map_dh: 3-D (d, B*n_dir, L) fp32; map_dxin: like map_x but over dx.
 // DIR is a template parameter so the per-chunk register arrays are indexed
 // with compile-time constants.
-template <typename UT, typename DUT, bool ACC_DX, int DIR>
-__global__ void __launch_bounds__(kRecCJ) sru_bwd_seq_kernel(
+template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ>
+__global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
     const __grid_constant__ CUtensorMap map_dh, const __grid_constant__ CUtensorMap map_dxin,
     const float* __restrict__ v, const float* __restrict__ bias, const uint8_t* __restrict__ mask,
     const float* __restrict__ ckpt, const float* __restrict__ dc_T, DUT* __restrict__ dU,
     float* __restrict__ dx, double* __restrict__ partial, float* __restrict__ dc0, int L, int B, int d,
     int n_dir, float alpha) {
-    using Lay = BwdLayout<UT, ACC_DX>;
+    using Lay = BwdLayout<UT, ACC_DX, CJ>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
 
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int j0 = blockIdx.x * kRecCJ, j = j0 + tid;
+    const int tid = threadIdx.x, lane = tid & 31, cj = 2 * tid;
+    const int j0 = blockIdx.x * CJ, j = j0 + cj;
     constexpr int dir = DIR;
     const int b = blockIdx.y;
     const int bd = b * n_dir + dir;
     const bool jok = j < d;
     const int nch = (L + kChunkT - 1) / kChunkT;
 
-    GateParams p = make_gate_params(0.f, 0.f, 0.f, 0.f);
-    float g = 0.f;
+    GateParams2 p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
+    float2 g = f2(0.f);
     if (jok) {
-        p = make_gate_params(v[(dir * 2 + 0) * d + j], v[(dir * 2 + 1) * d + j], bias[(dir * 2 + 0) * d + j],
-                             bias[(dir * 2 + 1) * d + j]);
-        if (dc_T != nullptr) g = dc_T[(size_t)bd * d + j];
+        p = make_gate_params2(load_pair(v + (dir * 2 + 0) * d + j), load_pair(v + (dir * 2 + 1) * d + j),
+                              load_pair(bias + (dir * 2 + 0) * d + j), load_pair(bias + (dir * 2 + 1) * d + j));
+        if (dc_T != nullptr) g = load_pair(dc_T + (size_t)bd * d + j);
     }
+    const float2 alpha2 = f2(alpha);
     if (tid == 0) {
         for (int s = 0; s < kBwdStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
@@ -387,7 +413,7 @@ __global__ void __launch_bounds__(kRecCJ) sru_bwd_seq_kernel(
     auto issue = [&](int k) {
         const int t0 = time_chunk(k) * kChunkT;
         const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
-        if (lane == 0 && valid != 0u) {
+        if (tid == 0 && valid != 0u) {
             const int s = k % kBwdStages;
             pending |= 1u << s;
             uint8_t* st = smem + s * Lay::STAGE;
@@ -401,7 +427,7 @@ __global__ void __launch_bounds__(kRecCJ) sru_bwd_seq_kernel(
     if (tid < 32)
         for (int k = 0; k < kBwdStages && k < nch; ++k) issue(k);
 
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    double acc[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
     uint32_t phase_bits = 0;
     const size_t u_tstride = (size_t)B * n_dir * 3 * d;
     const size_t x_tstride = (size_t)B * d;
@@ -428,33 +454,29 @@ __global__ void __launch_bounds__(kRecCJ) sru_bwd_seq_kernel(
 
         const UT* us = reinterpret_cast<const UT*>(smem + s * Lay::STAGE);
         const float* xs = reinterpret_cast<const float*>(smem + s * Lay::STAGE + Lay::U_BYTES);
-        const float* dhs = xs + kChunkT * kRecCJ;
-        const float* dxin = dhs + kChunkT * kRecCJ;
-        const float c_start = jok ? ckpt[((size_t)tc * B * n_dir + bd) * d + j] : 0.f;
-        bwd_chunk<UT, DUT, ACC_DX, DIR>(us, xs, dhs, dxin, valid, inrange, c_start, p, alpha, g, acc, dUp, dxp,
-                                        u_tstride, x_tstride, d, jok, tid);
+        const float* dhs = xs + kChunkT * CJ;
+        const float* dxin = dhs + kChunkT * CJ;
+        const float2 c_start = jok ? load_pair(ckpt + ((size_t)tc * B * n_dir + bd) * d + j) : f2(0.f);
+        bwd_chunk<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, dxin, valid, inrange, c_start, p, alpha2, g, acc, dUp,
+                                            dxp, u_tstride, x_tstride, d, jok, cj);
         __syncthreads();
         if (tid < 32 && k + kBwdStages < nch) issue(k + kBwdStages);
     }
     if (jok) {
-        dc0[(size_t)bd * d + j] = g;
-        double* pp = partial + (size_t)bd * 4 * d + j;
-        pp[0] = acc[0];
-        pp[(size_t)d] = acc[1];
-        pp[(size_t)2 * d] = acc[2];
-        pp[(size_t)3 * d] = acc[3];
+        store_pair(dc0 + (size_t)bd * d + j, g);
+        store_partials(partial + (size_t)bd * 4 * d + j, acc, d);
     }
 }
 
-// dv, db = sum over b of the per-row partial sums, in increasing b (deterministic).
-// partial: (B, n_dir, 4, d) doubles, rows [dv_f, dv_r, db_f, db_r].
-__global__ void sru_reduce_dvdb_kernel(const double* __restrict__ partial, int B, int d, int n_dir,
+// dv, db = sum over rows of the per-row partial sums, in increasing row order
+// (deterministic).  partial: (rows, n_dir, 4, d) doubles, [dv_f, dv_r, db_f, db_r].
+__global__ void sru_reduce_dvdb_kernel(const double* __restrict__ partial, int rows, int d, int n_dir,
                                        float* __restrict__ dv, float* __restrict__ db) {
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= n_dir * 4 * d) return;
     const int dir = idx / (4 * d), q = (idx / d) % 4, j = idx % d;
     double s = 0.0;
-    for (int bb = 0; bb < B; ++bb) s += partial[(((size_t)bb * n_dir + dir) * 4 + q) * d + j];
+    for (int rr = 0; rr < rows; ++rr) s += partial[(((size_t)rr * n_dir + dir) * 4 + q) * d + j];
     if (q < 2)
         dv[(dir * 2 + q) * d + j] = (float)s;
     else

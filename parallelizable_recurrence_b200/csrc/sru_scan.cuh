@@ -41,15 +41,15 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
 __device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
-__device__ __forceinline__ float ld_relaxed_gpu(const float* p) {
-    float v;
-    asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+__device__ __forceinline__ float2 ld_relaxed_gpu2(const float* p) {
+    float2 v;
+    asm volatile("ld.relaxed.gpu.global.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p) : "memory");
     return v;
 }
 
 struct ScanState {
     unsigned* flags;  // n_items flags, then the ticket counter
-    float* agg_a;     // n_items * CJ
+    float* agg_a;     // n_items * CJ (one value per channel)
     float* agg_b;
     float* prefix;
 };
@@ -87,23 +87,23 @@ __device__ __forceinline__ unsigned scan_wait_flag(const unsigned* flag, unsigne
 }
 
 // Decoupled look-back: the composition of the affine maps of items
-// k-1, k-2, ... (same tile) applied to the first available inclusive prefix.
-// Returns false on abort.
-__device__ __forceinline__ bool scan_lookback(const ScanState& ss, int k, int tile, int n_tiles, int tid,
-                                              unsigned* s_flag, float& carry) {
-    float a_acc = 1.f, b_acc = 0.f;
+// k-1, k-2, ... (same tile) applied to the first available inclusive prefix,
+// for this thread's channel pair (offset cj).  Returns false on abort.
+__device__ __forceinline__ bool scan_lookback(const ScanState& ss, int k, int tile, int n_tiles, int cj,
+                                              unsigned* s_flag, float2& carry) {
+    float2 a_acc = f2(1.f), b_acc = f2(0.f);
     for (int p = k - 1; p >= 0; --p) {
         const size_t item = (size_t)p * n_tiles + tile;
         const unsigned f = scan_wait_flag(&ss.flags[item], s_flag);
         if (f == kFlagAbort) return false;
         if (f == kFlagPrefix) {
-            carry = fmaf(a_acc, ld_relaxed_gpu(&ss.prefix[item * kRecCJ + tid]), b_acc);
+            carry = fma2(a_acc, ld_relaxed_gpu2(&ss.prefix[item * kRecCJ + cj]), b_acc);
             return true;
         }
-        const float a = ld_relaxed_gpu(&ss.agg_a[item * kRecCJ + tid]);
-        const float bb = ld_relaxed_gpu(&ss.agg_b[item * kRecCJ + tid]);
-        b_acc = fmaf(a_acc, bb, b_acc);
-        a_acc *= a;
+        const float2 a = ld_relaxed_gpu2(&ss.agg_a[item * kRecCJ + cj]);
+        const float2 bb = ld_relaxed_gpu2(&ss.agg_b[item * kRecCJ + cj]);
+        b_acc = fma2(a_acc, bb, b_acc);
+        a_acc = mul2(a_acc, a);
     }
     carry = b_acc;  // unreachable in practice: item 0 always publishes a prefix
     return true;
@@ -124,7 +124,7 @@ struct FwdScanLayout {
 
 // Forward, v = 0.  1-D grid of n_items = ceil(L/kScanT) * ceil(d/CJ) * B * n_dir CTAs.
 template <typename UT>
-__global__ void __launch_bounds__(kRecCJ) sru_fwd_scan_kernel(
+__global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
     const float* __restrict__ bias, const float* __restrict__ c0, const uint8_t* __restrict__ mask,
     float* __restrict__ h, float* __restrict__ c_T, float* __restrict__ ckpt, ScanState ss, int L, int B, int d,
@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kRecCJ) sru_fwd_scan_kernel(
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
     unsigned* s_misc = reinterpret_cast<unsigned*>(bar + 1);  // [0] ticket, [1] flag
 
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid, cj = 2 * lane;
     const int n_jt = (d + kRecCJ - 1) / kRecCJ;
     const int n_tiles = n_jt * B * n_dir;
     const int n_items = gridDim.x;
@@ -152,12 +152,14 @@ __global__ void __launch_bounds__(kRecCJ) sru_fwd_scan_kernel(
     const int nchs = (L + kScanT - 1) / kScanT;
     const int tc = dir == 0 ? k : nchs - 1 - k;
     const int t0 = tc * kScanT;
-    const int j0 = jt * kRecCJ, j = j0 + tid;
+    const int j0 = jt * kRecCJ, j = j0 + cj;
     const bool jok = j < d;
     const int nch16 = (L + kChunkT - 1) / kChunkT;
 
-    GateParams p = make_gate_params(0.f, 0.f, 0.f, 0.f);
-    if (jok) p = make_gate_params(0.f, 0.f, bias[(dir * 2 + 0) * d + j], bias[(dir * 2 + 1) * d + j]);
+    GateParams2 p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
+    if (jok)
+        p = make_gate_params2(f2(0.f), f2(0.f), load_pair(bias + (dir * 2 + 0) * d + j),
+                              load_pair(bias + (dir * 2 + 1) * d + j));
     uint32_t valid[kScanSub], inrange[kScanSub];
     bool any = false;
 #pragma unroll
@@ -190,7 +192,7 @@ __global__ void __launch_bounds__(kRecCJ) sru_fwd_scan_kernel(
     }
 
     // 1. the chunk as an affine map of the entering state: c_out = A c_in + Bc
-    float A = 1.f, Bc = 0.f;
+    float2 A = f2(1.f), Bc = f2(0.f);
 #pragma unroll
     for (int qq = 0; qq < kScanSub; ++qq) {
         const int q = dir == 0 ? qq : kScanSub - 1 - qq;
@@ -199,32 +201,34 @@ __global__ void __launch_bounds__(kRecCJ) sru_fwd_scan_kernel(
         for (int r = 0; r < kChunkT; ++r) {
             const int i = dir == 0 ? r : kChunkT - 1 - r;
             if ((valid[q] >> i) & 1u) {
-                const float uc = to_f32(us[(i * 3 + 0) * kRecCJ + tid]);
-                const float f = sigmoid_nl2(__fmaf_rn(to_f32(us[(i * 3 + 1) * kRecCJ + tid]), kNegLog2e, p.nbf));
-                A *= f;
-                Bc = fmaf(f, Bc - uc, uc);
+                const float2 uc = load_pair(us + (i * 3 + 0) * kRecCJ + cj);
+                const float2 f =
+                    sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 1) * kRecCJ + cj), f2(kNegLog2e), p.nbf));
+                A = mul2(A, f);
+                Bc = fma2(f, sub2(Bc, uc), uc);
             }
         }
     }
     // 2. state entering the chunk
-    float c_in = 0.f;
-    const size_t me = (size_t)w * kRecCJ + tid;
+    float2 c_in = f2(0.f);
+    const size_t me = (size_t)w * kRecCJ + cj;
     if (k == 0) {
-        c_in = (jok && c0 != nullptr) ? c0[(size_t)bd * d + j] : 0.f;
+        c_in = (jok && c0 != nullptr) ? load_pair(c0 + (size_t)bd * d + j) : f2(0.f);
     } else {
-        ss.agg_a[me] = A;
-        ss.agg_b[me] = Bc;
+        store_pair(ss.agg_a + me, A);
+        store_pair(ss.agg_b + me, Bc);
         scan_publish(&ss.flags[w], kFlagAgg);
-        if (!scan_lookback(ss, k, tile, n_tiles, tid, s_misc + 1, c_in)) {
+        if (!scan_lookback(ss, k, tile, n_tiles, cj, s_misc + 1, c_in)) {
             scan_publish(&ss.flags[w], kFlagAbort);
             return;
         }
     }
-    ss.prefix[me] = fmaf(A, c_in, Bc);
+    store_pair(ss.prefix + me, fma2(A, c_in, Bc));
     scan_publish(&ss.flags[w], kFlagPrefix);
 
     // 3. walk the chunk again from shared memory: h and the 16-step checkpoints
-    float c = c_in;
+    float2 c = c_in;
+    const float2 alpha2 = f2(alpha);
     const size_t h_tstride = (size_t)B * n_dir * d;
 #pragma unroll
     for (int qq = 0; qq < kScanSub; ++qq) {
@@ -232,13 +236,13 @@ __global__ void __launch_bounds__(kRecCJ) sru_fwd_scan_kernel(
         const int ts = t0 + q * kChunkT;
         if (ts >= L) continue;
         const int c16 = tc * kScanSub + q;
-        if (ckpt != nullptr && jok && c16 < nch16) ckpt[((size_t)c16 * B * n_dir + bd) * d + j] = c;
+        if (ckpt != nullptr && jok && c16 < nch16) store_pair(ckpt + ((size_t)c16 * B * n_dir + bd) * d + j, c);
         const UT* us = reinterpret_cast<const UT*>(smem + q * Lay::STAGE);
         const float* xs = reinterpret_cast<const float*>(smem + q * Lay::STAGE + FwdLayout<UT>::U_BYTES);
         float* hp = h + (size_t)ts * h_tstride + (size_t)bd * d + j;
-        c = fwd_chunk<UT>(us, xs, valid[q], inrange[q], c, p, alpha, dir, hp, h_tstride, jok, tid);
+        c = fwd_chunk<UT, kRecCJ>(us, xs, valid[q], inrange[q], c, p, alpha2, dir, hp, h_tstride, jok, cj);
     }
-    if (k == nchs - 1 && jok) c_T[(size_t)bd * d + j] = c;
+    if (k == nchs - 1 && jok) store_pair(c_T + (size_t)bd * d + j, c);
 }
 
 template <typename UT, bool ACC_DX>
@@ -251,7 +255,7 @@ struct BwdScanLayout {
 // Backward of direction DIR, v = 0.  1-D grid of n_items = ceil(L/kScanT) * ceil(d/CJ) * B.
 // partial: (nchs * B, n_dir, 4, d) doubles.
 template <typename UT, typename DUT, bool ACC_DX, int DIR>
-__global__ void __launch_bounds__(kRecCJ) sru_bwd_scan_kernel(
+__global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
     const __grid_constant__ CUtensorMap map_dh, const __grid_constant__ CUtensorMap map_dxin,
     const float* __restrict__ bias, const uint8_t* __restrict__ mask, const float* __restrict__ ckpt,
@@ -264,7 +268,7 @@ __global__ void __launch_bounds__(kRecCJ) sru_bwd_scan_kernel(
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
     unsigned* s_misc = reinterpret_cast<unsigned*>(bar + 1);
 
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid, cj = 2 * lane;
     const int n_jt = (d + kRecCJ - 1) / kRecCJ;
     const int n_tiles = n_jt * B;
     const int n_items = gridDim.x;
@@ -281,11 +285,13 @@ __global__ void __launch_bounds__(kRecCJ) sru_bwd_scan_kernel(
     const int nchs = (L + kScanT - 1) / kScanT;
     const int tc = DIR == 0 ? nchs - 1 - k : k;  // backward walks direction 0 from the end
     const int t0 = tc * kScanT;
-    const int j0 = jt * kRecCJ, j = j0 + tid;
+    const int j0 = jt * kRecCJ, j = j0 + cj;
     const bool jok = j < d;
 
-    GateParams p = make_gate_params(0.f, 0.f, 0.f, 0.f);
-    if (jok) p = make_gate_params(0.f, 0.f, bias[(DIR * 2 + 0) * d + j], bias[(DIR * 2 + 1) * d + j]);
+    GateParams2 p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
+    if (jok)
+        p = make_gate_params2(f2(0.f), f2(0.f), load_pair(bias + (DIR * 2 + 0) * d + j),
+                              load_pair(bias + (DIR * 2 + 1) * d + j));
     uint32_t valid[kScanSub], inrange[kScanSub];
     bool any = false;
 #pragma unroll
@@ -322,7 +328,7 @@ __global__ void __launch_bounds__(kRecCJ) sru_bwd_scan_kernel(
 
     // 1. the chunk as an affine map of the state gradient: g_out = A g_in + Bg,
     //    g <- f (g + dh r) per valid row, in backward order
-    float A = 1.f, Bg = 0.f;
+    float2 A = f2(1.f), Bg = f2(0.f);
 #pragma unroll
     for (int qq = 0; qq < kScanSub; ++qq) {
         const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
@@ -332,33 +338,36 @@ __global__ void __launch_bounds__(kRecCJ) sru_bwd_scan_kernel(
         for (int r = 0; r < kChunkT; ++r) {
             const int i = DIR == 0 ? kChunkT - 1 - r : r;
             if ((valid[q] >> i) & 1u) {
-                const float f = sigmoid_nl2(__fmaf_rn(to_f32(us[(i * 3 + 1) * kRecCJ + tid]), kNegLog2e, p.nbf));
-                const float rr = sigmoid_nl2(__fmaf_rn(to_f32(us[(i * 3 + 2) * kRecCJ + tid]), kNegLog2e, p.nbr));
-                A *= f;
-                Bg = f * fmaf(dhs[i * kRecCJ + tid], rr, Bg);
+                const float2 f =
+                    sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 1) * kRecCJ + cj), f2(kNegLog2e), p.nbf));
+                const float2 rr =
+                    sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 2) * kRecCJ + cj), f2(kNegLog2e), p.nbr));
+                A = mul2(A, f);
+                Bg = mul2(f, fma2(load_pair(dhs + i * kRecCJ + cj), rr, Bg));
             }
         }
     }
     // 2. state gradient entering the chunk (from later times)
-    float g_in = 0.f;
-    const size_t me = (size_t)w * kRecCJ + tid;
+    float2 g_in = f2(0.f);
+    const size_t me = (size_t)w * kRecCJ + cj;
     if (k == 0) {
-        g_in = (jok && dc_T != nullptr) ? dc_T[(size_t)bd * d + j] : 0.f;
+        g_in = (jok && dc_T != nullptr) ? load_pair(dc_T + (size_t)bd * d + j) : f2(0.f);
     } else {
-        ss.agg_a[me] = A;
-        ss.agg_b[me] = Bg;
+        store_pair(ss.agg_a + me, A);
+        store_pair(ss.agg_b + me, Bg);
         scan_publish(&ss.flags[w], kFlagAgg);
-        if (!scan_lookback(ss, k, tile, n_tiles, tid, s_misc + 1, g_in)) {
+        if (!scan_lookback(ss, k, tile, n_tiles, cj, s_misc + 1, g_in)) {
             scan_publish(&ss.flags[w], kFlagAbort);
             return;
         }
     }
-    ss.prefix[me] = fmaf(A, g_in, Bg);
+    store_pair(ss.prefix + me, fma2(A, g_in, Bg));
     scan_publish(&ss.flags[w], kFlagPrefix);
 
     // 3. gradients of every row, sub-chunk by sub-chunk in backward order
-    float g = g_in;
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    float2 g = g_in;
+    const float2 alpha2 = f2(alpha);
+    double acc[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
     const size_t u_tstride = (size_t)B * n_dir * 3 * d;
     const size_t x_tstride = (size_t)B * d;
 #pragma unroll
@@ -377,17 +386,13 @@ __global__ void __launch_bounds__(kRecCJ) sru_bwd_scan_kernel(
         const float* dhs = xs + kChunkT * kRecCJ;
         const float* dxin = dhs + kChunkT * kRecCJ;
         const int c16 = tc * kScanSub + q;
-        const float c_start = jok ? ckpt[((size_t)c16 * B * n_dir + bd) * d + j] : 0.f;
-        bwd_chunk<UT, DUT, ACC_DX, DIR>(us, xs, dhs, dxin, valid[q], inrange[q], c_start, p, alpha, g, acc, dUp,
-                                        dxp, u_tstride, x_tstride, d, jok, tid);
+        const float2 c_start = jok ? load_pair(ckpt + ((size_t)c16 * B * n_dir + bd) * d + j) : f2(0.f);
+        bwd_chunk<UT, DUT, ACC_DX, DIR, kRecCJ>(us, xs, dhs, dxin, valid[q], inrange[q], c_start, p, alpha2, g, acc, dUp,
+                                        dxp, u_tstride, x_tstride, d, jok, cj);
     }
     if (jok) {
-        if (k == nchs - 1) dc0[(size_t)bd * d + j] = g;
-        double* pp = partial + (((size_t)tc * B + b) * n_dir + DIR) * 4 * d + j;
-        pp[0] = acc[0];
-        pp[(size_t)d] = acc[1];
-        pp[(size_t)2 * d] = acc[2];
-        pp[(size_t)3 * d] = acc[3];
+        if (k == nchs - 1) store_pair(dc0 + (size_t)bd * d + j, g);
+        store_partials(partial + (((size_t)tc * B + b) * n_dir + DIR) * 4 * d + j, acc, d);
     }
 }
 
