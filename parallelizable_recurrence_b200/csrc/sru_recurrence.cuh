@@ -104,6 +104,25 @@ __device__ __forceinline__ void store_pair(__nv_bfloat16* p, float2 v) {
     *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v.x, v.y);
 }
 
+// A channel pair of U as held in registers before use: the raw bf16x2 word
+// (one 32-bit register) or the fp32 pair.
+template <typename UT>
+struct PairWord;
+template <>
+struct PairWord<__nv_bfloat16> {
+    using T = uint32_t;
+    static __device__ __forceinline__ T load(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
+    static __device__ __forceinline__ float2 unpack(T w) {
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    }
+};
+template <>
+struct PairWord<float> {
+    using T = float2;
+    static __device__ __forceinline__ T load(const float* p) { return *reinterpret_cast<const float2*>(p); }
+    static __device__ __forceinline__ float2 unpack(T w) { return w; }
+};
+
 // Bit i set: row t0+i of this chunk exists (t < L) and is not padded.  Whole warp calls.
 __device__ __forceinline__ uint32_t chunk_valid_bits(const uint8_t* __restrict__ mask, int t0, int L, int B,
                                                      int b, int lane) {
@@ -130,24 +149,51 @@ __device__ __forceinline__ void drain_pending_loads(uint64_t* full, uint32_t pen
 // (us: [T][3][CJ] gate blocks, xs: [T][CJ]), walked in the direction's time
 // order from state c, for this thread's channel pair (offset cj in the tile).
 // Writes h for the rows that exist (0 at padded rows); returns the state.
+// Fast path of fwd_chunk for a chunk whose 16 rows all exist and are valid,
+// in direction DIR's time order: the chunk's operands are first copied from
+// shared memory into registers, the 16 dependent steps then run on registers
+// only, and the outputs are stored last.  With about one warp per SM
+// sub-partition the serial chain of a step (two MUFU round trips) must not
+// also wait on shared-memory loads or store addressing.
+template <typename UT, int CJ, int DIR>
+__device__ __forceinline__ float2 fwd_chunk_full(const UT* __restrict__ us, const float* __restrict__ xs, float2 c,
+                                                 const GateParams2& p, float2 alpha, float* __restrict__ hp,
+                                                 size_t h_tstride, bool jok, int cj) {
+    using PW = PairWord<UT>;
+    typename PW::T wc[kChunkT], wf[kChunkT], wr[kChunkT];
+    float2 wx[kChunkT];
+#pragma unroll
+    for (int i = 0; i < kChunkT; ++i) {
+        wc[i] = PW::load(us + (i * 3 + 0) * CJ + cj);
+        wf[i] = PW::load(us + (i * 3 + 1) * CJ + cj);
+        wr[i] = PW::load(us + (i * 3 + 2) * CJ + cj);
+        wx[i] = load_pair(xs + i * CJ + cj);
+    }
+    float2 hv[kChunkT];
+#pragma unroll
+    for (int q = 0; q < kChunkT; ++q) {
+        const int i = DIR == 0 ? q : kChunkT - 1 - q;
+        float2 f, r;
+        c = sru_cell2(c, PW::unpack(wc[i]), PW::unpack(wf[i]), PW::unpack(wr[i]), p, f, r);
+        const float2 ax = mul2(alpha, wx[i]);
+        hv[i] = fma2(r, sub2(c, ax), ax);  // Eq. (5)
+    }
+    if (jok) {
+#pragma unroll
+        for (int i = 0; i < kChunkT; ++i) store_pair(hp + (size_t)i * h_tstride, hv[i]);
+    }
+    return c;
+}
+
 template <typename UT, int CJ = kRecCJ>
 __device__ __forceinline__ float2 fwd_chunk(const UT* __restrict__ us, const float* __restrict__ xs,
                                             uint32_t valid, uint32_t inrange, float2 c, const GateParams2& p,
                                             float2 alpha, int dir, float* __restrict__ hp, size_t h_tstride,
                                             bool jok, int cj) {
     constexpr uint32_t kFull = (1u << kChunkT) - 1u;
-    if (valid == kFull) {  // every row present and unpadded: no per-row predicates
-#pragma unroll
-        for (int q = 0; q < kChunkT; ++q) {
-            const int i = dir == 0 ? q : kChunkT - 1 - q;
-            float2 f, r;
-            c = sru_cell2(c, load_pair(us + (i * 3 + 0) * CJ + cj), load_pair(us + (i * 3 + 1) * CJ + cj),
-                          load_pair(us + (i * 3 + 2) * CJ + cj), p, f, r);
-            const float2 ax = mul2(alpha, load_pair(xs + i * CJ + cj));
-            if (jok) store_pair(hp + (size_t)i * h_tstride, fma2(r, sub2(c, ax), ax));  // Eq. (5)
-        }
-        return c;
-    }
+    if (valid == kFull)
+        return dir == 0 ? fwd_chunk_full<UT, CJ, 0>(us, xs, c, p, alpha, hp, h_tstride, jok, cj)
+                        : fwd_chunk_full<UT, CJ, 1>(us, xs, c, p, alpha, hp, h_tstride, jok, cj);
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
         const int i = dir == 0 ? q : kChunkT - 1 - q;
@@ -265,7 +311,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
 // the dv/db partial sums in acc[q] = {dv_f, dv_r, db_f, db_r} (per channel of
 // the pair), and updates g.
 template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ = kRecCJ>
-__device__ __forceinline__ void bwd_chunk(const UT* __restrict__ us, const float* __restrict__ xs,
+__device__ __forceinline__ void bwd_chunk_any(const UT* __restrict__ us, const float* __restrict__ xs,
                                           const float* __restrict__ dhs, const float* __restrict__ dxin,
                                           uint32_t valid, uint32_t inrange, float2 c, const GateParams2& p,
                                           float2 alpha, float2& g, double (&acc)[4][2], DUT* __restrict__ dUp,
@@ -330,6 +376,89 @@ __device__ __forceinline__ void bwd_chunk(const UT* __restrict__ us, const float
     acc[2][1] += (double)s_bf.y;
     acc[3][0] += (double)s_br.x;
     acc[3][1] += (double)s_br.y;
+}
+
+// Fast path of bwd_chunk for a chunk whose 16 rows all exist and are valid:
+// the state chain's operands are copied from shared memory into registers
+// before the chain runs, and no row carries a predicate.
+template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ>
+__device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const float* __restrict__ xs,
+                                               const float* __restrict__ dhs, const float* __restrict__ dxin,
+                                               float2 c, const GateParams2& p, float2 alpha, float2& g,
+                                               double (&acc)[4][2], DUT* __restrict__ dUp, float* __restrict__ dxp,
+                                               size_t u_tstride, size_t x_tstride, int d, bool jok, int cj) {
+    using PW = PairWord<UT>;
+    typename PW::T wc[kChunkT], wf[kChunkT], wr[kChunkT];
+    float2 wx[kChunkT], wdh[kChunkT];
+#pragma unroll
+    for (int i = 0; i < kChunkT; ++i) {
+        wc[i] = PW::load(us + (i * 3 + 0) * CJ + cj);
+        wf[i] = PW::load(us + (i * 3 + 1) * CJ + cj);
+        wr[i] = PW::load(us + (i * 3 + 2) * CJ + cj);
+        wx[i] = load_pair(xs + i * CJ + cj);
+        wdh[i] = load_pair(dhs + i * CJ + cj);
+    }
+    float2 cp[kChunkT], fs[kChunkT], rs[kChunkT];
+#pragma unroll
+    for (int q = 0; q < kChunkT; ++q) {
+        const int i = DIR == 0 ? q : kChunkT - 1 - q;
+        cp[i] = c;
+        c = sru_cell2(c, PW::unpack(wc[i]), PW::unpack(wf[i]), PW::unpack(wr[i]), p, fs[i], rs[i]);
+    }
+    float2 s_vf = f2(0.f), s_vr = f2(0.f), s_bf = f2(0.f), s_br = f2(0.f);
+#pragma unroll
+    for (int q = 0; q < kChunkT; ++q) {
+        const int i = DIR == 0 ? kChunkT - 1 - q : q;
+        const float2 f = fs[i], r = rs[i], cpv = cp[i];
+        const float2 uc = PW::unpack(wc[i]);
+        const float2 ax = mul2(alpha, wx[i]);
+        const float2 dhv = wdh[i];
+        const float2 cmu = sub2(cpv, uc);
+        const float2 cn = fma2(f, cmu, uc);
+        const float2 G = fma2(dhv, r, g);  // dLoss/dc[t]
+        const float2 omr = sub2(f2(1.f), r), omf = sub2(f2(1.f), f);
+        const float2 dxv = mul2(mul2(dhv, omr), alpha);
+        const float2 dzf = mul2(mul2(G, cmu), mul2(f, omf));
+        const float2 dzr = mul2(mul2(dhv, sub2(cn, ax)), mul2(r, omr));
+        const float2 duc = mul2(G, omf);
+        g = fma2(dzr, p.vr, fma2(dzf, p.vf, mul2(G, f)));  // dLoss/dc[t-1]
+        s_vf = fma2(dzf, cpv, s_vf);
+        s_vr = fma2(dzr, cpv, s_vr);
+        s_bf = add2(s_bf, dzf);
+        s_br = add2(s_br, dzr);
+        if (jok) {
+            store_pair(dUp + (size_t)i * u_tstride, duc);
+            store_pair(dUp + (size_t)i * u_tstride + d, dzf);
+            store_pair(dUp + (size_t)i * u_tstride + 2 * d, dzr);
+            if (ACC_DX)
+                store_pair(dxp + (size_t)i * x_tstride, add2(load_pair(dxin + i * CJ + cj), dxv));
+            else
+                store_pair(dxp + (size_t)i * x_tstride, dxv);
+        }
+    }
+    acc[0][0] += (double)s_vf.x;
+    acc[0][1] += (double)s_vf.y;
+    acc[1][0] += (double)s_vr.x;
+    acc[1][1] += (double)s_vr.y;
+    acc[2][0] += (double)s_bf.x;
+    acc[2][1] += (double)s_bf.y;
+    acc[3][0] += (double)s_br.x;
+    acc[3][1] += (double)s_br.y;
+}
+
+template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ = kRecCJ>
+__device__ __forceinline__ void bwd_chunk(const UT* __restrict__ us, const float* __restrict__ xs,
+                                          const float* __restrict__ dhs, const float* __restrict__ dxin,
+                                          uint32_t valid, uint32_t inrange, float2 c, const GateParams2& p,
+                                          float2 alpha, float2& g, double (&acc)[4][2], DUT* __restrict__ dUp,
+                                          float* __restrict__ dxp, size_t u_tstride, size_t x_tstride, int d,
+                                          bool jok, int cj) {
+    if (valid == (1u << kChunkT) - 1u)
+        bwd_chunk_full<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, dxin, c, p, alpha, g, acc, dUp, dxp, u_tstride,
+                                                 x_tstride, d, jok, cj);
+    else
+        bwd_chunk_any<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, dxin, valid, inrange, c, p, alpha, g, acc, dUp, dxp,
+                                                u_tstride, x_tstride, d, jok, cj);
 }
 
 // A chunk with no valid row: zero dU (and dx unless accumulating); g passes through.
