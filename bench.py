@@ -223,30 +223,32 @@ def run_ours(args):
     dW = torch.empty(N, K, device=dev)
     stream = torch.cuda.current_stream(dev)
     reducer = None
+    from parallelizable_recurrence_b200.dist import GradReducer
     if world > 1:
-        from parallelizable_recurrence_b200.dist import GradReducer
         reducer = GradReducer([dW, dv, db])  # one NCCL all-reduce of the parameter gradients
 
-    def step(ev=None):
+    def step(ev=None, bufs=None):
+        """One training step; bufs = (X, x, dh, dW, dv, db, dc0, reducer) or the default set."""
+        Xb, xb, dhb, dWb, dvb, dbb, dc0b, red = bufs if bufs is not None else (X, x, dh, dW, dv, db, dc0, reducer)
         if ev is not None:
             ev[0].record(stream)
-        sru.sru_project(X, W, U)
+        sru.sru_project(Xb, W, U)
         if ev is not None:
             ev[1].record(stream)
-        sru.sru_forward(U, x, v, b, h, cT, c0=c0, workspace=ws)
+        sru.sru_forward(U, xb, v, b, h, cT, c0=c0, workspace=ws)
         if ev is not None:
             ev[2].record(stream)
-        sru.sru_backward(U, x, v, b, dh, ws, dU, dx, dv, db, dc0, c0=c0)
+        sru.sru_backward(U, xb, v, b, dhb, ws, dU, dx, dvb, dbb, dc0b, c0=c0)
         if ev is not None:
             ev[3].record(stream)
-        sru.sru_project_backward(dU, X, W, dX=dx, accumulate=True)
+        sru.sru_project_backward(dU, Xb, W, dX=dx, accumulate=True)
         if ev is not None:
             ev[4].record(stream)
-        sru.sru_project_backward(dU, X, W, dW=dW)
+        sru.sru_project_backward(dU, Xb, W, dW=dWb)
         if ev is not None:
             ev[5].record(stream)
-        if reducer is not None:  # data-parallel gradient sum over ranks (batch sharding)
-            reducer()
+        if red is not None:  # data-parallel gradient sum over ranks (batch sharding)
+            red()
 
     for _ in range(args.warmup):
         step()
@@ -281,35 +283,70 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     elapsed_ms = float(t.item())
 
-    # ---- end to end: per-step inputs from pinned host memory, gradients back
+    # ---- end to end: every step copies its inputs (X bf16, x and dh fp32) from
+    # pinned host memory and reads its gradients (dW, dv, db, dc0) back.  The
+    # copies run on their own streams, double-buffered, so step k+1's inputs
+    # travel while step k computes and step k's gradients travel back while
+    # step k+1 computes (PCIe is full duplex).
     hX = torch.from_numpy(np.ascontiguousarray(inp["X"]).view(np.int16)).pin_memory()
     hx = torch.from_numpy(inp["x"]).pin_memory()
     hdh = torch.from_numpy(inp["dh"]).pin_memory()
-    out_dW = torch.empty(N, K).pin_memory()
-    out_small = torch.empty(4 * d + B * d).pin_memory()
-    small = torch.empty(4 * d + B * d, device=dev)
-    Xi = X.view(torch.int16)
+    sets = []
+    for i in range(2):
+        Xi = X if i == 0 else torch.empty_like(X)
+        xi = x if i == 0 else torch.empty_like(x)
+        dhi = dh if i == 0 else torch.empty_like(dh)
+        dWi = dW if i == 0 else torch.empty_like(dW)
+        dvi = dv if i == 0 else torch.empty_like(dv)
+        dbi = db if i == 0 else torch.empty_like(db)
+        dc0i = dc0 if i == 0 else torch.empty_like(dc0)
+        red = reducer if i == 0 or world == 1 else GradReducer([dWi, dvi, dbi])
+        small = torch.empty(4 * d + B * d, device=dev)
+        out_dW = torch.empty(N, K).pin_memory()
+        out_small = torch.empty(4 * d + B * d).pin_memory()
+        sets.append(dict(bufs=(Xi, xi, dhi, dWi, dvi, dbi, dc0i, red), small=small, out_dW=out_dW,
+                         out_small=out_small))
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in_ready", "computed", "out_done")}
 
-    def e2e_step():
-        Xi.copy_(hX, non_blocking=True)
-        x.copy_(hx, non_blocking=True)
-        dh.copy_(hdh, non_blocking=True)
-        step()
-        small[:2 * d].copy_(dv.view(-1))
-        small[2 * d:4 * d].copy_(db.view(-1))
-        small[4 * d:].copy_(dc0.view(-1))
-        out_dW.copy_(dW, non_blocking=True)
-        out_small.copy_(small, non_blocking=True)
+    def e2e_run(nsteps, start_ev=None):
+        if start_ev is not None:
+            s_h2d.wait_event(start_ev)
+        for k in range(nsteps):
+            i = k % 2
+            st_ = sets[i]
+            Xi, xi, dhi, dWi, dvi, dbi, dc0i, _ = st_["bufs"]
+            if k >= 2:
+                s_h2d.wait_event(ev["computed"][i])  # step k-2 is done reading this input set
+            with torch.cuda.stream(s_h2d):
+                Xi.view(torch.int16).copy_(hX, non_blocking=True)
+                xi.copy_(hx, non_blocking=True)
+                dhi.copy_(hdh, non_blocking=True)
+                ev["in_ready"][i].record(s_h2d)
+            stream.wait_event(ev["in_ready"][i])
+            if k >= 2:
+                stream.wait_event(ev["out_done"][i])  # step k-2's gradients have left this set
+            step(bufs=st_["bufs"])
+            sm = st_["small"]
+            sm[:2 * d].copy_(dvi.view(-1))
+            sm[2 * d:4 * d].copy_(dbi.view(-1))
+            sm[4 * d:].copy_(dc0i.view(-1))
+            ev["computed"][i].record(stream)
+            s_d2h.wait_event(ev["computed"][i])
+            with torch.cuda.stream(s_d2h):
+                st_["out_dW"].copy_(dWi, non_blocking=True)
+                st_["out_small"].copy_(sm, non_blocking=True)
+                ev["out_done"][i].record(s_d2h)
+        stream.wait_stream(s_h2d)
+        stream.wait_stream(s_d2h)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    e2e_run(max(2, args.warmup))
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    e2e_run(args.steps, start_ev=e0)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
@@ -319,12 +356,18 @@ def run_ours(args):
         dist.barrier()
     e2e_ms = float(t.item())
     h2d = hX.numel() * 2 + hx.numel() * 4 + hdh.numel() * 4
-    d2h = out_dW.numel() * 4 + out_small.numel() * 4
+    d2h = sets[0]["out_dW"].numel() * 4 + sets[0]["out_small"].numel() * 4
+    st = sru.sru_sync_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} in the end-to-end region")
 
     if rank == 0:
         tokens = cfg.tokens * world * args.steps
         value = tokens / (elapsed_ms / 1e3)
         gemm_flops = 2.0 * M * N * K
+        # DRAM read + write per launch from the ncu captures summarised in
+        # profiles/tc_gemm_pair_lm_train.md (same kernels, this workload)
+        gemm_traffic = {"project": 252.1e6, "project_dX": 542.4e6, "project_dW": 461.4e6}
         gemm_ms = {n: phase_ms[n] for n in ("project", "project_dX", "project_dW")}
         dom = max(gemm_ms, key=gemm_ms.get)
         peak_tc = peaks["bf16_tflops_sustained"]
@@ -339,15 +382,17 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 GEMM + f32 recurrence",
             "data": "synthetic", "config": config,
             "roofline": {"bound": "tensor", "kernel": f"tc_gemm ({dom})", "achieved": ach_tc, "peak": peak_tc,
-                         "unit": "TFLOP/s", "frac": ach_tc / peak_tc, "traffic": None,
+                         "unit": "TFLOP/s", "frac": ach_tc / peak_tc, "traffic": gemm_traffic[dom],
+                         "traffic_unit": "bytes per launch (ncu dram read+write)",
                          "peak_source": f"{peaks['source']} bf16 sustained (kernel inside a long step)",
                          "algorithmic_per_launch": f"2*M*N*K = {gemm_flops:.4g} flop"},
             "roofline_recurrence": {
                 "bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
                 "forward": {"achieved": ach_f, "frac": ach_f / peaks["hbm_gbs"], "bytes": fwd_bytes,
-                            "ms": phase_ms["forward"]},
+                            "ms": phase_ms["forward"], "traffic": 450.2e6},
                 "backward": {"achieved": ach_b, "frac": ach_b / peaks["hbm_gbs"], "bytes": bwd_bytes,
-                             "ms": phase_ms["backward"]},
+                             "ms": phase_ms["backward"], "traffic": 773.3e6},
+                "traffic_source": "ncu dram read+write per launch, profiles/sru_{fwd,bwd}_seq_lm_train.md",
                 "frac_of_nominal_8TBs": {"forward": ach_f / 8000.0, "backward": ach_b / 8000.0}},
             "phase_ms": phase_ms,
             "e2e": {"value": cfg.tokens * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",

@@ -64,10 +64,14 @@ typedef enum {
 
 typedef enum { SRU_F32 = 0, SRU_BF16 = 1 } sru_dtype;
 
-/* Caller asserts v == 0 (all entries): the recurrence is then linear in c and
- * may run as a chunked associative scan over t (sru_forward / sru_backward). */
+/* Caller asserts v == 0 (all entries): the state recurrence is then linear in c
+ * and sru_forward may run as a chunked associative scan over t.  (sru_backward
+ * may use its chunked scan for any v: the state-gradient recurrence is affine.)
+ * The library picks a scan when the sequential kernels would leave SMs idle
+ * (fewer than two 64-channel CTAs per SM). */
 #define SRU_FLAG_V_ZERO 0x1u
-/* With SRU_FLAG_V_ZERO: force the scan path / force the sequential path. */
+/* Force the scan paths (the forward scan only with SRU_FLAG_V_ZERO) / force the
+ * sequential paths. */
 #define SRU_FLAG_FORCE_SCAN 0x2u
 #define SRU_FLAG_FORCE_SEQUENTIAL 0x4u
 
@@ -82,9 +86,11 @@ int sru_version(void);
 
 /*
  * Bytes of caller-provided device workspace that sru_forward and sru_backward
- * need for a layer of these sizes and flags.  The workspace carries state
+ * need for a layer of these sizes and flags on the current device (the choice
+ * of scan paths depends on its SM count).  The workspace carries state
  * checkpoints from sru_forward to sru_backward (pass the same buffer to both)
- * and holds the backward's per-row partial sums.  Returns 0 on bad sizes.
+ * and holds the backward's partial sums and the scans' flags and carries.
+ * Returns 0 on bad sizes.
  */
 size_t sru_workspace_bytes(int64_t L, int64_t B, int64_t d, int bidirectional, unsigned flags);
 

@@ -70,8 +70,13 @@ constexpr int kMaxDevices = 64;
 
 int sm_count() {
     static int cache[kMaxDevices] = {0};
+    static bool no_device = false;  // CUDA unavailable: do not retry its (slow) initialisation
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (no_device) return 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        if (cudaGetLastError() == cudaErrorNoDevice || dev < 0) no_device = true;
+        return 148;
+    }
     if (cache[dev] == 0) {
         int n = 0;
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -112,11 +117,13 @@ struct WsLayout {
 
 int64_t scan_chunks(int64_t L) { return (L + sru::kScanT - 1) / sru::kScanT; }
 
+bool ws_has_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir);
+
 WsLayout ws_layout(int64_t L, int64_t B, int64_t d, int n_dir, unsigned flags) {
     WsLayout w{};
     const int64_t nch = (L + sru::kChunkT - 1) / sru::kChunkT;
     const int64_t n_jt = (d + sru::kRecCJ - 1) / sru::kRecCJ;
-    const bool scan = (flags & SRU_FLAG_V_ZERO) != 0;
+    const bool scan = ws_has_scan(flags, L, B, d, n_dir);
     size_t off = 0;
     w.ckpt_off = off;
     off += round256((size_t)nch * B * n_dir * d * sizeof(float));
@@ -148,14 +155,30 @@ sru::ScanState scan_state(void* workspace, const WsLayout& w) {
     return ss;
 }
 
-// The chunked scan pays off when the sequential kernel would leave SMs idle:
-// fewer than two 64-channel CTAs per SM.  Only with SRU_FLAG_V_ZERO.
-bool use_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir) {
+// The chunked scans pay off when the sequential kernels would leave SMs idle:
+// fewer than two 64-channel CTAs per SM.  The forward scan needs
+// SRU_FLAG_V_ZERO (linear state recurrence); the backward scan is exact for
+// any v (the state-gradient recurrence is affine).  FORCE flags override.
+bool seq_underfills(int64_t L, int64_t B, int64_t d, int n_dir_per_launch) {
+    const int64_t seq_ctas = ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B * n_dir_per_launch;
+    return L >= 2 * sru::kScanT && seq_ctas < 2 * (int64_t)sm_count();
+}
+bool use_fwd_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir) {
     if (!(flags & SRU_FLAG_V_ZERO)) return false;
     if (flags & SRU_FLAG_FORCE_SCAN) return true;
     if (flags & SRU_FLAG_FORCE_SEQUENTIAL) return false;
-    const int64_t seq_ctas = ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B * n_dir;
-    return L >= 2 * sru::kScanT && seq_ctas < 2 * (int64_t)sm_count();
+    return seq_underfills(L, B, d, n_dir);
+}
+bool use_bwd_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir) {
+    (void)n_dir;
+    if (flags & SRU_FLAG_FORCE_SCAN) return true;
+    if (flags & SRU_FLAG_FORCE_SEQUENTIAL) return false;
+    return seq_underfills(L, B, d, 1);  // one direction per backward launch
+}
+// Whether a workspace for these sizes and flags carries the scan regions.
+bool ws_has_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir) {
+    return use_fwd_scan(flags, L, B, d, n_dir) || use_bwd_scan(flags, L, B, d, n_dir) ||
+           (flags & SRU_FLAG_V_ZERO) != 0;
 }
 
 sru_status check_layer_sizes(int64_t L, int64_t B, int64_t d) {
@@ -354,35 +377,49 @@ sru_status launch_fwd_scan(const RecMaps& mp, const float* b, const float* c0, c
     return SRU_OK;
 }
 
-template <typename UT, typename DUT, bool ACC, int DIR>
-sru_status launch_bwd_scan_dir(const RecMaps& mp, const float* b, const uint8_t* mask, const float* ckpt,
+template <typename UT, typename DUT, bool ACC, int DIR, bool VZ>
+sru_status launch_bwd_scan_dir(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
+                               const float* ckpt,
                                const float* dc_T, DUT* dU, float* dx, double* partial, float* dc0,
                                const sru::ScanState& ss, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
                                cudaStream_t st) {
     using Lay = sru::BwdScanLayout<UT, ACC>;
-    auto kern = sru::sru_bwd_scan_kernel<UT, DUT, ACC, DIR>;
+    auto kern = sru::sru_bwd_scan_kernel<UT, DUT, ACC, DIR, VZ>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
     const int64_t items = scan_chunks(L) * ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B;
     if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
     sru_status s = reset_scan_flags(ss.flags, items + 1, st);
     if (s != SRU_OK) return s;
-    kern<<<(unsigned)items, sru::kRecThreads, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.dx, b, mask, ckpt, dc_T, dU, dx,
+    kern<<<(unsigned)items, sru::kRecThreads, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.dx, v, b, mask, ckpt, dc_T, dU, dx,
                                                           partial, dc0, ss, (int)L, (int)B, (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
 
+template <typename UT, typename DUT, bool VZ>
+sru_status launch_bwd_scan_vz(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
+                              const float* ckpt, const float* dc_T, DUT* du, float* dx, double* partial, float* dc0,
+                              const sru::ScanState& ss, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
+                              cudaStream_t st) {
+    sru_status s = launch_bwd_scan_dir<UT, DUT, false, 0, VZ>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, ss,
+                                                             L, B, d, n_dir, alpha, st);
+    if (s != SRU_OK || n_dir == 1) return s;
+    return launch_bwd_scan_dir<UT, DUT, true, 1, VZ>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, ss, L, B, d,
+                                                    n_dir, alpha, st);
+}
+
+// v_zero: the caller asserted v == 0 (SRU_FLAG_V_ZERO), so the chunk maps need no state.
 template <typename UT, typename DUT>
-sru_status launch_bwd_scan(const RecMaps& mp, const float* b, const uint8_t* mask, const float* ckpt,
+sru_status launch_bwd_scan(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask, const float* ckpt,
                            const float* dc_T, void* dU, float* dx, double* partial, float* dc0,
                            const sru::ScanState& ss, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool v_zero) {
     DUT* du = reinterpret_cast<DUT*>(dU);
-    sru_status s = launch_bwd_scan_dir<UT, DUT, false, 0>(mp, b, mask, ckpt, dc_T, du, dx, partial, dc0, ss, L, B,
-                                                         d, n_dir, alpha, st);
-    if (s != SRU_OK || n_dir == 1) return s;
-    return launch_bwd_scan_dir<UT, DUT, true, 1>(mp, b, mask, ckpt, dc_T, du, dx, partial, dc0, ss, L, B, d, n_dir,
-                                                alpha, st);
+    if (v_zero)
+        return launch_bwd_scan_vz<UT, DUT, true>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, ss, L, B, d,
+                                                 n_dir, alpha, st);
+    return launch_bwd_scan_vz<UT, DUT, false>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, ss, L, B, d, n_dir,
+                                              alpha, st);
 }
 
 }  // namespace
@@ -543,7 +580,7 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
     }
     if (!U || !x || !h || !aligned16(U) || !aligned16(x) || !aligned16(h)) return SRU_ERR_INVALID;
     const WsLayout w = ws_layout(L, B, d, n_dir, flags);
-    const bool scan = use_scan(flags, L, B, d, n_dir);
+    const bool scan = use_fwd_scan(flags, L, B, d, n_dir);
     if (workspace) {
         if (!aligned16(workspace) || workspace_bytes < w.total) return SRU_ERR_INVALID;
     } else if (scan) {
@@ -595,7 +632,7 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
         return SRU_ERR_INVALID;
     const WsLayout w = ws_layout(L, B, d, n_dir, flags);
     if (workspace_bytes < w.total) return SRU_ERR_INVALID;
-    const bool scan = use_scan(flags, L, B, d, n_dir);
+    const bool scan = use_bwd_scan(flags, L, B, d, n_dir);
     const int cj = scan ? sru::kRecCJ : pick_seq_cj(B, d, 1);
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj) ||
@@ -608,15 +645,15 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     if (scan) {
         const sru::ScanState ss = scan_state(workspace, w);
         if (ub)
-            s = db16 ? launch_bwd_scan<__nv_bfloat16, __nv_bfloat16>(mp, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss,
-                                                                     L, B, d, n_dir, alpha, st)
-                     : launch_bwd_scan<__nv_bfloat16, float>(mp, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss, L, B,
-                                                             d, n_dir, alpha, st);
+            s = db16 ? launch_bwd_scan<__nv_bfloat16, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss,
+                                                                     L, B, d, n_dir, alpha, st, (flags & SRU_FLAG_V_ZERO) != 0)
+                     : launch_bwd_scan<__nv_bfloat16, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss, L, B,
+                                                             d, n_dir, alpha, st, (flags & SRU_FLAG_V_ZERO) != 0);
         else
-            s = db16 ? launch_bwd_scan<float, __nv_bfloat16>(mp, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss, L, B,
-                                                             d, n_dir, alpha, st)
-                     : launch_bwd_scan<float, float>(mp, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss, L, B, d, n_dir,
-                                                     alpha, st);
+            s = db16 ? launch_bwd_scan<float, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss, L, B,
+                                                             d, n_dir, alpha, st, (flags & SRU_FLAG_V_ZERO) != 0)
+                     : launch_bwd_scan<float, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss, L, B, d, n_dir,
+                                                     alpha, st, (flags & SRU_FLAG_V_ZERO) != 0);
     } else {
         if (ub)
             s = db16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(cj, mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L,

@@ -20,8 +20,12 @@
 // releases every successor, records kErrTimeoutScan and returns.
 // The chunk is then walked again from shared memory with the carried-in state
 // (forward: h, checkpoints; backward: dU, dx, dv/db partials).
-// The backward uses the same scheme on the state gradient, which for v = 0 is
-// the linear recurrence g[t-1] = f[t] (g[t] + dh[t] r[t]).
+// The backward uses the same scheme on the state gradient g = dLoss/dc, whose
+// recurrence is affine in g for ANY v (the peepholes only make its
+// coefficients depend on the forward state, which each chunk recomputes from
+// the forward's checkpoints): g[t-1] = a[t] g[t] + b[t].  So the backward scan
+// serves every layer whose sequential grid would underfill the GPU, not only
+// v = 0; the forward scan needs v = 0.
 #pragma once
 
 #include "sru_recurrence.cuh"
@@ -254,13 +258,14 @@ struct BwdScanLayout {
 
 // Backward of direction DIR, v = 0.  1-D grid of n_items = ceil(L/kScanT) * ceil(d/CJ) * B.
 // partial: (nchs * B, n_dir, 4, d) doubles.
-template <typename UT, typename DUT, bool ACC_DX, int DIR>
+template <typename UT, typename DUT, bool ACC_DX, int DIR, bool VZERO>
 __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
     const __grid_constant__ CUtensorMap map_dh, const __grid_constant__ CUtensorMap map_dxin,
-    const float* __restrict__ bias, const uint8_t* __restrict__ mask, const float* __restrict__ ckpt,
-    const float* __restrict__ dc_T, DUT* __restrict__ dU, float* __restrict__ dx, double* __restrict__ partial,
-    float* __restrict__ dc0, ScanState ss, int L, int B, int d, int n_dir, float alpha) {
+    const float* __restrict__ v, const float* __restrict__ bias, const uint8_t* __restrict__ mask,
+    const float* __restrict__ ckpt, const float* __restrict__ dc_T, DUT* __restrict__ dU, float* __restrict__ dx,
+    double* __restrict__ partial, float* __restrict__ dc0, ScanState ss, int L, int B, int d, int n_dir,
+    float alpha) {
     using Lay = BwdScanLayout<UT, ACC_DX>;
     using SL = BwdLayout<UT, ACC_DX>;
     extern __shared__ uint8_t smem_raw[];
@@ -290,8 +295,10 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
 
     GateParams2 p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
     if (jok)
-        p = make_gate_params2(f2(0.f), f2(0.f), load_pair(bias + (DIR * 2 + 0) * d + j),
-                              load_pair(bias + (DIR * 2 + 1) * d + j));
+        p = make_gate_params2(load_pair(v + (DIR * 2 + 0) * d + j), load_pair(v + (DIR * 2 + 1) * d + j),
+                              load_pair(bias + (DIR * 2 + 0) * d + j), load_pair(bias + (DIR * 2 + 1) * d + j));
+    const float2 alpha2 = f2(alpha);
+    const int nch16 = (L + kChunkT - 1) / kChunkT;
     uint32_t valid[kScanSub], inrange[kScanSub];
     bool any = false;
 #pragma unroll
@@ -326,24 +333,68 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
         }
     }
 
-    // 1. the chunk as an affine map of the state gradient: g_out = A g_in + Bg,
-    //    g <- f (g + dh r) per valid row, in backward order
+    // 1. the chunk as an affine map of the state gradient, g_out = A g_in + Bg.
+    //    Each valid row maps g to a g + b with (see bwd_chunk)
+    //      a = f + (c' - u) f(1-f) v_f,  b = a dh r + dh (c - alpha x) r(1-r) v_r,
+    //    which needs the row's forward state: every 16-step sub-chunk is re-run
+    //    from its checkpoint (bit-identical to the forward), then walked back.
     float2 A = f2(1.f), Bg = f2(0.f);
+    if (VZERO) {
+        // v = 0: the gates do not read c, so a = f and b = f dh r need no state
 #pragma unroll
-    for (int qq = 0; qq < kScanSub; ++qq) {
-        const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
-        const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
-        const float* dhs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES + SL::V_BYTES);
+        for (int qq = 0; qq < kScanSub; ++qq) {
+            const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
+            const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
+            const float* dhs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES + SL::V_BYTES);
 #pragma unroll
-        for (int r = 0; r < kChunkT; ++r) {
-            const int i = DIR == 0 ? kChunkT - 1 - r : r;
-            if ((valid[q] >> i) & 1u) {
-                const float2 f =
-                    sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 1) * kRecCJ + cj), f2(kNegLog2e), p.nbf));
-                const float2 rr =
-                    sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 2) * kRecCJ + cj), f2(kNegLog2e), p.nbr));
-                A = mul2(A, f);
-                Bg = mul2(f, fma2(load_pair(dhs + i * kRecCJ + cj), rr, Bg));
+            for (int r = 0; r < kChunkT; ++r) {
+                const int i = DIR == 0 ? kChunkT - 1 - r : r;
+                if ((valid[q] >> i) & 1u) {
+                    const float2 f =
+                        sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 1) * kRecCJ + cj), f2(kNegLog2e), p.nbf));
+                    const float2 rr =
+                        sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 2) * kRecCJ + cj), f2(kNegLog2e), p.nbr));
+                    A = mul2(A, f);
+                    Bg = mul2(f, fma2(load_pair(dhs + i * kRecCJ + cj), rr, Bg));
+                }
+            }
+        }
+    } else {
+    #pragma unroll
+        for (int qq = 0; qq < kScanSub; ++qq) {
+            const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
+            if (valid[q] == 0u) continue;
+            const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
+            const float* xs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES);
+            const float* dhs = xs + kChunkT * kRecCJ;
+            const int c16 = tc * kScanSub + q;
+            float2 c = (jok && c16 < nch16) ? load_pair(ckpt + ((size_t)c16 * B * n_dir + bd) * d + j) : f2(0.f);
+            float2 cp[kChunkT], fs[kChunkT], rs[kChunkT];
+    #pragma unroll
+            for (int r = 0; r < kChunkT; ++r) {
+                const int i = DIR == 0 ? r : kChunkT - 1 - r;
+                cp[i] = c;
+                fs[i] = f2(0.f);
+                rs[i] = f2(0.f);
+                if ((valid[q] >> i) & 1u)
+                    c = sru_cell2(c, load_pair(us + (i * 3 + 0) * kRecCJ + cj), load_pair(us + (i * 3 + 1) * kRecCJ + cj),
+                                  load_pair(us + (i * 3 + 2) * kRecCJ + cj), p, fs[i], rs[i]);
+            }
+    #pragma unroll
+            for (int r = 0; r < kChunkT; ++r) {
+                const int i = DIR == 0 ? kChunkT - 1 - r : r;
+                if (!((valid[q] >> i) & 1u)) continue;
+                const float2 f = fs[i], rr = rs[i];
+                const float2 uc = load_pair(us + (i * 3 + 0) * kRecCJ + cj);
+                const float2 ax = mul2(alpha2, load_pair(xs + i * kRecCJ + cj));
+                const float2 dhv = load_pair(dhs + i * kRecCJ + cj);
+                const float2 cmu = sub2(cp[i], uc);
+                const float2 cn = fma2(f, cmu, uc);
+                const float2 dzr = mul2(mul2(dhv, sub2(cn, ax)), mul2(rr, sub2(f2(1.f), rr)));
+                const float2 a = fma2(mul2(cmu, mul2(f, sub2(f2(1.f), f))), p.vf, f);
+                const float2 bb = fma2(dzr, p.vr, mul2(a, mul2(dhv, rr)));
+                A = mul2(a, A);
+                Bg = fma2(a, Bg, bb);
             }
         }
     }
@@ -366,7 +417,6 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
 
     // 3. gradients of every row, sub-chunk by sub-chunk in backward order
     float2 g = g_in;
-    const float2 alpha2 = f2(alpha);
     double acc[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
     const size_t u_tstride = (size_t)B * n_dir * 3 * d;
     const size_t x_tstride = (size_t)B * d;

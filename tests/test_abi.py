@@ -95,7 +95,10 @@ def test_invalid_arguments_return_before_any_launch(lib):
     assert st == 1
     st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, fake, fake, need - 1, None)
     assert st == 1
-    # the scan path needs a workspace sized with SRU_FLAG_V_ZERO
-    assert lib.sru_workspace_bytes(4096, 2, 64, 0, 1) > lib.sru_workspace_bytes(4096, 2, 64, 0, 0)
+    # the scan regions: always with SRU_FLAG_V_ZERO; without it only where the
+    # backward would take the scan (a small batch*width); not for a wide layer
+    assert lib.sru_workspace_bytes(4096, 64, 4096, 0, 1) > lib.sru_workspace_bytes(4096, 64, 4096, 0, 0)
+    small = lib.sru_workspace_bytes(4096, 2, 64, 0, 0)
+    assert small >= 4096 // 64 * 2 * (4 + 3 * 64 * 4)
     st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4096, 2, 64, 1.0, 0, 1 | 2, fake, fake, None, 0, None)
     assert st == 1
