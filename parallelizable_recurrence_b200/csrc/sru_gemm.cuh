@@ -287,7 +287,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 // "empty" and "accumulator full" barriers (commit with .multicast::cluster);
 // both CTAs' epilogue warps release the accumulator on the leader's barrier.
 // No TMA load uses cluster multicast.
-constexpr int P_BM = 256, P_BN = 256, P_STAGES = 6;   // per pair (BK as above)
+#ifndef SRU_GEMM_PAIR_STAGES
+#define SRU_GEMM_PAIR_STAGES 6
+#endif
+constexpr int P_BM = 256, P_BN = 256, P_STAGES = SRU_GEMM_PAIR_STAGES;  // per pair (BK as above)
 constexpr int P_CM = 128, P_CN = 128;                  // per CTA
 constexpr uint32_t P_A_BYTES = P_CM * BK * 2;          // 16 KB
 constexpr uint32_t P_B_BYTES = P_CN * BK * 2;          // 16 KB
