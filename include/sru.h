@@ -74,6 +74,14 @@ typedef enum { SRU_F32 = 0, SRU_BF16 = 1 } sru_dtype;
  * sequential paths. */
 #define SRU_FLAG_FORCE_SCAN 0x2u
 #define SRU_FLAG_FORCE_SEQUENTIAL 0x4u
+/* Fault injection, for tests of the failure path only: on a chunked-scan
+ * launch the first work item publishes no carry, so the bounded waits of the
+ * CTAs that look back to it expire (after about 2 s).  They publish an abort
+ * that releases their successors, and return; the call's outputs are then
+ * undefined and the next sru_sync_status() returns SRU_ERR_TIMEOUT.  No fault,
+ * trap or hang is involved, and the context stays usable.  Has no effect on
+ * the sequential kernels. */
+#define SRU_FLAG_TEST_WITHHOLD_CARRY 0x8u
 
 /* Human-readable name of a status code (static string). */
 const char* sru_status_string(int status);

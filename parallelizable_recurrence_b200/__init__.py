@@ -27,6 +27,7 @@ SRU_F32, SRU_BF16 = 0, 1
 SRU_FLAG_V_ZERO = 0x1
 SRU_FLAG_FORCE_SCAN = 0x2
 SRU_FLAG_FORCE_SEQUENTIAL = 0x4
+SRU_FLAG_TEST_WITHHOLD_CARRY = 0x8
 
 # every symbol include/sru.h declares
 EXPORTED = ("sru_status_string", "sru_get_last_cuda_error", "sru_version", "sru_workspace_bytes",

@@ -145,9 +145,10 @@ WsLayout ws_layout(int64_t L, int64_t B, int64_t d, int n_dir, unsigned flags) {
     return w;
 }
 
-sru::ScanState scan_state(void* workspace, const WsLayout& w) {
+sru::ScanState scan_state(void* workspace, const WsLayout& w, unsigned flags) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     sru::ScanState ss;
+    ss.withhold = (flags & SRU_FLAG_TEST_WITHHOLD_CARRY) ? 0 : -1;
     ss.flags = reinterpret_cast<unsigned*>(ws + w.flags_off);
     ss.agg_a = reinterpret_cast<float*>(ws + w.agg_a_off);
     ss.agg_b = reinterpret_cast<float*>(ws + w.agg_b_off);
@@ -276,82 +277,133 @@ bool map_f32_rows(CUtensorMap* m, const float* p, int64_t L, int64_t rows, int64
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// Channel-tile width of the sequential kernels.  Measured on B200 for the
-// language-model training layer (L1024 B16 d2048) and the bidirectional
-// layer (L2048 B64 d1024): 64 channels per CTA beat 128 and 256 (wider rows
-// per TMA box gave 4-25% less bandwidth), so 64 is used throughout.
-int pick_seq_cj(int64_t B, int64_t d, int n_dir) {
-    (void)B;
-    (void)d;
-    (void)n_dir;
-#ifdef SRU_FORCE_CJ
-    return SRU_FORCE_CJ;
-#else
-    return 64;
-#endif
+// CTAs of a kernel (launched with `threads` threads and `smem` bytes of
+// dynamic shared memory) that fit on one SM; cached per (kernel, device).
+int resident_ctas(const void* kernel, int threads, size_t smem) {
+    static std::mutex mu;
+    static const void* known_kernel[256];
+    static int known_dev[256], known_n[256];
+    static int nknown = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < nknown; ++i)
+            if (known_kernel[i] == kernel && known_dev[i] == dev) return known_n[i];
+    }
+    int n = 0;
+    if (ensure_smem(kernel, smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess)
+        n = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (nknown < 256) {
+        known_kernel[nknown] = kernel;
+        known_dev[nknown] = dev;
+        known_n[nknown] = n;
+        ++nknown;
+    }
+    return n;
 }
 
-template <typename UT, int CJ>
-sru_status launch_fwd_seq_cj(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
-                             float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d, int n_dir,
-                             float alpha, cudaStream_t st) {
-    using Lay = sru::FwdLayout<UT, CJ>;
-    auto kern = sru::sru_fwd_seq_kernel<UT, CJ>;
+// Stage count for a sequential-kernel grid of `ctas` CTAs: the fewest waves
+// of resident CTAs, then the deepest ring.  resident[S] = CTAs per SM at S
+// stages (S = 2 .. smax).
+int pick_stages(int64_t ctas, const int* resident, int smax) {
+    int best = smax;
+    int64_t best_waves = INT64_MAX;
+    for (int S = smax; S >= 2; --S) {
+        if (resident[S] <= 0) continue;
+        const int64_t per_wave = (int64_t)sm_count() * resident[S];
+        const int64_t waves = (ctas + per_wave - 1) / per_wave;
+        if (waves < best_waves) {
+            best_waves = waves;
+            best = S;
+        }
+    }
+    return best;
+}
+
+constexpr int kSeqCJ = sru::kRecCJ;  // channels per CTA of the sequential kernels
+
+template <typename UT, int S>
+sru_status launch_fwd_seq_s(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
+                            float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d, int n_dir,
+                            float alpha, cudaStream_t st) {
+    using Lay = sru::FwdLayout<UT, kSeqCJ, S>;
+    auto kern = sru::sru_fwd_seq_kernel<UT, kSeqCJ, S>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
-    dim3 grid((unsigned)((d + CJ - 1) / CJ), (unsigned)B, (unsigned)n_dir);
-    kern<<<grid, CJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, v, b, c0, mask, h, c_T, ckpt, (int)L, (int)B, (int)d, n_dir,
-                                          alpha);
+    dim3 grid((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)B, (unsigned)n_dir);
+    kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, v, b, c0, mask, h, c_T, ckpt, (int)L, (int)B, (int)d,
+                                              n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
+}
+
+template <typename UT, int S>
+int fwd_resident() {
+    return resident_ctas(reinterpret_cast<const void*>(sru::sru_fwd_seq_kernel<UT, kSeqCJ, S>), kSeqCJ / 2,
+                         sru::FwdLayout<UT, kSeqCJ, S>::SMEM);
 }
 
 template <typename UT>
-sru_status launch_fwd_seq(int cj, const RecMaps& mp, const float* v, const float* b, const float* c0,
-                          const uint8_t* mask, float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d,
-                          int n_dir, float alpha, cudaStream_t st) {
-    if (cj == 256) return launch_fwd_seq_cj<UT, 256>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
-    if (cj == 128) return launch_fwd_seq_cj<UT, 128>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
-    return launch_fwd_seq_cj<UT, 64>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+sru_status launch_fwd_seq(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
+                          float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
+                          cudaStream_t st) {
+    static_assert(sru::kFwdStages == 4, "stage dispatch below covers 2..4");
+    const int resident[5] = {0, 0, fwd_resident<UT, 2>(), fwd_resident<UT, 3>(), fwd_resident<UT, 4>()};
+    const int64_t ctas = ((d + kSeqCJ - 1) / kSeqCJ) * B * n_dir;
+    switch (pick_stages(ctas, resident, 4)) {
+        case 2: return launch_fwd_seq_s<UT, 2>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+        case 3: return launch_fwd_seq_s<UT, 3>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+        default: return launch_fwd_seq_s<UT, 4>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+    }
 }
 
-template <typename UT, typename DUT, bool ACC, int DIR, int CJ>
-sru_status launch_bwd_seq_dir(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
-                              const float* ckpt, const float* dc_T, DUT* dU, float* dx, double* partial, float* dc0,
-                              int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
-    using Lay = sru::BwdLayout<UT, ACC, CJ>;
-    auto kern = sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR, CJ>;
+template <typename UT, typename DUT, bool ACC, int DIR, int S>
+sru_status launch_bwd_seq_s(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
+                            const float* ckpt, const float* dc_T, DUT* dU, float* dx, double* partial, float* dc0,
+                            int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
+    using Lay = sru::BwdLayout<UT, ACC, kSeqCJ, S>;
+    auto kern = sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR, kSeqCJ, S>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
-    dim3 grid((unsigned)((d + CJ - 1) / CJ), (unsigned)B, 1);
-    kern<<<grid, CJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.dx, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
-                                          (int)L, (int)B, (int)d, n_dir, alpha);
+    dim3 grid((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)B, 1);
+    kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.dx, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
+                                              (int)L, (int)B, (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
 
-template <typename UT, typename DUT, int CJ>
-sru_status launch_bwd_seq_cj(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
-                             const float* ckpt, const float* dc_T, DUT* du, float* dx, double* partial, float* dc0,
-                             int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
-    sru_status s = launch_bwd_seq_dir<UT, DUT, false, 0, CJ>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B,
-                                                            d, n_dir, alpha, st);
-    if (s != SRU_OK || n_dir == 1) return s;
-    return launch_bwd_seq_dir<UT, DUT, true, 1, CJ>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d,
-                                                   n_dir, alpha, st);
+template <typename UT, typename DUT, bool ACC, int DIR, int S>
+int bwd_resident() {
+    return resident_ctas(reinterpret_cast<const void*>(sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR, kSeqCJ, S>),
+                         kSeqCJ / 2, sru::BwdLayout<UT, ACC, kSeqCJ, S>::SMEM);
+}
+
+// One direction's backward launch.  ACC: dx += this direction's part.
+template <typename UT, typename DUT, bool ACC, int DIR>
+sru_status launch_bwd_seq_dir(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
+                              const float* ckpt, const float* dc_T, DUT* du, float* dx, double* partial, float* dc0,
+                              int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
+    static_assert(sru::kBwdStages == 3, "stage dispatch below covers 2..3");
+    const int resident[4] = {0, 0, bwd_resident<UT, DUT, ACC, DIR, 2>(), bwd_resident<UT, DUT, ACC, DIR, 3>()};
+    const int64_t ctas = ((d + kSeqCJ - 1) / kSeqCJ) * B;
+    if (pick_stages(ctas, resident, 3) == 2)
+        return launch_bwd_seq_s<UT, DUT, ACC, DIR, 2>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d,
+                                                      n_dir, alpha, st);
+    return launch_bwd_seq_s<UT, DUT, ACC, DIR, 3>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir,
+                                                  alpha, st);
 }
 
 template <typename UT, typename DUT>
-sru_status launch_bwd_seq(int cj, const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
-                          const float* ckpt, const float* dc_T, void* dU, float* dx, double* partial, float* dc0,
-                          int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
+sru_status launch_bwd_seq(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask, const float* ckpt,
+                          const float* dc_T, void* dU, float* dx, double* partial, float* dc0, int64_t L, int64_t B,
+                          int64_t d, int n_dir, float alpha, cudaStream_t st) {
     DUT* du = reinterpret_cast<DUT*>(dU);
-    if (cj == 256)
-        return launch_bwd_seq_cj<UT, DUT, 256>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir,
-                                               alpha, st);
-    if (cj == 128)
-        return launch_bwd_seq_cj<UT, DUT, 128>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir,
-                                               alpha, st);
-    return launch_bwd_seq_cj<UT, DUT, 64>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir, alpha,
-                                          st);
+    sru_status s = launch_bwd_seq_dir<UT, DUT, false, 0>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d,
+                                                         n_dir, alpha, st);
+    if (s != SRU_OK || n_dir == 1) return s;
+    return launch_bwd_seq_dir<UT, DUT, true, 1>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir,
+                                                alpha, st);
 }
 
 sru_status reset_scan_flags(unsigned* flags, int64_t n, cudaStream_t st) {
@@ -586,20 +638,20 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
     } else if (scan) {
         return SRU_ERR_INVALID;  // the scan needs its flags and aggregates
     }
-    const int cj = scan ? sru::kRecCJ : pick_seq_cj(B, d, n_dir);
+    const int cj = kSeqCJ;  // the scan kernels use the same 64-channel tiles
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj))
         return SRU_ERR_INVALID;
     float* ckpt = workspace ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.ckpt_off) : nullptr;
     if (scan) {
-        const sru::ScanState ss = scan_state(workspace, w);
+        const sru::ScanState ss = scan_state(workspace, w, flags);
         if (u_t == SRU_BF16)
             return launch_fwd_scan<__nv_bfloat16>(mp, b, c0, mask, h, c_T, ckpt, ss, L, B, d, n_dir, alpha, st);
         return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, ckpt, ss, L, B, d, n_dir, alpha, st);
     }
     if (u_t == SRU_BF16)
-        return launch_fwd_seq<__nv_bfloat16>(cj, mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
-    return launch_fwd_seq<float>(cj, mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+        return launch_fwd_seq<__nv_bfloat16>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+    return launch_fwd_seq<float>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
 }
 
 sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, const float* b, const float* c0,
@@ -633,7 +685,7 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     const WsLayout w = ws_layout(L, B, d, n_dir, flags);
     if (workspace_bytes < w.total) return SRU_ERR_INVALID;
     const bool scan = use_bwd_scan(flags, L, B, d, n_dir);
-    const int cj = scan ? sru::kRecCJ : pick_seq_cj(B, d, 1);
+    const int cj = kSeqCJ;
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj) ||
         !map_f32_rows(&mp.dh, dh, L, B * n_dir, d, cj) || !map_f32_rows(&mp.dx, dx, L, B, d, cj))
@@ -643,7 +695,7 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     double* partial = reinterpret_cast<double*>(ws + w.partial_off);
     const bool ub = u_t == SRU_BF16, db16 = du_t == SRU_BF16;
     if (scan) {
-        const sru::ScanState ss = scan_state(workspace, w);
+        const sru::ScanState ss = scan_state(workspace, w, flags);
         if (ub)
             s = db16 ? launch_bwd_scan<__nv_bfloat16, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss,
                                                                      L, B, d, n_dir, alpha, st, (flags & SRU_FLAG_V_ZERO) != 0)
@@ -656,14 +708,14 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
                                                      alpha, st, (flags & SRU_FLAG_V_ZERO) != 0);
     } else {
         if (ub)
-            s = db16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(cj, mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L,
+            s = db16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L,
                                                                     B, d, n_dir, alpha, st)
-                     : launch_bwd_seq<__nv_bfloat16, float>(cj, mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
+                     : launch_bwd_seq<__nv_bfloat16, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
                                                             n_dir, alpha, st);
         else
-            s = db16 ? launch_bwd_seq<float, __nv_bfloat16>(cj, mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
+            s = db16 ? launch_bwd_seq<float, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
                                                             n_dir, alpha, st)
-                     : launch_bwd_seq<float, float>(cj, mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d, n_dir,
+                     : launch_bwd_seq<float, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d, n_dir,
                                                     alpha, st);
     }
     if (s != SRU_OK) return s;
@@ -703,6 +755,7 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
     ss.agg_a = reinterpret_cast<float*>(base + agg_a_off);
     ss.agg_b = reinterpret_cast<float*>(base + agg_b_off);
     ss.prefix = reinterpret_cast<float*>(base + prefix_off);
+    ss.withhold = -1;
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, sru::kRecCJ) || !map_f32_rows(&mp.x, x, L, B, d, sru::kRecCJ))
         return SRU_ERR_INVALID;

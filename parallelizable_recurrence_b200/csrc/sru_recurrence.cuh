@@ -28,14 +28,12 @@ namespace sru {
 constexpr int kChunkT = 16;          // time steps per pipeline stage == checkpoint interval
 constexpr int kRecCJ = 64;           // channels per CTA
 constexpr int kRecThreads = 32;      // one warp; thread i owns channels 2i and 2i+1 of the tile
-#ifndef SRU_FWD_STAGES
-#define SRU_FWD_STAGES 4
-#endif
-#ifndef SRU_BWD_STAGES
-#define SRU_BWD_STAGES 3
-#endif
-constexpr int kFwdStages = SRU_FWD_STAGES;  // TMA ring depth (build-time tuning knobs)
-constexpr int kBwdStages = SRU_BWD_STAGES;
+// TMA ring depth of the sequential kernels: a template parameter S, from 2 up
+// to these maxima, picked per launch so that the grid needs as few waves of
+// resident CTAs as possible (each CTA walks the whole sequence, so a second,
+// partly filled wave costs as much as the first).
+constexpr int kFwdStages = 4;
+constexpr int kBwdStages = 3;
 constexpr float kNegLog2e = -1.4426950408889634f;
 
 // ------------------------------------------------------------ scalar helpers
@@ -211,25 +209,25 @@ __device__ __forceinline__ float2 fwd_chunk(const UT* __restrict__ us, const flo
     return c;
 }
 
-template <typename UT, int CJ = kRecCJ>
+template <typename UT, int CJ = kRecCJ, int S = kFwdStages>
 struct FwdLayout {
     static constexpr int U_BYTES = kChunkT * 3 * CJ * (int)sizeof(UT);
     static constexpr int X_BYTES = kChunkT * CJ * 4;
     static constexpr int STAGE = U_BYTES + X_BYTES;
-    static constexpr int BAR_OFF = kFwdStages * STAGE;
+    static constexpr int BAR_OFF = S * STAGE;
     static constexpr int SMEM = BAR_OFF + 64 + 128;  // barriers + alignment slack
 };
 
 // Forward.  Grid (ceil(d/CJ), B, n_dir), CJ/2 threads (CJ/64 warps) per CTA.
 //   map_u: 4-D (d, 3, B*n_dir, L) of UT, box (CJ, 3, 1, T)
 //   map_x: 3-D (d, B, L) fp32, box (CJ, 1, T)
-template <typename UT, int CJ>
+template <typename UT, int CJ, int S>
 __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
     const float* __restrict__ v, const float* __restrict__ bias, const float* __restrict__ c0,
     const uint8_t* __restrict__ mask, float* __restrict__ h, float* __restrict__ c_T, float* __restrict__ ckpt,
     int L, int B, int d, int n_dir, float alpha) {
-    using Lay = FwdLayout<UT, CJ>;
+    using Lay = FwdLayout<UT, CJ, S>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
@@ -250,7 +248,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
     }
     const float2 alpha2 = f2(alpha);
     if (tid == 0) {
-        for (int s = 0; s < kFwdStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
         tma_prefetch_desc(&map_u);
         tma_prefetch_desc(&map_x);
@@ -264,7 +262,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
         const int t0 = time_chunk(k) * kChunkT;
         const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
         if (tid == 0 && valid != 0u) {
-            const int s = k % kFwdStages;
+            const int s = k % S;
             pending |= 1u << s;
             uint8_t* st = smem + s * Lay::STAGE;
             mbar_arrive_expect_tx(&full[s], Lay::STAGE);
@@ -273,12 +271,12 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
         }
     };
     if (tid < 32)
-        for (int k = 0; k < kFwdStages && k < nch; ++k) issue(k);
+        for (int k = 0; k < S && k < nch; ++k) issue(k);
 
     uint32_t phase_bits = 0;
     const size_t h_tstride = (size_t)B * n_dir * d;
     for (int k = 0; k < nch; ++k) {
-        const int s = k % kFwdStages;
+        const int s = k % S;
         const int tc = time_chunk(k), t0 = tc * kChunkT;
         const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
         const uint32_t inrange = chunk_inrange_bits(t0, L);
@@ -286,7 +284,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
         if (valid != 0u) {
             const bool ok = mbar_wait(&full[s], (phase_bits >> s) & 1u, kErrTimeoutLoad);
             if (__syncthreads_or(!ok)) {  // a load never landed: give up (error recorded)
-                if (tid == 0) drain_pending_loads<kFwdStages>(full, pending, phase_bits);
+                if (tid == 0) drain_pending_loads<S>(full, pending, phase_bits);
                 return;
             }
             phase_bits ^= 1u << s;
@@ -297,9 +295,32 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
         float* hp = h + (size_t)t0 * h_tstride + (size_t)bd * d + j;
         c = fwd_chunk<UT, CJ>(us, xs, valid, inrange, c, p, alpha2, dir, hp, h_tstride, jok, cj);
         __syncthreads();  // every thread is done with stage s
-        if (tid < 32 && k + kFwdStages < nch) issue(k + kFwdStages);
+        if (tid < 32 && k + S < nch) issue(k + S);
     }
     if (jok) store_pair(c_T + (size_t)bd * d + j, c);
+}
+
+// fp64 totals of a thread's dv/db partial sums, acc[q][e] for
+// q in {dv_f, dv_r, db_f, db_r} and channel e of the pair: in registers, or
+// (SmemPartials) in shared memory, thread-interleaved, so that they hold no
+// registers across a long chunk loop.
+__device__ __forceinline__ void fold_partials(double (&acc)[4][2], const float2 (&s)[4]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        acc[q][0] += (double)s[q].x;
+        acc[q][1] += (double)s[q].y;
+    }
+}
+struct SmemPartials {
+    double* p;  // this thread's first total; total k at p[k * n]
+    int n;      // threads of the CTA
+};
+__device__ __forceinline__ void fold_partials(SmemPartials& acc, const float2 (&s)[4]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        acc.p[(2 * q) * acc.n] += (double)s[q].x;
+        acc.p[(2 * q + 1) * acc.n] += (double)s[q].y;
+    }
 }
 
 // ---------------------------------------------------------------- backward
@@ -310,11 +331,11 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
 // walks it in reverse: writes dU and dx for the rows that exist, accumulates
 // the dv/db partial sums in acc[q] = {dv_f, dv_r, db_f, db_r} (per channel of
 // the pair), and updates g.
-template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ = kRecCJ>
+template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ = kRecCJ, typename ACC>
 __device__ __forceinline__ void bwd_chunk_any(const UT* __restrict__ us, const float* __restrict__ xs,
                                           const float* __restrict__ dhs, const float* __restrict__ dxin,
                                           uint32_t valid, uint32_t inrange, float2 c, const GateParams2& p,
-                                          float2 alpha, float2& g, double (&acc)[4][2], DUT* __restrict__ dUp,
+                                          float2 alpha, float2& g, ACC& acc, DUT* __restrict__ dUp,
                                           float* __restrict__ dxp, size_t u_tstride, size_t x_tstride, int d,
                                           bool jok, int cj) {
     constexpr uint32_t kFull = (1u << kChunkT) - 1u;
@@ -368,24 +389,18 @@ __device__ __forceinline__ void bwd_chunk_any(const UT* __restrict__ us, const f
             }
         }
     }
-    acc[0][0] += (double)s_vf.x;
-    acc[0][1] += (double)s_vf.y;
-    acc[1][0] += (double)s_vr.x;
-    acc[1][1] += (double)s_vr.y;
-    acc[2][0] += (double)s_bf.x;
-    acc[2][1] += (double)s_bf.y;
-    acc[3][0] += (double)s_br.x;
-    acc[3][1] += (double)s_br.y;
+    const float2 s4[4] = {s_vf, s_vr, s_bf, s_br};
+    fold_partials(acc, s4);
 }
 
 // Fast path of bwd_chunk for a chunk whose 16 rows all exist and are valid:
 // the state chain's operands are copied from shared memory into registers
 // before the chain runs, and no row carries a predicate.
-template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ>
+template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ, typename ACC>
 __device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const float* __restrict__ xs,
                                                const float* __restrict__ dhs, const float* __restrict__ dxin,
                                                float2 c, const GateParams2& p, float2 alpha, float2& g,
-                                               double (&acc)[4][2], DUT* __restrict__ dUp, float* __restrict__ dxp,
+                                               ACC& acc, DUT* __restrict__ dUp, float* __restrict__ dxp,
                                                size_t u_tstride, size_t x_tstride, int d, bool jok, int cj) {
     using PW = PairWord<UT>;
     typename PW::T wc[kChunkT], wf[kChunkT], wr[kChunkT];
@@ -436,21 +451,15 @@ __device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const 
                 store_pair(dxp + (size_t)i * x_tstride, dxv);
         }
     }
-    acc[0][0] += (double)s_vf.x;
-    acc[0][1] += (double)s_vf.y;
-    acc[1][0] += (double)s_vr.x;
-    acc[1][1] += (double)s_vr.y;
-    acc[2][0] += (double)s_bf.x;
-    acc[2][1] += (double)s_bf.y;
-    acc[3][0] += (double)s_br.x;
-    acc[3][1] += (double)s_br.y;
+    const float2 s4[4] = {s_vf, s_vr, s_bf, s_br};
+    fold_partials(acc, s4);
 }
 
-template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ = kRecCJ>
+template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ = kRecCJ, typename ACC>
 __device__ __forceinline__ void bwd_chunk(const UT* __restrict__ us, const float* __restrict__ xs,
                                           const float* __restrict__ dhs, const float* __restrict__ dxin,
                                           uint32_t valid, uint32_t inrange, float2 c, const GateParams2& p,
-                                          float2 alpha, float2& g, double (&acc)[4][2], DUT* __restrict__ dUp,
+                                          float2 alpha, float2& g, ACC& acc, DUT* __restrict__ dUp,
                                           float* __restrict__ dxp, size_t u_tstride, size_t x_tstride, int d,
                                           bool jok, int cj) {
     if (valid == (1u << kChunkT) - 1u)
@@ -481,13 +490,19 @@ __device__ __forceinline__ void store_partials(double* __restrict__ pp, const do
 #pragma unroll
     for (int q = 0; q < 4; ++q) *reinterpret_cast<double2*>(pp + (size_t)q * d) = make_double2(acc[q][0], acc[q][1]);
 }
+__device__ __forceinline__ void store_partials(double* __restrict__ pp, const SmemPartials& acc, int d) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<double2*>(pp + (size_t)q * d) = make_double2(acc.p[(2 * q) * acc.n], acc.p[(2 * q + 1) * acc.n]);
+}
 
-template <typename UT, bool ACC_DX, int CJ = kRecCJ>
+template <typename UT, bool ACC_DX, int CJ = kRecCJ, int S = kBwdStages>
 struct BwdLayout {
     static constexpr int U_BYTES = kChunkT * 3 * CJ * (int)sizeof(UT);
     static constexpr int V_BYTES = kChunkT * CJ * 4;  // one fp32 (T, CJ) tile
     static constexpr int STAGE = U_BYTES + V_BYTES * (ACC_DX ? 3 : 2);
-    static constexpr int BAR_OFF = kBwdStages * STAGE;
+    static constexpr int ACC_OFF = S * STAGE;  // SmemPartials: 8 doubles per thread
+    static constexpr int BAR_OFF = ACC_OFF + (CJ / 2) * 8 * 8;
     static constexpr int SMEM = BAR_OFF + 64 + 128;
 };
 
@@ -497,7 +512,7 @@ struct BwdLayout {
 //   map_dh: 3-D (d, B*n_dir, L) fp32; map_dxin: like map_x but over dx.
 // DIR is a template parameter so the per-chunk register arrays are indexed
 // with compile-time constants.
-template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ>
+template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ, int S>
 __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
     const __grid_constant__ CUtensorMap map_dh, const __grid_constant__ CUtensorMap map_dxin,
@@ -505,7 +520,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     const float* __restrict__ ckpt, const float* __restrict__ dc_T, DUT* __restrict__ dU,
     float* __restrict__ dx, double* __restrict__ partial, float* __restrict__ dc0, int L, int B, int d,
     int n_dir, float alpha) {
-    using Lay = BwdLayout<UT, ACC_DX, CJ>;
+    using Lay = BwdLayout<UT, ACC_DX, CJ, S>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
@@ -527,7 +542,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     }
     const float2 alpha2 = f2(alpha);
     if (tid == 0) {
-        for (int s = 0; s < kBwdStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
         tma_prefetch_desc(&map_u);
         tma_prefetch_desc(&map_x);
@@ -543,7 +558,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
         const int t0 = time_chunk(k) * kChunkT;
         const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
         if (tid == 0 && valid != 0u) {
-            const int s = k % kBwdStages;
+            const int s = k % S;
             pending |= 1u << s;
             uint8_t* st = smem + s * Lay::STAGE;
             mbar_arrive_expect_tx(&full[s], Lay::STAGE);
@@ -554,42 +569,56 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
         }
     };
     if (tid < 32)
-        for (int k = 0; k < kBwdStages && k < nch; ++k) issue(k);
+        for (int k = 0; k < S && k < nch; ++k) issue(k);
 
-    double acc[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
+    SmemPartials acc{reinterpret_cast<double*>(smem + Lay::ACC_OFF) + tid, CJ / 2};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc.p[q * acc.n] = 0.0;  // read and written by this thread only
     uint32_t phase_bits = 0;
     const size_t u_tstride = (size_t)B * n_dir * 3 * d;
     const size_t x_tstride = (size_t)B * d;
+    // Checkpoint (state entering the chunk in time order) of backward chunk k.
+    // Loaded two chunks ahead of use so its global-memory latency is not on
+    // the chain.
+    auto ckpt_of = [&](int k) {
+        return (jok && k < nch) ? load_pair(ckpt + ((size_t)time_chunk(k) * B * n_dir + bd) * d + j) : f2(0.f);
+    };
+    // Waits for stage s's load; on expiry every thread leaves (after lane 0
+    // drained the loads in flight).
+    auto wait_stage = [&](int s) {
+        const bool ok = mbar_wait(&full[s], (phase_bits >> s) & 1u, kErrTimeoutLoad);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) drain_pending_loads<S>(full, pending, phase_bits);
+            return false;
+        }
+        return true;
+    };
+    float2 ck0 = ckpt_of(0), ck1 = ckpt_of(1);
     for (int k = 0; k < nch; ++k) {
-        const int s = k % kBwdStages;
+        const int s = k % S;
         const int tc = time_chunk(k), t0 = tc * kChunkT;
         const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
         const uint32_t inrange = chunk_inrange_bits(t0, L);
+        const float2 ck2 = ckpt_of(k + 2);
         DUT* dUp = dU + (size_t)t0 * u_tstride + (size_t)bd * 3 * d + j;
         float* dxp = dx + (size_t)t0 * x_tstride + (size_t)b * d + j;
         if (valid == 0u) {
             bwd_chunk_padded<DUT, ACC_DX>(inrange, dUp, dxp, u_tstride, x_tstride, d, jok);
-            __syncthreads();
-            if (tid < 32 && k + kBwdStages < nch) issue(k + kBwdStages);
-            continue;
+        } else {
+            if (!wait_stage(s)) return;
+            phase_bits ^= 1u << s;
+            pending &= ~(1u << s);
+            const UT* us = reinterpret_cast<const UT*>(smem + s * Lay::STAGE);
+            const float* xs = reinterpret_cast<const float*>(smem + s * Lay::STAGE + Lay::U_BYTES);
+            const float* dhs = xs + kChunkT * CJ;
+            const float* dxin = dhs + kChunkT * CJ;
+            bwd_chunk<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, dxin, valid, inrange, ck0, p, alpha2, g, acc, dUp, dxp,
+                                                u_tstride, x_tstride, d, jok, cj);
         }
-        const bool ok = mbar_wait(&full[s], (phase_bits >> s) & 1u, kErrTimeoutLoad);
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) drain_pending_loads<kBwdStages>(full, pending, phase_bits);
-            return;
-        }
-        phase_bits ^= 1u << s;
-        pending &= ~(1u << s);
-
-        const UT* us = reinterpret_cast<const UT*>(smem + s * Lay::STAGE);
-        const float* xs = reinterpret_cast<const float*>(smem + s * Lay::STAGE + Lay::U_BYTES);
-        const float* dhs = xs + kChunkT * CJ;
-        const float* dxin = dhs + kChunkT * CJ;
-        const float2 c_start = jok ? load_pair(ckpt + ((size_t)tc * B * n_dir + bd) * d + j) : f2(0.f);
-        bwd_chunk<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, dxin, valid, inrange, c_start, p, alpha2, g, acc, dUp,
-                                            dxp, u_tstride, x_tstride, d, jok, cj);
         __syncthreads();
-        if (tid < 32 && k + kBwdStages < nch) issue(k + kBwdStages);
+        if (tid < 32 && k + S < nch) issue(k + S);
+        ck0 = ck1;
+        ck1 = ck2;
     }
     if (jok) {
         store_pair(dc0 + (size_t)bd * d + j, g);

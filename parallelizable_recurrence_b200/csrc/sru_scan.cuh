@@ -56,6 +56,7 @@ struct ScanState {
     float* agg_a;     // n_items * CJ (one value per channel)
     float* agg_b;
     float* prefix;
+    int withhold;     // item that publishes no carry (fault injection for tests); -1 = none
 };
 
 // Whole CTA: publish this item's value(s) (already stored by every thread) under flag f.
@@ -227,6 +228,7 @@ __global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
             return;
         }
     }
+    if (w == ss.withhold) return;  // successors' waits expire (test hook)
     store_pair(ss.prefix + me, fma2(A, c_in, Bc));
     scan_publish(&ss.flags[w], kFlagPrefix);
 
@@ -412,6 +414,7 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
             return;
         }
     }
+    if (w == ss.withhold) return;  // successors' waits expire (test hook)
     store_pair(ss.prefix + me, fma2(A, g_in, Bg));
     scan_publish(&ss.flags[w], kFlagPrefix);
 
