@@ -391,7 +391,7 @@ def run_ours(args):
                 "forward": {"achieved": ach_f, "frac": ach_f / peaks["hbm_gbs"], "bytes": fwd_bytes,
                             "ms": phase_ms["forward"], "traffic": 450.2e6},
                 "backward": {"achieved": ach_b, "frac": ach_b / peaks["hbm_gbs"], "bytes": bwd_bytes,
-                             "ms": phase_ms["backward"], "traffic": 773.3e6},
+                             "ms": phase_ms["backward"], "traffic": 772.0e6},
                 "traffic_source": "ncu dram read+write per launch, profiles/sru_{fwd,bwd}_seq_lm_train.md",
                 "frac_of_nominal_8TBs": {"forward": ach_f / 8000.0, "backward": ach_b / 8000.0}},
             "phase_ms": phase_ms,

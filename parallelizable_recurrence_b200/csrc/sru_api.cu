@@ -68,9 +68,10 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base
 // ------------------------------------------------------------- device facts
 constexpr int kMaxDevices = 64;
 
+bool no_device = false;  // CUDA unavailable: do not retry its (slow) initialisation
+
 int sm_count() {
     static int cache[kMaxDevices] = {0};
-    static bool no_device = false;  // CUDA unavailable: do not retry its (slow) initialisation
     int dev = 0;
     if (no_device) return 148;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -156,30 +157,79 @@ sru::ScanState scan_state(void* workspace, const WsLayout& w, unsigned flags) {
     return ss;
 }
 
-// The chunked scans pay off when the sequential kernels would leave SMs idle:
-// fewer than two 64-channel CTAs per SM.  The forward scan needs
-// SRU_FLAG_V_ZERO (linear state recurrence); the backward scan is exact for
-// any v (the state-gradient recurrence is affine).  FORCE flags override.
-bool seq_underfills(int64_t L, int64_t B, int64_t d, int n_dir_per_launch) {
-    const int64_t seq_ctas = ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B * n_dir_per_launch;
-    return L >= 2 * sru::kScanT && seq_ctas < 2 * (int64_t)sm_count();
+// ------------------------------------------------ sequential kernel or scan
+// The sequential kernels give every CTA a whole sequence (L/16 chunks walked
+// one after another); the chunked scans cut time into kScanT-step work items
+// at the price of a second pass over each item and a look-back.  Measured on
+// B200 over layers from L256 B32 d512 to L8192 B4 d512: one wave of resident
+// scan CTAs costs about as much as kScanWaveChunks sequential 16-step chunks
+// (forward 20 us vs 1.5 us, backward 27 us vs 2.45 us per chunk), so a scan is
+// taken when its waves cost fewer chunks than the sequence has.  Only grids
+// that leave SMs idle (fewer than two sequential CTAs per SM) are candidates.
+// The forward scan needs SRU_FLAG_V_ZERO (linear state recurrence); the
+// backward scan is exact for any v (the state-gradient recurrence is affine).
+// The FORCE flags override.
+constexpr int64_t kScanWaveChunks = 12;
+
+int64_t seq_ctas(int64_t B, int64_t d, int n_dir_per_launch) {
+    return ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B * n_dir_per_launch;
 }
-bool use_fwd_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir) {
+bool scan_candidate(int64_t B, int64_t d, int n_dir_per_launch) {
+    return seq_ctas(B, d, n_dir_per_launch) < 2 * (int64_t)sm_count();
+}
+// Scan CTAs (one warp, `smem` bytes) resident per SM: shared memory bounds it
+// (1 KB per CTA is reserved by the system), and 255-register warps at 8.
+int smem_resident(size_t smem) {
+    static int cap[kMaxDevices] = {0};
+    int dev = 0;
+    int bytes = 228 * 1024;
+    sm_count();  // sets no_device when CUDA is unavailable
+    if (!no_device && cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) {
+        if (cap[dev] == 0) {
+            int n = 0;
+            cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+            cap[dev] = n > 0 ? n : bytes;
+        }
+        bytes = cap[dev];
+    }
+    const int n = (int)(bytes / (smem + 1024));
+    return n < 1 ? 1 : (n > 8 ? 8 : n);
+}
+bool scan_pays(int64_t L, int64_t ctas, size_t scan_smem) {
+    const int64_t per_wave = (int64_t)sm_count() * smem_resident(scan_smem);
+    const int64_t items = ((L + sru::kScanT - 1) / sru::kScanT) * ctas;
+    const int64_t waves = (items + per_wave - 1) / per_wave;
+    return waves * kScanWaveChunks < (L + sru::kChunkT - 1) / sru::kChunkT;
+}
+size_t fwd_scan_smem(int u_t) {
+    return u_t == SRU_BF16 ? sru::FwdScanLayout<__nv_bfloat16>::SMEM : sru::FwdScanLayout<float>::SMEM;
+}
+size_t bwd_scan_smem(int u_t, bool acc_dx) {
+    if (u_t == SRU_BF16)
+        return acc_dx ? sru::BwdScanLayout<__nv_bfloat16, true>::SMEM : sru::BwdScanLayout<__nv_bfloat16, false>::SMEM;
+    return acc_dx ? sru::BwdScanLayout<float, true>::SMEM : sru::BwdScanLayout<float, false>::SMEM;
+}
+bool use_fwd_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir, int u_t) {
     if (!(flags & SRU_FLAG_V_ZERO)) return false;
     if (flags & SRU_FLAG_FORCE_SCAN) return true;
     if (flags & SRU_FLAG_FORCE_SEQUENTIAL) return false;
-    return seq_underfills(L, B, d, n_dir);
+    return scan_candidate(B, d, n_dir) && scan_pays(L, seq_ctas(B, d, n_dir), fwd_scan_smem(u_t));
 }
-bool use_bwd_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir) {
-    (void)n_dir;
+bool use_bwd_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir, int u_t) {
     if (flags & SRU_FLAG_FORCE_SCAN) return true;
     if (flags & SRU_FLAG_FORCE_SEQUENTIAL) return false;
-    return seq_underfills(L, B, d, 1);  // one direction per backward launch
+    // one direction per backward launch
+    return scan_candidate(B, d, 1) && scan_pays(L, seq_ctas(B, d, 1), bwd_scan_smem(u_t, n_dir == 2));
 }
-// Whether a workspace for these sizes and flags carries the scan regions.
+// Whether a workspace for these sizes and flags carries the scan regions: a
+// superset of the layers that take a scan (it depends on sizes and flags only,
+// not on the U dtype).
 bool ws_has_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir) {
-    return use_fwd_scan(flags, L, B, d, n_dir) || use_bwd_scan(flags, L, B, d, n_dir) ||
-           (flags & SRU_FLAG_V_ZERO) != 0;
+    (void)L;
+    (void)n_dir;
+    if (flags & (SRU_FLAG_FORCE_SCAN | SRU_FLAG_V_ZERO)) return true;
+    if (flags & SRU_FLAG_FORCE_SEQUENTIAL) return false;
+    return scan_candidate(B, d, 1);
 }
 
 sru_status check_layer_sizes(int64_t L, int64_t B, int64_t d) {
@@ -632,7 +682,7 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
     }
     if (!U || !x || !h || !aligned16(U) || !aligned16(x) || !aligned16(h)) return SRU_ERR_INVALID;
     const WsLayout w = ws_layout(L, B, d, n_dir, flags);
-    const bool scan = use_fwd_scan(flags, L, B, d, n_dir);
+    const bool scan = use_fwd_scan(flags, L, B, d, n_dir, u_t);
     if (workspace) {
         if (!aligned16(workspace) || workspace_bytes < w.total) return SRU_ERR_INVALID;
     } else if (scan) {
@@ -684,7 +734,7 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
         return SRU_ERR_INVALID;
     const WsLayout w = ws_layout(L, B, d, n_dir, flags);
     if (workspace_bytes < w.total) return SRU_ERR_INVALID;
-    const bool scan = use_bwd_scan(flags, L, B, d, n_dir);
+    const bool scan = use_bwd_scan(flags, L, B, d, n_dir, u_t);
     const int cj = kSeqCJ;
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj) ||
@@ -721,7 +771,8 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     if (s != SRU_OK) return s;
     const int64_t rows = scan ? scan_chunks(L) * B : B;
     const size_t nred = (size_t)n_dir * 4 * d;
-    sru::sru_reduce_dvdb_kernel<<<blocks_for(nred, 256), 256, 0, st>>>(partial, (int)rows, (int)d, n_dir, dv, db);
+    sru::sru_reduce_dvdb_kernel<<<blocks_for(nred, sru::kRedCols), sru::kRedCols * sru::kRedSlices, 0, st>>>(
+        partial, (int)rows, (int)d, n_dir, dv, db);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }

@@ -626,19 +626,33 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     }
 }
 
-// dv, db = sum over rows of the per-row partial sums, in increasing row order
-// (deterministic).  partial: (rows, n_dir, 4, d) doubles, [dv_f, dv_r, db_f, db_r].
-__global__ void sru_reduce_dvdb_kernel(const double* __restrict__ partial, int rows, int d, int n_dir,
-                                       float* __restrict__ dv, float* __restrict__ db) {
-    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= n_dir * 4 * d) return;
-    const int dir = idx / (4 * d), q = (idx / d) % 4, j = idx % d;
+// dv, db = sum over rows of the per-row partial sums.  partial: (rows,
+// n_dir, 4, d) doubles, [dv_f, dv_r, db_f, db_r].  A block owns
+// kRedCols consecutive output columns; its kRedSlices row slices each sum
+// rows slice, slice + kRedSlices, ... in increasing order, and the slices are
+// then added in increasing order: a fixed order, so the result is the same
+// on every run.
+constexpr int kRedCols = 32, kRedSlices = 8;
+__global__ void __launch_bounds__(kRedCols * kRedSlices) sru_reduce_dvdb_kernel(
+    const double* __restrict__ partial, int rows, int d, int n_dir, float* __restrict__ dv, float* __restrict__ db) {
+    __shared__ double part[kRedSlices][kRedCols];
+    const int col = threadIdx.x % kRedCols, slice = threadIdx.x / kRedCols;
+    const int idx = blockIdx.x * kRedCols + col;
+    const int ncols = n_dir * 4 * d;
     double s = 0.0;
-    for (int rr = 0; rr < rows; ++rr) s += partial[(((size_t)rr * n_dir + dir) * 4 + q) * d + j];
+    if (idx < ncols)
+        for (int rr = slice; rr < rows; rr += kRedSlices) s += partial[(size_t)rr * ncols + idx];
+    part[slice][col] = s;
+    __syncthreads();
+    if (slice != 0 || idx >= ncols) return;
+    double t = 0.0;
+#pragma unroll
+    for (int k = 0; k < kRedSlices; ++k) t += part[k][col];
+    const int dir = idx / (4 * d), q = (idx / d) % 4, j = idx % d;
     if (q < 2)
-        dv[(dir * 2 + q) * d + j] = (float)s;
+        dv[(dir * 2 + q) * d + j] = (float)t;
     else
-        db[(dir * 2 + q - 2) * d + j] = (float)s;
+        db[(dir * 2 + q - 2) * d + j] = (float)t;
 }
 
 // L == 0: the final state is the initial state.

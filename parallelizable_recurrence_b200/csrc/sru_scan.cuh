@@ -34,6 +34,14 @@ namespace sru {
 
 constexpr int kScanSub = 4;                 // 16-step sub-chunks per scan chunk
 constexpr int kScanT = kScanSub * kChunkT;  // steps per scan chunk
+static_assert(kScanT <= 64, "sub-chunk row bits are packed in one 64-bit word");
+
+// Row bits of sub-chunk q from a packed word (kChunkT bits per sub-chunk), so
+// that loops over sub-chunks need not be unrolled: four unrolled copies of the
+// chunk code overflow the instruction cache.
+__device__ __forceinline__ uint32_t sub_bits(uint64_t packed, int q) {
+    return (uint32_t)(packed >> (kChunkT * q)) & ((1u << kChunkT) - 1u);
+}
 
 enum ScanFlag : unsigned { kFlagNone = 0, kFlagAgg = 1, kFlagPrefix = 2, kFlagAbort = 3 };
 
@@ -187,6 +195,12 @@ __global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
             tma_load_3d(st + FwdLayout<UT>::U_BYTES, &map_x, bar, j0, b, t0 + q * kChunkT);
         }
     }
+    uint64_t valid_all = 0, inrange_all = 0;
+#pragma unroll
+    for (int q = 0; q < kScanSub; ++q) {
+        valid_all |= (uint64_t)valid[q] << (kChunkT * q);
+        inrange_all |= (uint64_t)inrange[q] << (kChunkT * q);
+    }
     if (any) {
         const bool ok = mbar_wait(bar, 0, kErrTimeoutLoad);
         if (__syncthreads_or(!ok)) {
@@ -198,14 +212,14 @@ __global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
 
     // 1. the chunk as an affine map of the entering state: c_out = A c_in + Bc
     float2 A = f2(1.f), Bc = f2(0.f);
-#pragma unroll
+#pragma unroll 1
     for (int qq = 0; qq < kScanSub; ++qq) {
         const int q = dir == 0 ? qq : kScanSub - 1 - qq;
         const UT* us = reinterpret_cast<const UT*>(smem + q * Lay::STAGE);
 #pragma unroll
         for (int r = 0; r < kChunkT; ++r) {
             const int i = dir == 0 ? r : kChunkT - 1 - r;
-            if ((valid[q] >> i) & 1u) {
+            if ((sub_bits(valid_all, q) >> i) & 1u) {
                 const float2 uc = load_pair(us + (i * 3 + 0) * kRecCJ + cj);
                 const float2 f =
                     sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 1) * kRecCJ + cj), f2(kNegLog2e), p.nbf));
@@ -236,7 +250,7 @@ __global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
     float2 c = c_in;
     const float2 alpha2 = f2(alpha);
     const size_t h_tstride = (size_t)B * n_dir * d;
-#pragma unroll
+#pragma unroll 1
     for (int qq = 0; qq < kScanSub; ++qq) {
         const int q = dir == 0 ? qq : kScanSub - 1 - qq;
         const int ts = t0 + q * kChunkT;
@@ -246,7 +260,7 @@ __global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
         const UT* us = reinterpret_cast<const UT*>(smem + q * Lay::STAGE);
         const float* xs = reinterpret_cast<const float*>(smem + q * Lay::STAGE + FwdLayout<UT>::U_BYTES);
         float* hp = h + (size_t)ts * h_tstride + (size_t)bd * d + j;
-        c = fwd_chunk<UT, kRecCJ>(us, xs, valid[q], inrange[q], c, p, alpha2, dir, hp, h_tstride, jok, cj);
+        c = fwd_chunk<UT, kRecCJ>(us, xs, sub_bits(valid_all, q), sub_bits(inrange_all, q), c, p, alpha2, dir, hp, h_tstride, jok, cj);
     }
     if (k == nchs - 1 && jok) store_pair(c_T + (size_t)bd * d + j, c);
 }
@@ -254,7 +268,9 @@ __global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
 template <typename UT, bool ACC_DX>
 struct BwdScanLayout {
     static constexpr int STAGE = BwdLayout<UT, ACC_DX>::STAGE;
-    static constexpr int BAR_OFF = kScanSub * STAGE;
+    static constexpr int CK_OFF = kScanSub * STAGE;             // checkpoints: [kScanSub][CJ] fp32
+    static constexpr int ACC_OFF = CK_OFF + kScanSub * kRecCJ * 4;  // SmemPartials: 8 doubles per thread
+    static constexpr int BAR_OFF = ACC_OFF + kRecThreads * 8 * 8;
     static constexpr int SMEM = BAR_OFF + 64 + 128;
 };
 
@@ -326,6 +342,19 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
             if (ACC_DX) tma_load_3d(st + SL::U_BYTES + 2 * SL::V_BYTES, &map_dxin, bar, j0, b, ts);
         }
     }
+    uint64_t valid_all = 0, inrange_all = 0;
+#pragma unroll
+    for (int q = 0; q < kScanSub; ++q) {
+        valid_all |= (uint64_t)valid[q] << (kChunkT * q);
+        inrange_all |= (uint64_t)inrange[q] << (kChunkT * q);
+    }
+    // the sub-chunks' forward checkpoints, fetched while the tiles load
+    float2* s_ck = reinterpret_cast<float2*>(smem + Lay::CK_OFF) + lane;  // sub-chunk q at s_ck[q * 32]
+#pragma unroll
+    for (int q = 0; q < kScanSub; ++q) {
+        const int c16 = tc * kScanSub + q;
+        s_ck[q * 32] = (jok && c16 < nch16) ? load_pair(ckpt + ((size_t)c16 * B * n_dir + bd) * d + j) : f2(0.f);
+    }
     if (any) {
         const bool ok = mbar_wait(bar, 0, kErrTimeoutLoad);
         if (__syncthreads_or(!ok)) {
@@ -343,7 +372,7 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
     float2 A = f2(1.f), Bg = f2(0.f);
     if (VZERO) {
         // v = 0: the gates do not read c, so a = f and b = f dh r need no state
-#pragma unroll
+#pragma unroll 1
         for (int qq = 0; qq < kScanSub; ++qq) {
             const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
             const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
@@ -351,7 +380,7 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
 #pragma unroll
             for (int r = 0; r < kChunkT; ++r) {
                 const int i = DIR == 0 ? kChunkT - 1 - r : r;
-                if ((valid[q] >> i) & 1u) {
+                if ((sub_bits(valid_all, q) >> i) & 1u) {
                     const float2 f =
                         sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 1) * kRecCJ + cj), f2(kNegLog2e), p.nbf));
                     const float2 rr =
@@ -362,15 +391,14 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
             }
         }
     } else {
-    #pragma unroll
+    #pragma unroll 1
         for (int qq = 0; qq < kScanSub; ++qq) {
             const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
-            if (valid[q] == 0u) continue;
+            if (sub_bits(valid_all, q) == 0u) continue;
             const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
             const float* xs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES);
             const float* dhs = xs + kChunkT * kRecCJ;
-            const int c16 = tc * kScanSub + q;
-            float2 c = (jok && c16 < nch16) ? load_pair(ckpt + ((size_t)c16 * B * n_dir + bd) * d + j) : f2(0.f);
+            float2 c = s_ck[q * 32];
             float2 cp[kChunkT], fs[kChunkT], rs[kChunkT];
     #pragma unroll
             for (int r = 0; r < kChunkT; ++r) {
@@ -378,14 +406,14 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
                 cp[i] = c;
                 fs[i] = f2(0.f);
                 rs[i] = f2(0.f);
-                if ((valid[q] >> i) & 1u)
+                if ((sub_bits(valid_all, q) >> i) & 1u)
                     c = sru_cell2(c, load_pair(us + (i * 3 + 0) * kRecCJ + cj), load_pair(us + (i * 3 + 1) * kRecCJ + cj),
                                   load_pair(us + (i * 3 + 2) * kRecCJ + cj), p, fs[i], rs[i]);
             }
     #pragma unroll
             for (int r = 0; r < kChunkT; ++r) {
                 const int i = DIR == 0 ? kChunkT - 1 - r : r;
-                if (!((valid[q] >> i) & 1u)) continue;
+                if (!((sub_bits(valid_all, q) >> i) & 1u)) continue;
                 const float2 f = fs[i], rr = rs[i];
                 const float2 uc = load_pair(us + (i * 3 + 0) * kRecCJ + cj);
                 const float2 ax = mul2(alpha2, load_pair(xs + i * kRecCJ + cj));
@@ -420,28 +448,29 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
 
     // 3. gradients of every row, sub-chunk by sub-chunk in backward order
     float2 g = g_in;
-    double acc[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
+    SmemPartials acc{reinterpret_cast<double*>(smem + Lay::ACC_OFF) + lane, kRecThreads};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc.p[q * acc.n] = 0.0;  // read and written by this thread only
     const size_t u_tstride = (size_t)B * n_dir * 3 * d;
     const size_t x_tstride = (size_t)B * d;
-#pragma unroll
+#pragma unroll 1
     for (int qq = 0; qq < kScanSub; ++qq) {
         const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
         const int ts = t0 + q * kChunkT;
         if (ts >= L) continue;
         DUT* dUp = dU + (size_t)ts * u_tstride + (size_t)bd * 3 * d + j;
         float* dxp = dx + (size_t)ts * x_tstride + (size_t)b * d + j;
-        if (valid[q] == 0u) {
-            bwd_chunk_padded<DUT, ACC_DX>(inrange[q], dUp, dxp, u_tstride, x_tstride, d, jok);
+        if (sub_bits(valid_all, q) == 0u) {
+            bwd_chunk_padded<DUT, ACC_DX>(sub_bits(inrange_all, q), dUp, dxp, u_tstride, x_tstride, d, jok);
             continue;
         }
         const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
         const float* xs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES);
         const float* dhs = xs + kChunkT * kRecCJ;
         const float* dxin = dhs + kChunkT * kRecCJ;
-        const int c16 = tc * kScanSub + q;
-        const float2 c_start = jok ? load_pair(ckpt + ((size_t)c16 * B * n_dir + bd) * d + j) : f2(0.f);
-        bwd_chunk<UT, DUT, ACC_DX, DIR, kRecCJ>(us, xs, dhs, dxin, valid[q], inrange[q], c_start, p, alpha2, g, acc, dUp,
-                                        dxp, u_tstride, x_tstride, d, jok, cj);
+        bwd_chunk<UT, DUT, ACC_DX, DIR, kRecCJ>(us, xs, dhs, dxin, sub_bits(valid_all, q), sub_bits(inrange_all, q),
+                                                s_ck[q * 32], p, alpha2, g, acc, dUp, dxp, u_tstride, x_tstride, d,
+                                                jok, cj);
     }
     if (jok) {
         if (k == nchs - 1) store_pair(dc0 + (size_t)bd * d + j, g);
