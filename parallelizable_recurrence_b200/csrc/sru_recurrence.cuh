@@ -101,6 +101,10 @@ __device__ __forceinline__ void store_pair(float* p, float2 v) { *reinterpret_ca
 __device__ __forceinline__ void store_pair(__nv_bfloat16* p, float2 v) {
     *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v.x, v.y);
 }
+// p[0..1] += v with one 8-byte atomic (sm_90+ vector atomicAdd): used where
+// exactly one addend arrives per element, so the result does not depend on
+// timing.
+__device__ __forceinline__ void add_pair(float* p, float2 v) { atomicAdd(reinterpret_cast<float2*>(p), v); }
 
 // A channel pair of U as held in registers before use: the raw bf16x2 word
 // (one 32-bit register) or the fp32 pair.
@@ -324,16 +328,18 @@ __device__ __forceinline__ void fold_partials(SmemPartials& acc, const float2 (&
 }
 
 // ---------------------------------------------------------------- backward
-// Backward over one chunk staged in shared memory (us, xs, dhs and, with
-// ACC_DX, the dx the other direction already wrote in dxin), given the state c
-// entering the chunk in forward order and the state gradient g leaving it.
+// Backward over one chunk staged in shared memory (us, xs, dhs), given the
+// state c entering the chunk in forward order and the state gradient g leaving
+// it.  With ACC_DX the highway gradient is added onto the dx the other
+// direction already wrote (one atomic add per element, after that launch
+// completed on the same stream: the same single fp32 addition every run).
 // Re-runs the forward over the chunk keeping c, f and r in registers, then
 // walks it in reverse: writes dU and dx for the rows that exist, accumulates
 // the dv/db partial sums in acc[q] = {dv_f, dv_r, db_f, db_r} (per channel of
 // the pair), and updates g.
 template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ = kRecCJ, typename ACC>
 __device__ __forceinline__ void bwd_chunk_any(const UT* __restrict__ us, const float* __restrict__ xs,
-                                          const float* __restrict__ dhs, const float* __restrict__ dxin,
+                                          const float* __restrict__ dhs,
                                           uint32_t valid, uint32_t inrange, float2 c, const GateParams2& p,
                                           float2 alpha, float2& g, ACC& acc, DUT* __restrict__ dUp,
                                           float* __restrict__ dxp, size_t u_tstride, size_t x_tstride, int d,
@@ -383,7 +389,7 @@ __device__ __forceinline__ void bwd_chunk_any(const UT* __restrict__ us, const f
             store_pair(dUp + (size_t)i * u_tstride + d, dzf);
             store_pair(dUp + (size_t)i * u_tstride + 2 * d, dzr);
             if (ACC_DX) {
-                if (row) store_pair(dxp + (size_t)i * x_tstride, add2(load_pair(dxin + i * CJ + cj), dxv));
+                if (row) add_pair(dxp + (size_t)i * x_tstride, dxv);
             } else {
                 store_pair(dxp + (size_t)i * x_tstride, dxv);
             }
@@ -398,7 +404,7 @@ __device__ __forceinline__ void bwd_chunk_any(const UT* __restrict__ us, const f
 // before the chain runs, and no row carries a predicate.
 template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ, typename ACC>
 __device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const float* __restrict__ xs,
-                                               const float* __restrict__ dhs, const float* __restrict__ dxin,
+                                               const float* __restrict__ dhs,
                                                float2 c, const GateParams2& p, float2 alpha, float2& g,
                                                ACC& acc, DUT* __restrict__ dUp, float* __restrict__ dxp,
                                                size_t u_tstride, size_t x_tstride, int d, bool jok, int cj) {
@@ -446,7 +452,7 @@ __device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const 
             store_pair(dUp + (size_t)i * u_tstride + d, dzf);
             store_pair(dUp + (size_t)i * u_tstride + 2 * d, dzr);
             if (ACC_DX)
-                store_pair(dxp + (size_t)i * x_tstride, add2(load_pair(dxin + i * CJ + cj), dxv));
+                add_pair(dxp + (size_t)i * x_tstride, dxv);
             else
                 store_pair(dxp + (size_t)i * x_tstride, dxv);
         }
@@ -457,16 +463,16 @@ __device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const 
 
 template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ = kRecCJ, typename ACC>
 __device__ __forceinline__ void bwd_chunk(const UT* __restrict__ us, const float* __restrict__ xs,
-                                          const float* __restrict__ dhs, const float* __restrict__ dxin,
+                                          const float* __restrict__ dhs,
                                           uint32_t valid, uint32_t inrange, float2 c, const GateParams2& p,
                                           float2 alpha, float2& g, ACC& acc, DUT* __restrict__ dUp,
                                           float* __restrict__ dxp, size_t u_tstride, size_t x_tstride, int d,
                                           bool jok, int cj) {
     if (valid == (1u << kChunkT) - 1u)
-        bwd_chunk_full<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, dxin, c, p, alpha, g, acc, dUp, dxp, u_tstride,
+        bwd_chunk_full<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, c, p, alpha, g, acc, dUp, dxp, u_tstride,
                                                  x_tstride, d, jok, cj);
     else
-        bwd_chunk_any<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, dxin, valid, inrange, c, p, alpha, g, acc, dUp, dxp,
+        bwd_chunk_any<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, valid, inrange, c, p, alpha, g, acc, dUp, dxp,
                                                 u_tstride, x_tstride, d, jok, cj);
 }
 
@@ -500,7 +506,7 @@ template <typename UT, bool ACC_DX, int CJ = kRecCJ, int S = kBwdStages>
 struct BwdLayout {
     static constexpr int U_BYTES = kChunkT * 3 * CJ * (int)sizeof(UT);
     static constexpr int V_BYTES = kChunkT * CJ * 4;  // one fp32 (T, CJ) tile
-    static constexpr int STAGE = U_BYTES + V_BYTES * (ACC_DX ? 3 : 2);
+    static constexpr int STAGE = U_BYTES + 2 * V_BYTES;  // U, x, dh
     static constexpr int ACC_OFF = S * STAGE;  // SmemPartials: 8 doubles per thread
     static constexpr int BAR_OFF = ACC_OFF + (CJ / 2) * 8 * 8;
     static constexpr int SMEM = BAR_OFF + 64 + 128;
@@ -509,15 +515,16 @@ struct BwdLayout {
 // Backward of direction DIR.  Grid (ceil(d/CJ), B), CJ/2 threads (CJ/64 warps) per CTA.
 // ACC_DX: dx += this direction's highway gradient (dx already holds the other
 // direction's, written by an earlier launch on the same stream), else dx = it.
-//   map_dh: 3-D (d, B*n_dir, L) fp32; map_dxin: like map_x but over dx.
+// Adding with 8-byte atomics instead of staging dx keeps a stage at U + x + dh,
+// so as many CTAs fit on an SM as in the first direction's launch.
+//   map_dh: 3-D (d, B*n_dir, L) fp32.
 // DIR is a template parameter so the per-chunk register arrays are indexed
 // with compile-time constants.
 template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ, int S>
 __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
-    const __grid_constant__ CUtensorMap map_dh, const __grid_constant__ CUtensorMap map_dxin,
-    const float* __restrict__ v, const float* __restrict__ bias, const uint8_t* __restrict__ mask,
-    const float* __restrict__ ckpt, const float* __restrict__ dc_T, DUT* __restrict__ dU,
+    const __grid_constant__ CUtensorMap map_dh, const float* __restrict__ v, const float* __restrict__ bias,
+    const uint8_t* __restrict__ mask, const float* __restrict__ ckpt, const float* __restrict__ dc_T, DUT* __restrict__ dU,
     float* __restrict__ dx, double* __restrict__ partial, float* __restrict__ dc0, int L, int B, int d,
     int n_dir, float alpha) {
     using Lay = BwdLayout<UT, ACC_DX, CJ, S>;
@@ -547,7 +554,6 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
         tma_prefetch_desc(&map_u);
         tma_prefetch_desc(&map_x);
         tma_prefetch_desc(&map_dh);
-        if (ACC_DX) tma_prefetch_desc(&map_dxin);
     }
     __syncthreads();
 
@@ -565,7 +571,6 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
             tma_load_4d(st, &map_u, &full[s], j0, 0, bd, t0);
             tma_load_3d(st + Lay::U_BYTES, &map_x, &full[s], j0, b, t0);
             tma_load_3d(st + Lay::U_BYTES + Lay::V_BYTES, &map_dh, &full[s], j0, bd, t0);
-            if (ACC_DX) tma_load_3d(st + Lay::U_BYTES + 2 * Lay::V_BYTES, &map_dxin, &full[s], j0, b, t0);
         }
     };
     if (tid < 32)
@@ -611,8 +616,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
             const UT* us = reinterpret_cast<const UT*>(smem + s * Lay::STAGE);
             const float* xs = reinterpret_cast<const float*>(smem + s * Lay::STAGE + Lay::U_BYTES);
             const float* dhs = xs + kChunkT * CJ;
-            const float* dxin = dhs + kChunkT * CJ;
-            bwd_chunk<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, dxin, valid, inrange, ck0, p, alpha2, g, acc, dUp, dxp,
+            bwd_chunk<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, valid, inrange, ck0, p, alpha2, g, acc, dUp, dxp,
                                                 u_tstride, x_tstride, d, jok, cj);
         }
         __syncthreads();

@@ -279,7 +279,7 @@ struct BwdScanLayout {
 template <typename UT, typename DUT, bool ACC_DX, int DIR, bool VZERO>
 __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
-    const __grid_constant__ CUtensorMap map_dh, const __grid_constant__ CUtensorMap map_dxin,
+    const __grid_constant__ CUtensorMap map_dh,
     const float* __restrict__ v, const float* __restrict__ bias, const uint8_t* __restrict__ mask,
     const float* __restrict__ ckpt, const float* __restrict__ dc_T, DUT* __restrict__ dU, float* __restrict__ dx,
     double* __restrict__ partial, float* __restrict__ dc0, ScanState ss, int L, int B, int d, int n_dir,
@@ -339,7 +339,6 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
             tma_load_4d(st, &map_u, bar, j0, 0, bd, ts);
             tma_load_3d(st + SL::U_BYTES, &map_x, bar, j0, b, ts);
             tma_load_3d(st + SL::U_BYTES + SL::V_BYTES, &map_dh, bar, j0, bd, ts);
-            if (ACC_DX) tma_load_3d(st + SL::U_BYTES + 2 * SL::V_BYTES, &map_dxin, bar, j0, b, ts);
         }
     }
     uint64_t valid_all = 0, inrange_all = 0;
@@ -467,8 +466,7 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
         const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
         const float* xs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES);
         const float* dhs = xs + kChunkT * kRecCJ;
-        const float* dxin = dhs + kChunkT * kRecCJ;
-        bwd_chunk<UT, DUT, ACC_DX, DIR, kRecCJ>(us, xs, dhs, dxin, sub_bits(valid_all, q), sub_bits(inrange_all, q),
+        bwd_chunk<UT, DUT, ACC_DX, DIR, kRecCJ>(us, xs, dhs, sub_bits(valid_all, q), sub_bits(inrange_all, q),
                                                 s_ck[q * 32], p, alpha2, g, acc, dUp, dxp, u_tstride, x_tstride, d,
                                                 jok, cj);
     }
