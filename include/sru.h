@@ -192,6 +192,30 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
                                     const float* c0, const uint8_t* mask, int64_t L, int64_t B, int64_t d,
                                     float alpha, int bidirectional, float* h, float* c_T, void* stream);
 
+/*
+ * One time step of a unidirectional layer for inference (token-by-token
+ * decoding), with the projection fused in.  The page notes that SRU-based
+ * models run as an RNN at inference time (one token per step); there the
+ * product of Eq. (1) degenerates to a matrix-vector product per step, and
+ * this call does that product and Eqs. (2)-(5) in one kernel:
+ *   u[b, g, j] = sum_k X_t[b, k] * W_cat[g*d + j, k]     (fp32, never stored)
+ *   c[b, j], h_t[b, j] <- Eqs. (2)-(5) from c[b, j], u, x_t[b, j], v, b, alpha
+ * for b < B, j < d.  u is kept in fp32 (sru_project + sru_forward round U to
+ * the U dtype in between; here no U exists).
+ *   X_t  (B, d) bf16     projection input of this step
+ *   W    (3*d, d) bf16   W_cat of one direction (gate blocks as above)
+ *   x_t  (B, d) fp32     highway input of this step
+ *   v, b (2, d) fp32     forget / reset peepholes and biases
+ *   c    (B, d) fp32     state: read as c[t-1], overwritten with c[t]
+ *   h_t  (B, d) fp32     output
+ * Each W element is read once per call (the step streams 6*d*d bytes of W for
+ * any B <= 16; larger B is processed 16 rows at a time).  Same pointer rules as
+ * above; X_t, W, x_t, c and h_t must not overlap.  B = 0 is a no-op.
+ * Limits: d % 8 == 0, d <= 2^24, B <= 2^20, else SRU_ERR_UNSUPPORTED.
+ */
+sru_status sru_decode_step(const void* X_t, const void* W, const float* x_t, const float* v, const float* b,
+                           float* c, float* h_t, int64_t B, int64_t d, float alpha, void* stream);
+
 /* Synchronise `stream`, then read and clear the device error word of the
  * current device: SRU_ERR_TIMEOUT if a bounded wait expired since the last
  * call, SRU_ERR_CUDA if the stream reported an error, else SRU_OK. */

@@ -32,7 +32,7 @@ SRU_FLAG_TEST_WITHHOLD_CARRY = 0x8
 # every symbol include/sru.h declares
 EXPORTED = ("sru_status_string", "sru_get_last_cuda_error", "sru_version", "sru_workspace_bytes",
             "sru_project", "sru_project_backward", "sru_forward", "sru_backward", "sru_forward_scan_noalloc",
-            "sru_sync_status")
+            "sru_decode_step", "sru_sync_status")
 
 
 class SRUError(RuntimeError):
@@ -80,6 +80,8 @@ def load_library(path: str = LIB_PATH):
     lib.sru_forward_scan_noalloc.restype = _int
     lib.sru_forward_scan_noalloc.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _f32, _int,
                                              _vp, _vp, _vp]
+    lib.sru_decode_step.restype = _int
+    lib.sru_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _vp]
     lib.sru_sync_status.restype = _int
     lib.sru_sync_status.argtypes = [_vp]
     _lib = lib
@@ -203,6 +205,22 @@ def sru_forward_scan_noalloc(U, x, b, h, c_T, c0=None, mask=None, alpha: float =
                                         _ptr(c_T, torch.float32), _stream(stream)),
            "sru_forward_scan_noalloc")
     return h, c_T
+
+
+def sru_decode_step(X_t, W, x_t, v, b, c, h_t, alpha: float = 1.0, stream=None):
+    """One inference step of a unidirectional layer with the projection fused:
+    u = X_t W^T (fp32, never stored), then Eqs. (2)-(5).  X_t (B, d) bf16,
+    W (3d, d) bf16, x_t (B, d) fp32, v and b (2, d) fp32 (a (1, 2, d) slice is
+    fine), c (B, d) fp32 state updated in place, h_t (B, d) fp32 output."""
+    lib = load_library()
+    B, d = X_t.shape
+    if W.shape[0] != 3 * d or W.shape[1] != d:
+        raise ValueError("W must be (3*d, d)")
+    _check(lib.sru_decode_step(_ptr(X_t, torch.bfloat16), _ptr(W, torch.bfloat16), _ptr(x_t, torch.float32),
+                               _ptr(v, torch.float32), _ptr(b, torch.float32), _ptr(c, torch.float32),
+                               _ptr(h_t, torch.float32), B, d, float(alpha), _stream(stream)),
+           "sru_decode_step")
+    return h_t, c
 
 
 def sru_sync_status(stream=None) -> int:

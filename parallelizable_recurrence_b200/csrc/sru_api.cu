@@ -12,6 +12,7 @@
 #include "../../include/sru.h"
 #include "sru_gemm.cuh"
 #include "sru_recurrence.cuh"
+#include "sru_decode.cuh"
 #include "sru_scan.cuh"
 
 namespace {
@@ -524,6 +525,25 @@ sru_status launch_bwd_scan(const RecMaps& mp, const float* v, const float* b, co
                                               alpha, st);
 }
 
+// ------------------------------------------------------------ decode step
+template <int NB>
+sru_status launch_decode_nb(const void* X_t, const void* W, const float* x_t, const float* v, const float* b,
+                            float* c, float* h_t, int64_t B, int64_t d, float alpha, cudaStream_t st) {
+    const dim3 grid((unsigned)((d + sru::kDecWarps - 1) / sru::kDecWarps), (unsigned)((B + NB - 1) / NB));
+    sru::sru_decode_step_kernel<NB><<<grid, sru::kDecThreads, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(X_t), reinterpret_cast<const __nv_bfloat16*>(W), x_t, v, b, c, h_t,
+        (int)B, (int)d, alpha);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+// Batch rows per pass over W: the smallest instantiated count covering B (at most 16).
+int decode_rows_per_pass(int64_t B) {
+    int nb = 1;
+    while (nb < B && nb < sru::kDecMaxNB) nb *= 2;
+    return nb;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -813,6 +833,27 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
     if (u_t == SRU_BF16)
         return launch_fwd_scan<__nv_bfloat16>(mp, b, c0, mask, h, c_T, nullptr, ss, L, B, d, n_dir, alpha, st);
     return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, nullptr, ss, L, B, d, n_dir, alpha, st);
+}
+
+sru_status sru_decode_step(const void* X_t, const void* W, const float* x_t, const float* v, const float* b,
+                           float* c, float* h_t, int64_t B, int64_t d, float alpha, void* stream) {
+    if (B < 0 || d < 1) return SRU_ERR_INVALID;
+    if (d % 8 != 0) return SRU_ERR_UNSUPPORTED;
+    if (B == 0) return SRU_OK;
+    if (!X_t || !W || !x_t || !v || !b || !c || !h_t) return SRU_ERR_INVALID;
+    if (!aligned16(X_t) || !aligned16(W) || !aligned16(x_t) || !aligned16(c) || !aligned16(h_t))
+        return SRU_ERR_INVALID;
+    if (d > ((int64_t)1 << 24) || B > ((int64_t)1 << 20)) return SRU_ERR_UNSUPPORTED;
+    const int nb = decode_rows_per_pass(B);
+    if ((B + nb - 1) / nb > 65535) return SRU_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    switch (nb) {
+        case 1: return launch_decode_nb<1>(X_t, W, x_t, v, b, c, h_t, B, d, alpha, st);
+        case 2: return launch_decode_nb<2>(X_t, W, x_t, v, b, c, h_t, B, d, alpha, st);
+        case 4: return launch_decode_nb<4>(X_t, W, x_t, v, b, c, h_t, B, d, alpha, st);
+        case 8: return launch_decode_nb<8>(X_t, W, x_t, v, b, c, h_t, B, d, alpha, st);
+        default: return launch_decode_nb<16>(X_t, W, x_t, v, b, c, h_t, B, d, alpha, st);
+    }
 }
 
 sru_status sru_sync_status(void* stream) {

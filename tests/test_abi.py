@@ -102,3 +102,15 @@ def test_invalid_arguments_return_before_any_launch(lib):
     assert small >= 4096 // 64 * 2 * (4 + 3 * 64 * 4)
     st = lib.sru_forward(fake, 1, fake, fake, fake, None, None, 4096, 2, 64, 1.0, 0, 1 | 2, fake, fake, None, 0, None)
     assert st == 1
+
+
+def test_decode_step_checks_arguments_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)
+    args = [fake] * 7
+    assert lib.sru_decode_step(*args, 0, 64, 1.0, None) == 0          # B = 0: nothing to do
+    assert lib.sru_decode_step(*args, 2, 12, 1.0, None) == 4          # d % 8 != 0
+    assert lib.sru_decode_step(*args, -1, 64, 1.0, None) == 1         # negative B
+    assert lib.sru_decode_step(None, *args[1:], 2, 64, 1.0, None) == 1  # null X_t
+    assert lib.sru_decode_step(vp(0x1008), *args[1:], 2, 64, 1.0, None) == 1  # misaligned X_t
+    assert lib.sru_decode_step(*args, 1, 1 << 25, 1.0, None) == 4     # d beyond the size limit
