@@ -193,6 +193,30 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
                                     float alpha, int bidirectional, float* h, float* c_T, void* stream);
 
 /*
+ * Factorised projection: the page's variant of Eq. (1) with a low-rank
+ * projection (Figure 2, the SRU layer "with projection trick"):
+ *   P = X Wq^T        (M, Kp)  Wq (Kp, K): projects d down to d' = Kp
+ *   U = P Wo^T        (M, N)   Wo (N, Kp): back up to the n_dir * 3d gate columns
+ * X, Wq, Wo bf16; P is a caller-provided bf16 buffer that receives the
+ * intermediate (kept for the backward); U of type u_t (BF16 or F32).  Two
+ * chained tensor-core products with fp32 accumulation; P is rounded to bf16
+ * in between.  K, Kp and N must be multiples of 8 (SRU_ERR_UNSUPPORTED).
+ */
+sru_status sru_project_factored(const void* X, const void* Wq, const void* Wo, void* P, void* U, int u_t,
+                                int64_t M, int64_t N, int64_t K, int64_t Kp, void* stream);
+
+/*
+ * Gradients of sru_project_factored for a bf16 dU (M, N):
+ *   dWo = dU^T P (N, Kp) fp32;   dP = dU Wo (M, Kp) written to the caller's bf16 buffer dP;
+ *   dWq = dP^T X (Kp, K) fp32;   dX = dP Wq (M, K) fp32, added onto dX when accumulate != 0.
+ * P is the intermediate the forward wrote.  Any of dX, dWq, dWo may be NULL
+ * (not computed); dP is always written.
+ */
+sru_status sru_project_factored_backward(const void* dU, const void* X, const void* Wq, const void* Wo,
+                                         const void* P, void* dP, float* dX, int accumulate, float* dWq,
+                                         float* dWo, int64_t M, int64_t N, int64_t K, int64_t Kp, void* stream);
+
+/*
  * One time step of a unidirectional layer for inference (token-by-token
  * decoding), with the projection fused in.  The page notes that SRU-based
  * models run as an RNN at inference time (one token per step); there the

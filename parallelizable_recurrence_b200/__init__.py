@@ -32,7 +32,7 @@ SRU_FLAG_TEST_WITHHOLD_CARRY = 0x8
 # every symbol include/sru.h declares
 EXPORTED = ("sru_status_string", "sru_get_last_cuda_error", "sru_version", "sru_workspace_bytes",
             "sru_project", "sru_project_backward", "sru_forward", "sru_backward", "sru_forward_scan_noalloc",
-            "sru_decode_step", "sru_sync_status")
+            "sru_project_factored", "sru_project_factored_backward", "sru_decode_step", "sru_sync_status")
 
 
 class SRUError(RuntimeError):
@@ -80,6 +80,11 @@ def load_library(path: str = LIB_PATH):
     lib.sru_forward_scan_noalloc.restype = _int
     lib.sru_forward_scan_noalloc.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _f32, _int,
                                              _vp, _vp, _vp]
+    lib.sru_project_factored.restype = _int
+    lib.sru_project_factored.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp]
+    lib.sru_project_factored_backward.restype = _int
+    lib.sru_project_factored_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _i64, _i64,
+                                                  _i64, _i64, _vp]
     lib.sru_decode_step.restype = _int
     lib.sru_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _vp]
     lib.sru_sync_status.restype = _int
@@ -205,6 +210,34 @@ def sru_forward_scan_noalloc(U, x, b, h, c_T, c0=None, mask=None, alpha: float =
                                         _ptr(c_T, torch.float32), _stream(stream)),
            "sru_forward_scan_noalloc")
     return h, c_T
+
+
+def sru_project_factored(X, Wq, Wo, P, U, stream=None):
+    """P = X Wq^T (bf16, written to P), U = P Wo^T.  X (M, K), Wq (Kp, K), Wo (N, Kp) bf16."""
+    lib = load_library()
+    M, K = X.shape
+    Kp, N = Wq.shape[0], Wo.shape[0]
+    if Wq.shape[1] != K or Wo.shape[1] != Kp or tuple(P.shape) != (M, Kp) or U.numel() != M * N:
+        raise ValueError("shape mismatch")
+    _check(lib.sru_project_factored(_ptr(X, torch.bfloat16), _ptr(Wq, torch.bfloat16), _ptr(Wo, torch.bfloat16),
+                                    _ptr(P, torch.bfloat16), _ptr(U), _dtype_code(U), M, N, K, Kp,
+                                    _stream(stream)), "sru_project_factored")
+    return U
+
+
+def sru_project_factored_backward(dU, X, Wq, Wo, P, dP, dX=None, accumulate: bool = False, dWq=None, dWo=None,
+                                  stream=None):
+    """dWo = dU^T P, dP = dU Wo (bf16, into dP), dWq = dP^T X, dX (+)= dP Wq (fp32 outputs)."""
+    lib = load_library()
+    M, K = X.shape
+    Kp, N = Wq.shape[0], Wo.shape[0]
+    _check(lib.sru_project_factored_backward(_ptr(dU, torch.bfloat16), _ptr(X, torch.bfloat16),
+                                             _ptr(Wq, torch.bfloat16), _ptr(Wo, torch.bfloat16),
+                                             _ptr(P, torch.bfloat16), _ptr(dP, torch.bfloat16),
+                                             _ptr(dX, torch.float32), int(bool(accumulate)),
+                                             _ptr(dWq, torch.float32), _ptr(dWo, torch.float32), M, N, K, Kp,
+                                             _stream(stream)), "sru_project_factored_backward")
+    return dX, dWq, dWo
 
 
 def sru_decode_step(X_t, W, x_t, v, b, c, h_t, alpha: float = 1.0, stream=None):

@@ -835,6 +835,52 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
     return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, nullptr, ss, L, B, d, n_dir, alpha, st);
 }
 
+sru_status sru_project_factored(const void* X, const void* Wq, const void* Wo, void* P, void* U, int u_t,
+                                int64_t M, int64_t N, int64_t K, int64_t Kp, void* stream) {
+    if (M < 0 || N < 0 || K < 1 || Kp < 1) return SRU_ERR_INVALID;
+    if (!X || !Wq || !Wo || !P || !U) return SRU_ERR_INVALID;
+    if (u_t != SRU_BF16 && u_t != SRU_F32) return SRU_ERR_INVALID;
+    if (K % 8 != 0 || Kp % 8 != 0 || N % 8 != 0) return SRU_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0) return SRU_OK;
+    sru_status s = sru_project(X, SRU_BF16, Wq, SRU_BF16, P, SRU_BF16, M, Kp, K, stream);
+    if (s != SRU_OK) return s;
+    return sru_project(P, SRU_BF16, Wo, SRU_BF16, U, u_t, M, N, Kp, stream);
+}
+
+sru_status sru_project_factored_backward(const void* dU, const void* X, const void* Wq, const void* Wo,
+                                         const void* P, void* dP, float* dX, int accumulate, float* dWq,
+                                         float* dWo, int64_t M, int64_t N, int64_t K, int64_t Kp, void* stream) {
+    if (M < 0 || N < 1 || K < 1 || Kp < 1) return SRU_ERR_INVALID;
+    if (!dU || !Wo || !dP || !aligned16(dU) || !aligned16(Wo) || !aligned16(dP)) return SRU_ERR_INVALID;
+    if (dWo && (!P || !aligned16(P) || !aligned16(dWo))) return SRU_ERR_INVALID;
+    if (dWq && (!X || !aligned16(X) || !aligned16(dWq))) return SRU_ERR_INVALID;
+    if (dX && (!Wq || !aligned16(Wq) || !aligned16(dX))) return SRU_ERR_INVALID;
+    if (K % 8 != 0 || Kp % 8 != 0 || N % 8 != 0) return SRU_ERR_UNSUPPORTED;
+    if (M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31) || Kp >= ((int64_t)1 << 31))
+        return SRU_ERR_UNSUPPORTED;
+    cudaStream_t st = as_stream(stream);
+    if (M == 0) {
+        if (dWo) { sru_status s = zero_f32(dWo, (size_t)N * Kp, st); if (s) return s; }
+        if (dWq) return zero_f32(dWq, (size_t)Kp * K, st);
+        return SRU_OK;
+    }
+    CUtensorMap ma, mb;
+    // dWo = dU^T P: A(r = n, red = m) = dU[m][n] MN-major; B(c = kp, red = m) = P[m][kp] MN-major
+    if (dWo) {
+        if (!map_mnmajor(&ma, dU, N, M, N) || !map_mnmajor(&mb, P, Kp, M, Kp)) return SRU_ERR_INVALID;
+        sru_status s = launch_tc_gemm<true, true, sru::gemm::kOutF32>(ma, mb, dWo, N, Kp, M, st);
+        if (s != SRU_OK) return s;
+    }
+    // dP = dU Wo (bf16): A = dU K-major over n; B(c = kp, red = n) = Wo[n][kp] MN-major
+    {
+        if (!map_kmajor(&ma, dU, M, N, sru::gemm::BM) || !map_mnmajor(&mb, Wo, Kp, N, Kp)) return SRU_ERR_INVALID;
+        sru_status s = launch_tc_gemm<false, true, sru::gemm::kOutBF16>(ma, mb, dP, M, Kp, N, st);
+        if (s != SRU_OK) return s;
+    }
+    // dWq = dP^T X and dX (+)= dP Wq: the gradients of the first product
+    return sru_project_backward(dP, X, Wq, SRU_BF16, dX, accumulate, dWq, M, Kp, K, stream);
+}
+
 sru_status sru_decode_step(const void* X_t, const void* W, const float* x_t, const float* v, const float* b,
                            float* c, float* h_t, int64_t B, int64_t d, float alpha, void* stream) {
     if (B < 0 || d < 1) return SRU_ERR_INVALID;
