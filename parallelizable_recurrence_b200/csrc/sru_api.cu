@@ -253,18 +253,21 @@ constexpr bool kGemmPair = SRU_GEMM_USE_PAIR != 0;
 // rows of B staged per CTA for a K-major B operand
 constexpr uint32_t kGemmBRows = kGemmPair ? (uint32_t)sru::gemm::P_CN : (uint32_t)sru::gemm::BN;
 
+// splits = 2 (pair kernel, OUT == kOutF32Red only): each output tile's
+// reduction is cut in two halves that add into the zeroed output.
 template <bool A_MN, bool B_MN, int OUT>
 sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
-                          int64_t Kr, cudaStream_t st) {
+                          int64_t Kr, cudaStream_t st, int splits = 1) {
     if (kGemmPair) {
         auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT>;
         SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
-        const int64_t tiles =
-            ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN);
-        const int64_t pairs = tiles < sm_count() / 2 ? tiles : sm_count() / 2;
+        const int64_t units =
+            ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN) * splits;
+        const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
         kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(ma, mb, out, (int)R, (int)C,
-                                                                                       (int)Kr, (int)C);
+                                                                                       (int)Kr, (int)C, splits);
     } else {
+        if (splits != 1) return SRU_ERR_UNSUPPORTED;
         auto kern = sru::gemm::tc_gemm_kernel<A_MN, B_MN, OUT>;
         SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::SMEM_BYTES));
         const int64_t tiles = ((R + sru::gemm::BM - 1) / sru::gemm::BM) * ((C + sru::gemm::BN - 1) / sru::gemm::BN);
@@ -273,6 +276,18 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
     }
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
+}
+
+// Whether an fp32-output product with few output tiles and a long reduction
+// runs faster as two K halves: when the halves fill the SM pairs' waves
+// better (e.g. 96 tiles on 74 pairs: 65% of the second wave idle, versus 192
+// halves in 3 waves at 86%), and each half keeps at least 16 k-blocks.
+bool gemm_split_pays(int64_t R, int64_t C, int64_t Kr) {
+    if (!kGemmPair || Kr < 32 * sru::gemm::BK) return false;
+    const int64_t tiles = ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN);
+    const int64_t P = sm_count() / 2;
+    auto eff = [&](int64_t u) { return (double)u / (double)(((u + P - 1) / P) * P); };
+    return eff(2 * tiles) > eff(tiles) + 0.05;
 }
 
 // K-major operand (rows x K), contiguous K: box (64, box_rows)
@@ -678,6 +693,10 @@ sru_status sru_project_backward(const void* dU, const void* X, const void* W, in
         CUtensorMap ma, mb;
         // A(r = n, red = m) = dU[m][n]: MN-major, ld = N; B(c = k, red = m) = X[m][k]: MN-major, ld = K
         if (!map_mnmajor(&ma, dU, N, M, N) || !map_mnmajor(&mb, X, K, M, K)) return SRU_ERR_INVALID;
+        if (gemm_split_pays(N, K, M)) {
+            SRU_CUDA_TRY(cudaMemsetAsync(dW, 0, (size_t)N * K * sizeof(float), st));
+            return launch_tc_gemm<true, true, sru::gemm::kOutF32Red>(ma, mb, dW, N, K, M, st, 2);
+        }
         return launch_tc_gemm<true, true, sru::gemm::kOutF32>(ma, mb, dW, N, K, M, st);
     }
     return SRU_OK;

@@ -38,7 +38,10 @@ constexpr uint32_t TMEM_COLS = 2 * BN;  // two fp32 accumulators
 constexpr uint32_t MN_BOX_BYTES = 64 * 64 * 2;  // one (64 x 64) MN-major box
 constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
-enum OutMode : int { kOutBF16 = 0, kOutF32 = 1, kOutF32Acc = 2 };
+// kOutF32Red: add into an fp32 output with vector atomics (the two K halves of
+// a split tile, onto an output the host zeroed: 0 + a + b rounds the same in
+// either order, so the sum does not depend on which half lands first).
+enum OutMode : int { kOutBF16 = 0, kOutF32 = 1, kOutF32Acc = 2, kOutF32Red = 3 };
 
 // Shared-memory matrix descriptor (tcgen05 "smem descriptor"): start address,
 // leading- and stride-dimension byte offsets (16-byte units), descriptor
@@ -88,6 +91,10 @@ __device__ __forceinline__ void epilogue_store_row32(void* __restrict__ out, int
             if (col0 + g * 4 < N) {
                 float4 val = make_float4(__uint_as_float(r[g * 4 + 0]), __uint_as_float(r[g * 4 + 1]),
                                          __uint_as_float(r[g * 4 + 2]), __uint_as_float(r[g * 4 + 3]));
+                if (OUT == kOutF32Red) {
+                    atomicAdd(reinterpret_cast<float4*>(o + g * 4), val);
+                    continue;
+                }
                 if (OUT == kOutF32Acc) {
                     const float4 old = *reinterpret_cast<const float4*>(o + g * 4);
                     val.x += old.x;
@@ -306,7 +313,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16_pair(bool a_mn, bool b_mn) {
 template <bool A_MN, bool B_MN, int OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                        void* __restrict__ out, int M, int N, int K, int ldo) {
+                        void* __restrict__ out, int M, int N, int K, int ldo, int splits) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
@@ -324,6 +331,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int m_tiles = (M + P_BM - 1) / P_BM, n_tiles = (N + P_BN - 1) / P_BN;
     const int tiles = m_tiles * n_tiles;
     const int kblocks = (K + BK - 1) / BK;
+    // work unit u = (tile u / splits, K part u % splits); splits > 1 only with
+    // kOutF32Red and at least one k-block per part (the host checks both)
+    const int units = tiles * splits;
+    const int kper = (kblocks + splits - 1) / splits;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < P_STAGES; ++s) {
@@ -358,10 +369,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             uint32_t issued = 0;
             int stage = 0;
             uint32_t phase = 0;
-            for (int tile = pair_id; tile < tiles && !*abort_flag; tile += n_pairs) {
+            for (int u = pair_id; u < units && !*abort_flag; u += n_pairs) {
+                const int tile = u / splits, kb_lo = (u % splits) * kper;
+                const int kb_hi = min(kblocks, kb_lo + kper);
                 const int m0 = (tile / n_tiles) * P_BM + (int)rank * P_CM;
                 const int n0 = (tile % n_tiles) * P_BN + (int)rank * P_CN;
-                for (int kb = 0; kb < kblocks; ++kb) {
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, kErrTimeoutMma) || *abort_flag) {
                         *abort_flag = 1;
                         break;
@@ -402,7 +415,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             int stage = 0;
             uint32_t phase = 0, nconsumed = 0;
             int it = 0;
-            for (int tile = pair_id; tile < tiles && !*abort_flag; tile += n_pairs, ++it) {
+            for (int u = pair_id; u < units && !*abort_flag; u += n_pairs, ++it) {
+                const int kb_lo = (u % splits) * kper, kb_hi = min(kblocks, kb_lo + kper);
                 const int acc = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, kErrTimeoutEpilogue)) {
@@ -412,7 +426,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + acc * P_BN;
                 bool ok = true;
-                for (int kb = 0; kb < kblocks; ++kb) {
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!mbar_wait(&full[stage], phase, kErrTimeoutLoad)) {
                         ok = false;
                         break;
@@ -426,7 +440,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                                                     : smem_desc_sw128(a_addr + kk * 32, 16, 1024);
                         const uint64_t bdesc = B_MN ? smem_desc_sw128(b_addr + kk * 2048, MN_BOX_BYTES, 1024)
                                                     : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-                        tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        tc_mma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb != kb_lo || kk != 0) ? 1u : 0u);
                     }
                     tc_commit_pair_mc(&empty[stage], 0x3);  // frees this stage in both CTAs
                     *consumed = ++nconsumed;
@@ -448,7 +462,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // ---------------------------------------------------------- epilogue (both CTAs)
         const int quarter = warp & 3;
         int it = 0;
-        for (int tile = pair_id; tile < tiles; tile += n_pairs, ++it) {
+        for (int u = pair_id; u < units; u += n_pairs, ++it) {
+            const int tile = u / splits;
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             const int m0 = (tile / n_tiles) * P_BM + (int)rank * P_CM, n0 = (tile % n_tiles) * P_BN;

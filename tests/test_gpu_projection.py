@@ -102,3 +102,20 @@ def test_project_large_k_sampled(sru):
     ref = oracle.project_dW_entries(dUb, Xb, rows, cols)
     absref = oracle.project_dW_entries(tl.abs_operand(dUb), tl.abs_operand(Xb), rows, cols)
     tl.assert_close_sum("dW sampled", tl.host_f64(dW)[rows, cols], ref, absref)
+
+
+def test_split_reduction_dw_is_deterministic(sru):
+    """dW with few output tiles and a long reduction is computed as two K halves
+    added into the zeroed output; with two addends per element the fp32 sum is
+    the same whichever half lands first, so repeated calls agree bit for bit."""
+    rng = np.random.default_rng(5)
+    M, N, K = 8192, 768, 256          # 3 output tiles, 128 k-blocks: the split is taken
+    Xd, dUd = tl.to_dev_bf16(_bf16(rng, (M, K))), tl.to_dev_bf16(_bf16(rng, (M, N)))
+    Wd = tl.to_dev_bf16(_bf16(rng, (N, K)))
+    outs = []
+    for _ in range(3):
+        dW = torch.full((N, K), float("nan"), device="cuda")
+        sru.sru_project_backward(dUd, Xd, Wd, dW=dW)
+        outs.append(dW)
+    assert sru.sru_sync_status() == 0
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
