@@ -214,3 +214,48 @@ def project_dW_entries(dU, X, rows, cols):
     M, N = dU.shape
     K = X.shape[1]
     return gemm_entries(rows, cols, M, dU, 1, N, X, 1, K)
+
+
+def _as_f64(a):
+    a = np.asarray(a)
+    if a.dtype == np.uint16:  # bf16 bits, widened exactly
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def attention_project(X, Wq, Wk, Wv, Wo, alpha, L, B, causal=True, ln_gamma=None, ln_beta=None, ln_eps=1e-5):
+    """SRU++'s producer of U ("When Attention Meets Fast Recurrence", SRU++
+    section: attention replaces the linear map of Eq. (1)), in fp64:
+
+      Q = X Wq^T, K = Q Wk^T, V = Q Wv^T         (rows = tokens; Wq (d', d), Wk, Wv (d', d'))
+      per batch row b, over its L tokens:
+        A_b = softmax(Q_b K_b^T / sqrt(d')) V_b   (scaled dot-product attention;
+                                                   with causal=True token t sees tokens <= t)
+      R = Q + alpha A, or layernorm(Q + alpha A) over the d' features
+          (ln_gamma, ln_beta given; the page's post-attention normalisation)
+      U = R Wo^T                                  (Wo (N, d'))
+
+    X is (L*B, d) time-major (row t*B + b), bf16 bits or floats; returns U
+    (L*B, N) float64.  Every product is a plain matrix product; the softmax
+    subtracts the row maximum before exponentiating (the same value).
+    """
+    X, Wq, Wk, Wv, Wo = (_as_f64(a) for a in (X, Wq, Wk, Wv, Wo))
+    Q = X @ Wq.T
+    K = Q @ Wk.T
+    V = Q @ Wv.T
+    dp = Q.shape[1]
+    A = np.zeros_like(Q)
+    for b in range(B):
+        rows = np.arange(L) * B + b
+        Qb, Kb, Vb = Q[rows], K[rows], V[rows]
+        for t in range(L):
+            n = t + 1 if causal else L
+            s = Kb[:n] @ Qb[t] / np.sqrt(dp)
+            p = np.exp(s - s.max())
+            A[rows[t]] = (p / p.sum()) @ Vb[:n]
+    R = Q + alpha * A
+    if ln_gamma is not None:
+        mu = R.mean(axis=1, keepdims=True)
+        var = ((R - mu) ** 2).mean(axis=1, keepdims=True)
+        R = (R - mu) / np.sqrt(var + ln_eps) * _as_f64(ln_gamma) + _as_f64(ln_beta)
+    return R @ Wo.T

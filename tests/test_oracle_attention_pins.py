@@ -1,0 +1,86 @@
+"""Pins of the oracle's SRU++ attention producer (oracle.attention_project),
+each against a fact the page or the mathematics fixes, not against the
+oracle's own formula."""
+import numpy as np
+
+import oracle
+
+
+def _w(rng, *shape):
+    return rng.standard_normal(shape) / np.sqrt(shape[-1])
+
+
+def _case(seed=0, L=5, B=3, d=12, dp=4, N=18):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((L * B, d)), _w(rng, dp, d), _w(rng, dp, dp), _w(rng, dp, dp), _w(rng, N, dp), L, B)
+
+
+def test_alpha_zero_is_the_factorised_linear_map():
+    # the page: with alpha = 0, U = Wo Q = (Wo Wq) X^T, the attention is skipped
+    X, Wq, Wk, Wv, Wo, L, B = _case()
+    U = oracle.attention_project(X, Wq, Wk, Wv, Wo, 0.0, L, B)
+    np.testing.assert_allclose(U, X @ (Wo @ Wq).T, rtol=1e-12, atol=1e-12)
+
+
+def test_single_token_attends_only_to_itself():
+    # L = 1: the softmax of one score is 1, so A = V = Q Wv^T and U = Wo (Q + alpha V)
+    X, Wq, Wk, Wv, Wo, _, B = _case(L=1)
+    alpha = 0.7
+    Q = X @ Wq.T
+    U = oracle.attention_project(X, Wq, Wk, Wv, Wo, alpha, 1, B)
+    np.testing.assert_allclose(U, (Q + alpha * (Q @ Wv.T)) @ Wo.T, rtol=1e-12, atol=1e-12)
+
+
+def test_constant_sequence_averages_identical_values():
+    # every token of a row equal: all V_t equal, so any convex weights give A_t = V_t
+    X, Wq, Wk, Wv, Wo, L, B = _case(L=6)
+    X = np.repeat(X[:B][None], L, axis=0).reshape(L * B, -1)
+    alpha = -1.3
+    Q = X @ Wq.T
+    for causal in (True, False):
+        U = oracle.attention_project(X, Wq, Wk, Wv, Wo, alpha, L, B, causal=causal)
+        np.testing.assert_allclose(U, (Q + alpha * (Q @ Wv.T)) @ Wo.T, rtol=1e-12, atol=1e-12)
+
+
+def test_causal_output_ignores_later_tokens_and_rows():
+    X, Wq, Wk, Wv, Wo, L, B = _case(L=7, B=2)
+    U = oracle.attention_project(X, Wq, Wk, Wv, Wo, 0.9, L, B)
+    Y = X.copy()
+    Y[4 * B + 1] += 3.0                      # token t = 4 of batch row 1
+    V = oracle.attention_project(Y, Wq, Wk, Wv, Wo, 0.9, L, B)
+    rows_b1 = np.arange(L) * B + 1
+    np.testing.assert_array_equal(U[:4 * B], V[:4 * B])              # earlier tokens: unchanged
+    np.testing.assert_array_equal(U[np.arange(L) * B], V[np.arange(L) * B])  # other batch row: unchanged
+    assert np.abs(U[rows_b1[4:]] - V[rows_b1[4:]]).max() > 1e-3       # this and later tokens move
+
+
+def test_last_token_is_the_same_with_or_without_the_causal_mask():
+    X, Wq, Wk, Wv, Wo, L, B = _case(L=6)
+    U = oracle.attention_project(X, Wq, Wk, Wv, Wo, 1.1, L, B, causal=True)
+    V = oracle.attention_project(X, Wq, Wk, Wv, Wo, 1.1, L, B, causal=False)
+    last = (L - 1) * B + np.arange(B)
+    np.testing.assert_allclose(U[last], V[last], rtol=1e-12, atol=1e-12)
+    assert np.abs(U[:B] - V[:B]).max() > 1e-6
+
+
+def test_two_token_softmax_by_hand():
+    # L = 2, d = d' = 1, N = 1, every weight 1 except Wv: scores are q_t q_s, A_1 mixes V_0, V_1
+    X = np.array([[0.5], [2.0]])             # B = 1: tokens 0 and 1
+    one = np.ones((1, 1))
+    Wv = np.array([[3.0]])
+    U = oracle.attention_project(X, one, one, Wv, one, 1.0, 2, 1)
+    q0, q1 = 0.5, 2.0
+    w0, w1 = np.exp(q1 * q0), np.exp(q1 * q1)   # sqrt(d') = 1
+    a1 = (w0 * 3 * q0 + w1 * 3 * q1) / (w0 + w1)
+    np.testing.assert_allclose(U[:, 0], [q0 + 3 * q0, q1 + a1], rtol=1e-12)
+
+
+def test_layernorm_single_token_closed_form():
+    X, Wq, Wk, Wv, Wo, _, B = _case(L=1, dp=6)
+    g = np.linspace(0.5, 1.5, 6)
+    be = np.linspace(-0.2, 0.3, 6)
+    Q = X @ Wq.T
+    R = Q + 0.4 * (Q @ Wv.T)
+    Rn = (R - R.mean(1, keepdims=True)) / np.sqrt(R.var(1, keepdims=True) + 1e-5) * g + be
+    U = oracle.attention_project(X, Wq, Wk, Wv, Wo, 0.4, 1, B, ln_gamma=g, ln_beta=be)
+    np.testing.assert_allclose(U, Rn @ Wo.T, rtol=1e-11, atol=1e-12)
