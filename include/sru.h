@@ -217,6 +217,28 @@ sru_status sru_project_factored_backward(const void* dU, const void* X, const vo
                                          float* dWo, int64_t M, int64_t N, int64_t K, int64_t Kp, void* stream);
 
 /*
+ * SRU++'s producer of U: single-head attention in place of the linear map of
+ * Eq. (1) (the page's SRU++ section).  With d' the attention width:
+ *   Q = X Wq^T                  (L*B, d')   Wq  (d', d)
+ *   [K | V] = Q Wkv^T           (L*B, 2d')  Wkv (2d', d') = [Wk; Wv]
+ *   per batch row b, over its L tokens (rows t*B + b):
+ *     A_b = softmax(Q_b K_b^T / sqrt(d')) V_b, token t seeing tokens <= t when causal
+ *   R = Q + alpha A, or layernorm(Q + alpha A) * gamma + beta over the d' features
+ *       (eps 1e-5) when ln_gamma and ln_beta are given (both or neither)
+ *   U = R Wo^T                  (L*B, N)    Wo  (N, d'), U of type u_t (BF16 or F32)
+ * X, Wq, Wkv, Wo bf16; X and U time-major as everywhere.  Q, [K | V], P and R
+ * are rounded to bf16 (they are tensor-core operands), scores and A are fp32.
+ * The workspace (>= sru_attention_workspace_bytes(L, B, d')) holds Q, K, V,
+ * one batch row's scores and probabilities, A and R.  Limits: d, d', N and L
+ * multiples of 8, L <= 65536.  The per-batch products are separate launches.
+ */
+size_t sru_attention_workspace_bytes(int64_t L, int64_t B, int64_t dp);
+sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv, const void* Wo, float alpha,
+                                 const float* ln_gamma, const float* ln_beta, int causal, void* U, int u_t,
+                                 int64_t L, int64_t B, int64_t d, int64_t dp, int64_t N, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
  * One time step of a unidirectional layer for inference (token-by-token
  * decoding), with the projection fused in.  The page notes that SRU-based
  * models run as an RNN at inference time (one token per step); there the

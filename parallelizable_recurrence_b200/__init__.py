@@ -32,7 +32,8 @@ SRU_FLAG_TEST_WITHHOLD_CARRY = 0x8
 # every symbol include/sru.h declares
 EXPORTED = ("sru_status_string", "sru_get_last_cuda_error", "sru_version", "sru_workspace_bytes",
             "sru_project", "sru_project_backward", "sru_forward", "sru_backward", "sru_forward_scan_noalloc",
-            "sru_project_factored", "sru_project_factored_backward", "sru_decode_step", "sru_sync_status")
+            "sru_project_factored", "sru_project_factored_backward", "sru_attention_workspace_bytes",
+            "sru_attention_project", "sru_decode_step", "sru_sync_status")
 
 
 class SRUError(RuntimeError):
@@ -85,6 +86,11 @@ def load_library(path: str = LIB_PATH):
     lib.sru_project_factored_backward.restype = _int
     lib.sru_project_factored_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _i64, _i64,
                                                   _i64, _i64, _vp]
+    lib.sru_attention_workspace_bytes.restype = ctypes.c_size_t
+    lib.sru_attention_workspace_bytes.argtypes = [_i64, _i64, _i64]
+    lib.sru_attention_project.restype = _int
+    lib.sru_attention_project.argtypes = [_vp, _vp, _vp, _vp, _f32, _vp, _vp, _int, _vp, _int, _i64, _i64, _i64,
+                                          _i64, _i64, _vp, ctypes.c_size_t, _vp]
     lib.sru_decode_step.restype = _int
     lib.sru_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _vp]
     lib.sru_sync_status.restype = _int
@@ -238,6 +244,30 @@ def sru_project_factored_backward(dU, X, Wq, Wo, P, dP, dX=None, accumulate: boo
                                              _ptr(dWq, torch.float32), _ptr(dWo, torch.float32), M, N, K, Kp,
                                              _stream(stream)), "sru_project_factored_backward")
     return dX, dWq, dWo
+
+
+def sru_attention_project(X, Wq, Wkv, Wo, U, L: int, B: int, alpha: float, ln_gamma=None, ln_beta=None,
+                          causal: bool = True, workspace=None, stream=None):
+    """SRU++ attention producer of U (see sru.h).  X (L*B, d) bf16 time-major,
+    Wq (d', d), Wkv (2d', d') = [Wk; Wv], Wo (N, d') bf16; U (L*B, N) bf16 or
+    fp32.  A workspace of sru_attention_workspace_bytes bytes is allocated when
+    none is given."""
+    lib = load_library()
+    M, d = X.shape
+    dp, N = Wq.shape[0], Wo.shape[0]
+    if M != L * B or Wq.shape[1] != d or tuple(Wkv.shape) != (2 * dp, dp) or Wo.shape[1] != dp:
+        raise ValueError("shape mismatch")
+    if workspace is None:
+        n = int(lib.sru_attention_workspace_bytes(L, B, dp))
+        if n == 0:
+            raise SRUError(SRU_ERR_UNSUPPORTED, "sru_attention_workspace_bytes", lib)
+        workspace = torch.empty(n, dtype=torch.uint8, device=X.device)
+    _check(lib.sru_attention_project(_ptr(X, torch.bfloat16), _ptr(Wq, torch.bfloat16), _ptr(Wkv, torch.bfloat16),
+                                     _ptr(Wo, torch.bfloat16), float(alpha), _ptr(ln_gamma, torch.float32),
+                                     _ptr(ln_beta, torch.float32), int(bool(causal)), _ptr(U), _dtype_code(U),
+                                     L, B, d, dp, N, _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "sru_attention_project")
+    return U
 
 
 def sru_decode_step(X_t, W, x_t, v, b, c, h_t, alpha: float = 1.0, stream=None):

@@ -12,6 +12,7 @@
 #include "../../include/sru.h"
 #include "sru_gemm.cuh"
 #include "sru_recurrence.cuh"
+#include "sru_attention.cuh"
 #include "sru_decode.cuh"
 #include "sru_scan.cuh"
 
@@ -255,9 +256,11 @@ constexpr uint32_t kGemmBRows = kGemmPair ? (uint32_t)sru::gemm::P_CN : (uint32_
 
 // splits = 2 (pair kernel, OUT == kOutF32Red only): each output tile's
 // reduction is cut in two halves that add into the zeroed output.
+// ldo: output row stride in elements (default C).
 template <bool A_MN, bool B_MN, int OUT>
 sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
-                          int64_t Kr, cudaStream_t st, int splits = 1) {
+                          int64_t Kr, cudaStream_t st, int splits = 1, int64_t ldo = -1) {
+    if (ldo < 0) ldo = C;
     if (kGemmPair) {
         auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT>;
         SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
@@ -265,17 +268,69 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
             ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN) * splits;
         const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
         kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(ma, mb, out, (int)R, (int)C,
-                                                                                       (int)Kr, (int)C, splits);
+                                                                                       (int)Kr, (int)ldo, splits, 1,
+                                                                                       0LL);
     } else {
         if (splits != 1) return SRU_ERR_UNSUPPORTED;
         auto kern = sru::gemm::tc_gemm_kernel<A_MN, B_MN, OUT>;
         SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::SMEM_BYTES));
         const int64_t tiles = ((R + sru::gemm::BM - 1) / sru::gemm::BM) * ((C + sru::gemm::BN - 1) / sru::gemm::BN);
         const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-        kern<<<grid, sru::gemm::THREADS, sru::gemm::SMEM_BYTES, st>>>(ma, mb, out, (int)R, (int)C, (int)Kr, (int)C);
+        kern<<<grid, sru::gemm::THREADS, sru::gemm::SMEM_BYTES, st>>>(ma, mb, out, (int)R, (int)C, (int)Kr, (int)ldo);
     }
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
+}
+
+// `batches` products of one shape in one launch of the pair kernel (operand
+// maps from map_kmajor_b / map_mnmajor_b with the batch at coordinate BPA /
+// BPB); product z writes out + z * out_bstride elements.
+template <bool A_MN, bool B_MN, int OUT, int BPA, int BPB>
+sru_status launch_tc_gemm_batched(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
+                                  int64_t Kr, int64_t ldo, int64_t batches, int64_t out_bstride, cudaStream_t st) {
+    if (!kGemmPair) return SRU_ERR_UNSUPPORTED;
+    auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT, BPA, BPB>;
+    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
+    const int64_t units =
+        ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN) * batches;
+    if (units >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
+    const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
+    kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
+        ma, mb, out, (int)R, (int)C, (int)Kr, (int)ldo, 1, (int)batches, (long long)out_bstride);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
+// Batched K-major operand: element (row r, k) of batch z at
+// p[z * batch_ld + r * row_ld + k]; the batch is coordinate bpos (1: dims
+// (K, batches, rows), 2: dims (K, rows, batches)) -- whichever keeps the
+// strides increasing.
+bool map_kmajor_b(CUtensorMap* m, const void* p, int64_t rows, int64_t K, int64_t row_ld, int64_t batches,
+                  int64_t batch_ld, uint32_t box_rows, int bpos) {
+    if (bpos == 1) {
+        const uint64_t dims[3] = {(uint64_t)K, (uint64_t)batches, (uint64_t)rows};
+        const uint64_t strides[2] = {(uint64_t)batch_ld * 2, (uint64_t)row_ld * 2};
+        const uint32_t box[3] = {64, 1, box_rows};
+        return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    const uint64_t dims[3] = {(uint64_t)K, (uint64_t)rows, (uint64_t)batches};
+    const uint64_t strides[2] = {(uint64_t)row_ld * 2, (uint64_t)batch_ld * 2};
+    const uint32_t box[3] = {64, box_rows, 1};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// Batched MN-major operand: element (r, k) of batch z at p[z * batch_ld + k * ld + r].
+bool map_mnmajor_b(CUtensorMap* m, const void* p, int64_t rows, int64_t K, int64_t ld, int64_t batches,
+                   int64_t batch_ld, int bpos) {
+    if (bpos == 1) {
+        const uint64_t dims[3] = {(uint64_t)rows, (uint64_t)batches, (uint64_t)K};
+        const uint64_t strides[2] = {(uint64_t)batch_ld * 2, (uint64_t)ld * 2};
+        const uint32_t box[3] = {64, 1, 64};
+        return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    const uint64_t dims[3] = {(uint64_t)rows, (uint64_t)K, (uint64_t)batches};
+    const uint64_t strides[2] = {(uint64_t)ld * 2, (uint64_t)batch_ld * 2};
+    const uint32_t box[3] = {64, 64, 1};
+    return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Whether an fp32-output product with few output tiles and a long reduction
@@ -290,10 +345,11 @@ bool gemm_split_pays(int64_t R, int64_t C, int64_t Kr) {
     return eff(2 * tiles) > eff(tiles) + 0.05;
 }
 
-// K-major operand (rows x K), contiguous K: box (64, box_rows)
-bool map_kmajor(CUtensorMap* m, const void* p, int64_t rows, int64_t K, uint32_t box_rows) {
+// K-major operand (rows x K), contiguous K, rows ld elements apart (ld >= K;
+// default K): box (64, box_rows)
+bool map_kmajor(CUtensorMap* m, const void* p, int64_t rows, int64_t K, uint32_t box_rows, int64_t ld = -1) {
     const uint64_t dims[2] = {(uint64_t)K, (uint64_t)rows};
-    const uint64_t strides[1] = {(uint64_t)K * 2};
+    const uint64_t strides[1] = {(uint64_t)(ld < 0 ? K : ld) * 2};
     const uint32_t box[2] = {64, box_rows};
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
@@ -898,6 +954,92 @@ sru_status sru_project_factored_backward(const void* dU, const void* X, const vo
     }
     // dWq = dP^T X and dX (+)= dP Wq: the gradients of the first product
     return sru_project_backward(dP, X, Wq, SRU_BF16, dX, accumulate, dWq, M, Kp, K, stream);
+}
+
+// ---- SRU++ attention producer
+// Batch rows are processed in groups of G: one batched launch each for the
+// scores, the softmax and A; G bounds the scores and probabilities buffers.
+constexpr size_t kAttnGroupBytes = (size_t)256 << 20;
+int64_t attn_group(int64_t L, int64_t B) {
+    const int64_t g = (int64_t)(kAttnGroupBytes / ((size_t)L * L * 6));
+    return g < 1 ? 1 : (g > B ? B : g);
+}
+struct AttnWs {
+    size_t q, kv, s, p, a, r, total;
+};
+AttnWs attn_ws(int64_t L, int64_t B, int64_t dp) {
+    AttnWs w{};
+    const int64_t M = L * B, G = attn_group(L, B);
+    size_t off = 0;
+    w.q = off;  off += round256((size_t)M * dp * 2);
+    w.kv = off; off += round256((size_t)M * 2 * dp * 2);
+    w.s = off;  off += round256((size_t)G * L * L * 4);
+    w.p = off;  off += round256((size_t)G * L * L * 2);
+    w.a = off;  off += round256((size_t)M * dp * 4);
+    w.r = off;  off += round256((size_t)M * dp * 2);
+    w.total = off;
+    return w;
+}
+
+size_t sru_attention_workspace_bytes(int64_t L, int64_t B, int64_t dp) {
+    if (L < 1 || B < 1 || dp < 8 || dp % 8 != 0 || L % 8 != 0) return 0;
+    return attn_ws(L, B, dp).total;
+}
+
+sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv, const void* Wo, float alpha,
+                                 const float* ln_gamma, const float* ln_beta, int causal, void* U, int u_t,
+                                 int64_t L, int64_t B, int64_t d, int64_t dp, int64_t N, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    if (L < 1 || B < 1 || d < 1 || dp < 1 || N < 1) return SRU_ERR_INVALID;
+    if (!X || !Wq || !Wkv || !Wo || !U || !workspace || !aligned16(workspace)) return SRU_ERR_INVALID;
+    if ((ln_gamma == nullptr) != (ln_beta == nullptr)) return SRU_ERR_INVALID;
+    if (u_t != SRU_BF16 && u_t != SRU_F32) return SRU_ERR_INVALID;
+    if (d % 8 != 0 || dp % 8 != 0 || N % 8 != 0 || L % 8 != 0) return SRU_ERR_UNSUPPORTED;
+    const int64_t M = L * B;
+    if (M >= ((int64_t)1 << 31) || L > 65536) return SRU_ERR_UNSUPPORTED;
+    const AttnWs w = attn_ws(L, B, dp);
+    if (workspace_bytes < w.total) return SRU_ERR_INVALID;
+    cudaStream_t st = as_stream(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    __nv_bfloat16* Q = reinterpret_cast<__nv_bfloat16*>(ws + w.q);
+    __nv_bfloat16* KV = reinterpret_cast<__nv_bfloat16*>(ws + w.kv);
+    float* S = reinterpret_cast<float*>(ws + w.s);
+    __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(ws + w.p);
+    float* A = reinterpret_cast<float*>(ws + w.a);
+    __nv_bfloat16* R = reinterpret_cast<__nv_bfloat16*>(ws + w.r);
+    // Q = X Wq^T, then [K | V] = Q [Wk; Wv]^T
+    sru_status s = sru_project(X, SRU_BF16, Wq, SRU_BF16, Q, SRU_BF16, M, dp, d, stream);
+    if (s != SRU_OK) return s;
+    s = sru_project(Q, SRU_BF16, Wkv, SRU_BF16, KV, SRU_BF16, M, 2 * dp, dp, stream);
+    if (s != SRU_OK) return s;
+    const float scale = 1.0f / sqrtf((float)dp);
+    const int64_t G = attn_group(L, B);
+    // batch row b's tokens are rows t*B + b of the time-major Q, K, V and A
+    for (int64_t b0 = 0; b0 < B; b0 += G) {
+        const int64_t g = B - b0 < G ? B - b0 : G;
+        CUtensorMap ma, mb;
+        // S_z = Q_z K_z^T (z = 0 .. g-1): K-major over d'; batch stride d' / 2d', row stride B d' / 2B d'
+        if (!map_kmajor_b(&ma, Q + b0 * dp, L, dp, B * dp, g, dp, sru::gemm::BM, 1) ||
+            !map_kmajor_b(&mb, KV + b0 * 2 * dp, L, dp, B * 2 * dp, g, 2 * dp, kGemmBRows, 1))
+            return SRU_ERR_INVALID;
+        s = launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st);
+        if (s != SRU_OK) return s;
+        sru::sru_softmax_rows_kernel<<<blocks_for((size_t)(g * L), sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+            S, P, (int)L, (int)(g * L), scale, causal ? 1 : 0);
+        SRU_CUDA_TRY(cudaGetLastError());
+        // A_z = P_z V_z: P_z K-major over s (batch outermost); V_z(c = j, red = s) at
+        // KV[(s*B + b0 + z)*2d' + d' + j]: MN-major, batch stride 2d'
+        if (!map_kmajor_b(&ma, P, L, L, L, g, L * L, sru::gemm::BM, 2) ||
+            !map_mnmajor_b(&mb, KV + b0 * 2 * dp + dp, dp, L, B * 2 * dp, g, 2 * dp, 1))
+            return SRU_ERR_INVALID;
+        s = launch_tc_gemm_batched<false, true, sru::gemm::kOutF32, 2, 1>(ma, mb, A + b0 * dp, L, dp, L, B * dp, g,
+                                                                           dp, st);
+        if (s != SRU_OK) return s;
+    }
+    sru::sru_residual_norm_kernel<<<blocks_for((size_t)M, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+        Q, A, alpha, ln_gamma, ln_beta, R, (int)M, (int)dp);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return sru_project(R, SRU_BF16, Wo, SRU_BF16, U, u_t, M, N, dp, stream);
 }
 
 sru_status sru_decode_step(const void* X_t, const void* W, const float* x_t, const float* v, const float* b,

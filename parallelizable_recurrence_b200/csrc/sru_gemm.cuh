@@ -310,10 +310,27 @@ __host__ __device__ constexpr uint32_t idesc_bf16_pair(bool a_mn, bool b_mn) {
            ((uint32_t)(P_BN >> 3) << 17) | ((uint32_t)(P_BM >> 4) << 24);
 }
 
-template <bool A_MN, bool B_MN, int OUT>
+// Batched form (BAT): `batches` independent products of the same shape.  The
+// operands' tensor maps are 3-D with the batch index as coordinate bpos_a /
+// bpos_b (1 or 2) and the 2-D tile coordinates in the other two, so a box
+// lands in shared memory exactly as in the 2-D case; batch z writes
+// out + z * out_bstride.
+template <int BPOS>
+__device__ __forceinline__ void tma_load_tile_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                                   int z) {
+    if (BPOS == 0)
+        tma_load_2d_pair(dst, map, bar, x, y);
+    else if (BPOS == 1)
+        tma_load_3d_pair(dst, map, bar, x, z, y);
+    else
+        tma_load_3d_pair(dst, map, bar, x, y, z);
+}
+
+template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                        void* __restrict__ out, int M, int N, int K, int ldo, int splits) {
+                        void* __restrict__ out, int M, int N, int K, int ldo, int splits, int batches,
+                        long long out_bstride) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
@@ -333,7 +350,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int kblocks = (K + BK - 1) / BK;
     // work unit u = (tile u / splits, K part u % splits); splits > 1 only with
     // kOutF32Red and at least one k-block per part (the host checks both)
-    const int units = tiles * splits;
+    const int units = tiles * splits * batches;  // batch-major, then tile, then K part
     const int kper = (kblocks + splits - 1) / splits;
 
     if (threadIdx.x == 0) {
@@ -370,7 +387,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             for (int u = pair_id; u < units && !*abort_flag; u += n_pairs) {
-                const int tile = u / splits, kb_lo = (u % splits) * kper;
+                const int z = u / (tiles * splits), uu = u % (tiles * splits);
+                const int tile = uu / splits, kb_lo = (uu % splits) * kper;
                 const int kb_hi = min(kblocks, kb_lo + kper);
                 const int m0 = (tile / n_tiles) * P_BM + (int)rank * P_CM;
                 const int n0 = (tile % n_tiles) * P_BN + (int)rank * P_CN;
@@ -385,16 +403,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t bar = leader_full0 + (uint32_t)stage * 8u;
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
                     if (!A_MN) {
-                        tma_load_2d_pair(a_dst, &map_a, bar, k0, m0);
+                        tma_load_tile_pair<BPA>(a_dst, &map_a, bar, k0, m0, z);
                     } else {
-                        tma_load_2d_pair(a_dst, &map_a, bar, m0, k0);
-                        tma_load_2d_pair(a_dst + MN_BOX_BYTES, &map_a, bar, m0 + 64, k0);
+                        tma_load_tile_pair<BPA>(a_dst, &map_a, bar, m0, k0, z);
+                        tma_load_tile_pair<BPA>(a_dst + MN_BOX_BYTES, &map_a, bar, m0 + 64, k0, z);
                     }
                     if (!B_MN) {
-                        tma_load_2d_pair(b_dst, &map_b, bar, k0, n0);
+                        tma_load_tile_pair<BPB>(b_dst, &map_b, bar, k0, n0, z);
                     } else {
-                        tma_load_2d_pair(b_dst, &map_b, bar, n0, k0);
-                        tma_load_2d_pair(b_dst + MN_BOX_BYTES, &map_b, bar, n0 + 64, k0);
+                        tma_load_tile_pair<BPB>(b_dst, &map_b, bar, n0, k0, z);
+                        tma_load_tile_pair<BPB>(b_dst + MN_BOX_BYTES, &map_b, bar, n0 + 64, k0, z);
                     }
                     ++issued;
                     if (++stage == P_STAGES) {
@@ -416,7 +434,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             uint32_t phase = 0, nconsumed = 0;
             int it = 0;
             for (int u = pair_id; u < units && !*abort_flag; u += n_pairs, ++it) {
-                const int kb_lo = (u % splits) * kper, kb_hi = min(kblocks, kb_lo + kper);
+                const int kb_lo = (u % splits) * kper, kb_hi = min(kblocks, kb_lo + kper);  // (units per batch % splits == 0)
                 const int acc = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, kErrTimeoutEpilogue)) {
@@ -463,7 +481,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int quarter = warp & 3;
         int it = 0;
         for (int u = pair_id; u < units; u += n_pairs, ++it) {
-            const int tile = u / splits;
+            const int z = u / (tiles * splits);
+            const int tile = (u % (tiles * splits)) / splits;
+            void* const zout = (BPA | BPB) != 0 ? static_cast<void*>(static_cast<uint8_t*>(out) +
+                                                             (size_t)z * (size_t)out_bstride * (OUT == kOutBF16 ? 2 : 4))
+                                        : out;
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             const int m0 = (tile / n_tiles) * P_BM + (int)rank * P_CM, n0 = (tile % n_tiles) * P_BN;
@@ -480,7 +502,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * P_BN + ch * 32, r);
                 tc_wait_ld();
-                epilogue_store_row32<OUT>(out, row, col0, M, N, ldo, r);
+                epilogue_store_row32<OUT>(zout, row, col0, M, N, ldo, r);
             }
             tc_fence_before_sync();
             __syncwarp();

@@ -10,8 +10,9 @@ every timed call) of:
     (14 B and 24 B per element, bf16 U and dU; padded positions excluded);
   - where the forward scan applies (v = 0), both forced paths;
   - for bf16-projection workloads, sru_project, sru_project_backward (dX and
-    dW separately) and sru_project_factored (d' = d/4) in TFLOP/s, beside
-    torch.matmul (cuBLAS) on the same product.
+    dW separately), sru_project_factored (d' = d/4) and, for unidirectional
+    layers, SRU++'s attention producer sru_attention_project (d' = d/4,
+    causal) in TFLOP/s, beside torch.matmul (cuBLAS) on the same product.
 Inputs come from the seeded generator; nothing here checks numerics (the
 tests do).
 """
@@ -112,6 +113,15 @@ def time_workload(name: str) -> dict:
         t_f = _timeit(lambda: sru.sru_project_factored(X, Wq, Wo, P, Uo), flush=False)
         t_fb = _timeit(lambda: sru.sru_project_factored_backward(dUo, X, Wq, Wo, P, dP, dX=dX, accumulate=True,
                                                                  dWq=dWq, dWo=dWo), flush=False)
+        t_att = None
+        if nd == 1 and L % 8 == 0:
+            Wkv = (torch.randn(2 * Kp, Kp, device="cuda", generator=g) / Kp ** 0.5).bfloat16()
+            aws = torch.empty(int(sru.load_library().sru_attention_workspace_bytes(L, B, Kp)), dtype=torch.uint8,
+                              device="cuda")
+            t_att = _timeit(lambda: sru.sru_attention_project(X, Wq, Wkv, Wo, Uo, L, B, 0.5, workspace=aws),
+                            flush=False)
+        # attention producer flops: Q, [K|V], U products + per batch row 2 L^2 d' (scores) + 2 L^2 d' (A)
+        afl = 2.0 * M * Kp * (K + 2 * Kp + N) + 4.0 * B * L * L * Kp
         out["gemm"] = {"M": M, "N": N, "K": K,
                        "project_us": t_u * 1e3, "project_TFs": fl / t_u / 1e9,
                        "dX_us": t_dx * 1e3, "dX_TFs": fl / t_dx / 1e9,
@@ -119,6 +129,8 @@ def time_workload(name: str) -> dict:
                        "cublas_project_TFs": fl / t_cu / 1e9,
                        "factored_Kp": Kp, "factored_us": t_f * 1e3, "factored_TFs": ffl / t_f / 1e9,
                        "factored_backward_us": t_fb * 1e3, "factored_backward_TFs": 2 * ffl / t_fb / 1e9}
+        if t_att is not None:
+            out["gemm"].update(attention_us=t_att * 1e3, attention_TFs=afl / t_att / 1e9)
     status = sru.sru_sync_status()
     if status != 0:
         raise RuntimeError(f"device status {status}")
