@@ -445,7 +445,13 @@ int pick_stages(int64_t ctas, const int* resident, int smax) {
     return best;
 }
 
-constexpr int kSeqCJ = sru::kRecCJ;  // channels per CTA of the sequential kernels
+// Channels per CTA of the sequential kernels (CJ/2 threads; at least 32 so
+// that a CTA has a lane for each of a chunk's 16 rows).
+#ifndef SRU_SEQ_CJ
+#define SRU_SEQ_CJ 64
+#endif
+constexpr int kSeqCJ = SRU_SEQ_CJ;
+static_assert(kSeqCJ >= 32 && kSeqCJ % 32 == 0, "sequential tile width");
 
 template <typename UT, int S>
 sru_status launch_fwd_seq_s(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
@@ -783,7 +789,7 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
     } else if (scan) {
         return SRU_ERR_INVALID;  // the scan needs its flags and aggregates
     }
-    const int cj = kSeqCJ;  // the scan kernels use the same 64-channel tiles
+    const int cj = scan ? sru::kRecCJ : kSeqCJ;  // TMA box width of the kernel that runs
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj))
         return SRU_ERR_INVALID;
@@ -830,7 +836,7 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     const WsLayout w = ws_layout(L, B, d, n_dir, flags);
     if (workspace_bytes < w.total) return SRU_ERR_INVALID;
     const bool scan = use_bwd_scan(flags, L, B, d, n_dir, u_t);
-    const int cj = kSeqCJ;
+    const int cj = scan ? sru::kRecCJ : kSeqCJ;
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj) ||
         !map_f32_rows(&mp.dh, dh, L, B * n_dir, d, cj))

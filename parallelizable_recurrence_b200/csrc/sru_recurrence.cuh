@@ -125,12 +125,15 @@ struct PairWord<float> {
     static __device__ __forceinline__ float2 unpack(T w) { return w; }
 };
 
-// Bit i set: row t0+i of this chunk exists (t < L) and is not padded.  Whole warp calls.
+// Bit i set: row t0+i of this chunk exists (t < L) and is not padded.  Every
+// thread of the warp (or of a CTA smaller than a warp) calls.
 __device__ __forceinline__ uint32_t chunk_valid_bits(const uint8_t* __restrict__ mask, int t0, int L, int B,
                                                      int b, int lane) {
     bool ok = lane < kChunkT && t0 + lane < L;
     if (ok && mask != nullptr) ok = mask[(size_t)(t0 + lane) * B + b] == 0;
-    return __ballot_sync(0xffffffffu, ok);
+    // CTAs of fewer than 32 threads (at least kChunkT) vote with their own lanes
+    const unsigned lanes = blockDim.x >= 32 ? 0xffffffffu : ((1u << blockDim.x) - 1u);
+    return __ballot_sync(lanes, ok);
 }
 __device__ __forceinline__ uint32_t chunk_inrange_bits(int t0, int L) {
     const int n = L - t0;
