@@ -264,12 +264,22 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
     if (kGemmPair) {
         auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT>;
         SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
+        // the output as the epilogue's TMA store target: box 32 x 32, swizzled like the staging buffers
+        CUtensorMap mo;
+        {
+            const bool bf = OUT == sru::gemm::kOutBF16;
+            const uint64_t dims[2] = {(uint64_t)C, (uint64_t)R};
+            const uint64_t strides[1] = {(uint64_t)ldo * (bf ? 2 : 4)};
+            const uint32_t box[2] = {32, 32};
+            if (!make_map(&mo, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, dims,
+                          strides, box, bf ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
+                return SRU_ERR_INVALID;
+        }
         const int64_t units =
             ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN) * splits;
         const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
-        kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(ma, mb, out, (int)R, (int)C,
-                                                                                       (int)Kr, (int)ldo, splits, 1,
-                                                                                       0LL);
+        kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
+            ma, mb, mo, out, (int)R, (int)C, (int)Kr, (int)ldo, splits, 1, 0LL);
     } else {
         if (splits != 1) return SRU_ERR_UNSUPPORTED;
         auto kern = sru::gemm::tc_gemm_kernel<A_MN, B_MN, OUT>;
@@ -295,8 +305,10 @@ sru_status launch_tc_gemm_batched(const CUtensorMap& ma, const CUtensorMap& mb, 
         ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN) * batches;
     if (units >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
     const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
+    CUtensorMap unused;  // batched launches store directly (no output map)
+    std::memset(&unused, 0, sizeof(unused));
     kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
-        ma, mb, out, (int)R, (int)C, (int)Kr, (int)ldo, 1, (int)batches, (long long)out_bstride);
+        ma, mb, unused, out, (int)R, (int)C, (int)Kr, (int)ldo, 1, (int)batches, (long long)out_bstride);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }

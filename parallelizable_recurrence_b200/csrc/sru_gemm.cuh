@@ -303,7 +303,41 @@ constexpr uint32_t P_A_BYTES = P_CM * BK * 2;          // 16 KB
 constexpr uint32_t P_B_BYTES = P_CN * BK * 2;          // 16 KB
 constexpr uint32_t P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
 constexpr uint32_t P_TMEM_COLS = 2 * P_BN;             // two 128 x 256 fp32 accumulators per CTA
-constexpr size_t P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024 + 256;
+// Epilogue staging (non-batched launches): each of the 4 epilogue warps owns
+// two 4 KB buffers; a 32 x 32 output chunk is written there in the TMA swizzle
+// pattern and leaves by one TMA store (or TMA reduce-add), so the output goes
+// out as whole lines instead of 16-byte pieces of 32 different rows.
+constexpr uint32_t P_EPI_BUF = 4096;
+constexpr uint32_t P_EPI_BYTES = 4 * 2 * P_EPI_BUF;
+constexpr size_t P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + P_EPI_BYTES + 1024 + 256;
+static_assert(P_SMEM_BYTES <= 232448, "pair GEMM shared memory");
+
+// Write one row's 32 accumulator columns (r, fp32 bits) into a staging buffer
+// laid out as the TMA tensor's 32 x 32 box with its swizzle: fp32 rows of
+// 128 B with 128-byte swizzle (16-byte chunk c of row i at chunk c ^ (i % 8)),
+// bf16 rows of 64 B with 64-byte swizzle (chunk c at c ^ ((i / 2) % 4)).
+// Either way the 32 rows' stores of one chunk fall in distinct banks.
+template <int OUT>
+__device__ __forceinline__ void epilogue_stage_row32(uint32_t buf, int i, const uint32_t (&r)[32]) {
+    if (OUT == kOutBF16) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 two = __floats2bfloat162_rn(__uint_as_float(r[c * 8 + 2 * e]),
+                                                           __uint_as_float(r[c * 8 + 2 * e + 1]));
+                w[e] = *reinterpret_cast<uint32_t*>(&two);
+            }
+            st_shared_v4(buf + (uint32_t)i * 64u + ((uint32_t)(c ^ ((i >> 1) & 3)) << 4), w[0], w[1], w[2], w[3]);
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            st_shared_v4(buf + (uint32_t)i * 128u + ((uint32_t)(c ^ (i & 7)) << 4), r[4 * c], r[4 * c + 1],
+                         r[4 * c + 2], r[4 * c + 3]);
+    }
+}
 
 __host__ __device__ constexpr uint32_t idesc_bf16_pair(bool a_mn, bool b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
@@ -326,14 +360,19 @@ __device__ __forceinline__ void tma_load_tile_pair(void* dst, const CUtensorMap*
         tma_load_3d_pair(dst, map, bar, x, y, z);
 }
 
+// map_out (non-batched launches): the output as a 2-D tensor (N columns, M
+// rows, row stride ldo) of the output type, box 32 x 32, swizzle 64 B (bf16)
+// or 128 B (fp32).  Batched launches store directly and ignore it.
 template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                        void* __restrict__ out, int M, int N, int K, int ldo, int splits, int batches,
-                        long long out_bstride) {
+                        const __grid_constant__ CUtensorMap map_out, void* __restrict__ out, int M, int N, int K,
+                        int ldo, int splits, int batches, long long out_bstride) {
+    constexpr bool kTmaOut = (BPA | BPB) == 0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
+    uint8_t* epi = smem + P_STAGES * P_STAGE_BYTES;  // 1024-aligned staging buffers
+    uint64_t* full = reinterpret_cast<uint64_t*>(epi + P_EPI_BYTES);
     uint64_t* empty = full + P_STAGES;
     uint64_t* tfull = empty + P_STAGES;
     uint64_t* tempty = tfull + 2;
@@ -368,6 +407,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         fence_mbar_init();
         tma_prefetch_desc(&map_a);
         tma_prefetch_desc(&map_b);
+        if (kTmaOut) tma_prefetch_desc(&map_out);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, P_TMEM_COLS);
@@ -480,6 +520,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // ---------------------------------------------------------- epilogue (both CTAs)
         const int quarter = warp & 3;
         int it = 0;
+        uint32_t nstaged = 0;  // chunks this warp has handed to TMA stores
         for (int u = pair_id; u < units; u += n_pairs, ++it) {
             const int z = u / (tiles * splits);
             const int tile = (u % (tiles * splits)) / splits;
@@ -502,12 +543,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * P_BN + ch * 32, r);
                 tc_wait_ld();
-                epilogue_store_row32<OUT>(zout, row, col0, M, N, ldo, r);
+                if (kTmaOut) {
+                    // buffer (nstaged & 1) was last read by the store issued two chunks ago
+                    const uint32_t buf = smem_u32(epi) + (uint32_t)(quarter * 2 + (nstaged & 1)) * P_EPI_BUF;
+                    if (nstaged >= 2) {
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                    }
+                    epilogue_stage_row32<OUT>(buf, lane, r);
+                    fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const void* src = epi + (size_t)(quarter * 2 + (nstaged & 1)) * P_EPI_BUF;
+                        if (OUT == kOutF32Acc || OUT == kOutF32Red)
+                            tma_reduce_add_2d(&map_out, src, col0, m0 + quarter * 32);
+                        else
+                            tma_store_2d(&map_out, src, col0, m0 + quarter * 32);
+                        bulk_commit_group();
+                    }
+                    ++nstaged;
+                } else {
+                    epilogue_store_row32<OUT>(zout, row, col0, M, N, ldo, r);
+                }
             }
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)acc * 8u);
         }
+        if (kTmaOut && lane == 0) bulk_wait_group<0>();  // every store of this warp has landed
     }
     tc_fence_before_sync();
     __syncthreads();
