@@ -393,6 +393,7 @@ sru_status zero_f32(float* p, size_t n, cudaStream_t st) {
 // ------------------------------------------------------- recurrence launch
 struct RecMaps {
     CUtensorMap u, x, dh;
+    CUtensorMap du, dxo;  // backward outputs, for the kernels that store them with TMA
 };
 
 bool map_u_tensor(CUtensorMap* m, const void* U, int u_t, int64_t L, int64_t B, int64_t d, int n_dir, int cj) {
@@ -507,7 +508,7 @@ sru_status launch_bwd_seq_s(const RecMaps& mp, const float* v, const float* b, c
     auto kern = sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR, kSeqCJ, S>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
     dim3 grid((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)B, 1);
-    kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
+    kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.du, mp.dxo, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
                                               (int)L, (int)B, (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
@@ -851,7 +852,8 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     const int cj = scan ? sru::kRecCJ : kSeqCJ;
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj) ||
-        !map_f32_rows(&mp.dh, dh, L, B * n_dir, d, cj))
+        !map_f32_rows(&mp.dh, dh, L, B * n_dir, d, cj) || !map_u_tensor(&mp.du, dU, du_t, L, B, d, n_dir, cj) ||
+        !map_f32_rows(&mp.dxo, dx, L, B, d, cj))
         return SRU_ERR_INVALID;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const float* ckpt = reinterpret_cast<const float*>(ws + w.ckpt_off);

@@ -405,12 +405,17 @@ __device__ __forceinline__ void bwd_chunk_any(const UT* __restrict__ us, const f
 // Fast path of bwd_chunk for a chunk whose 16 rows all exist and are valid:
 // the state chain's operands are copied from shared memory into registers
 // before the chain runs, and no row carries a predicate.
-template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ, typename ACC>
+// STAGE (DUT == UT): dU and dx are not stored to global memory here but
+// written over this thread's own U and x values in the chunk's shared-memory
+// stage (same layout; the values were copied to registers first), for the
+// caller to send out with two TMA stores.
+template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ, typename ACC, bool STAGE = false>
 __device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const float* __restrict__ xs,
                                                const float* __restrict__ dhs,
                                                float2 c, const GateParams2& p, float2 alpha, float2& g,
                                                ACC& acc, DUT* __restrict__ dUp, float* __restrict__ dxp,
                                                size_t u_tstride, size_t x_tstride, int d, bool jok, int cj) {
+    static_assert(!STAGE || sizeof(DUT) == sizeof(UT), "staged dU reuses the U tile");
     using PW = PairWord<UT>;
     typename PW::T wc[kChunkT], wf[kChunkT], wr[kChunkT];
     float2 wx[kChunkT], wdh[kChunkT];
@@ -422,6 +427,7 @@ __device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const 
         wx[i] = load_pair(xs + i * CJ + cj);
         wdh[i] = load_pair(dhs + i * CJ + cj);
     }
+    if (STAGE) asm volatile("" ::: "memory");  // every read of the tile precedes the writes over it
     float2 cp[kChunkT], fs[kChunkT], rs[kChunkT];
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
@@ -450,7 +456,13 @@ __device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const 
         s_vr = fma2(dzr, cpv, s_vr);
         s_bf = add2(s_bf, dzf);
         s_br = add2(s_br, dzr);
-        if (jok) {
+        if (STAGE) {
+            DUT* su = reinterpret_cast<DUT*>(const_cast<UT*>(us));
+            store_pair(su + (i * 3 + 0) * CJ + cj, duc);
+            store_pair(su + (i * 3 + 1) * CJ + cj, dzf);
+            store_pair(su + (i * 3 + 2) * CJ + cj, dzr);
+            store_pair(const_cast<float*>(xs) + i * CJ + cj, dxv);
+        } else if (jok) {
             store_pair(dUp + (size_t)i * u_tstride, duc);
             store_pair(dUp + (size_t)i * u_tstride + d, dzf);
             store_pair(dUp + (size_t)i * u_tstride + 2 * d, dzr);
@@ -526,11 +538,17 @@ struct BwdLayout {
 template <typename UT, typename DUT, bool ACC_DX, int DIR, int CJ, int S>
 __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
-    const __grid_constant__ CUtensorMap map_dh, const float* __restrict__ v, const float* __restrict__ bias,
+    const __grid_constant__ CUtensorMap map_dh, const __grid_constant__ CUtensorMap map_du,
+    const __grid_constant__ CUtensorMap map_dxo, const float* __restrict__ v, const float* __restrict__ bias,
     const uint8_t* __restrict__ mask, const float* __restrict__ ckpt, const float* __restrict__ dc_T, DUT* __restrict__ dU,
     float* __restrict__ dx, double* __restrict__ partial, float* __restrict__ dc0, int L, int B, int d,
     int n_dir, float alpha) {
     using Lay = BwdLayout<UT, ACC_DX, CJ, S>;
+    // Full chunks leave through TMA stores of the stage they came in on (dU over
+    // U, dx over x): a stage is refilled one iteration after its store was
+    // issued, so loads run S - 1 chunks ahead (needs S >= 3 to overlap).
+    constexpr bool kStage = sizeof(UT) == sizeof(DUT) && S >= 3;
+    constexpr int kAhead = kStage ? S - 1 : S;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
@@ -557,6 +575,10 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
         tma_prefetch_desc(&map_u);
         tma_prefetch_desc(&map_x);
         tma_prefetch_desc(&map_dh);
+        if (kStage) {
+            tma_prefetch_desc(&map_du);
+            tma_prefetch_desc(&map_dxo);
+        }
     }
     __syncthreads();
 
@@ -577,7 +599,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
         }
     };
     if (tid < 32)
-        for (int k = 0; k < S && k < nch; ++k) issue(k);
+        for (int k = 0; k < kAhead && k < nch; ++k) issue(k);
 
     SmemPartials acc{reinterpret_cast<double*>(smem + Lay::ACC_OFF) + tid, CJ / 2};
 #pragma unroll
@@ -596,7 +618,10 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     auto wait_stage = [&](int s) {
         const bool ok = mbar_wait(&full[s], (phase_bits >> s) & 1u, kErrTimeoutLoad);
         if (__syncthreads_or(!ok)) {
-            if (tid == 0) drain_pending_loads<S>(full, pending, phase_bits);
+            if (tid == 0) {
+                drain_pending_loads<S>(full, pending, phase_bits);
+                if (kStage) bulk_wait_group<0>();  // stores still reading shared memory
+            }
             return false;
         }
         return true;
@@ -610,6 +635,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
         const float2 ck2 = ckpt_of(k + 2);
         DUT* dUp = dU + (size_t)t0 * u_tstride + (size_t)bd * 3 * d + j;
         float* dxp = dx + (size_t)t0 * x_tstride + (size_t)b * d + j;
+        bool staged = false;
         if (valid == 0u) {
             bwd_chunk_padded<DUT, ACC_DX>(inrange, dUp, dxp, u_tstride, x_tstride, d, jok);
         } else {
@@ -619,14 +645,43 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
             const UT* us = reinterpret_cast<const UT*>(smem + s * Lay::STAGE);
             const float* xs = reinterpret_cast<const float*>(smem + s * Lay::STAGE + Lay::U_BYTES);
             const float* dhs = xs + kChunkT * CJ;
-            bwd_chunk<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, valid, inrange, ck0, p, alpha2, g, acc, dUp, dxp,
-                                                u_tstride, x_tstride, d, jok, cj);
+            if constexpr (kStage) {
+                if (valid == (1u << kChunkT) - 1u) {
+                    bwd_chunk_full<UT, DUT, ACC_DX, DIR, CJ, SmemPartials, true>(us, xs, dhs, ck0, p, alpha2, g, acc,
+                                                                                 dUp, dxp, u_tstride, x_tstride, d,
+                                                                                 jok, cj);
+                    fence_proxy_async_shared();  // the tile's new contents, visible to the TMA unit
+                    staged = true;
+                }
+            }
+            if (!staged)
+                bwd_chunk<UT, DUT, ACC_DX, DIR, CJ>(us, xs, dhs, valid, inrange, ck0, p, alpha2, g, acc, dUp, dxp,
+                                                    u_tstride, x_tstride, d, jok, cj);
         }
         __syncthreads();
-        if (tid < 32 && k + S < nch) issue(k + S);
+        if (kStage && tid == 0) {
+            if (staged) {
+                const uint8_t* st = smem + s * Lay::STAGE;
+                tma_store_4d(&map_du, st, j0, 0, bd, t0);
+                if (ACC_DX)
+                    tma_reduce_add_3d(&map_dxo, st + Lay::U_BYTES, j0, b, t0);
+                else
+                    tma_store_3d(&map_dxo, st + Lay::U_BYTES, j0, b, t0);
+                bulk_commit_group();
+            }
+            // the next load goes to the stage chunk k-1 used: its store must be done reading it
+            if (k + kAhead < nch) {
+                if (staged)
+                    bulk_wait_group_read<1>();
+                else
+                    bulk_wait_group_read<0>();
+            }
+        }
+        if (tid < 32 && k + kAhead < nch) issue(k + kAhead);
         ck0 = ck1;
         ck1 = ck2;
     }
+    if (kStage && tid == 0) bulk_wait_group<0>();  // every store has landed
     if (jok) {
         store_pair(dc0 + (size_t)bd * d + j, g);
         store_partials(partial + (size_t)bd * 4 * d + j, acc, d);
