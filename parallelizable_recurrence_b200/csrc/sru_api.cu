@@ -394,6 +394,7 @@ sru_status zero_f32(float* p, size_t n, cudaStream_t st) {
 struct RecMaps {
     CUtensorMap u, x, dh;
     CUtensorMap du, dxo;  // backward outputs, for the kernels that store them with TMA
+    CUtensorMap h;        // forward output, likewise
 };
 
 bool map_u_tensor(CUtensorMap* m, const void* U, int u_t, int64_t L, int64_t B, int64_t d, int n_dir, int cj) {
@@ -466,16 +467,16 @@ int pick_stages(int64_t ctas, const int* resident, int smax) {
 constexpr int kSeqCJ = SRU_SEQ_CJ;
 static_assert(kSeqCJ >= 32 && kSeqCJ % 32 == 0, "sequential tile width");
 
-template <typename UT, int S>
+template <typename UT, int S, bool STAGE_H = false>
 sru_status launch_fwd_seq_s(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
                             float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d, int n_dir,
                             float alpha, cudaStream_t st) {
     using Lay = sru::FwdLayout<UT, kSeqCJ, S>;
-    auto kern = sru::sru_fwd_seq_kernel<UT, kSeqCJ, S>;
+    auto kern = sru::sru_fwd_seq_kernel<UT, kSeqCJ, S, STAGE_H>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
     dim3 grid((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)B, (unsigned)n_dir);
-    kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, v, b, c0, mask, h, c_T, ckpt, (int)L, (int)B, (int)d,
-                                              n_dir, alpha);
+    kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.h, v, b, c0, mask, h, c_T, ckpt, (int)L, (int)B,
+                                              (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
@@ -493,7 +494,12 @@ sru_status launch_fwd_seq(const RecMaps& mp, const float* v, const float* b, con
     static_assert(sru::kFwdStages == 4, "stage dispatch below covers 2..4");
     const int resident[5] = {0, 0, fwd_resident<UT, 2>(), fwd_resident<UT, 3>(), fwd_resident<UT, 4>()};
     const int64_t ctas = ((d + kSeqCJ - 1) / kSeqCJ) * B * n_dir;
-    switch (pick_stages(ctas, resident, 4)) {
+    const int S = pick_stages(ctas, resident, 4);
+    // h through TMA stores: for unmasked grids of about 5 or more CTAs per SM (measured)
+    if (S >= 3 && mask == nullptr && ctas * 10 >= (int64_t)sm_count() * 48)
+        return S == 3 ? launch_fwd_seq_s<UT, 3, true>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st)
+                      : launch_fwd_seq_s<UT, 4, true>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+    switch (S) {
         case 2: return launch_fwd_seq_s<UT, 2>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
         case 3: return launch_fwd_seq_s<UT, 3>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
         default: return launch_fwd_seq_s<UT, 4>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
@@ -804,7 +810,8 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
     }
     const int cj = scan ? sru::kRecCJ : kSeqCJ;  // TMA box width of the kernel that runs
     RecMaps mp;
-    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj))
+    if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj) ||
+        !map_f32_rows(&mp.h, h, L, B * n_dir, d, cj))
         return SRU_ERR_INVALID;
     float* ckpt = workspace ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.ckpt_off) : nullptr;
     if (scan) {

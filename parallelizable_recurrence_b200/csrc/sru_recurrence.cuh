@@ -160,7 +160,10 @@ __device__ __forceinline__ void drain_pending_loads(uint64_t* full, uint32_t pen
 // only, and the outputs are stored last.  With about one warp per SM
 // sub-partition the serial chain of a step (two MUFU round trips) must not
 // also wait on shared-memory loads or store addressing.
-template <typename UT, int CJ, int DIR>
+// STAGE: h is written over this thread's own x values in the chunk's
+// shared-memory stage (copied to registers first) for the caller to store
+// with TMA, instead of to global memory.
+template <typename UT, int CJ, int DIR, bool STAGE = false>
 __device__ __forceinline__ float2 fwd_chunk_full(const UT* __restrict__ us, const float* __restrict__ xs, float2 c,
                                                  const GateParams2& p, float2 alpha, float* __restrict__ hp,
                                                  size_t h_tstride, bool jok, int cj) {
@@ -183,22 +186,27 @@ __device__ __forceinline__ float2 fwd_chunk_full(const UT* __restrict__ us, cons
         const float2 ax = mul2(alpha, wx[i]);
         hv[i] = fma2(r, sub2(c, ax), ax);  // Eq. (5)
     }
-    if (jok) {
+    if (STAGE) {
+        asm volatile("" ::: "memory");  // the x reads above precede the writes over them
+#pragma unroll
+        for (int i = 0; i < kChunkT; ++i) store_pair(const_cast<float*>(xs) + i * CJ + cj, hv[i]);
+    } else if (jok) {
 #pragma unroll
         for (int i = 0; i < kChunkT; ++i) store_pair(hp + (size_t)i * h_tstride, hv[i]);
     }
     return c;
 }
 
-template <typename UT, int CJ = kRecCJ>
+template <typename UT, int CJ = kRecCJ, bool STAGE = false>
 __device__ __forceinline__ float2 fwd_chunk(const UT* __restrict__ us, const float* __restrict__ xs,
                                             uint32_t valid, uint32_t inrange, float2 c, const GateParams2& p,
                                             float2 alpha, int dir, float* __restrict__ hp, size_t h_tstride,
                                             bool jok, int cj) {
     constexpr uint32_t kFull = (1u << kChunkT) - 1u;
+    // (with STAGE, only full chunks come here)
     if (valid == kFull)
-        return dir == 0 ? fwd_chunk_full<UT, CJ, 0>(us, xs, c, p, alpha, hp, h_tstride, jok, cj)
-                        : fwd_chunk_full<UT, CJ, 1>(us, xs, c, p, alpha, hp, h_tstride, jok, cj);
+        return dir == 0 ? fwd_chunk_full<UT, CJ, 0, STAGE>(us, xs, c, p, alpha, hp, h_tstride, jok, cj)
+                        : fwd_chunk_full<UT, CJ, 1, STAGE>(us, xs, c, p, alpha, hp, h_tstride, jok, cj);
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
         const int i = dir == 0 ? q : kChunkT - 1 - q;
@@ -228,13 +236,21 @@ struct FwdLayout {
 // Forward.  Grid (ceil(d/CJ), B, n_dir), CJ/2 threads (CJ/64 warps) per CTA.
 //   map_u: 4-D (d, 3, B*n_dir, L) of UT, box (CJ, 3, 1, T)
 //   map_x: 3-D (d, B, L) fp32, box (CJ, 1, T)
-template <typename UT, int CJ, int S>
+template <typename UT, int CJ, int S, bool STAGE_H = false>
 __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
-    const float* __restrict__ v, const float* __restrict__ bias, const float* __restrict__ c0,
-    const uint8_t* __restrict__ mask, float* __restrict__ h, float* __restrict__ c_T, float* __restrict__ ckpt,
-    int L, int B, int d, int n_dir, float alpha) {
+    const __grid_constant__ CUtensorMap map_h, const float* __restrict__ v, const float* __restrict__ bias,
+    const float* __restrict__ c0, const uint8_t* __restrict__ mask, float* __restrict__ h, float* __restrict__ c_T,
+    float* __restrict__ ckpt, int L, int B, int d, int n_dir, float alpha) {
     using Lay = FwdLayout<UT, CJ, S>;
+    // STAGE_H: full chunks leave through a TMA store of h written over the
+    // stage's x tile; a stage is refilled one iteration after its store was
+    // issued, so loads run S - 1 chunks ahead (rings of 3 or more stages).
+    // Measured on B200 it pays only where the per-thread h stores throttle a
+    // dense grid (L1024 B16 d3072: 138 -> 128 us) and costs elsewhere
+    // (L1024 B16 d2048: 94 -> 105 us), so the host chooses per launch.
+    constexpr bool kStage = STAGE_H && S >= 3;
+    constexpr int kAhead = kStage ? S - 1 : S;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
@@ -259,6 +275,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
         fence_mbar_init();
         tma_prefetch_desc(&map_u);
         tma_prefetch_desc(&map_x);
+        if (kStage) tma_prefetch_desc(&map_h);
     }
     __syncthreads();
 
@@ -278,7 +295,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
         }
     };
     if (tid < 32)
-        for (int k = 0; k < S && k < nch; ++k) issue(k);
+        for (int k = 0; k < kAhead && k < nch; ++k) issue(k);
 
     uint32_t phase_bits = 0;
     const size_t h_tstride = (size_t)B * n_dir * d;
@@ -291,7 +308,10 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
         if (valid != 0u) {
             const bool ok = mbar_wait(&full[s], (phase_bits >> s) & 1u, kErrTimeoutLoad);
             if (__syncthreads_or(!ok)) {  // a load never landed: give up (error recorded)
-                if (tid == 0) drain_pending_loads<S>(full, pending, phase_bits);
+                if (tid == 0) {
+                    drain_pending_loads<S>(full, pending, phase_bits);
+                    if (kStage) bulk_wait_group<0>();  // stores still reading shared memory
+                }
                 return;
             }
             phase_bits ^= 1u << s;
@@ -300,10 +320,30 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
         const UT* us = reinterpret_cast<const UT*>(smem + s * Lay::STAGE);
         const float* xs = reinterpret_cast<const float*>(smem + s * Lay::STAGE + Lay::U_BYTES);
         float* hp = h + (size_t)t0 * h_tstride + (size_t)bd * d + j;
-        c = fwd_chunk<UT, CJ>(us, xs, valid, inrange, c, p, alpha2, dir, hp, h_tstride, jok, cj);
+        const bool staged = kStage && valid == (1u << kChunkT) - 1u;
+        if (staged) {
+            c = fwd_chunk<UT, CJ, true>(us, xs, valid, inrange, c, p, alpha2, dir, hp, h_tstride, jok, cj);
+            fence_proxy_async_shared();  // h over the x tile, visible to the TMA unit
+        } else {
+            c = fwd_chunk<UT, CJ>(us, xs, valid, inrange, c, p, alpha2, dir, hp, h_tstride, jok, cj);
+        }
         __syncthreads();  // every thread is done with stage s
-        if (tid < 32 && k + S < nch) issue(k + S);
+        if (kStage && tid == 0) {
+            if (staged) {
+                tma_store_3d(&map_h, smem + s * Lay::STAGE + Lay::U_BYTES, j0, bd, t0);
+                bulk_commit_group();
+            }
+            // the next load goes to the stage chunk k-1 used: its store must be done reading it
+            if (k + kAhead < nch) {
+                if (staged)
+                    bulk_wait_group_read<1>();
+                else
+                    bulk_wait_group_read<0>();
+            }
+        }
+        if (tid < 32 && k + kAhead < nch) issue(k + kAhead);
     }
+    if (kStage && tid == 0) bulk_wait_group<0>();  // every store has landed
     if (jok) store_pair(c_T + (size_t)bd * d + j, c);
 }
 
