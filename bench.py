@@ -367,7 +367,7 @@ def run_ours(args):
         gemm_flops = 2.0 * M * N * K
         # DRAM read + write per launch from the ncu capture summarised in
         # profiles/launches_lm_train_step.md (same kernels, this workload)
-        gemm_traffic = {"project": 263.0e6, "project_dX": 536.6e6, "project_dW": 457.1e6}
+        gemm_traffic = {"project": 266.2e6, "project_dX": 535.9e6, "project_dW": 457.2e6}
         gemm_ms = {n: phase_ms[n] for n in ("project", "project_dX", "project_dW")}
         dom = max(gemm_ms, key=gemm_ms.get)
         peak_tc = peaks["bf16_tflops_sustained"]
@@ -391,7 +391,7 @@ def run_ours(args):
                 "forward": {"achieved": ach_f, "frac": ach_f / peaks["hbm_gbs"], "bytes": fwd_bytes,
                             "ms": phase_ms["forward"], "traffic": 446.4e6},
                 "backward": {"achieved": ach_b, "frac": ach_b / peaks["hbm_gbs"], "bytes": bwd_bytes,
-                             "ms": phase_ms["backward"], "traffic": 768.5e6},
+                             "ms": phase_ms["backward"], "traffic": 771.2e6},
                 "traffic_source": "ncu dram read+write per launch, profiles/launches_lm_train_step.md",
                 "frac_of_nominal_8TBs": {"forward": ach_f / 8000.0, "backward": ach_b / 8000.0}},
             "phase_ms": phase_ms,
