@@ -14,7 +14,9 @@
 //   warp 1        TMEM allocator and MMA issuer (one elected lane)
 //   warps 2..5    epilogue, one TMEM lane quarter each
 // Two 128 x 256 fp32 accumulators (512 TMEM columns) let the epilogue of tile
-// i overlap the main loop of tile i+1.
+// i overlap the main loop of tile i+1.  (tc_gemm_kernel is the single-SM
+// variant kept for comparison builds; the default is tc_gemm_pair_kernel
+// below, whose epilogue stores through shared memory with TMA.)
 //
 // Operand majorness (which index is contiguous in global memory):
 //   U  = X  W^T : A = X  (M x K, K-major), B = W (N x K, K-major)

@@ -13,7 +13,9 @@
 // kChunkT consecutive steps are brought into shared memory by TMA
 // (cp.async.bulk.tensor) through an S-stage mbarrier ring, so (S-1)*kChunkT
 // steps of input are in flight while kChunkT steps are computed.  Outputs are
-// written with coalesced 8-byte (fp32 pair) / 4-byte (bf16 pair) stores.
+// written with coalesced 8-byte (fp32 pair) / 4-byte (bf16 pair) stores, or,
+// for full chunks where it pays, over the chunk's input tile in shared memory
+// and out by TMA stores (see the kernels).
 //
 // The backward re-runs the forward over one chunk from the state checkpoint
 // the forward stored at the chunk start (keeping c, f and r of the chunk in
