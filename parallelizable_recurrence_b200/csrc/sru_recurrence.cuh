@@ -5,7 +5,7 @@
 // channel j) stream is independent; each is walked sequentially over t with
 // its state c in a register.
 //
-// Layout of the work: a CTA owns CJ (64, 128 or 256) consecutive channels of
+// Layout of the work: a CTA owns CJ (64; a build knob allows 32) consecutive channels of
 // one (b, direction), CJ/2 threads; each thread owns two adjacent channels and
 // advances both with the packed fp32x2 instructions of sm_100 (__ffma2_rn,
 // __fadd2_rn, __fmul2_rn), so the two independent recurrences interleave and
