@@ -538,8 +538,11 @@ def run_reference(args):
     cfg, config = workload_config()
     per_step = []
     desc = ""
+    budget = args.ref_step_budget
+    if budget is None:
+        budget = min(2.0, 150.0 / max(1, args.warmup + args.steps))
     for k in range(args.warmup + args.steps):
-        tps, desc, full = cpu_baseline(cfg, budget_s=args.ref_step_budget, seed=k)
+        tps, desc, full = cpu_baseline(cfg, budget_s=budget, seed=k)
         if k >= args.warmup:
             per_step.append(full)
     full_s = statistics.mean(per_step)
@@ -562,7 +565,9 @@ def main():
     ap.add_argument("--workload", choices=["train", "decode"], default="train",
                     help="train: the layer training step (the headline); decode: batch-1 token steps")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--ref-step-budget", type=float, default=2.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--ref-step-budget", type=float, default=None,
+                    help="seconds of oracle work per reference step (default: 2 s, less so that the whole "
+                         "--impl reference run stays near 150 s)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
