@@ -116,6 +116,30 @@ def test_mask_equals_truncated_rows_on_gpu(sru):
         np.testing.assert_array_equal(full["dc0"][bb], part["dc0"][0])
 
 
+def test_reverse_direction_equals_forward_on_flipped_input(sru):
+    """Direction 1 walks t = L-1 .. 0: given direction 0's inputs mirrored in
+    time (its U block, dh, and a palindromic x, which both directions read),
+    and the same v, b and c0, it produces direction 0's outputs mirrored in
+    time.  L is a multiple of the 16-step chunk, so the two walks perform the
+    same operations in mirrored order."""
+    L, B, d = 64, 3, 200
+    cfg = _cfg(L=L, B=B, d=d, n_dir=2, masked=False)
+    inp = generate(cfg, u_direct=True)
+    inp["U"][:, :, 1] = inp["U"][::-1, :, 0]
+    x = inp["x"]
+    inp["x"] = np.ascontiguousarray(np.concatenate([x[: L // 2], x[: L // 2][::-1]]))  # x[t] == x[L-1-t]
+    inp["dh"][:, :, 1] = inp["dh"][::-1, :, 0]
+    inp["v"][1], inp["bias"][1] = inp["v"][0], inp["bias"][0]
+    inp["c0"][:, 1] = inp["c0"][:, 0]
+    gpu = tl.run_gpu_recurrence(sru, inp, 2, 0.75)
+    np.testing.assert_array_equal(gpu["h"][:, :, 1], gpu["h"][::-1, :, 0])
+    np.testing.assert_array_equal(gpu["cT"][:, 1], gpu["cT"][:, 0])
+    np.testing.assert_array_equal(gpu["dU"][:, :, 1], gpu["dU"][::-1, :, 0])
+    np.testing.assert_array_equal(gpu["dc0"][:, 1], gpu["dc0"][:, 0])
+    np.testing.assert_array_equal(gpu["dv"][1], gpu["dv"][0])
+    np.testing.assert_array_equal(gpu["db"][1], gpu["db"][0])
+
+
 def test_invalid_arguments_are_rejected(sru):
     x = torch.zeros(4, 2, 12, device="cuda")  # d = 12 is not a multiple of 8
     U = torch.zeros(4, 2, 1, 3, 12, device="cuda")
