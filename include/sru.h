@@ -257,10 +257,18 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
  * Each W element is read once per call (the step streams 6*d*d bytes of W for
  * any B <= 16; larger B is processed 16 rows at a time).  Same pointer rules as
  * above; X_t, W, x_t, c and h_t must not overlap.  B = 0 is a no-op.
+ * workspace / workspace_bytes (nullable): see sru_decode_workspace_bytes; with
+ * one, batches of 8, 16, 24, ... rows take the tensor-core path.
  * Limits: d % 8 == 0, d <= 2^24, B <= 2^20, else SRU_ERR_UNSUPPORTED.
  */
 sru_status sru_decode_step(const void* X_t, const void* W, const float* x_t, const float* v, const float* b,
-                           float* c, float* h_t, int64_t B, int64_t d, float alpha, void* stream);
+                           float* c, float* h_t, int64_t B, int64_t d, float alpha, void* workspace,
+                           size_t workspace_bytes, void* stream);
+/* Bytes of workspace with which sru_decode_step runs a batched step's product
+ * on the tensor cores (u = W_cat X_t^T as 3d x B fp32, then the cell update):
+ * nonzero when B is a multiple of 8, at least 8.  With workspace NULL (or any
+ * other B) the step runs the fused kernel above. */
+size_t sru_decode_workspace_bytes(int64_t B, int64_t d);
 
 /* Synchronise `stream`, then read and clear the device error word of the
  * current device: SRU_ERR_TIMEOUT if a bounded wait expired since the last

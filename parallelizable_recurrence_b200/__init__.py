@@ -33,7 +33,7 @@ SRU_FLAG_TEST_WITHHOLD_CARRY = 0x8
 EXPORTED = ("sru_status_string", "sru_get_last_cuda_error", "sru_version", "sru_workspace_bytes",
             "sru_project", "sru_project_backward", "sru_forward", "sru_backward", "sru_forward_scan_noalloc",
             "sru_project_factored", "sru_project_factored_backward", "sru_attention_workspace_bytes",
-            "sru_attention_project", "sru_decode_step", "sru_sync_status")
+            "sru_attention_project", "sru_decode_workspace_bytes", "sru_decode_step", "sru_sync_status")
 
 
 class SRUError(RuntimeError):
@@ -92,7 +92,9 @@ def load_library(path: str = LIB_PATH):
     lib.sru_attention_project.argtypes = [_vp, _vp, _vp, _vp, _f32, _vp, _vp, _int, _vp, _int, _i64, _i64, _i64,
                                           _i64, _i64, _vp, ctypes.c_size_t, _vp]
     lib.sru_decode_step.restype = _int
-    lib.sru_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _vp]
+    lib.sru_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _vp, ctypes.c_size_t, _vp]
+    lib.sru_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.sru_decode_workspace_bytes.argtypes = [_i64, _i64]
     lib.sru_sync_status.restype = _int
     lib.sru_sync_status.argtypes = [_vp]
     _lib = lib
@@ -270,18 +272,25 @@ def sru_attention_project(X, Wq, Wkv, Wo, U, L: int, B: int, alpha: float, ln_ga
     return U
 
 
-def sru_decode_step(X_t, W, x_t, v, b, c, h_t, alpha: float = 1.0, stream=None):
-    """One inference step of a unidirectional layer with the projection fused:
-    u = X_t W^T (fp32, never stored), then Eqs. (2)-(5).  X_t (B, d) bf16,
-    W (3d, d) bf16, x_t (B, d) fp32, v and b (2, d) fp32 (a (1, 2, d) slice is
-    fine), c (B, d) fp32 state updated in place, h_t (B, d) fp32 output."""
+def sru_decode_step(X_t, W, x_t, v, b, c, h_t, alpha: float = 1.0, workspace=None, stream=None):
+    """One inference step of a unidirectional layer: u = X_t W^T (fp32), then
+    Eqs. (2)-(5).  X_t (B, d) bf16, W (3d, d) bf16, x_t (B, d) fp32, v and b
+    (2, d) fp32 (a (1, 2, d) slice is fine), c (B, d) fp32 state updated in
+    place, h_t (B, d) fp32 output.  One fused kernel, except for batches of
+    8, 16, 24, ... rows, whose product runs on the tensor cores in a workspace
+    of sru_decode_workspace_bytes bytes (allocated when none is given)."""
     lib = load_library()
     B, d = X_t.shape
     if W.shape[0] != 3 * d or W.shape[1] != d:
         raise ValueError("W must be (3*d, d)")
+    if workspace is None:
+        n = int(lib.sru_decode_workspace_bytes(B, d))
+        if n:
+            workspace = torch.empty(n, dtype=torch.uint8, device=X_t.device)
     _check(lib.sru_decode_step(_ptr(X_t, torch.bfloat16), _ptr(W, torch.bfloat16), _ptr(x_t, torch.float32),
                                _ptr(v, torch.float32), _ptr(b, torch.float32), _ptr(c, torch.float32),
-                               _ptr(h_t, torch.float32), B, d, float(alpha), _stream(stream)),
+                               _ptr(h_t, torch.float32), B, d, float(alpha), _ptr(workspace), _nbytes(workspace),
+                               _stream(stream)),
            "sru_decode_step")
     return h_t, c
 

@@ -1069,8 +1069,22 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
     return sru_project(R, SRU_BF16, Wo, SRU_BF16, U, u_t, M, N, dp, stream);
 }
 
+// Batch rows from which the step's product runs on the tensor cores (measured:
+// the fused CUDA-core kernel's registers per channel grow with B).
+constexpr int64_t kDecodeTensorMinB = 8;
+
+// (B a multiple of 8: u's rows, B floats each, are a tensor-core output whose
+// row pitch must be a multiple of 16 bytes)
+bool decode_tensor_path(int64_t B) { return B >= kDecodeTensorMinB && B % 8 == 0; }
+
+size_t sru_decode_workspace_bytes(int64_t B, int64_t d) {
+    if (!decode_tensor_path(B) || d < 1) return 0;
+    return round256((size_t)3 * d * B * sizeof(float));
+}
+
 sru_status sru_decode_step(const void* X_t, const void* W, const float* x_t, const float* v, const float* b,
-                           float* c, float* h_t, int64_t B, int64_t d, float alpha, void* stream) {
+                           float* c, float* h_t, int64_t B, int64_t d, float alpha, void* workspace,
+                           size_t workspace_bytes, void* stream) {
     if (B < 0 || d < 1) return SRU_ERR_INVALID;
     if (d % 8 != 0) return SRU_ERR_UNSUPPORTED;
     if (B == 0) return SRU_OK;
@@ -1078,6 +1092,19 @@ sru_status sru_decode_step(const void* X_t, const void* W, const float* x_t, con
     if (!aligned16(X_t) || !aligned16(W) || !aligned16(x_t) || !aligned16(c) || !aligned16(h_t))
         return SRU_ERR_INVALID;
     if (d > ((int64_t)1 << 24) || B > ((int64_t)1 << 20)) return SRU_ERR_UNSUPPORTED;
+    if (workspace != nullptr && decode_tensor_path(B)) {
+        // u = W_cat X_t^T (3d x B) on the tensor cores, then the cell update
+        if (!aligned16(workspace) || workspace_bytes < sru_decode_workspace_bytes(B, d)) return SRU_ERR_INVALID;
+        if (3 * d >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
+        float* u = static_cast<float*>(workspace);
+        sru_status s = sru_project(W, SRU_BF16, X_t, SRU_BF16, u, SRU_F32, 3 * d, B, d, stream);
+        if (s != SRU_OK) return s;
+        const size_t n = (size_t)B * d;
+        sru::sru_decode_cell_kernel<<<blocks_for(n, 256), 256, 0, as_stream(stream)>>>(u, x_t, v, b, c, h_t, (int)B,
+                                                                                        (int)d, alpha);
+        SRU_CUDA_TRY(cudaGetLastError());
+        return SRU_OK;
+    }
     const int nb = decode_rows_per_pass(B);
     if ((B + nb - 1) / nb > 65535) return SRU_ERR_UNSUPPORTED;
     cudaStream_t st = as_stream(stream);

@@ -123,4 +123,24 @@ __global__ void __launch_bounds__(kDecThreads) sru_decode_step_kernel(
     }
 }
 
+// Batched decoding (B rows per step): u = W_cat X_t^T has been computed on the
+// tensor cores into u (3d x B fp32, row g*d + j, column b); this applies
+// Eqs. (2)-(5) to every (b, j) with the same operations as sru_cell1.
+// One thread per (j, b), b fastest (consecutive threads read consecutive u).
+__global__ void __launch_bounds__(256) sru_decode_cell_kernel(const float* __restrict__ u,
+                                                              const float* __restrict__ x,
+                                                              const float* __restrict__ v,
+                                                              const float* __restrict__ bias,
+                                                              float* __restrict__ c, float* __restrict__ h, int B,
+                                                              int d, float alpha) {
+    const size_t i = (size_t)blockIdx.x * 256 + threadIdx.x;
+    if (i >= (size_t)B * d) return;
+    const int b = (int)(i % B), j = (int)(i / B);
+    const float uc = u[(size_t)j * B + b], uf = u[((size_t)d + j) * B + b], ur = u[((size_t)2 * d + j) * B + b];
+    const size_t e = (size_t)b * d + j;
+    float hv;
+    c[e] = sru_cell1(c[e], uc, uf, ur, v[j], v[d + j], bias[j], bias[d + j], __fmul_rn(alpha, x[e]), hv);
+    h[e] = hv;
+}
+
 }  // namespace sru

@@ -108,9 +108,15 @@ def test_decode_step_checks_arguments_before_any_launch(lib):
     vp = ctypes.c_void_p
     fake = vp(0x1000)
     args = [fake] * 7
-    assert lib.sru_decode_step(*args, 0, 64, 1.0, None) == 0          # B = 0: nothing to do
-    assert lib.sru_decode_step(*args, 2, 12, 1.0, None) == 4          # d % 8 != 0
-    assert lib.sru_decode_step(*args, -1, 64, 1.0, None) == 1         # negative B
-    assert lib.sru_decode_step(None, *args[1:], 2, 64, 1.0, None) == 1  # null X_t
-    assert lib.sru_decode_step(vp(0x1008), *args[1:], 2, 64, 1.0, None) == 1  # misaligned X_t
-    assert lib.sru_decode_step(*args, 1, 1 << 25, 1.0, None) == 4     # d beyond the size limit
+    assert lib.sru_decode_step(*args, 0, 64, 1.0, None, 0, None) == 0          # B = 0: nothing to do
+    assert lib.sru_decode_step(*args, 2, 12, 1.0, None, 0, None) == 4          # d % 8 != 0
+    assert lib.sru_decode_step(*args, -1, 64, 1.0, None, 0, None) == 1         # negative B
+    assert lib.sru_decode_step(None, *args[1:], 2, 64, 1.0, None, 0, None) == 1  # null X_t
+    assert lib.sru_decode_step(vp(0x1008), *args[1:], 2, 64, 1.0, None, 0, None) == 1  # misaligned X_t
+    assert lib.sru_decode_step(*args, 1, 1 << 25, 1.0, None, 0, None) == 4     # d beyond the size limit
+    # the batched tensor-core path: its workspace size, and a short workspace rejected
+    assert lib.sru_decode_workspace_bytes(4, 64) == 0
+    assert lib.sru_decode_workspace_bytes(21, 64) == 0                # not a multiple of 8
+    need = lib.sru_decode_workspace_bytes(16, 64)
+    assert need >= 3 * 64 * 16 * 4
+    assert lib.sru_decode_step(*args, 16, 64, 1.0, fake, need - 256, None) == 1

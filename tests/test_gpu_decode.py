@@ -61,7 +61,9 @@ def _check(name, got, ref, extra):
     assert not bad.any(), f"{name}: {bad.sum()} of {bad.size} beyond tolerance, worst {np.max(err - tol):.3g}"
 
 
-@pytest.mark.parametrize("B,d", [(1, 8), (1, 2048), (3, 136), (16, 512), (21, 264), (2, 4096)])
+# B = 8, 16, 24 take the tensor-core product (a multiple of 8, at least 8); the rest the fused kernel
+@pytest.mark.parametrize("B,d", [(1, 8), (1, 2048), (3, 136), (16, 512), (21, 264), (2, 4096), (8, 2048),
+                                 (24, 1024), (16, 4096)])
 def test_decode_step_matches_oracle(sru, B, d):
     alpha = 1.0 if B != 3 else 0.5
     Xb, Wb, x, v, bias, c = _inputs(B, d, seed=B * 1000 + d)
