@@ -84,3 +84,17 @@ def test_layernorm_single_token_closed_form():
     Rn = (R - R.mean(1, keepdims=True)) / np.sqrt(R.var(1, keepdims=True) + 1e-5) * g + be
     U = oracle.attention_project(X, Wq, Wk, Wv, Wo, 0.4, 1, B, ln_gamma=g, ln_beta=be)
     np.testing.assert_allclose(U, Rn @ Wo.T, rtol=1e-11, atol=1e-12)
+
+
+def test_two_token_softmax_scaled_by_sqrt_dprime():
+    # d = d' = N = 4, Wq = Wk = Wo = I, Wv = 3 I: Q = K = X, V = 3 X; only feature 0 is nonzero.
+    # Token 1's scores are q1.k0 / sqrt(4) and q1.k1 / sqrt(4) (the 1/sqrt(d') matters here).
+    a, b = 0.5, 2.0
+    X = np.zeros((2, 4))
+    X[0, 0], X[1, 0] = a, b                  # B = 1: tokens 0 and 1
+    eye = np.eye(4)
+    U = oracle.attention_project(X, eye, eye, 3 * eye, eye, 1.0, 2, 1)
+    w0, w1 = np.exp(b * a / 2.0), np.exp(b * b / 2.0)
+    a1 = (w0 * 3 * a + w1 * 3 * b) / (w0 + w1)
+    np.testing.assert_allclose(U[:, 0], [a + 3 * a, b + a1], rtol=1e-12)
+    np.testing.assert_array_equal(U[:, 1:], 0.0)
