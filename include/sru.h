@@ -68,7 +68,9 @@ typedef enum { SRU_F32 = 0, SRU_BF16 = 1 } sru_dtype;
  * and sru_forward may run as a chunked associative scan over t.  (sru_backward
  * may use its chunked scan for any v: the state-gradient recurrence is affine.)
  * The library picks a scan when the sequential kernels would leave SMs idle
- * (fewer than two 64-channel CTAs per SM). */
+ * (fewer than two 64-channel CTAs per SM) and the scan's waves of resident
+ * CTAs cost less than the sequence's 16-step chunks (a measured ratio of 12
+ * chunks per wave on B200). */
 #define SRU_FLAG_V_ZERO 0x1u
 /* Force the scan paths (the forward scan only with SRU_FLAG_V_ZERO) / force the
  * sequential paths. */
@@ -132,8 +134,8 @@ sru_status sru_project_backward(const void* dU, const void* X, const void* W, in
  *   SRU_ERR_INVALID if smaller), or NULL for inference only (then no
  *   checkpoints are written, sru_backward cannot follow, and the scan path is
  *   not available).  flags: SRU_FLAG_* above.  With SRU_FLAG_V_ZERO the
- *   library runs the chunked scan when the sequential kernel would leave SMs
- *   idle (fewer than two 64-channel CTAs per SM), or when forced.
+ *   library runs the chunked scan where it pays (see SRU_FLAG_V_ZERO), or
+ *   when forced.
  */
 sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, const float* b,
                        const float* c0, const uint8_t* mask, int64_t L, int64_t B, int64_t d,
