@@ -12,7 +12,7 @@ with inputs resident in HBM; `e2e` is the same step through the same C-ABI
 calls with the per-step inputs copied from pinned host memory and the
 gradients copied back inside the timed region.
 
---impl reference times the fp64 CPU oracle (the baseline this build is
+--impl reference times the fp64 CPU oracle (the baseline the library is
 checked against) on the host cores, on a bounded sample per step.
 """
 from __future__ import annotations

@@ -59,7 +59,7 @@ typedef enum {
     SRU_ERR_INVALID = 1,      /* bad pointer, size, alignment or dtype */
     SRU_ERR_CUDA = 2,         /* a CUDA runtime/driver call failed */
     SRU_ERR_TIMEOUT = 3,      /* a bounded device-side wait expired */
-    SRU_ERR_UNSUPPORTED = 4   /* valid request this build does not implement */
+    SRU_ERR_UNSUPPORTED = 4   /* valid request outside the library's limits */
 } sru_status;
 
 typedef enum { SRU_F32 = 0, SRU_BF16 = 1 } sru_dtype;

@@ -694,7 +694,7 @@ const char* sru_status_string(int status) {
         case SRU_ERR_INVALID: return "SRU_ERR_INVALID: bad pointer, size, alignment or dtype";
         case SRU_ERR_CUDA: return "SRU_ERR_CUDA: a CUDA call failed";
         case SRU_ERR_TIMEOUT: return "SRU_ERR_TIMEOUT: a bounded device-side wait expired";
-        case SRU_ERR_UNSUPPORTED: return "SRU_ERR_UNSUPPORTED: request outside this build's limits";
+        case SRU_ERR_UNSUPPORTED: return "SRU_ERR_UNSUPPORTED: request outside the library's limits";
         default: return "unknown sru_status";
     }
 }
