@@ -1,4 +1,4 @@
-"""Benchmark of the SRU layer training step on B200.
+"""Benchmark of the SRU layer on B200.
 
 One step = one pass of the whole hot path over one batch: the projection
 U = X W_cat^T (tcgen05 GEMM), the forward recurrence, the backward recurrence
@@ -9,11 +9,18 @@ B = 16 tokens-per-step rows, d = 2048, bf16 projection and fp32 recurrence
 
 Prints ONE JSON line (rank 0).  `value` is device-timed throughput (tokens/s)
 with inputs resident in HBM; `e2e` is the same step through the same C-ABI
-calls with the per-step inputs copied from pinned host memory and the
-gradients copied back inside the timed region.
+calls with the per-step inputs copied from pinned host memory and every
+gradient (dx, dW, dv, db, dc0) copied back inside the timed region.
+`workloads` holds device-timed results of every other layer workload (the
+forward-only layer, the bidirectional masked layer, the recurrence-only layer
+with v != 0 and v = 0, and a layer in the chunked scan's regime), each kernel
+against its roofline.  The tensor-core peak is chosen from the clock samples
+taken while the kernels ran: the burst figure when the SM clock stayed within
+5 % of its maximum with no power-cap sample, the sustained one otherwise.
 
 --impl reference times the fp64 CPU oracle (the baseline the library is
-checked against) on the host cores, on a bounded sample per step.
+checked against) on the host cores, on a bounded sample per step, and
+extrapolates to the full step (said so in its line).
 """
 from __future__ import annotations
 
@@ -23,7 +30,6 @@ import os
 import statistics
 import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -44,6 +50,65 @@ def load_peaks():
                     bf16_tflops_sustained=float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
                     source="measured")
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+def tensor_peak(peaks, clocks):
+    """The bf16 peak that applies to kernels run under these sampled clocks:
+    the burst figure (cuBLAS timed alone at full clock) when the median SM clock
+    stayed within 5 % of its maximum and no sample saw the power cap, else the
+    sustained figure (a seconds-long loop under the power cap)."""
+    sm, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    burst = (sm is not None and mx and sm >= 0.95 * mx and "sw_power_cap" not in clocks.get("reasons", []))
+    if burst:
+        return "burst", peaks["bf16_tflops"]
+    return "sustained", peaks["bf16_tflops_sustained"]
+
+
+SRC_DIRS = (os.path.join(ROOT, "parallelizable_recurrence_b200", "csrc"), os.path.join(ROOT, "include"))
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+
+
+def library_source_hash() -> str:
+    """sha256 over the library's CUDA/C sources (file names and contents, sorted)."""
+    import hashlib
+    h = hashlib.sha256()
+    for d in SRC_DIRS:
+        for name in sorted(os.listdir(d)):
+            if name.endswith((".cu", ".cuh", ".h")):
+                h.update(name.encode())
+                with open(os.path.join(d, name), "rb") as fh:
+                    h.update(fh.read())
+    return h.hexdigest()
+
+
+def load_traffic():
+    """ncu DRAM bytes (read + write) per launch, keyed by workload and phase, from
+    the capture recorded beside the profiles -- only if that capture was taken of
+    these exact library sources (same hash); otherwise {} and traffic is null."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return {}, "no ncu capture recorded"
+    with open(TRAFFIC_FILE) as fh:
+        rec = json.load(fh)
+    if rec.get("source_hash") != library_source_hash():
+        return {}, "ncu capture was of other library sources (stale): traffic not reported"
+    return rec.get("bytes_per_launch", {}), rec.get("command", "")
+
+
+def host_info():
+    model = None
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
 
 
 def workload_config():
@@ -135,7 +200,8 @@ class ClockSampler:
 def cpu_baseline(cfg, budget_s: float = 10.0, seed: int = 0):
     """Time the fp64 oracle on a bounded sample of the workload on one host core
     and extrapolate to the full step (projection, its two gradients, forward and
-    backward recurrence over every channel).  Returns (tokens/s, description)."""
+    backward recurrence over every channel).  Returns (tokens/s, description,
+    extrapolated seconds per full step, seconds of oracle work measured)."""
     import oracle
     from synthetic import f32_to_bf16_bits
     rng = np.random.default_rng(seed)
@@ -148,7 +214,7 @@ def cpu_baseline(cfg, budget_s: float = 10.0, seed: int = 0):
     v = rng.uniform(-0.5, 0.5, (1, 2, n_ch))
     bias = 0.1 * rng.standard_normal((1, 2, n_ch))
     dh = rng.standard_normal((L, B, 1, n_ch))
-    t0 = time.perf_counter()
+    t_start = t0 = time.perf_counter()
     reps = 0
     while True:
         oracle.forward(U, x, v, bias)
@@ -170,11 +236,211 @@ def cpu_baseline(cfg, budget_s: float = 10.0, seed: int = 0):
         if time.perf_counter() - t0 > budget_s * 0.7:
             break
     t_mac = (time.perf_counter() - t0) / (n_ent * K)                # s per multiply-add
+    measured = time.perf_counter() - t_start
     full = t_rec * B * d * cfg.n_dir + t_mac * 3 * M * N * K
     desc = (f"fp64 oracle, 1 thread: recurrence fwd+bwd on {n_ch} channels x {B} rows x L={L} "
-            f"({reps} reps), projection plain sums {n_ent} entries x K={K}; extrapolated to the full step "
-            f"({B * d * cfg.n_dir} channels, 3 products of {M}x{N}x{K})")
-    return cfg.tokens / full, desc, full
+            f"({reps} reps), projection plain sums {n_ent} entries x K={K}, {measured:.1f} s measured; "
+            f"extrapolated to the full step ({B * d * cfg.n_dir} channels, 3 products of {M}x{N}x{K})")
+    return cfg.tokens / full, desc, full, measured
+
+
+# ------------------------------------------------------ per-workload block
+def _time_ms(fn, flush, reps=10, warm=3):
+    """Median device time (ms) of fn() on torch's current stream, CUDA events,
+    after `warm` untimed calls; `flush` (a buffer larger than L2) is rewritten
+    before every timed call so that no input is served from L2."""
+    import torch
+    st = torch.cuda.current_stream()
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        fn()
+        b.record(st)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return float(statistics.median(ts))
+
+
+def _lengths(L, B, seed):
+    """Sequence lengths of a padded batch: integers uniform on [L/2, L]."""
+    return np.random.default_rng(seed).integers(L // 2, L, size=B, endpoint=True)
+
+
+def _hbm_entry(kernel, ms, nbytes):
+    return {"kernel": kernel, "bound": "hbm", "ms": ms, "algorithmic_bytes": nbytes,
+            "achieved": nbytes / (ms / 1e3) / 1e9, "unit": "GB/s"}
+
+
+def _tc_entry(kernel, ms, flops):
+    return {"kernel": kernel, "bound": "tensor", "ms": ms, "algorithmic_flops": flops,
+            "achieved": flops / (ms / 1e3) / 1e12, "unit": "TFLOP/s"}
+
+
+class _Layer:
+    """Device buffers of one layer workload, drawn on the device from a seeded
+    generator with the workload's distributions (U or X and W, x, v, b, c0, dh,
+    padding lengths)."""
+
+    def __init__(self, L, B, d, nd, seed, dev, masked=False, v_zero=False, project=False, c0=False):
+        import torch
+        import parallelizable_recurrence_b200 as sru
+        self.L, self.B, self.d, self.nd = L, B, d, nd
+        g = torch.Generator(device=dev).manual_seed(seed)
+        self.x = torch.randn(L, B, d, device=dev, generator=g)
+        if project:
+            a = (3.0 / d) ** 0.5
+            self.X = self.x.view(L * B, d).to(torch.bfloat16)
+            self.W = ((torch.rand(nd * 3 * d, d, device=dev, generator=g) * 2 - 1) * a).to(torch.bfloat16)
+        self.U = torch.randn(L, B, nd, 3, d, device=dev, generator=g).to(torch.bfloat16)
+        self.v = torch.zeros(nd, 2, d, device=dev) if v_zero else torch.rand(nd, 2, d, device=dev, generator=g) - 0.5
+        self.b = 0.1 * torch.randn(nd, 2, d, device=dev, generator=g)
+        self.c0 = torch.randn(B, nd, d, device=dev, generator=g) if c0 else None
+        self.dh = torch.randn(L, B, nd, d, device=dev, generator=g)
+        self.mask = None
+        self.valid = 1.0
+        if masked:
+            lengths = _lengths(L, B, seed)
+            m = (np.arange(L)[:, None] >= lengths[None, :]).astype(np.uint8)
+            self.mask = torch.from_numpy(m).to(dev)
+            self.valid = float((m == 0).mean())
+        self.h = torch.empty(L, B, nd, d, device=dev)
+        self.cT = torch.empty(B, nd, d, device=dev)
+        self.dU = torch.empty(L, B, nd, 3, d, device=dev, dtype=torch.bfloat16)
+        self.dx = torch.empty(L, B, d, device=dev)
+        self.dv = torch.empty(nd, 2, d, device=dev)
+        self.db = torch.empty(nd, 2, d, device=dev)
+        self.dc0 = torch.empty(B, nd, d, device=dev)
+        flags = (sru.SRU_FLAG_V_ZERO | sru.SRU_FLAG_FORCE_SCAN) if v_zero else sru.SRU_FLAG_FORCE_SCAN
+        self.ws = sru.alloc_workspace(L, B, d, nd == 2, flags, device=dev)
+
+    @property
+    def elements(self):
+        return self.L * self.B * self.d * self.nd
+
+    def fwd_bytes(self):
+        """U 6 + x 4 + h 4 bytes per valid element; h (zeros) 4 per padded one."""
+        e = self.elements
+        return 14.0 * e * self.valid + 4.0 * e * (1 - self.valid)
+
+    def bwd_bytes(self):
+        """U 6 + x 4 + dh 4 + dU 6 + dx 4 bytes per valid element; per padded one the
+        zero dU (6) and, once per position for both directions, the zero dx (4)."""
+        e = self.elements
+        return 24.0 * e * self.valid + (6.0 + 4.0 / self.nd) * e * (1 - self.valid)
+
+    def forward(self, flags=0):
+        import parallelizable_recurrence_b200 as sru
+        sru.sru_forward(self.U, self.x, self.v, self.b, self.h, self.cT, c0=self.c0, mask=self.mask,
+                        bidirectional=self.nd == 2, flags=flags, workspace=self.ws)
+
+    def backward(self, flags=0):
+        import parallelizable_recurrence_b200 as sru
+        sru.sru_backward(self.U, self.x, self.v, self.b, self.dh, self.ws, self.dU, self.dx, self.dv, self.db,
+                         self.dc0, c0=self.c0, mask=self.mask, bidirectional=self.nd == 2, flags=flags)
+
+
+def _recurrence_entries(lay, flush, variants, tag=""):
+    out = {}
+    for name, fl in variants:
+        tf = _time_ms(lambda: lay.forward(fl), flush)
+        lay.forward(fl)  # the backward reads this variant's checkpoints
+        tb = _time_ms(lambda: lay.backward(fl), flush)
+        out[f"forward{tag}{name}"] = _hbm_entry("sru_forward", tf, lay.fwd_bytes())
+        out[f"backward{tag}{name}"] = _hbm_entry("sru_backward", tb, lay.bwd_bytes())
+    return out
+
+
+def _gemm_entries(lay, flush):
+    import torch
+    import parallelizable_recurrence_b200 as sru
+    M, N, K = lay.L * lay.B, lay.nd * 3 * lay.d, lay.d
+    fl = 2.0 * M * N * K
+    Uv = lay.U.view(M, N)
+    dX = torch.empty(M, K, device=lay.x.device)
+    dW = torch.empty(N, K, device=lay.x.device)
+    dUv = lay.dU.view(M, N).copy_(Uv)
+    t_u = _time_ms(lambda: sru.sru_project(lay.X, lay.W, Uv), flush)
+    t_dx = _time_ms(lambda: sru.sru_project_backward(dUv, lay.X, lay.W, dX=dX, accumulate=True), flush)
+    t_dw = _time_ms(lambda: sru.sru_project_backward(dUv, lay.X, lay.W, dW=dW), flush)
+    return {"project": _tc_entry("sru_project (U = X W^T)", t_u, fl),
+            "project_dX": _tc_entry("sru_project_backward (dX += dU W)", t_dx, fl),
+            "project_dW": _tc_entry("sru_project_backward (dW = dU^T X)", t_dw, fl)}
+
+
+def measure_workloads(dev, peaks):
+    """Device-timed kernels of the other layer workloads, each alone with L2
+    flushed before every timed call (median of 10 after 3 warm-up calls)."""
+    import torch
+    import parallelizable_recurrence_b200 as sru
+    VZ, SCAN, SEQ = sru.SRU_FLAG_V_ZERO, sru.SRU_FLAG_FORCE_SCAN, sru.SRU_FLAG_FORCE_SEQUENTIAL
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    with ClockSampler(dev.index if dev.index is not None else 0, period_s=0.02) as clk:
+        # forward-only language-model layer: L256 B32 d512, bf16 projection
+        lay = _Layer(256, 32, 512, 1, 1, dev, project=True)
+        e = _gemm_entries(lay, flush)
+        e = {"project": e["project"]}
+        t = _time_ms(lambda: lay.forward(0), flush)
+        e["forward"] = _hbm_entry("sru_forward", t, lay.fwd_bytes())
+        t_step = _time_ms(lambda: (sru.sru_project(lay.X, lay.W, lay.U.view(256 * 32, 1536)), lay.forward(0)), flush)
+        e["layer_forward"] = {"ms": t_step, "tokens_per_s": 256 * 32 / (t_step / 1e3),
+                              "calls": "sru_project + sru_forward"}
+        res["lm_fwd L256 B32 d512 forward"] = e
+        del lay
+        torch.cuda.empty_cache()
+        # bidirectional padded layer: L2048 B64 d1024 x 2 directions
+        lay = _Layer(2048, 64, 1024, 2, 3, dev, masked=True, project=True)
+        e = _gemm_entries(lay, flush)
+        e.update(_recurrence_entries(lay, flush, [("", 0)], tag="_masked"))
+        e["valid_fraction"] = lay.valid
+        mask = lay.mask
+        lay.mask, lay.valid = None, 1.0
+        e.update(_recurrence_entries(lay, flush, [("", 0)], tag="_unmasked"))
+        lay.mask = mask
+        res["bidir_masked L2048 B64 d1024 x2"] = e
+        del lay, mask
+        torch.cuda.empty_cache()
+        # recurrence-only layer, U given: L1024 B16 d3072, v != 0, then v = 0
+        lay = _Layer(1024, 16, 3072, 1, 4, dev)
+        res["rec_only L1024 B16 d3072 v!=0"] = _recurrence_entries(lay, flush, [("", 0)])
+        lay.v.zero_()
+        res["rec_only_v0 L1024 B16 d3072 v=0"] = _recurrence_entries(
+            lay, flush, [("_dispatched", VZ), ("_scan_forced", VZ | SCAN), ("_sequential_forced", VZ | SEQ)])
+        del lay
+        torch.cuda.empty_cache()
+        # a layer in the chunked scan's regime (B*d too small to fill the GPU): L2048 B4 d2048, v = 0
+        lay = _Layer(2048, 4, 2048, 1, 5, dev, v_zero=True)
+        res["scan_regime L2048 B4 d2048 v=0"] = _recurrence_entries(
+            lay, flush, [("_dispatched", VZ), ("_sequential_forced", VZ | SEQ)])
+        del lay
+        torch.cuda.empty_cache()
+    clocks = clk.summary()
+    st = sru.sru_sync_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} in the workload block")
+    src, tc_peak = tensor_peak(peaks, clocks)
+    for entries in res.values():
+        for k, ent in entries.items():
+            if not isinstance(ent, dict) or "bound" not in ent:
+                continue
+            if ent["bound"] == "hbm":
+                ent["peak"] = peaks["hbm_gbs"]
+                ent["frac"] = ent["achieved"] / peaks["hbm_gbs"]
+                ent["frac_of_nominal_8TBs"] = ent["achieved"] / NOMINAL_HBM_GBS
+            else:
+                ent["peak"] = tc_peak
+                ent["frac"] = ent["achieved"] / tc_peak
+                ent["frac_of_nominal_2250"] = ent["achieved"] / NOMINAL_BF16_TFLOPS
+    return {"timing": "each kernel alone, median of 10 after 3 warm-up calls, 512 MB written before every "
+                      "timed call (L2 flushed); inputs drawn on the device from seeded generators",
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": tc_peak, "bf16_peak_kind": src,
+                      "source": peaks["source"]},
+            "clocks": clocks, "layers": res}
 
 
 # ------------------------------------------------------------ GPU arm
@@ -228,8 +494,9 @@ def run_ours(args):
         reducer = GradReducer([dW, dv, db])  # one NCCL all-reduce of the parameter gradients
 
     def step(ev=None, bufs=None):
-        """One training step; bufs = (X, x, dh, dW, dv, db, dc0, reducer) or the default set."""
-        Xb, xb, dhb, dWb, dvb, dbb, dc0b, red = bufs if bufs is not None else (X, x, dh, dW, dv, db, dc0, reducer)
+        """One training step; bufs = (X, x, dh, dx, dW, dv, db, dc0, reducer) or the default set."""
+        Xb, xb, dhb, dxb, dWb, dvb, dbb, dc0b, red = (bufs if bufs is not None
+                                                      else (X, x, dh, dx, dW, dv, db, dc0, reducer))
         if ev is not None:
             ev[0].record(stream)
         sru.sru_project(Xb, W, U)
@@ -238,10 +505,10 @@ def run_ours(args):
         sru.sru_forward(U, xb, v, b, h, cT, c0=c0, workspace=ws)
         if ev is not None:
             ev[2].record(stream)
-        sru.sru_backward(U, xb, v, b, dhb, ws, dU, dx, dvb, dbb, dc0b, c0=c0)
+        sru.sru_backward(U, xb, v, b, dhb, ws, dU, dxb, dvb, dbb, dc0b, c0=c0)
         if ev is not None:
             ev[3].record(stream)
-        sru.sru_project_backward(dU, Xb, W, dX=dx, accumulate=True)
+        sru.sru_project_backward(dU, Xb, W, dX=dxb, accumulate=True)
         if ev is not None:
             ev[4].record(stream)
         sru.sru_project_backward(dU, Xb, W, dW=dWb)
@@ -284,7 +551,7 @@ def run_ours(args):
     elapsed_ms = float(t.item())
 
     # ---- end to end: every step copies its inputs (X bf16, x and dh fp32) from
-    # pinned host memory and reads its gradients (dW, dv, db, dc0) back.  The
+    # pinned host memory and reads its gradients (dx, dW, dv, db, dc0) back.  The
     # copies run on their own streams, double-buffered, so step k+1's inputs
     # travel while step k computes and step k's gradients travel back while
     # step k+1 computes (PCIe is full duplex).
@@ -296,6 +563,7 @@ def run_ours(args):
         Xi = X if i == 0 else torch.empty_like(X)
         xi = x if i == 0 else torch.empty_like(x)
         dhi = dh if i == 0 else torch.empty_like(dh)
+        dxi = dx if i == 0 else torch.empty_like(dx)
         dWi = dW if i == 0 else torch.empty_like(dW)
         dvi = dv if i == 0 else torch.empty_like(dv)
         dbi = db if i == 0 else torch.empty_like(db)
@@ -303,9 +571,10 @@ def run_ours(args):
         red = reducer if i == 0 or world == 1 else GradReducer([dWi, dvi, dbi])
         small = torch.empty(4 * d + B * d, device=dev)
         out_dW = torch.empty(N, K).pin_memory()
+        out_dx = torch.empty(L, B, d).pin_memory()
         out_small = torch.empty(4 * d + B * d).pin_memory()
-        sets.append(dict(bufs=(Xi, xi, dhi, dWi, dvi, dbi, dc0i, red), small=small, out_dW=out_dW,
-                         out_small=out_small))
+        sets.append(dict(bufs=(Xi, xi, dhi, dxi, dWi, dvi, dbi, dc0i, red), small=small, out_dW=out_dW,
+                         out_dx=out_dx, out_small=out_small))
     s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in_ready", "computed", "out_done")}
 
@@ -315,7 +584,7 @@ def run_ours(args):
         for k in range(nsteps):
             i = k % 2
             st_ = sets[i]
-            Xi, xi, dhi, dWi, dvi, dbi, dc0i, _ = st_["bufs"]
+            Xi, xi, dhi, dxi, dWi, dvi, dbi, dc0i, _ = st_["bufs"]
             if k >= 2:
                 s_h2d.wait_event(ev["computed"][i])  # step k-2 is done reading this input set
             with torch.cuda.stream(s_h2d):
@@ -335,6 +604,7 @@ def run_ours(args):
             s_d2h.wait_event(ev["computed"][i])
             with torch.cuda.stream(s_d2h):
                 st_["out_dW"].copy_(dWi, non_blocking=True)
+                st_["out_dx"].copy_(dxi, non_blocking=True)
                 st_["out_small"].copy_(sm, non_blocking=True)
                 ev["out_done"][i].record(s_d2h)
         stream.wait_stream(s_h2d)
@@ -356,54 +626,66 @@ def run_ours(args):
         dist.barrier()
     e2e_ms = float(t.item())
     h2d = hX.numel() * 2 + hx.numel() * 4 + hdh.numel() * 4
-    d2h = sets[0]["out_dW"].numel() * 4 + sets[0]["out_small"].numel() * 4
+    d2h = (sets[0]["out_dW"].numel() + sets[0]["out_dx"].numel() + sets[0]["out_small"].numel()) * 4
     st = sru.sru_sync_status()
     if st != 0:
         raise RuntimeError(f"device status {st} in the end-to-end region")
+
+    workloads = None
+    if rank == 0 and world == 1 and not args.skip_workloads:
+        workloads = measure_workloads(dev, peaks)
 
     if rank == 0:
         tokens = cfg.tokens * world * args.steps
         value = tokens / (elapsed_ms / 1e3)
         gemm_flops = 2.0 * M * N * K
-        # DRAM read + write per launch from the ncu capture summarised in
-        # profiles/launches_lm_train_step.md (same kernels, this workload)
-        gemm_traffic = {"project": 266.2e6, "project_dX": 535.9e6, "project_dW": 457.2e6}
+        traffic, traffic_src = load_traffic()
+        traffic = traffic.get(WORKLOAD, {})
         gemm_ms = {n: phase_ms[n] for n in ("project", "project_dX", "project_dW")}
         dom = max(gemm_ms, key=gemm_ms.get)
-        peak_tc = peaks["bf16_tflops_sustained"]
+        peak_kind, peak_tc = tensor_peak(peaks, clocks)
         ach_tc = gemm_flops / (gemm_ms[dom] / 1e3) / 1e12
         fwd_bytes = 14.0 * L * B * d
         bwd_bytes = 24.0 * L * B * d
         ach_f = fwd_bytes / (phase_ms["forward"] / 1e3) / 1e9
         ach_b = bwd_bytes / (phase_ms["backward"] / 1e3) / 1e9
+        sm = clocks.get("sm_mhz")
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 GEMM + f32 recurrence",
             "data": "synthetic", "config": config,
-            "roofline": {"bound": "tensor", "kernel": f"tc_gemm ({dom})", "achieved": ach_tc, "peak": peak_tc,
-                         "unit": "TFLOP/s", "frac": ach_tc / peak_tc, "traffic": gemm_traffic[dom],
-                         "traffic_unit": "bytes per launch (ncu dram read+write)",
-                         "peak_source": f"{peaks['source']} bf16 sustained (kernel inside a long step)",
+            "roofline": {"bound": "tensor", "kernel": f"tc_gemm_pair_kernel ({dom})", "achieved": ach_tc,
+                         "peak": peak_tc, "unit": "TFLOP/s", "frac": ach_tc / peak_tc,
+                         "traffic": traffic.get(dom), "traffic_unit": "bytes per launch (ncu dram read+write)",
+                         "traffic_source": traffic_src,
+                         "peak_source": f"{peaks['source']} bf16 {peak_kind} (chosen from this run's clocks: "
+                                        f"median {sm} MHz, reasons {clocks.get('reasons')})",
+                         "frac_of_burst": ach_tc / peaks["bf16_tflops"],
+                         "frac_of_sustained": ach_tc / peaks["bf16_tflops_sustained"],
+                         "frac_of_nominal_2250": ach_tc / NOMINAL_BF16_TFLOPS,
+                         "ms_x_sm_mhz": gemm_ms[dom] * sm if sm else None,
                          "algorithmic_per_launch": f"2*M*N*K = {gemm_flops:.4g} flop"},
             "roofline_recurrence": {
                 "bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
                 "forward": {"achieved": ach_f, "frac": ach_f / peaks["hbm_gbs"], "bytes": fwd_bytes,
-                            "ms": phase_ms["forward"], "traffic": 446.4e6},
+                            "ms": phase_ms["forward"], "traffic": traffic.get("forward")},
                 "backward": {"achieved": ach_b, "frac": ach_b / peaks["hbm_gbs"], "bytes": bwd_bytes,
-                             "ms": phase_ms["backward"], "traffic": 771.2e6},
-                "traffic_source": "ncu dram read+write per launch, profiles/launches_lm_train_step.md",
-                "frac_of_nominal_8TBs": {"forward": ach_f / 8000.0, "backward": ach_b / 8000.0}},
+                             "ms": phase_ms["backward"], "traffic": traffic.get("backward")},
+                "traffic_source": traffic_src,
+                "frac_of_nominal_8TBs": {"forward": ach_f / NOMINAL_HBM_GBS, "backward": ach_b / NOMINAL_HBM_GBS}},
             "phase_ms": phase_ms,
             "e2e": {"value": cfg.tokens * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 6 * args.steps,
             "clocks": clocks,
         }
+        if workloads is not None:
+            line["workloads"] = workloads
         if world == 1:
-            cpu_tps, desc, _ = cpu_baseline(cfg, budget_s=args.cpu_budget)
+            cpu_tps, desc, _, measured = cpu_baseline(cfg, budget_s=args.cpu_budget)
             line["cpu_baseline"] = {"value": cpu_tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                    "sample": desc}
+                                    "sample": desc, "extrapolated": True, "measured_s": measured, **host_info()}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -541,16 +823,23 @@ def run_reference(args):
     budget = args.ref_step_budget
     if budget is None:
         budget = min(2.0, 150.0 / max(1, args.warmup + args.steps))
+    measured = []
     for k in range(args.warmup + args.steps):
-        tps, desc, full = cpu_baseline(cfg, budget_s=budget, seed=k)
+        tps, desc, full, meas = cpu_baseline(cfg, budget_s=budget, seed=k)
         if k >= args.warmup:
             per_step.append(full)
+            measured.append(meas)
     full_s = statistics.mean(per_step)
     value = cfg.tokens / full_s
+    # ms_per_step is extrapolated from the measured sample (a full step of the
+    # oracle would take hours); the seconds actually measured are given beside it
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": full_s * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config, "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
+            "warmup": args.warmup, "ms_per_step": full_s * 1e3, "extrapolated": True,
+            "measured_sample_s_per_step": statistics.mean(measured), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc,
+                             "extrapolated": True, "measured_s": statistics.mean(measured), **host_info()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
@@ -565,6 +854,8 @@ def main():
     ap.add_argument("--workload", choices=["train", "decode"], default="train",
                     help="train: the layer training step (the headline); decode: batch-1 token steps")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--skip-workloads", action="store_true",
+                    help="leave out the per-workload block (the headline step only)")
     ap.add_argument("--ref-step-budget", type=float, default=None,
                     help="seconds of oracle work per reference step (default: 2 s, less so that the whole "
                          "--impl reference run stays near 150 s)")

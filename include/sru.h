@@ -31,7 +31,9 @@
  * gradient (dU = 0, no dx contribution); the state gradient passes through it.
  *
  * Pointers: every data pointer is a DEVICE pointer owned by the caller, at
- * least 16-byte aligned, to densely packed memory of the stated layout.
+ * least 16-byte aligned, to densely packed memory of the stated layout (the
+ * calls check 16 bytes for the (L, B, ...) tensors and at least 8 bytes for the
+ * per-channel vectors v, b, c0, c_T and their gradients; SRU_ERR_INVALID).
  * The library allocates no device memory.  `stream` is a cudaStream_t (NULL =
  * legacy default stream); calls are stream-ordered and asynchronous (none
  * synchronises).  Size limits: d % 8 == 0, 1 <= d, 0 <= L, 0 <= B, L*B < 2^31.
@@ -184,7 +186,9 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
  * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
  * call).  Its first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, once per device, with that device current); make
- * that first call before any stream capture.  Every call zeroes the flags it
+ * that first call before any stream capture: a first call on a device whose
+ * stream is capturing is refused with SRU_ERR_INVALID, before anything is
+ * launched.  Every call zeroes the flags it
  * uses before launching and otherwise reuses whatever the previous call left
  * in the array, so calls that overlap on the GPU (concurrent streams, or
  * several host threads on the same device) race on the shared scratch and

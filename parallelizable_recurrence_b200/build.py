@@ -2,6 +2,7 @@
 from __future__ import annotations
 
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -11,7 +12,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsru.so")
 SOURCES = ["sru_api.cu"]
-DEPS = ["sru_api.cu", "sru_ptx.cuh", "sru_recurrence.cuh", "sru_gemm.cuh", "sru_scan.cuh"]
+_INCLUDE_RE = re.compile(r'^\s*#\s*include\s*"([^"]+)"', re.M)
 
 
 def nvcc() -> str:
@@ -19,12 +20,25 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else (shutil.which("nvcc") or "nvcc")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def deps(csrc: str = CSRC) -> list:
+    """Every file the library build reads: the sources and, transitively, each
+    file they #include "..." (paths resolved against the including file)."""
+    seen, todo = [], [os.path.join(csrc, s) for s in SOURCES]
+    while todo:
+        f = os.path.normpath(todo.pop())
+        if f in seen or not os.path.exists(f):
+            continue
+        seen.append(f)
+        with open(f) as fh:
+            todo += [os.path.join(os.path.dirname(f), inc) for inc in _INCLUDE_RE.findall(fh.read())]
+    return seen
+
+
+def _stale(lib: str = LIB, csrc: str = CSRC) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
-    srcs = [os.path.join(CSRC, f) for f in DEPS] + [os.path.join(ROOT, "include", "sru.h")]
-    return any(os.path.exists(s) and os.path.getmtime(s) > t for s in srcs)
+    t = os.path.getmtime(lib)
+    return any(os.path.getmtime(s) > t for s in deps(csrc))
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

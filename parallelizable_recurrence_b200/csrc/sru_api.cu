@@ -32,6 +32,9 @@ sru_status cuda_fail(cudaError_t e) {
     } while (0)
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// the per-channel vectors (v, b, c0, c_T and their gradients) are read and
+// written as 8-byte channel pairs; a null (optional) pointer passes
+inline bool aligned8_or_null(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -664,23 +667,30 @@ size_t noalloc_scan_bytes(int64_t items, size_t* agg_a_off, size_t* agg_b_off, s
 
 // Device address of the scratch on the current device, looked up once per
 // device.  In host code g_noalloc_scratch names a host-side stand-in, never
-// the device array, so kernels only ever receive this looked-up address.
-cudaError_t noalloc_scratch_address(void** out) {
+// the device array, so kernels only ever receive this looked-up address.  The
+// lookup is not a stream operation, but it may load the library's module on
+// the device, which a stream capture in progress does not allow: a first call
+// on a device made while `st` is capturing is refused with SRU_ERR_INVALID.
+sru_status noalloc_scratch_address(cudaStream_t st, void** out) {
     static std::mutex mu;
     static void* addr[kMaxDevices] = {nullptr};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return cuda_fail(cudaErrorInvalidDevice);
     std::lock_guard<std::mutex> lock(mu);
     if (addr[dev] == nullptr) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        e = cudaStreamIsCapturing(st, &cs);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (cs != cudaStreamCaptureStatusNone) return SRU_ERR_INVALID;  // first call during a capture
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) return cuda_fail(e);
         addr[dev] = p;
     }
     *out = addr[dev];
-    return cudaSuccess;
+    return SRU_OK;
 }
 
 }  // namespace
@@ -793,6 +803,8 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
     const int n_dir = bidirectional ? 2 : 1;
     if (B == 0) return SRU_OK;
     if (!v || !b || !c_T) return SRU_ERR_INVALID;
+    if (!aligned8_or_null(v) || !aligned8_or_null(b) || !aligned8_or_null(c0) || !aligned8_or_null(c_T))
+        return SRU_ERR_INVALID;
     cudaStream_t st = as_stream(stream);
     if (L == 0) {
         const size_t n = (size_t)B * n_dir * d;
@@ -837,6 +849,9 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     if (du_t != SRU_F32 && du_t != SRU_BF16) return SRU_ERR_INVALID;
     const int n_dir = bidirectional ? 2 : 1;
     if (!v || !b || !dv || !db) return SRU_ERR_INVALID;
+    if (!aligned8_or_null(v) || !aligned8_or_null(b) || !aligned8_or_null(dc_T) || !aligned8_or_null(dv) ||
+        !aligned8_or_null(db) || !aligned8_or_null(dc0))
+        return SRU_ERR_INVALID;
     cudaStream_t st = as_stream(stream);
     if (B == 0 || L == 0) {
         // no steps: dv = db = 0, dc0 = dc_T
@@ -908,6 +923,7 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
     const int n_dir = bidirectional ? 2 : 1;
     if (B == 0) return SRU_OK;
     if (!b || !c_T) return SRU_ERR_INVALID;
+    if (!aligned8_or_null(b) || !aligned8_or_null(c0) || !aligned8_or_null(c_T)) return SRU_ERR_INVALID;
     if (L > 0 && (!U || !x || !h || !aligned16(U) || !aligned16(x) || !aligned16(h))) return SRU_ERR_INVALID;
     const int64_t items = scan_chunks(L) * ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B * n_dir;
     size_t agg_a_off = 0, agg_b_off = 0, prefix_off = 0;
@@ -921,7 +937,8 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
         return SRU_OK;
     }
     void* scratch = nullptr;
-    SRU_CUDA_TRY(noalloc_scratch_address(&scratch));
+    s = noalloc_scratch_address(st, &scratch);
+    if (s != SRU_OK) return s;
     uint8_t* base = static_cast<uint8_t*>(scratch);
     sru::ScanState ss;
     ss.flags = reinterpret_cast<unsigned*>(base);

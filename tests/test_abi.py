@@ -120,3 +120,24 @@ def test_decode_step_checks_arguments_before_any_launch(lib):
     need = lib.sru_decode_workspace_bytes(16, 64)
     assert need >= 3 * 64 * 16 * 4
     assert lib.sru_decode_step(*args, 16, 64, 1.0, fake, need - 256, None) == 1
+
+
+def test_per_channel_vectors_must_be_pair_aligned(lib):
+    """v, b, c0, c_T (and dc_T, dv, db, dc0) are read and written as 8-byte channel
+    pairs: a pointer off an 8-byte boundary is rejected before any launch."""
+    vp = ctypes.c_void_p
+    fake, odd = vp(0x1000), vp(0x1004)
+    for pos in (3, 4, 5, 14):  # v, b, c0, c_T
+        args = [fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, fake, None, 0, None]
+        args[pos] = odd
+        assert lib.sru_forward(*args) == 1, pos
+    need = lib.sru_workspace_bytes(4, 2, 16, 0, 0)
+    for pos in (3, 4, 14, 20, 21, 22):  # v, b, dc_T, dv, db, dc0
+        args = [fake, 1, fake, fake, fake, None, None, 4, 2, 16, 1.0, 0, 0, fake, fake, fake, need,
+                fake, 1, fake, fake, fake, fake, None]
+        args[pos] = odd
+        assert lib.sru_backward(*args) == 1, pos
+    for pos in (3, 4, 12):  # b, c0, c_T
+        args = [fake, 1, fake, fake, fake, None, 4, 2, 64, 1.0, 0, fake, fake, None]
+        args[pos] = odd
+        assert lib.sru_forward_scan_noalloc(*args) == 1, pos
