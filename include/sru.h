@@ -199,6 +199,34 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
                                     float alpha, int bidirectional, float* h, float* c_T, void* stream);
 
 /*
+ * Eq. (1) and Eqs. (2)-(5) in one kernel (the page's Figure 2(a): the grouped
+ * matrix multiplication and the element-wise recurrence, fused): computes what
+ *   sru_project(X, BF16, W, BF16, U, BF16, L*B, n_dir*3*d, d) followed by
+ *   sru_forward(U, BF16, x, v, b, c0, mask, L, B, d, alpha, bidirectional, 0,
+ *               h, c_T, workspace)
+ * computes, without reading U back from memory: each 32-step x 4-row x
+ * 64-channel tile of the product is rounded to bf16 (as U is stored on the
+ * two-call path) and the recurrence runs on it from shared memory.
+ *   X (L*B, d) bf16 time-major, W (n_dir*3*d, d) bf16 (W_cat, gate blocks as
+ *   above), x, v, b, c0, mask, h, c_T as for sru_forward.
+ *   U nullable: when given ((L, B, n_dir, 3, d) bf16), the projection is also
+ *   stored there and the state checkpoints are written to the workspace, so
+ *   that sru_backward (flags 0, same workspace) can follow; when NULL, nothing
+ *   of U is stored (inference).
+ *   workspace: at least sru_workspace_bytes(L, B, d, bidirectional, flags) bytes
+ *   for any flags (it also carries the state from one time tile to the next;
+ *   its flags are cleared on the stream before the launch).
+ * The kernel keeps one CTA on every SM of the device and hands the state of a
+ * sequence between CTAs: do not run it concurrently with other work on the
+ * same GPU (its bounded waits would expire: SRU_ERR_TIMEOUT at the next
+ * sru_sync_status).  Limits as for sru_forward (d % 8 == 0).
+ */
+sru_status sru_forward_fused(const void* X, const void* W, const float* x, const float* v, const float* b,
+                             const float* c0, const uint8_t* mask, int64_t L, int64_t B, int64_t d, float alpha,
+                             int bidirectional, float* h, float* c_T, void* U, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
  * Factorised projection: the page's variant of Eq. (1) with a low-rank
  * projection (Figure 2, the SRU layer "with projection trick"):
  *   P = X Wq^T        (M, Kp)  Wq (Kp, K): projects d down to d' = Kp

@@ -32,6 +32,7 @@ SRU_FLAG_TEST_WITHHOLD_CARRY = 0x8
 # every symbol include/sru.h declares
 EXPORTED = ("sru_status_string", "sru_get_last_cuda_error", "sru_version", "sru_workspace_bytes",
             "sru_project", "sru_project_backward", "sru_forward", "sru_backward", "sru_forward_scan_noalloc",
+            "sru_forward_fused",
             "sru_project_factored", "sru_project_factored_backward", "sru_attention_workspace_bytes",
             "sru_attention_project", "sru_decode_workspace_bytes", "sru_decode_step", "sru_sync_status")
 
@@ -81,6 +82,9 @@ def load_library(path: str = LIB_PATH):
     lib.sru_forward_scan_noalloc.restype = _int
     lib.sru_forward_scan_noalloc.argtypes = [_vp, _int, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _f32, _int,
                                              _vp, _vp, _vp]
+    lib.sru_forward_fused.restype = _int
+    lib.sru_forward_fused.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _f32, _int,
+                                      _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
     lib.sru_project_factored.restype = _int
     lib.sru_project_factored.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp]
     lib.sru_project_factored_backward.restype = _int
@@ -217,6 +221,23 @@ def sru_forward_scan_noalloc(U, x, b, h, c_T, c0=None, mask=None, alpha: float =
                                         int(bool(bidirectional)), _ptr(h, torch.float32),
                                         _ptr(c_T, torch.float32), _stream(stream)),
            "sru_forward_scan_noalloc")
+    return h, c_T
+
+
+def sru_forward_fused(X, W, x, v, b, h, c_T, workspace, c0=None, mask=None, alpha: float = 1.0,
+                      bidirectional: bool = False, U=None, stream=None):
+    """Eq. (1) and Eqs. (2)-(5) in one kernel: X (L*B, d) bf16, W (n_dir*3d, d)
+    bf16, x (L, B, d) fp32, v and b (n_dir, 2, d); h (L, B, n_dir, d) and c_T
+    (B, n_dir, d) written in place.  With U ((L, B, n_dir, 3, d) bf16) the
+    projection and the checkpoints are stored for sru_backward (same workspace)."""
+    lib = load_library()
+    L, B, d = x.shape
+    _check(lib.sru_forward_fused(_ptr(X, torch.bfloat16), _ptr(W, torch.bfloat16), _ptr(x, torch.float32),
+                                 _ptr(v, torch.float32), _ptr(b, torch.float32), _ptr(c0, torch.float32),
+                                 _ptr(mask, torch.uint8), L, B, d, float(alpha), int(bool(bidirectional)),
+                                 _ptr(h, torch.float32), _ptr(c_T, torch.float32), _ptr(U, torch.bfloat16),
+                                 _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "sru_forward_fused")
     return h, c_T
 
 

@@ -15,6 +15,7 @@
 #include "sru_attention.cuh"
 #include "sru_decode.cuh"
 #include "sru_scan.cuh"
+#include "sru_fused.cuh"
 
 namespace {
 
@@ -114,10 +115,12 @@ cudaError_t ensure_smem(const void* kernel, size_t bytes) {
 }
 
 // ---------------------------------------------------------- workspace layout
-// [checkpoints | dv/db partial sums | scan flags | scan aggregates A, B, prefix]
-// The scan regions exist only when SRU_FLAG_V_ZERO is set.
+// [checkpoints | fused-forward carries and flags | dv/db partial sums | scan
+//  flags | scan aggregates A, B, prefix].  The scan regions exist only when a
+// scan can run (see ws_has_scan); the offsets of the first two regions do not
+// depend on the flags.
 struct WsLayout {
-    size_t ckpt_off, partial_off, flags_off, agg_a_off, agg_b_off, prefix_off, total;
+    size_t ckpt_off, carry_off, fflags_off, partial_off, flags_off, agg_a_off, agg_b_off, prefix_off, total;
     int64_t scan_items;
 };
 
@@ -133,6 +136,10 @@ WsLayout ws_layout(int64_t L, int64_t B, int64_t d, int n_dir, unsigned flags) {
     size_t off = 0;
     w.ckpt_off = off;
     off += round256((size_t)nch * B * n_dir * d * sizeof(float));
+    w.carry_off = off;
+    off += round256((size_t)B * n_dir * d * sizeof(float));
+    w.fflags_off = off;
+    off += round256((size_t)B * n_dir * ((d + sru::fused::kCh - 1) / sru::fused::kCh) * sizeof(unsigned));
     w.partial_off = off;
     const int64_t partial_rows = scan ? scan_chunks(L) * B : B;
     off += round256((size_t)partial_rows * n_dir * 4 * d * sizeof(double));
@@ -693,6 +700,31 @@ sru_status noalloc_scratch_address(cudaStream_t st, void** out) {
     return SRU_OK;
 }
 
+// CTA pairs of the fused forward that the device can hold at once (the
+// kernel hands the state between CTAs, so its whole grid must be resident):
+// the occupancy calculator's count of co-resident 2-CTA clusters, cached per
+// device.
+int64_t fused_resident_pairs() {
+    static std::mutex mu;
+    static int cache[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == 0) {
+        auto kern = sru::fused::sru_fused_fwd_kernel;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * (sm_count() / 2)), 1, 1);
+        cfg.blockDim = dim3(sru::fused::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = sru::fused::kSmemBytes;
+        int n = 0;
+        if (ensure_smem(reinterpret_cast<const void*>(kern), sru::fused::kSmemBytes) != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(kern), &cfg) != cudaSuccess)
+            n = 0;
+        cache[dev] = n > 0 ? (n < sm_count() / 2 ? n : sm_count() / 2) : -1;
+    }
+    return cache[dev];
+}
+
 }  // namespace
 
 // =========================================================================
@@ -952,6 +984,89 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
     if (u_t == SRU_BF16)
         return launch_fwd_scan<__nv_bfloat16>(mp, b, c0, mask, h, c_T, nullptr, ss, L, B, d, n_dir, alpha, st);
     return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, nullptr, ss, L, B, d, n_dir, alpha, st);
+}
+
+sru_status sru_forward_fused(const void* X, const void* W, const float* x, const float* v, const float* b,
+                             const float* c0, const uint8_t* mask, int64_t L, int64_t B, int64_t d, float alpha,
+                             int bidirectional, float* h, float* c_T, void* U, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    sru_status s = check_layer_sizes(L, B, d);
+    if (s != SRU_OK) return s;
+    const int n_dir = bidirectional ? 2 : 1;
+    if (B == 0) return SRU_OK;
+    if (!v || !b || !c_T) return SRU_ERR_INVALID;
+    if (!aligned8_or_null(v) || !aligned8_or_null(b) || !aligned8_or_null(c0) || !aligned8_or_null(c_T))
+        return SRU_ERR_INVALID;
+    cudaStream_t st = as_stream(stream);
+    if (L == 0) {
+        const size_t n = (size_t)B * n_dir * d;
+        sru::sru_copy_state_kernel<<<blocks_for(n, 256), 256, 0, st>>>(c0, c_T, n);
+        SRU_CUDA_TRY(cudaGetLastError());
+        return SRU_OK;
+    }
+    if (!X || !W || !x || !h || !workspace) return SRU_ERR_INVALID;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(x) || !aligned16(h) || !aligned16(workspace) ||
+        (U && !aligned16(U)))
+        return SRU_ERR_INVALID;
+    const WsLayout w = ws_layout(L, B, d, n_dir, SRU_FLAG_FORCE_SEQUENTIAL);  // the smallest layout
+    if (workspace_bytes < w.total) return SRU_ERR_INVALID;
+    const int64_t nT = (L + sru::fused::kTt - 1) / sru::fused::kTt;
+    const int64_t njs = (d + sru::fused::kCh - 1) / sru::fused::kCh;
+    const int64_t nbgp = (B + 2 * sru::fused::kBb - 1) / (2 * sru::fused::kBb);
+    const int64_t items = nT * n_dir * nbgp * njs;
+    if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
+    CUtensorMap mx, mw, mu;
+    {
+        const uint64_t dims[3] = {(uint64_t)d, (uint64_t)B, (uint64_t)L};
+        const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)B * d * 2};
+        const uint32_t box[3] = {64, (uint32_t)sru::fused::kBb, (uint32_t)sru::fused::kTt};
+        if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return SRU_ERR_INVALID;
+    }
+    {
+        const uint64_t dims[3] = {(uint64_t)d, (uint64_t)d, (uint64_t)(3 * n_dir)};
+        const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)d * d * 2};
+        const uint32_t box[3] = {64, (uint32_t)(sru::fused::kCh / 2), 3};
+        if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, W, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return SRU_ERR_INVALID;
+    }
+    std::memset(&mu, 0, sizeof(mu));
+    if (U) {
+        const uint64_t dims[5] = {(uint64_t)d, 3, (uint64_t)n_dir, (uint64_t)B, (uint64_t)L};
+        const uint64_t strides[4] = {(uint64_t)d * 2, (uint64_t)3 * d * 2, (uint64_t)n_dir * 3 * d * 2,
+                                     (uint64_t)B * n_dir * 3 * d * 2};
+        const uint32_t box[5] = {(uint32_t)sru::fused::kCh, 3, 1, (uint32_t)sru::fused::kBb,
+                                 (uint32_t)sru::fused::kTt};
+        if (!make_map(&mu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, U, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return SRU_ERR_INVALID;
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    sru::fused::FusedArgs fa;
+    fa.x = x;
+    fa.v = v;
+    fa.bias = b;
+    fa.c0 = c0;
+    fa.mask = mask;
+    fa.h = h;
+    fa.c_T = c_T;
+    fa.ckpt = U ? reinterpret_cast<float*>(ws + w.ckpt_off) : nullptr;
+    fa.carry = reinterpret_cast<float*>(ws + w.carry_off);
+    fa.flags = reinterpret_cast<unsigned*>(ws + w.fflags_off);
+    fa.L = (int)L;
+    fa.B = (int)B;
+    fa.d = (int)d;
+    fa.n_dir = n_dir;
+    fa.alpha = alpha;
+    fa.write_u = U != nullptr;
+    SRU_CUDA_TRY(cudaMemsetAsync(fa.flags, 0, (size_t)B * n_dir * njs * sizeof(unsigned), st));
+    auto kern = sru::fused::sru_fused_fwd_kernel;
+    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::fused::kSmemBytes));
+    const int64_t max_pairs = fused_resident_pairs();
+    if (max_pairs < 1) return cuda_fail(cudaErrorLaunchOutOfResources);
+    const int64_t pairs = items < max_pairs ? items : max_pairs;
+    kern<<<(unsigned)(2 * pairs), sru::fused::kThreads, sru::fused::kSmemBytes, st>>>(mx, mw, mu, fa);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
 }
 
 sru_status sru_project_factored(const void* X, const void* Wq, const void* Wo, void* P, void* U, int u_t,
