@@ -372,75 +372,131 @@ def _gemm_entries(lay, flush):
             "project_dW": _tc_entry("sru_project_backward (dW = dU^T X)", t_dw, fl)}
 
 
-def measure_workloads(dev, peaks):
+def _fused_entry(lay, ms, with_u):
+    """The fused forward against the roofline of a kernel that is both a product
+    and a stream: its time bound is the larger of flops / tensor peak and
+    algorithmic bytes / HBM peak (bytes: X 2 B per (t, b, k), W_cat once, x 4 and
+    h 4 per element, + U 6 per element when it is stored)."""
+    L, B, d, nd = lay.L, lay.B, lay.d, lay.nd
+    flops = 2.0 * L * B * nd * 3 * d * d
+    nbytes = 2.0 * L * B * d + 2.0 * nd * 3 * d * d + (4.0 + (6.0 if with_u else 0.0)) * lay.elements + 4.0 * L * B * d
+    return {"kernel": "sru_forward_fused" + (" (U stored)" if with_u else " (inference: no U)"), "bound": "mixed",
+            "ms": ms, "algorithmic_flops": flops, "algorithmic_bytes": nbytes,
+            "achieved_tflops": flops / (ms / 1e3) / 1e12, "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+            "tokens_per_s": L * B / (ms / 1e3)}
+
+
+def _layer_rec_only(dev, flush, sru):
+    lay = _Layer(1024, 16, 3072, 1, 4, dev)
+    out = {"rec_only L1024 B16 d3072 v!=0": _recurrence_entries(lay, flush, [("", 0)])}
+    lay.v.zero_()
+    VZ, SCAN, SEQ = sru.SRU_FLAG_V_ZERO, sru.SRU_FLAG_FORCE_SCAN, sru.SRU_FLAG_FORCE_SEQUENTIAL
+    out["rec_only_v0 L1024 B16 d3072 v=0"] = _recurrence_entries(
+        lay, flush, [("_dispatched", VZ), ("_scan_forced", VZ | SCAN), ("_sequential_forced", VZ | SEQ)])
+    return out
+
+
+def _layer_scan_regime(dev, flush, sru):
+    # a layer in the chunked scan's regime (B*d too small to fill the GPU), v = 0
+    lay = _Layer(2048, 4, 2048, 1, 5, dev, v_zero=True)
+    VZ, SEQ = sru.SRU_FLAG_V_ZERO, sru.SRU_FLAG_FORCE_SEQUENTIAL
+    return {"scan_regime L2048 B4 d2048 v=0": _recurrence_entries(
+        lay, flush, [("_dispatched", VZ), ("_sequential_forced", VZ | SEQ)])}
+
+
+def _layer_lm_fwd(dev, flush, sru):
+    # forward-only language-model layer, bf16 projection
+    L, B, d = 256, 32, 512
+    lay = _Layer(L, B, d, 1, 1, dev, project=True)
+    e = {"project": _gemm_entries(lay, flush)["project"]}
+    e["forward"] = _hbm_entry("sru_forward", _time_ms(lambda: lay.forward(0), flush), lay.fwd_bytes())
+    t_step = _time_ms(lambda: (sru.sru_project(lay.X, lay.W, lay.U.view(L * B, 3 * d)), lay.forward(0)), flush)
+    e["layer_two_calls"] = {"ms": t_step, "tokens_per_s": L * B / (t_step / 1e3), "calls": "sru_project + sru_forward"}
+    t_f = _time_ms(lambda: sru.sru_forward_fused(lay.X, lay.W, lay.x, lay.v, lay.b, lay.h, lay.cT, lay.ws), flush)
+    e["layer_fused"] = _fused_entry(lay, t_f, with_u=False)
+    return {"lm_fwd L256 B32 d512 forward": e}
+
+
+def _layer_lm_train_fused(dev, flush, sru):
+    # the training layer's forward: two calls vs fused (U and checkpoints stored for the backward)
+    L, B, d = 1024, 16, 2048
+    lay = _Layer(L, B, d, 1, 2, dev, project=True, c0=True)
+    t2 = _time_ms(lambda: (sru.sru_project(lay.X, lay.W, lay.U.view(L * B, 3 * d)), lay.forward(0)), flush)
+    t_f = _time_ms(lambda: sru.sru_forward_fused(lay.X, lay.W, lay.x, lay.v, lay.b, lay.h, lay.cT, lay.ws,
+                                                 c0=lay.c0, U=lay.U), flush)
+    t_i = _time_ms(lambda: sru.sru_forward_fused(lay.X, lay.W, lay.x, lay.v, lay.b, lay.h, lay.cT, lay.ws,
+                                                 c0=lay.c0), flush)
+    return {"lm_train L1024 B16 d2048 forward": {
+        "layer_two_calls": {"ms": t2, "tokens_per_s": L * B / (t2 / 1e3), "calls": "sru_project + sru_forward"},
+        "layer_fused_with_U": _fused_entry(lay, t_f, with_u=True),
+        "layer_fused_inference": _fused_entry(lay, t_i, with_u=False)}}
+
+
+def _layer_bidir(dev, flush, sru):
+    # bidirectional padded layer, 2 directions
+    lay = _Layer(2048, 64, 1024, 2, 3, dev, masked=True, project=True)
+    e = _gemm_entries(lay, flush)
+    e.update(_recurrence_entries(lay, flush, [("", 0)], tag="_masked"))
+    e["valid_fraction"] = lay.valid
+    t_f = _time_ms(lambda: sru.sru_forward_fused(lay.X, lay.W, lay.x, lay.v, lay.b, lay.h, lay.cT, lay.ws,
+                                                 mask=lay.mask, bidirectional=True, U=lay.U), flush)
+    e["layer_fused_with_U_masked"] = _fused_entry(lay, t_f, with_u=True)
+    lay.mask, lay.valid = None, 1.0
+    e.update(_recurrence_entries(lay, flush, [("", 0)], tag="_unmasked"))
+    return {"bidir_masked L2048 B64 d1024 x2": e}
+
+
+# recurrence-only layers first, the product-heavy ones last (so that a power
+# cap reached under the products does not slow the latency-bound recurrences)
+WORKLOAD_LAYERS = {"rec_only": _layer_rec_only, "scan_regime": _layer_scan_regime, "lm_fwd": _layer_lm_fwd,
+                   "lm_train_fused": _layer_lm_train_fused, "bidir_masked": _layer_bidir}
+
+
+def measure_workloads(dev, peaks, only=None):
     """Device-timed kernels of the other layer workloads, each alone with L2
-    flushed before every timed call (median of 10 after 3 warm-up calls)."""
+    flushed before every timed call (median of 10 after 3 warm-up calls).  The
+    clocks are sampled per layer and each layer's tensor peak chosen from them."""
     import torch
     import parallelizable_recurrence_b200 as sru
-    VZ, SCAN, SEQ = sru.SRU_FLAG_V_ZERO, sru.SRU_FLAG_FORCE_SCAN, sru.SRU_FLAG_FORCE_SEQUENTIAL
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    res = {}
-    with ClockSampler(dev.index if dev.index is not None else 0, period_s=0.02) as clk:
-        # forward-only language-model layer: L256 B32 d512, bf16 projection
-        lay = _Layer(256, 32, 512, 1, 1, dev, project=True)
-        e = _gemm_entries(lay, flush)
-        e = {"project": e["project"]}
-        t = _time_ms(lambda: lay.forward(0), flush)
-        e["forward"] = _hbm_entry("sru_forward", t, lay.fwd_bytes())
-        t_step = _time_ms(lambda: (sru.sru_project(lay.X, lay.W, lay.U.view(256 * 32, 1536)), lay.forward(0)), flush)
-        e["layer_forward"] = {"ms": t_step, "tokens_per_s": 256 * 32 / (t_step / 1e3),
-                              "calls": "sru_project + sru_forward"}
-        res["lm_fwd L256 B32 d512 forward"] = e
-        del lay
+    res, clocks_by_layer = {}, {}
+    for key, fn in WORKLOAD_LAYERS.items():
+        if only is not None and key != only:
+            continue
+        with ClockSampler(dev.index if dev.index is not None else 0, period_s=0.01) as clk:
+            out = fn(dev, flush, sru)
+            torch.cuda.synchronize()
         torch.cuda.empty_cache()
-        # bidirectional padded layer: L2048 B64 d1024 x 2 directions
-        lay = _Layer(2048, 64, 1024, 2, 3, dev, masked=True, project=True)
-        e = _gemm_entries(lay, flush)
-        e.update(_recurrence_entries(lay, flush, [("", 0)], tag="_masked"))
-        e["valid_fraction"] = lay.valid
-        mask = lay.mask
-        lay.mask, lay.valid = None, 1.0
-        e.update(_recurrence_entries(lay, flush, [("", 0)], tag="_unmasked"))
-        lay.mask = mask
-        res["bidir_masked L2048 B64 d1024 x2"] = e
-        del lay, mask
-        torch.cuda.empty_cache()
-        # recurrence-only layer, U given: L1024 B16 d3072, v != 0, then v = 0
-        lay = _Layer(1024, 16, 3072, 1, 4, dev)
-        res["rec_only L1024 B16 d3072 v!=0"] = _recurrence_entries(lay, flush, [("", 0)])
-        lay.v.zero_()
-        res["rec_only_v0 L1024 B16 d3072 v=0"] = _recurrence_entries(
-            lay, flush, [("_dispatched", VZ), ("_scan_forced", VZ | SCAN), ("_sequential_forced", VZ | SEQ)])
-        del lay
-        torch.cuda.empty_cache()
-        # a layer in the chunked scan's regime (B*d too small to fill the GPU): L2048 B4 d2048, v = 0
-        lay = _Layer(2048, 4, 2048, 1, 5, dev, v_zero=True)
-        res["scan_regime L2048 B4 d2048 v=0"] = _recurrence_entries(
-            lay, flush, [("_dispatched", VZ), ("_sequential_forced", VZ | SEQ)])
-        del lay
-        torch.cuda.empty_cache()
-    clocks = clk.summary()
+        clocks = clk.summary()
+        kind, tc_peak = tensor_peak(peaks, clocks)
+        for name, entries in out.items():
+            clocks_by_layer[name] = dict(clocks, bf16_peak_kind=kind, bf16_peak=tc_peak)
+            for ent in entries.values():
+                if not isinstance(ent, dict) or "bound" not in ent:
+                    continue
+                if ent["bound"] == "hbm":
+                    ent["peak"] = peaks["hbm_gbs"]
+                    ent["frac"] = ent["achieved"] / peaks["hbm_gbs"]
+                    ent["frac_of_nominal_8TBs"] = ent["achieved"] / NOMINAL_HBM_GBS
+                elif ent["bound"] == "tensor":
+                    ent["peak"] = tc_peak
+                    ent["frac"] = ent["achieved"] / tc_peak
+                    ent["frac_of_nominal_2250"] = ent["achieved"] / NOMINAL_BF16_TFLOPS
+                else:  # a product and a stream: the larger of the two bounds
+                    t_bound = max(ent["algorithmic_flops"] / (tc_peak * 1e12),
+                                  ent["algorithmic_bytes"] / (peaks["hbm_gbs"] * 1e9))
+                    ent["roofline_ms"] = t_bound * 1e3
+                    ent["frac"] = t_bound / (ent["ms"] / 1e3)
+            res[name] = entries
+        time.sleep(0.5)  # let the power state settle before the next layer
     st = sru.sru_sync_status()
     if st != 0:
         raise RuntimeError(f"device status {st} in the workload block")
-    src, tc_peak = tensor_peak(peaks, clocks)
-    for entries in res.values():
-        for k, ent in entries.items():
-            if not isinstance(ent, dict) or "bound" not in ent:
-                continue
-            if ent["bound"] == "hbm":
-                ent["peak"] = peaks["hbm_gbs"]
-                ent["frac"] = ent["achieved"] / peaks["hbm_gbs"]
-                ent["frac_of_nominal_8TBs"] = ent["achieved"] / NOMINAL_HBM_GBS
-            else:
-                ent["peak"] = tc_peak
-                ent["frac"] = ent["achieved"] / tc_peak
-                ent["frac_of_nominal_2250"] = ent["achieved"] / NOMINAL_BF16_TFLOPS
     return {"timing": "each kernel alone, median of 10 after 3 warm-up calls, 512 MB written before every "
                       "timed call (L2 flushed); inputs drawn on the device from seeded generators",
-            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": tc_peak, "bf16_peak_kind": src,
-                      "source": peaks["source"]},
-            "clocks": clocks, "layers": res}
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_burst": peaks["bf16_tflops"],
+                      "bf16_sustained": peaks["bf16_tflops_sustained"], "source": peaks["source"]},
+            "clocks": clocks_by_layer, "layers": res}
 
 
 # ------------------------------------------------------------ GPU arm
@@ -845,6 +901,16 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_only(args):
+    """One layer of the per-workload block alone (e.g. under ncu -k <kernel>)."""
+    import torch
+    import parallelizable_recurrence_b200 as sru
+    torch.cuda.set_device(0)
+    sru.load_library()
+    out = measure_workloads(torch.device("cuda", 0), load_peaks(), only=args.only)
+    print(json.dumps({"only": args.only, **out}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -854,6 +920,8 @@ def main():
     ap.add_argument("--workload", choices=["train", "decode"], default="train",
                     help="train: the layer training step (the headline); decode: batch-1 token steps")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--only", choices=sorted(WORKLOAD_LAYERS), default=None,
+                    help="run only this layer of the per-workload block and print it (for profiling one kernel)")
     ap.add_argument("--skip-workloads", action="store_true",
                     help="leave out the per-workload block (the headline step only)")
     ap.add_argument("--ref-step-budget", type=float, default=None,
@@ -862,7 +930,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.only is not None:
+        run_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.workload == "decode":
         run_decode(args)

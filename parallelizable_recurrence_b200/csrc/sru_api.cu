@@ -115,12 +115,12 @@ cudaError_t ensure_smem(const void* kernel, size_t bytes) {
 }
 
 // ---------------------------------------------------------- workspace layout
-// [checkpoints | fused-forward carries and flags | dv/db partial sums | scan
+// [checkpoints | fused-forward carries and flags | launch order | dv/db partial sums | scan
 //  flags | scan aggregates A, B, prefix].  The scan regions exist only when a
 // scan can run (see ws_has_scan); the offsets of the first two regions do not
 // depend on the flags.
 struct WsLayout {
-    size_t ckpt_off, carry_off, fflags_off, partial_off, flags_off, agg_a_off, agg_b_off, prefix_off, total;
+    size_t ckpt_off, carry_off, fflags_off, order_off, partial_off, flags_off, agg_a_off, agg_b_off, prefix_off, total;
     int64_t scan_items;
 };
 
@@ -140,6 +140,8 @@ WsLayout ws_layout(int64_t L, int64_t B, int64_t d, int n_dir, unsigned flags) {
     off += round256((size_t)B * n_dir * d * sizeof(float));
     w.fflags_off = off;
     off += round256((size_t)B * n_dir * ((d + sru::fused::kCh - 1) / sru::fused::kCh) * sizeof(unsigned));
+    w.order_off = off;
+    off += round256((size_t)B * n_dir * sizeof(int));
     w.partial_off = off;
     const int64_t partial_rows = scan ? scan_chunks(L) * B : B;
     off += round256((size_t)partial_rows * n_dir * 4 * d * sizeof(double));
@@ -479,13 +481,14 @@ static_assert(kSeqCJ >= 32 && kSeqCJ % 32 == 0, "sequential tile width");
 
 template <typename UT, int S, bool STAGE_H = false>
 sru_status launch_fwd_seq_s(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
-                            float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d, int n_dir,
-                            float alpha, cudaStream_t st) {
+                            float* h, float* c_T, float* ckpt, const int* order, int64_t L, int64_t B, int64_t d,
+                            int n_dir, float alpha, cudaStream_t st) {
     using Lay = sru::FwdLayout<UT, kSeqCJ, S>;
     auto kern = sru::sru_fwd_seq_kernel<UT, kSeqCJ, S, STAGE_H>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
-    dim3 grid((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)B, (unsigned)n_dir);
-    kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.h, v, b, c0, mask, h, c_T, ckpt, (int)L, (int)B,
+    const dim3 grid = order != nullptr ? dim3((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)(B * n_dir), 1)
+                                       : dim3((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)B, (unsigned)n_dir);
+    kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.h, v, b, c0, mask, h, c_T, ckpt, order, (int)L, (int)B,
                                               (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
@@ -497,35 +500,52 @@ int fwd_resident() {
                          sru::FwdLayout<UT, kSeqCJ, S>::SMEM);
 }
 
+// A padded layer whose grid needs more than one wave of resident CTAs takes
+// its (batch row, direction) streams longest first (sru_length_order_kernel,
+// into the workspace's order region); returns the order, or null to keep the
+// natural one.
+sru_status maybe_order(const uint8_t* mask, int* order_ws, int64_t L, int64_t B, int n_dir, int64_t ctas,
+                       int64_t per_wave, cudaStream_t st, const int** order) {
+    *order = nullptr;
+    if (mask == nullptr || order_ws == nullptr || B > sru::kOrderMaxB || B < 2 || ctas <= per_wave) return SRU_OK;
+    sru::sru_length_order_kernel<<<1, sru::kOrderThreads, 0, st>>>(mask, (int)L, (int)B, n_dir, order_ws);
+    SRU_CUDA_TRY(cudaGetLastError());
+    *order = order_ws;
+    return SRU_OK;
+}
+
 template <typename UT>
 sru_status launch_fwd_seq(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
-                          float* h, float* c_T, float* ckpt, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
-                          cudaStream_t st) {
+                          float* h, float* c_T, float* ckpt, int* order_ws, int64_t L, int64_t B, int64_t d, int n_dir,
+                          float alpha, cudaStream_t st) {
     static_assert(sru::kFwdStages == 4, "stage dispatch below covers 2..4");
     const int resident[5] = {0, 0, fwd_resident<UT, 2>(), fwd_resident<UT, 3>(), fwd_resident<UT, 4>()};
     const int64_t ctas = ((d + kSeqCJ - 1) / kSeqCJ) * B * n_dir;
     const int S = pick_stages(ctas, resident, 4);
+    const int* order = nullptr;
+    sru_status s = maybe_order(mask, order_ws, L, B, n_dir, ctas, (int64_t)sm_count() * resident[S], st, &order);
+    if (s != SRU_OK) return s;
     // h through TMA stores: for unmasked grids of about 5 or more CTAs per SM (measured)
     if (S >= 3 && mask == nullptr && ctas * 10 >= (int64_t)sm_count() * 48)
-        return S == 3 ? launch_fwd_seq_s<UT, 3, true>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st)
-                      : launch_fwd_seq_s<UT, 4, true>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+        return S == 3 ? launch_fwd_seq_s<UT, 3, true>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st)
+                      : launch_fwd_seq_s<UT, 4, true>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
     switch (S) {
-        case 2: return launch_fwd_seq_s<UT, 2>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
-        case 3: return launch_fwd_seq_s<UT, 3>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
-        default: return launch_fwd_seq_s<UT, 4>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+        case 2: return launch_fwd_seq_s<UT, 2>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
+        case 3: return launch_fwd_seq_s<UT, 3>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
+        default: return launch_fwd_seq_s<UT, 4>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
     }
 }
 
 template <typename UT, typename DUT, bool ACC, int DIR, int S>
 sru_status launch_bwd_seq_s(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
                             const float* ckpt, const float* dc_T, DUT* dU, float* dx, double* partial, float* dc0,
-                            int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
+                            const int* order, int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
     using Lay = sru::BwdLayout<UT, ACC, kSeqCJ, S>;
     auto kern = sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR, kSeqCJ, S>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
     dim3 grid((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)B, 1);
     kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.du, mp.dxo, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
-                                              (int)L, (int)B, (int)d, n_dir, alpha);
+                                              order, (int)L, (int)B, (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
@@ -540,27 +560,34 @@ int bwd_resident() {
 template <typename UT, typename DUT, bool ACC, int DIR>
 sru_status launch_bwd_seq_dir(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
                               const float* ckpt, const float* dc_T, DUT* du, float* dx, double* partial, float* dc0,
-                              int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
+                              int* order_ws, const int** order, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
+                              cudaStream_t st) {
     static_assert(sru::kBwdStages == 3, "stage dispatch below covers 2..3");
     const int resident[4] = {0, 0, bwd_resident<UT, DUT, ACC, DIR, 2>(), bwd_resident<UT, DUT, ACC, DIR, 3>()};
     const int64_t ctas = ((d + kSeqCJ - 1) / kSeqCJ) * B;
-    if (pick_stages(ctas, resident, 3) == 2)
-        return launch_bwd_seq_s<UT, DUT, ACC, DIR, 2>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d,
-                                                      n_dir, alpha, st);
-    return launch_bwd_seq_s<UT, DUT, ACC, DIR, 3>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir,
-                                                  alpha, st);
+    const int S = pick_stages(ctas, resident, 3);
+    if (DIR == 0) {  // one order for both directions' launches
+        sru_status s = maybe_order(mask, order_ws, L, B, n_dir, ctas, (int64_t)sm_count() * resident[S], st, order);
+        if (s != SRU_OK) return s;
+    }
+    if (S == 2)
+        return launch_bwd_seq_s<UT, DUT, ACC, DIR, 2>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, *order, L, B,
+                                                      d, n_dir, alpha, st);
+    return launch_bwd_seq_s<UT, DUT, ACC, DIR, 3>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, *order, L, B, d,
+                                                  n_dir, alpha, st);
 }
 
 template <typename UT, typename DUT>
 sru_status launch_bwd_seq(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask, const float* ckpt,
-                          const float* dc_T, void* dU, float* dx, double* partial, float* dc0, int64_t L, int64_t B,
-                          int64_t d, int n_dir, float alpha, cudaStream_t st) {
+                          const float* dc_T, void* dU, float* dx, double* partial, float* dc0, int* order_ws,
+                          int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
     DUT* du = reinterpret_cast<DUT*>(dU);
-    sru_status s = launch_bwd_seq_dir<UT, DUT, false, 0>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d,
-                                                         n_dir, alpha, st);
+    const int* order = nullptr;
+    sru_status s = launch_bwd_seq_dir<UT, DUT, false, 0>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, order_ws,
+                                                         &order, L, B, d, n_dir, alpha, st);
     if (s != SRU_OK || n_dir == 1) return s;
-    return launch_bwd_seq_dir<UT, DUT, true, 1>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, L, B, d, n_dir,
-                                                alpha, st);
+    return launch_bwd_seq_dir<UT, DUT, true, 1>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, order_ws, &order, L,
+                                                B, d, n_dir, alpha, st);
 }
 
 sru_status reset_scan_flags(unsigned* flags, int64_t n, cudaStream_t st) {
@@ -858,6 +885,7 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
         !map_f32_rows(&mp.h, h, L, B * n_dir, d, cj))
         return SRU_ERR_INVALID;
     float* ckpt = workspace ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.ckpt_off) : nullptr;
+    int* order_ws = workspace ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + w.order_off) : nullptr;
     if (scan) {
         const sru::ScanState ss = scan_state(workspace, w, flags);
         if (u_t == SRU_BF16)
@@ -865,8 +893,8 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
         return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, ckpt, ss, L, B, d, n_dir, alpha, st);
     }
     if (u_t == SRU_BF16)
-        return launch_fwd_seq<__nv_bfloat16>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
-    return launch_fwd_seq<float>(mp, v, b, c0, mask, h, c_T, ckpt, L, B, d, n_dir, alpha, st);
+        return launch_fwd_seq<__nv_bfloat16>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st);
+    return launch_fwd_seq<float>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st);
 }
 
 sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, const float* b, const float* c0,
@@ -912,6 +940,7 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const float* ckpt = reinterpret_cast<const float*>(ws + w.ckpt_off);
     double* partial = reinterpret_cast<double*>(ws + w.partial_off);
+    int* order_ws = reinterpret_cast<int*>(ws + w.order_off);
     const bool ub = u_t == SRU_BF16, db16 = du_t == SRU_BF16;
     if (scan) {
         const sru::ScanState ss = scan_state(workspace, w, flags);
@@ -927,14 +956,14 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
                                                      alpha, st, (flags & SRU_FLAG_V_ZERO) != 0);
     } else {
         if (ub)
-            s = db16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L,
+            s = db16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, order_ws, L,
                                                                     B, d, n_dir, alpha, st)
-                     : launch_bwd_seq<__nv_bfloat16, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
+                     : launch_bwd_seq<__nv_bfloat16, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, order_ws, L, B, d,
                                                             n_dir, alpha, st);
         else
-            s = db16 ? launch_bwd_seq<float, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d,
+            s = db16 ? launch_bwd_seq<float, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, order_ws, L, B, d,
                                                             n_dir, alpha, st)
-                     : launch_bwd_seq<float, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, L, B, d, n_dir,
+                     : launch_bwd_seq<float, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, order_ws, L, B, d, n_dir,
                                                     alpha, st);
     }
     if (s != SRU_OK) return s;

@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
     const __grid_constant__ CUtensorMap map_h, const float* __restrict__ v, const float* __restrict__ bias,
     const float* __restrict__ c0, const uint8_t* __restrict__ mask, float* __restrict__ h, float* __restrict__ c_T,
-    float* __restrict__ ckpt, int L, int B, int d, int n_dir, float alpha) {
+    float* __restrict__ ckpt, const int* __restrict__ order, int L, int B, int d, int n_dir, float alpha) {
     using Lay = FwdLayout<UT, CJ, S>;
     // STAGE_H: full chunks leave through a TMA store of h written over the
     // stage's x tile; a stage is refilled one iteration after its store was
@@ -259,8 +259,10 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
 
     const int tid = threadIdx.x, lane = tid & 31, cj = 2 * tid;
     const int j0 = blockIdx.x * CJ, j = j0 + cj;
-    const int b = blockIdx.y, dir = blockIdx.z;
-    const int bd = b * n_dir + dir;
+    // grid (d tiles, B, n_dir), or with `order` (d tiles, B * n_dir): the
+    // (batch row, direction) streams longest first (padded layers)
+    const int bd = order != nullptr ? order[blockIdx.y] : (int)(blockIdx.y * n_dir + blockIdx.z);
+    const int b = bd / n_dir, dir = bd % n_dir;
     const bool jok = j < d;  // d is even, so the pair is either in or out
     const int nch = (L + kChunkT - 1) / kChunkT;
 
@@ -583,8 +585,8 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     const __grid_constant__ CUtensorMap map_dh, const __grid_constant__ CUtensorMap map_du,
     const __grid_constant__ CUtensorMap map_dxo, const float* __restrict__ v, const float* __restrict__ bias,
     const uint8_t* __restrict__ mask, const float* __restrict__ ckpt, const float* __restrict__ dc_T, DUT* __restrict__ dU,
-    float* __restrict__ dx, double* __restrict__ partial, float* __restrict__ dc0, int L, int B, int d,
-    int n_dir, float alpha) {
+    float* __restrict__ dx, double* __restrict__ partial, float* __restrict__ dc0, const int* __restrict__ order, int L,
+    int B, int d, int n_dir, float alpha) {
     using Lay = BwdLayout<UT, ACC_DX, CJ, S>;
     // Full chunks leave through TMA stores of the stage they came in on (dU over
     // U, dx over x): a stage is refilled one iteration after its store was
@@ -598,7 +600,8 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     const int tid = threadIdx.x, lane = tid & 31, cj = 2 * tid;
     const int j0 = blockIdx.x * CJ, j = j0 + cj;
     constexpr int dir = DIR;
-    const int b = blockIdx.y;
+    // with `order`, the batch rows longest first (its entries are (b, dir) streams, n_dir per row)
+    const int b = order != nullptr ? order[blockIdx.y * n_dir] / n_dir : (int)blockIdx.y;
     const int bd = b * n_dir + dir;
     const bool jok = j < d;
     const int nch = (L + kChunkT - 1) / kChunkT;
@@ -757,6 +760,41 @@ __global__ void __launch_bounds__(kRedCols * kRedSlices) sru_reduce_dvdb_kernel(
         dv[(dir * 2 + q) * d + j] = (float)t;
     else
         db[(dir * 2 + q - 2) * d + j] = (float)t;
+}
+
+// Launch order of a padded layer's (batch row, direction) streams, longest
+// first.  A row's work is its number of kChunkT-step chunks holding a valid
+// (unpadded) step: padded chunks cost only their zero outputs.  With every
+// CTA walking a whole sequence, taking the long rows first lets the short ones
+// fill the SMs behind them (longest-processing-time-first), instead of each
+// wave of resident CTAs lasting as long as its longest row.  One block; rows
+// of equal work keep their index order, so the order is deterministic.
+//   order[r * n_dir + dir] = b * n_dir + dir for the row b of rank r.
+constexpr int kOrderThreads = 1024;
+constexpr int kOrderMaxB = 2048;
+__global__ void __launch_bounds__(kOrderThreads) sru_length_order_kernel(const uint8_t* __restrict__ mask, int L,
+                                                                         int B, int n_dir, int* __restrict__ order) {
+    __shared__ int work[kOrderMaxB];
+    const int nch = (L + kChunkT - 1) / kChunkT;
+    for (int b = threadIdx.x; b < B; b += blockDim.x) work[b] = 0;
+    __syncthreads();
+    for (long long idx = threadIdx.x; idx < (long long)B * nch; idx += blockDim.x) {
+        const int b = (int)(idx % B), c = (int)(idx / B);  // consecutive threads: consecutive rows, coalesced
+        const int t1 = min(L, (c + 1) * kChunkT);
+        bool any = false;
+        for (int t = c * kChunkT; t < t1; ++t) any |= mask[(size_t)t * B + b] == 0;
+        if (any) atomicAdd(&work[b], 1);
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        const int wb = work[b];
+        int rank = 0;
+        for (int o = 0; o < B; ++o) {
+            const int wo = work[o];
+            rank += (wo > wb) || (wo == wb && o < b);
+        }
+        for (int dir = 0; dir < n_dir; ++dir) order[rank * n_dir + dir] = b * n_dir + dir;
+    }
 }
 
 // L == 0: the final state is the initial state.
