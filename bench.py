@@ -435,14 +435,17 @@ def _layer_lm_train_fused(dev, flush, sru):
 def _layer_bidir(dev, flush, sru):
     # bidirectional padded layer, 2 directions
     lay = _Layer(2048, 64, 1024, 2, 3, dev, masked=True, project=True)
-    e = _gemm_entries(lay, flush)
-    e.update(_recurrence_entries(lay, flush, [("", 0)], tag="_masked"))
+    # the latency-bound recurrences first, before the products draw the power cap
+    e = _recurrence_entries(lay, flush, [("", 0)], tag="_masked")
     e["valid_fraction"] = lay.valid
+    mask = lay.mask
+    lay.mask, lay.valid = None, 1.0
+    e.update(_recurrence_entries(lay, flush, [("", 0)], tag="_unmasked"))
+    lay.mask = mask
+    e.update(_gemm_entries(lay, flush))
     t_f = _time_ms(lambda: sru.sru_forward_fused(lay.X, lay.W, lay.x, lay.v, lay.b, lay.h, lay.cT, lay.ws,
                                                  mask=lay.mask, bidirectional=True, U=lay.U), flush)
     e["layer_fused_with_U_masked"] = _fused_entry(lay, t_f, with_u=True)
-    lay.mask, lay.valid = None, 1.0
-    e.update(_recurrence_entries(lay, flush, [("", 0)], tag="_unmasked"))
     return {"bidir_masked L2048 B64 d1024 x2": e}
 
 
@@ -549,27 +552,34 @@ def run_ours(args):
     if world > 1:
         reducer = GradReducer([dW, dv, db])  # one NCCL all-reduce of the parameter gradients
 
+    fused = args.forward == "fused"
+    names = (["forward_fused"] if fused else ["project", "forward"]) + ["backward", "project_dX", "project_dW"]
+
     def step(ev=None, bufs=None):
-        """One training step; bufs = (X, x, dh, dx, dW, dv, db, dc0, reducer) or the default set."""
+        """One training step; bufs = (X, x, dh, dx, dW, dv, db, dc0, reducer) or the default set.
+        ev: CUDA events recorded between the phases (len(names) + 1)."""
         Xb, xb, dhb, dxb, dWb, dvb, dbb, dc0b, red = (bufs if bufs is not None
                                                       else (X, x, dh, dx, dW, dv, db, dc0, reducer))
-        if ev is not None:
-            ev[0].record(stream)
-        sru.sru_project(Xb, W, U)
-        if ev is not None:
-            ev[1].record(stream)
-        sru.sru_forward(U, xb, v, b, h, cT, c0=c0, workspace=ws)
-        if ev is not None:
-            ev[2].record(stream)
+        marks = iter(ev) if ev is not None else None
+
+        def mark():
+            if marks is not None:
+                next(marks).record(stream)
+        mark()
+        if fused:  # Eq. (1) and Eqs. (2)-(5) in one kernel; U and the checkpoints stored for the backward
+            sru.sru_forward_fused(Xb, W, xb, v, b, h, cT, ws, c0=c0, U=U)
+            mark()
+        else:
+            sru.sru_project(Xb, W, U)
+            mark()
+            sru.sru_forward(U, xb, v, b, h, cT, c0=c0, workspace=ws)
+            mark()
         sru.sru_backward(U, xb, v, b, dhb, ws, dU, dxb, dvb, dbb, dc0b, c0=c0)
-        if ev is not None:
-            ev[3].record(stream)
+        mark()
         sru.sru_project_backward(dU, Xb, W, dX=dxb, accumulate=True)
-        if ev is not None:
-            ev[4].record(stream)
+        mark()
         sru.sru_project_backward(dU, Xb, W, dW=dWb)
-        if ev is not None:
-            ev[5].record(stream)
+        mark()
         if red is not None:  # data-parallel gradient sum over ranks (batch sharding)
             red()
 
@@ -580,7 +590,7 @@ def run_ours(args):
         raise RuntimeError(f"device status {st} after warm-up")
 
     # ---- device-timed region
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -598,7 +608,6 @@ def run_ours(args):
     st = sru.sru_sync_status()
     if st != 0:
         raise RuntimeError(f"device status {st} in the timed region")
-    names = ["project", "forward", "backward", "project_dX", "project_dW"]
     phase_ms = {n: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
                 for i, n in enumerate(names)}
     t = torch.tensor([elapsed_ms], device=dev)
@@ -697,13 +706,16 @@ def run_ours(args):
         gemm_flops = 2.0 * M * N * K
         traffic, traffic_src = load_traffic()
         traffic = traffic.get(WORKLOAD, {})
-        gemm_ms = {n: phase_ms[n] for n in ("project", "project_dX", "project_dW")}
+        tensor_phases = [n for n in ("forward_fused", "project", "project_dX", "project_dW") if n in phase_ms]
+        gemm_ms = {n: phase_ms[n] for n in tensor_phases}
         dom = max(gemm_ms, key=gemm_ms.get)
         peak_kind, peak_tc = tensor_peak(peaks, clocks)
         ach_tc = gemm_flops / (gemm_ms[dom] / 1e3) / 1e12
         fwd_bytes = 14.0 * L * B * d
         bwd_bytes = 24.0 * L * B * d
-        ach_f = fwd_bytes / (phase_ms["forward"] / 1e3) / 1e9
+        # the fused forward moves X, W, x, h and U (stored for the backward) instead of U twice
+        fused_bytes = 2.0 * L * B * d + 6.0 * d * d + 14.0 * L * B * d
+        ach_f = (fused_bytes if fused else fwd_bytes) / (phase_ms["forward_fused" if fused else "forward"] / 1e3) / 1e9
         ach_b = bwd_bytes / (phase_ms["backward"] / 1e3) / 1e9
         sm = clocks.get("sm_mhz")
         line = {
@@ -711,7 +723,9 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16 GEMM + f32 recurrence",
             "data": "synthetic", "config": config,
-            "roofline": {"bound": "tensor", "kernel": f"tc_gemm_pair_kernel ({dom})", "achieved": ach_tc,
+            "roofline": {"bound": "tensor",
+                         "kernel": ("sru_fused_fwd_kernel (forward_fused)" if dom == "forward_fused"
+                                    else f"tc_gemm_pair_kernel ({dom})"), "achieved": ach_tc,
                          "peak": peak_tc, "unit": "TFLOP/s", "frac": ach_tc / peak_tc,
                          "traffic": traffic.get(dom), "traffic_unit": "bytes per launch (ncu dram read+write)",
                          "traffic_source": traffic_src,
@@ -724,8 +738,12 @@ def run_ours(args):
                          "algorithmic_per_launch": f"2*M*N*K = {gemm_flops:.4g} flop"},
             "roofline_recurrence": {
                 "bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
-                "forward": {"achieved": ach_f, "frac": ach_f / peaks["hbm_gbs"], "bytes": fwd_bytes,
-                            "ms": phase_ms["forward"], "traffic": traffic.get("forward")},
+                "forward": {"achieved": ach_f, "frac": ach_f / peaks["hbm_gbs"],
+                            "bytes": fused_bytes if fused else fwd_bytes,
+                            "kernel": "sru_fused_fwd_kernel (projection fused; the product bounds it)" if fused
+                            else "sru_fwd_seq_kernel",
+                            "ms": phase_ms["forward_fused" if fused else "forward"],
+                            "traffic": traffic.get("forward_fused" if fused else "forward")},
                 "backward": {"achieved": ach_b, "frac": ach_b / peaks["hbm_gbs"], "bytes": bwd_bytes,
                              "ms": phase_ms["backward"], "traffic": traffic.get("backward")},
                 "traffic_source": traffic_src,
@@ -733,7 +751,8 @@ def run_ours(args):
             "phase_ms": phase_ms,
             "e2e": {"value": cfg.tokens * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 6 * args.steps,
+            "gpu_launches": (5 if fused else 6) * args.steps,
+            "forward_path": args.forward,
             "clocks": clocks,
         }
         if workloads is not None:
@@ -920,6 +939,9 @@ def main():
     ap.add_argument("--workload", choices=["train", "decode"], default="train",
                     help="train: the layer training step (the headline); decode: batch-1 token steps")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--forward", choices=["fused", "separate"], default="separate",
+                    help="training step's forward: sru_forward_fused (projection and recurrence in one kernel) or "
+                         "sru_project then sru_forward")
     ap.add_argument("--only", choices=sorted(WORKLOAD_LAYERS), default=None,
                     help="run only this layer of the per-workload block and print it (for profiling one kernel)")
     ap.add_argument("--skip-workloads", action="store_true",

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/sru.h"
 #include "sru_gemm.cuh"
@@ -472,32 +473,37 @@ int pick_stages(int64_t ctas, const int* resident, int smax) {
 }
 
 // Channels per CTA of the sequential kernels (CJ/2 threads; at least 32 so
-// that a CTA has a lane for each of a chunk's 16 rows).
-#ifndef SRU_SEQ_CJ
-#define SRU_SEQ_CJ 64
+// that a CTA has a lane for each of a chunk's 16 rows): 64 (one warp), or 32
+// (half a warp) for grids that leave SMs idle at 64 -- fewer than two CTAs
+// per SM -- so that the same channels spread over twice as many CTAs.
+// SRU_SEQ_CJ_FORCE (32 or 64) fixes the width at build time for measurements.
+#ifndef SRU_SEQ_CJ_FORCE
+#define SRU_SEQ_CJ_FORCE 0
 #endif
-constexpr int kSeqCJ = SRU_SEQ_CJ;
-static_assert(kSeqCJ >= 32 && kSeqCJ % 32 == 0, "sequential tile width");
+int seq_cj(int64_t B, int64_t d, int n_dir_per_launch) {
+    if (SRU_SEQ_CJ_FORCE == 32 || SRU_SEQ_CJ_FORCE == 64) return SRU_SEQ_CJ_FORCE;
+    return ((d + 63) / 64) * B * n_dir_per_launch < 2 * (int64_t)sm_count() ? 32 : 64;
+}
 
-template <typename UT, int S, bool STAGE_H = false>
+template <typename UT, int CJ, int S, bool STAGE_H = false>
 sru_status launch_fwd_seq_s(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
                             float* h, float* c_T, float* ckpt, const int* order, int64_t L, int64_t B, int64_t d,
                             int n_dir, float alpha, cudaStream_t st) {
-    using Lay = sru::FwdLayout<UT, kSeqCJ, S>;
-    auto kern = sru::sru_fwd_seq_kernel<UT, kSeqCJ, S, STAGE_H>;
+    using Lay = sru::FwdLayout<UT, CJ, S>;
+    auto kern = sru::sru_fwd_seq_kernel<UT, CJ, S, STAGE_H>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
-    const dim3 grid = order != nullptr ? dim3((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)(B * n_dir), 1)
-                                       : dim3((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)B, (unsigned)n_dir);
-    kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.h, v, b, c0, mask, h, c_T, ckpt, order, (int)L, (int)B,
+    const dim3 grid = order != nullptr ? dim3((unsigned)((d + CJ - 1) / CJ), (unsigned)(B * n_dir), 1)
+                                       : dim3((unsigned)((d + CJ - 1) / CJ), (unsigned)B, (unsigned)n_dir);
+    kern<<<grid, CJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.h, v, b, c0, mask, h, c_T, ckpt, order, (int)L, (int)B,
                                               (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
 
-template <typename UT, int S>
+template <typename UT, int CJ, int S>
 int fwd_resident() {
-    return resident_ctas(reinterpret_cast<const void*>(sru::sru_fwd_seq_kernel<UT, kSeqCJ, S>), kSeqCJ / 2,
-                         sru::FwdLayout<UT, kSeqCJ, S>::SMEM);
+    return resident_ctas(reinterpret_cast<const void*>(sru::sru_fwd_seq_kernel<UT, CJ, S>), CJ / 2,
+                         sru::FwdLayout<UT, CJ, S>::SMEM);
 }
 
 // A padded layer whose grid needs more than one wave of resident CTAs takes
@@ -514,79 +520,79 @@ sru_status maybe_order(const uint8_t* mask, int* order_ws, int64_t L, int64_t B,
     return SRU_OK;
 }
 
-template <typename UT>
+template <typename UT, int CJ>
 sru_status launch_fwd_seq(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
                           float* h, float* c_T, float* ckpt, int* order_ws, int64_t L, int64_t B, int64_t d, int n_dir,
                           float alpha, cudaStream_t st) {
     static_assert(sru::kFwdStages == 4, "stage dispatch below covers 2..4");
-    const int resident[5] = {0, 0, fwd_resident<UT, 2>(), fwd_resident<UT, 3>(), fwd_resident<UT, 4>()};
-    const int64_t ctas = ((d + kSeqCJ - 1) / kSeqCJ) * B * n_dir;
+    const int resident[5] = {0, 0, fwd_resident<UT, CJ, 2>(), fwd_resident<UT, CJ, 3>(), fwd_resident<UT, CJ, 4>()};
+    const int64_t ctas = ((d + CJ - 1) / CJ) * B * n_dir;
     const int S = pick_stages(ctas, resident, 4);
     const int* order = nullptr;
     sru_status s = maybe_order(mask, order_ws, L, B, n_dir, ctas, (int64_t)sm_count() * resident[S], st, &order);
     if (s != SRU_OK) return s;
     // h through TMA stores: for unmasked grids of about 5 or more CTAs per SM (measured)
     if (S >= 3 && mask == nullptr && ctas * 10 >= (int64_t)sm_count() * 48)
-        return S == 3 ? launch_fwd_seq_s<UT, 3, true>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st)
-                      : launch_fwd_seq_s<UT, 4, true>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
+        return S == 3 ? launch_fwd_seq_s<UT, CJ, 3, true>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st)
+                      : launch_fwd_seq_s<UT, CJ, 4, true>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
     switch (S) {
-        case 2: return launch_fwd_seq_s<UT, 2>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
-        case 3: return launch_fwd_seq_s<UT, 3>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
-        default: return launch_fwd_seq_s<UT, 4>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
+        case 2: return launch_fwd_seq_s<UT, CJ, 2>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
+        case 3: return launch_fwd_seq_s<UT, CJ, 3>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
+        default: return launch_fwd_seq_s<UT, CJ, 4>(mp, v, b, c0, mask, h, c_T, ckpt, order, L, B, d, n_dir, alpha, st);
     }
 }
 
-template <typename UT, typename DUT, bool ACC, int DIR, int S>
+template <typename UT, typename DUT, bool ACC, int DIR, int CJ, int S>
 sru_status launch_bwd_seq_s(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
                             const float* ckpt, const float* dc_T, DUT* dU, float* dx, double* partial, float* dc0,
                             const int* order, int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
-    using Lay = sru::BwdLayout<UT, ACC, kSeqCJ, S>;
-    auto kern = sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR, kSeqCJ, S>;
+    using Lay = sru::BwdLayout<UT, ACC, CJ, S>;
+    auto kern = sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR, CJ, S>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), Lay::SMEM));
-    dim3 grid((unsigned)((d + kSeqCJ - 1) / kSeqCJ), (unsigned)B, 1);
-    kern<<<grid, kSeqCJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.du, mp.dxo, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
+    dim3 grid((unsigned)((d + CJ - 1) / CJ), (unsigned)B, 1);
+    kern<<<grid, CJ / 2, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, mp.du, mp.dxo, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
                                               order, (int)L, (int)B, (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
 
-template <typename UT, typename DUT, bool ACC, int DIR, int S>
+template <typename UT, typename DUT, bool ACC, int DIR, int CJ, int S>
 int bwd_resident() {
-    return resident_ctas(reinterpret_cast<const void*>(sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR, kSeqCJ, S>),
-                         kSeqCJ / 2, sru::BwdLayout<UT, ACC, kSeqCJ, S>::SMEM);
+    return resident_ctas(reinterpret_cast<const void*>(sru::sru_bwd_seq_kernel<UT, DUT, ACC, DIR, CJ, S>),
+                         CJ / 2, sru::BwdLayout<UT, ACC, CJ, S>::SMEM);
 }
 
 // One direction's backward launch.  ACC: dx += this direction's part.
-template <typename UT, typename DUT, bool ACC, int DIR>
+template <typename UT, typename DUT, bool ACC, int DIR, int CJ>
 sru_status launch_bwd_seq_dir(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask,
                               const float* ckpt, const float* dc_T, DUT* du, float* dx, double* partial, float* dc0,
                               int* order_ws, const int** order, int64_t L, int64_t B, int64_t d, int n_dir, float alpha,
                               cudaStream_t st) {
     static_assert(sru::kBwdStages == 3, "stage dispatch below covers 2..3");
-    const int resident[4] = {0, 0, bwd_resident<UT, DUT, ACC, DIR, 2>(), bwd_resident<UT, DUT, ACC, DIR, 3>()};
-    const int64_t ctas = ((d + kSeqCJ - 1) / kSeqCJ) * B;
+    const int resident[4] = {0, 0, bwd_resident<UT, DUT, ACC, DIR, CJ, 2>(), bwd_resident<UT, DUT, ACC, DIR, CJ, 3>()};
+    const int64_t ctas = ((d + CJ - 1) / CJ) * B;
     const int S = pick_stages(ctas, resident, 3);
     if (DIR == 0) {  // one order for both directions' launches
         sru_status s = maybe_order(mask, order_ws, L, B, n_dir, ctas, (int64_t)sm_count() * resident[S], st, order);
         if (s != SRU_OK) return s;
     }
     if (S == 2)
-        return launch_bwd_seq_s<UT, DUT, ACC, DIR, 2>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, *order, L, B,
+        return launch_bwd_seq_s<UT, DUT, ACC, DIR, CJ, 2>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, *order, L, B,
                                                       d, n_dir, alpha, st);
-    return launch_bwd_seq_s<UT, DUT, ACC, DIR, 3>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, *order, L, B, d,
+    return launch_bwd_seq_s<UT, DUT, ACC, DIR, CJ, 3>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, *order, L, B, d,
                                                   n_dir, alpha, st);
 }
 
-template <typename UT, typename DUT>
+template <typename UT, typename DUT, int CJ>
 sru_status launch_bwd_seq(const RecMaps& mp, const float* v, const float* b, const uint8_t* mask, const float* ckpt,
                           const float* dc_T, void* dU, float* dx, double* partial, float* dc0, int* order_ws,
                           int64_t L, int64_t B, int64_t d, int n_dir, float alpha, cudaStream_t st) {
     DUT* du = reinterpret_cast<DUT*>(dU);
     const int* order = nullptr;
-    sru_status s = launch_bwd_seq_dir<UT, DUT, false, 0>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, order_ws,
+    sru_status s = launch_bwd_seq_dir<UT, DUT, false, 0, CJ>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, order_ws,
                                                          &order, L, B, d, n_dir, alpha, st);
     if (s != SRU_OK || n_dir == 1) return s;
-    return launch_bwd_seq_dir<UT, DUT, true, 1>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, order_ws, &order, L,
+    return launch_bwd_seq_dir<UT, DUT, true, 1, CJ>(mp, v, b, mask, ckpt, dc_T, du, dx, partial, dc0, order_ws, &order, L,
                                                 B, d, n_dir, alpha, st);
 }
 
@@ -879,7 +885,7 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
     } else if (scan) {
         return SRU_ERR_INVALID;  // the scan needs its flags and aggregates
     }
-    const int cj = scan ? sru::kRecCJ : kSeqCJ;  // TMA box width of the kernel that runs
+    const int cj = scan ? sru::kRecCJ : seq_cj(B, d, n_dir);  // TMA box width of the kernel that runs
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj) ||
         !map_f32_rows(&mp.h, h, L, B * n_dir, d, cj))
@@ -892,9 +898,13 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
             return launch_fwd_scan<__nv_bfloat16>(mp, b, c0, mask, h, c_T, ckpt, ss, L, B, d, n_dir, alpha, st);
         return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, ckpt, ss, L, B, d, n_dir, alpha, st);
     }
-    if (u_t == SRU_BF16)
-        return launch_fwd_seq<__nv_bfloat16>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st);
-    return launch_fwd_seq<float>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st);
+    if (cj == 32)
+        return u_t == SRU_BF16
+                   ? launch_fwd_seq<__nv_bfloat16, 32>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st)
+                   : launch_fwd_seq<float, 32>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st);
+    return u_t == SRU_BF16
+               ? launch_fwd_seq<__nv_bfloat16, 64>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st)
+               : launch_fwd_seq<float, 64>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st);
 }
 
 sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, const float* b, const float* c0,
@@ -931,7 +941,7 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
     const WsLayout w = ws_layout(L, B, d, n_dir, flags);
     if (workspace_bytes < w.total) return SRU_ERR_INVALID;
     const bool scan = use_bwd_scan(flags, L, B, d, n_dir, u_t);
-    const int cj = scan ? sru::kRecCJ : kSeqCJ;
+    const int cj = scan ? sru::kRecCJ : seq_cj(B, d, 1);
     RecMaps mp;
     if (!map_u_tensor(&mp.u, U, u_t, L, B, d, n_dir, cj) || !map_f32_rows(&mp.x, x, L, B, d, cj) ||
         !map_f32_rows(&mp.dh, dh, L, B * n_dir, d, cj) || !map_u_tensor(&mp.du, dU, du_t, L, B, d, n_dir, cj) ||
@@ -955,16 +965,20 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
                      : launch_bwd_scan<float, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, ss, L, B, d, n_dir,
                                                      alpha, st, (flags & SRU_FLAG_V_ZERO) != 0);
     } else {
-        if (ub)
-            s = db16 ? launch_bwd_seq<__nv_bfloat16, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, order_ws, L,
-                                                                    B, d, n_dir, alpha, st)
-                     : launch_bwd_seq<__nv_bfloat16, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, order_ws, L, B, d,
-                                                            n_dir, alpha, st);
+        // one (U type, dU type, channel width) instantiation per combination
+        auto run = [&](auto ut, auto dut, auto cjc) {
+            using UT = decltype(ut);
+            using DUT = decltype(dut);
+            return launch_bwd_seq<UT, DUT, decltype(cjc)::value>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
+                                                                 order_ws, L, B, d, n_dir, alpha, st);
+        };
+        using C32 = std::integral_constant<int, 32>;
+        using C64 = std::integral_constant<int, 64>;
+        const __nv_bfloat16 hb{};
+        if (cj == 32)
+            s = ub ? (db16 ? run(hb, hb, C32{}) : run(hb, 0.f, C32{})) : (db16 ? run(0.f, hb, C32{}) : run(0.f, 0.f, C32{}));
         else
-            s = db16 ? launch_bwd_seq<float, __nv_bfloat16>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, order_ws, L, B, d,
-                                                            n_dir, alpha, st)
-                     : launch_bwd_seq<float, float>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0, order_ws, L, B, d, n_dir,
-                                                    alpha, st);
+            s = ub ? (db16 ? run(hb, hb, C64{}) : run(hb, 0.f, C64{})) : (db16 ? run(0.f, hb, C64{}) : run(0.f, 0.f, C64{}));
     }
     if (s != SRU_OK) return s;
     const int64_t rows = scan ? scan_chunks(L) * B : B;

@@ -135,24 +135,31 @@ struct FusedArgs {
     int write_u;           // store the U tile with map_u
 };
 
+// x of one tile half (rows i0 .. i0+15, those before L), for one thread's
+// channel pair; loaded ahead of use so that its latency is off the chain.
+__device__ __forceinline__ void load_x_half(float2 (&wx)[kChunkT], const float* __restrict__ xp, int i0, int nrows,
+                                            size_t tstride_x, bool jok) {
+#pragma unroll
+    for (int i = 0; i < kChunkT; ++i)
+        wx[i] = (jok && i0 + i < nrows) ? load_pair(xp + (size_t)(i0 + i) * tstride_x) : f2(0.f);
+}
+
 // Walk kChunkT steps of one tile half (rows i0 .. i0+15 of the tile in time
-// order, visited in the direction's order) for one thread's channel pair.
+// order, visited in the direction's order) for one thread's channel pair,
+// with the half's x already in registers.
 template <int DIR>
 __device__ __forceinline__ float2 fused_chunk(uint32_t utile, int q, int l, int i0, uint32_t valid16, float2 c,
-                                              const GateParams2& p, float2 alpha2, const float* __restrict__ xp,
-                                              float* __restrict__ hp, size_t tstride_x, size_t tstride_h, bool jok,
-                                              int nrows) {
+                                              const GateParams2& p, float2 alpha2, const float2 (&wx)[kChunkT],
+                                              float* __restrict__ hp, size_t tstride_h, bool jok, int nrows) {
     constexpr uint32_t kFull = (1u << kChunkT) - 1u;
     if (valid16 == kFull) {
         uint32_t wc[kChunkT], wf[kChunkT], wr[kChunkT];
-        float2 wx[kChunkT];
 #pragma unroll
         for (int i = 0; i < kChunkT; ++i) {
             const int r = (i0 + i) * kBb + q;
             wc[i] = lds_u32(utile_word(utile, r, 0, l));
             wf[i] = lds_u32(utile_word(utile, r, 1, l));
             wr[i] = lds_u32(utile_word(utile, r, 2, l));
-            wx[i] = jok ? load_pair(xp + (size_t)(i0 + i) * tstride_x) : f2(0.f);
         }
         float2 hv[kChunkT];
 #pragma unroll
@@ -180,7 +187,7 @@ __device__ __forceinline__ float2 fused_chunk(uint32_t utile, int q, int l, int 
             c = sru_cell2(c, bf16x2_to_float2(lds_u32(utile_word(utile, r, 0, l))),
                           bf16x2_to_float2(lds_u32(utile_word(utile, r, 1, l))),
                           bf16x2_to_float2(lds_u32(utile_word(utile, r, 2, l))), p, f, rr);
-            const float2 ax = mul2(alpha2, jok ? load_pair(xp + (size_t)(i0 + i) * tstride_x) : f2(0.f));
+            const float2 ax = mul2(alpha2, wx[i]);
             hv = fma2(rr, sub2(c, ax), ax);
         }
         if (jok) store_pair(hp + (size_t)(i0 + i) * tstride_h, hv);
@@ -361,28 +368,71 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after_sync();
+            // ---- this warp's stream: batch row b, channel pair (j, j+1).  Everything the
+            // walk reads from global memory is requested now, so that its latency passes
+            // under the accumulator transpose below.
+            const int b0 = bgp * 2 * kBb + (int)rank * kBb;
+            const int js0 = js * kCh;
+            const int b = b0 + q;
+            const bool brow = b < B;
+            const int j = js0 + cj;
+            const bool jok = brow && j < d;
+            const int bd = b * n_dir + dir;
+            const int t_base = tp * kTt;
+            const int nrows = min(kTt, L - t_base);
+            const int i_first = dir == 0 ? 0 : kTt - kChunkT;  // first tile half in walk order
+            unsigned* flag = a.flags + (size_t)bd * njs + js;
+            const float* xp = a.x + (size_t)t_base * tstride_x + (size_t)b * d + j;
+            float2 xa[kChunkT];
+            load_x_half(xa, xp, i_first, nrows, tstride_x, jok);
+            GateParams2 p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
+            float2 c = f2(0.f);
+            unsigned seen = (unsigned)tt;  // tiles of this stream already published
+            if (jok) {
+                p = make_gate_params2(load_pair(a.v + (dir * 2 + 0) * d + j), load_pair(a.v + (dir * 2 + 1) * d + j),
+                                      load_pair(a.bias + (dir * 2 + 0) * d + j),
+                                      load_pair(a.bias + (dir * 2 + 1) * d + j));
+            }
+            if (brow) {
+                if (tt == 0) {
+                    if (jok && a.c0 != nullptr) c = load_pair(a.c0 + (size_t)bd * d + j);
+                } else {
+                    // the carry is read after the flag's acquire: valid if the flag already says so
+                    seen = ld_acquire_gpu(flag);
+                    if (jok) c = ld_relaxed_gpu2(a.carry + (size_t)bd * d + j);
+                }
+            }
+            // rows of this tile that exist (t < L) and are not padded, bit i = step t_base + i
+            bool vrow = brow && lane < nrows;
+            if (vrow && a.mask != nullptr) vrow = a.mask[(size_t)(t_base + lane) * B + b] == 0;
+            const uint32_t valid = __ballot_sync(0xffffffffu, vrow);
             // ---- accumulator rows (t, b) -> bf16 U tile, 128-byte swizzled lines [t][b][gate]
             {
                 const int r = q * 32 + lane;
 #pragma unroll 1
-                for (int c6 = 0; c6 < 6; ++c6) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * kAccCols + c6 * 32,
-                                       v);
+                for (int c2 = 0; c2 < 3; ++c2) {
+                    uint32_t v[2][32];
+                    const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * kAccCols + c2 * 64;
+                    tmem_ld_32x32b_x32(taddr, v[0]);
+                    tmem_ld_32x32b_x32(taddr + 32, v[1]);
                     tc_wait_ld();
-                    const int half = c6 / 3, g = c6 % 3;
-                    const uint32_t line = (uint32_t)(r * 3 + g);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        uint32_t w[4];
+                    for (int k = 0; k < 2; ++k) {
+                        const int c6 = 2 * c2 + k;
+                        const int half = c6 / 3, g = c6 % 3;
+                        const uint32_t line = (uint32_t)(r * 3 + g);
 #pragma unroll
-                        for (int k2 = 0; k2 < 4; ++k2) {
-                            __nv_bfloat162 two = __floats2bfloat162_rn(__uint_as_float(v[e * 8 + 2 * k2]),
-                                                                       __uint_as_float(v[e * 8 + 2 * k2 + 1]));
-                            w[k2] = *reinterpret_cast<uint32_t*>(&two);
+                        for (int e = 0; e < 4; ++e) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int k2 = 0; k2 < 4; ++k2) {
+                                __nv_bfloat162 two = __floats2bfloat162_rn(__uint_as_float(v[k][e * 8 + 2 * k2]),
+                                                                           __uint_as_float(v[k][e * 8 + 2 * k2 + 1]));
+                                w[k2] = *reinterpret_cast<uint32_t*>(&two);
+                            }
+                            const uint32_t chunk = (uint32_t)(half * 4 + e);
+                            st_shared_v4(utile + line * 128u + ((chunk ^ (line & 7u)) << 4), w[0], w[1], w[2], w[3]);
                         }
-                        const uint32_t chunk = (uint32_t)(half * 4 + e);
-                        st_shared_v4(utile + line * 128u + ((chunk ^ (line & 7u)) << 4), w[0], w[1], w[2], w[3]);
                     }
                 }
             }
@@ -391,77 +441,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)acc * 8u);  // accumulator free
             fence_proxy_async_shared();  // the tile's writes, visible to the TMA store
             epi_sync();
-            const int b0 = bgp * 2 * kBb + (int)rank * kBb;
-            const int js0 = js * kCh;
             if (issuer && a.write_u && b0 < B) {  // (a group wholly beyond B has no rows to store)
-                tma_store_5d(&map_u, utile_p, js0, 0, dir, b0, tp * kTt);
+                tma_store_5d(&map_u, utile_p, js0, 0, dir, b0, t_base);
                 bulk_commit_group();
                 stored = true;
             }
-            // ---- Eqs. (2)-(5) for batch row b over the tile's steps, channel pair (j, j+1)
-            const int b = b0 + q;
-            if (b < B) {
-                const int j = js0 + cj;
-                const bool jok = j < d;
-                const int bd = b * n_dir + dir;
-                GateParams2 p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
-                if (jok)
-                    p = make_gate_params2(load_pair(a.v + (dir * 2 + 0) * d + j), load_pair(a.v + (dir * 2 + 1) * d + j),
-                                          load_pair(a.bias + (dir * 2 + 0) * d + j),
-                                          load_pair(a.bias + (dir * 2 + 1) * d + j));
-                // state entering the tile: c0, or the carry the previous tile of this stream published
-                unsigned* flag = a.flags + (size_t)bd * njs + js;
-                float2 c = f2(0.f);
-                if (tt == 0) {
-                    if (jok && a.c0 != nullptr) c = load_pair(a.c0 + (size_t)bd * d + j);
-                } else {
-                    if (lane == 0) {
-                        if (ld_acquire_gpu(flag) < (unsigned)tt) {
-                            const uint64_t t0 = globaltimer_ns();
-                            while (ld_acquire_gpu(flag) < (unsigned)tt) {
-                                if (*reinterpret_cast<volatile unsigned*>(&g_error_word) != 0u) break;
-                                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                                    record_error(kErrTimeoutScan);
-                                    break;
-                                }
-                                __nanosleep(32);
-                            }
+            if (!brow) continue;
+            // ---- Eqs. (2)-(5) over the tile's steps in the direction's order
+            if (__any_sync(0xffffffffu, seen < (unsigned)tt)) {
+                // the previous tile of this stream has not published yet: wait (bounded), re-read
+                if (lane == 0) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_gpu(flag) < (unsigned)tt) {
+                        if (*reinterpret_cast<volatile unsigned*>(&g_error_word) != 0u) break;
+                        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                            record_error(kErrTimeoutScan);
+                            break;
                         }
+                        __nanosleep(32);
                     }
-                    __syncwarp();
-                    if (jok) c = ld_relaxed_gpu2(a.carry + (size_t)bd * d + j);
                 }
-                // rows of this tile that exist (t < L) and are not padded, bit i = step tp*kTt + i
-                const int t_base = tp * kTt;
-                bool vrow = t_base + lane < L;
-                if (vrow && a.mask != nullptr) vrow = a.mask[(size_t)(t_base + lane) * B + b] == 0;
-                const uint32_t valid = __ballot_sync(0xffffffffu, vrow);
-                const int nrows = min(kTt, L - t_base);
-                const float* xp = a.x + (size_t)t_base * tstride_x + (size_t)b * d + j;
-                float* hp = a.h + (size_t)t_base * tstride_h + (size_t)bd * d + j;
-#pragma unroll 1
-                for (int hh = 0; hh < kTt / kChunkT; ++hh) {
-                    const int half = dir == 0 ? hh : kTt / kChunkT - 1 - hh;
-                    const int i0 = half * kChunkT;
-                    const int tc = (t_base + i0) / kChunkT;
-                    if (tc >= nch) continue;  // wholly beyond L
-                    if (a.ckpt != nullptr && jok) store_pair(a.ckpt + ((size_t)tc * B * n_dir + bd) * d + j, c);
-                    const uint32_t v16 = (valid >> i0) & ((1u << kChunkT) - 1u);
-                    c = dir == 0 ? fused_chunk<0>(utile, q, lane, i0, v16, c, p, alpha2, xp, hp, tstride_x, tstride_h,
-                                                  jok, nrows)
-                                 : fused_chunk<1>(utile, q, lane, i0, v16, c, p, alpha2, xp, hp, tstride_x, tstride_h,
-                                                  jok, nrows);
-                }
-                if (tt + 1 < nT) {
-                    if (jok) st_relaxed_gpu2(a.carry + (size_t)bd * d + j, c);
-                    __syncwarp();
-                    if (lane == 0) {
-                        __threadfence();
-                        st_release_gpu(flag, (unsigned)(tt + 1));
-                    }
-                } else if (jok) {
-                    store_pair(a.c_T + (size_t)bd * d + j, c);
-                }
+                __syncwarp();
+                (void)ld_acquire_gpu(flag);
+                if (jok) c = ld_relaxed_gpu2(a.carry + (size_t)bd * d + j);
+            }
+            float* hp = a.h + (size_t)t_base * tstride_h + (size_t)bd * d + j;
+            float2 xb[kChunkT];
+            const int i_second = kTt - kChunkT - i_first;
+            load_x_half(xb, xp, i_second, nrows, tstride_x, jok);  // under the first half's walk
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int i0 = hh == 0 ? i_first : i_second;
+                const int tc = (t_base + i0) / kChunkT;
+                if (tc >= nch) continue;  // wholly beyond L
+                if (a.ckpt != nullptr && jok) store_pair(a.ckpt + ((size_t)tc * B * n_dir + bd) * d + j, c);
+                const uint32_t v16 = (valid >> i0) & ((1u << kChunkT) - 1u);
+                if (dir == 0)
+                    c = fused_chunk<0>(utile, q, lane, i0, v16, c, p, alpha2, hh == 0 ? xa : xb, hp, tstride_h, jok,
+                                       nrows);
+                else
+                    c = fused_chunk<1>(utile, q, lane, i0, v16, c, p, alpha2, hh == 0 ? xa : xb, hp, tstride_h, jok,
+                                       nrows);
+            }
+            if (tt + 1 < nT) {
+                if (jok) st_relaxed_gpu2(a.carry + (size_t)bd * d + j, c);
+                __syncwarp();
+                if (lane == 0) st_release_gpu(flag, (unsigned)(tt + 1));  // orders the warp's carry stores before it
+            } else if (jok) {
+                store_pair(a.c_T + (size_t)bd * d + j, c);
             }
         }
         if (issuer && stored) bulk_wait_group<0>();  // every U store has landed
