@@ -264,7 +264,9 @@ sru_status sru_project_factored_backward(const void* dU, const void* X, const vo
  * are rounded to bf16 (they are tensor-core operands), scores and A are fp32.
  * The workspace (>= sru_attention_workspace_bytes(L, B, d')) holds Q, K, V,
  * one batch row's scores and probabilities, A and R.  Limits: d, d', N and L
- * multiples of 8, L <= 65536.  The per-batch products are separate launches.
+ * multiples of 8, L <= 65536.  With causal, the score tiles wholly above the
+ * diagonal and P V's reduction beyond each row tile's diagonal are skipped
+ * (those probabilities are 0).
  */
 size_t sru_attention_workspace_bytes(int64_t L, int64_t B, int64_t dp);
 sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv, const void* Wo, float alpha,

@@ -308,14 +308,18 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
 // `batches` products of one shape in one launch of the pair kernel (operand
 // maps from map_kmajor_b / map_mnmajor_b with the batch at coordinate BPA /
 // BPB); product z writes out + z * out_bstride elements.
-template <bool A_MN, bool B_MN, int OUT, int BPA, int BPB>
+// CAUSAL (square causal attention products, see sru::gemm::pair_unit): 1 = only
+// the output tiles on or below the diagonal, 2 = reduction cut at each row
+// tile's diagonal.
+template <bool A_MN, bool B_MN, int OUT, int BPA, int BPB, int CAUSAL = 0>
 sru_status launch_tc_gemm_batched(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
                                   int64_t Kr, int64_t ldo, int64_t batches, int64_t out_bstride, cudaStream_t st) {
     if (!kGemmPair) return SRU_ERR_UNSUPPORTED;
-    auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT, BPA, BPB>;
+    auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT, BPA, BPB, CAUSAL>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
-    const int64_t units =
-        ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN) * batches;
+    const int64_t mt = (R + sru::gemm::P_BM - 1) / sru::gemm::P_BM, nt = (C + sru::gemm::P_BN - 1) / sru::gemm::P_BN;
+    if (CAUSAL == 1 && R != C) return SRU_ERR_UNSUPPORTED;
+    const int64_t units = (CAUSAL == 1 ? mt * (mt + 1) / 2 : mt * nt) * batches;
     if (units >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
     const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
     CUtensorMap unused;  // batched launches store directly (no output map)
@@ -472,18 +476,13 @@ int pick_stages(int64_t ctas, const int* resident, int smax) {
     return best;
 }
 
-// Channels per CTA of the sequential kernels (CJ/2 threads; at least 32 so
-// that a CTA has a lane for each of a chunk's 16 rows): 64 (one warp), or 32
-// (half a warp) for grids that leave SMs idle at 64 -- fewer than two CTAs
-// per SM -- so that the same channels spread over twice as many CTAs.
-// SRU_SEQ_CJ_FORCE (32 or 64) fixes the width at build time for measurements.
-#ifndef SRU_SEQ_CJ_FORCE
-#define SRU_SEQ_CJ_FORCE 0
-#endif
-int seq_cj(int64_t B, int64_t d, int n_dir_per_launch) {
-    if (SRU_SEQ_CJ_FORCE == 32 || SRU_SEQ_CJ_FORCE == 64) return SRU_SEQ_CJ_FORCE;
-    return ((d + 63) / 64) * B * n_dir_per_launch < 2 * (int64_t)sm_count() ? 32 : 64;
-}
+// Channels per CTA of the sequential kernels: 64 (one warp, two channels per
+// thread).  Measured on B200, a 32-channel (half-warp) CTA was no faster where
+// the 64-channel grid leaves SMs idle (L256 B32 d512: 38.9 us forward and
+// 48.1 us backward at either width) and slower for the backward of dense grids
+// (L1024 B16 d2048: 163 -> 194 us), so the kernels are built at 64 only.
+constexpr int kSeqCJ = 64;
+int seq_cj(int64_t, int64_t, int) { return kSeqCJ; }
 
 template <typename UT, int CJ, int S, bool STAGE_H = false>
 sru_status launch_fwd_seq_s(const RecMaps& mp, const float* v, const float* b, const float* c0, const uint8_t* mask,
@@ -898,13 +897,10 @@ sru_status sru_forward(const void* U, int u_t, const float* x, const float* v, c
             return launch_fwd_scan<__nv_bfloat16>(mp, b, c0, mask, h, c_T, ckpt, ss, L, B, d, n_dir, alpha, st);
         return launch_fwd_scan<float>(mp, b, c0, mask, h, c_T, ckpt, ss, L, B, d, n_dir, alpha, st);
     }
-    if (cj == 32)
-        return u_t == SRU_BF16
-                   ? launch_fwd_seq<__nv_bfloat16, 32>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st)
-                   : launch_fwd_seq<float, 32>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st);
     return u_t == SRU_BF16
-               ? launch_fwd_seq<__nv_bfloat16, 64>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st)
-               : launch_fwd_seq<float, 64>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st);
+               ? launch_fwd_seq<__nv_bfloat16, kSeqCJ>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha,
+                                                        st)
+               : launch_fwd_seq<float, kSeqCJ>(mp, v, b, c0, mask, h, c_T, ckpt, order_ws, L, B, d, n_dir, alpha, st);
 }
 
 sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, const float* b, const float* c0,
@@ -972,13 +968,9 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
             return launch_bwd_seq<UT, DUT, decltype(cjc)::value>(mp, v, b, mask, ckpt, dc_T, dU, dx, partial, dc0,
                                                                  order_ws, L, B, d, n_dir, alpha, st);
         };
-        using C32 = std::integral_constant<int, 32>;
-        using C64 = std::integral_constant<int, 64>;
+        using C64 = std::integral_constant<int, kSeqCJ>;
         const __nv_bfloat16 hb{};
-        if (cj == 32)
-            s = ub ? (db16 ? run(hb, hb, C32{}) : run(hb, 0.f, C32{})) : (db16 ? run(0.f, hb, C32{}) : run(0.f, 0.f, C32{}));
-        else
-            s = ub ? (db16 ? run(hb, hb, C64{}) : run(hb, 0.f, C64{})) : (db16 ? run(0.f, hb, C64{}) : run(0.f, 0.f, C64{}));
+        s = ub ? (db16 ? run(hb, hb, C64{}) : run(hb, 0.f, C64{})) : (db16 ? run(0.f, hb, C64{}) : run(0.f, 0.f, C64{}));
     }
     if (s != SRU_OK) return s;
     const int64_t rows = scan ? scan_chunks(L) * B : B;
@@ -1224,7 +1216,8 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
         if (!map_kmajor_b(&ma, Q + b0 * dp, L, dp, B * dp, g, dp, sru::gemm::BM, 1) ||
             !map_kmajor_b(&mb, KV + b0 * 2 * dp, L, dp, B * 2 * dp, g, 2 * dp, kGemmBRows, 1))
             return SRU_ERR_INVALID;
-        s = launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st);
+        s = causal ? launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st)
+                   : launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st);
         if (s != SRU_OK) return s;
         sru::sru_softmax_rows_kernel<<<blocks_for((size_t)(g * L), sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
             S, P, (int)L, (int)(g * L), scale, causal ? 1 : 0);
@@ -1234,8 +1227,10 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
         if (!map_kmajor_b(&ma, P, L, L, L, g, L * L, sru::gemm::BM, 2) ||
             !map_mnmajor_b(&mb, KV + b0 * 2 * dp + dp, dp, L, B * 2 * dp, g, 2 * dp, 1))
             return SRU_ERR_INVALID;
-        s = launch_tc_gemm_batched<false, true, sru::gemm::kOutF32, 2, 1>(ma, mb, A + b0 * dp, L, dp, L, B * dp, g,
-                                                                           dp, st);
+        s = causal ? launch_tc_gemm_batched<false, true, sru::gemm::kOutF32, 2, 1, 2>(ma, mb, A + b0 * dp, L, dp, L,
+                                                                                     B * dp, g, dp, st)
+                   : launch_tc_gemm_batched<false, true, sru::gemm::kOutF32, 2, 1>(ma, mb, A + b0 * dp, L, dp, L, B * dp,
+                                                                                 g, dp, st);
         if (s != SRU_OK) return s;
     }
     sru::sru_residual_norm_kernel<<<blocks_for((size_t)M, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(

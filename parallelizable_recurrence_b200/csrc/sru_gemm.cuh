@@ -365,7 +365,44 @@ __device__ __forceinline__ void tma_load_tile_pair(void* dst, const CUtensorMap*
 // map_out (non-batched launches): the output as a 2-D tensor (N columns, M
 // rows, row stride ldo) of the output type, box 32 x 32, swizzle 64 B (bf16)
 // or 128 B (fp32).  Batched launches store directly and ignore it.
-template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0>
+// A work unit of the pair kernel: output tile (tm, tn) of batch z and its
+// k-block range [kb_lo, kb_hi).  CAUSAL (batched square products of SRU++'s
+// causal attention, tiles of P_BM = P_BN rows):
+//   1  scores S = Q K^T: only the tiles on or below the diagonal (tn <= tm);
+//      the tiles above it hold only masked entries, which the softmax never reads;
+//   2  A = P V: the reduction over s stops at the end of the row tile, past
+//      which every probability is 0.
+struct PairUnit {
+    int z, tm, tn, kb_lo, kb_hi;
+};
+template <int CAUSAL>
+__device__ __forceinline__ PairUnit pair_unit(int u, int m_tiles, int n_tiles, int splits, int kblocks, int kper) {
+    PairUnit w;
+    if (CAUSAL == 1) {
+        const int tri = m_tiles * (m_tiles + 1) / 2;
+        w.z = u / tri;
+        const int t = u % tri;
+        int tm = (int)((sqrtf(8.0f * (float)t + 1.0f) - 1.0f) * 0.5f);
+        while (tm * (tm + 1) / 2 > t) --tm;
+        while ((tm + 1) * (tm + 2) / 2 <= t) ++tm;
+        w.tm = tm;
+        w.tn = t - tm * (tm + 1) / 2;
+        w.kb_lo = 0;
+        w.kb_hi = kblocks;
+        return w;
+    }
+    const int tiles = m_tiles * n_tiles;
+    w.z = u / (tiles * splits);
+    const int uu = u % (tiles * splits), tile = uu / splits;
+    w.tm = tile / n_tiles;
+    w.tn = tile % n_tiles;
+    w.kb_lo = (uu % splits) * kper;
+    w.kb_hi = min(kblocks, w.kb_lo + kper);
+    if (CAUSAL == 2) w.kb_hi = min(w.kb_hi, ((w.tm + 1) * P_BM + BK - 1) / BK);
+    return w;
+}
+
+template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0, int CAUSAL = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                         const __grid_constant__ CUtensorMap map_out, void* __restrict__ out, int M, int N, int K,
@@ -391,7 +428,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int kblocks = (K + BK - 1) / BK;
     // work unit u = (tile u / splits, K part u % splits); splits > 1 only with
     // kOutF32Red and at least one k-block per part (the host checks both)
-    const int units = tiles * splits * batches;  // batch-major, then tile, then K part
+    // batch-major, then tile, then K part (causal scores: the lower-triangle tiles only)
+    const int units = (CAUSAL == 1 ? m_tiles * (m_tiles + 1) / 2 : tiles * splits) * batches;
     const int kper = (kblocks + splits - 1) / splits;
 
     if (threadIdx.x == 0) {
@@ -429,11 +467,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             for (int u = pair_id; u < units && !*abort_flag; u += n_pairs) {
-                const int z = u / (tiles * splits), uu = u % (tiles * splits);
-                const int tile = uu / splits, kb_lo = (uu % splits) * kper;
-                const int kb_hi = min(kblocks, kb_lo + kper);
-                const int m0 = (tile / n_tiles) * P_BM + (int)rank * P_CM;
-                const int n0 = (tile % n_tiles) * P_BN + (int)rank * P_CN;
+                const PairUnit w = pair_unit<CAUSAL>(u, m_tiles, n_tiles, splits, kblocks, kper);
+                const int z = w.z, kb_lo = w.kb_lo, kb_hi = w.kb_hi;
+                const int m0 = w.tm * P_BM + (int)rank * P_CM;
+                const int n0 = w.tn * P_BN + (int)rank * P_CN;
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, kErrTimeoutMma) || *abort_flag) {
                         *abort_flag = 1;
@@ -476,7 +513,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             uint32_t phase = 0, nconsumed = 0;
             int it = 0;
             for (int u = pair_id; u < units && !*abort_flag; u += n_pairs, ++it) {
-                const int kb_lo = (u % splits) * kper, kb_hi = min(kblocks, kb_lo + kper);  // (units per batch % splits == 0)
+                const PairUnit w = pair_unit<CAUSAL>(u, m_tiles, n_tiles, splits, kblocks, kper);
+                const int kb_lo = w.kb_lo, kb_hi = w.kb_hi;
                 const int acc = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, kErrTimeoutEpilogue)) {
@@ -524,14 +562,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         int it = 0;
         uint32_t nstaged = 0;  // chunks this warp has handed to TMA stores
         for (int u = pair_id; u < units; u += n_pairs, ++it) {
-            const int z = u / (tiles * splits);
-            const int tile = (u % (tiles * splits)) / splits;
+            const PairUnit w = pair_unit<CAUSAL>(u, m_tiles, n_tiles, splits, kblocks, kper);
+            const int z = w.z;
             void* const zout = (BPA | BPB) != 0 ? static_cast<void*>(static_cast<uint8_t*>(out) +
                                                              (size_t)z * (size_t)out_bstride * (OUT == kOutBF16 ? 2 : 4))
                                         : out;
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
-            const int m0 = (tile / n_tiles) * P_BM + (int)rank * P_CM, n0 = (tile % n_tiles) * P_BN;
+            const int m0 = w.tm * P_BM + (int)rank * P_CM, n0 = w.tn * P_BN;
             const bool ok = mbar_wait(&tfull[acc], acc_phase, kErrTimeoutMma);
             if (!__all_sync(0xffffffffu, ok) || *abort_flag) {
                 *abort_flag = 1;

@@ -40,6 +40,8 @@ def _dev(bits):
     (256, 4, 512, 128, 0.25, True, False),
     (64, 2, 128, 32, 0.0, True, False),
     (4096, 3, 64, 16, 0.5, True, False),   # long rows: batch rows go in groups of 2 (score buffer bound)
+    (600, 2, 128, 32, 0.5, True, True),    # causal over 3 score tiles, the last one ragged
+    (600, 2, 128, 32, 0.5, False, False),  # the same without the mask: every tile computed
 ])
 def test_attention_producer_matches_oracle(sru, L, B, d, dp, alpha, causal, ln):
     rng = np.random.default_rng(L + B + d + dp)
