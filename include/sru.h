@@ -215,7 +215,7 @@ sru_status sru_forward_scan_noalloc(const void* U, int u_t, const float* x, cons
  *   of U is stored (inference).
  *   workspace: at least sru_workspace_bytes(L, B, d, bidirectional, flags) bytes
  *   for any flags (it also carries the state from one time tile to the next;
- *   its flags are cleared on the stream before the launch).
+ *   that region is cleared on the stream before the launch).
  * The kernel keeps one CTA on every SM of the device and hands the state of a
  * sequence between CTAs: do not run it concurrently with other work on the
  * same GPU (its bounded waits would expire: SRU_ERR_TIMEOUT at the next

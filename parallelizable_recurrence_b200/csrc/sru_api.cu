@@ -116,12 +116,12 @@ cudaError_t ensure_smem(const void* kernel, size_t bytes) {
 }
 
 // ---------------------------------------------------------- workspace layout
-// [checkpoints | fused-forward carries and flags | launch order | dv/db partial sums | scan
+// [checkpoints | fused-forward carry words | launch order | dv/db partial sums | scan
 //  flags | scan aggregates A, B, prefix].  The scan regions exist only when a
 // scan can run (see ws_has_scan); the offsets of the first two regions do not
 // depend on the flags.
 struct WsLayout {
-    size_t ckpt_off, carry_off, fflags_off, order_off, partial_off, flags_off, agg_a_off, agg_b_off, prefix_off, total;
+    size_t ckpt_off, carry_off, order_off, partial_off, flags_off, agg_a_off, agg_b_off, prefix_off, total;
     int64_t scan_items;
 };
 
@@ -138,9 +138,7 @@ WsLayout ws_layout(int64_t L, int64_t B, int64_t d, int n_dir, unsigned flags) {
     w.ckpt_off = off;
     off += round256((size_t)nch * B * n_dir * d * sizeof(float));
     w.carry_off = off;
-    off += round256((size_t)B * n_dir * d * sizeof(float));
-    w.fflags_off = off;
-    off += round256((size_t)B * n_dir * ((d + sru::fused::kCh - 1) / sru::fused::kCh) * sizeof(unsigned));
+    off += round256((size_t)B * n_dir * d * sizeof(unsigned long long));
     w.order_off = off;
     off += round256((size_t)B * n_dir * sizeof(int));
     w.partial_off = off;
@@ -1085,15 +1083,14 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
     fa.h = h;
     fa.c_T = c_T;
     fa.ckpt = U ? reinterpret_cast<float*>(ws + w.ckpt_off) : nullptr;
-    fa.carry = reinterpret_cast<float*>(ws + w.carry_off);
-    fa.flags = reinterpret_cast<unsigned*>(ws + w.fflags_off);
+    fa.carry = reinterpret_cast<unsigned long long*>(ws + w.carry_off);
     fa.L = (int)L;
     fa.B = (int)B;
     fa.d = (int)d;
     fa.n_dir = n_dir;
     fa.alpha = alpha;
     fa.write_u = U != nullptr;
-    SRU_CUDA_TRY(cudaMemsetAsync(fa.flags, 0, (size_t)B * n_dir * njs * sizeof(unsigned), st));
+    SRU_CUDA_TRY(cudaMemsetAsync(fa.carry, 0, (size_t)B * n_dir * d * sizeof(unsigned long long), st));
     auto kern = sru::fused::sru_fused_fwd_kernel;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::fused::kSmemBytes));
     const int64_t max_pairs = fused_resident_pairs();

@@ -29,11 +29,15 @@
 // Time tiles of one (batch row, direction, channel slice) stream are walked
 // in order but may run on different CTAs: items are dealt round-robin in
 // (time tile, stream) order, and the state leaving a tile is handed to the
-// next by a carry slot and a flag (release / acquire at GPU scope).  The MMAs
-// of every item run without waiting; only the epilogue's walk waits for its
-// predecessor's carry, which was dealt earlier.  Every CTA of the grid must be
-// resident (one per SM, grid <= SM count); waits are bounded (2 s) so that a
-// GPU shared with other work cannot hang the kernel.
+// next through one 64-bit word per channel holding the state and the number
+// of the tile that wrote it (tile + 1; the words are zeroed before the
+// launch).  An aligned 64-bit access is single-copy atomic, so the reader
+// that sees its predecessor's tile number in a word has that tile's state in
+// the same word: no flag, fence or second round trip.  The MMAs of every item
+// run without waiting; only the epilogue's walk waits for its predecessor's
+// carry, which was dealt earlier.  Every CTA of the grid must be resident
+// (one per SM, grid <= SM count); waits are bounded (2 s) so that a GPU
+// shared with other work cannot hang the kernel.
 #pragma once
 
 #include "sru_recurrence.cuh"
@@ -104,6 +108,21 @@ __device__ __forceinline__ void st_relaxed_gpu2(float* p, float2 v) {
     asm volatile("st.relaxed.gpu.global.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(v.x), "f"(v.y) : "memory");
 }
 
+// Tagged carry words of a channel pair: (tag << 32) | float bits, one 16-byte
+// access of two single-copy-atomic 64-bit elements.
+__device__ __forceinline__ void ld_carry2(const unsigned long long* p, unsigned& tag0, unsigned& tag1, float2& c) {
+    unsigned long long w0, w1;
+    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(w0), "=l"(w1) : "l"(p) : "memory");
+    tag0 = (unsigned)(w0 >> 32);
+    tag1 = (unsigned)(w1 >> 32);
+    c = make_float2(__uint_as_float((unsigned)w0), __uint_as_float((unsigned)w1));
+}
+__device__ __forceinline__ void st_carry2(unsigned long long* p, unsigned tag, float2 c) {
+    const unsigned long long hi = (unsigned long long)tag << 32;
+    const unsigned long long w0 = hi | __float_as_uint(c.x), w1 = hi | __float_as_uint(c.y);
+    asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(w0), "l"(w1) : "memory");
+}
+
 // Shared-memory address of the 32-bit word holding channels (2l, 2l+1) of
 // gate g at accumulator row r in the swizzled U tile.
 __device__ __forceinline__ uint32_t utile_word(uint32_t utile, int r, int g, int l) {
@@ -128,8 +147,8 @@ struct FusedArgs {
     float* h;              // (L, B, n_dir, d)
     float* c_T;            // (B, n_dir, d)
     float* ckpt;           // (ceil(L/16), B, n_dir, d) or null
-    float* carry;          // (B, n_dir, d): state handed from a time tile to the next
-    unsigned* flags;       // (B, n_dir, ceil(d/64)): time tiles published so far (zeroed before launch)
+    unsigned long long* carry;  // (B, n_dir, d): (tile + 1) << 32 | state bits, from a tile to the next
+                                //  (zeroed before the launch)
     int L, B, d, n_dir;
     float alpha;
     int write_u;           // store the U tile with map_u
@@ -381,13 +400,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int t_base = tp * kTt;
             const int nrows = min(kTt, L - t_base);
             const int i_first = dir == 0 ? 0 : kTt - kChunkT;  // first tile half in walk order
-            unsigned* flag = a.flags + (size_t)bd * njs + js;
+            unsigned long long* cw = a.carry + (size_t)bd * d + j;  // this pair's carry words
             const float* xp = a.x + (size_t)t_base * tstride_x + (size_t)b * d + j;
             float2 xa[kChunkT];
             load_x_half(xa, xp, i_first, nrows, tstride_x, jok);
             GateParams2 p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
             float2 c = f2(0.f);
-            unsigned seen = (unsigned)tt;  // tiles of this stream already published
+            bool have = true;  // the state entering the tile is known
             if (jok) {
                 p = make_gate_params2(load_pair(a.v + (dir * 2 + 0) * d + j), load_pair(a.v + (dir * 2 + 1) * d + j),
                                       load_pair(a.bias + (dir * 2 + 0) * d + j),
@@ -396,10 +415,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (brow) {
                 if (tt == 0) {
                     if (jok && a.c0 != nullptr) c = load_pair(a.c0 + (size_t)bd * d + j);
-                } else {
-                    // the carry is read after the flag's acquire: valid if the flag already says so
-                    seen = ld_acquire_gpu(flag);
-                    if (jok) c = ld_relaxed_gpu2(a.carry + (size_t)bd * d + j);
+                } else if (jok) {
+                    unsigned g0, g1;
+                    ld_carry2(cw, g0, g1, c);
+                    have = g0 == (unsigned)tt && g1 == (unsigned)tt;  // written by tile tt - 1
                 }
             }
             // rows of this tile that exist (t < L) and are not padded, bit i = step t_base + i
@@ -448,22 +467,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             if (!brow) continue;
             // ---- Eqs. (2)-(5) over the tile's steps in the direction's order
-            if (__any_sync(0xffffffffu, seen < (unsigned)tt)) {
-                // the previous tile of this stream has not published yet: wait (bounded), re-read
-                if (lane == 0) {
-                    const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire_gpu(flag) < (unsigned)tt) {
-                        if (*reinterpret_cast<volatile unsigned*>(&g_error_word) != 0u) break;
-                        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                            record_error(kErrTimeoutScan);
-                            break;
-                        }
-                        __nanosleep(32);
+            if (!have) {
+                // the previous tile of this stream has not handed over yet: re-read (bounded)
+                const uint64_t t0 = globaltimer_ns();
+                for (;;) {
+                    unsigned g0, g1;
+                    ld_carry2(cw, g0, g1, c);
+                    if (g0 == (unsigned)tt && g1 == (unsigned)tt) break;
+                    if (*reinterpret_cast<volatile unsigned*>(&g_error_word) != 0u) break;
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                        record_error(kErrTimeoutScan);
+                        break;
                     }
                 }
-                __syncwarp();
-                (void)ld_acquire_gpu(flag);
-                if (jok) c = ld_relaxed_gpu2(a.carry + (size_t)bd * d + j);
             }
             float* hp = a.h + (size_t)t_base * tstride_h + (size_t)bd * d + j;
             float2 xb[kChunkT];
@@ -484,9 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                        nrows);
             }
             if (tt + 1 < nT) {
-                if (jok) st_relaxed_gpu2(a.carry + (size_t)bd * d + j, c);
-                __syncwarp();
-                if (lane == 0) st_release_gpu(flag, (unsigned)(tt + 1));  // orders the warp's carry stores before it
+                if (jok) st_carry2(cw, (unsigned)(tt + 1), c);
             } else if (jok) {
                 store_pair(a.c_T + (size_t)bd * d + j, c);
             }
