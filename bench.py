@@ -939,7 +939,7 @@ def main():
     ap.add_argument("--workload", choices=["train", "decode"], default="train",
                     help="train: the layer training step (the headline); decode: batch-1 token steps")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--forward", choices=["fused", "separate"], default="separate",
+    ap.add_argument("--forward", choices=["fused", "separate"], default="fused",
                     help="training step's forward: sru_forward_fused (projection and recurrence in one kernel) or "
                          "sru_project then sru_forward")
     ap.add_argument("--only", choices=sorted(WORKLOAD_LAYERS), default=None,

@@ -734,6 +734,7 @@ sru_status noalloc_scratch_address(cudaStream_t st, void** out) {
 // kernel hands the state between CTAs, so its whole grid must be resident):
 // the occupancy calculator's count of co-resident 2-CTA clusters, cached per
 // device.
+template <int NS>
 int64_t fused_resident_pairs() {
     static std::mutex mu;
     static int cache[kMaxDevices] = {0};
@@ -741,18 +742,38 @@ int64_t fused_resident_pairs() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
     std::lock_guard<std::mutex> lock(mu);
     if (cache[dev] == 0) {
-        auto kern = sru::fused::sru_fused_fwd_kernel;
+        auto kern = sru::fused::sru_fused_fwd_kernel<NS>;
+        constexpr size_t smem = sru::fused::FusedShape<NS>::kSmem;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(2 * (sm_count() / 2)), 1, 1);
         cfg.blockDim = dim3(sru::fused::kThreads, 1, 1);
-        cfg.dynamicSmemBytes = sru::fused::kSmemBytes;
+        cfg.dynamicSmemBytes = smem;
         int n = 0;
-        if (ensure_smem(reinterpret_cast<const void*>(kern), sru::fused::kSmemBytes) != cudaSuccess ||
+        if (ensure_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess ||
             cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(kern), &cfg) != cudaSuccess)
             n = 0;
         cache[dev] = n > 0 ? (n < sm_count() / 2 ? n : sm_count() / 2) : -1;
     }
     return cache[dev];
+}
+
+template <int NS>
+sru_status launch_fused(const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& mu,
+                        const sru::fused::FusedArgs& fa, int64_t L, int64_t B, int64_t d, int n_dir, cudaStream_t st) {
+    const int64_t nT = (L + sru::fused::kTt - 1) / sru::fused::kTt;
+    const int64_t njg = ((d + sru::fused::kCh - 1) / sru::fused::kCh + NS - 1) / NS;
+    const int64_t nbgp = (B + 2 * sru::fused::kBb - 1) / (2 * sru::fused::kBb);
+    const int64_t items = nT * n_dir * nbgp * njg;
+    if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
+    auto kern = sru::fused::sru_fused_fwd_kernel<NS>;
+    constexpr size_t smem = sru::fused::FusedShape<NS>::kSmem;
+    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
+    const int64_t max_pairs = fused_resident_pairs<NS>();
+    if (max_pairs < 1) return cuda_fail(cudaErrorLaunchOutOfResources);
+    const int64_t pairs = items < max_pairs ? items : max_pairs;
+    kern<<<(unsigned)(2 * pairs), sru::fused::kThreads, smem, st>>>(mx, mw, mu, fa);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
 }
 
 }  // namespace
@@ -1043,11 +1064,6 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
         return SRU_ERR_INVALID;
     const WsLayout w = ws_layout(L, B, d, n_dir, SRU_FLAG_FORCE_SEQUENTIAL);  // the smallest layout
     if (workspace_bytes < w.total) return SRU_ERR_INVALID;
-    const int64_t nT = (L + sru::fused::kTt - 1) / sru::fused::kTt;
-    const int64_t njs = (d + sru::fused::kCh - 1) / sru::fused::kCh;
-    const int64_t nbgp = (B + 2 * sru::fused::kBb - 1) / (2 * sru::fused::kBb);
-    const int64_t items = nT * n_dir * nbgp * njs;
-    if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
     CUtensorMap mx, mw, mu;
     {
         const uint64_t dims[3] = {(uint64_t)d, (uint64_t)B, (uint64_t)L};
@@ -1091,14 +1107,10 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
     fa.alpha = alpha;
     fa.write_u = U != nullptr;
     SRU_CUDA_TRY(cudaMemsetAsync(fa.carry, 0, (size_t)B * n_dir * d * sizeof(unsigned long long), st));
-    auto kern = sru::fused::sru_fused_fwd_kernel;
-    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::fused::kSmemBytes));
-    const int64_t max_pairs = fused_resident_pairs();
-    if (max_pairs < 1) return cuda_fail(cudaErrorLaunchOutOfResources);
-    const int64_t pairs = items < max_pairs ? items : max_pairs;
-    kern<<<(unsigned)(2 * pairs), sru::fused::kThreads, sru::fused::kSmemBytes, st>>>(mx, mw, mu, fa);
-    SRU_CUDA_TRY(cudaGetLastError());
-    return SRU_OK;
+    // two 64-channel slices per work item where the per-item product is long
+    // enough to hide two slices' walks (d >= 1024); one otherwise
+    if (d >= 1024) return launch_fused<2>(mx, mw, mu, fa, L, B, d, n_dir, st);
+    return launch_fused<1>(mx, mw, mu, fa, L, B, d, n_dir, st);
 }
 
 sru_status sru_project_factored(const void* X, const void* Wq, const void* Wo, void* P, void* U, int u_t,

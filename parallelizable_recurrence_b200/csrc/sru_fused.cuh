@@ -52,16 +52,12 @@ constexpr int kCh = 64;                  // channels per item
 constexpr int kRows = kTt * kBb;         // 128 accumulator rows per CTA
 constexpr int kN = 3 * kCh;              // 192 accumulator columns
 constexpr int kBK = 64;                  // k per stage (one 128-byte swizzle row)
-constexpr int kStages = 6;
 constexpr uint32_t kABytes = kRows * kBK * 2;          // 16 KB of X per CTA
-constexpr uint32_t kBBytes = (kN / 2) * kBK * 2;       // 12 KB of W_cat per CTA
-constexpr uint32_t kStageBytes = kABytes + kBBytes;    // 28 KB
-constexpr uint32_t kUTileBytes = kRows * 3 * 128;      // 48 KB: [t][b][gate] lines of 64 bf16
+constexpr uint32_t kBBytes = (kN / 2) * kBK * 2;       // 12 KB of W_cat per CTA and slice
+constexpr uint32_t kUTileBytes = kRows * 3 * 128;      // 48 KB per slice: [t][b][gate] lines of 64 bf16
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCols = 256;                      // column offset of the second accumulator
+constexpr uint32_t kAccCols = 256;                      // column stride of accumulators
 constexpr int kThreads = 192;
-constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + kUTileBytes + 1024 + 256;
-static_assert(kSmemBytes <= 232448, "fused kernel shared memory");
 static_assert(kTt == 32, "one ballot covers a tile's rows");
 static_assert(kTt % kChunkT == 0, "checkpoint interval divides the tile");
 
@@ -214,21 +210,42 @@ __device__ __forceinline__ float2 fused_chunk(uint32_t utile, int q, int l, int 
     return c;
 }
 
+// Shape of a work item: NS 64-channel slices side by side (N = 192 * NS
+// accumulator columns as NS MMAs of N = 192 sharing the X tile).  NS = 2
+// halves the X traffic per flop (the L2-to-SM feed bounds a 192-column
+// product) at the price of a single-buffered accumulator and a ring of 3
+// stages; NS = 1 keeps two accumulators and 6 stages, for layers whose
+// per-item product is short and whose chains lie on the critical path.
+template <int NS>
+struct FusedShape {
+    static constexpr int kStages = NS == 1 ? 6 : 3;
+    static constexpr uint32_t kStageBytes = kABytes + NS * kBBytes;
+    static constexpr int kAccBufs = NS == 1 ? 2 : 1;  // accumulators in flight
+    static constexpr size_t kSmem = (size_t)kStages * kStageBytes + NS * kUTileBytes + 1024 + 256;
+    static_assert(kSmem <= 232448, "fused kernel shared memory");
+    static_assert(NS == 1 || NS == 2, "slices per item");
+};
+
 // map_x: X as 3-D (d, B, L) bf16, box (64, kBb, kTt), 128-byte swizzle.
 // map_w: W_cat as 3-D (d, d, n_dir*3) bf16, box (64, 32, 3), 128-byte swizzle.
 // map_u: U as 5-D (d, 3, n_dir, B, L) bf16, box (64, 3, 1, kBb, kTt), 128-byte
 //        swizzle (only used when a.write_u).
+template <int NS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     sru_fused_fwd_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                          const __grid_constant__ CUtensorMap map_u, const FusedArgs a) {
+    using Sh = FusedShape<NS>;
+    constexpr int kStages = Sh::kStages;
+    constexpr uint32_t kStageBytes = Sh::kStageBytes;
+    constexpr int kAccBufs = Sh::kAccBufs;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* utile_p = smem + kStages * kStageBytes;  // 1024-aligned
-    uint64_t* full = reinterpret_cast<uint64_t*>(utile_p + kUTileBytes);
+    uint8_t* utile_p = smem + kStages * kStageBytes;  // 1024-aligned; NS tiles of kUTileBytes
+    uint64_t* full = reinterpret_cast<uint64_t*>(utile_p + NS * kUTileBytes);
     uint64_t* empty = full + kStages;
     uint64_t* tfull = empty + kStages;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* drain = tempty + 2;
+    uint64_t* tempty = tfull + kAccBufs;
+    uint64_t* drain = tempty + kAccBufs;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     volatile uint32_t* consumed = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
@@ -239,8 +256,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int L = a.L, B = a.B, d = a.d, n_dir = a.n_dir;
     const int nT = (L + kTt - 1) / kTt;                     // time tiles
     const int njs = (d + kCh - 1) / kCh;                    // channel slices
+    const int njg = (njs + NS - 1) / NS;                    // groups of NS slices (one item each)
     const int nbgp = (B + 2 * kBb - 1) / (2 * kBb);         // pairs of batch groups
-    const int streams = n_dir * nbgp * njs;
+    const int streams = n_dir * nbgp * njg;
     const int items = nT * streams;
     const int kblocks = (d + kBK - 1) / kBK;
 
@@ -249,7 +267,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int acc = 0; acc < 2; ++acc) {
+        for (int acc = 0; acc < kAccBufs; ++acc) {
             mbar_init(&tfull[acc], 1);
             mbar_init(&tempty[acc], 8);  // leader's: the 4 epilogue warps of each CTA
         }
@@ -272,15 +290,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
     const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
 
-    // item u -> (walk-order time tile, direction, batch-group pair, channel slice)
-    auto decode = [&](int u, int& tt, int& dir, int& bgp, int& js) {
+    // item u -> (walk-order time tile, direction, batch-group pair, slice group)
+    auto decode = [&](int u, int& tt, int& dir, int& bgp, int& jg) {
         tt = u / streams;
         int s = u % streams;
-        js = s % njs;
-        s /= njs;
+        jg = s % njg;
+        s /= njg;
         bgp = s % nbgp;
         dir = s / nbgp;
     };
+    // accumulator of buffer acc, slice s: TMEM columns from (acc + s) * kAccCols
+    // (one of acc, s is always 0)
 
     if (warp == 0) {
         if (lane == 0) {
@@ -289,11 +309,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             for (int u = pair_id; u < items && !*abort_flag; u += n_pairs) {
-                int tt, dir, bgp, js;
-                decode(u, tt, dir, bgp, js);
+                int tt, dir, bgp, jg;
+                decode(u, tt, dir, bgp, jg);
                 const int tp = dir == 0 ? tt : nT - 1 - tt;
                 const int b0 = bgp * 2 * kBb + (int)rank * kBb;
-                const int j0 = js * kCh + (int)rank * (kCh / 2);
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, kErrTimeoutMma) || *abort_flag) {
                         *abort_flag = 1;
@@ -303,7 +322,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t bar = leader_full0 + (uint32_t)stage * 8u;
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
                     tma_load_3d_pair(a_dst, &map_x, bar, kb * kBK, b0, tp * kTt);
-                    tma_load_3d_pair(a_dst + kABytes, &map_w, bar, kb * kBK, j0, dir * 3);
+#pragma unroll
+                    for (int s = 0; s < NS; ++s)
+                        tma_load_3d_pair(a_dst + kABytes + s * kBBytes, &map_w, bar, kb * kBK,
+                                         (jg * NS + s) * kCh + (int)rank * (kCh / 2), dir * 3);
                     ++issued;
                     if (++stage == kStages) {
                         stage = 0;
@@ -324,14 +346,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             uint32_t phase = 0, nconsumed = 0;
             int it = 0;
             for (int u = pair_id; u < items && !*abort_flag; u += n_pairs, ++it) {
-                const int acc = it & 1;
-                const uint32_t acc_phase = (it >> 1) & 1;
+                const int acc = it % kAccBufs;
+                const uint32_t acc_phase = (it / kAccBufs) & 1;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, kErrTimeoutEpilogue)) {
                     *abort_flag = 1;
                     break;
                 }
                 tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + (uint32_t)acc * kAccCols;
                 bool ok = true;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&full[stage], phase, kErrTimeoutLoad)) {
@@ -340,11 +361,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after_sync();
                     const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
-                    const uint32_t b_addr = a_addr + kABytes;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
-                        tc_mma_bf16_pair(d_tmem, sdesc_sw128(a_addr + kk * 32), sdesc_sw128(b_addr + kk * 32), idesc,
-                                         (kb | kk) != 0 ? 1u : 0u);
+#pragma unroll
+                        for (int s = 0; s < NS; ++s)
+                            tc_mma_bf16_pair(tmem_base + (uint32_t)(acc + s) * kAccCols, sdesc_sw128(a_addr + kk * 32),
+                                             sdesc_sw128(a_addr + kABytes + s * kBBytes + kk * 32), idesc,
+                                             (kb | kk) != 0 ? 1u : 0u);
                     tc_commit_pair_mc(&empty[stage], 0x3);
                     *consumed = ++nconsumed;
                     if (++stage == kStages) {
@@ -364,8 +387,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else {
         // ---------------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;  // TMEM lane quarter = this warp's batch row in the group
-        const uint32_t utile = smem_u32(utile_p);
-        const bool issuer = warp == 2 && lane == 0;  // sends the U tile by TMA
+        const uint32_t utile0 = smem_u32(utile_p);
+        const bool issuer = warp == 2 && lane == 0;  // sends the U tiles by TMA
         const int cj = 2 * lane;
         const float2 alpha2 = f2(a.alpha);
         const size_t tstride_x = (size_t)B * d;
@@ -374,70 +397,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         int it = 0;
         bool stored = false;
         for (int u = pair_id; u < items; u += n_pairs, ++it) {
-            int tt, dir, bgp, js;
-            decode(u, tt, dir, bgp, js);
+            int tt, dir, bgp, jg;
+            decode(u, tt, dir, bgp, jg);
             const int tp = dir == 0 ? tt : nT - 1 - tt;
-            const int acc = it & 1;
-            const uint32_t acc_phase = (it >> 1) & 1;
+            const int acc = it % kAccBufs;
+            const uint32_t acc_phase = (it / kAccBufs) & 1;
             const bool ok = mbar_wait(&tfull[acc], acc_phase, kErrTimeoutMma);
-            // the previous item's U store must be done reading the tile before it is rewritten
+            // the previous item's U stores must be done reading the tiles before they are rewritten
             if (issuer && stored) bulk_wait_group_read<0>();
             if (epi_sync_or(!__all_sync(0xffffffffu, ok) || *abort_flag)) {
                 *abort_flag = 1;
                 break;
             }
             tc_fence_after_sync();
-            // ---- this warp's stream: batch row b, channel pair (j, j+1).  Everything the
-            // walk reads from global memory is requested now, so that its latency passes
-            // under the accumulator transpose below.
+            // ---- this warp's streams: batch row b, channel pair (j, j+1) of each slice.
+            // What the first slice's walk reads from global memory is requested now, so
+            // that its latency passes under the accumulator transpose below.
             const int b0 = bgp * 2 * kBb + (int)rank * kBb;
-            const int js0 = js * kCh;
             const int b = b0 + q;
             const bool brow = b < B;
-            const int j = js0 + cj;
-            const bool jok = brow && j < d;
             const int bd = b * n_dir + dir;
             const int t_base = tp * kTt;
             const int nrows = min(kTt, L - t_base);
             const int i_first = dir == 0 ? 0 : kTt - kChunkT;  // first tile half in walk order
-            unsigned long long* cw = a.carry + (size_t)bd * d + j;  // this pair's carry words
-            const float* xp = a.x + (size_t)t_base * tstride_x + (size_t)b * d + j;
+            const int i_second = kTt - kChunkT - i_first;
             float2 xa[kChunkT];
-            load_x_half(xa, xp, i_first, nrows, tstride_x, jok);
-            GateParams2 p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
-            float2 c = f2(0.f);
-            bool have = true;  // the state entering the tile is known
-            if (jok) {
-                p = make_gate_params2(load_pair(a.v + (dir * 2 + 0) * d + j), load_pair(a.v + (dir * 2 + 1) * d + j),
-                                      load_pair(a.bias + (dir * 2 + 0) * d + j),
-                                      load_pair(a.bias + (dir * 2 + 1) * d + j));
-            }
-            if (brow) {
-                if (tt == 0) {
-                    if (jok && a.c0 != nullptr) c = load_pair(a.c0 + (size_t)bd * d + j);
-                } else if (jok) {
-                    unsigned g0, g1;
-                    ld_carry2(cw, g0, g1, c);
-                    have = g0 == (unsigned)tt && g1 == (unsigned)tt;  // written by tile tt - 1
+            GateParams2 p;
+            float2 c;
+            bool have;
+            int j;
+            bool jok;
+            // x of the first half, gate parameters and entering state of slice s
+            auto prefetch = [&](int s) {
+                j = (jg * NS + s) * kCh + cj;
+                jok = brow && j < d;
+                load_x_half(xa, a.x + (size_t)t_base * tstride_x + (size_t)b * d + j, i_first, nrows, tstride_x, jok);
+                p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
+                c = f2(0.f);
+                have = true;
+                if (jok) {
+                    p = make_gate_params2(load_pair(a.v + (dir * 2 + 0) * d + j), load_pair(a.v + (dir * 2 + 1) * d + j),
+                                          load_pair(a.bias + (dir * 2 + 0) * d + j),
+                                          load_pair(a.bias + (dir * 2 + 1) * d + j));
+                    if (tt == 0) {
+                        if (a.c0 != nullptr) c = load_pair(a.c0 + (size_t)bd * d + j);
+                    } else {
+                        unsigned g0, g1;
+                        ld_carry2(a.carry + (size_t)bd * d + j, g0, g1, c);
+                        have = g0 == (unsigned)tt && g1 == (unsigned)tt;  // written by tile tt - 1
+                    }
                 }
-            }
+            };
+            prefetch(0);
             // rows of this tile that exist (t < L) and are not padded, bit i = step t_base + i
             bool vrow = brow && lane < nrows;
             if (vrow && a.mask != nullptr) vrow = a.mask[(size_t)(t_base + lane) * B + b] == 0;
             const uint32_t valid = __ballot_sync(0xffffffffu, vrow);
-            // ---- accumulator rows (t, b) -> bf16 U tile, 128-byte swizzled lines [t][b][gate]
+            // ---- accumulator rows (t, b) -> bf16 U tiles, 128-byte swizzled lines [t][b][gate]
             {
                 const int r = q * 32 + lane;
 #pragma unroll 1
-                for (int c2 = 0; c2 < 3; ++c2) {
+                for (int c2 = 0; c2 < 3 * NS; ++c2) {
+                    const int s = c2 / 3;
                     uint32_t v[2][32];
-                    const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * kAccCols + c2 * 64;
+                    const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc + s) * kAccCols +
+                                           (c2 % 3) * 64;
                     tmem_ld_32x32b_x32(taddr, v[0]);
                     tmem_ld_32x32b_x32(taddr + 32, v[1]);
                     tc_wait_ld();
+                    const uint32_t utile = utile0 + (uint32_t)s * kUTileBytes;
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
-                        const int c6 = 2 * c2 + k;
+                        const int c6 = 2 * (c2 % 3) + k;
                         const int half = c6 / 3, g = c6 % 3;
                         const uint32_t line = (uint32_t)(r * 3 + g);
 #pragma unroll
@@ -458,51 +489,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)acc * 8u);  // accumulator free
-            fence_proxy_async_shared();  // the tile's writes, visible to the TMA store
+            fence_proxy_async_shared();  // the tiles' writes, visible to the TMA store
             epi_sync();
             if (issuer && a.write_u && b0 < B) {  // (a group wholly beyond B has no rows to store)
-                tma_store_5d(&map_u, utile_p, js0, 0, dir, b0, t_base);
+#pragma unroll
+                for (int s = 0; s < NS; ++s)
+                    if ((jg * NS + s) < njs)
+                        tma_store_5d(&map_u, utile_p + s * kUTileBytes, (jg * NS + s) * kCh, 0, dir, b0, t_base);
                 bulk_commit_group();
                 stored = true;
             }
             if (!brow) continue;
-            // ---- Eqs. (2)-(5) over the tile's steps in the direction's order
-            if (!have) {
-                // the previous tile of this stream has not handed over yet: re-read (bounded)
-                const uint64_t t0 = globaltimer_ns();
-                for (;;) {
-                    unsigned g0, g1;
-                    ld_carry2(cw, g0, g1, c);
-                    if (g0 == (unsigned)tt && g1 == (unsigned)tt) break;
-                    if (*reinterpret_cast<volatile unsigned*>(&g_error_word) != 0u) break;
-                    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                        record_error(kErrTimeoutScan);
-                        break;
+            // ---- Eqs. (2)-(5) over the tile's steps in the direction's order, slice by slice
+#pragma unroll 1
+            for (int s = 0; s < NS; ++s) {
+                if (s > 0) prefetch(s);
+                if ((jg * NS + s) >= njs) break;  // a slice wholly beyond d
+                unsigned long long* cw = a.carry + (size_t)bd * d + j;  // this pair's carry words
+                if (!have) {
+                    // the previous tile of this stream has not handed over yet: re-read (bounded)
+                    const uint64_t t0 = globaltimer_ns();
+                    for (;;) {
+                        unsigned g0, g1;
+                        ld_carry2(cw, g0, g1, c);
+                        if (g0 == (unsigned)tt && g1 == (unsigned)tt) break;
+                        if (*reinterpret_cast<volatile unsigned*>(&g_error_word) != 0u) break;
+                        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                            record_error(kErrTimeoutScan);
+                            break;
+                        }
                     }
                 }
-            }
-            float* hp = a.h + (size_t)t_base * tstride_h + (size_t)bd * d + j;
-            float2 xb[kChunkT];
-            const int i_second = kTt - kChunkT - i_first;
-            load_x_half(xb, xp, i_second, nrows, tstride_x, jok);  // under the first half's walk
+                const uint32_t utile = utile0 + (uint32_t)s * kUTileBytes;
+                const float* xp = a.x + (size_t)t_base * tstride_x + (size_t)b * d + j;
+                float* hp = a.h + (size_t)t_base * tstride_h + (size_t)bd * d + j;
+                float2 xb[kChunkT];
+                load_x_half(xb, xp, i_second, nrows, tstride_x, jok);  // under the first half's walk
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int i0 = hh == 0 ? i_first : i_second;
-                const int tc = (t_base + i0) / kChunkT;
-                if (tc >= nch) continue;  // wholly beyond L
-                if (a.ckpt != nullptr && jok) store_pair(a.ckpt + ((size_t)tc * B * n_dir + bd) * d + j, c);
-                const uint32_t v16 = (valid >> i0) & ((1u << kChunkT) - 1u);
-                if (dir == 0)
-                    c = fused_chunk<0>(utile, q, lane, i0, v16, c, p, alpha2, hh == 0 ? xa : xb, hp, tstride_h, jok,
-                                       nrows);
-                else
-                    c = fused_chunk<1>(utile, q, lane, i0, v16, c, p, alpha2, hh == 0 ? xa : xb, hp, tstride_h, jok,
-                                       nrows);
-            }
-            if (tt + 1 < nT) {
-                if (jok) st_carry2(cw, (unsigned)(tt + 1), c);
-            } else if (jok) {
-                store_pair(a.c_T + (size_t)bd * d + j, c);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int i0 = hh == 0 ? i_first : i_second;
+                    const int tc = (t_base + i0) / kChunkT;
+                    if (tc >= nch) continue;  // wholly beyond L
+                    if (a.ckpt != nullptr && jok) store_pair(a.ckpt + ((size_t)tc * B * n_dir + bd) * d + j, c);
+                    const uint32_t v16 = (valid >> i0) & ((1u << kChunkT) - 1u);
+                    if (dir == 0)
+                        c = fused_chunk<0>(utile, q, lane, i0, v16, c, p, alpha2, hh == 0 ? xa : xb, hp, tstride_h, jok,
+                                           nrows);
+                    else
+                        c = fused_chunk<1>(utile, q, lane, i0, v16, c, p, alpha2, hh == 0 ? xa : xb, hp, tstride_h, jok,
+                                           nrows);
+                }
+                if (tt + 1 < nT) {
+                    if (jok) st_carry2(cw, (unsigned)(tt + 1), c);
+                } else if (jok) {
+                    store_pair(a.c_T + (size_t)bd * d + j, c);
+                }
             }
         }
         if (issuer && stored) bulk_wait_group<0>();  // every U store has landed
