@@ -123,7 +123,7 @@ def test_fused_without_u_is_inference_only_and_equal(sru):
 
 
 def test_fused_repeated_calls_reuse_the_workspace(sru):
-    """The tile hand-over flags are cleared before every launch: a second call on
+    """The carry words are cleared before every launch: a second call on
     the same workspace gives the same result."""
     cfg, inp = _inputs(200, 8, 256, 1, 17, False, True)
     f = _run_fused(sru, cfg, inp, 1.0)
