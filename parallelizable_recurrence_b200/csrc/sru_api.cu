@@ -256,24 +256,19 @@ sru_status check_layer_sizes(int64_t L, int64_t B, int64_t d) {
 inline unsigned blocks_for(size_t n, unsigned threads) { return (unsigned)((n + threads - 1) / threads); }
 
 // ------------------------------------------------------------- GEMM launch
-// The CTA-pair kernel (256 x 256 tiles over two SMs) is the default; the
-// single-CTA kernel (128 x 256) remains for comparison builds.
-#ifndef SRU_GEMM_USE_PAIR
-#define SRU_GEMM_USE_PAIR 1
-#endif
-constexpr bool kGemmPair = SRU_GEMM_USE_PAIR != 0;
-// rows of B staged per CTA for a K-major B operand
-constexpr uint32_t kGemmBRows = kGemmPair ? (uint32_t)sru::gemm::P_CN : (uint32_t)sru::gemm::BN;
+// The CTA-pair kernel: 256 x 256 output tiles over two SMs; a K-major B
+// operand is staged as 128 rows per CTA.
+constexpr uint32_t kGemmBRows = (uint32_t)sru::gemm::P_CN;
 
-// splits = 2 (pair kernel, OUT == kOutF32Red only): each output tile's
-// reduction is cut in two halves that add into the zeroed output.
-// ldo: output row stride in elements (default C).
-template <bool A_MN, bool B_MN, int OUT>
+// tail_split (pair kernel, OUT == kOutF32 only): the output tiles of the last,
+// partial round of CTA pairs are cut in two k-pieces that add onto regions
+// zeroed here first (see sru::gemm::pair_next).
+template <bool A_MN, bool B_MN, int OUT, int L2HINT = 0>
 sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
-                          int64_t Kr, cudaStream_t st, int splits = 1, int64_t ldo = -1) {
+                          int64_t Kr, cudaStream_t st, int splits = 1, int64_t ldo = -1, bool tail_split = false) {
     if (ldo < 0) ldo = C;
-    if (kGemmPair) {
-        auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT>;
+    {
+        auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT, 0, 0, 0, L2HINT>;
         SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
         // the output as the epilogue's TMA store target: box 32 x 32, swizzled like the staging buffers
         CUtensorMap mo;
@@ -286,18 +281,23 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
                           strides, box, bf ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
                 return SRU_ERR_INVALID;
         }
-        const int64_t units =
-            ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN) * splits;
+        const int64_t n_tiles = (C + sru::gemm::P_BN - 1) / sru::gemm::P_BN;
+        const int64_t tiles = ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * n_tiles;
+        const int64_t units = tiles * splits;
         const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
+        int tail_s = 0;
+        const int64_t kblocks = (Kr + sru::gemm::BK - 1) / sru::gemm::BK;
+        if (tail_split && OUT == sru::gemm::kOutF32 && splits == 1 && tiles > pairs && tiles % pairs != 0 &&
+            kblocks >= 6) {
+            const int64_t F = tiles / pairs, Rt = tiles % pairs;
+            tail_s = (int)(2 * Rt <= pairs ? kblocks / 2 : kblocks / 3);
+            sru::gemm::zero_tail_tiles_kernel<<<(unsigned)Rt, 256, 0, st>>>(reinterpret_cast<float*>(out), (int)R,
+                                                                          (int)C, (long long)ldo, (int)n_tiles,
+                                                                          (int)(F * pairs));
+            SRU_CUDA_TRY(cudaGetLastError());
+        }
         kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
-            ma, mb, mo, out, (int)R, (int)C, (int)Kr, (int)ldo, splits, 1, 0LL);
-    } else {
-        if (splits != 1) return SRU_ERR_UNSUPPORTED;
-        auto kern = sru::gemm::tc_gemm_kernel<A_MN, B_MN, OUT>;
-        SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::SMEM_BYTES));
-        const int64_t tiles = ((R + sru::gemm::BM - 1) / sru::gemm::BM) * ((C + sru::gemm::BN - 1) / sru::gemm::BN);
-        const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-        kern<<<grid, sru::gemm::THREADS, sru::gemm::SMEM_BYTES, st>>>(ma, mb, out, (int)R, (int)C, (int)Kr, (int)ldo);
+            ma, mb, mo, out, (int)R, (int)C, (int)Kr, (int)ldo, splits, 1, 0LL, tail_s);
     }
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
@@ -312,7 +312,6 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
 template <bool A_MN, bool B_MN, int OUT, int BPA, int BPB, int CAUSAL = 0>
 sru_status launch_tc_gemm_batched(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
                                   int64_t Kr, int64_t ldo, int64_t batches, int64_t out_bstride, cudaStream_t st) {
-    if (!kGemmPair) return SRU_ERR_UNSUPPORTED;
     auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT, BPA, BPB, CAUSAL>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
     const int64_t mt = (R + sru::gemm::P_BM - 1) / sru::gemm::P_BM, nt = (C + sru::gemm::P_BN - 1) / sru::gemm::P_BN;
@@ -323,7 +322,7 @@ sru_status launch_tc_gemm_batched(const CUtensorMap& ma, const CUtensorMap& mb, 
     CUtensorMap unused;  // batched launches store directly (no output map)
     std::memset(&unused, 0, sizeof(unused));
     kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
-        ma, mb, unused, out, (int)R, (int)C, (int)Kr, (int)ldo, 1, (int)batches, (long long)out_bstride);
+        ma, mb, unused, out, (int)R, (int)C, (int)Kr, (int)ldo, 1, (int)batches, (long long)out_bstride, 0);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
@@ -358,18 +357,6 @@ bool map_mnmajor_b(CUtensorMap* m, const void* p, int64_t rows, int64_t K, int64
     const uint64_t strides[2] = {(uint64_t)ld * 2, (uint64_t)batch_ld * 2};
     const uint32_t box[3] = {64, 64, 1};
     return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
-// Whether an fp32-output product with few output tiles and a long reduction
-// runs faster as two K halves: when the halves fill the SM pairs' waves
-// better (e.g. 96 tiles on 74 pairs: 65% of the second wave idle, versus 192
-// halves in 3 waves at 86%), and each half keeps at least 16 k-blocks.
-bool gemm_split_pays(int64_t R, int64_t C, int64_t Kr) {
-    if (!kGemmPair || Kr < 32 * sru::gemm::BK) return false;
-    const int64_t tiles = ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN);
-    const int64_t P = sm_count() / 2;
-    auto eff = [&](int64_t u) { return (double)u / (double)(((u + P - 1) / P) * P); };
-    return eff(2 * tiles) > eff(tiles) + 0.05;
 }
 
 // K-major operand (rows x K), contiguous K, rows ld elements apart (ld >= K;
@@ -817,7 +804,7 @@ sru_status sru_project(const void* X, int x_t, const void* W, int w_t, void* U, 
     if (x_t != SRU_BF16 || w_t != SRU_BF16 || (u_t != SRU_BF16 && u_t != SRU_F32)) return SRU_ERR_INVALID;
     if (K == 0) return SRU_ERR_UNSUPPORTED;
     CUtensorMap ma, mb;
-    if (!map_kmajor(&ma, X, M, K, sru::gemm::BM) || !map_kmajor(&mb, W, N, K, kGemmBRows)) return SRU_ERR_INVALID;
+    if (!map_kmajor(&ma, X, M, K, sru::gemm::P_CM) || !map_kmajor(&mb, W, N, K, kGemmBRows)) return SRU_ERR_INVALID;
     if (u_t == SRU_BF16) return launch_tc_gemm<false, false, sru::gemm::kOutBF16>(ma, mb, U, M, N, K, st);
     return launch_tc_gemm<false, false, sru::gemm::kOutF32>(ma, mb, U, M, N, K, st);
 }
@@ -856,7 +843,7 @@ sru_status sru_project_backward(const void* dU, const void* X, const void* W, in
         } else {
             CUtensorMap ma, mb;
             // A = dU (M x N) K-major; B(c = k, red = n) = W[n][k]: MN-major with ld = K
-            if (!map_kmajor(&ma, dU, M, N, sru::gemm::BM) || !map_mnmajor(&mb, W, K, N, K)) return SRU_ERR_INVALID;
+            if (!map_kmajor(&ma, dU, M, N, sru::gemm::P_CM) || !map_mnmajor(&mb, W, K, N, K)) return SRU_ERR_INVALID;
             sru_status s = accumulate ? launch_tc_gemm<false, true, sru::gemm::kOutF32Acc>(ma, mb, dX, M, K, N, st)
                                       : launch_tc_gemm<false, true, sru::gemm::kOutF32>(ma, mb, dX, M, K, N, st);
             if (s != SRU_OK) return s;
@@ -867,11 +854,8 @@ sru_status sru_project_backward(const void* dU, const void* X, const void* W, in
         CUtensorMap ma, mb;
         // A(r = n, red = m) = dU[m][n]: MN-major, ld = N; B(c = k, red = m) = X[m][k]: MN-major, ld = K
         if (!map_mnmajor(&ma, dU, N, M, N) || !map_mnmajor(&mb, X, K, M, K)) return SRU_ERR_INVALID;
-        if (gemm_split_pays(N, K, M)) {
-            SRU_CUDA_TRY(cudaMemsetAsync(dW, 0, (size_t)N * K * sizeof(float), st));
-            return launch_tc_gemm<true, true, sru::gemm::kOutF32Red>(ma, mb, dW, N, K, M, st, 2);
-        }
-        return launch_tc_gemm<true, true, sru::gemm::kOutF32>(ma, mb, dW, N, K, M, st);
+        // dW = dU^T X: dU read once (evict first), X read by every round of tiles (kept)
+        return launch_tc_gemm<true, true, sru::gemm::kOutF32, 1>(ma, mb, dW, N, K, M, st, 1, -1, /*tail_split=*/true);
     }
     return SRU_OK;
 }
@@ -1154,7 +1138,7 @@ sru_status sru_project_factored_backward(const void* dU, const void* X, const vo
     }
     // dP = dU Wo (bf16): A = dU K-major over n; B(c = kp, red = n) = Wo[n][kp] MN-major
     {
-        if (!map_kmajor(&ma, dU, M, N, sru::gemm::BM) || !map_mnmajor(&mb, Wo, Kp, N, Kp)) return SRU_ERR_INVALID;
+        if (!map_kmajor(&ma, dU, M, N, sru::gemm::P_CM) || !map_mnmajor(&mb, Wo, Kp, N, Kp)) return SRU_ERR_INVALID;
         sru_status s = launch_tc_gemm<false, true, sru::gemm::kOutBF16>(ma, mb, dP, M, Kp, N, st);
         if (s != SRU_OK) return s;
     }
@@ -1225,7 +1209,7 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
         const int64_t g = B - b0 < G ? B - b0 : G;
         CUtensorMap ma, mb;
         // S_z = Q_z K_z^T (z = 0 .. g-1): K-major over d'; batch stride d' / 2d', row stride B d' / 2B d'
-        if (!map_kmajor_b(&ma, Q + b0 * dp, L, dp, B * dp, g, dp, sru::gemm::BM, 1) ||
+        if (!map_kmajor_b(&ma, Q + b0 * dp, L, dp, B * dp, g, dp, sru::gemm::P_CM, 1) ||
             !map_kmajor_b(&mb, KV + b0 * 2 * dp, L, dp, B * 2 * dp, g, 2 * dp, kGemmBRows, 1))
             return SRU_ERR_INVALID;
         s = causal ? launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st)
@@ -1236,7 +1220,7 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
         SRU_CUDA_TRY(cudaGetLastError());
         // A_z = P_z V_z: P_z K-major over s (batch outermost); V_z(c = j, red = s) at
         // KV[(s*B + b0 + z)*2d' + d' + j]: MN-major, batch stride 2d'
-        if (!map_kmajor_b(&ma, P, L, L, L, g, L * L, sru::gemm::BM, 2) ||
+        if (!map_kmajor_b(&ma, P, L, L, L, g, L * L, sru::gemm::P_CM, 2) ||
             !map_mnmajor_b(&mb, KV + b0 * 2 * dp + dp, dp, L, B * 2 * dp, g, 2 * dp, 1))
             return SRU_ERR_INVALID;
         s = causal ? launch_tc_gemm_batched<false, true, sru::gemm::kOutF32, 2, 1, 2>(ma, mb, A + b0 * dp, L, dp, L,

@@ -4,19 +4,19 @@
 // the three per-step matrix-vector products of all L steps are grouped into one
 // product U^T = [W; W'; W''] X^T, the only dense contraction of the layer.
 //
-// tc_gemm_kernel computes  out[r, c] (+)= sum_k A(r, k) * B(c, k)  on the
+// tc_gemm_pair_kernel computes  out[r, c] (+)= sum_k A(r, k) * B(c, k)  on the
 // 5th-generation tensor cores: bf16 operands staged by TMA into 128-byte
 // swizzled shared memory, tcgen05.mma issued by a single thread into a fp32
 // accumulator in tensor memory (TMEM), and an epilogue that reads TMEM with
-// tcgen05.ld.  The kernel is persistent (one CTA per SM walking output tiles)
-// and warp specialised:
-//   warp 0        TMA producer (one elected lane), STAGES-deep smem ring
-//   warp 1        TMEM allocator and MMA issuer (one elected lane)
+// tcgen05.ld and sends the output through shared memory with TMA stores.  A
+// cluster of two CTAs (two SMs) computes each 256 x 256 output tile with
+// tcgen05.mma.cta_group::2; the kernel is persistent (one pair per two SMs
+// walking output tiles) and warp specialised:
+//   warp 0        TMA producer (one elected lane), P_STAGES-deep smem ring
+//   warp 1        TMEM allocator and MMA issuer (one elected lane, pair leader)
 //   warps 2..5    epilogue, one TMEM lane quarter each
-// Two 128 x 256 fp32 accumulators (512 TMEM columns) let the epilogue of tile
-// i overlap the main loop of tile i+1.  (tc_gemm_kernel is the single-SM
-// variant kept for comparison builds; the default is tc_gemm_pair_kernel
-// below, whose epilogue stores through shared memory with TMA.)
+// Two 128 x 256 fp32 accumulators per CTA (512 TMEM columns) let the epilogue
+// of tile i overlap the main loop of tile i+1.
 //
 // Operand majorness (which index is contiguous in global memory):
 //   U  = X  W^T : A = X  (M x K, K-major), B = W (N x K, K-major)
@@ -31,19 +31,11 @@
 namespace sru {
 namespace gemm {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KB
-constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KB
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int BK = 64;           // k per stage: one 128-byte swizzle row of bf16
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 2 * BN;  // two fp32 accumulators
 constexpr uint32_t MN_BOX_BYTES = 64 * 64 * 2;  // one (64 x 64) MN-major box
-constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-
-// kOutF32Red: add into an fp32 output with vector atomics (the two K halves of
-// a split tile, onto an output the host zeroed: 0 + a + b rounds the same in
-// either order, so the sum does not depend on which half lands first).
-enum OutMode : int { kOutBF16 = 0, kOutF32 = 1, kOutF32Acc = 2, kOutF32Red = 3 };
+// kOutF32Acc: add onto the existing fp32 output (TMA reduce-add).
+enum OutMode : int { kOutBF16 = 0, kOutF32 = 1, kOutF32Acc = 2 };
 
 // Shared-memory matrix descriptor (tcgen05 "smem descriptor"): start address,
 // leading- and stride-dimension byte offsets (16-byte units), descriptor
@@ -56,13 +48,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     d |= 1ull << 46;  // version for sm_100
     d |= 2ull << 61;  // SWIZZLE_128B
     return d;
-}
-
-// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B,
-// operand majorness, N >> 3 and M >> 4.
-__host__ __device__ constexpr uint32_t idesc_bf16(bool a_mn, bool b_mn) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
-           ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
 // Store 32 consecutive accumulator columns (r[0..31]) of one output row.
@@ -93,10 +78,6 @@ __device__ __forceinline__ void epilogue_store_row32(void* __restrict__ out, int
             if (col0 + g * 4 < N) {
                 float4 val = make_float4(__uint_as_float(r[g * 4 + 0]), __uint_as_float(r[g * 4 + 1]),
                                          __uint_as_float(r[g * 4 + 2]), __uint_as_float(r[g * 4 + 3]));
-                if (OUT == kOutF32Red) {
-                    atomicAdd(reinterpret_cast<float4*>(o + g * 4), val);
-                    continue;
-                }
                 if (OUT == kOutF32Acc) {
                     const float4 old = *reinterpret_cast<const float4*>(o + g * 4);
                     val.x += old.x;
@@ -110,183 +91,8 @@ __device__ __forceinline__ void epilogue_store_row32(void* __restrict__ out, int
     }
 }
 
-template <bool A_MN, bool B_MN, int OUT>
-__global__ void __launch_bounds__(THREADS, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                   void* __restrict__ out, int M, int N, int K, int ldo) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-    uint64_t* empty = full + STAGES;
-    uint64_t* tfull = empty + STAGES;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile uint32_t* consumed = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m_tiles = (M + BM - 1) / BM, n_tiles = (N + BN - 1) / BN;
-    const int tiles = m_tiles * n_tiles;
-    const int kblocks = (K + BK - 1) / BK;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 4);
-        }
-        mbar_init(drain, 1);
-        *abort_flag = 0;
-        *consumed = 0;
-        fence_mbar_init();
-        tma_prefetch_desc(&map_a);
-        tma_prefetch_desc(&map_b);
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem_base = *tmem_slot;
-
-    if (warp == 0) {
-        if (lane == 0) {
-            // ------------------------------------------------------ producer
-            uint32_t issued = 0;
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x) {
-                const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
-                for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1u, kErrTimeoutMma) || *abort_flag) {
-                        *abort_flag = 1;
-                        break;
-                    }
-                    uint8_t* a_dst = smem + stage * STAGE_BYTES;
-                    uint8_t* b_dst = a_dst + A_BYTES;
-                    const int k0 = kb * BK;
-                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-                    if (!A_MN) {
-                        tma_load_2d(a_dst, &map_a, &full[stage], k0, m0);
-                    } else {
-                        tma_load_2d(a_dst, &map_a, &full[stage], m0, k0);
-                        tma_load_2d(a_dst + MN_BOX_BYTES, &map_a, &full[stage], m0 + 64, k0);
-                    }
-                    if (!B_MN) {
-                        tma_load_2d(b_dst, &map_b, &full[stage], k0, n0);
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < BN / 64; ++q)
-                            tma_load_2d(b_dst + q * MN_BOX_BYTES, &map_b, &full[stage], n0 + 64 * q, k0);
-                    }
-                    ++issued;
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-            }
-            if (*abort_flag) {
-                // wait (bounded) for the loads still in flight before this CTA may exit
-                for (uint32_t q = *consumed; q < issued; ++q)
-                    mbar_wait(&full[q % STAGES], (q / STAGES) & 1u, kErrTimeoutLoad);
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            // ------------------------------------------------------ MMA issuer
-            constexpr uint32_t idesc = idesc_bf16(A_MN, B_MN);
-            int stage = 0;
-            uint32_t phase = 0, nconsumed = 0;
-            int it = 0;
-            for (int tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x, ++it) {
-                const int acc = it & 1;
-                const uint32_t acc_phase = (it >> 1) & 1;
-                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, kErrTimeoutEpilogue)) {
-                    *abort_flag = 1;
-                    break;
-                }
-                tc_fence_after_sync();
-                const uint32_t d_tmem = tmem_base + acc * BN;
-                bool ok = true;
-                for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, kErrTimeoutLoad)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    const uint32_t a_addr = smem_u32(smem + stage * STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + A_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t adesc = A_MN ? smem_desc_sw128(a_addr + kk * 2048, MN_BOX_BYTES, 1024)
-                                                    : smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-                        const uint64_t bdesc = B_MN ? smem_desc_sw128(b_addr + kk * 2048, MN_BOX_BYTES, 1024)
-                                                    : smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-                        tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
-                    }
-                    tc_commit(&empty[stage]);  // frees the smem stage once these MMAs retire
-                    *consumed = ++nconsumed;
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-                if (!ok) {
-                    *abort_flag = 1;
-                    break;
-                }
-                tc_commit(&tfull[acc]);  // accumulator ready for the epilogue
-            }
-            // every MMA this thread issued has retired before TMEM is released
-            tc_commit(drain);
-            mbar_wait(drain, 0, kErrTimeoutMma);
-        }
-    } else {
-        // ---------------------------------------------------------- epilogue
-        const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
-        int it = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++it) {
-            const int acc = it & 1;
-            const uint32_t acc_phase = (it >> 1) & 1;
-            const int m0 = (tile / n_tiles) * BM, n0 = (tile % n_tiles) * BN;
-            const bool ok = mbar_wait(&tfull[acc], acc_phase, kErrTimeoutMma);
-            if (!__all_sync(0xffffffffu, ok) || *abort_flag) {
-                *abort_flag = 1;
-                break;
-            }
-            tc_fence_after_sync();
-            const int row = m0 + quarter * 32 + lane;
-            for (int ch = 0; ch < BN / 32; ++ch) {
-                const int col0 = n0 + ch * 32;
-                if (col0 >= N) break;  // uniform across the warp
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN + ch * 32, r);
-                tc_wait_ld();
-                epilogue_store_row32<OUT>(out, row, col0, M, N, ldo, r);
-            }
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
-        }
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after_sync();
-        tmem_dealloc(tmem_base, TMEM_COLS);
-    }
-}
-
-
 // ---------------------------------------------------------------------------
-// CTA-pair variant: a cluster of two CTAs (two SMs) computes one 256 x 256
+// A cluster of two CTAs (two SMs) computes one 256 x 256
 // output tile with tcgen05.mma.cta_group::2 (M = 256).  Each CTA stages its own
 // 128 rows of A and its own 128 columns of B (32 KB per k-block instead of
 // 48 KB for a 128 x 256 tile on one SM), and holds its 128 rows of the
@@ -353,8 +159,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16_pair(bool a_mn, bool b_mn) {
 // out + z * out_bstride.
 template <int BPOS>
 __device__ __forceinline__ void tma_load_tile_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y,
-                                                   int z) {
-    if (BPOS == 0)
+                                                   int z, uint64_t policy = 0) {
+    if (BPOS == 0 && policy != 0)
+        tma_load_2d_pair_hint(dst, map, bar, x, y, policy);
+    else if (BPOS == 0)
         tma_load_2d_pair(dst, map, bar, x, y);
     else if (BPOS == 1)
         tma_load_3d_pair(dst, map, bar, x, z, y);
@@ -374,6 +182,7 @@ __device__ __forceinline__ void tma_load_tile_pair(void* dst, const CUtensorMap*
 //      which every probability is 0.
 struct PairUnit {
     int z, tm, tn, kb_lo, kb_hi;
+    bool reduce;  // add onto the output (a piece of a tile split in two) instead of storing
 };
 template <int CAUSAL>
 __device__ __forceinline__ PairUnit pair_unit(int u, int m_tiles, int n_tiles, int splits, int kblocks, int kper) {
@@ -399,14 +208,65 @@ __device__ __forceinline__ PairUnit pair_unit(int u, int m_tiles, int n_tiles, i
     w.kb_lo = (uu % splits) * kper;
     w.kb_hi = min(kblocks, w.kb_lo + kper);
     if (CAUSAL == 2) w.kb_hi = min(w.kb_hi, ((w.tm + 1) * P_BM + BK - 1) / BK);
+    w.reduce = false;
     return w;
 }
 
-template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0, int CAUSAL = 0>
+// The i-th work unit of pair p (of P).  Without a tail split (tail_s == 0) the
+// units are dealt round-robin: unit p + i P.  With one (fp32 outputs, one
+// batch, no K split): the tiles = F P + R fill F whole rounds round-robin, and
+// the R tiles of the last, partial round are cut in two k-pieces, [0, s) and
+// [s, K), that both add onto an output region zeroed beforehand (0 + a + b
+// rounds the same in either order, so the result is deterministic):
+//   pair p < R              the piece [s, K) of tail tile p
+//   R <= p < 2R             the piece [0, s) of tail tile p - R
+//   and, when 2R > P, pair p with p - R < 2R - P also the piece [0, s) of tail
+//   tile (P - R) + (p - R).
+// The host takes s = K/2 when 2R <= P (every piece its own pair) and s = K/3
+// otherwise (some pairs take two short pieces): the tail then costs half or
+// two thirds of a round instead of a whole one.
+template <int CAUSAL>
+__device__ __forceinline__ bool pair_next(int i, int p, int P, int units, int m_tiles, int n_tiles, int splits,
+                                          int kblocks, int kper, int tail_s, PairUnit& w) {
+    if (tail_s == 0) {
+        const int u = p + i * P;
+        if (u >= units) return false;
+        w = pair_unit<CAUSAL>(u, m_tiles, n_tiles, splits, kblocks, kper);
+        return true;
+    }
+    const int tiles = m_tiles * n_tiles, F = tiles / P, R = tiles % P;
+    int tile = -1;
+    bool large = false;
+    if (i < F) {
+        tile = p + i * P;
+    } else if (i == F) {
+        if (p < R) {
+            tile = F * P + p;
+            large = true;
+        } else if (p - R < R) {
+            tile = F * P + (p - R);
+        }
+    } else if (i == F + 1) {
+        if (p >= R && p - R < 2 * R - P) tile = F * P + (P - R) + (p - R);
+    }
+    if (tile < 0) return false;
+    w.z = 0;
+    w.tm = tile / n_tiles;
+    w.tn = tile % n_tiles;
+    w.reduce = i >= F;
+    w.kb_lo = (i < F || !large) ? 0 : tail_s;
+    w.kb_hi = (i < F || large) ? kblocks : tail_s;
+    return true;
+}
+
+// L2HINT (non-batched launches): 1 = the A operand is read once (its loads
+// evicted first) and the B operand is read again by later rounds of tiles
+// (kept in L2): dW = dU^T X, where every round re-reads all of X.
+template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0, int CAUSAL = 0, int L2HINT = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                         const __grid_constant__ CUtensorMap map_out, void* __restrict__ out, int M, int N, int K,
-                        int ldo, int splits, int batches, long long out_bstride) {
+                        int ldo, int splits, int batches, long long out_bstride, int tail_s) {
     constexpr bool kTmaOut = (BPA | BPB) == 0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -426,8 +286,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int m_tiles = (M + P_BM - 1) / P_BM, n_tiles = (N + P_BN - 1) / P_BN;
     const int tiles = m_tiles * n_tiles;
     const int kblocks = (K + BK - 1) / BK;
-    // work unit u = (tile u / splits, K part u % splits); splits > 1 only with
-    // kOutF32Red and at least one k-block per part (the host checks both)
+    // work unit u = (tile u / splits, K part u % splits); the host passes splits = 1
     // batch-major, then tile, then K part (causal scores: the lower-triangle tiles only)
     const int units = (CAUSAL == 1 ? m_tiles * (m_tiles + 1) / 2 : tiles * splits) * batches;
     const int kper = (kblocks + splits - 1) / splits;
@@ -466,8 +325,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             uint32_t issued = 0;
             int stage = 0;
             uint32_t phase = 0;
-            for (int u = pair_id; u < units && !*abort_flag; u += n_pairs) {
-                const PairUnit w = pair_unit<CAUSAL>(u, m_tiles, n_tiles, splits, kblocks, kper);
+            const uint64_t pol_a = L2HINT == 1 ? l2_policy_evict_first() : 0;
+            const uint64_t pol_b = L2HINT == 1 ? l2_policy_evict_last() : 0;
+            PairUnit w;
+            for (int i = 0; !*abort_flag &&
+                            pair_next<CAUSAL>(i, pair_id, n_pairs, units, m_tiles, n_tiles, splits, kblocks, kper,
+                                              tail_s, w);
+                 ++i) {
                 const int z = w.z, kb_lo = w.kb_lo, kb_hi = w.kb_hi;
                 const int m0 = w.tm * P_BM + (int)rank * P_CM;
                 const int n0 = w.tn * P_BN + (int)rank * P_CN;
@@ -482,16 +346,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t bar = leader_full0 + (uint32_t)stage * 8u;
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
                     if (!A_MN) {
-                        tma_load_tile_pair<BPA>(a_dst, &map_a, bar, k0, m0, z);
+                        tma_load_tile_pair<BPA>(a_dst, &map_a, bar, k0, m0, z, pol_a);
                     } else {
-                        tma_load_tile_pair<BPA>(a_dst, &map_a, bar, m0, k0, z);
-                        tma_load_tile_pair<BPA>(a_dst + MN_BOX_BYTES, &map_a, bar, m0 + 64, k0, z);
+                        tma_load_tile_pair<BPA>(a_dst, &map_a, bar, m0, k0, z, pol_a);
+                        tma_load_tile_pair<BPA>(a_dst + MN_BOX_BYTES, &map_a, bar, m0 + 64, k0, z, pol_a);
                     }
                     if (!B_MN) {
-                        tma_load_tile_pair<BPB>(b_dst, &map_b, bar, k0, n0, z);
+                        tma_load_tile_pair<BPB>(b_dst, &map_b, bar, k0, n0, z, pol_b);
                     } else {
-                        tma_load_tile_pair<BPB>(b_dst, &map_b, bar, n0, k0, z);
-                        tma_load_tile_pair<BPB>(b_dst + MN_BOX_BYTES, &map_b, bar, n0 + 64, k0, z);
+                        tma_load_tile_pair<BPB>(b_dst, &map_b, bar, n0, k0, z, pol_b);
+                        tma_load_tile_pair<BPB>(b_dst + MN_BOX_BYTES, &map_b, bar, n0 + 64, k0, z, pol_b);
                     }
                     ++issued;
                     if (++stage == P_STAGES) {
@@ -512,8 +376,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             int stage = 0;
             uint32_t phase = 0, nconsumed = 0;
             int it = 0;
-            for (int u = pair_id; u < units && !*abort_flag; u += n_pairs, ++it) {
-                const PairUnit w = pair_unit<CAUSAL>(u, m_tiles, n_tiles, splits, kblocks, kper);
+            PairUnit w;
+            for (int i = 0; !*abort_flag &&
+                            pair_next<CAUSAL>(i, pair_id, n_pairs, units, m_tiles, n_tiles, splits, kblocks, kper,
+                                              tail_s, w);
+                 ++i, ++it) {
                 const int kb_lo = w.kb_lo, kb_hi = w.kb_hi;
                 const int acc = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
@@ -561,8 +428,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int quarter = warp & 3;
         int it = 0;
         uint32_t nstaged = 0;  // chunks this warp has handed to TMA stores
-        for (int u = pair_id; u < units; u += n_pairs, ++it) {
-            const PairUnit w = pair_unit<CAUSAL>(u, m_tiles, n_tiles, splits, kblocks, kper);
+        PairUnit w;
+        for (int i = 0; pair_next<CAUSAL>(i, pair_id, n_pairs, units, m_tiles, n_tiles, splits, kblocks, kper, tail_s, w);
+             ++i, ++it) {
             const int z = w.z;
             void* const zout = (BPA | BPB) != 0 ? static_cast<void*>(static_cast<uint8_t*>(out) +
                                                              (size_t)z * (size_t)out_bstride * (OUT == kOutBF16 ? 2 : 4))
@@ -595,7 +463,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     __syncwarp();
                     if (lane == 0) {
                         const void* src = epi + (size_t)(quarter * 2 + (nstaged & 1)) * P_EPI_BUF;
-                        if (OUT == kOutF32Acc || OUT == kOutF32Red)
+                        if (OUT == kOutF32Acc || w.reduce)
                             tma_reduce_add_2d(&map_out, src, col0, m0 + quarter * 32);
                         else
                             tma_store_2d(&map_out, src, col0, m0 + quarter * 32);
@@ -618,6 +486,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (warp == 1) {
         tc_fence_after_sync();
         tmem_dealloc_pair(tmem_base, P_TMEM_COLS);
+    }
+}
+
+// Zero the output regions of the tail tiles (tiles first_tile .. first_tile +
+// gridDim.x - 1 of P_BM x P_BN, clipped to R x C, row stride ldo floats) that
+// the tail split's two pieces then add onto.
+__global__ void __launch_bounds__(256) zero_tail_tiles_kernel(float* __restrict__ out, int R, int C, long long ldo,
+                                                              int n_tiles, int first_tile) {
+    const int tile = first_tile + blockIdx.x;
+    const int r0 = (tile / n_tiles) * P_BM, c0 = (tile % n_tiles) * P_BN;
+    const int rows = min(P_BM, R - r0), cols = min(P_BN, C - c0);  // C % 8 == 0: cols a multiple of 4
+    for (int e = threadIdx.x; e < rows * (cols / 4); e += blockDim.x) {
+        const int r = e / (cols / 4), c4 = e % (cols / 4);
+        *reinterpret_cast<float4*>(out + (size_t)(r0 + r) * ldo + c0 + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
 }
 

@@ -104,14 +104,18 @@ def test_project_large_k_sampled(sru):
     tl.assert_close_sum("dW sampled", tl.host_f64(dW)[rows, cols], ref, absref)
 
 
-def test_split_reduction_dw_is_deterministic(sru):
-    """dW with few output tiles and a long reduction is computed as two K halves
-    added into the zeroed output; with two addends per element the fp32 sum is
-    the same whichever half lands first, so repeated calls agree bit for bit."""
+@pytest.mark.parametrize("N,K", [(6144, 2048), (3072, 2048)])
+def test_tail_split_dw_matches_oracle_and_is_deterministic(sru, N, K):
+    """dW whose output tiles do not fill whole rounds of the 74 CTA pairs: the
+    tiles of the last, partial round are cut in two k-pieces that add onto a
+    zeroed region (192 tiles: pieces of K/3 and 2K/3, some pairs taking two short
+    pieces; 96 tiles: halves).  Entries of those tiles and of whole tiles match
+    the oracle's plain sums, and with two addends per element the fp32 result is
+    the same whichever piece lands first: repeated calls agree bit for bit."""
     rng = np.random.default_rng(5)
-    M, N, K = 8192, 768, 256          # 3 output tiles, 128 k-blocks: the split is taken
-    Xd, dUd = tl.to_dev_bf16(_bf16(rng, (M, K))), tl.to_dev_bf16(_bf16(rng, (M, N)))
-    Wd = tl.to_dev_bf16(_bf16(rng, (N, K)))
+    M = 1024                          # 16 k-blocks: pieces of 5 and 11, or 8 and 8
+    Xb, dUb = _bf16(rng, (M, K)), _bf16(rng, (M, N))
+    Xd, dUd, Wd = tl.to_dev_bf16(Xb), tl.to_dev_bf16(dUb), tl.to_dev_bf16(_bf16(rng, (N, K)))
     outs = []
     for _ in range(3):
         dW = torch.full((N, K), float("nan"), device="cuda")
@@ -119,3 +123,10 @@ def test_split_reduction_dw_is_deterministic(sru):
         outs.append(dW)
     assert sru.sru_sync_status() == 0
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    got = tl.host_f64(outs[0])
+    # sampled entries anywhere, and every entry of one row and one column of the last tiles
+    rows = np.concatenate([rng.integers(0, N, 2048), np.full(K, N - 1), np.arange(N - 256, N)])
+    cols = np.concatenate([rng.integers(0, K, 2048), np.arange(K), np.full(256, K - 1)])
+    ref = oracle.project_dW_entries(dUb, Xb, rows, cols)
+    absref = oracle.project_dW_entries(tl.abs_operand(dUb), tl.abs_operand(Xb), rows, cols)
+    tl.assert_close_sum("dW sampled", got[rows, cols], ref, absref)
