@@ -176,14 +176,22 @@ __device__ __forceinline__ float2 fused_chunk(uint32_t utile, int q, int l, int 
             wf[i] = lds_u32(utile_word(utile, r, 1, l));
             wr[i] = lds_u32(utile_word(utile, r, 2, l));
         }
-        float2 hv[kChunkT];
+        // pass 1: the state chain (forget gate and c only); pass 2: reset gate and h
+        float2 cprev[kChunkT], cs[kChunkT];
 #pragma unroll
         for (int s = 0; s < kChunkT; ++s) {
             const int i = DIR == 0 ? s : kChunkT - 1 - s;
-            float2 f, r;
-            c = sru_cell2(c, bf16x2_to_float2(wc[i]), bf16x2_to_float2(wf[i]), bf16x2_to_float2(wr[i]), p, f, r);
+            cprev[i] = c;
+            const float2 uc = bf16x2_to_float2(wc[i]);
+            c = fma2(sru_forget2(c, bf16x2_to_float2(wf[i]), p), sub2(c, uc), uc);  // Eq. (4)
+            cs[i] = c;
+        }
+        float2 hv[kChunkT];
+#pragma unroll
+        for (int i = 0; i < kChunkT; ++i) {
+            const float2 r = sru_reset2(cprev[i], bf16x2_to_float2(wr[i]), p);
             const float2 ax = mul2(alpha2, wx[i]);
-            hv[i] = fma2(r, sub2(c, ax), ax);  // Eq. (5)
+            hv[i] = fma2(r, sub2(cs[i], ax), ax);  // Eq. (5)
         }
         if (jok) {
 #pragma unroll

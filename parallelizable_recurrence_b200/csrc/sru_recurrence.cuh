@@ -93,6 +93,17 @@ __device__ __forceinline__ float2 sru_cell2(float2 c, float2 uc, float2 uf, floa
     return fma2(f, sub2(c, uc), uc);
 }
 
+// The two halves of sru_cell2, for chunks walked in two passes: the state
+// chain needs only the forget gate (Eqs. (2), (4)); the reset gate (Eq. (3))
+// and h (Eq. (5)) of every step of a chunk can then be computed without a
+// dependency between steps.  Same operations as sru_cell2, so the same bits.
+__device__ __forceinline__ float2 sru_forget2(float2 c, float2 uf, const GateParams2& p) {
+    return sigmoid2_nl2(fma2(p.nvf, c, fma2(uf, f2(kNegLog2e), p.nbf)));
+}
+__device__ __forceinline__ float2 sru_reset2(float2 c, float2 ur, const GateParams2& p) {
+    return sigmoid2_nl2(fma2(p.nvr, c, fma2(ur, f2(kNegLog2e), p.nbr)));
+}
+
 // Loads/stores of a channel pair (2 adjacent elements, 4- or 8-byte aligned).
 __device__ __forceinline__ float2 load_pair(const __nv_bfloat16* p) {
     const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
@@ -179,14 +190,23 @@ __device__ __forceinline__ float2 fwd_chunk_full(const UT* __restrict__ us, cons
         wr[i] = PW::load(us + (i * 3 + 2) * CJ + cj);
         wx[i] = load_pair(xs + i * CJ + cj);
     }
-    float2 hv[kChunkT];
+    // pass 1: the state chain (forget gate and c only)
+    float2 cprev[kChunkT], cs[kChunkT];
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
         const int i = DIR == 0 ? q : kChunkT - 1 - q;
-        float2 f, r;
-        c = sru_cell2(c, PW::unpack(wc[i]), PW::unpack(wf[i]), PW::unpack(wr[i]), p, f, r);
+        cprev[i] = c;
+        const float2 uc = PW::unpack(wc[i]);
+        c = fma2(sru_forget2(c, PW::unpack(wf[i]), p), sub2(c, uc), uc);  // Eq. (4)
+        cs[i] = c;
+    }
+    // pass 2: reset gate and h of every step, independent of one another
+    float2 hv[kChunkT];
+#pragma unroll
+    for (int i = 0; i < kChunkT; ++i) {
+        const float2 r = sru_reset2(cprev[i], PW::unpack(wr[i]), p);
         const float2 ax = mul2(alpha, wx[i]);
-        hv[i] = fma2(r, sub2(c, ax), ax);  // Eq. (5)
+        hv[i] = fma2(r, sub2(cs[i], ax), ax);  // Eq. (5)
     }
     if (STAGE) {
         asm volatile("" ::: "memory");  // the x reads above precede the writes over them
@@ -474,11 +494,15 @@ __device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const 
     if (STAGE) asm volatile("" ::: "memory");  // every read of the tile precedes the writes over it
     float2 cp[kChunkT], fs[kChunkT], rs[kChunkT];
 #pragma unroll
-    for (int q = 0; q < kChunkT; ++q) {
+    for (int q = 0; q < kChunkT; ++q) {  // the state chain (forget gate and c)
         const int i = DIR == 0 ? q : kChunkT - 1 - q;
         cp[i] = c;
-        c = sru_cell2(c, PW::unpack(wc[i]), PW::unpack(wf[i]), PW::unpack(wr[i]), p, fs[i], rs[i]);
+        const float2 uc = PW::unpack(wc[i]);
+        fs[i] = sru_forget2(c, PW::unpack(wf[i]), p);
+        c = fma2(fs[i], sub2(c, uc), uc);
     }
+#pragma unroll
+    for (int i = 0; i < kChunkT; ++i) rs[i] = sru_reset2(cp[i], PW::unpack(wr[i]), p);  // no chain
     float2 s_vf = f2(0.f), s_vr = f2(0.f), s_bf = f2(0.f), s_br = f2(0.f);
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
