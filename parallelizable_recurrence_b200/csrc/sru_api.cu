@@ -263,12 +263,12 @@ constexpr uint32_t kGemmBRows = (uint32_t)sru::gemm::P_CN;
 // tail_split (pair kernel, OUT == kOutF32 only): the output tiles of the last,
 // partial round of CTA pairs are cut in two k-pieces that add onto regions
 // zeroed here first (see sru::gemm::pair_next).
-template <bool A_MN, bool B_MN, int OUT, int L2HINT = 0>
+template <bool A_MN, bool B_MN, int OUT>
 sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
                           int64_t Kr, cudaStream_t st, int splits = 1, int64_t ldo = -1, bool tail_split = false) {
     if (ldo < 0) ldo = C;
     {
-        auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT, 0, 0, 0, L2HINT>;
+        auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT>;
         SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
         // the output as the epilogue's TMA store target: box 32 x 32, swizzled like the staging buffers
         CUtensorMap mo;
@@ -854,8 +854,7 @@ sru_status sru_project_backward(const void* dU, const void* X, const void* W, in
         CUtensorMap ma, mb;
         // A(r = n, red = m) = dU[m][n]: MN-major, ld = N; B(c = k, red = m) = X[m][k]: MN-major, ld = K
         if (!map_mnmajor(&ma, dU, N, M, N) || !map_mnmajor(&mb, X, K, M, K)) return SRU_ERR_INVALID;
-        // dW = dU^T X: dU read once (evict first), X read by every round of tiles (kept)
-        return launch_tc_gemm<true, true, sru::gemm::kOutF32, 1>(ma, mb, dW, N, K, M, st, 1, -1, /*tail_split=*/true);
+        return launch_tc_gemm<true, true, sru::gemm::kOutF32>(ma, mb, dW, N, K, M, st, 1, -1, /*tail_split=*/true);
     }
     return SRU_OK;
 }

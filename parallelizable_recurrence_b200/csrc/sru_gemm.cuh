@@ -159,10 +159,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16_pair(bool a_mn, bool b_mn) {
 // out + z * out_bstride.
 template <int BPOS>
 __device__ __forceinline__ void tma_load_tile_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y,
-                                                   int z, uint64_t policy = 0) {
-    if (BPOS == 0 && policy != 0)
-        tma_load_2d_pair_hint(dst, map, bar, x, y, policy);
-    else if (BPOS == 0)
+                                                   int z) {
+    if (BPOS == 0)
         tma_load_2d_pair(dst, map, bar, x, y);
     else if (BPOS == 1)
         tma_load_3d_pair(dst, map, bar, x, z, y);
@@ -259,10 +257,7 @@ __device__ __forceinline__ bool pair_next(int i, int p, int P, int units, int m_
     return true;
 }
 
-// L2HINT (non-batched launches): 1 = the A operand is read once (its loads
-// evicted first) and the B operand is read again by later rounds of tiles
-// (kept in L2): dW = dU^T X, where every round re-reads all of X.
-template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0, int CAUSAL = 0, int L2HINT = 0>
+template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0, int CAUSAL = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                         const __grid_constant__ CUtensorMap map_out, void* __restrict__ out, int M, int N, int K,
@@ -325,8 +320,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             uint32_t issued = 0;
             int stage = 0;
             uint32_t phase = 0;
-            const uint64_t pol_a = L2HINT == 1 ? l2_policy_evict_first() : 0;
-            const uint64_t pol_b = L2HINT == 1 ? l2_policy_evict_last() : 0;
             PairUnit w;
             for (int i = 0; !*abort_flag &&
                             pair_next<CAUSAL>(i, pair_id, n_pairs, units, m_tiles, n_tiles, splits, kblocks, kper,
@@ -346,16 +339,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     const uint32_t bar = leader_full0 + (uint32_t)stage * 8u;
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
                     if (!A_MN) {
-                        tma_load_tile_pair<BPA>(a_dst, &map_a, bar, k0, m0, z, pol_a);
+                        tma_load_tile_pair<BPA>(a_dst, &map_a, bar, k0, m0, z);
                     } else {
-                        tma_load_tile_pair<BPA>(a_dst, &map_a, bar, m0, k0, z, pol_a);
-                        tma_load_tile_pair<BPA>(a_dst + MN_BOX_BYTES, &map_a, bar, m0 + 64, k0, z, pol_a);
+                        tma_load_tile_pair<BPA>(a_dst, &map_a, bar, m0, k0, z);
+                        tma_load_tile_pair<BPA>(a_dst + MN_BOX_BYTES, &map_a, bar, m0 + 64, k0, z);
                     }
                     if (!B_MN) {
-                        tma_load_tile_pair<BPB>(b_dst, &map_b, bar, k0, n0, z, pol_b);
+                        tma_load_tile_pair<BPB>(b_dst, &map_b, bar, k0, n0, z);
                     } else {
-                        tma_load_tile_pair<BPB>(b_dst, &map_b, bar, n0, k0, z, pol_b);
-                        tma_load_tile_pair<BPB>(b_dst + MN_BOX_BYTES, &map_b, bar, n0 + 64, k0, z, pol_b);
+                        tma_load_tile_pair<BPB>(b_dst, &map_b, bar, n0, k0, z);
+                        tma_load_tile_pair<BPB>(b_dst + MN_BOX_BYTES, &map_b, bar, n0 + 64, k0, z);
                     }
                     ++issued;
                     if (++stage == P_STAGES) {

@@ -494,15 +494,11 @@ __device__ __forceinline__ void bwd_chunk_full(const UT* __restrict__ us, const 
     if (STAGE) asm volatile("" ::: "memory");  // every read of the tile precedes the writes over it
     float2 cp[kChunkT], fs[kChunkT], rs[kChunkT];
 #pragma unroll
-    for (int q = 0; q < kChunkT; ++q) {  // the state chain (forget gate and c)
+    for (int q = 0; q < kChunkT; ++q) {
         const int i = DIR == 0 ? q : kChunkT - 1 - q;
         cp[i] = c;
-        const float2 uc = PW::unpack(wc[i]);
-        fs[i] = sru_forget2(c, PW::unpack(wf[i]), p);
-        c = fma2(fs[i], sub2(c, uc), uc);
+        c = sru_cell2(c, PW::unpack(wc[i]), PW::unpack(wf[i]), PW::unpack(wr[i]), p, fs[i], rs[i]);
     }
-#pragma unroll
-    for (int i = 0; i < kChunkT; ++i) rs[i] = sru_reset2(cp[i], PW::unpack(wr[i]), p);  // no chain
     float2 s_vf = f2(0.f), s_vr = f2(0.f), s_bf = f2(0.f), s_br = f2(0.f);
 #pragma unroll
     for (int q = 0; q < kChunkT; ++q) {
