@@ -721,7 +721,8 @@ sru_status noalloc_scratch_address(cudaStream_t st, void** out) {
 // kernel hands the state between CTAs, so its whole grid must be resident):
 // the occupancy calculator's count of co-resident 2-CTA clusters, cached per
 // device.
-template <int NS>
+// WIDE: the kernel with 4-slice items (sru_fused_wide_kernel), else sru_fused_fwd_kernel<1>.
+template <bool WIDE>
 int64_t fused_resident_pairs() {
     static std::mutex mu;
     static int cache[kMaxDevices] = {0};
@@ -729,36 +730,41 @@ int64_t fused_resident_pairs() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
     std::lock_guard<std::mutex> lock(mu);
     if (cache[dev] == 0) {
-        auto kern = sru::fused::sru_fused_fwd_kernel<NS>;
-        constexpr size_t smem = sru::fused::FusedShape<NS>::kSmem;
+        const void* kern = WIDE ? reinterpret_cast<const void*>(sru::fused::sru_fused_wide_kernel)
+                                : reinterpret_cast<const void*>(sru::fused::sru_fused_fwd_kernel<1>);
+        const size_t smem = WIDE ? sru::fused::kWideSmem : sru::fused::FusedShape<1>::kSmem;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(2 * (sm_count() / 2)), 1, 1);
         cfg.blockDim = dim3(sru::fused::kThreads, 1, 1);
         cfg.dynamicSmemBytes = smem;
         int n = 0;
-        if (ensure_smem(reinterpret_cast<const void*>(kern), smem) != cudaSuccess ||
-            cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(kern), &cfg) != cudaSuccess)
+        if (ensure_smem(kern, smem) != cudaSuccess || cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess)
             n = 0;
         cache[dev] = n > 0 ? (n < sm_count() / 2 ? n : sm_count() / 2) : -1;
     }
     return cache[dev];
 }
 
-template <int NS>
+template <bool WIDE>
 sru_status launch_fused(const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& mu,
                         const sru::fused::FusedArgs& fa, int64_t L, int64_t B, int64_t d, int n_dir, cudaStream_t st) {
+    const int per = WIDE ? sru::fused::kWideSlices : 1;  // 64-channel slices per work item
     const int64_t nT = (L + sru::fused::kTt - 1) / sru::fused::kTt;
-    const int64_t njg = ((d + sru::fused::kCh - 1) / sru::fused::kCh + NS - 1) / NS;
+    const int64_t ngrp = ((d + sru::fused::kCh - 1) / sru::fused::kCh + per - 1) / per;
     const int64_t nbgp = (B + 2 * sru::fused::kBb - 1) / (2 * sru::fused::kBb);
-    const int64_t items = nT * n_dir * nbgp * njg;
+    const int64_t items = nT * n_dir * nbgp * ngrp;
     if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
-    auto kern = sru::fused::sru_fused_fwd_kernel<NS>;
-    constexpr size_t smem = sru::fused::FusedShape<NS>::kSmem;
-    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), smem));
-    const int64_t max_pairs = fused_resident_pairs<NS>();
+    const void* kern = WIDE ? reinterpret_cast<const void*>(sru::fused::sru_fused_wide_kernel)
+                            : reinterpret_cast<const void*>(sru::fused::sru_fused_fwd_kernel<1>);
+    const size_t smem = WIDE ? sru::fused::kWideSmem : sru::fused::FusedShape<1>::kSmem;
+    SRU_CUDA_TRY(ensure_smem(kern, smem));
+    const int64_t max_pairs = fused_resident_pairs<WIDE>();
     if (max_pairs < 1) return cuda_fail(cudaErrorLaunchOutOfResources);
     const int64_t pairs = items < max_pairs ? items : max_pairs;
-    kern<<<(unsigned)(2 * pairs), sru::fused::kThreads, smem, st>>>(mx, mw, mu, fa);
+    if (WIDE)
+        sru::fused::sru_fused_wide_kernel<<<(unsigned)(2 * pairs), sru::fused::kThreads, smem, st>>>(mx, mw, mu, fa);
+    else
+        sru::fused::sru_fused_fwd_kernel<1><<<(unsigned)(2 * pairs), sru::fused::kThreads, smem, st>>>(mx, mw, mu, fa);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
@@ -1047,6 +1053,8 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
         return SRU_ERR_INVALID;
     const WsLayout w = ws_layout(L, B, d, n_dir, SRU_FLAG_FORCE_SEQUENTIAL);  // the smallest layout
     if (workspace_bytes < w.total) return SRU_ERR_INVALID;
+    // wide items (4 slices, N = 256 products) where the per-item product is long: d >= 1024
+    const bool wide = d >= 1024;
     CUtensorMap mx, mw, mu;
     {
         const uint64_t dims[3] = {(uint64_t)d, (uint64_t)B, (uint64_t)L};
@@ -1058,7 +1066,8 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
     {
         const uint64_t dims[3] = {(uint64_t)d, (uint64_t)d, (uint64_t)(3 * n_dir)};
         const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)d * d * 2};
-        const uint32_t box[3] = {64, (uint32_t)(sru::fused::kCh / 2), 3};
+        // one gate block of 64 channels (wide), or half a slice's 32 channels of all 3 gates
+        const uint32_t box[3] = {64, wide ? 64u : (uint32_t)(sru::fused::kCh / 2), wide ? 1u : 3u};
         if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, W, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return SRU_ERR_INVALID;
     }
@@ -1067,7 +1076,7 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
         const uint64_t dims[5] = {(uint64_t)d, 3, (uint64_t)n_dir, (uint64_t)B, (uint64_t)L};
         const uint64_t strides[4] = {(uint64_t)d * 2, (uint64_t)3 * d * 2, (uint64_t)n_dir * 3 * d * 2,
                                      (uint64_t)B * n_dir * 3 * d * 2};
-        const uint32_t box[5] = {(uint32_t)sru::fused::kCh, 3, 1, (uint32_t)sru::fused::kBb,
+        const uint32_t box[5] = {(uint32_t)sru::fused::kCh, wide ? 1u : 3u, 1, (uint32_t)sru::fused::kBb,
                                  (uint32_t)sru::fused::kTt};
         if (!make_map(&mu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, U, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return SRU_ERR_INVALID;
@@ -1090,13 +1099,8 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
     fa.alpha = alpha;
     fa.write_u = U != nullptr;
     SRU_CUDA_TRY(cudaMemsetAsync(fa.carry, 0, (size_t)B * n_dir * d * sizeof(unsigned long long), st));
-    // Two 64-channel slices per work item only for inference layers of d >= 2048
-    // (measured on B200, L1024 B16 d2048: 310 against 325 us).  With U stored,
-    // the single accumulator buffer that two slices need holds the next item's
-    // products behind two walks and the U stores, and one slice per item is
-    // faster (333 against 337 us there; L2048 B64 d1024 x2: 1653 against 1859).
-    if (U == nullptr && d >= 2048) return launch_fused<2>(mx, mw, mu, fa, L, B, d, n_dir, st);
-    return launch_fused<1>(mx, mw, mu, fa, L, B, d, n_dir, st);
+    if (wide) return launch_fused<true>(mx, mw, mu, fa, L, B, d, n_dir, st);
+    return launch_fused<false>(mx, mw, mu, fa, L, B, d, n_dir, st);
 }
 
 sru_status sru_project_factored(const void* X, const void* Wq, const void* Wo, void* P, void* U, int u_t,
