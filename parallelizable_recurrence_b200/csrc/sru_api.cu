@@ -721,8 +721,6 @@ sru_status noalloc_scratch_address(cudaStream_t st, void** out) {
 // kernel hands the state between CTAs, so its whole grid must be resident):
 // the occupancy calculator's count of co-resident 2-CTA clusters, cached per
 // device.
-// WIDE: the kernel with 4-slice items (sru_fused_wide_kernel), else sru_fused_fwd_kernel<1>.
-template <bool WIDE>
 int64_t fused_resident_pairs() {
     static std::mutex mu;
     static int cache[kMaxDevices] = {0};
@@ -730,43 +728,18 @@ int64_t fused_resident_pairs() {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
     std::lock_guard<std::mutex> lock(mu);
     if (cache[dev] == 0) {
-        const void* kern = WIDE ? reinterpret_cast<const void*>(sru::fused::sru_fused_wide_kernel)
-                                : reinterpret_cast<const void*>(sru::fused::sru_fused_fwd_kernel<1>);
-        const size_t smem = WIDE ? sru::fused::kWideSmem : sru::fused::FusedShape<1>::kSmem;
+        const void* kern = reinterpret_cast<const void*>(sru::fused::sru_fused_fwd_kernel);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(2 * (sm_count() / 2)), 1, 1);
         cfg.blockDim = dim3(sru::fused::kThreads, 1, 1);
-        cfg.dynamicSmemBytes = smem;
+        cfg.dynamicSmemBytes = sru::fused::kSmemBytes;
         int n = 0;
-        if (ensure_smem(kern, smem) != cudaSuccess || cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess)
+        if (ensure_smem(kern, sru::fused::kSmemBytes) != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess)
             n = 0;
         cache[dev] = n > 0 ? (n < sm_count() / 2 ? n : sm_count() / 2) : -1;
     }
     return cache[dev];
-}
-
-template <bool WIDE>
-sru_status launch_fused(const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& mu,
-                        const sru::fused::FusedArgs& fa, int64_t L, int64_t B, int64_t d, int n_dir, cudaStream_t st) {
-    const int per = WIDE ? sru::fused::kWideSlices : 1;  // 64-channel slices per work item
-    const int64_t nT = (L + sru::fused::kTt - 1) / sru::fused::kTt;
-    const int64_t ngrp = ((d + sru::fused::kCh - 1) / sru::fused::kCh + per - 1) / per;
-    const int64_t nbgp = (B + 2 * sru::fused::kBb - 1) / (2 * sru::fused::kBb);
-    const int64_t items = nT * n_dir * nbgp * ngrp;
-    if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
-    const void* kern = WIDE ? reinterpret_cast<const void*>(sru::fused::sru_fused_wide_kernel)
-                            : reinterpret_cast<const void*>(sru::fused::sru_fused_fwd_kernel<1>);
-    const size_t smem = WIDE ? sru::fused::kWideSmem : sru::fused::FusedShape<1>::kSmem;
-    SRU_CUDA_TRY(ensure_smem(kern, smem));
-    const int64_t max_pairs = fused_resident_pairs<WIDE>();
-    if (max_pairs < 1) return cuda_fail(cudaErrorLaunchOutOfResources);
-    const int64_t pairs = items < max_pairs ? items : max_pairs;
-    if (WIDE)
-        sru::fused::sru_fused_wide_kernel<<<(unsigned)(2 * pairs), sru::fused::kThreads, smem, st>>>(mx, mw, mu, fa);
-    else
-        sru::fused::sru_fused_fwd_kernel<1><<<(unsigned)(2 * pairs), sru::fused::kThreads, smem, st>>>(mx, mw, mu, fa);
-    SRU_CUDA_TRY(cudaGetLastError());
-    return SRU_OK;
 }
 
 }  // namespace
@@ -1053,8 +1026,6 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
         return SRU_ERR_INVALID;
     const WsLayout w = ws_layout(L, B, d, n_dir, SRU_FLAG_FORCE_SEQUENTIAL);  // the smallest layout
     if (workspace_bytes < w.total) return SRU_ERR_INVALID;
-    // wide items (4 slices, N = 256 products) where the per-item product is long: d >= 1024
-    const bool wide = d >= 1024;
     CUtensorMap mx, mw, mu;
     {
         const uint64_t dims[3] = {(uint64_t)d, (uint64_t)B, (uint64_t)L};
@@ -1066,8 +1037,8 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
     {
         const uint64_t dims[3] = {(uint64_t)d, (uint64_t)d, (uint64_t)(3 * n_dir)};
         const uint64_t strides[2] = {(uint64_t)d * 2, (uint64_t)d * d * 2};
-        // one gate block of 64 channels (wide), or half a slice's 32 channels of all 3 gates
-        const uint32_t box[3] = {64, wide ? 64u : (uint32_t)(sru::fused::kCh / 2), wide ? 1u : 3u};
+        // half a slice's 32 channels of all 3 gates
+        const uint32_t box[3] = {64, (uint32_t)(sru::fused::kCh / 2), 3};
         if (!make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, W, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return SRU_ERR_INVALID;
     }
@@ -1076,7 +1047,7 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
         const uint64_t dims[5] = {(uint64_t)d, 3, (uint64_t)n_dir, (uint64_t)B, (uint64_t)L};
         const uint64_t strides[4] = {(uint64_t)d * 2, (uint64_t)3 * d * 2, (uint64_t)n_dir * 3 * d * 2,
                                      (uint64_t)B * n_dir * 3 * d * 2};
-        const uint32_t box[5] = {(uint32_t)sru::fused::kCh, wide ? 1u : 3u, 1, (uint32_t)sru::fused::kBb,
+        const uint32_t box[5] = {(uint32_t)sru::fused::kCh, 3, 1, (uint32_t)sru::fused::kBb,
                                  (uint32_t)sru::fused::kTt};
         if (!make_map(&mu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, U, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
             return SRU_ERR_INVALID;
@@ -1099,8 +1070,20 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
     fa.alpha = alpha;
     fa.write_u = U != nullptr;
     SRU_CUDA_TRY(cudaMemsetAsync(fa.carry, 0, (size_t)B * n_dir * d * sizeof(unsigned long long), st));
-    if (wide) return launch_fused<true>(mx, mw, mu, fa, L, B, d, n_dir, st);
-    return launch_fused<false>(mx, mw, mu, fa, L, B, d, n_dir, st);
+    const int64_t nT = (L + sru::fused::kTt - 1) / sru::fused::kTt;
+    const int64_t njs = (d + sru::fused::kCh - 1) / sru::fused::kCh;
+    const int64_t nbgp = (B + 2 * sru::fused::kBb - 1) / (2 * sru::fused::kBb);
+    const int64_t items = nT * n_dir * nbgp * njs;
+    if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
+    const void* kern = reinterpret_cast<const void*>(sru::fused::sru_fused_fwd_kernel);
+    SRU_CUDA_TRY(ensure_smem(kern, sru::fused::kSmemBytes));
+    const int64_t max_pairs = fused_resident_pairs();
+    if (max_pairs < 1) return cuda_fail(cudaErrorLaunchOutOfResources);
+    const int64_t pairs = items < max_pairs ? items : max_pairs;
+    sru::fused::sru_fused_fwd_kernel<<<(unsigned)(2 * pairs), sru::fused::kThreads, sru::fused::kSmemBytes, st>>>(
+        mx, mw, mu, fa);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
 }
 
 sru_status sru_project_factored(const void* X, const void* Wq, const void* Wo, void* P, void* U, int u_t,

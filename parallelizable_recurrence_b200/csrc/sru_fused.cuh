@@ -219,37 +219,23 @@ __device__ __forceinline__ float2 fused_chunk(WordAddr word, int q, int i0, uint
     return c;
 }
 
-// Shape of a work item: NS 64-channel slices side by side (N = 192 * NS
-// accumulator columns as NS MMAs of N = 192 sharing the X tile).  NS = 2
-// halves the X traffic per flop (the L2-to-SM feed bounds a 192-column
-// product) at the price of a single-buffered accumulator and a ring of 3
-// stages; NS = 1 keeps two accumulators and 6 stages, for layers whose
-// per-item product is short and whose chains lie on the critical path.
-template <int NS>
-struct FusedShape {
-    static constexpr int kStages = NS == 1 ? 6 : 3;
-    static constexpr uint32_t kStageBytes = kABytes + NS * kBBytes;
-    static constexpr int kAccBufs = NS == 1 ? 2 : 1;  // accumulators in flight
-    static constexpr size_t kSmem = (size_t)kStages * kStageBytes + NS * kUTileBytes + 1024 + 256;
-    static_assert(kSmem <= 232448, "fused kernel shared memory");
-    static_assert(NS == 1 || NS == 2, "slices per item");
-};
+constexpr int kStages = 6;
+constexpr uint32_t kStageBytes = kABytes + kBBytes;  // 28 KB: X tile + this CTA's half of the W_cat rows
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + kUTileBytes + 1024 + 256;
+static_assert(kSmemBytes <= 232448, "fused kernel shared memory");
 
 // map_x: X as 3-D (d, B, L) bf16, box (64, kBb, kTt), 128-byte swizzle.
 // map_w: W_cat as 3-D (d, d, n_dir*3) bf16, box (64, 32, 3), 128-byte swizzle.
 // map_u: U as 5-D (d, 3, n_dir, B, L) bf16, box (64, 3, 1, kBb, kTt), 128-byte
 //        swizzle (only used when a.write_u).
-template <int NS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     sru_fused_fwd_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                          const __grid_constant__ CUtensorMap map_u, const FusedArgs a) {
-    using Sh = FusedShape<NS>;
-    constexpr int kStages = Sh::kStages;
-    constexpr uint32_t kStageBytes = Sh::kStageBytes;
-    constexpr int kAccBufs = Sh::kAccBufs;
+    constexpr int kAccBufs = 2;  // accumulators in flight
+    constexpr int NS = 1;        // 64-channel slices per work item (the loops below take any count; one measured fastest)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* utile_p = smem + kStages * kStageBytes;  // 1024-aligned; NS tiles of kUTileBytes
+    uint8_t* utile_p = smem + kStages * kStageBytes;  // 1024-aligned U tile(s)
     uint64_t* full = reinterpret_cast<uint64_t*>(utile_p + NS * kUTileBytes);
     uint64_t* empty = full + kStages;
     uint64_t* tfull = empty + kStages;
@@ -551,354 +537,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     if (jok) st_carry2(cw, (unsigned)(tt + 1), c);
                 } else if (jok) {
                     store_pair(a.c_T + (size_t)bd * d + j, c);
-                }
-            }
-        }
-        if (issuer && stored) bulk_wait_group<0>();  // every U store has landed
-    }
-    tc_fence_before_sync();
-    __syncthreads();
-    cluster_sync_all();  // no CTA leaves while its peer may still signal its barriers
-    if (warp == 1) {
-        tc_fence_after_sync();
-        tmem_dealloc_pair(tmem_base, kTmemCols);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Wide work items, for layers whose per-item products are long (d >= 1024):
-// 4 channel slices (256 channels) per item, whose 12 gate blocks of 64 W_cat
-// rows -- in [slice][gate] order -- are multiplied as three MMA chunks of
-// N = 256 (the standalone projection's tile shape; a 192-column product moves
-// 17 % more bytes from L2 per flop and measured 306 against 250 us for the
-// training layer's projection).  Chunk k's accumulator holds blocks 4k .. 4k+3
-// (CTA 0 supplies the first two blocks' W rows, CTA 1 the other two); the
-// epilogue copies each block into one of 6 staging buffers [t][b][64 ch]
-// (block i of the item into buffer i % 6, so slice s uses buffers 3(s % 2) ..
-// 3(s % 2) + 2), and walks a slice as soon as its three gate blocks are in:
-// slice 0 after chunk 0, slice 1 after chunk 1, slices 2 and 3 after chunk 2.
-// The accumulator is double-buffered (2 x 256 TMEM columns), so the next
-// chunk's products run under the transpose and the walks.
-constexpr int kWideSlices = 4;
-constexpr int kWideChunks = 3;                          // 12 gate blocks / 4 per chunk
-constexpr int kWideStages = 4;
-constexpr uint32_t kWideBlockBytes = kRows * 128;       // 16 KB: 128 (t, b) rows x 64 bf16
-constexpr uint32_t kWideStageBytes = kABytes + 2 * (64 * kBK * 2);  // X 16 KB + 2 W blocks 16 KB
-constexpr int kWideBufs = 6;
-constexpr size_t kWideSmem = (size_t)kWideStages * kWideStageBytes + kWideBufs * kWideBlockBytes + 1024 + 256;
-static_assert(kWideSmem <= 232448, "wide fused kernel shared memory");
-
-__host__ __device__ constexpr uint32_t idesc_wide() {  // N = 256, M = 256 (cta_group::2), bf16 -> fp32
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
-}
-// address of this thread's bf16 pair (lane l) at row r of a staging block buffer
-__device__ __forceinline__ uint32_t block_word(uint32_t buf, int r, int l) {
-    return buf + (uint32_t)r * 128u + ((((uint32_t)l >> 2) ^ ((uint32_t)r & 7u)) << 4) + ((uint32_t)l & 3u) * 4u;
-}
-
-// map_x: X as 3-D (d, B, L) bf16, box (64, kBb, kTt), 128-byte swizzle.
-// map_w: W_cat as 3-D (d, d, n_dir*3) bf16, box (64, 64, 1), 128-byte swizzle.
-// map_u: U as 5-D (d, 3, n_dir, B, L) bf16, box (64, 1, 1, kBb, kTt), 128-byte
-//        swizzle (only used when a.write_u).
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    sru_fused_wide_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
-                          const __grid_constant__ CUtensorMap map_u, const FusedArgs a) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* stage_p = smem + kWideStages * kWideStageBytes;  // 1024-aligned: 6 staging blocks
-    uint64_t* full = reinterpret_cast<uint64_t*>(stage_p + kWideBufs * kWideBlockBytes);
-    uint64_t* empty = full + kWideStages;
-    uint64_t* tfull = empty + kWideStages;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile uint32_t* consumed = reinterpret_cast<volatile uint32_t*>(tmem_slot + 2);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();  // 0 = leader
-    const int pair_id = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
-    const int L = a.L, B = a.B, d = a.d, n_dir = a.n_dir;
-    const int nT = (L + kTt - 1) / kTt;
-    const int njs = (d + kCh - 1) / kCh;
-    const int ngrp = (njs + kWideSlices - 1) / kWideSlices;  // groups of 4 slices (one item each)
-    const int nbgp = (B + 2 * kBb - 1) / (2 * kBb);
-    const int streams = n_dir * nbgp * ngrp;
-    const int items = nT * streams;
-    const int kblocks = (d + kBK - 1) / kBK;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kWideStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        for (int acc = 0; acc < 2; ++acc) {
-            mbar_init(&tfull[acc], 1);
-            mbar_init(&tempty[acc], 8);  // leader's: the 4 epilogue warps of each CTA
-        }
-        mbar_init(drain, 1);
-        *abort_flag = 0;
-        *consumed = 0;
-        fence_mbar_init();
-        tma_prefetch_desc(&map_x);
-        tma_prefetch_desc(&map_w);
-        if (a.write_u) tma_prefetch_desc(&map_u);
-    }
-    if (warp == 1) {
-        tmem_alloc_pair(tmem_slot, kTmemCols);
-        tmem_relinquish_pair();
-    }
-    tc_fence_before_sync();
-    cluster_sync_all();
-    tc_fence_after_sync();
-    const uint32_t tmem_base = *tmem_slot;
-    const uint32_t leader_full0 = mapa_shared(smem_u32(&full[0]), 0);
-    const uint32_t leader_tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
-
-    auto decode = [&](int u, int& tt, int& dir, int& bgp, int& grp) {
-        tt = u / streams;
-        int s = u % streams;
-        grp = s % ngrp;
-        s /= ngrp;
-        bgp = s % nbgp;
-        dir = s / nbgp;
-    };
-
-    if (warp == 0) {
-        if (lane == 0) {
-            // ------------------------------------------------------ producer (both CTAs)
-            uint32_t issued = 0;
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int u = pair_id; u < items && !*abort_flag; u += n_pairs) {
-                int tt, dir, bgp, grp;
-                decode(u, tt, dir, bgp, grp);
-                const int tp = dir == 0 ? tt : nT - 1 - tt;
-                const int b0 = bgp * 2 * kBb + (int)rank * kBb;
-                for (int ck = 0; ck < kWideChunks && !*abort_flag; ++ck) {
-                    for (int kb = 0; kb < kblocks; ++kb) {
-                        if (!mbar_wait(&empty[stage], phase ^ 1u, kErrTimeoutMma) || *abort_flag) {
-                            *abort_flag = 1;
-                            break;
-                        }
-                        uint8_t* a_dst = smem + stage * kWideStageBytes;
-                        const uint32_t bar = leader_full0 + (uint32_t)stage * 8u;
-                        if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kWideStageBytes);
-                        tma_load_3d_pair(a_dst, &map_x, bar, kb * kBK, b0, tp * kTt);
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {  // this CTA's two gate blocks of the chunk
-                            const int blk = ck * 4 + (int)rank * 2 + e;
-                            const int sl = blk / 3, g = blk % 3;
-                            tma_load_3d_pair(a_dst + kABytes + e * (64 * kBK * 2), &map_w, bar, kb * kBK,
-                                             (grp * kWideSlices + sl) * kCh, dir * 3 + g);
-                        }
-                        ++issued;
-                        if (++stage == kWideStages) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
-                    }
-                }
-            }
-            if (*abort_flag && rank == 0) {
-                for (uint32_t qd = *consumed; qd < issued; ++qd)
-                    mbar_wait(&full[qd % kWideStages], (qd / kWideStages) & 1u, kErrTimeoutLoad);
-            }
-        }
-    } else if (warp == 1) {
-        if (lane == 0 && rank == 0) {
-            // ------------------------------------------------------ MMA issuer (leader)
-            constexpr uint32_t idesc = idesc_wide();
-            int stage = 0;
-            uint32_t phase = 0, nconsumed = 0;
-            int ic = 0;  // chunks issued
-            for (int u = pair_id; u < items && !*abort_flag; u += n_pairs) {
-                for (int ck = 0; ck < kWideChunks && !*abort_flag; ++ck, ++ic) {
-                    const int acc = ic & 1;
-                    const uint32_t acc_phase = (ic >> 1) & 1;
-                    if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, kErrTimeoutEpilogue)) {
-                        *abort_flag = 1;
-                        break;
-                    }
-                    tc_fence_after_sync();
-                    bool ok = true;
-                    for (int kb = 0; kb < kblocks; ++kb) {
-                        if (!mbar_wait(&full[stage], phase, kErrTimeoutLoad)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after_sync();
-                        const uint32_t a_addr = smem_u32(smem + stage * kWideStageBytes);
-#pragma unroll
-                        for (int kk = 0; kk < kBK / 16; ++kk)
-                            tc_mma_bf16_pair(tmem_base + (uint32_t)acc * kAccCols, sdesc_sw128(a_addr + kk * 32),
-                                             sdesc_sw128(a_addr + kABytes + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
-                        tc_commit_pair_mc(&empty[stage], 0x3);
-                        *consumed = ++nconsumed;
-                        if (++stage == kWideStages) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
-                    }
-                    if (!ok) {
-                        *abort_flag = 1;
-                        break;
-                    }
-                    tc_commit_pair_mc(&tfull[acc], 0x3);
-                }
-            }
-            tc_commit_pair_mc(drain, 0x1);
-            mbar_wait(drain, 0, kErrTimeoutMma);
-        }
-    } else {
-        // ---------------------------------------------------------- epilogue (both CTAs)
-        const int q = warp & 3;  // TMEM lane quarter = this warp's batch row in the group
-        const uint32_t stage0 = smem_u32(stage_p);
-        const bool issuer = warp == 2 && lane == 0;  // sends the U blocks by TMA
-        const int cj = 2 * lane;
-        const float2 alpha2 = f2(a.alpha);
-        const size_t tstride_x = (size_t)B * d;
-        const size_t tstride_h = (size_t)B * n_dir * d;
-        const int nch = (L + kChunkT - 1) / kChunkT;
-        int ic = 0;
-        bool stored = false, aborted = false;
-        for (int u = pair_id; u < items && !aborted; u += n_pairs) {
-            int tt, dir, bgp, grp;
-            decode(u, tt, dir, bgp, grp);
-            const int tp = dir == 0 ? tt : nT - 1 - tt;
-            const int b0 = bgp * 2 * kBb + (int)rank * kBb;
-            const int b = b0 + q;
-            const bool brow = b < B;
-            const int bd = b * n_dir + dir;
-            const int t_base = tp * kTt;
-            const int nrows = min(kTt, L - t_base);
-            const int i_first = dir == 0 ? 0 : kTt - kChunkT;
-            const int i_second = kTt - kChunkT - i_first;
-            // rows of this tile that exist (t < L) and are not padded, bit i = step t_base + i
-            bool vrow = brow && lane < nrows;
-            if (vrow && a.mask != nullptr) vrow = a.mask[(size_t)(t_base + lane) * B + b] == 0;
-            const uint32_t valid = __ballot_sync(0xffffffffu, vrow);
-            for (int ck = 0; ck < kWideChunks; ++ck, ++ic) {
-                const int acc = ic & 1;
-                const uint32_t acc_phase = (ic >> 1) & 1;
-                const bool ok = mbar_wait(&tfull[acc], acc_phase, kErrTimeoutMma);
-                // earlier U stores must be done reading the staging blocks before they are rewritten
-                if (issuer && stored) bulk_wait_group_read<0>();
-                if (epi_sync_or(!__all_sync(0xffffffffu, ok) || *abort_flag)) {
-                    *abort_flag = 1;
-                    aborted = true;
-                    break;
-                }
-                tc_fence_after_sync();
-                // ---- the chunk's 4 gate blocks -> staging buffers (block i of the item -> buffer i % 6)
-                {
-                    const int r = q * 32 + lane;
-#pragma unroll 1
-                    for (int c2 = 0; c2 < 4; ++c2) {  // one 64-column gate block per pass
-                        uint32_t v[2][32];
-                        const uint32_t taddr =
-                            tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)acc * kAccCols + (uint32_t)c2 * 64;
-                        tmem_ld_32x32b_x32(taddr, v[0]);
-                        tmem_ld_32x32b_x32(taddr + 32, v[1]);
-                        tc_wait_ld();
-                        const uint32_t buf = stage0 + (uint32_t)((ck * 4 + c2) % kWideBufs) * kWideBlockBytes;
-#pragma unroll
-                        for (int k = 0; k < 2; ++k) {
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                uint32_t w[4];
-#pragma unroll
-                                for (int k2 = 0; k2 < 4; ++k2) {
-                                    __nv_bfloat162 two = __floats2bfloat162_rn(__uint_as_float(v[k][e * 8 + 2 * k2]),
-                                                                               __uint_as_float(v[k][e * 8 + 2 * k2 + 1]));
-                                    w[k2] = *reinterpret_cast<uint32_t*>(&two);
-                                }
-                                const uint32_t chunk = (uint32_t)(k * 4 + e);
-                                st_shared_v4(buf + (uint32_t)r * 128u + ((chunk ^ ((uint32_t)r & 7u)) << 4), w[0], w[1],
-                                             w[2], w[3]);
-                            }
-                        }
-                    }
-                }
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)acc * 8u);  // accumulator free
-                fence_proxy_async_shared();  // the blocks' writes, visible to the TMA stores
-                epi_sync();
-                // slices whose three gate blocks are now staged: [s_lo, s_hi)
-                const int s_lo = ck == 0 ? 0 : ck, s_hi = ck == 0 ? 1 : (ck == 1 ? 2 : 4);
-                if (issuer && a.write_u && b0 < B) {
-                    for (int sl = s_lo; sl < s_hi; ++sl) {
-                        if (grp * kWideSlices + sl >= njs) break;
-#pragma unroll
-                        for (int g = 0; g < 3; ++g)
-                            tma_store_5d(&map_u, stage_p + ((sl * 3 + g) % kWideBufs) * kWideBlockBytes,
-                                         (grp * kWideSlices + sl) * kCh, g, dir, b0, t_base);
-                    }
-                    bulk_commit_group();
-                    stored = true;
-                }
-                if (!brow) continue;
-                // ---- Eqs. (2)-(5) for each completed slice, channel pair (j, j+1)
-#pragma unroll 1
-                for (int sl = s_lo; sl < s_hi; ++sl) {
-                    const int js = grp * kWideSlices + sl;
-                    if (js >= njs) break;  // a slice wholly beyond d
-                    const int j = js * kCh + cj;
-                    const bool jok = j < d;
-                    const float* xp = a.x + (size_t)t_base * tstride_x + (size_t)b * d + j;
-                    float* hp = a.h + (size_t)t_base * tstride_h + (size_t)bd * d + j;
-                    unsigned long long* cw = a.carry + (size_t)bd * d + j;
-                    float2 xa[kChunkT], xb[kChunkT];
-                    load_x_half(xa, xp, i_first, nrows, tstride_x, jok);
-                    GateParams2 p = make_gate_params2(f2(0.f), f2(0.f), f2(0.f), f2(0.f));
-                    float2 c = f2(0.f);
-                    if (jok) {
-                        p = make_gate_params2(load_pair(a.v + (dir * 2 + 0) * d + j),
-                                              load_pair(a.v + (dir * 2 + 1) * d + j),
-                                              load_pair(a.bias + (dir * 2 + 0) * d + j),
-                                              load_pair(a.bias + (dir * 2 + 1) * d + j));
-                        if (tt == 0) {
-                            if (a.c0 != nullptr) c = load_pair(a.c0 + (size_t)bd * d + j);
-                        } else {
-                            // the state the previous tile of this stream handed over (bounded wait)
-                            const uint64_t t0 = globaltimer_ns();
-                            for (;;) {
-                                unsigned g0, g1;
-                                ld_carry2(cw, g0, g1, c);
-                                if (g0 == (unsigned)tt && g1 == (unsigned)tt) break;
-                                if (*reinterpret_cast<volatile unsigned*>(&g_error_word) != 0u) break;
-                                if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                                    record_error(kErrTimeoutScan);
-                                    break;
-                                }
-                            }
-                        }
-                    }
-                    load_x_half(xb, xp, i_second, nrows, tstride_x, jok);
-                    const uint32_t bc = stage0 + (uint32_t)((sl * 3 + 0) % kWideBufs) * kWideBlockBytes;
-                    const uint32_t bf = stage0 + (uint32_t)((sl * 3 + 1) % kWideBufs) * kWideBlockBytes;
-                    const uint32_t br = stage0 + (uint32_t)((sl * 3 + 2) % kWideBufs) * kWideBlockBytes;
-                    auto word = [&](int r, int g) { return block_word(g == 0 ? bc : (g == 1 ? bf : br), r, lane); };
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int i0 = hh == 0 ? i_first : i_second;
-                        const int tc = (t_base + i0) / kChunkT;
-                        if (tc >= nch) continue;  // wholly beyond L
-                        if (a.ckpt != nullptr && jok) store_pair(a.ckpt + ((size_t)tc * B * n_dir + bd) * d + j, c);
-                        const uint32_t v16 = (valid >> i0) & ((1u << kChunkT) - 1u);
-                        if (dir == 0)
-                            c = fused_chunk<0>(word, q, i0, v16, c, p, alpha2, hh == 0 ? xa : xb, hp, tstride_h, jok,
-                                               nrows);
-                        else
-                            c = fused_chunk<1>(word, q, i0, v16, c, p, alpha2, hh == 0 ? xa : xb, hp, tstride_h, jok,
-                                               nrows);
-                    }
-                    if (tt + 1 < nT) {
-                        if (jok) st_carry2(cw, (unsigned)(tt + 1), c);
-                    } else if (jok) {
-                        store_pair(a.c_T + (size_t)bd * d + j, c);
-                    }
                 }
             }
         }

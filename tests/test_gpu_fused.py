@@ -13,9 +13,8 @@ Checks per case:
     bit-identical gradients (the checkpoints are the same).
 Cases span several time tiles (32 steps), ragged L, B (not a multiple of the
 8 rows of a CTA pair) and d (not a multiple of the 64-channel slice), masks
-with holes, both directions, c0 given or not, alpha != 1, and both item
-shapes (one 64-channel slice per item for d < 1024; from d = 1024, four slices
-whose gate blocks are multiplied as three 256-column chunks).
+with holes, both directions, c0 given or not, alpha != 1, and widths from one
+64-channel slice to 32 slices per direction.
 """
 import numpy as np
 import pytest
@@ -64,9 +63,9 @@ CASES = [  # L, B, d, n_dir, seed, masked, c0, alpha
     (130, 12, 200, 2, 13, True, True, 0.5),     # ragged everything, both directions, mask with a hole
     (257, 16, 64, 2, 14, True, False, 1.0),     # many time tiles handed between CTAs
     (33, 9, 512, 1, 15, True, True, -2.0),      # L one past a tile, B one past a pair
-    (40, 5, 1088, 2, 18, True, True, 0.75),     # wide items (d >= 1024): 4 slices each, the last one's 3 beyond d
-    (70, 8, 1024, 1, 19, False, False, 1.0),    # wide items, whole groups of 4 slices
-    (100, 3, 2048, 1, 20, True, True, 1.0),     # wide items over several time tiles, a lone batch group
+    (40, 5, 1088, 2, 18, True, True, 0.75),     # 17 slices, the last one 64 wide; both directions
+    (70, 8, 1024, 1, 19, False, False, 1.0),    # 16 whole slices
+    (100, 3, 2048, 1, 20, True, True, 1.0),     # 32 slices over several time tiles, a lone batch group
 ]
 
 
