@@ -449,10 +449,48 @@ def _layer_bidir(dev, flush, sru):
     return {"bidir_masked L2048 B64 d1024 x2": e}
 
 
+def _layer_producers(dev, flush, sru):
+    # the other producers of U at the training layer's shape (d' = d/4): the factorised
+    # projection (forward and backward) and SRU++'s attention producer
+    import torch
+    L, B, d = 1024, 16, 2048
+    dp, M, N = d // 4, L * B, 3 * d
+    g = torch.Generator(device=dev).manual_seed(6)
+    X = torch.randn(M, d, device=dev, generator=g).to(torch.bfloat16)
+    Wq = ((torch.rand(dp, d, device=dev, generator=g) * 2 - 1) * (3.0 / d) ** 0.5).to(torch.bfloat16)
+    Wo = ((torch.rand(N, dp, device=dev, generator=g) * 2 - 1) * (3.0 / dp) ** 0.5).to(torch.bfloat16)
+    Wkv = ((torch.rand(2 * dp, dp, device=dev, generator=g) * 2 - 1) * (3.0 / dp) ** 0.5).to(torch.bfloat16)
+    P = torch.empty(M, dp, device=dev, dtype=torch.bfloat16)
+    U = torch.empty(M, N, device=dev, dtype=torch.bfloat16)
+    dU = torch.randn(M, N, device=dev, generator=g).to(torch.bfloat16)
+    dP = torch.empty(M, dp, device=dev, dtype=torch.bfloat16)
+    dX = torch.zeros(M, d, device=dev)
+    dWq, dWo = torch.empty(dp, d, device=dev), torch.empty(N, dp, device=dev)
+    ffl = 2.0 * M * dp * (d + N)
+    t_f = _time_ms(lambda: sru.sru_project_factored(X, Wq, Wo, P, U), flush)
+    t_fb = _time_ms(lambda: sru.sru_project_factored_backward(dU, X, Wq, Wo, P, dP, dX=dX, accumulate=True,
+                                                              dWq=dWq, dWo=dWo), flush)
+    aws = torch.empty(int(sru.load_library().sru_attention_workspace_bytes(L, B, dp)), dtype=torch.uint8,
+                      device=dev)
+    proj = 2.0 * M * dp * (d + 2 * dp + N)  # Q, [K | V] and the output products
+    e = {"factored": _tc_entry("sru_project_factored (U = (X Wq^T) Wo^T)", t_f, ffl),
+         "factored_backward": _tc_entry("sru_project_factored_backward (dX, dWq, dWo)", t_fb, 2.0 * ffl)}
+    for causal in (True, False):
+        # scores and P.V: 2 L^2 d' flops each per batch row, or only the (t, s <= t) entries when causal
+        att = 2.0 * 2.0 * B * dp * (L * (L + 1) / 2.0 if causal else float(L * L))
+        t_a = _time_ms(lambda: sru.sru_attention_project(X, Wq, Wkv, Wo, U, L, B, 0.5, causal=causal,
+                                                         workspace=aws), flush)
+        ent = _tc_entry("sru_attention_project (" + ("causal" if causal else "full") + " attention)", t_a,
+                        proj + att)
+        ent["tokens_per_s"] = M / (t_a / 1e3)
+        e["attention_causal" if causal else "attention_full"] = ent
+    return {"producers L1024 B16 d2048 d'512": e}
+
+
 # recurrence-only layers first, the product-heavy ones last (so that a power
 # cap reached under the products does not slow the latency-bound recurrences)
 WORKLOAD_LAYERS = {"rec_only": _layer_rec_only, "scan_regime": _layer_scan_regime, "lm_fwd": _layer_lm_fwd,
-                   "lm_train_fused": _layer_lm_train_fused, "bidir_masked": _layer_bidir}
+                   "lm_train_fused": _layer_lm_train_fused, "producers": _layer_producers, "bidir_masked": _layer_bidir}
 
 
 def measure_workloads(dev, peaks, only=None):
