@@ -259,3 +259,83 @@ def attention_project(X, Wq, Wk, Wv, Wo, alpha, L, B, causal=True, ln_gamma=None
         var = ((R - mu) ** 2).mean(axis=1, keepdims=True)
         R = (R - mu) / np.sqrt(var + ln_eps) * _as_f64(ln_gamma) + _as_f64(ln_beta)
     return R @ Wo.T
+
+
+def attention_project_backward(dU, X, Wq, Wk, Wv, Wo, alpha, L, B, causal=True, ln_gamma=None, ln_beta=None,
+                               ln_eps=1e-5):
+    """Reverse-mode derivative of attention_project for Loss = sum(dU * U), in
+    fp64, taking the forward's steps backwards one at a time (the chain rule on
+    each line of attention_project; the forward values are recomputed here):
+
+      U = R Wo^T                     dWo = dU^T R,  dR = dU Wo
+      R = layernorm(Z) g + b         dg = sum_m dR * Zhat,  db = sum_m dR,
+                                     dZ = (dZhat - mean(dZhat) - Zhat mean(dZhat * Zhat)) / sigma,
+                                     dZhat = dR g   (or dZ = dR without the norm)
+      Z = Q + alpha A                dQ = dZ,  dA = alpha dZ
+      A_t = sum_s p_ts V_s           dV_s += p_ts dA_t,  dp_ts = V_s . dA_t
+      p_t = softmax(q_t K^T / sqrt(d'))
+                                     ds_ts = p_ts (dp_ts - sum_s' p_ts' dp_ts') / sqrt(d')
+                                     dQ_t += sum_s ds_ts K_s,  dK_s += ds_ts Q_t
+      K = Q Wk^T, V = Q Wv^T         dQ += dK Wk + dV Wv,  dWk = dK^T Q,  dWv = dV^T Q
+      Q = X Wq^T                     dWq = dQ^T X,  dX = dQ Wq
+
+    Returns a dict with dX (L*B, d), dWq, dWk, dWv, dWo and, with the norm,
+    dgamma and dbeta (d',), all float64.
+    """
+    dU, X, Wq, Wk, Wv, Wo = (_as_f64(a) for a in (dU, X, Wq, Wk, Wv, Wo))
+    Q = X @ Wq.T
+    K = Q @ Wk.T
+    V = Q @ Wv.T
+    dp = Q.shape[1]
+    A = np.zeros_like(Q)
+    probs = {}
+    for b in range(B):
+        rows = np.arange(L) * B + b
+        Qb, Kb, Vb = Q[rows], K[rows], V[rows]
+        for t in range(L):
+            n = t + 1 if causal else L
+            s = Kb[:n] @ Qb[t] / np.sqrt(dp)
+            p = np.exp(s - s.max())
+            p = p / p.sum()
+            probs[(b, t)] = p
+            A[rows[t]] = p @ Vb[:n]
+    Z = Q + alpha * A
+    out = {}
+    if ln_gamma is not None:
+        g = _as_f64(ln_gamma)
+        mu = Z.mean(axis=1, keepdims=True)
+        sigma = np.sqrt(((Z - mu) ** 2).mean(axis=1, keepdims=True) + ln_eps)
+        Zhat = (Z - mu) / sigma
+        R = Zhat * g + _as_f64(ln_beta)
+    else:
+        R = Z
+    out["dWo"] = dU.T @ R
+    dR = dU @ Wo
+    if ln_gamma is not None:
+        out["dgamma"] = (dR * Zhat).sum(axis=0)
+        out["dbeta"] = dR.sum(axis=0)
+        dZhat = dR * g
+        dZ = (dZhat - dZhat.mean(axis=1, keepdims=True) - Zhat * (dZhat * Zhat).mean(axis=1, keepdims=True)) / sigma
+    else:
+        dZ = dR
+    dQ = dZ.copy()
+    dA = alpha * dZ
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    for b in range(B):
+        rows = np.arange(L) * B + b
+        Qb, Kb, Vb = Q[rows], K[rows], V[rows]
+        for t in range(L):
+            n = t + 1 if causal else L
+            p = probs[(b, t)]
+            dV[rows[:n]] += np.outer(p, dA[rows[t]])
+            dpt = Vb[:n] @ dA[rows[t]]
+            ds = p * (dpt - p @ dpt) / np.sqrt(dp)
+            dQ[rows[t]] += ds @ Kb[:n]
+            dK[rows[:n]] += np.outer(ds, Qb[t])
+    dQ += dK @ Wk + dV @ Wv
+    out["dWk"] = dK.T @ Q
+    out["dWv"] = dV.T @ Q
+    out["dWq"] = dQ.T @ X
+    out["dX"] = dQ @ Wq
+    return out

@@ -98,3 +98,65 @@ def test_two_token_softmax_scaled_by_sqrt_dprime():
     a1 = (w0 * 3 * a + w1 * 3 * b) / (w0 + w1)
     np.testing.assert_allclose(U[:, 0], [a + 3 * a, b + a1], rtol=1e-12)
     np.testing.assert_array_equal(U[:, 1:], 0.0)
+
+
+# ------------------------------------------------------------ the backward
+def _loss(dU, *args, **kw):
+    return float((dU * oracle.attention_project(*args, **kw)).sum())
+
+
+def _central(f, arr, idx, h=1e-6):
+    old = arr[idx]
+    arr[idx] = old + h
+    up = f()
+    arr[idx] = old - h
+    dn = f()
+    arr[idx] = old
+    return (up - dn) / (2 * h)
+
+
+def _check_backward_against_differences(causal, with_ln, alpha, seed):
+    # every input element's gradient against a central difference of the
+    # forward oracle's loss sum(dU * U): pins each step of the chain rule
+    X, Wq, Wk, Wv, Wo, L, B = _case(seed=seed, L=4, B=2, d=6, dp=4, N=5)
+    rng = np.random.default_rng(100 + seed)
+    dU = rng.standard_normal((L * B, Wo.shape[0]))
+    g = 1.0 + 0.3 * rng.standard_normal(Wq.shape[0]) if with_ln else None
+    be = 0.2 * rng.standard_normal(Wq.shape[0]) if with_ln else None
+    kw = dict(causal=causal, ln_gamma=g, ln_beta=be)
+    got = oracle.attention_project_backward(dU, X, Wq, Wk, Wv, Wo, alpha, L, B, **kw)
+    named = {"dX": X, "dWq": Wq, "dWk": Wk, "dWv": Wv, "dWo": Wo}
+    if with_ln:
+        named.update(dgamma=g, dbeta=be)
+    else:
+        assert "dgamma" not in got and "dbeta" not in got
+    for name, arr in named.items():
+        assert got[name].shape == arr.shape, name
+        for idx in np.ndindex(arr.shape):
+            fd = _central(lambda: _loss(dU, X, Wq, Wk, Wv, Wo, alpha, L, B, **kw), arr, idx)
+            assert abs(got[name][idx] - fd) <= 1e-6 * (1 + abs(fd)), (name, idx, got[name][idx], fd)
+
+
+def test_backward_matches_central_differences_causal():
+    _check_backward_against_differences(True, False, 0.8, 1)
+
+
+def test_backward_matches_central_differences_full_attention_with_norm():
+    _check_backward_against_differences(False, True, -0.6, 2)
+
+
+def test_backward_matches_central_differences_causal_with_norm():
+    _check_backward_against_differences(True, True, 1.3, 3)
+
+
+def test_backward_at_alpha_zero_is_the_factorised_maps_gradient():
+    # alpha = 0: U = X (Wo Wq)^T, so dX = dU Wo Wq, dWo = dU^T Q, dWq = (dU Wo)^T X,
+    # and the attention weights receive nothing
+    X, Wq, Wk, Wv, Wo, L, B = _case(seed=4)
+    dU = np.random.default_rng(5).standard_normal((L * B, Wo.shape[0]))
+    got = oracle.attention_project_backward(dU, X, Wq, Wk, Wv, Wo, 0.0, L, B)
+    Q = X @ Wq.T
+    np.testing.assert_allclose(got["dX"], dU @ Wo @ Wq, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(got["dWo"], dU.T @ Q, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(got["dWq"], (dU @ Wo).T @ X, rtol=1e-12, atol=1e-12)
+    assert np.abs(got["dWk"]).max() == 0 and np.abs(got["dWv"]).max() == 0
