@@ -484,6 +484,22 @@ def _layer_producers(dev, flush, sru):
                         proj + att)
         ent["tokens_per_s"] = M / (t_a / 1e3)
         e["attention_causal" if causal else "attention_full"] = ent
+    # the producer's backward (causal, with the norm): the gradients of the four
+    # projections (two products each) and of the attention (dP, dV, dK, dQ: four
+    # products of the scores' size); the recomputation of the scores is not counted
+    bws = torch.empty(int(sru.load_library().sru_attention_backward_workspace_bytes(L, B, d, dp, N)),
+                      dtype=torch.uint8, device=dev)
+    gam, bet = torch.ones(dp, device=dev), torch.zeros(dp, device=dev)
+    dgam, dbet = torch.empty(dp, device=dev), torch.empty(dp, device=dev)
+    dWkv = torch.empty(2 * dp, dp, device=dev)
+    sru.sru_attention_project(X, Wq, Wkv, Wo, U, L, B, 0.5, ln_gamma=gam, ln_beta=bet, workspace=aws)
+    t_ab = _time_ms(lambda: sru.sru_attention_project_backward(dU, X, Wq, Wkv, Wo, L, B, 0.5, aws, dX, dWq, dWkv, dWo,
+                                                               ln_gamma=gam, ln_beta=bet, dgamma=dgam, dbeta=dbet,
+                                                               workspace=bws), flush)
+    ent = _tc_entry("sru_attention_project_backward (causal, layer norm)", t_ab,
+                    2.0 * proj + 4.0 * 2.0 * B * dp * (L * (L + 1) / 2.0))
+    ent["tokens_per_s"] = M / (t_ab / 1e3)
+    e["attention_backward_causal"] = ent
     return {"producers L1024 B16 d2048 d'512": e}
 
 

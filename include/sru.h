@@ -71,8 +71,8 @@ typedef enum { SRU_F32 = 0, SRU_BF16 = 1 } sru_dtype;
  * may use its chunked scan for any v: the state-gradient recurrence is affine.)
  * The library picks a scan when the sequential kernels would leave SMs idle
  * (fewer than two 64-channel CTAs per SM) and the scan's waves of resident
- * CTAs cost less than the sequence's 16-step chunks (a measured ratio of 12
- * chunks per wave on B200). */
+ * CTAs cost less than the sequence's 16-step chunks (measured on B200: a wave
+ * costs about 8 chunks forward, 5 backward). */
 #define SRU_FLAG_V_ZERO 0x1u
 /* Force the scan paths (the forward scan only with SRU_FLAG_V_ZERO) / force the
  * sequential paths. */
@@ -245,10 +245,18 @@ sru_status sru_project_factored(const void* X, const void* Wq, const void* Wo, v
  *   dWq = dP^T X (Kp, K) fp32;   dX = dP Wq (M, K) fp32, added onto dX when accumulate != 0.
  * P is the intermediate the forward wrote.  Any of dX, dWq, dWo may be NULL
  * (not computed); dP is always written.
+ * workspace / workspace_bytes (nullable; 16-byte aligned): with at least
+ * sru_project_factored_backward_workspace_bytes(M, N, K, Kp) bytes, a weight
+ * gradient whose output tiles cannot fill the GPU (dWq and dWo of a narrow d')
+ * is cut along its reduction over the M tokens, each part written to its own
+ * slab of the workspace and the slabs summed in a fixed order (the same bits
+ * every run); without one it runs as a single product.
  */
+size_t sru_project_factored_backward_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t Kp);
 sru_status sru_project_factored_backward(const void* dU, const void* X, const void* Wq, const void* Wo,
                                          const void* P, void* dP, float* dX, int accumulate, float* dWq,
-                                         float* dWo, int64_t M, int64_t N, int64_t K, int64_t Kp, void* stream);
+                                         float* dWo, int64_t M, int64_t N, int64_t K, int64_t Kp, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 
 /*
  * SRU++'s producer of U: single-head attention in place of the linear map of
@@ -273,6 +281,47 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
                                  const float* ln_gamma, const float* ln_beta, int causal, void* U, int u_t,
                                  int64_t L, int64_t B, int64_t d, int64_t dp, int64_t N, void* workspace,
                                  size_t workspace_bytes, void* stream);
+
+/*
+ * Backward of sru_attention_project for Loss = sum(dU * U) (the reverse-mode
+ * derivative of the SRU++ producer above; the page trains it end to end):
+ *   dWo = dU^T R,  dR = dU Wo
+ *   dZ from dR through the layer norm (or dZ = dR), Z = Q + alpha A;
+ *   dgamma = sum over tokens of dR * Zhat, dbeta = sum of dR (with the norm)
+ *   dQ = dZ;  dA = alpha dZ
+ *   per batch row: dP = dA V^T, dS = P * (dP - rowsum(P * dP)) / sqrt(d'),
+ *     dV = P^T dA, dK = dS^T Q, dQ += dS K
+ *   dQ += [dK | dV] Wkv;  dWkv = [dK | dV]^T Q
+ *   dWq = dQ^T X;  dX (+)= dQ Wq
+ *   dU (L*B, N) bf16; X, Wq, Wkv, Wo, alpha, ln_gamma, ln_beta, causal and
+ *   the sizes exactly as given to the forward call.
+ *   fwd_workspace: the workspace of that forward call, unchanged since (its Q,
+ *   [K | V], A and R are read; the probabilities are recomputed here one group
+ *   of batch rows at a time).
+ *   dX (L*B, d) fp32, written, or added onto when accumulate != 0 (so that the
+ *   highway part from sru_backward can be summed in place).
+ *   dWq (d', d), dWkv (2d', d'), dWo (N, d') fp32, written.
+ *   dgamma, dbeta (d',) fp32, written when ln_gamma / ln_beta are given (both
+ *   required then; ignored otherwise).  The sums over tokens are taken in a
+ *   fixed order: the same bits on every run.
+ *   workspace: >= sru_attention_backward_workspace_bytes(L, B, d, d', N) bytes,
+ *   16-byte aligned (dQ, dA, the per-group probabilities and their gradients,
+ *   [dK | dV], and the k slabs of the weight gradients: a weight gradient with
+ *   fewer output tiles than the GPU has CTA pairs is cut along its reduction over
+ *   the tokens, each part written to its own slab, and the slabs summed in a
+ *   fixed order).  0 for unsupported sizes.
+ * dA, dP's softmax gradient dS, [dK | dV] and dQ are rounded to bf16 where they
+ * become tensor-core operands.  Limits as for the forward.  Null or misaligned
+ * pointers and a short workspace: SRU_ERR_INVALID, before any launch.
+ */
+size_t sru_attention_backward_workspace_bytes(int64_t L, int64_t B, int64_t d, int64_t dp, int64_t N);
+sru_status sru_attention_project_backward(const void* dU, const void* X, const void* Wq, const void* Wkv,
+                                          const void* Wo, float alpha, const float* ln_gamma,
+                                          const float* ln_beta, int causal, const void* fwd_workspace,
+                                          size_t fwd_workspace_bytes, float* dX, int accumulate, float* dWq,
+                                          float* dWkv, float* dWo, float* dgamma, float* dbeta, int64_t L,
+                                          int64_t B, int64_t d, int64_t dp, int64_t N, void* workspace,
+                                          size_t workspace_bytes, void* stream);
 
 /*
  * One time step of a unidirectional layer for inference (token-by-token

@@ -33,8 +33,10 @@ SRU_FLAG_TEST_WITHHOLD_CARRY = 0x8
 EXPORTED = ("sru_status_string", "sru_get_last_cuda_error", "sru_version", "sru_workspace_bytes",
             "sru_project", "sru_project_backward", "sru_forward", "sru_backward", "sru_forward_scan_noalloc",
             "sru_forward_fused",
-            "sru_project_factored", "sru_project_factored_backward", "sru_attention_workspace_bytes",
-            "sru_attention_project", "sru_decode_workspace_bytes", "sru_decode_step", "sru_sync_status")
+            "sru_project_factored", "sru_project_factored_backward", "sru_project_factored_backward_workspace_bytes",
+            "sru_attention_workspace_bytes",
+            "sru_attention_project", "sru_attention_backward_workspace_bytes", "sru_attention_project_backward",
+            "sru_decode_workspace_bytes", "sru_decode_step", "sru_sync_status")
 
 
 class SRUError(RuntimeError):
@@ -89,12 +91,20 @@ def load_library(path: str = LIB_PATH):
     lib.sru_project_factored.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp]
     lib.sru_project_factored_backward.restype = _int
     lib.sru_project_factored_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _i64, _i64,
-                                                  _i64, _i64, _vp]
+                                                  _i64, _i64, _vp, ctypes.c_size_t, _vp]
+    lib.sru_project_factored_backward_workspace_bytes.restype = ctypes.c_size_t
+    lib.sru_project_factored_backward_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64]
     lib.sru_attention_workspace_bytes.restype = ctypes.c_size_t
     lib.sru_attention_workspace_bytes.argtypes = [_i64, _i64, _i64]
     lib.sru_attention_project.restype = _int
     lib.sru_attention_project.argtypes = [_vp, _vp, _vp, _vp, _f32, _vp, _vp, _int, _vp, _int, _i64, _i64, _i64,
                                           _i64, _i64, _vp, ctypes.c_size_t, _vp]
+    lib.sru_attention_backward_workspace_bytes.restype = ctypes.c_size_t
+    lib.sru_attention_backward_workspace_bytes.argtypes = [_i64, _i64, _i64, _i64, _i64]
+    lib.sru_attention_project_backward.restype = _int
+    lib.sru_attention_project_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _int, _vp, ctypes.c_size_t,
+                                                   _vp, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64,
+                                                   _vp, ctypes.c_size_t, _vp]
     lib.sru_decode_step.restype = _int
     lib.sru_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _vp, ctypes.c_size_t, _vp]
     lib.sru_decode_workspace_bytes.restype = ctypes.c_size_t
@@ -255,16 +265,24 @@ def sru_project_factored(X, Wq, Wo, P, U, stream=None):
 
 
 def sru_project_factored_backward(dU, X, Wq, Wo, P, dP, dX=None, accumulate: bool = False, dWq=None, dWo=None,
-                                  stream=None):
-    """dWo = dU^T P, dP = dU Wo (bf16, into dP), dWq = dP^T X, dX (+)= dP Wq (fp32 outputs)."""
+                                  workspace=None, stream=None):
+    """dWo = dU^T P, dP = dU Wo (bf16, into dP), dWq = dP^T X, dX (+)= dP Wq (fp32 outputs).
+    A workspace of sru_project_factored_backward_workspace_bytes bytes (the
+    split weight gradients' slabs) is allocated when none is given; an empty
+    tensor runs without one."""
     lib = load_library()
     M, K = X.shape
     Kp, N = Wq.shape[0], Wo.shape[0]
+    if workspace is None:
+        n = int(lib.sru_project_factored_backward_workspace_bytes(M, N, K, Kp))
+        workspace = torch.empty(n, dtype=torch.uint8, device=dU.device)
+    ws_ptr = _ptr(workspace) if workspace.numel() > 0 else None
     _check(lib.sru_project_factored_backward(_ptr(dU, torch.bfloat16), _ptr(X, torch.bfloat16),
                                              _ptr(Wq, torch.bfloat16), _ptr(Wo, torch.bfloat16),
                                              _ptr(P, torch.bfloat16), _ptr(dP, torch.bfloat16),
                                              _ptr(dX, torch.float32), int(bool(accumulate)),
                                              _ptr(dWq, torch.float32), _ptr(dWo, torch.float32), M, N, K, Kp,
+                                             ws_ptr, _nbytes(workspace) if ws_ptr is not None else 0,
                                              _stream(stream)), "sru_project_factored_backward")
     return dX, dWq, dWo
 
@@ -291,6 +309,39 @@ def sru_attention_project(X, Wq, Wkv, Wo, U, L: int, B: int, alpha: float, ln_ga
                                      L, B, d, dp, N, _ptr(workspace), _nbytes(workspace), _stream(stream)),
            "sru_attention_project")
     return U
+
+
+def sru_attention_project_backward(dU, X, Wq, Wkv, Wo, L: int, B: int, alpha: float, fwd_workspace, dX, dWq, dWkv,
+                                   dWo, accumulate: bool = False, ln_gamma=None, ln_beta=None, dgamma=None,
+                                   dbeta=None, causal: bool = True, workspace=None, stream=None):
+    """Backward of sru_attention_project (see sru.h).  dU (L*B, N) bf16; X, Wq,
+    Wkv, Wo, alpha, ln_gamma, ln_beta and causal as given to the forward, whose
+    workspace (unchanged since) is fwd_workspace.  Writes dX (L*B, d) fp32 (or
+    adds onto it with accumulate), dWq (d', d), dWkv (2d', d'), dWo (N, d') and,
+    with the norm, dgamma, dbeta (d',), all fp32.  A workspace of
+    sru_attention_backward_workspace_bytes bytes is allocated when none is given."""
+    lib = load_library()
+    M, d = X.shape
+    dp, N = Wq.shape[0], Wo.shape[0]
+    if M != L * B or tuple(dU.shape) != (M, N) or Wq.shape[1] != d or tuple(Wkv.shape) != (2 * dp, dp) \
+            or Wo.shape[1] != dp:
+        raise ValueError("shape mismatch")
+    if tuple(dX.shape) != (M, d) or tuple(dWq.shape) != (dp, d) or tuple(dWkv.shape) != (2 * dp, dp) \
+            or tuple(dWo.shape) != (N, dp):
+        raise ValueError("gradient shape mismatch")
+    if workspace is None:
+        n = int(lib.sru_attention_backward_workspace_bytes(L, B, d, dp, N))
+        if n == 0:
+            raise SRUError(SRU_ERR_UNSUPPORTED, "sru_attention_backward_workspace_bytes", lib)
+        workspace = torch.empty(n, dtype=torch.uint8, device=X.device)
+    _check(lib.sru_attention_project_backward(
+        _ptr(dU, torch.bfloat16), _ptr(X, torch.bfloat16), _ptr(Wq, torch.bfloat16), _ptr(Wkv, torch.bfloat16),
+        _ptr(Wo, torch.bfloat16), float(alpha), _ptr(ln_gamma, torch.float32), _ptr(ln_beta, torch.float32),
+        int(bool(causal)), _ptr(fwd_workspace), _nbytes(fwd_workspace), _ptr(dX, torch.float32),
+        int(bool(accumulate)), _ptr(dWq, torch.float32), _ptr(dWkv, torch.float32), _ptr(dWo, torch.float32),
+        _ptr(dgamma, torch.float32), _ptr(dbeta, torch.float32), L, B, d, dp, N, _ptr(workspace),
+        _nbytes(workspace), _stream(stream)), "sru_attention_project_backward")
+    return dX, dWq, dWkv, dWo
 
 
 def sru_decode_step(X_t, W, x_t, v, b, c, h_t, alpha: float = 1.0, workspace=None, stream=None):

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -175,14 +176,16 @@ sru::ScanState scan_state(void* workspace, const WsLayout& w, unsigned flags) {
 // one after another); the chunked scans cut time into kScanT-step work items
 // at the price of a second pass over each item and a look-back.  Measured on
 // B200 over layers from L256 B32 d512 to L8192 B4 d512: one wave of resident
-// scan CTAs costs about as much as kScanWaveChunks sequential 16-step chunks
-// (forward 20 us vs 1.5 us, backward 27 us vs 2.45 us per chunk), so a scan is
-// taken when its waves cost fewer chunks than the sequence has.  Only grids
-// that leave SMs idle (fewer than two sequential CTAs per SM) are candidates.
-// The forward scan needs SRU_FLAG_V_ZERO (linear state recurrence); the
-// backward scan is exact for any v (the state-gradient recurrence is affine).
-// The FORCE flags override.
-constexpr int64_t kScanWaveChunks = 12;
+// forward-scan CTAs costs about as much as kScanWaveChunksFwd sequential
+// 16-step chunks (about 12 us against 1.5-2 us per chunk), one wave of
+// backward-scan CTAs about kScanWaveChunksBwd (about 12-15 us against 2.3-3
+// us), so a scan is taken when its waves cost fewer chunks than the sequence
+// has.  Only grids that leave SMs idle (fewer than two sequential CTAs per SM)
+// are candidates.  The forward scan needs SRU_FLAG_V_ZERO (linear state
+// recurrence); the backward scan is exact for any v (the state-gradient
+// recurrence is affine).  The FORCE flags override.
+constexpr int64_t kScanWaveChunksFwd = 8;
+constexpr int64_t kScanWaveChunksBwd = 5;
 
 int64_t seq_ctas(int64_t B, int64_t d, int n_dir_per_launch) {
     return ((d + sru::kRecCJ - 1) / sru::kRecCJ) * B * n_dir_per_launch;
@@ -190,8 +193,9 @@ int64_t seq_ctas(int64_t B, int64_t d, int n_dir_per_launch) {
 bool scan_candidate(int64_t B, int64_t d, int n_dir_per_launch) {
     return seq_ctas(B, d, n_dir_per_launch) < 2 * (int64_t)sm_count();
 }
-// Scan CTAs (one warp, `smem` bytes) resident per SM: shared memory bounds it
-// (1 KB per CTA is reserved by the system), and 255-register warps at 8.
+// Scan CTAs (kScanThreads threads, `smem` bytes) resident per SM without a
+// device to ask: shared memory bounds it (1 KB per CTA is reserved by the
+// system).
 int smem_resident(size_t smem) {
     static int cap[kMaxDevices] = {0};
     int dev = 0;
@@ -208,31 +212,58 @@ int smem_resident(size_t smem) {
     const int n = (int)(bytes / (smem + 1024));
     return n < 1 ? 1 : (n > 8 ? 8 : n);
 }
-bool scan_pays(int64_t L, int64_t ctas, size_t scan_smem) {
-    const int64_t per_wave = (int64_t)sm_count() * smem_resident(scan_smem);
+// A scan kernel's CTAs resident per SM (registers and shared memory), from the
+// occupancy calculator; the shared-memory bound when it cannot answer.
+int scan_resident(const void* kern, size_t smem) {
+    if (no_device || ensure_smem(kern, smem) != cudaSuccess) return smem_resident(smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, sru::kScanThreads, smem) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        return smem_resident(smem);
+    }
+    return n;
+}
+bool scan_pays(int64_t L, int64_t ctas, int per_sm, int64_t wave_chunks) {
+    const int64_t per_wave = (int64_t)sm_count() * per_sm;
     const int64_t items = ((L + sru::kScanT - 1) / sru::kScanT) * ctas;
     const int64_t waves = (items + per_wave - 1) / per_wave;
-    return waves * kScanWaveChunks < (L + sru::kChunkT - 1) / sru::kChunkT;
+    return waves * wave_chunks < (L + sru::kChunkT - 1) / sru::kChunkT;
 }
-size_t fwd_scan_smem(int u_t) {
-    return u_t == SRU_BF16 ? sru::FwdScanLayout<__nv_bfloat16>::SMEM : sru::FwdScanLayout<float>::SMEM;
-}
-size_t bwd_scan_smem(int u_t, bool acc_dx) {
+int fwd_scan_resident(int u_t) {
     if (u_t == SRU_BF16)
-        return acc_dx ? sru::BwdScanLayout<__nv_bfloat16, true>::SMEM : sru::BwdScanLayout<__nv_bfloat16, false>::SMEM;
-    return acc_dx ? sru::BwdScanLayout<float, true>::SMEM : sru::BwdScanLayout<float, false>::SMEM;
+        return scan_resident(reinterpret_cast<const void*>(sru::sru_fwd_scan_kernel<__nv_bfloat16>),
+                             sru::FwdScanLayout<__nv_bfloat16>::SMEM);
+    return scan_resident(reinterpret_cast<const void*>(sru::sru_fwd_scan_kernel<float>),
+                         sru::FwdScanLayout<float>::SMEM);
+}
+// (the first direction's kernel with a U-typed dU stands for every variant)
+int bwd_scan_resident(int u_t, bool v_zero) {
+    if (u_t == SRU_BF16)
+        return v_zero ? scan_resident(reinterpret_cast<const void*>(
+                                          sru::sru_bwd_scan_kernel<__nv_bfloat16, __nv_bfloat16, false, 0, true>),
+                                      sru::BwdScanLayout<__nv_bfloat16, false>::SMEM)
+                      : scan_resident(reinterpret_cast<const void*>(
+                                          sru::sru_bwd_scan_kernel<__nv_bfloat16, __nv_bfloat16, false, 0, false>),
+                                      sru::BwdScanLayout<__nv_bfloat16, false>::SMEM);
+    return v_zero ? scan_resident(reinterpret_cast<const void*>(sru::sru_bwd_scan_kernel<float, float, false, 0, true>),
+                                  sru::BwdScanLayout<float, false>::SMEM)
+                  : scan_resident(reinterpret_cast<const void*>(sru::sru_bwd_scan_kernel<float, float, false, 0, false>),
+                                  sru::BwdScanLayout<float, false>::SMEM);
 }
 bool use_fwd_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir, int u_t) {
     if (!(flags & SRU_FLAG_V_ZERO)) return false;
     if (flags & SRU_FLAG_FORCE_SCAN) return true;
     if (flags & SRU_FLAG_FORCE_SEQUENTIAL) return false;
-    return scan_candidate(B, d, n_dir) && scan_pays(L, seq_ctas(B, d, n_dir), fwd_scan_smem(u_t));
+    return scan_candidate(B, d, n_dir) &&
+           scan_pays(L, seq_ctas(B, d, n_dir), fwd_scan_resident(u_t), kScanWaveChunksFwd);
 }
 bool use_bwd_scan(unsigned flags, int64_t L, int64_t B, int64_t d, int n_dir, int u_t) {
     if (flags & SRU_FLAG_FORCE_SCAN) return true;
     if (flags & SRU_FLAG_FORCE_SEQUENTIAL) return false;
     // one direction per backward launch
-    return scan_candidate(B, d, 1) && scan_pays(L, seq_ctas(B, d, 1), bwd_scan_smem(u_t, n_dir == 2));
+    return scan_candidate(B, d, 1) &&
+           scan_pays(L, seq_ctas(B, d, 1), bwd_scan_resident(u_t, (flags & SRU_FLAG_V_ZERO) != 0),
+                     kScanWaveChunksBwd);
 }
 // Whether a workspace for these sizes and flags carries the scan regions: a
 // superset of the layers that take a scan (it depends on sizes and flags only,
@@ -270,15 +301,16 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
     {
         auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT>;
         SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
-        // the output as the epilogue's TMA store target: box 32 x 32, swizzled like the staging buffers
+        // the output as the epilogue's TMA store target: boxes of 32 rows x 128 bytes
+        // (64 bf16 or 32 fp32 columns), swizzled like the staging buffers
         CUtensorMap mo;
         {
             const bool bf = OUT == sru::gemm::kOutBF16;
             const uint64_t dims[2] = {(uint64_t)C, (uint64_t)R};
             const uint64_t strides[1] = {(uint64_t)ldo * (bf ? 2 : 4)};
-            const uint32_t box[2] = {32, 32};
+            const uint32_t box[2] = {(uint32_t)sru::gemm::EpiChunk<OUT>::kCols, 32};
             if (!make_map(&mo, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, dims,
-                          strides, box, bf ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
+                          strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
                 return SRU_ERR_INVALID;
         }
         const int64_t n_tiles = (C + sru::gemm::P_BN - 1) / sru::gemm::P_BN;
@@ -297,7 +329,7 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
             SRU_CUDA_TRY(cudaGetLastError());
         }
         kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
-            ma, mb, mo, out, (int)R, (int)C, (int)Kr, (int)ldo, splits, 1, 0LL, tail_s);
+            ma, mb, mo, out, (int)R, (int)C, (int)Kr, (int)ldo, splits, 1, 0LL, tail_s, 0);
     }
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
@@ -322,7 +354,7 @@ sru_status launch_tc_gemm_batched(const CUtensorMap& ma, const CUtensorMap& mb, 
     CUtensorMap unused;  // batched launches store directly (no output map)
     std::memset(&unused, 0, sizeof(unused));
     kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
-        ma, mb, unused, out, (int)R, (int)C, (int)Kr, (int)ldo, 1, (int)batches, (long long)out_bstride, 0);
+        ma, mb, unused, out, (int)R, (int)C, (int)Kr, (int)ldo, 1, (int)batches, (long long)out_bstride, 0, 0);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
@@ -597,8 +629,8 @@ sru_status launch_fwd_scan(const RecMaps& mp, const float* b, const float* c0, c
     if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
     sru_status s = reset_scan_flags(ss.flags, items + 1, st);
     if (s != SRU_OK) return s;
-    kern<<<(unsigned)items, sru::kRecThreads, Lay::SMEM, st>>>(mp.u, mp.x, b, c0, mask, h, c_T, ckpt, ss, (int)L, (int)B,
-                                                          (int)d, n_dir, alpha);
+    kern<<<(unsigned)items, sru::kScanThreads, Lay::SMEM, st>>>(mp.u, mp.x, b, c0, mask, h, c_T, ckpt, ss, (int)L,
+                                                           (int)B, (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
@@ -616,8 +648,8 @@ sru_status launch_bwd_scan_dir(const RecMaps& mp, const float* v, const float* b
     if (items >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
     sru_status s = reset_scan_flags(ss.flags, items + 1, st);
     if (s != SRU_OK) return s;
-    kern<<<(unsigned)items, sru::kRecThreads, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, v, b, mask, ckpt, dc_T, dU, dx,
-                                                          partial, dc0, ss, (int)L, (int)B, (int)d, n_dir, alpha);
+    kern<<<(unsigned)items, sru::kScanThreads, Lay::SMEM, st>>>(mp.u, mp.x, mp.dh, v, b, mask, ckpt, dc_T, dU, dx,
+                                                           partial, dc0, ss, (int)L, (int)B, (int)d, n_dir, alpha);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
@@ -1086,6 +1118,79 @@ sru_status sru_forward_fused(const void* X, const void* W, const float* x, const
     return SRU_OK;
 }
 
+// Split-K for fp32 products with fewer output tiles than CTA pairs and a long
+// reduction (the weight gradients dW = dU^T X of narrow layers): k part s of
+// every tile is written to slab s of a scratch buffer (rows s * R_pad ..,
+// R_pad = R rounded up to whole tiles), then splitk_reduce_kernel sums the
+// slabs in order into the output, so the result is the same bits every run.
+// S comes from a time model measured on B200: a round of units costs
+// kper k-blocks at 0.35 us each plus 2 us of fill and epilogue, and the slabs
+// cost their bytes twice (written, then read by the sum) at 5 TB/s plus 3 us
+// for the sum's launch; S = 1 means no split pays.
+struct SplitPlan {
+    int64_t splits, slab_rows;
+    size_t bytes;
+};
+static SplitPlan split_plan(int64_t R, int64_t C, int64_t Kr) {
+    constexpr double kKblockUs = 0.35, kUnitUs = 2.0, kSlabBytesPerUs = 5.0e6, kSumUs = 3.0;
+    const int64_t P = sm_count() / 2;
+    const int64_t tiles = ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((C + sru::gemm::P_BN - 1) / sru::gemm::P_BN);
+    const int64_t kblocks = (Kr + sru::gemm::BK - 1) / sru::gemm::BK;
+    SplitPlan pl{1, ((R + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * sru::gemm::P_BM, 0};
+    auto model_us = [&](int64_t S) {
+        const int64_t kper = (kblocks + S - 1) / S;
+        const double slabs = S > 1 ? (double)S * pl.slab_rows * C * 4 * 2 / kSlabBytesPerUs + kSumUs : 0.0;
+        return (double)((tiles * S + P - 1) / P) * (kper * kKblockUs + kUnitUs) + slabs;
+    };
+    double best = model_us(1);
+    for (int64_t S0 = 2; S0 <= 32 && S0 * 4 <= kblocks; ++S0) {
+        // the kernel gives part s the k-blocks [s kper, (s + 1) kper) with kper =
+        // ceil(kblocks / S): take S so that no part is empty (an empty part would
+        // store an accumulator no MMA wrote)
+        const int64_t S = (kblocks + (kblocks + S0 - 1) / S0 - 1) / ((kblocks + S0 - 1) / S0);
+        const double t = model_us(S);
+        if (t < best) {
+            best = t;
+            pl.splits = S;
+        }
+    }
+    pl.bytes = pl.splits > 1 ? (size_t)pl.splits * pl.slab_rows * C * 4 : 0;
+    return pl;
+}
+// dW[N, K] = dU[M, N]^T X[M, K] (bf16 operands, fp32 output) with the split
+// plan above when `scratch` holds its slabs, else as sru_project_backward does.
+static sru_status project_dW_split(const void* dU, const void* X, float* dW, int64_t M, int64_t N, int64_t K, void* scratch,
+                            size_t scratch_bytes, cudaStream_t st) {
+    if (M == 0) return zero_f32(dW, (size_t)N * K, st);
+    CUtensorMap ma, mb;
+    if (!map_mnmajor(&ma, dU, N, M, N) || !map_mnmajor(&mb, X, K, M, K)) return SRU_ERR_INVALID;
+    const SplitPlan pl = split_plan(N, K, M);
+    if (pl.splits <= 1 || scratch == nullptr || scratch_bytes < pl.bytes)
+        return launch_tc_gemm<true, true, sru::gemm::kOutF32>(ma, mb, dW, N, K, M, st, 1, -1, /*tail_split=*/true);
+    auto kern = sru::gemm::tc_gemm_pair_kernel<true, true, sru::gemm::kOutF32>;
+    SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
+    CUtensorMap mo;
+    {
+        const uint64_t dims[2] = {(uint64_t)K, (uint64_t)(pl.slab_rows * pl.splits)};
+        const uint64_t strides[1] = {(uint64_t)K * 4};
+        const uint32_t box[2] = {(uint32_t)sru::gemm::EpiChunk<sru::gemm::kOutF32>::kCols, 32};
+        if (!make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, scratch, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return SRU_ERR_INVALID;
+    }
+    const int64_t tiles = ((N + sru::gemm::P_BM - 1) / sru::gemm::P_BM) * ((K + sru::gemm::P_BN - 1) / sru::gemm::P_BN);
+    const int64_t units = tiles * pl.splits;
+    const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
+    kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
+        ma, mb, mo, scratch, (int)N, (int)K, (int)M, (int)K, (int)pl.splits, 1, 0LL, 0, (int)pl.slab_rows);
+    SRU_CUDA_TRY(cudaGetLastError());
+    const size_t n4 = (size_t)N * K / 4;
+    sru::gemm::splitk_reduce_kernel<<<(unsigned)std::min<size_t>(blocks_for(n4, 256), (size_t)sm_count() * 8), 256, 0,
+                                      st>>>(reinterpret_cast<const float4*>(scratch), reinterpret_cast<float4*>(dW),
+                                            (int)N, (int)(K / 4), (int)pl.slab_rows, (int)pl.splits);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
 sru_status sru_project_factored(const void* X, const void* Wq, const void* Wo, void* P, void* U, int u_t,
                                 int64_t M, int64_t N, int64_t K, int64_t Kp, void* stream) {
     if (M < 0 || N < 0 || K < 1 || Kp < 1) return SRU_ERR_INVALID;
@@ -1098,11 +1203,20 @@ sru_status sru_project_factored(const void* X, const void* Wq, const void* Wo, v
     return sru_project(P, SRU_BF16, Wo, SRU_BF16, U, u_t, M, N, Kp, stream);
 }
 
+size_t sru_project_factored_backward_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t Kp) {
+    if (M < 1 || N < 8 || K < 8 || Kp < 8 || N % 8 != 0 || K % 8 != 0 || Kp % 8 != 0) return 0;
+    if (M >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31) || Kp >= ((int64_t)1 << 31))
+        return 0;
+    return round256(std::max(split_plan(N, Kp, M).bytes, split_plan(Kp, K, M).bytes));
+}
+
 sru_status sru_project_factored_backward(const void* dU, const void* X, const void* Wq, const void* Wo,
                                          const void* P, void* dP, float* dX, int accumulate, float* dWq,
-                                         float* dWo, int64_t M, int64_t N, int64_t K, int64_t Kp, void* stream) {
+                                         float* dWo, int64_t M, int64_t N, int64_t K, int64_t Kp, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
     if (M < 0 || N < 1 || K < 1 || Kp < 1) return SRU_ERR_INVALID;
     if (!dU || !Wo || !dP || !aligned16(dU) || !aligned16(Wo) || !aligned16(dP)) return SRU_ERR_INVALID;
+    if (workspace != nullptr && !aligned16(workspace)) return SRU_ERR_INVALID;
     if (dWo && (!P || !aligned16(P) || !aligned16(dWo))) return SRU_ERR_INVALID;
     if (dWq && (!X || !aligned16(X) || !aligned16(dWq))) return SRU_ERR_INVALID;
     if (dX && (!Wq || !aligned16(Wq) || !aligned16(dX))) return SRU_ERR_INVALID;
@@ -1116,10 +1230,10 @@ sru_status sru_project_factored_backward(const void* dU, const void* X, const vo
         return SRU_OK;
     }
     CUtensorMap ma, mb;
-    // dWo = dU^T P: A(r = n, red = m) = dU[m][n] MN-major; B(c = kp, red = m) = P[m][kp] MN-major
+    // dWo = dU^T P (split along the tokens when its tiles cannot fill the GPU and
+    // the workspace holds the slabs)
     if (dWo) {
-        if (!map_mnmajor(&ma, dU, N, M, N) || !map_mnmajor(&mb, P, Kp, M, Kp)) return SRU_ERR_INVALID;
-        sru_status s = launch_tc_gemm<true, true, sru::gemm::kOutF32>(ma, mb, dWo, N, Kp, M, st);
+        sru_status s = project_dW_split(dU, P, dWo, M, N, Kp, workspace, workspace_bytes, st);
         if (s != SRU_OK) return s;
     }
     // dP = dU Wo (bf16): A = dU K-major over n; B(c = kp, red = n) = Wo[n][kp] MN-major
@@ -1129,7 +1243,9 @@ sru_status sru_project_factored_backward(const void* dU, const void* X, const vo
         if (s != SRU_OK) return s;
     }
     // dWq = dP^T X and dX (+)= dP Wq: the gradients of the first product
-    return sru_project_backward(dP, X, Wq, SRU_BF16, dX, accumulate, dWq, M, Kp, K, stream);
+    sru_status s = sru_project_backward(dP, X, Wq, SRU_BF16, dX, accumulate, nullptr, M, Kp, K, stream);
+    if (s != SRU_OK || !dWq) return s;
+    return project_dW_split(dP, X, dWq, M, Kp, K, workspace, workspace_bytes, st);
 }
 
 // ---- SRU++ attention producer
@@ -1219,6 +1335,176 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
         Q, A, alpha, ln_gamma, ln_beta, R, (int)M, (int)dp);
     SRU_CUDA_TRY(cudaGetLastError());
     return sru_project(R, SRU_BF16, Wo, SRU_BF16, U, u_t, M, N, dp, stream);
+}
+
+// ------------------------------------------------- attention producer backward
+// Batch rows per group of the backward: scores / their gradient (fp32), P and
+// dS (bf16) of one group stay under the same budget as the forward's.
+static int64_t attn_bwd_group(int64_t L, int64_t B) {
+    const int64_t g = (int64_t)(kAttnGroupBytes / ((size_t)L * L * 8));
+    return g < 1 ? 1 : (g > B ? B : g);
+}
+constexpr int kNormSlices = 128;  // row slices of the norm's parameter-gradient sums
+struct AttnBwdWs {
+    size_t dr, dq, da, dkv, dqb, s, p, ds, stats, part, split, split_bytes, total;
+};
+static AttnBwdWs attn_bwd_ws(int64_t L, int64_t B, int64_t d, int64_t dp, int64_t N) {
+    AttnBwdWs w{};
+    const int64_t M = L * B, G = attn_bwd_group(L, B);
+    // slabs of the split-K weight gradients dWo (N x d'), dWkv (2d' x d'), dWq (d' x d)
+    w.split_bytes = std::max(split_plan(N, dp, M).bytes, std::max(split_plan(2 * dp, dp, M).bytes,
+                                                                  split_plan(dp, d, M).bytes));
+    size_t off = 0;
+    w.dr = off;    off += round256((size_t)M * dp * 4);
+    w.dq = off;    off += round256((size_t)M * dp * 4);
+    w.da = off;    off += round256((size_t)M * dp * 2);
+    w.dkv = off;   off += round256((size_t)M * 2 * dp * 2);
+    w.dqb = off;   off += round256((size_t)M * dp * 2);
+    w.s = off;     off += round256((size_t)G * L * L * 4);
+    w.p = off;     off += round256((size_t)G * L * L * 2);
+    w.ds = off;    off += round256((size_t)G * L * L * 2);
+    w.stats = off; off += round256((size_t)M * 8);
+    w.part = off;  off += round256((size_t)kNormSlices * 2 * dp * 4);
+    w.split = off; off += round256(w.split_bytes);
+    w.total = off;
+    return w;
+}
+
+size_t sru_attention_backward_workspace_bytes(int64_t L, int64_t B, int64_t d, int64_t dp, int64_t N) {
+    if (L < 1 || B < 1 || d < 8 || dp < 8 || N < 8 || d % 8 != 0 || dp % 8 != 0 || N % 8 != 0 || L % 8 != 0)
+        return 0;
+    if (L * B >= ((int64_t)1 << 31) || L > 65536) return 0;
+    return attn_bwd_ws(L, B, d, dp, N).total;
+}
+
+sru_status sru_attention_project_backward(const void* dU, const void* X, const void* Wq, const void* Wkv,
+                                          const void* Wo, float alpha, const float* ln_gamma,
+                                          const float* ln_beta, int causal, const void* fwd_workspace,
+                                          size_t fwd_workspace_bytes, float* dX, int accumulate, float* dWq,
+                                          float* dWkv, float* dWo, float* dgamma, float* dbeta, int64_t L,
+                                          int64_t B, int64_t d, int64_t dp, int64_t N, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+    if (L < 1 || B < 1 || d < 1 || dp < 1 || N < 1) return SRU_ERR_INVALID;
+    if (!dU || !X || !Wq || !Wkv || !Wo || !fwd_workspace || !dX || !dWq || !dWkv || !dWo || !workspace)
+        return SRU_ERR_INVALID;
+    if (!aligned16(dU) || !aligned16(X) || !aligned16(Wq) || !aligned16(Wkv) || !aligned16(Wo) ||
+        !aligned16(fwd_workspace) || !aligned16(dX) || !aligned16(dWq) || !aligned16(dWkv) || !aligned16(dWo) ||
+        !aligned16(workspace))
+        return SRU_ERR_INVALID;
+    if ((ln_gamma == nullptr) != (ln_beta == nullptr)) return SRU_ERR_INVALID;
+    const bool norm = ln_gamma != nullptr;
+    if (norm && (!dgamma || !dbeta)) return SRU_ERR_INVALID;
+    if (d % 8 != 0 || dp % 8 != 0 || N % 8 != 0 || L % 8 != 0) return SRU_ERR_UNSUPPORTED;
+    const int64_t M = L * B;
+    if (M >= ((int64_t)1 << 31) || L > 65536) return SRU_ERR_UNSUPPORTED;
+    const AttnWs fw = attn_ws(L, B, dp);
+    const AttnBwdWs w = attn_bwd_ws(L, B, d, dp, N);
+    if (fwd_workspace_bytes < fw.total || workspace_bytes < w.total) return SRU_ERR_INVALID;
+    cudaStream_t st = as_stream(stream);
+    const uint8_t* fws = static_cast<const uint8_t*>(fwd_workspace);
+    const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(fws + fw.q);
+    const __nv_bfloat16* KV = reinterpret_cast<const __nv_bfloat16*>(fws + fw.kv);
+    const float* A = reinterpret_cast<const float*>(fws + fw.a);
+    const __nv_bfloat16* R = reinterpret_cast<const __nv_bfloat16*>(fws + fw.r);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* dR = reinterpret_cast<float*>(ws + w.dr);
+    float* dQ = reinterpret_cast<float*>(ws + w.dq);
+    __nv_bfloat16* dA = reinterpret_cast<__nv_bfloat16*>(ws + w.da);
+    __nv_bfloat16* dKV = reinterpret_cast<__nv_bfloat16*>(ws + w.dkv);
+    __nv_bfloat16* dQb = reinterpret_cast<__nv_bfloat16*>(ws + w.dqb);
+    float* S = reinterpret_cast<float*>(ws + w.s);
+    __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(ws + w.p);
+    __nv_bfloat16* dS = reinterpret_cast<__nv_bfloat16*>(ws + w.ds);
+    float2* stats = reinterpret_cast<float2*>(ws + w.stats);
+    float* part = reinterpret_cast<float*>(ws + w.part);
+    void* split = ws + w.split;
+
+    // U = R Wo^T:  dR = dU Wo,  dWo = dU^T R
+    sru_status s = sru_project_backward(dU, R, Wo, SRU_BF16, dR, 0, nullptr, M, N, dp, stream);
+    if (s != SRU_OK) return s;
+    s = project_dW_split(dU, R, dWo, M, N, dp, split, w.split_bytes, st);
+    if (s != SRU_OK) return s;
+    // through the norm (or the identity): dQ = dZ, dA = alpha dZ
+    sru::sru_norm_backward_kernel<<<blocks_for((size_t)M, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+        dR, Q, A, alpha, ln_gamma, dQ, dA, stats, (int)M, (int)dp);
+    SRU_CUDA_TRY(cudaGetLastError());
+    if (norm) {
+        const int rows_per = (int)((M + kNormSlices - 1) / kNormSlices);
+        const dim3 grid(blocks_for((size_t)dp, sru::kNormParamThreads), (unsigned)((M + rows_per - 1) / rows_per));
+        sru::sru_norm_param_partial_kernel<<<grid, sru::kNormParamThreads, 0, st>>>(dR, Q, A, alpha, stats, part,
+                                                                                   (int)M, (int)dp, rows_per);
+        SRU_CUDA_TRY(cudaGetLastError());
+        sru::sru_norm_param_reduce_kernel<<<blocks_for((size_t)dp, 256), 256, 0, st>>>(part, (int)grid.y, (int)dp,
+                                                                                       dgamma, dbeta);
+        SRU_CUDA_TRY(cudaGetLastError());
+    }
+    const float scale = 1.0f / sqrtf((float)dp);
+    const int64_t G = attn_bwd_group(L, B);
+    // batch row b's tokens are rows t*B + b of the time-major Q, K, V, dA, dQ and [dK | dV]
+    for (int64_t b0 = 0; b0 < B; b0 += G) {
+        const int64_t g = B - b0 < G ? B - b0 : G;
+        CUtensorMap ma, mb;
+        // the forward's probabilities of this group: S = Q K^T, softmax
+        if (!map_kmajor_b(&ma, Q + b0 * dp, L, dp, B * dp, g, dp, sru::gemm::P_CM, 1) ||
+            !map_kmajor_b(&mb, KV + b0 * 2 * dp, L, dp, B * 2 * dp, g, 2 * dp, kGemmBRows, 1))
+            return SRU_ERR_INVALID;
+        s = causal ? launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st)
+                   : launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st);
+        if (s != SRU_OK) return s;
+        sru::sru_softmax_rows_kernel<<<blocks_for((size_t)(g * L), sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+            S, P, (int)L, (int)(g * L), scale, causal ? 1 : 0);
+        SRU_CUDA_TRY(cudaGetLastError());
+        // dP = dA V^T (into S), then dS
+        if (!map_kmajor_b(&ma, dA + b0 * dp, L, dp, B * dp, g, dp, sru::gemm::P_CM, 1) ||
+            !map_kmajor_b(&mb, KV + b0 * 2 * dp + dp, L, dp, B * 2 * dp, g, 2 * dp, kGemmBRows, 1))
+            return SRU_ERR_INVALID;
+        s = causal ? launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st)
+                   : launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st);
+        if (s != SRU_OK) return s;
+        sru::sru_softmax_backward_rows_kernel<<<blocks_for((size_t)(g * L), sru::kRowWarps), sru::kRowWarps * 32, 0,
+                                                st>>>(S, P, dS, (int)L, (int)(g * L), scale, causal ? 1 : 0);
+        SRU_CUDA_TRY(cudaGetLastError());
+        // dV = P^T dA and dK = dS^T Q (bf16, into [dK | dV]): the first operand read
+        // MN-major (element (s, t) of batch z at z L^2 + t L + s), the second too
+        // (element (j, t) at (t B + b0 + z) d' + j)
+        __nv_bfloat16* dK0 = dKV + b0 * 2 * dp;
+        if (!map_mnmajor_b(&ma, P, L, L, L, g, L * L, 2) || !map_mnmajor_b(&mb, dA + b0 * dp, dp, L, B * dp, g, dp, 1))
+            return SRU_ERR_INVALID;
+        s = causal ? launch_tc_gemm_batched<true, true, sru::gemm::kOutBF16, 2, 1, 3>(ma, mb, dK0 + dp, L, dp, L,
+                                                                                     B * 2 * dp, g, 2 * dp, st)
+                   : launch_tc_gemm_batched<true, true, sru::gemm::kOutBF16, 2, 1>(ma, mb, dK0 + dp, L, dp, L,
+                                                                                  B * 2 * dp, g, 2 * dp, st);
+        if (s != SRU_OK) return s;
+        if (!map_mnmajor_b(&ma, dS, L, L, L, g, L * L, 2) || !map_mnmajor_b(&mb, Q + b0 * dp, dp, L, B * dp, g, dp, 1))
+            return SRU_ERR_INVALID;
+        s = causal ? launch_tc_gemm_batched<true, true, sru::gemm::kOutBF16, 2, 1, 3>(ma, mb, dK0, L, dp, L,
+                                                                                     B * 2 * dp, g, 2 * dp, st)
+                   : launch_tc_gemm_batched<true, true, sru::gemm::kOutBF16, 2, 1>(ma, mb, dK0, L, dp, L, B * 2 * dp,
+                                                                                  g, 2 * dp, st);
+        if (s != SRU_OK) return s;
+        // dQ += dS K: dS K-major over s; K (c = j, red = s) at KV[(s B + b0 + z) 2d' + j]: MN-major
+        if (!map_kmajor_b(&ma, dS, L, L, L, g, L * L, sru::gemm::P_CM, 2) ||
+            !map_mnmajor_b(&mb, KV + b0 * 2 * dp, dp, L, B * 2 * dp, g, 2 * dp, 1))
+            return SRU_ERR_INVALID;
+        s = causal ? launch_tc_gemm_batched<false, true, sru::gemm::kOutF32Acc, 2, 1, 2>(ma, mb, dQ + b0 * dp, L, dp, L,
+                                                                                        B * dp, g, dp, st)
+                   : launch_tc_gemm_batched<false, true, sru::gemm::kOutF32Acc, 2, 1>(ma, mb, dQ + b0 * dp, L, dp, L,
+                                                                                     B * dp, g, dp, st);
+        if (s != SRU_OK) return s;
+    }
+    // [K | V] = Q Wkv^T:  dQ += [dK | dV] Wkv,  dWkv = [dK | dV]^T Q
+    s = sru_project_backward(dKV, Q, Wkv, SRU_BF16, dQ, 1, nullptr, M, 2 * dp, dp, stream);
+    if (s != SRU_OK) return s;
+    s = project_dW_split(dKV, Q, dWkv, M, 2 * dp, dp, split, w.split_bytes, st);
+    if (s != SRU_OK) return s;
+    // Q = X Wq^T:  dWq = dQ^T X,  dX (+)= dQ Wq  (dQ rounded to bf16 as the products' operand)
+    const size_t n4 = (size_t)M * dp / 4;
+    sru::sru_f32_to_bf16_kernel<<<(unsigned)std::min<size_t>(blocks_for(n4, 256), (size_t)sm_count() * 8), 256, 0,
+                                  st>>>(reinterpret_cast<const float4*>(dQ), reinterpret_cast<uint2*>(dQb), n4);
+    SRU_CUDA_TRY(cudaGetLastError());
+    s = sru_project_backward(dQb, X, Wq, SRU_BF16, dX, accumulate, nullptr, M, dp, d, stream);
+    if (s != SRU_OK) return s;
+    return project_dW_split(dQb, X, dWq, M, dp, d, split, w.split_bytes, st);
 }
 
 // Batch rows from which the step's product runs on the tensor cores (measured:

@@ -6,9 +6,12 @@
 //   A^T = softmax(Q^T K / sqrt(d')) V^T,
 //   U^T = W_o (Q + alpha A)      or  W_o layernorm(Q + alpha A)
 // (post-attention normalisation).  The products run on the tensor-core GEMM
-// (sru_gemm.cuh); this file holds the two row-wise steps between them: the
+// (sru_gemm.cuh); this file holds the row-wise steps between them: the
 // scaled, optionally causal softmax of one batch row's L x L scores, and the
-// residual Q + alpha A with the optional layer norm.  One warp per row.
+// residual Q + alpha A with the optional layer norm, and, for the backward
+// (the reverse-mode derivative of those two steps), the softmax's and the
+// norm's gradients.  One warp per row, except the column sums of the norm's
+// parameter gradients.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -81,6 +84,132 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_residual_norm_kernel(
     for (int j = lane; j < dp; j += 32) {
         const float z = fmaf(alpha, a[j], __bfloat162float(q[j])) - mean;
         r[j] = __float2bfloat16_rn(fmaf(z * rstd, gamma[j], beta[j]));
+    }
+}
+
+// ------------------------------------------------------------------ backward
+// Softmax gradient of one row t: with p = P[t][.] (the bf16 probabilities the
+// forward multiplied by V) and g = dP[t][.],
+//   dS[t][s] = p_s (g_s - sum_s' p_s' g_s') * scale       for the visible s,
+// and 0 for the others (so that products reading up to the end of a row's
+// tile see zeros).  The scale is the forward's 1/sqrt(d'): the scores'
+// gradient is taken with respect to Q K^T itself.
+__global__ void __launch_bounds__(kRowWarps * 32) sru_softmax_backward_rows_kernel(
+    const float* __restrict__ dP, const __nv_bfloat16* __restrict__ P, __nv_bfloat16* __restrict__ dS, int L, int rows,
+    float scale, int causal) {
+    const int row = blockIdx.x * kRowWarps + threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (row >= rows) return;
+    const int t = row % L;
+    const float* grow = dP + (size_t)row * L;
+    const __nv_bfloat16* prow = P + (size_t)row * L;
+    __nv_bfloat16* drow = dS + (size_t)row * L;
+    const int n = causal ? t + 1 : L;
+    float dot = 0.f;
+    for (int s = lane; s < n; s += 32) dot = fmaf(__bfloat162float(prow[s]), grow[s], dot);
+    dot = warp_sum(dot);
+    for (int s = lane; s < L; s += 32)
+        drow[s] = __float2bfloat16_rn(s < n ? __bfloat162float(prow[s]) * (grow[s] - dot) * scale : 0.f);
+}
+
+// Gradient through R = Z (no norm) or R = layernorm(Z) gamma + beta, with
+// Z = Q + alpha A recomputed exactly as the forward did.  Row m:
+//   no norm:  dZ = dR
+//   norm:     Zhat = (Z - mean) * rstd,  dZhat = dR * gamma,
+//             dZ = rstd * (dZhat - mean(dZhat) - Zhat * mean(dZhat * Zhat))
+// writes dQ = dZ (fp32; the attention and projection terms are added later)
+// and dA = bf16(alpha dZ), and, with the norm, the row's mean and rstd (for
+// the parameter gradients).
+__global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_kernel(
+    const float* __restrict__ dR, const __nv_bfloat16* __restrict__ Q, const float* __restrict__ A, float alpha,
+    const float* __restrict__ gamma, float* __restrict__ dQ, __nv_bfloat16* __restrict__ dA,
+    float2* __restrict__ stats, int M, int dp) {
+    const int m = blockIdx.x * kRowWarps + threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (m >= M) return;
+    const float* dr = dR + (size_t)m * dp;
+    float* dq = dQ + (size_t)m * dp;
+    __nv_bfloat16* da = dA + (size_t)m * dp;
+    if (gamma == nullptr) {
+        for (int j = lane; j < dp; j += 32) {
+            const float g = dr[j];
+            dq[j] = g;
+            da[j] = __float2bfloat16_rn(alpha * g);
+        }
+        return;
+    }
+    const __nv_bfloat16* q = Q + (size_t)m * dp;
+    const float* a = A + (size_t)m * dp;
+    float sum = 0.f;
+    for (int j = lane; j < dp; j += 32) sum += fmaf(alpha, a[j], __bfloat162float(q[j]));
+    const float mean = warp_sum(sum) / (float)dp;
+    float sq = 0.f;
+    for (int j = lane; j < dp; j += 32) {
+        const float z = fmaf(alpha, a[j], __bfloat162float(q[j])) - mean;
+        sq = fmaf(z, z, sq);
+    }
+    const float rstd = rsqrtf(warp_sum(sq) / (float)dp + kLayerNormEps);
+    float s1 = 0.f, s2 = 0.f;
+    for (int j = lane; j < dp; j += 32) {
+        const float zh = (fmaf(alpha, a[j], __bfloat162float(q[j])) - mean) * rstd;
+        const float g = dr[j] * gamma[j];
+        s1 += g;
+        s2 = fmaf(g, zh, s2);
+    }
+    s1 = warp_sum(s1) / (float)dp;
+    s2 = warp_sum(s2) / (float)dp;
+    for (int j = lane; j < dp; j += 32) {
+        const float zh = (fmaf(alpha, a[j], __bfloat162float(q[j])) - mean) * rstd;
+        const float g = dr[j] * gamma[j];
+        const float dz = rstd * (g - s1 - zh * s2);
+        dq[j] = dz;
+        da[j] = __float2bfloat16_rn(alpha * dz);
+    }
+    if (lane == 0) stats[m] = make_float2(mean, rstd);
+}
+
+// The norm's parameter gradients, first stage: slice y of the rows (rows
+// [y * rows_per, (y + 1) * rows_per)) summed per feature j in fp32, in row
+// order, into part[y][0][j] (dgamma: dR * Zhat) and part[y][1][j] (dbeta: dR).
+constexpr int kNormParamThreads = 256;
+__global__ void __launch_bounds__(kNormParamThreads) sru_norm_param_partial_kernel(
+    const float* __restrict__ dR, const __nv_bfloat16* __restrict__ Q, const float* __restrict__ A, float alpha,
+    const float2* __restrict__ stats, float* __restrict__ part, int M, int dp, int rows_per) {
+    const int j = blockIdx.x * kNormParamThreads + threadIdx.x;
+    if (j >= dp) return;
+    const int m0 = blockIdx.y * rows_per, m1 = min(M, m0 + rows_per);
+    float sg = 0.f, sb = 0.f;
+    for (int m = m0; m < m1; ++m) {
+        const size_t e = (size_t)m * dp + j;
+        const float2 st = stats[m];
+        const float zh = (fmaf(alpha, A[e], __bfloat162float(Q[e])) - st.x) * st.y;
+        sg = fmaf(dR[e], zh, sg);
+        sb += dR[e];
+    }
+    part[((size_t)blockIdx.y * 2 + 0) * dp + j] = sg;
+    part[((size_t)blockIdx.y * 2 + 1) * dp + j] = sb;
+}
+
+// Second stage: the slices' partial sums per feature in slice order, in fp64.
+__global__ void __launch_bounds__(256) sru_norm_param_reduce_kernel(const float* __restrict__ part, int slices, int dp,
+                                                                    float* __restrict__ dgamma,
+                                                                    float* __restrict__ dbeta) {
+    const int j = blockIdx.x * 256 + threadIdx.x;
+    if (j >= dp) return;
+    double sg = 0.0, sb = 0.0;
+    for (int y = 0; y < slices; ++y) {
+        sg += (double)part[((size_t)y * 2 + 0) * dp + j];
+        sb += (double)part[((size_t)y * 2 + 1) * dp + j];
+    }
+    dgamma[j] = (float)sg;
+    dbeta[j] = (float)sb;
+}
+
+// out[i] = bf16(in[i]), four at a time (n a multiple of 4, both 16-byte aligned).
+__global__ void __launch_bounds__(256) sru_f32_to_bf16_kernel(const float4* __restrict__ in,
+                                                              uint2* __restrict__ out, size_t n4) {
+    for (size_t i = blockIdx.x * (size_t)256 + threadIdx.x; i < n4; i += (size_t)gridDim.x * 256) {
+        const float4 v = in[i];
+        __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+        out[i] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
     }
 }
 

@@ -112,24 +112,25 @@ constexpr uint32_t P_B_BYTES = P_CN * BK * 2;          // 16 KB
 constexpr uint32_t P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
 constexpr uint32_t P_TMEM_COLS = 2 * P_BN;             // two 128 x 256 fp32 accumulators per CTA
 // Epilogue staging (non-batched launches): each of the 4 epilogue warps owns
-// two 4 KB buffers; a 32 x 32 output chunk is written there in the TMA swizzle
-// pattern and leaves by one TMA store (or TMA reduce-add), so the output goes
-// out as whole lines instead of 16-byte pieces of 32 different rows.
+// two 4 KB buffers; a chunk of 32 rows x 128 bytes (64 bf16 or 32 fp32 output
+// columns) is written there in the TMA swizzle pattern and leaves by one TMA
+// store (or TMA reduce-add), so the output goes out as whole lines instead of
+// 16-byte pieces of 32 different rows.
 constexpr uint32_t P_EPI_BUF = 4096;
 constexpr uint32_t P_EPI_BYTES = 4 * 2 * P_EPI_BUF;
 constexpr size_t P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + P_EPI_BYTES + 1024 + 256;
 static_assert(P_SMEM_BYTES <= 232448, "pair GEMM shared memory");
 
-// Write one row's 32 accumulator columns (r, fp32 bits) into a staging buffer
-// laid out as the TMA tensor's 32 x 32 box with its swizzle: fp32 rows of
-// 128 B with 128-byte swizzle (16-byte chunk c of row i at chunk c ^ (i % 8)),
-// bf16 rows of 64 B with 64-byte swizzle (chunk c at c ^ ((i / 2) % 4)).
-// Either way the 32 rows' stores of one chunk fall in distinct banks.
+// Write one row's accumulator columns (r, fp32 bits) into a staging buffer laid
+// out as the TMA tensor's box with 128-byte swizzle: each output row is 128 B
+// (64 bf16 or 32 fp32 columns), and its 16-byte chunk c sits at chunk
+// c ^ (i % 8) of row i, so the 32 rows' stores of one chunk fall in distinct banks.
 template <int OUT>
-__device__ __forceinline__ void epilogue_stage_row32(uint32_t buf, int i, const uint32_t (&r)[32]) {
-    if (OUT == kOutBF16) {
+__device__ __forceinline__ void epilogue_stage_row(uint32_t buf, int i, const uint32_t* r) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 8; ++c) {
+        const uint32_t dst = buf + (uint32_t)i * 128u + ((uint32_t)(c ^ (i & 7)) << 4);
+        if (OUT == kOutBF16) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -137,14 +138,25 @@ __device__ __forceinline__ void epilogue_stage_row32(uint32_t buf, int i, const 
                                                            __uint_as_float(r[c * 8 + 2 * e + 1]));
                 w[e] = *reinterpret_cast<uint32_t*>(&two);
             }
-            st_shared_v4(buf + (uint32_t)i * 64u + ((uint32_t)(c ^ ((i >> 1) & 3)) << 4), w[0], w[1], w[2], w[3]);
+            st_shared_v4(dst, w[0], w[1], w[2], w[3]);
+        } else {
+            st_shared_v4(dst, r[4 * c], r[4 * c + 1], r[4 * c + 2], r[4 * c + 3]);
         }
-    } else {
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-            st_shared_v4(buf + (uint32_t)i * 128u + ((uint32_t)(c ^ (i & 7)) << 4), r[4 * c], r[4 * c + 1],
-                         r[4 * c + 2], r[4 * c + 3]);
     }
+}
+
+// Accumulator columns per staged box: one 128-byte row per output row.
+template <int OUT>
+struct EpiChunk {
+    static constexpr int kCols = OUT == kOutBF16 ? 64 : 32;
+};
+
+// Load kCols consecutive accumulator columns of this warp's 32 TMEM lanes.
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NC]) {
+    static_assert(NC == 32 || NC == 64, "columns per load");
+    tmem_ld_32x32b_x32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+    if (NC == 64) tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[NC == 64 ? 32 : 0]));
 }
 
 __host__ __device__ constexpr uint32_t idesc_bf16_pair(bool a_mn, bool b_mn) {
@@ -176,10 +188,13 @@ __device__ __forceinline__ void tma_load_tile_pair(void* dst, const CUtensorMap*
 // causal attention, tiles of P_BM = P_BN rows):
 //   1  scores S = Q K^T: only the tiles on or below the diagonal (tn <= tm);
 //      the tiles above it hold only masked entries, which the softmax never reads;
-//   2  A = P V: the reduction over s stops at the end of the row tile, past
-//      which every probability is 0.
+//   2  A = P V (and dQ = dS K): the reduction over s stops at the end of the
+//      row tile, past which every probability (gradient) is 0;
+//   3  dV = P^T dA (and dK = dS^T Q): output row tile s0.. reduces over
+//      t >= s0 only, since P[t][s] = 0 for t < s.
 struct PairUnit {
     int z, tm, tn, kb_lo, kb_hi;
+    int split;    // k part of a split-K launch (0 otherwise)
     bool reduce;  // add onto the output (a piece of a tile split in two) instead of storing
 };
 template <int CAUSAL>
@@ -196,6 +211,8 @@ __device__ __forceinline__ PairUnit pair_unit(int u, int m_tiles, int n_tiles, i
         w.tn = t - tm * (tm + 1) / 2;
         w.kb_lo = 0;
         w.kb_hi = kblocks;
+        w.split = 0;
+        w.reduce = false;
         return w;
     }
     const int tiles = m_tiles * n_tiles;
@@ -203,9 +220,11 @@ __device__ __forceinline__ PairUnit pair_unit(int u, int m_tiles, int n_tiles, i
     const int uu = u % (tiles * splits), tile = uu / splits;
     w.tm = tile / n_tiles;
     w.tn = tile % n_tiles;
-    w.kb_lo = (uu % splits) * kper;
+    w.split = uu % splits;
+    w.kb_lo = w.split * kper;
     w.kb_hi = min(kblocks, w.kb_lo + kper);
     if (CAUSAL == 2) w.kb_hi = min(w.kb_hi, ((w.tm + 1) * P_BM + BK - 1) / BK);
+    if (CAUSAL == 3) w.kb_lo = max(w.kb_lo, (w.tm * P_BM) / BK);
     w.reduce = false;
     return w;
 }
@@ -252,6 +271,7 @@ __device__ __forceinline__ bool pair_next(int i, int p, int P, int units, int m_
     w.tm = tile / n_tiles;
     w.tn = tile % n_tiles;
     w.reduce = i >= F;
+    w.split = 0;
     w.kb_lo = (i < F || !large) ? 0 : tail_s;
     w.kb_hi = (i < F || large) ? kblocks : tail_s;
     return true;
@@ -261,7 +281,7 @@ template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0, int CAUSAL = 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                         const __grid_constant__ CUtensorMap map_out, void* __restrict__ out, int M, int N, int K,
-                        int ldo, int splits, int batches, long long out_bstride, int tail_s) {
+                        int ldo, int splits, int batches, long long out_bstride, int tail_s, int slab_rows) {
     constexpr bool kTmaOut = (BPA | BPB) == 0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -438,12 +458,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             tc_fence_after_sync();
             const int row = m0 + quarter * 32 + lane;
-            for (int ch = 0; ch < P_BN / 32; ++ch) {
-                const int col0 = n0 + ch * 32;
-                if (col0 >= N) break;  // uniform across the warp
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * P_BN + ch * 32, r);
-                tc_wait_ld();
+            // the accumulator leaves in chunks of kCols columns; the TMEM load of chunk
+            // g + 1 is issued before chunk g is converted and stored, so its latency
+            // overlaps that work
+            constexpr int NC = EpiChunk<OUT>::kCols, NG = P_BN / NC;
+            const int ng = min(NG, (N - n0 + NC - 1) / NC);  // chunks that start inside N (>= 1)
+            const uint32_t tacc = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * P_BN;
+            uint32_t r0[NC], r1[NC];
+            tmem_ld_cols<NC>(tacc, r0);
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+                if (g >= ng) break;  // uniform across the warp
+                uint32_t(&cur)[NC] = (g & 1) ? r1 : r0;
+                uint32_t(&nxt)[NC] = (g & 1) ? r0 : r1;
+                tc_wait_ld();  // chunk g (and nothing else) is in flight
+                if (g + 1 < ng) tmem_ld_cols<NC>(tacc + (g + 1) * NC, nxt);
+                const int col0 = n0 + g * NC;
                 if (kTmaOut) {
                     // buffer (nstaged & 1) was last read by the store issued two chunks ago
                     const uint32_t buf = smem_u32(epi) + (uint32_t)(quarter * 2 + (nstaged & 1)) * P_EPI_BUF;
@@ -451,20 +481,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         if (lane == 0) bulk_wait_group_read<1>();
                         __syncwarp();
                     }
-                    epilogue_stage_row32<OUT>(buf, lane, r);
+                    epilogue_stage_row<OUT>(buf, lane, cur);
                     fence_proxy_async_shared();
                     __syncwarp();
                     if (lane == 0) {
                         const void* src = epi + (size_t)(quarter * 2 + (nstaged & 1)) * P_EPI_BUF;
+                        // split-K: k part s lands in slab s, rows s * slab_rows ..
+                        const int orow = m0 + quarter * 32 + w.split * slab_rows;
                         if (OUT == kOutF32Acc || w.reduce)
-                            tma_reduce_add_2d(&map_out, src, col0, m0 + quarter * 32);
+                            tma_reduce_add_2d(&map_out, src, col0, orow);
                         else
-                            tma_store_2d(&map_out, src, col0, m0 + quarter * 32);
+                            tma_store_2d(&map_out, src, col0, orow);
                         bulk_commit_group();
                     }
                     ++nstaged;
                 } else {
-                    epilogue_store_row32<OUT>(zout, row, col0, M, N, ldo, r);
+#pragma unroll
+                    for (int h = 0; h < NC / 32; ++h)
+                        if (col0 + h * 32 < N)
+                            epilogue_store_row32<OUT>(zout, row, col0 + h * 32, M, N, ldo,
+                                                      *reinterpret_cast<const uint32_t(*)[32]>(&cur[h * 32]));
                 }
             }
             tc_fence_before_sync();
@@ -493,6 +529,25 @@ __global__ void __launch_bounds__(256) zero_tail_tiles_kernel(float* __restrict_
     for (int e = threadIdx.x; e < rows * (cols / 4); e += blockDim.x) {
         const int r = e / (cols / 4), c4 = e % (cols / 4);
         *reinterpret_cast<float4*>(out + (size_t)(r0 + r) * ldo + c0 + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+// Split-K: out[r][c] = sum over s = 0, 1, .. of slabs[s * slab_rows + r][c], in
+// that order (the same bits every run); four columns per thread (C % 4 == 0).
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float4* __restrict__ slabs, float4* __restrict__ out,
+                                                            int R, int C4, int slab_rows, int splits) {
+    const size_t n = (size_t)R * C4;
+    for (size_t e = blockIdx.x * (size_t)256 + threadIdx.x; e < n; e += (size_t)gridDim.x * 256) {
+        const size_t r = e / C4, c = e % C4;
+        float4 acc = slabs[r * C4 + c];
+        for (int sp = 1; sp < splits; ++sp) {
+            const float4 v = slabs[((size_t)sp * slab_rows + r) * C4 + c];
+            acc.x += v.x;
+            acc.y += v.y;
+            acc.z += v.z;
+            acc.w += v.w;
+        }
+        out[e] = acc;
     }
 }
 

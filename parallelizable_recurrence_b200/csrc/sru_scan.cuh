@@ -128,16 +128,32 @@ __global__ void sru_scan_reset_kernel(unsigned* __restrict__ flags, int n) {
     if (i < n) flags[i] = 0u;
 }
 
+// A scan CTA has one warp per 16-step sub-chunk of its item: warp q stages,
+// reduces and re-walks sub-chunk q, so the item's 64 dependent steps run as
+// four chains of 16 in parallel.  The sub-chunks' affine maps meet in shared
+// memory (one float4 (A.x, A.y, B.x, B.y) per lane and sub-chunk) and are
+// composed there, in the direction's time order, into the item's map and into
+// the state entering each sub-chunk.
+constexpr int kScanThreads = kScanSub * 32;
+
+// (A, B) of the maps applied one after another: first (a0, b0), then (a1, b1).
+__device__ __forceinline__ void compose_after(float2& a0, float2& b0, float2 a1, float2 b1) {
+    b0 = fma2(a1, b0, b1);
+    a0 = mul2(a1, a0);
+}
+
 template <typename UT>
 struct FwdScanLayout {
     static constexpr int STAGE = FwdLayout<UT>::STAGE;
-    static constexpr int BAR_OFF = kScanSub * STAGE;
-    static constexpr int SMEM = BAR_OFF + 64 + 128;
+    static constexpr int MAP_OFF = kScanSub * STAGE;
+    static constexpr int BAR_OFF = MAP_OFF + kScanSub * 32 * 16;
+    static constexpr int SMEM = BAR_OFF + kScanSub * 8 + 64 + 128;
 };
 
-// Forward, v = 0.  1-D grid of n_items = ceil(L/kScanT) * ceil(d/CJ) * B * n_dir CTAs.
+// Forward, v = 0.  1-D grid of n_items = ceil(L/kScanT) * ceil(d/CJ) * B * n_dir
+// CTAs of kScanThreads threads.
 template <typename UT>
-__global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
+__global__ void __launch_bounds__(kScanThreads) sru_fwd_scan_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
     const float* __restrict__ bias, const float* __restrict__ c0, const uint8_t* __restrict__ mask,
     float* __restrict__ h, float* __restrict__ c_T, float* __restrict__ ckpt, ScanState ss, int L, int B, int d,
@@ -145,16 +161,17 @@ __global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
     using Lay = FwdScanLayout<UT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
-    unsigned* s_misc = reinterpret_cast<unsigned*>(bar + 1);  // [0] ticket, [1] flag
+    float4* s_map = reinterpret_cast<float4*>(smem + Lay::MAP_OFF);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);    // one per sub-chunk
+    unsigned* s_misc = reinterpret_cast<unsigned*>(bar + kScanSub);       // [0] ticket, [1] flag
 
-    const int tid = threadIdx.x, lane = tid, cj = 2 * lane;
+    const int tid = threadIdx.x, q = tid >> 5, lane = tid & 31, cj = 2 * lane;
     const int n_jt = (d + kRecCJ - 1) / kRecCJ;
     const int n_tiles = n_jt * B * n_dir;
     const int n_items = gridDim.x;
     if (tid == 0) {
         s_misc[0] = atomicAdd(&ss.flags[n_items], 1u);
-        mbar_init(bar, 1);
+        for (int i = 0; i < kScanSub; ++i) mbar_init(&bar[i], 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -173,69 +190,60 @@ __global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
     if (jok)
         p = make_gate_params2(f2(0.f), f2(0.f), load_pair(bias + (dir * 2 + 0) * d + j),
                               load_pair(bias + (dir * 2 + 1) * d + j));
-    uint32_t valid[kScanSub], inrange[kScanSub];
-    bool any = false;
-#pragma unroll
-    for (int q = 0; q < kScanSub; ++q) {
-        const int ts = t0 + q * kChunkT;
-        valid[q] = ts < L ? chunk_valid_bits(mask, ts, L, B, b, lane) : 0u;
-        inrange[q] = ts < L ? chunk_inrange_bits(ts, L) : 0u;
-        any |= valid[q] != 0u;
+    // this warp's sub-chunk: rows ts .. ts + 15
+    const int ts = t0 + q * kChunkT;
+    const uint32_t valid = ts < L ? chunk_valid_bits(mask, ts, L, B, b, lane) : 0u;
+    const uint32_t inrange = ts < L ? chunk_inrange_bits(ts, L) : 0u;
+    uint8_t* st = smem + q * Lay::STAGE;
+    if (lane == 0 && valid != 0u) {
+        mbar_arrive_expect_tx(&bar[q], (uint32_t)Lay::STAGE);
+        tma_load_4d(st, &map_u, &bar[q], j0, 0, bd, ts);
+        tma_load_3d(st + FwdLayout<UT>::U_BYTES, &map_x, &bar[q], j0, b, ts);
     }
-    if (tid == 0 && any) {
-        uint32_t bytes = 0;
-#pragma unroll
-        for (int q = 0; q < kScanSub; ++q) bytes += valid[q] ? (uint32_t)Lay::STAGE : 0u;
-        mbar_arrive_expect_tx(bar, bytes);
-#pragma unroll
-        for (int q = 0; q < kScanSub; ++q) {
-            if (!valid[q]) continue;
-            uint8_t* st = smem + q * Lay::STAGE;
-            tma_load_4d(st, &map_u, bar, j0, 0, bd, t0 + q * kChunkT);
-            tma_load_3d(st + FwdLayout<UT>::U_BYTES, &map_x, bar, j0, b, t0 + q * kChunkT);
-        }
-    }
-    uint64_t valid_all = 0, inrange_all = 0;
-#pragma unroll
-    for (int q = 0; q < kScanSub; ++q) {
-        valid_all |= (uint64_t)valid[q] << (kChunkT * q);
-        inrange_all |= (uint64_t)inrange[q] << (kChunkT * q);
-    }
-    if (any) {
-        const bool ok = mbar_wait(bar, 0, kErrTimeoutLoad);
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) mbar_wait(bar, 0, kErrTimeoutLoad);
-            scan_publish(&ss.flags[w], kFlagAbort);
-            return;
-        }
+    const bool ok = valid == 0u || mbar_wait(&bar[q], 0, kErrTimeoutLoad);
+    if (__syncthreads_or(!ok)) {
+        if (lane == 0 && valid != 0u) mbar_wait(&bar[q], 0, kErrTimeoutLoad);
+        scan_publish(&ss.flags[w], kFlagAbort);
+        return;
     }
 
-    // 1. the chunk as an affine map of the entering state: c_out = A c_in + Bc
+    // 1. this sub-chunk as an affine map of its entering state, then the item's
+    const UT* us = reinterpret_cast<const UT*>(st);
     float2 A = f2(1.f), Bc = f2(0.f);
-#pragma unroll 1
-    for (int qq = 0; qq < kScanSub; ++qq) {
-        const int q = dir == 0 ? qq : kScanSub - 1 - qq;
-        const UT* us = reinterpret_cast<const UT*>(smem + q * Lay::STAGE);
 #pragma unroll
-        for (int r = 0; r < kChunkT; ++r) {
-            const int i = dir == 0 ? r : kChunkT - 1 - r;
-            if ((sub_bits(valid_all, q) >> i) & 1u) {
-                const float2 uc = load_pair(us + (i * 3 + 0) * kRecCJ + cj);
-                const float2 f =
-                    sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 1) * kRecCJ + cj), f2(kNegLog2e), p.nbf));
-                A = mul2(A, f);
-                Bc = fma2(f, sub2(Bc, uc), uc);
-            }
+    for (int r = 0; r < kChunkT; ++r) {
+        const int i = dir == 0 ? r : kChunkT - 1 - r;
+        if ((valid >> i) & 1u) {
+            const float2 uc = load_pair(us + (i * 3 + 0) * kRecCJ + cj);
+            const float2 f = sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 1) * kRecCJ + cj), f2(kNegLog2e), p.nbf));
+            A = mul2(A, f);
+            Bc = fma2(f, sub2(Bc, uc), uc);
         }
     }
-    // 2. state entering the chunk
+    s_map[q * 32 + lane] = make_float4(A.x, A.y, Bc.x, Bc.y);
+    __syncthreads();
+    // item map and the map of the sub-chunks before this one, in time order
+    float2 Ai = f2(1.f), Bi = f2(0.f), Ab = f2(1.f), Bb = f2(0.f);
+#pragma unroll
+    for (int qq = 0; qq < kScanSub; ++qq) {
+        const int qs = dir == 0 ? qq : kScanSub - 1 - qq;
+        if (qs == q) {
+            Ab = Ai;
+            Bb = Bi;
+        }
+        const float4 m = s_map[qs * 32 + lane];
+        compose_after(Ai, Bi, make_float2(m.x, m.y), make_float2(m.z, m.w));
+    }
+    // 2. state entering the item
     float2 c_in = f2(0.f);
     const size_t me = (size_t)w * kRecCJ + cj;
     if (k == 0) {
         c_in = (jok && c0 != nullptr) ? load_pair(c0 + (size_t)bd * d + j) : f2(0.f);
     } else {
-        store_pair(ss.agg_a + me, A);
-        store_pair(ss.agg_b + me, Bc);
+        if (q == 0) {
+            store_pair(ss.agg_a + me, Ai);
+            store_pair(ss.agg_b + me, Bi);
+        }
         scan_publish(&ss.flags[w], kFlagAgg);
         if (!scan_lookback(ss, k, tile, n_tiles, cj, s_misc + 1, c_in)) {
             scan_publish(&ss.flags[w], kFlagAbort);
@@ -243,41 +251,37 @@ __global__ void __launch_bounds__(kRecThreads) sru_fwd_scan_kernel(
         }
     }
     if (w == ss.withhold) return;  // successors' waits expire (test hook)
-    store_pair(ss.prefix + me, fma2(A, c_in, Bc));
+    if (q == 0) store_pair(ss.prefix + me, fma2(Ai, c_in, Bi));
     scan_publish(&ss.flags[w], kFlagPrefix);
 
-    // 3. walk the chunk again from shared memory: h and the 16-step checkpoints
-    float2 c = c_in;
-    const float2 alpha2 = f2(alpha);
+    // 3. walk this sub-chunk again from its entering state: h and its checkpoint
+    if (ts >= L) return;
+    float2 c = fma2(Ab, c_in, Bb);
+    const int c16 = tc * kScanSub + q;
+    if (ckpt != nullptr && jok && c16 < nch16) store_pair(ckpt + ((size_t)c16 * B * n_dir + bd) * d + j, c);
     const size_t h_tstride = (size_t)B * n_dir * d;
-#pragma unroll 1
-    for (int qq = 0; qq < kScanSub; ++qq) {
-        const int q = dir == 0 ? qq : kScanSub - 1 - qq;
-        const int ts = t0 + q * kChunkT;
-        if (ts >= L) continue;
-        const int c16 = tc * kScanSub + q;
-        if (ckpt != nullptr && jok && c16 < nch16) store_pair(ckpt + ((size_t)c16 * B * n_dir + bd) * d + j, c);
-        const UT* us = reinterpret_cast<const UT*>(smem + q * Lay::STAGE);
-        const float* xs = reinterpret_cast<const float*>(smem + q * Lay::STAGE + FwdLayout<UT>::U_BYTES);
-        float* hp = h + (size_t)ts * h_tstride + (size_t)bd * d + j;
-        c = fwd_chunk<UT, kRecCJ>(us, xs, sub_bits(valid_all, q), sub_bits(inrange_all, q), c, p, alpha2, dir, hp, h_tstride, jok, cj);
-    }
-    if (k == nchs - 1 && jok) store_pair(c_T + (size_t)bd * d + j, c);
+    const float* xs = reinterpret_cast<const float*>(st + FwdLayout<UT>::U_BYTES);
+    float* hp = h + (size_t)ts * h_tstride + (size_t)bd * d + j;
+    c = fwd_chunk<UT, kRecCJ>(us, xs, valid, inrange, c, p, f2(alpha), dir, hp, h_tstride, jok, cj);
+    // the last sub-chunk in walk order leaves c_T
+    const bool last = dir == 0 ? (ts + kChunkT >= L || q == kScanSub - 1) : q == 0;
+    if (k == nchs - 1 && last && jok) store_pair(c_T + (size_t)bd * d + j, c);
 }
 
 template <typename UT, bool ACC_DX>
 struct BwdScanLayout {
     static constexpr int STAGE = BwdLayout<UT, ACC_DX>::STAGE;
-    static constexpr int CK_OFF = kScanSub * STAGE;             // checkpoints: [kScanSub][CJ] fp32
-    static constexpr int ACC_OFF = CK_OFF + kScanSub * kRecCJ * 4;  // SmemPartials: 8 doubles per thread
-    static constexpr int BAR_OFF = ACC_OFF + kRecThreads * 8 * 8;
-    static constexpr int SMEM = BAR_OFF + 64 + 128;
+    static constexpr int ACC_OFF = kScanSub * STAGE;                  // SmemPartials: 8 doubles per thread
+    static constexpr int MAP_OFF = ACC_OFF + kScanThreads * 8 * 8;
+    static constexpr int BAR_OFF = MAP_OFF + kScanSub * 32 * 16;
+    static constexpr int SMEM = BAR_OFF + kScanSub * 8 + 64 + 128;
 };
 
-// Backward of direction DIR, v = 0.  1-D grid of n_items = ceil(L/kScanT) * ceil(d/CJ) * B.
+// Backward of direction DIR.  1-D grid of n_items = ceil(L/kScanT) * ceil(d/CJ) * B
+// CTAs of kScanThreads threads (warp q: sub-chunk q of the item).
 // partial: (nchs * B, n_dir, 4, d) doubles.
 template <typename UT, typename DUT, bool ACC_DX, int DIR, bool VZERO>
-__global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
+__global__ void __launch_bounds__(kScanThreads) sru_bwd_scan_kernel(
     const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_x,
     const __grid_constant__ CUtensorMap map_dh,
     const float* __restrict__ v, const float* __restrict__ bias, const uint8_t* __restrict__ mask,
@@ -288,16 +292,17 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
     using SL = BwdLayout<UT, ACC_DX>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    float4* s_map = reinterpret_cast<float4*>(smem + Lay::MAP_OFF);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
-    unsigned* s_misc = reinterpret_cast<unsigned*>(bar + 1);
+    unsigned* s_misc = reinterpret_cast<unsigned*>(bar + kScanSub);
 
-    const int tid = threadIdx.x, lane = tid, cj = 2 * lane;
+    const int tid = threadIdx.x, q = tid >> 5, lane = tid & 31, cj = 2 * lane;
     const int n_jt = (d + kRecCJ - 1) / kRecCJ;
     const int n_tiles = n_jt * B;
     const int n_items = gridDim.x;
     if (tid == 0) {
         s_misc[0] = atomicAdd(&ss.flags[n_items], 1u);
-        mbar_init(bar, 1);
+        for (int i = 0; i < kScanSub; ++i) mbar_init(&bar[i], 1);
         fence_mbar_init();
     }
     __syncthreads();
@@ -317,124 +322,103 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
                               load_pair(bias + (DIR * 2 + 0) * d + j), load_pair(bias + (DIR * 2 + 1) * d + j));
     const float2 alpha2 = f2(alpha);
     const int nch16 = (L + kChunkT - 1) / kChunkT;
-    uint32_t valid[kScanSub], inrange[kScanSub];
-    bool any = false;
-#pragma unroll
-    for (int q = 0; q < kScanSub; ++q) {
-        const int ts = t0 + q * kChunkT;
-        valid[q] = ts < L ? chunk_valid_bits(mask, ts, L, B, b, lane) : 0u;
-        inrange[q] = ts < L ? chunk_inrange_bits(ts, L) : 0u;
-        any |= valid[q] != 0u;
+    // this warp's sub-chunk: rows ts .. ts + 15
+    const int ts = t0 + q * kChunkT;
+    const uint32_t valid = ts < L ? chunk_valid_bits(mask, ts, L, B, b, lane) : 0u;
+    const uint32_t inrange = ts < L ? chunk_inrange_bits(ts, L) : 0u;
+    uint8_t* st = smem + q * SL::STAGE;
+    if (lane == 0 && valid != 0u) {
+        mbar_arrive_expect_tx(&bar[q], (uint32_t)SL::STAGE);
+        tma_load_4d(st, &map_u, &bar[q], j0, 0, bd, ts);
+        tma_load_3d(st + SL::U_BYTES, &map_x, &bar[q], j0, b, ts);
+        tma_load_3d(st + SL::U_BYTES + SL::V_BYTES, &map_dh, &bar[q], j0, bd, ts);
     }
-    if (tid == 0 && any) {
-        uint32_t bytes = 0;
-#pragma unroll
-        for (int q = 0; q < kScanSub; ++q) bytes += valid[q] ? (uint32_t)SL::STAGE : 0u;
-        mbar_arrive_expect_tx(bar, bytes);
-#pragma unroll
-        for (int q = 0; q < kScanSub; ++q) {
-            if (!valid[q]) continue;
-            uint8_t* st = smem + q * SL::STAGE;
-            const int ts = t0 + q * kChunkT;
-            tma_load_4d(st, &map_u, bar, j0, 0, bd, ts);
-            tma_load_3d(st + SL::U_BYTES, &map_x, bar, j0, b, ts);
-            tma_load_3d(st + SL::U_BYTES + SL::V_BYTES, &map_dh, bar, j0, bd, ts);
-        }
+    // the sub-chunk's forward checkpoint, fetched while the tiles load
+    const int c16 = tc * kScanSub + q;
+    const float2 ck = (jok && c16 < nch16) ? load_pair(ckpt + ((size_t)c16 * B * n_dir + bd) * d + j) : f2(0.f);
+    const bool ok = valid == 0u || mbar_wait(&bar[q], 0, kErrTimeoutLoad);
+    if (__syncthreads_or(!ok)) {
+        if (lane == 0 && valid != 0u) mbar_wait(&bar[q], 0, kErrTimeoutLoad);
+        scan_publish(&ss.flags[w], kFlagAbort);
+        return;
     }
-    uint64_t valid_all = 0, inrange_all = 0;
-#pragma unroll
-    for (int q = 0; q < kScanSub; ++q) {
-        valid_all |= (uint64_t)valid[q] << (kChunkT * q);
-        inrange_all |= (uint64_t)inrange[q] << (kChunkT * q);
-    }
-    // the sub-chunks' forward checkpoints, fetched while the tiles load
-    float2* s_ck = reinterpret_cast<float2*>(smem + Lay::CK_OFF) + lane;  // sub-chunk q at s_ck[q * 32]
-#pragma unroll
-    for (int q = 0; q < kScanSub; ++q) {
-        const int c16 = tc * kScanSub + q;
-        s_ck[q * 32] = (jok && c16 < nch16) ? load_pair(ckpt + ((size_t)c16 * B * n_dir + bd) * d + j) : f2(0.f);
-    }
-    if (any) {
-        const bool ok = mbar_wait(bar, 0, kErrTimeoutLoad);
-        if (__syncthreads_or(!ok)) {
-            if (tid == 0) mbar_wait(bar, 0, kErrTimeoutLoad);
-            scan_publish(&ss.flags[w], kFlagAbort);
-            return;
-        }
-    }
+    const UT* us = reinterpret_cast<const UT*>(st);
+    const float* xs = reinterpret_cast<const float*>(st + SL::U_BYTES);
+    const float* dhs = xs + kChunkT * kRecCJ;
 
-    // 1. the chunk as an affine map of the state gradient, g_out = A g_in + Bg.
+    // 1. this sub-chunk as an affine map of the state gradient, g_out = A g_in + Bg.
     //    Each valid row maps g to a g + b with (see bwd_chunk)
     //      a = f + (c' - u) f(1-f) v_f,  b = a dh r + dh (c - alpha x) r(1-r) v_r,
-    //    which needs the row's forward state: every 16-step sub-chunk is re-run
-    //    from its checkpoint (bit-identical to the forward), then walked back.
+    //    which needs the row's forward state: the sub-chunk is re-run from its
+    //    checkpoint (bit-identical to the forward), then walked back.
     float2 A = f2(1.f), Bg = f2(0.f);
     if (VZERO) {
         // v = 0: the gates do not read c, so a = f and b = f dh r need no state
-#pragma unroll 1
-        for (int qq = 0; qq < kScanSub; ++qq) {
-            const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
-            const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
-            const float* dhs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES + SL::V_BYTES);
 #pragma unroll
-            for (int r = 0; r < kChunkT; ++r) {
-                const int i = DIR == 0 ? kChunkT - 1 - r : r;
-                if ((sub_bits(valid_all, q) >> i) & 1u) {
-                    const float2 f =
-                        sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 1) * kRecCJ + cj), f2(kNegLog2e), p.nbf));
-                    const float2 rr =
-                        sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 2) * kRecCJ + cj), f2(kNegLog2e), p.nbr));
-                    A = mul2(A, f);
-                    Bg = mul2(f, fma2(load_pair(dhs + i * kRecCJ + cj), rr, Bg));
-                }
+        for (int r = 0; r < kChunkT; ++r) {
+            const int i = DIR == 0 ? kChunkT - 1 - r : r;
+            if ((valid >> i) & 1u) {
+                const float2 f = sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 1) * kRecCJ + cj), f2(kNegLog2e), p.nbf));
+                const float2 rr =
+                    sigmoid2_nl2(fma2(load_pair(us + (i * 3 + 2) * kRecCJ + cj), f2(kNegLog2e), p.nbr));
+                A = mul2(A, f);
+                Bg = mul2(f, fma2(load_pair(dhs + i * kRecCJ + cj), rr, Bg));
             }
         }
-    } else {
-    #pragma unroll 1
-        for (int qq = 0; qq < kScanSub; ++qq) {
-            const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
-            if (sub_bits(valid_all, q) == 0u) continue;
-            const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
-            const float* xs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES);
-            const float* dhs = xs + kChunkT * kRecCJ;
-            float2 c = s_ck[q * 32];
-            float2 cp[kChunkT], fs[kChunkT], rs[kChunkT];
-    #pragma unroll
-            for (int r = 0; r < kChunkT; ++r) {
-                const int i = DIR == 0 ? r : kChunkT - 1 - r;
-                cp[i] = c;
-                fs[i] = f2(0.f);
-                rs[i] = f2(0.f);
-                if ((sub_bits(valid_all, q) >> i) & 1u)
-                    c = sru_cell2(c, load_pair(us + (i * 3 + 0) * kRecCJ + cj), load_pair(us + (i * 3 + 1) * kRecCJ + cj),
-                                  load_pair(us + (i * 3 + 2) * kRecCJ + cj), p, fs[i], rs[i]);
-            }
-    #pragma unroll
-            for (int r = 0; r < kChunkT; ++r) {
-                const int i = DIR == 0 ? kChunkT - 1 - r : r;
-                if (!((sub_bits(valid_all, q) >> i) & 1u)) continue;
-                const float2 f = fs[i], rr = rs[i];
-                const float2 uc = load_pair(us + (i * 3 + 0) * kRecCJ + cj);
-                const float2 ax = mul2(alpha2, load_pair(xs + i * kRecCJ + cj));
-                const float2 dhv = load_pair(dhs + i * kRecCJ + cj);
-                const float2 cmu = sub2(cp[i], uc);
-                const float2 cn = fma2(f, cmu, uc);
-                const float2 dzr = mul2(mul2(dhv, sub2(cn, ax)), mul2(rr, sub2(f2(1.f), rr)));
-                const float2 a = fma2(mul2(cmu, mul2(f, sub2(f2(1.f), f))), p.vf, f);
-                const float2 bb = fma2(dzr, p.vr, mul2(a, mul2(dhv, rr)));
-                A = mul2(a, A);
-                Bg = fma2(a, Bg, bb);
-            }
+    } else if (valid != 0u) {
+        float2 c = ck;
+        float2 cp[kChunkT], fs[kChunkT], rs[kChunkT];
+#pragma unroll
+        for (int r = 0; r < kChunkT; ++r) {
+            const int i = DIR == 0 ? r : kChunkT - 1 - r;
+            cp[i] = c;
+            fs[i] = f2(0.f);
+            rs[i] = f2(0.f);
+            if ((valid >> i) & 1u)
+                c = sru_cell2(c, load_pair(us + (i * 3 + 0) * kRecCJ + cj), load_pair(us + (i * 3 + 1) * kRecCJ + cj),
+                              load_pair(us + (i * 3 + 2) * kRecCJ + cj), p, fs[i], rs[i]);
+        }
+#pragma unroll
+        for (int r = 0; r < kChunkT; ++r) {
+            const int i = DIR == 0 ? kChunkT - 1 - r : r;
+            if (!((valid >> i) & 1u)) continue;
+            const float2 f = fs[i], rr = rs[i];
+            const float2 uc = load_pair(us + (i * 3 + 0) * kRecCJ + cj);
+            const float2 ax = mul2(alpha2, load_pair(xs + i * kRecCJ + cj));
+            const float2 dhv = load_pair(dhs + i * kRecCJ + cj);
+            const float2 cmu = sub2(cp[i], uc);
+            const float2 cn = fma2(f, cmu, uc);
+            const float2 dzr = mul2(mul2(dhv, sub2(cn, ax)), mul2(rr, sub2(f2(1.f), rr)));
+            const float2 a = fma2(mul2(cmu, mul2(f, sub2(f2(1.f), f))), p.vf, f);
+            const float2 bb = fma2(dzr, p.vr, mul2(a, mul2(dhv, rr)));
+            A = mul2(a, A);
+            Bg = fma2(a, Bg, bb);
         }
     }
-    // 2. state gradient entering the chunk (from later times)
+    s_map[q * 32 + lane] = make_float4(A.x, A.y, Bg.x, Bg.y);
+    __syncthreads();
+    // item map and the map of the sub-chunks walked before this one (backward walk order)
+    float2 Ai = f2(1.f), Bi = f2(0.f), Ab = f2(1.f), Bb = f2(0.f);
+#pragma unroll
+    for (int qq = 0; qq < kScanSub; ++qq) {
+        const int qs = DIR == 0 ? kScanSub - 1 - qq : qq;
+        if (qs == q) {
+            Ab = Ai;
+            Bb = Bi;
+        }
+        const float4 m = s_map[qs * 32 + lane];
+        compose_after(Ai, Bi, make_float2(m.x, m.y), make_float2(m.z, m.w));
+    }
+    // 2. state gradient entering the item (from later times)
     float2 g_in = f2(0.f);
     const size_t me = (size_t)w * kRecCJ + cj;
     if (k == 0) {
         g_in = (jok && dc_T != nullptr) ? load_pair(dc_T + (size_t)bd * d + j) : f2(0.f);
     } else {
-        store_pair(ss.agg_a + me, A);
-        store_pair(ss.agg_b + me, Bg);
+        if (q == 0) {
+            store_pair(ss.agg_a + me, Ai);
+            store_pair(ss.agg_b + me, Bi);
+        }
         scan_publish(&ss.flags[w], kFlagAgg);
         if (!scan_lookback(ss, k, tile, n_tiles, cj, s_misc + 1, g_in)) {
             scan_publish(&ss.flags[w], kFlagAbort);
@@ -442,37 +426,43 @@ __global__ void __launch_bounds__(kRecThreads) sru_bwd_scan_kernel(
         }
     }
     if (w == ss.withhold) return;  // successors' waits expire (test hook)
-    store_pair(ss.prefix + me, fma2(A, g_in, Bg));
+    if (q == 0) store_pair(ss.prefix + me, fma2(Ai, g_in, Bi));
     scan_publish(&ss.flags[w], kFlagPrefix);
 
-    // 3. gradients of every row, sub-chunk by sub-chunk in backward order
-    float2 g = g_in;
-    SmemPartials acc{reinterpret_cast<double*>(smem + Lay::ACC_OFF) + lane, kRecThreads};
+    // 3. gradients of this sub-chunk's rows from the state gradient entering it
+    float2 g = fma2(Ab, g_in, Bb);
+    SmemPartials acc{reinterpret_cast<double*>(smem + Lay::ACC_OFF) + tid, kScanThreads};
 #pragma unroll
-    for (int q = 0; q < 8; ++q) acc.p[q * acc.n] = 0.0;  // read and written by this thread only
-    const size_t u_tstride = (size_t)B * n_dir * 3 * d;
-    const size_t x_tstride = (size_t)B * d;
-#pragma unroll 1
-    for (int qq = 0; qq < kScanSub; ++qq) {
-        const int q = DIR == 0 ? kScanSub - 1 - qq : qq;
-        const int ts = t0 + q * kChunkT;
-        if (ts >= L) continue;
+    for (int i = 0; i < 8; ++i) acc.p[i * acc.n] = 0.0;  // read and written by this thread only
+    if (ts < L) {
+        const size_t u_tstride = (size_t)B * n_dir * 3 * d;
+        const size_t x_tstride = (size_t)B * d;
         DUT* dUp = dU + (size_t)ts * u_tstride + (size_t)bd * 3 * d + j;
         float* dxp = dx + (size_t)ts * x_tstride + (size_t)b * d + j;
-        if (sub_bits(valid_all, q) == 0u) {
-            bwd_chunk_padded<DUT, ACC_DX>(sub_bits(inrange_all, q), dUp, dxp, u_tstride, x_tstride, d, jok);
-            continue;
-        }
-        const UT* us = reinterpret_cast<const UT*>(smem + q * SL::STAGE);
-        const float* xs = reinterpret_cast<const float*>(smem + q * SL::STAGE + SL::U_BYTES);
-        const float* dhs = xs + kChunkT * kRecCJ;
-        bwd_chunk<UT, DUT, ACC_DX, DIR, kRecCJ>(us, xs, dhs, sub_bits(valid_all, q), sub_bits(inrange_all, q),
-                                                s_ck[q * 32], p, alpha2, g, acc, dUp, dxp, u_tstride, x_tstride, d,
-                                                jok, cj);
+        if (valid == 0u)
+            bwd_chunk_padded<DUT, ACC_DX>(inrange, dUp, dxp, u_tstride, x_tstride, d, jok);
+        else
+            bwd_chunk<UT, DUT, ACC_DX, DIR, kRecCJ>(us, xs, dhs, valid, inrange, ck, p, alpha2, g, acc, dUp, dxp,
+                                                    u_tstride, x_tstride, d, jok, cj);
     }
-    if (jok) {
-        if (k == nchs - 1) store_pair(dc0 + (size_t)bd * d + j, g);
-        store_partials(partial + (((size_t)tc * B + b) * n_dir + DIR) * 4 * d + j, acc, d);
+    // the last sub-chunk in walk order leaves dc0
+    const bool last = DIR == 0 ? q == 0 : (ts + kChunkT >= L || q == kScanSub - 1);
+    if (k == nchs - 1 && last && ts < L && jok) store_pair(dc0 + (size_t)bd * d + j, g);
+    // the item's dv/db partial sums: the four warps' totals in sub-chunk order
+    __syncthreads();
+    if (q == 0 && jok) {
+        const double* base = reinterpret_cast<const double*>(smem + Lay::ACC_OFF);
+        double* pp = partial + (((size_t)tc * B + b) * n_dir + DIR) * 4 * d + j;
+#pragma unroll
+        for (int t4 = 0; t4 < 4; ++t4) {
+            double sx = 0.0, sy = 0.0;
+#pragma unroll
+            for (int qq = 0; qq < kScanSub; ++qq) {
+                sx += base[(2 * t4) * kScanThreads + qq * 32 + lane];
+                sy += base[(2 * t4 + 1) * kScanThreads + qq * 32 + lane];
+            }
+            *reinterpret_cast<double2*>(pp + (size_t)t4 * d) = make_double2(sx, sy);
+        }
     }
 }
 

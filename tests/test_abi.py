@@ -141,3 +141,33 @@ def test_per_channel_vectors_must_be_pair_aligned(lib):
         args = [fake, 1, fake, fake, fake, None, 4, 2, 64, 1.0, 0, fake, fake, None]
         args[pos] = odd
         assert lib.sru_forward_scan_noalloc(*args) == 1, pos
+
+
+def test_attention_backward_checks_arguments_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)
+    L, B, d, dp, N = 64, 2, 128, 32, 384
+    fneed = lib.sru_attention_workspace_bytes(L, B, dp)
+    need = lib.sru_attention_backward_workspace_bytes(L, B, d, dp, N)
+    # per group: scores or their gradient (fp32), P and dS (bf16) of each batch row
+    assert need >= B * L * L * 8 + L * B * dp * (4 + 4 + 2 + 4 + 2)
+    assert lib.sru_attention_backward_workspace_bytes(60, B, d, dp, N) == 0      # L % 8 != 0
+    assert lib.sru_attention_backward_workspace_bytes(L, B, d, 12, N) == 0       # d' % 8 != 0
+    assert lib.sru_attention_backward_workspace_bytes(L, B, 100, dp, N) == 0     # d % 8 != 0
+
+    def call(**kw):
+        a = dict(dU=fake, X=fake, Wq=fake, Wkv=fake, Wo=fake, alpha=0.5, g=None, b=None, causal=1, fws=fake,
+                 fwsb=fneed, dX=fake, acc=0, dWq=fake, dWkv=fake, dWo=fake, dg=None, db=None, L=L, B=B, d=d, dp=dp,
+                 N=N, ws=fake, wsb=need, st=None)
+        a.update(kw)
+        return lib.sru_attention_project_backward(*a.values())
+
+    assert call(dU=None) == 1                       # null input
+    assert call(dWkv=None) == 1                     # null output
+    assert call(dX=vp(0x1008)) == 1                 # misaligned output
+    assert call(fwsb=fneed - 256) == 1              # short forward workspace
+    assert call(wsb=need - 256) == 1                # short workspace
+    assert call(g=fake) == 1                        # gamma without beta
+    assert call(g=fake, b=fake) == 1                # the norm without its gradient outputs
+    assert call(d=100) == 4                         # d % 8 != 0
+    assert call(L=0) == 1                           # no tokens

@@ -46,7 +46,8 @@ def _check(name, got, ref, tol):
     assert not bad.any(), f"{name}: {bad.sum()} of {bad.size} beyond tolerance, worst {np.max(err - tol):.3g}"
 
 
-@pytest.mark.parametrize("M,K,Kp,N", [(111, 256, 64, 768), (256, 2048, 512, 6144), (9, 64, 16, 192)])
+@pytest.mark.parametrize("M,K,Kp,N", [(111, 256, 64, 768), (256, 2048, 512, 6144), (9, 64, 16, 192),
+                                       (4100, 512, 128, 1536)])  # few output tiles, long reduction: split
 def test_factored_projection_and_gradients(sru, M, K, Kp, N):
     rng = np.random.default_rng(M + K)
     Xb = _bits(rng, (M, K), 1.0)
@@ -111,3 +112,28 @@ def test_factored_equals_two_plain_projections(sru):
     assert sru.sru_sync_status() == 0
     assert torch.equal(P1.view(torch.int16), P2.view(torch.int16))
     assert torch.equal(U1.view(torch.int16), U2.view(torch.int16))
+
+
+def test_split_weight_gradients_are_deterministic_and_match_the_single_product(sru):
+    """dWq and dWo of a narrow d' over many tokens are cut along the tokens
+    into workspace slabs summed in a fixed order: the same bits on every run,
+    and the single product (no workspace) within fp32 summation-order error."""
+    rng = np.random.default_rng(5)
+    M, K, Kp, N = 8192, 256, 64, 768
+    Xd, Wqd, Wod = _dev(_bits(rng, (M, K), 1.0)), _dev(_bits(rng, (Kp, K), 0.06)), _dev(_bits(rng, (N, Kp), 0.1))
+    dUd = _dev(_bits(rng, (M, N), 1.0))
+    P = torch.empty(M, Kp, device="cuda", dtype=torch.bfloat16)
+    sru.sru_project_factored(Xd, Wqd, Wod, P, torch.empty(M, N, device="cuda", dtype=torch.bfloat16))
+    runs = []
+    for ws in (None, None, torch.empty(0, dtype=torch.uint8, device="cuda")):
+        dP = torch.empty(M, Kp, device="cuda", dtype=torch.bfloat16)
+        dWq, dWo = torch.empty(Kp, K, device="cuda"), torch.empty(N, Kp, device="cuda")
+        sru.sru_project_factored_backward(dUd, Xd, Wqd, Wod, P, dP, dWq=dWq, dWo=dWo, workspace=ws)
+        assert sru.sru_sync_status() == 0
+        runs.append((dWq, dWo))
+    assert sru.load_library().sru_project_factored_backward_workspace_bytes(M, N, K, Kp) > 0
+    for a, b in zip(runs[0], runs[1]):
+        assert torch.equal(a, b)
+    for a, b in zip(runs[0], runs[2]):
+        scale = b.abs().max().item()
+        assert (a - b).abs().max().item() <= 1e-5 * scale * 8
