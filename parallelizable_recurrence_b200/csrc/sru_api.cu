@@ -1344,9 +1344,9 @@ static int64_t attn_bwd_group(int64_t L, int64_t B) {
     const int64_t g = (int64_t)(kAttnGroupBytes / ((size_t)L * L * 8));
     return g < 1 ? 1 : (g > B ? B : g);
 }
-constexpr int kNormSlices = 128;  // row slices of the norm's parameter-gradient sums
 struct AttnBwdWs {
-    size_t dr, dq, da, dkv, dqb, s, p, ds, stats, part, split, split_bytes, total;
+    size_t dr, dq, dqa, da, dkv, dqb, s, p, ds, stats, part, split, split_bytes, total;
+    bool fwd_p;  // the forward's workspace holds every batch row's probabilities (one group)
 };
 static AttnBwdWs attn_bwd_ws(int64_t L, int64_t B, int64_t d, int64_t dp, int64_t N) {
     AttnBwdWs w{};
@@ -1354,17 +1354,19 @@ static AttnBwdWs attn_bwd_ws(int64_t L, int64_t B, int64_t d, int64_t dp, int64_
     // slabs of the split-K weight gradients dWo (N x d'), dWkv (2d' x d'), dWq (d' x d)
     w.split_bytes = std::max(split_plan(N, dp, M).bytes, std::max(split_plan(2 * dp, dp, M).bytes,
                                                                   split_plan(dp, d, M).bytes));
+    w.fwd_p = attn_group(L, B) >= B;
     size_t off = 0;
     w.dr = off;    off += round256((size_t)M * dp * 4);
     w.dq = off;    off += round256((size_t)M * dp * 4);
+    w.dqa = off;   off += round256((size_t)M * dp * 4);
     w.da = off;    off += round256((size_t)M * dp * 2);
     w.dkv = off;   off += round256((size_t)M * 2 * dp * 2);
     w.dqb = off;   off += round256((size_t)M * dp * 2);
     w.s = off;     off += round256((size_t)G * L * L * 4);
-    w.p = off;     off += round256((size_t)G * L * L * 2);
+    w.p = off;     off += w.fwd_p ? 0 : round256((size_t)G * L * L * 2);
     w.ds = off;    off += round256((size_t)G * L * L * 2);
     w.stats = off; off += round256((size_t)M * 8);
-    w.part = off;  off += round256((size_t)kNormSlices * 2 * dp * 4);
+    w.part = off;  off += round256((size_t)((M + sru::kNormRows - 1) / sru::kNormRows) * 2 * dp * 4);
     w.split = off; off += round256(w.split_bytes);
     w.total = off;
     return w;
@@ -1409,11 +1411,14 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* dR = reinterpret_cast<float*>(ws + w.dr);
     float* dQ = reinterpret_cast<float*>(ws + w.dq);
+    float* dQa = reinterpret_cast<float*>(ws + w.dqa);
     __nv_bfloat16* dA = reinterpret_cast<__nv_bfloat16*>(ws + w.da);
     __nv_bfloat16* dKV = reinterpret_cast<__nv_bfloat16*>(ws + w.dkv);
     __nv_bfloat16* dQb = reinterpret_cast<__nv_bfloat16*>(ws + w.dqb);
     float* S = reinterpret_cast<float*>(ws + w.s);
-    __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(ws + w.p);
+    // with one group the forward's probabilities of every batch row are still in its workspace
+    const __nv_bfloat16* Pf = reinterpret_cast<const __nv_bfloat16*>(fws + fw.p);
+    __nv_bfloat16* P = w.fwd_p ? nullptr : reinterpret_cast<__nv_bfloat16*>(ws + w.p);
     __nv_bfloat16* dS = reinterpret_cast<__nv_bfloat16*>(ws + w.ds);
     float2* stats = reinterpret_cast<float2*>(ws + w.stats);
     float* part = reinterpret_cast<float*>(ws + w.part);
@@ -1429,13 +1434,15 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
         dR, Q, A, alpha, ln_gamma, dQ, dA, stats, (int)M, (int)dp);
     SRU_CUDA_TRY(cudaGetLastError());
     if (norm) {
-        const int rows_per = (int)((M + kNormSlices - 1) / kNormSlices);
-        const dim3 grid(blocks_for((size_t)dp, sru::kNormParamThreads), (unsigned)((M + rows_per - 1) / rows_per));
+        const unsigned slices = (unsigned)((M + sru::kNormRows - 1) / sru::kNormRows);
+        if (slices > 65535u) return SRU_ERR_UNSUPPORTED;
+        const dim3 grid(blocks_for((size_t)dp, sru::kNormParamThreads), slices);
         sru::sru_norm_param_partial_kernel<<<grid, sru::kNormParamThreads, 0, st>>>(dR, Q, A, alpha, stats, part,
-                                                                                   (int)M, (int)dp, rows_per);
+                                                                                   (int)M, (int)dp);
         SRU_CUDA_TRY(cudaGetLastError());
-        sru::sru_norm_param_reduce_kernel<<<blocks_for((size_t)dp, 256), 256, 0, st>>>(part, (int)grid.y, (int)dp,
-                                                                                       dgamma, dbeta);
+        sru::sru_norm_param_reduce_kernel<<<blocks_for((size_t)(2 * dp), sru::kNormRedCols),
+                                            sru::kNormRedCols * sru::kNormRedGroups, 0, st>>>(part, (int)slices,
+                                                                                            (int)dp, dgamma, dbeta);
         SRU_CUDA_TRY(cudaGetLastError());
     }
     const float scale = 1.0f / sqrtf((float)dp);
@@ -1444,16 +1451,22 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
     for (int64_t b0 = 0; b0 < B; b0 += G) {
         const int64_t g = B - b0 < G ? B - b0 : G;
         CUtensorMap ma, mb;
-        // the forward's probabilities of this group: S = Q K^T, softmax
-        if (!map_kmajor_b(&ma, Q + b0 * dp, L, dp, B * dp, g, dp, sru::gemm::P_CM, 1) ||
-            !map_kmajor_b(&mb, KV + b0 * 2 * dp, L, dp, B * 2 * dp, g, 2 * dp, kGemmBRows, 1))
-            return SRU_ERR_INVALID;
-        s = causal ? launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st)
-                   : launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st);
-        if (s != SRU_OK) return s;
-        sru::sru_softmax_rows_kernel<<<blocks_for((size_t)(g * L), sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
-            S, P, (int)L, (int)(g * L), scale, causal ? 1 : 0);
-        SRU_CUDA_TRY(cudaGetLastError());
+        // the forward's probabilities of this group: still in the forward's workspace
+        // (one group there), else recomputed: S = Q K^T, softmax
+        const __nv_bfloat16* Pg = w.fwd_p ? Pf + b0 * L * L : P;
+        if (!w.fwd_p) {
+            if (!map_kmajor_b(&ma, Q + b0 * dp, L, dp, B * dp, g, dp, sru::gemm::P_CM, 1) ||
+                !map_kmajor_b(&mb, KV + b0 * 2 * dp, L, dp, B * 2 * dp, g, 2 * dp, kGemmBRows, 1))
+                return SRU_ERR_INVALID;
+            s = causal ? launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1, 1>(ma, mb, S, L, L, dp, L, g,
+                                                                                          L * L, st)
+                       : launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g,
+                                                                                       L * L, st);
+            if (s != SRU_OK) return s;
+            sru::sru_softmax_rows_kernel<<<blocks_for((size_t)(g * L), sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+                S, P, (int)L, (int)(g * L), scale, causal ? 1 : 0);
+            SRU_CUDA_TRY(cudaGetLastError());
+        }
         // dP = dA V^T (into S), then dS
         if (!map_kmajor_b(&ma, dA + b0 * dp, L, dp, B * dp, g, dp, sru::gemm::P_CM, 1) ||
             !map_kmajor_b(&mb, KV + b0 * 2 * dp + dp, L, dp, B * 2 * dp, g, 2 * dp, kGemmBRows, 1))
@@ -1462,13 +1475,13 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
                    : launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st);
         if (s != SRU_OK) return s;
         sru::sru_softmax_backward_rows_kernel<<<blocks_for((size_t)(g * L), sru::kRowWarps), sru::kRowWarps * 32, 0,
-                                                st>>>(S, P, dS, (int)L, (int)(g * L), scale, causal ? 1 : 0);
+                                                st>>>(S, Pg, dS, (int)L, (int)(g * L), scale, causal ? 1 : 0);
         SRU_CUDA_TRY(cudaGetLastError());
         // dV = P^T dA and dK = dS^T Q (bf16, into [dK | dV]): the first operand read
         // MN-major (element (s, t) of batch z at z L^2 + t L + s), the second too
         // (element (j, t) at (t B + b0 + z) d' + j)
         __nv_bfloat16* dK0 = dKV + b0 * 2 * dp;
-        if (!map_mnmajor_b(&ma, P, L, L, L, g, L * L, 2) || !map_mnmajor_b(&mb, dA + b0 * dp, dp, L, B * dp, g, dp, 1))
+        if (!map_mnmajor_b(&ma, Pg, L, L, L, g, L * L, 2) || !map_mnmajor_b(&mb, dA + b0 * dp, dp, L, B * dp, g, dp, 1))
             return SRU_ERR_INVALID;
         s = causal ? launch_tc_gemm_batched<true, true, sru::gemm::kOutBF16, 2, 1, 3>(ma, mb, dK0 + dp, L, dp, L,
                                                                                      B * 2 * dp, g, 2 * dp, st)
@@ -1482,14 +1495,15 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
                    : launch_tc_gemm_batched<true, true, sru::gemm::kOutBF16, 2, 1>(ma, mb, dK0, L, dp, L, B * 2 * dp,
                                                                                   g, 2 * dp, st);
         if (s != SRU_OK) return s;
-        // dQ += dS K: dS K-major over s; K (c = j, red = s) at KV[(s B + b0 + z) 2d' + j]: MN-major
+        // dS K (into dQa, added to dQ below): dS K-major over s; K (c = j, red = s) at
+        // KV[(s B + b0 + z) 2d' + j]: MN-major
         if (!map_kmajor_b(&ma, dS, L, L, L, g, L * L, sru::gemm::P_CM, 2) ||
             !map_mnmajor_b(&mb, KV + b0 * 2 * dp, dp, L, B * 2 * dp, g, 2 * dp, 1))
             return SRU_ERR_INVALID;
-        s = causal ? launch_tc_gemm_batched<false, true, sru::gemm::kOutF32Acc, 2, 1, 2>(ma, mb, dQ + b0 * dp, L, dp, L,
-                                                                                        B * dp, g, dp, st)
-                   : launch_tc_gemm_batched<false, true, sru::gemm::kOutF32Acc, 2, 1>(ma, mb, dQ + b0 * dp, L, dp, L,
-                                                                                     B * dp, g, dp, st);
+        s = causal ? launch_tc_gemm_batched<false, true, sru::gemm::kOutF32, 2, 1, 2>(ma, mb, dQa + b0 * dp, L, dp, L,
+                                                                                     B * dp, g, dp, st)
+                   : launch_tc_gemm_batched<false, true, sru::gemm::kOutF32, 2, 1>(ma, mb, dQa + b0 * dp, L, dp, L,
+                                                                                  B * dp, g, dp, st);
         if (s != SRU_OK) return s;
     }
     // [K | V] = Q Wkv^T:  dQ += [dK | dV] Wkv,  dWkv = [dK | dV]^T Q
@@ -1497,10 +1511,12 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
     if (s != SRU_OK) return s;
     s = project_dW_split(dKV, Q, dWkv, M, 2 * dp, dp, split, w.split_bytes, st);
     if (s != SRU_OK) return s;
-    // Q = X Wq^T:  dWq = dQ^T X,  dX (+)= dQ Wq  (dQ rounded to bf16 as the products' operand)
+    // Q = X Wq^T:  dWq = dQ^T X,  dX (+)= dQ Wq  (dQ = dZ + [dK | dV] Wkv + dS K rounded to
+    // bf16 as the products' operand)
     const size_t n4 = (size_t)M * dp / 4;
-    sru::sru_f32_to_bf16_kernel<<<(unsigned)std::min<size_t>(blocks_for(n4, 256), (size_t)sm_count() * 8), 256, 0,
-                                  st>>>(reinterpret_cast<const float4*>(dQ), reinterpret_cast<uint2*>(dQb), n4);
+    sru::sru_add_to_bf16_kernel<<<(unsigned)std::min<size_t>(blocks_for(n4, 256), (size_t)sm_count() * 8), 256, 0,
+                                  st>>>(reinterpret_cast<const float4*>(dQ), reinterpret_cast<const float4*>(dQa),
+                                        reinterpret_cast<uint2*>(dQb), n4);
     SRU_CUDA_TRY(cudaGetLastError());
     s = sru_project_backward(dQb, X, Wq, SRU_BF16, dX, accumulate, nullptr, M, dp, d, stream);
     if (s != SRU_OK) return s;

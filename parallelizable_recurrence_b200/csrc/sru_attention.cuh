@@ -167,15 +167,16 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_kernel(
 }
 
 // The norm's parameter gradients, first stage: slice y of the rows (rows
-// [y * rows_per, (y + 1) * rows_per)) summed per feature j in fp32, in row
+// [y * kNormRows, (y + 1) * kNormRows)) summed per feature j in fp32, in row
 // order, into part[y][0][j] (dgamma: dR * Zhat) and part[y][1][j] (dbeta: dR).
+constexpr int kNormRows = 16;
 constexpr int kNormParamThreads = 256;
 __global__ void __launch_bounds__(kNormParamThreads) sru_norm_param_partial_kernel(
     const float* __restrict__ dR, const __nv_bfloat16* __restrict__ Q, const float* __restrict__ A, float alpha,
-    const float2* __restrict__ stats, float* __restrict__ part, int M, int dp, int rows_per) {
+    const float2* __restrict__ stats, float* __restrict__ part, int M, int dp) {
     const int j = blockIdx.x * kNormParamThreads + threadIdx.x;
     if (j >= dp) return;
-    const int m0 = blockIdx.y * rows_per, m1 = min(M, m0 + rows_per);
+    const int m0 = blockIdx.y * kNormRows, m1 = min(M, m0 + kNormRows);
     float sg = 0.f, sb = 0.f;
     for (int m = m0; m < m1; ++m) {
         const size_t e = (size_t)m * dp + j;
@@ -188,27 +189,38 @@ __global__ void __launch_bounds__(kNormParamThreads) sru_norm_param_partial_kern
     part[((size_t)blockIdx.y * 2 + 1) * dp + j] = sb;
 }
 
-// Second stage: the slices' partial sums per feature in slice order, in fp64.
-__global__ void __launch_bounds__(256) sru_norm_param_reduce_kernel(const float* __restrict__ part, int slices, int dp,
-                                                                    float* __restrict__ dgamma,
-                                                                    float* __restrict__ dbeta) {
-    const int j = blockIdx.x * 256 + threadIdx.x;
-    if (j >= dp) return;
-    double sg = 0.0, sb = 0.0;
-    for (int y = 0; y < slices; ++y) {
-        sg += (double)part[((size_t)y * 2 + 0) * dp + j];
-        sb += (double)part[((size_t)y * 2 + 1) * dp + j];
-    }
-    dgamma[j] = (float)sg;
-    dbeta[j] = (float)sb;
+// Second stage: column c of the slices' partial sums (c < d': dgamma, else
+// dbeta), in fp64.  A block owns kNormRedCols columns; its kNormRedGroups
+// thread groups each sum slices g, g + kNormRedGroups, ... in increasing
+// order, and the groups are then added in increasing order: a fixed order,
+// so the result is the same on every run.
+constexpr int kNormRedCols = 32, kNormRedGroups = 8;
+__global__ void __launch_bounds__(kNormRedCols * kNormRedGroups) sru_norm_param_reduce_kernel(
+    const float* __restrict__ part, int slices, int dp, float* __restrict__ dgamma, float* __restrict__ dbeta) {
+    __shared__ double acc[kNormRedGroups][kNormRedCols];
+    const int col = threadIdx.x % kNormRedCols, grp = threadIdx.x / kNormRedCols;
+    const int c = blockIdx.x * kNormRedCols + col;
+    double sum = 0.0;
+    if (c < 2 * dp)
+        for (int y = grp; y < slices; y += kNormRedGroups) sum += (double)part[(size_t)y * 2 * dp + c];
+    acc[grp][col] = sum;
+    __syncthreads();
+    if (grp != 0 || c >= 2 * dp) return;
+    double t = 0.0;
+#pragma unroll
+    for (int k = 0; k < kNormRedGroups; ++k) t += acc[k][col];
+    if (c < dp)
+        dgamma[c] = (float)t;
+    else
+        dbeta[c - dp] = (float)t;
 }
 
-// out[i] = bf16(in[i]), four at a time (n a multiple of 4, both 16-byte aligned).
-__global__ void __launch_bounds__(256) sru_f32_to_bf16_kernel(const float4* __restrict__ in,
+// out[i] = bf16(a[i] + b[i]), four at a time (n a multiple of 4, all 16-byte aligned).
+__global__ void __launch_bounds__(256) sru_add_to_bf16_kernel(const float4* __restrict__ a, const float4* __restrict__ b,
                                                               uint2* __restrict__ out, size_t n4) {
     for (size_t i = blockIdx.x * (size_t)256 + threadIdx.x; i < n4; i += (size_t)gridDim.x * 256) {
-        const float4 v = in[i];
-        __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+        const float4 u = a[i], v = b[i];
+        __nv_bfloat162 lo = __floats2bfloat162_rn(u.x + v.x, u.y + v.y), hi = __floats2bfloat162_rn(u.z + v.z, u.w + v.w);
         out[i] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
     }
 }

@@ -42,6 +42,7 @@ def _dev(bits):
     (4096, 3, 64, 16, 0.5, True, False),   # long rows: batch rows go in groups of 2 (score buffer bound)
     (600, 2, 128, 32, 0.5, True, True),    # causal over 3 score tiles, the last one ragged
     (600, 2, 128, 32, 0.5, False, False),  # the same without the mask: every tile computed
+    (72, 3, 96, 40, 0.9, True, True),      # widths that are not multiples of a tile or a k-block
 ])
 def test_attention_producer_matches_oracle(sru, L, B, d, dp, alpha, causal, ln):
     rng = np.random.default_rng(L + B + d + dp)

@@ -96,7 +96,9 @@ def _compare(out, ref):
     (256, 3, 128, 64, 0.25, True, False),    # one full score tile
     (600, 2, 128, 32, 0.5, True, True),      # causal over 3 score tiles, the last one ragged
     (600, 2, 128, 32, -0.7, False, False),   # the same without the mask: every tile computed
-    (2048, 5, 64, 16, 0.5, True, False),     # long rows: batch rows go in groups of 2 (score buffer bound)
+    (2048, 5, 64, 16, 0.5, True, False),     # every batch row's probabilities kept by the forward (one group)
+    (4096, 3, 64, 16, 0.5, True, True),      # long rows in groups of 2: the probabilities are recomputed
+    (72, 3, 96, 40, 0.9, True, True),        # widths that are not multiples of a tile or a k-block
 ])
 def test_attention_backward_matches_oracle(sru, L, B, d, dp, alpha, causal, ln):
     out, ref = _run(sru, L, B, d, dp, alpha, causal, ln, seed=L + B + d + dp)
