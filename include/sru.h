@@ -268,7 +268,8 @@ sru_status sru_project_factored_backward(const void* dU, const void* X, const vo
  *   R = Q + alpha A, or layernorm(Q + alpha A) * gamma + beta over the d' features
  *       (eps 1e-5) when ln_gamma and ln_beta are given (both or neither)
  *   U = R Wo^T                  (L*B, N)    Wo  (N, d'), U of type u_t (BF16 or F32)
- * X, Wq, Wkv, Wo bf16; X and U time-major as everywhere.  Q, [K | V], P and R
+ * X, Wq, Wkv, Wo bf16; X and U time-major as everywhere; ln_gamma and ln_beta
+ * (d',) fp32, 16-byte aligned like every other pointer.  Q, [K | V], P and R
  * are rounded to bf16 (they are tensor-core operands), scores and A are fp32.
  * The workspace (>= sru_attention_workspace_bytes(L, B, d')) holds Q, K, V,
  * one batch row's scores and probabilities, A and R.  Limits: d, d', N and L

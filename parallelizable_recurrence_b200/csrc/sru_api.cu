@@ -777,6 +777,66 @@ int64_t fused_resident_pairs() {
 }  // namespace
 
 // =========================================================================
+template <int NV>
+void norm_backward_reg(const float* dR, const __nv_bfloat16* Q, const float* A, float alpha, const float* g, float* dQ,
+                       __nv_bfloat16* dA, float2* stats, int64_t M, int64_t dp, cudaStream_t st) {
+    sru::sru_norm_backward_reg_kernel<NV><<<blocks_for((size_t)M, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+        dR, Q, A, alpha, g, dQ, dA, stats, (int)M, (int)dp);
+}
+sru_status launch_norm_backward(const float* dR, const __nv_bfloat16* Q, const float* A, float alpha, const float* g,
+                                float* dQ, __nv_bfloat16* dA, float2* stats, int64_t M, int64_t dp, cudaStream_t st) {
+    const int64_t nv = (dp + 127) / 128;
+    if (nv <= 1) norm_backward_reg<1>(dR, Q, A, alpha, g, dQ, dA, stats, M, dp, st);
+    else if (nv <= 2) norm_backward_reg<2>(dR, Q, A, alpha, g, dQ, dA, stats, M, dp, st);
+    else if (nv <= 4) norm_backward_reg<4>(dR, Q, A, alpha, g, dQ, dA, stats, M, dp, st);
+    else if (nv <= 8) norm_backward_reg<8>(dR, Q, A, alpha, g, dQ, dA, stats, M, dp, st);
+    else
+        sru::sru_norm_backward_kernel<<<blocks_for((size_t)M, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+            dR, Q, A, alpha, g, dQ, dA, stats, (int)M, (int)dp);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+// The row-wise steps: the register-resident kernels for rows that fit (scores
+// rows of L <= 2048, d' <= 1024), the streaming ones otherwise.
+template <int NV>
+void softmax_reg(const float* S, __nv_bfloat16* P, int64_t L, int64_t rows, float scale, int causal, cudaStream_t st) {
+    sru::sru_softmax_rows_reg_kernel<NV><<<blocks_for((size_t)rows, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+        S, P, (int)L, (int)rows, scale, causal);
+}
+sru_status launch_softmax_rows(const float* S, __nv_bfloat16* P, int64_t L, int64_t rows, float scale, int causal,
+                               cudaStream_t st) {
+    const int64_t nv = (L + 127) / 128;
+    if (nv <= 1) softmax_reg<1>(S, P, L, rows, scale, causal, st);
+    else if (nv <= 2) softmax_reg<2>(S, P, L, rows, scale, causal, st);
+    else if (nv <= 4) softmax_reg<4>(S, P, L, rows, scale, causal, st);
+    else if (nv <= 8) softmax_reg<8>(S, P, L, rows, scale, causal, st);
+    else if (nv <= 16) softmax_reg<16>(S, P, L, rows, scale, causal, st);
+    else
+        sru::sru_softmax_rows_kernel<<<blocks_for((size_t)rows, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+            S, P, (int)L, (int)rows, scale, causal);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+template <int NV>
+void residual_norm_reg(const __nv_bfloat16* Q, const float* A, float alpha, const float* g, const float* b,
+                       __nv_bfloat16* R, int64_t M, int64_t dp, cudaStream_t st) {
+    sru::sru_residual_norm_reg_kernel<NV><<<blocks_for((size_t)M, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+        Q, A, alpha, g, b, R, (int)M, (int)dp);
+}
+sru_status launch_residual_norm(const __nv_bfloat16* Q, const float* A, float alpha, const float* g, const float* b,
+                                __nv_bfloat16* R, int64_t M, int64_t dp, cudaStream_t st) {
+    const int64_t nv = (dp + 127) / 128;
+    if (nv <= 1) residual_norm_reg<1>(Q, A, alpha, g, b, R, M, dp, st);
+    else if (nv <= 2) residual_norm_reg<2>(Q, A, alpha, g, b, R, M, dp, st);
+    else if (nv <= 4) residual_norm_reg<4>(Q, A, alpha, g, b, R, M, dp, st);
+    else if (nv <= 8) residual_norm_reg<8>(Q, A, alpha, g, b, R, M, dp, st);
+    else
+        sru::sru_residual_norm_kernel<<<blocks_for((size_t)M, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
+            Q, A, alpha, g, b, R, (int)M, (int)dp);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+
 extern "C" {
 
 const char* sru_status_string(int status) {
@@ -1285,6 +1345,7 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
     if (L < 1 || B < 1 || d < 1 || dp < 1 || N < 1) return SRU_ERR_INVALID;
     if (!X || !Wq || !Wkv || !Wo || !U || !workspace || !aligned16(workspace)) return SRU_ERR_INVALID;
     if ((ln_gamma == nullptr) != (ln_beta == nullptr)) return SRU_ERR_INVALID;
+    if (ln_gamma != nullptr && (!aligned16(ln_gamma) || !aligned16(ln_beta))) return SRU_ERR_INVALID;
     if (u_t != SRU_BF16 && u_t != SRU_F32) return SRU_ERR_INVALID;
     if (d % 8 != 0 || dp % 8 != 0 || N % 8 != 0 || L % 8 != 0) return SRU_ERR_UNSUPPORTED;
     const int64_t M = L * B;
@@ -1317,9 +1378,8 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
         s = causal ? launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st)
                    : launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st);
         if (s != SRU_OK) return s;
-        sru::sru_softmax_rows_kernel<<<blocks_for((size_t)(g * L), sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
-            S, P, (int)L, (int)(g * L), scale, causal ? 1 : 0);
-        SRU_CUDA_TRY(cudaGetLastError());
+        s = launch_softmax_rows(S, P, L, g * L, scale, causal ? 1 : 0, st);
+        if (s != SRU_OK) return s;
         // A_z = P_z V_z: P_z K-major over s (batch outermost); V_z(c = j, red = s) at
         // KV[(s*B + b0 + z)*2d' + d' + j]: MN-major, batch stride 2d'
         if (!map_kmajor_b(&ma, P, L, L, L, g, L * L, sru::gemm::P_CM, 2) ||
@@ -1331,9 +1391,8 @@ sru_status sru_attention_project(const void* X, const void* Wq, const void* Wkv,
                                                                                  g, dp, st);
         if (s != SRU_OK) return s;
     }
-    sru::sru_residual_norm_kernel<<<blocks_for((size_t)M, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
-        Q, A, alpha, ln_gamma, ln_beta, R, (int)M, (int)dp);
-    SRU_CUDA_TRY(cudaGetLastError());
+    s = launch_residual_norm(Q, A, alpha, ln_gamma, ln_beta, R, M, dp, st);
+    if (s != SRU_OK) return s;
     return sru_project(R, SRU_BF16, Wo, SRU_BF16, U, u_t, M, N, dp, stream);
 }
 
@@ -1394,6 +1453,7 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
         !aligned16(workspace))
         return SRU_ERR_INVALID;
     if ((ln_gamma == nullptr) != (ln_beta == nullptr)) return SRU_ERR_INVALID;
+    if (ln_gamma != nullptr && (!aligned16(ln_gamma) || !aligned16(ln_beta))) return SRU_ERR_INVALID;
     const bool norm = ln_gamma != nullptr;
     if (norm && (!dgamma || !dbeta)) return SRU_ERR_INVALID;
     if (d % 8 != 0 || dp % 8 != 0 || N % 8 != 0 || L % 8 != 0) return SRU_ERR_UNSUPPORTED;
@@ -1430,9 +1490,8 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
     s = project_dW_split(dU, R, dWo, M, N, dp, split, w.split_bytes, st);
     if (s != SRU_OK) return s;
     // through the norm (or the identity): dQ = dZ, dA = alpha dZ
-    sru::sru_norm_backward_kernel<<<blocks_for((size_t)M, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
-        dR, Q, A, alpha, ln_gamma, dQ, dA, stats, (int)M, (int)dp);
-    SRU_CUDA_TRY(cudaGetLastError());
+    s = launch_norm_backward(dR, Q, A, alpha, ln_gamma, dQ, dA, stats, M, dp, st);
+    if (s != SRU_OK) return s;
     if (norm) {
         const unsigned slices = (unsigned)((M + sru::kNormRows - 1) / sru::kNormRows);
         if (slices > 65535u) return SRU_ERR_UNSUPPORTED;
@@ -1463,9 +1522,8 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
                        : launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g,
                                                                                        L * L, st);
             if (s != SRU_OK) return s;
-            sru::sru_softmax_rows_kernel<<<blocks_for((size_t)(g * L), sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
-                S, P, (int)L, (int)(g * L), scale, causal ? 1 : 0);
-            SRU_CUDA_TRY(cudaGetLastError());
+            s = launch_softmax_rows(S, P, L, g * L, scale, causal ? 1 : 0, st);
+            if (s != SRU_OK) return s;
         }
         // dP = dA V^T (into S), then dS
         if (!map_kmajor_b(&ma, dA + b0 * dp, L, dp, B * dp, g, dp, sru::gemm::P_CM, 1) ||

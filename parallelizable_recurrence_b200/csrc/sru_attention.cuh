@@ -57,6 +57,119 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_softmax_rows_kernel(const 
         prow[s] = __float2bfloat16_rn(s < n ? expf(srow[s] * scale - m) * inv : 0.f);
 }
 
+// The same softmax with the row held in registers (rows of at most NV * 128
+// scores, read once with 16-byte loads): lane l owns scores 4l .. 4l + 3 of
+// every 128.  When causal, P is written only up to the end of the row's
+// 256-wide tile: the products that read P (P V up to the end of each row
+// tile, P^T dA from each row tile's diagonal on) never read further.
+template <int NV>
+__global__ void __launch_bounds__(kRowWarps * 32) sru_softmax_rows_reg_kernel(const float* __restrict__ S,
+                                                                            __nv_bfloat16* __restrict__ P, int L,
+                                                                            int rows, float scale, int causal) {
+    const int row = blockIdx.x * kRowWarps + threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (row >= rows) return;
+    const int t = row % L;
+    const float4* srow = reinterpret_cast<const float4*>(S + (size_t)row * L);
+    uint2* prow = reinterpret_cast<uint2*>(P + (size_t)row * L);
+    const int n = causal ? t + 1 : L;
+    const int end = causal ? min(L, (t / 256 + 1) * 256) : L;  // written: [0, end)
+    float4 v[NV];
+    float m = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int s0 = k * 128 + lane * 4;
+        v[k] = s0 < n ? srow[s0 / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[k].x = s0 + 0 < n ? v[k].x * scale : -INFINITY;
+        v[k].y = s0 + 1 < n ? v[k].y * scale : -INFINITY;
+        v[k].z = s0 + 2 < n ? v[k].z * scale : -INFINITY;
+        v[k].w = s0 + 3 < n ? v[k].w * scale : -INFINITY;
+        m = fmaxf(m, fmaxf(fmaxf(v[k].x, v[k].y), fmaxf(v[k].z, v[k].w)));
+    }
+    m = warp_max(m);
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        v[k].x = expf(v[k].x - m);
+        v[k].y = expf(v[k].y - m);
+        v[k].z = expf(v[k].z - m);
+        v[k].w = expf(v[k].w - m);
+        sum += (v[k].x + v[k].y) + (v[k].z + v[k].w);
+    }
+    const float inv = 1.0f / warp_sum(sum);
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int s0 = k * 128 + lane * 4;
+        if (s0 >= end) continue;
+        __nv_bfloat162 lo = __floats2bfloat162_rn(v[k].x * inv, v[k].y * inv);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(v[k].z * inv, v[k].w * inv);
+        prow[s0 / 4] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+    }
+}
+
+// The residual and norm with the row held in registers (d' at most NV * 128,
+// read once): lane l owns features 4l .. 4l + 3 of every 128.  gamma and beta
+// are read 16 bytes at a time.
+template <int NV>
+__global__ void __launch_bounds__(kRowWarps * 32) sru_residual_norm_reg_kernel(
+    const __nv_bfloat16* __restrict__ Q, const float* __restrict__ A, float alpha, const float* __restrict__ gamma,
+    const float* __restrict__ beta, __nv_bfloat16* __restrict__ R, int M, int dp) {
+    const int m = blockIdx.x * kRowWarps + threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (m >= M) return;
+    const uint2* q = reinterpret_cast<const uint2*>(Q + (size_t)m * dp);
+    const float4* a = reinterpret_cast<const float4*>(A + (size_t)m * dp);
+    uint2* r = reinterpret_cast<uint2*>(R + (size_t)m * dp);
+    float z[NV][4];
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int j0 = k * 128 + lane * 4;
+        if (j0 < dp) {
+            const uint2 qq = q[j0 / 4];
+            const float4 aa = a[j0 / 4];
+            const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qq.x));
+            const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qq.y));
+            z[k][0] = fmaf(alpha, aa.x, q01.x);
+            z[k][1] = fmaf(alpha, aa.y, q01.y);
+            z[k][2] = fmaf(alpha, aa.z, q23.x);
+            z[k][3] = fmaf(alpha, aa.w, q23.y);
+            sum += z[k][0] + z[k][1] + z[k][2] + z[k][3];
+        } else {
+            z[k][0] = z[k][1] = z[k][2] = z[k][3] = 0.f;
+        }
+    }
+    float mean = 0.f, rstd = 1.f;
+    if (gamma != nullptr) {
+        mean = warp_sum(sum) / (float)dp;
+        float sq = 0.f;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            if (k * 128 + lane * 4 >= dp) continue;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sq = fmaf(z[k][e] - mean, z[k][e] - mean, sq);
+        }
+        rstd = rsqrtf(warp_sum(sq) / (float)dp + kLayerNormEps);
+    }
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int j0 = k * 128 + lane * 4;
+        if (j0 >= dp) continue;
+        float o[4];
+        if (gamma == nullptr) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = z[k][e];
+        } else {
+            const float4 g4 = *reinterpret_cast<const float4*>(gamma + j0);
+            const float4 b4 = *reinterpret_cast<const float4*>(beta + j0);
+            o[0] = fmaf((z[k][0] - mean) * rstd, g4.x, b4.x);
+            o[1] = fmaf((z[k][1] - mean) * rstd, g4.y, b4.y);
+            o[2] = fmaf((z[k][2] - mean) * rstd, g4.z, b4.z);
+            o[3] = fmaf((z[k][3] - mean) * rstd, g4.w, b4.w);
+        }
+        __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]), hi = __floats2bfloat162_rn(o[2], o[3]);
+        r[j0 / 4] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+    }
+}
+
 // R[m][j] = bf16(z) with z = Q[m][j] + alpha * A[m][j], or, with gamma/beta,
 // bf16((z - mean_j z) / sqrt(var_j z + eps) * gamma[j] + beta[j]) over the
 // d' features of row m (two passes for the mean and the variance).
@@ -164,6 +277,91 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_kernel(
         da[j] = __float2bfloat16_rn(alpha * dz);
     }
     if (lane == 0) stats[m] = make_float2(mean, rstd);
+}
+
+// The same gradient with the row held in registers (d' at most NV * 128, each
+// input read once): lane l owns features 4l .. 4l + 3 of every 128.
+template <int NV>
+__global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_reg_kernel(
+    const float* __restrict__ dR, const __nv_bfloat16* __restrict__ Q, const float* __restrict__ A, float alpha,
+    const float* __restrict__ gamma, float* __restrict__ dQ, __nv_bfloat16* __restrict__ dA,
+    float2* __restrict__ stats, int M, int dp) {
+    const int m = blockIdx.x * kRowWarps + threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (m >= M) return;
+    const float4* dr = reinterpret_cast<const float4*>(dR + (size_t)m * dp);
+    float4* dq = reinterpret_cast<float4*>(dQ + (size_t)m * dp);
+    uint2* da = reinterpret_cast<uint2*>(dA + (size_t)m * dp);
+    float g[NV][4], z[NV][4];
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int j0 = k * 128 + lane * 4;
+        if (j0 >= dp) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) g[k][e] = z[k][e] = 0.f;
+            continue;
+        }
+        const float4 r4 = dr[j0 / 4];
+        g[k][0] = r4.x;
+        g[k][1] = r4.y;
+        g[k][2] = r4.z;
+        g[k][3] = r4.w;
+        if (gamma != nullptr) {
+            const uint2 qq = reinterpret_cast<const uint2*>(Q + (size_t)m * dp)[j0 / 4];
+            const float4 aa = reinterpret_cast<const float4*>(A + (size_t)m * dp)[j0 / 4];
+            const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qq.x));
+            const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qq.y));
+            z[k][0] = fmaf(alpha, aa.x, q01.x);
+            z[k][1] = fmaf(alpha, aa.y, q01.y);
+            z[k][2] = fmaf(alpha, aa.z, q23.x);
+            z[k][3] = fmaf(alpha, aa.w, q23.y);
+            sum += z[k][0] + z[k][1] + z[k][2] + z[k][3];
+        }
+    }
+    if (gamma != nullptr) {
+        const float mean = warp_sum(sum) / (float)dp;
+        float sq = 0.f;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            if (k * 128 + lane * 4 >= dp) continue;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sq = fmaf(z[k][e] - mean, z[k][e] - mean, sq);
+        }
+        const float rstd = rsqrtf(warp_sum(sq) / (float)dp + kLayerNormEps);
+        float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            const int j0 = k * 128 + lane * 4;
+            if (j0 >= dp) continue;
+            const float4 g4 = *reinterpret_cast<const float4*>(gamma + j0);
+            const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                z[k][e] = (z[k][e] - mean) * rstd;  // Zhat from here on
+                g[k][e] *= gv[e];                   // dZhat = dR * gamma
+                s1 += g[k][e];
+                s2 = fmaf(g[k][e], z[k][e], s2);
+            }
+        }
+        s1 = warp_sum(s1) / (float)dp;
+        s2 = warp_sum(s2) / (float)dp;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            if (k * 128 + lane * 4 >= dp) continue;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) g[k][e] = rstd * (g[k][e] - s1 - z[k][e] * s2);
+        }
+        if (lane == 0) stats[m] = make_float2(mean, rstd);
+    }
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int j0 = k * 128 + lane * 4;
+        if (j0 >= dp) continue;
+        dq[j0 / 4] = make_float4(g[k][0], g[k][1], g[k][2], g[k][3]);
+        __nv_bfloat162 lo = __floats2bfloat162_rn(alpha * g[k][0], alpha * g[k][1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(alpha * g[k][2], alpha * g[k][3]);
+        da[j0 / 4] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+    }
 }
 
 // The norm's parameter gradients, first stage: slice y of the rows (rows

@@ -169,5 +169,6 @@ def test_attention_backward_checks_arguments_before_any_launch(lib):
     assert call(wsb=need - 256) == 1                # short workspace
     assert call(g=fake) == 1                        # gamma without beta
     assert call(g=fake, b=fake) == 1                # the norm without its gradient outputs
+    assert call(g=vp(0x1004), b=fake, dg=fake, db=fake) == 1   # gamma off a 16-byte boundary
     assert call(d=100) == 4                         # d % 8 != 0
     assert call(L=0) == 1                           # no tokens
