@@ -357,12 +357,16 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
                 tma_store_3d(&map_h, smem + s * Lay::STAGE + Lay::U_BYTES, j0, bd, t0);
                 bulk_commit_group();
             }
-            // the next load goes to the stage chunk k-1 used: its store must be done reading it
             if (k + kAhead < nch) {
-                if (staged)
+                if (kAhead == S) {
+                    // the next load goes to this chunk's stage: its store must be done reading it
+                    if (staged) bulk_wait_group_read<0>();
+                } else if (staged) {
+                    // the next load goes to the stage chunk k-1 used: its store must be done reading it
                     bulk_wait_group_read<1>();
-                else
+                } else {
                     bulk_wait_group_read<0>();
+                }
             }
         }
         if (tid < 32 && k + kAhead < nch) issue(k + kAhead);
@@ -609,10 +613,12 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     int B, int d, int n_dir, float alpha) {
     using Lay = BwdLayout<UT, ACC_DX, CJ, S>;
     // Full chunks leave through TMA stores of the stage they came in on (dU over
-    // U, dx over x): a stage is refilled one iteration after its store was
-    // issued, so loads run S - 1 chunks ahead (needs S >= 3 to overlap).
-    constexpr bool kStage = sizeof(UT) == sizeof(DUT) && S >= 3;
-    constexpr int kAhead = kStage ? S - 1 : S;
+    // U, dx over x).  With S >= 3 a stage is refilled one iteration after its
+    // store was issued, so loads run S - 1 chunks ahead; with S = 2 loads run 2
+    // ahead and the stage just stored is refilled as soon as its store has read
+    // it (a wait of a few hundred cycles).
+    constexpr bool kStage = sizeof(UT) == sizeof(DUT) && S >= 2;
+    constexpr int kAhead = S >= 3 ? S - 1 : S;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
@@ -734,12 +740,16 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
                     tma_store_3d(&map_dxo, st + Lay::U_BYTES, j0, b, t0);
                 bulk_commit_group();
             }
-            // the next load goes to the stage chunk k-1 used: its store must be done reading it
             if (k + kAhead < nch) {
-                if (staged)
+                if (kAhead == S) {
+                    // the next load goes to this chunk's stage: its store must be done reading it
+                    if (staged) bulk_wait_group_read<0>();
+                } else if (staged) {
+                    // the next load goes to the stage chunk k-1 used: its store must be done reading it
                     bulk_wait_group_read<1>();
-                else
+                } else {
                     bulk_wait_group_read<0>();
+                }
             }
         }
         if (tid < 32 && k + kAhead < nch) issue(k + kAhead);
