@@ -100,9 +100,6 @@ __device__ __forceinline__ void tma_store_5d(const CUtensorMap* map, const void*
         "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
         : "memory");
 }
-__device__ __forceinline__ void st_relaxed_gpu2(float* p, float2 v) {
-    asm volatile("st.relaxed.gpu.global.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(v.x), "f"(v.y) : "memory");
-}
 
 // Tagged carry words of a channel pair: (tag << 32) | float bits, one 16-byte
 // access of two single-copy-atomic 64-bit elements.

@@ -34,14 +34,6 @@ namespace sru {
 
 constexpr int kScanSub = 4;                 // 16-step sub-chunks per scan chunk
 constexpr int kScanT = kScanSub * kChunkT;  // steps per scan chunk
-static_assert(kScanT <= 64, "sub-chunk row bits are packed in one 64-bit word");
-
-// Row bits of sub-chunk q from a packed word (kChunkT bits per sub-chunk), so
-// that loops over sub-chunks need not be unrolled: four unrolled copies of the
-// chunk code overflow the instruction cache.
-__device__ __forceinline__ uint32_t sub_bits(uint64_t packed, int q) {
-    return (uint32_t)(packed >> (kChunkT * q)) & ((1u << kChunkT) - 1u);
-}
 
 enum ScanFlag : unsigned { kFlagNone = 0, kFlagAgg = 1, kFlagPrefix = 2, kFlagAbort = 3 };
 
