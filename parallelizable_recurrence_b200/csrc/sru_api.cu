@@ -329,7 +329,7 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
             SRU_CUDA_TRY(cudaGetLastError());
         }
         kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
-            ma, mb, mo, out, (int)R, (int)C, (int)Kr, (int)ldo, splits, 1, 0LL, tail_s, 0);
+            ma, mb, mo, (int)R, (int)C, (int)Kr, splits, 1, tail_s, 0);
     }
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
@@ -337,26 +337,58 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
 
 // `batches` products of one shape in one launch of the pair kernel (operand
 // maps from map_kmajor_b / map_mnmajor_b with the batch at coordinate BPA /
-// BPB); product z writes out + z * out_bstride elements.
+// BPB); product z writes out + z * out_bstride elements, rows ldo apart, by
+// TMA stores through a 3-D output map (batch coordinate 1 when the batch
+// stride is below the row stride, else 2).
 // CAUSAL (square causal attention products, see sru::gemm::pair_unit): 1 = only
 // the output tiles on or below the diagonal, 2 = reduction cut at each row
-// tile's diagonal.
-template <bool A_MN, bool B_MN, int OUT, int BPA, int BPB, int CAUSAL = 0>
-sru_status launch_tc_gemm_batched(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
-                                  int64_t Kr, int64_t ldo, int64_t batches, int64_t out_bstride, cudaStream_t st) {
-    auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT, BPA, BPB, CAUSAL>;
+// tile's diagonal, 3 = reduction started at each row tile's diagonal.
+template <bool A_MN, bool B_MN, int OUT, int BPA, int BPB, int CAUSAL, int BPO>
+sru_status launch_batched_bpo(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
+                              int64_t Kr, int64_t ldo, int64_t batches, int64_t out_bstride, cudaStream_t st) {
+    auto kern = sru::gemm::tc_gemm_pair_kernel<A_MN, B_MN, OUT, BPA, BPB, CAUSAL, BPO>;
     SRU_CUDA_TRY(ensure_smem(reinterpret_cast<const void*>(kern), sru::gemm::P_SMEM_BYTES));
     const int64_t mt = (R + sru::gemm::P_BM - 1) / sru::gemm::P_BM, nt = (C + sru::gemm::P_BN - 1) / sru::gemm::P_BN;
     if (CAUSAL == 1 && R != C) return SRU_ERR_UNSUPPORTED;
     const int64_t units = (CAUSAL == 1 ? mt * (mt + 1) / 2 : mt * nt) * batches;
     if (units >= ((int64_t)1 << 31)) return SRU_ERR_UNSUPPORTED;
     const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
-    CUtensorMap unused;  // batched launches store directly (no output map)
-    std::memset(&unused, 0, sizeof(unused));
+    CUtensorMap mo;
+    {
+        const bool bf = OUT == sru::gemm::kOutBF16;
+        const uint64_t es = bf ? 2 : 4;
+        const uint32_t kc = (uint32_t)sru::gemm::EpiChunk<OUT>::kCols;
+        uint64_t dims[3], strides[2];
+        uint32_t box[3];
+        if (BPO == 1) {
+            dims[0] = (uint64_t)C; dims[1] = (uint64_t)batches; dims[2] = (uint64_t)R;
+            strides[0] = (uint64_t)out_bstride * es; strides[1] = (uint64_t)ldo * es;
+            box[0] = kc; box[1] = 1; box[2] = 32;
+        } else {
+            dims[0] = (uint64_t)C; dims[1] = (uint64_t)R; dims[2] = (uint64_t)batches;
+            strides[0] = (uint64_t)ldo * es; strides[1] = (uint64_t)out_bstride * es;
+            box[0] = kc; box[1] = 32; box[2] = 1;
+        }
+        if (!make_map(&mo, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, dims,
+                      strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return SRU_ERR_INVALID;
+    }
     kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
-        ma, mb, unused, out, (int)R, (int)C, (int)Kr, (int)ldo, 1, (int)batches, (long long)out_bstride, 0, 0);
+        ma, mb, mo, (int)R, (int)C, (int)Kr, 1, (int)batches, 0, 0);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
+}
+
+template <bool A_MN, bool B_MN, int OUT, int BPA, int BPB, int CAUSAL = 0>
+sru_status launch_tc_gemm_batched(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int64_t R, int64_t C,
+                                  int64_t Kr, int64_t ldo, int64_t batches, int64_t out_bstride, cudaStream_t st) {
+    if (out_bstride < ldo) {
+        if (C > out_bstride) return SRU_ERR_INVALID;  // the batches' columns would overlap
+        return launch_batched_bpo<A_MN, B_MN, OUT, BPA, BPB, CAUSAL, 1>(ma, mb, out, R, C, Kr, ldo, batches,
+                                                                       out_bstride, st);
+    }
+    return launch_batched_bpo<A_MN, B_MN, OUT, BPA, BPB, CAUSAL, 2>(ma, mb, out, R, C, Kr, ldo, batches, out_bstride,
+                                                                   st);
 }
 
 // Batched K-major operand: element (row r, k) of batch z at
@@ -1241,7 +1273,7 @@ static sru_status project_dW_split(const void* dU, const void* X, float* dW, int
     const int64_t units = tiles * pl.splits;
     const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
     kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(
-        ma, mb, mo, scratch, (int)N, (int)K, (int)M, (int)K, (int)pl.splits, 1, 0LL, 0, (int)pl.slab_rows);
+        ma, mb, mo, (int)N, (int)K, (int)M, (int)pl.splits, 1, 0, (int)pl.slab_rows);
     SRU_CUDA_TRY(cudaGetLastError());
     const size_t n4 = (size_t)N * K / 4;
     sru::gemm::splitk_reduce_kernel<<<(unsigned)std::min<size_t>(blocks_for(n4, 256), (size_t)sm_count() * 8), 256, 0,

@@ -50,47 +50,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
     return d;
 }
 
-// Store 32 consecutive accumulator columns (r[0..31]) of one output row.
-template <int OUT>
-__device__ __forceinline__ void epilogue_store_row32(void* __restrict__ out, int row, int col0, int M, int N, int ldo,
-                                                     const uint32_t (&r)[32]) {
-    if (row >= M) return;
-    if (OUT == kOutBF16) {
-        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * ldo + col0;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-            if (col0 + g * 8 < N) {
-                uint4 pk;
-                uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    __nv_bfloat162 two =
-                        __floats2bfloat162_rn(__uint_as_float(r[g * 8 + 2 * e]), __uint_as_float(r[g * 8 + 2 * e + 1]));
-                    w[e] = *reinterpret_cast<uint32_t*>(&two);
-                }
-                *reinterpret_cast<uint4*>(o + g * 8) = pk;
-            }
-        }
-    } else {
-        float* o = reinterpret_cast<float*>(out) + (size_t)row * ldo + col0;
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            if (col0 + g * 4 < N) {
-                float4 val = make_float4(__uint_as_float(r[g * 4 + 0]), __uint_as_float(r[g * 4 + 1]),
-                                         __uint_as_float(r[g * 4 + 2]), __uint_as_float(r[g * 4 + 3]));
-                if (OUT == kOutF32Acc) {
-                    const float4 old = *reinterpret_cast<const float4*>(o + g * 4);
-                    val.x += old.x;
-                    val.y += old.y;
-                    val.z += old.z;
-                    val.w += old.w;
-                }
-                *reinterpret_cast<float4*>(o + g * 4) = val;
-            }
-        }
-    }
-}
-
 // ---------------------------------------------------------------------------
 // A cluster of two CTAs (two SMs) computes one 256 x 256
 // output tile with tcgen05.mma.cta_group::2 (M = 256).  Each CTA stages its own
@@ -164,11 +123,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_pair(bool a_mn, bool b_mn) {
            ((uint32_t)(P_BN >> 3) << 17) | ((uint32_t)(P_BM >> 4) << 24);
 }
 
-// Batched form (BAT): `batches` independent products of the same shape.  The
+// Batched form: `batches` independent products of the same shape.  The
 // operands' tensor maps are 3-D with the batch index as coordinate bpos_a /
 // bpos_b (1 or 2) and the 2-D tile coordinates in the other two, so a box
-// lands in shared memory exactly as in the 2-D case; batch z writes
-// out + z * out_bstride.
+// lands in shared memory exactly as in the 2-D case; the output leaves the
+// same way through a 3-D map (BPO).
 template <int BPOS>
 __device__ __forceinline__ void tma_load_tile_pair(void* dst, const CUtensorMap* map, uint32_t bar, int x, int y,
                                                    int z) {
@@ -180,9 +139,11 @@ __device__ __forceinline__ void tma_load_tile_pair(void* dst, const CUtensorMap*
         tma_load_3d_pair(dst, map, bar, x, y, z);
 }
 
-// map_out (non-batched launches): the output as a 2-D tensor (N columns, M
-// rows, row stride ldo) of the output type, box 32 x 32, swizzle 64 B (bf16)
-// or 128 B (fp32).  Batched launches store directly and ignore it.
+// map_out: the output as a tensor of the output type that the epilogue's TMA
+// stores write, boxes of 32 rows x 128 bytes with 128-byte swizzle: 2-D (N
+// columns, M rows) for single products; for batched ones 3-D with the batch
+// index at coordinate BPO: 1 = between columns and rows (batch stride below
+// the row stride, e.g. time-major rows t B + b), 2 = outermost.
 // A work unit of the pair kernel: output tile (tm, tn) of batch z and its
 // k-block range [kb_lo, kb_hi).  CAUSAL (batched square products of SRU++'s
 // causal attention, tiles of P_BM = P_BN rows):
@@ -277,12 +238,12 @@ __device__ __forceinline__ bool pair_next(int i, int p, int P, int units, int m_
     return true;
 }
 
-template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0, int CAUSAL = 0>
+template <bool A_MN, bool B_MN, int OUT, int BPA = 0, int BPB = 0, int CAUSAL = 0, int BPO = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                        const __grid_constant__ CUtensorMap map_out, void* __restrict__ out, int M, int N, int K,
-                        int ldo, int splits, int batches, long long out_bstride, int tail_s, int slab_rows) {
-    constexpr bool kTmaOut = (BPA | BPB) == 0;
+                        const __grid_constant__ CUtensorMap map_out, int M, int N, int K, int splits, int batches,
+                        int tail_s, int slab_rows) {
+    static_assert(((BPA | BPB) == 0) == (BPO == 0), "batched launches store through a 3-D output map");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi = smem + P_STAGES * P_STAGE_BYTES;  // 1024-aligned staging buffers
@@ -321,7 +282,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         fence_mbar_init();
         tma_prefetch_desc(&map_a);
         tma_prefetch_desc(&map_b);
-        if (kTmaOut) tma_prefetch_desc(&map_out);
+        tma_prefetch_desc(&map_out);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, P_TMEM_COLS);
@@ -445,9 +406,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int i = 0; pair_next<CAUSAL>(i, pair_id, n_pairs, units, m_tiles, n_tiles, splits, kblocks, kper, tail_s, w);
              ++i, ++it) {
             const int z = w.z;
-            void* const zout = (BPA | BPB) != 0 ? static_cast<void*>(static_cast<uint8_t*>(out) +
-                                                             (size_t)z * (size_t)out_bstride * (OUT == kOutBF16 ? 2 : 4))
-                                        : out;
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             const int m0 = w.tm * P_BM + (int)rank * P_CM, n0 = w.tn * P_BN;
@@ -457,7 +415,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 break;
             }
             tc_fence_after_sync();
-            const int row = m0 + quarter * 32 + lane;
             // the accumulator leaves in chunks of kCols columns; the TMEM load of chunk
             // g + 1 is issued before chunk g is converted and stored, so its latency
             // overlaps that work
@@ -474,40 +431,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 tc_wait_ld();  // chunk g (and nothing else) is in flight
                 if (g + 1 < ng) tmem_ld_cols<NC>(tacc + (g + 1) * NC, nxt);
                 const int col0 = n0 + g * NC;
-                if (kTmaOut) {
-                    // buffer (nstaged & 1) was last read by the store issued two chunks ago
-                    const uint32_t buf = smem_u32(epi) + (uint32_t)(quarter * 2 + (nstaged & 1)) * P_EPI_BUF;
-                    if (nstaged >= 2) {
-                        if (lane == 0) bulk_wait_group_read<1>();
-                        __syncwarp();
-                    }
-                    epilogue_stage_row<OUT>(buf, lane, cur);
-                    fence_proxy_async_shared();
+                // buffer (nstaged & 1) was last read by the store issued two chunks ago
+                const uint32_t buf = smem_u32(epi) + (uint32_t)(quarter * 2 + (nstaged & 1)) * P_EPI_BUF;
+                if (nstaged >= 2) {
+                    if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();
-                    if (lane == 0) {
-                        const void* src = epi + (size_t)(quarter * 2 + (nstaged & 1)) * P_EPI_BUF;
-                        // split-K: k part s lands in slab s, rows s * slab_rows ..
-                        const int orow = m0 + quarter * 32 + w.split * slab_rows;
+                }
+                epilogue_stage_row<OUT>(buf, lane, cur);
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    const void* src = epi + (size_t)(quarter * 2 + (nstaged & 1)) * P_EPI_BUF;
+                    // split-K: k part s lands in slab s, rows s * slab_rows ..
+                    const int orow = m0 + quarter * 32 + w.split * slab_rows;
+                    if (BPO == 0) {
                         if (OUT == kOutF32Acc || w.reduce)
                             tma_reduce_add_2d(&map_out, src, col0, orow);
                         else
                             tma_store_2d(&map_out, src, col0, orow);
-                        bulk_commit_group();
+                    } else if (OUT == kOutF32Acc) {
+                        if (BPO == 1) tma_reduce_add_3d(&map_out, src, col0, z, orow);
+                        else tma_reduce_add_3d(&map_out, src, col0, orow, z);
+                    } else {
+                        if (BPO == 1) tma_store_3d(&map_out, src, col0, z, orow);
+                        else tma_store_3d(&map_out, src, col0, orow, z);
                     }
-                    ++nstaged;
-                } else {
-#pragma unroll
-                    for (int h = 0; h < NC / 32; ++h)
-                        if (col0 + h * 32 < N)
-                            epilogue_store_row32<OUT>(zout, row, col0 + h * 32, M, N, ldo,
-                                                      *reinterpret_cast<const uint32_t(*)[32]>(&cur[h * 32]));
+                    bulk_commit_group();
                 }
+                ++nstaged;
             }
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)acc * 8u);
         }
-        if (kTmaOut && lane == 0) bulk_wait_group<0>();  // every store of this warp has landed
+        if (lane == 0) bulk_wait_group<0>();  // every store of this warp has landed
     }
     tc_fence_before_sync();
     __syncthreads();

@@ -122,3 +122,12 @@ def test_attention_backward_alpha_zero_leaves_the_attention_weights_without_grad
     out, ref = _run(sru, 64, 2, 128, 32, 0.0, True, False, seed=11)
     assert torch.count_nonzero(out["dWkv"]).item() == 0
     _compare(out, ref)
+
+
+def test_attention_backward_at_the_training_layer_width(sru):
+    """d = 2048, d' = 512, N = 6144 as in the training layer, with the batch cut
+    to 2 rows so that the fp64 oracle finishes in seconds: every product at
+    its full width, the split weight gradients at their full reduction plans'
+    shapes (dWo 6144 x 512, dWkv 1024 x 512, dWq 512 x 2048)."""
+    out, ref = _run(sru, 1024, 2, 2048, 512, 0.5, True, True, seed=31)
+    _compare(out, ref)
