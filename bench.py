@@ -805,7 +805,9 @@ def run_ours(args):
             "phase_ms": phase_ms,
             "e2e": {"value": cfg.tokens * world * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": (5 if fused else 6) * args.steps,
+            # per step: [sru_project, sru_forward | sru_forward_fused], the backward recurrence, the dv/db
+            # reduction, dX, the zeroing of dW's split tail tiles, dW
+            "gpu_launches": (6 if fused else 7) * args.steps,
             "forward_path": args.forward,
             "clocks": clocks,
         }

@@ -323,9 +323,9 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
             kblocks >= 6) {
             const int64_t F = tiles / pairs, Rt = tiles % pairs;
             tail_s = (int)(2 * Rt <= pairs ? kblocks / 2 : kblocks / 3);
-            sru::gemm::zero_tail_tiles_kernel<<<(unsigned)Rt, 256, 0, st>>>(reinterpret_cast<float*>(out), (int)R,
-                                                                          (int)C, (long long)ldo, (int)n_tiles,
-                                                                          (int)(F * pairs));
+            const dim3 zgrid((unsigned)Rt, (unsigned)(sru::gemm::P_BM / sru::gemm::kZeroRows));
+            sru::gemm::zero_tail_tiles_kernel<<<zgrid, 256, 0, st>>>(reinterpret_cast<float*>(out), (int)R, (int)C,
+                                                                   (long long)ldo, (int)n_tiles, (int)(F * pairs));
             SRU_CUDA_TRY(cudaGetLastError());
         }
         kern<<<(unsigned)(2 * pairs), sru::gemm::THREADS, sru::gemm::P_SMEM_BYTES, st>>>(

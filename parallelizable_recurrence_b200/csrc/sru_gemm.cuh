@@ -477,12 +477,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
 // Zero the output regions of the tail tiles (tiles first_tile .. first_tile +
 // gridDim.x - 1 of P_BM x P_BN, clipped to R x C, row stride ldo floats) that
-// the tail split's two pieces then add onto.
+// the tail split's two pieces then add onto; P_BM / kZeroRows blocks per tile.
+// Block (x, y): tile first_tile + x, rows y * kZeroRows .. of it.
+constexpr int kZeroRows = 16;
 __global__ void __launch_bounds__(256) zero_tail_tiles_kernel(float* __restrict__ out, int R, int C, long long ldo,
                                                               int n_tiles, int first_tile) {
     const int tile = first_tile + blockIdx.x;
-    const int r0 = (tile / n_tiles) * P_BM, c0 = (tile % n_tiles) * P_BN;
-    const int rows = min(P_BM, R - r0), cols = min(P_BN, C - c0);  // C % 8 == 0: cols a multiple of 4
+    const int r0 = (tile / n_tiles) * P_BM + blockIdx.y * kZeroRows, c0 = (tile % n_tiles) * P_BN;
+    const int rows = min(kZeroRows, R - r0), cols = min(P_BN, C - c0);  // C % 8 == 0: cols a multiple of 4
     for (int e = threadIdx.x; e < rows * (cols / 4); e += blockDim.x) {
         const int r = e / (cols / 4), c4 = e % (cols / 4);
         *reinterpret_cast<float4*>(out + (size_t)(r0 + r) * ldo + c0 + 4 * c4) = make_float4(0.f, 0.f, 0.f, 0.f);
