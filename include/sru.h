@@ -180,7 +180,7 @@ sru_status sru_backward(const void* U, int u_t, const float* x, const float* v, 
  * exits.  The caller still passes all inputs and outputs (same layouts and
  * rules as sru_forward; v is not read and is taken as 0).
  *
- * Limit: ceil(L/64) * ceil(d/64) * B * n_dir work items, each needing 772
+ * Limit: ceil(L/128) * ceil(d/64) * B * n_dir work items, each needing 772
  * bytes of the scratch (about 10 800 items); a larger request returns
  * SRU_ERR_UNSUPPORTED before anything is launched.
  * The call allocates nothing (no cudaMalloc, cudaFree or allocating library

@@ -32,7 +32,7 @@
 
 namespace sru {
 
-constexpr int kScanSub = 4;                 // 16-step sub-chunks per scan chunk
+constexpr int kScanSub = 8;                 // 16-step sub-chunks per scan chunk
 constexpr int kScanT = kScanSub * kChunkT;  // steps per scan chunk
 
 enum ScanFlag : unsigned { kFlagNone = 0, kFlagAgg = 1, kFlagPrefix = 2, kFlagAbort = 3 };
@@ -121,8 +121,8 @@ __global__ void sru_scan_reset_kernel(unsigned* __restrict__ flags, int n) {
 }
 
 // A scan CTA has one warp per 16-step sub-chunk of its item: warp q stages,
-// reduces and re-walks sub-chunk q, so the item's 64 dependent steps run as
-// four chains of 16 in parallel.  The sub-chunks' affine maps meet in shared
+// reduces and re-walks sub-chunk q, so the item's 128 dependent steps run as
+// eight chains of 16 in parallel.  The sub-chunks' affine maps meet in shared
 // memory (one float4 (A.x, A.y, B.x, B.y) per lane and sub-chunk) and are
 // composed there, in the direction's time order, into the item's map and into
 // the state entering each sub-chunk.
@@ -440,7 +440,7 @@ __global__ void __launch_bounds__(kScanThreads) sru_bwd_scan_kernel(
     // the last sub-chunk in walk order leaves dc0
     const bool last = DIR == 0 ? q == 0 : (ts + kChunkT >= L || q == kScanSub - 1);
     if (k == nchs - 1 && last && ts < L && jok) store_pair(dc0 + (size_t)bd * d + j, g);
-    // the item's dv/db partial sums: the four warps' totals in sub-chunk order
+    // the item's dv/db partial sums: the warps' totals in sub-chunk order
     __syncthreads();
     if (q == 0 && jok) {
         const double* base = reinterpret_cast<const double*>(smem + Lay::ACC_OFF);

@@ -106,7 +106,7 @@ def test_noalloc_with_no_steps_returns_the_initial_state(sru):
 def test_noalloc_rejects_requests_beyond_its_scratch(sru):
     lib = sru.load_library()
     fake = ctypes.c_void_p(0x10000)
-    # ceil(4096/64) * ceil(1024/64) * 64 rows * 2 directions = 131072 work items >> the scratch
+    # ceil(4096/128) * ceil(1024/64) * 64 rows * 2 directions = 65536 work items >> the scratch
     status = lib.sru_forward_scan_noalloc(fake, sru.SRU_BF16, fake, fake, None, None, 4096, 64, 1024, 1.0, 1,
                                           fake, fake, None)
     assert status == sru.SRU_ERR_UNSUPPORTED
