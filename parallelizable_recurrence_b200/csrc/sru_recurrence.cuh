@@ -138,15 +138,25 @@ struct PairWord<float> {
     static __device__ __forceinline__ float2 unpack(T w) { return w; }
 };
 
+// Lane i's row of the chunk starting at t0 (lanes below kChunkT): it exists
+// (t < L) and is not padded.
+__device__ __forceinline__ bool chunk_row_ok(const uint8_t* __restrict__ mask, int t0, int L, int B, int b,
+                                             int lane) {
+    bool ok = lane < kChunkT && t0 + lane < L;
+    if (ok && mask != nullptr) ok = mask[(size_t)(t0 + lane) * B + b] == 0;
+    return ok;
+}
+// The warp's vote on chunk_row_ok: bit i set for row t0+i.  CTAs of fewer than
+// 32 threads (at least kChunkT) vote with their own lanes.
+__device__ __forceinline__ uint32_t chunk_vote(bool ok) {
+    const unsigned lanes = blockDim.x >= 32 ? 0xffffffffu : ((1u << blockDim.x) - 1u);
+    return __ballot_sync(lanes, ok);
+}
 // Bit i set: row t0+i of this chunk exists (t < L) and is not padded.  Every
 // thread of the warp (or of a CTA smaller than a warp) calls.
 __device__ __forceinline__ uint32_t chunk_valid_bits(const uint8_t* __restrict__ mask, int t0, int L, int B,
                                                      int b, int lane) {
-    bool ok = lane < kChunkT && t0 + lane < L;
-    if (ok && mask != nullptr) ok = mask[(size_t)(t0 + lane) * B + b] == 0;
-    // CTAs of fewer than 32 threads (at least kChunkT) vote with their own lanes
-    const unsigned lanes = blockDim.x >= 32 ? 0xffffffffu : ((1u << blockDim.x) - 1u);
-    return __ballot_sync(lanes, ok);
+    return chunk_vote(chunk_row_ok(mask, t0, L, B, b, lane));
 }
 __device__ __forceinline__ uint32_t chunk_inrange_bits(int t0, int L) {
     const int n = L - t0;
@@ -304,11 +314,15 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
     __syncthreads();
 
     auto time_chunk = [&](int k) { return dir == 0 ? k : nch - 1 - k; };
+    // the row-validity words of processing chunks k .. k + kAhead, slot k & 3: each is
+    // voted on when its chunk's loads are issued, from mask bytes fetched one chunk
+    // earlier, so no mask read sits on the chain
+    uint32_t* vring = reinterpret_cast<uint32_t*>(full + S);
     uint32_t pending = 0;  // thread 0: stages with a load in flight
     // warp 0 issues the loads of processing chunk k into stage k % S (skipped if fully padded)
-    auto issue = [&](int k) {
+    auto issue = [&](int k, uint32_t valid) {
+        if (lane == 0) vring[k & 3] = valid;
         const int t0 = time_chunk(k) * kChunkT;
-        const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
         if (tid == 0 && valid != 0u) {
             const int s = k % S;
             pending |= 1u << s;
@@ -319,14 +333,18 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
         }
     };
     if (tid < 32)
-        for (int k = 0; k < kAhead && k < nch; ++k) issue(k);
+        for (int k = 0; k < kAhead && k < nch; ++k)
+            issue(k, chunk_valid_bits(mask, time_chunk(k) * kChunkT, L, B, b, lane));
+    __syncthreads();
 
     uint32_t phase_bits = 0;
     const size_t h_tstride = (size_t)B * n_dir * d;
     for (int k = 0; k < nch; ++k) {
         const int s = k % S;
         const int tc = time_chunk(k), t0 = tc * kChunkT;
-        const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
+        const uint32_t valid = vring[k & 3];
+        // this lane's row of the chunk whose loads go out at the end of this iteration
+        const bool row_next = k + kAhead < nch && chunk_row_ok(mask, time_chunk(k + kAhead) * kChunkT, L, B, b, lane);
         const uint32_t inrange = chunk_inrange_bits(t0, L);
         if (ckpt != nullptr && jok) store_pair(ckpt + ((size_t)tc * B * n_dir + bd) * d + j, c);
         if (valid != 0u) {
@@ -357,19 +375,14 @@ __global__ void __launch_bounds__(CJ / 2) sru_fwd_seq_kernel(
                 tma_store_3d(&map_h, smem + s * Lay::STAGE + Lay::U_BYTES, j0, bd, t0);
                 bulk_commit_group();
             }
+            // the next load goes to the stage chunk k-1 used (kAhead = S - 1 here): its
+            // store must be done reading it
             if (k + kAhead < nch) {
-                if (kAhead == S) {
-                    // the next load goes to this chunk's stage: its store must be done reading it
-                    if (staged) bulk_wait_group_read<0>();
-                } else if (staged) {
-                    // the next load goes to the stage chunk k-1 used: its store must be done reading it
-                    bulk_wait_group_read<1>();
-                } else {
-                    bulk_wait_group_read<0>();
-                }
+                if (staged) bulk_wait_group_read<1>();
+                else bulk_wait_group_read<0>();
             }
         }
-        if (tid < 32 && k + kAhead < nch) issue(k + kAhead);
+        if (tid < 32 && k + kAhead < nch) issue(k + kAhead, chunk_vote(row_next));
     }
     if (kStage && tid == 0) bulk_wait_group<0>();  // every store has landed
     if (jok) store_pair(c_T + (size_t)bd * d + j, c);
@@ -655,10 +668,14 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
 
     // backward processing chunk k covers time chunk: dir 0 walks time chunks downwards
     auto time_chunk = [&](int k) { return dir == 0 ? nch - 1 - k : k; };
+    // the row-validity words of processing chunks k .. k + kAhead, slot k & 3: each is
+    // voted on when its chunk's loads are issued, from mask bytes fetched one chunk
+    // earlier, so no mask read sits on the chain
+    uint32_t* vring = reinterpret_cast<uint32_t*>(full + S);
     uint32_t pending = 0;  // thread 0: stages with a load in flight
-    auto issue = [&](int k) {
+    auto issue = [&](int k, uint32_t valid) {
+        if (lane == 0) vring[k & 3] = valid;
         const int t0 = time_chunk(k) * kChunkT;
-        const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
         if (tid == 0 && valid != 0u) {
             const int s = k % S;
             pending |= 1u << s;
@@ -670,7 +687,9 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
         }
     };
     if (tid < 32)
-        for (int k = 0; k < kAhead && k < nch; ++k) issue(k);
+        for (int k = 0; k < kAhead && k < nch; ++k)
+            issue(k, chunk_valid_bits(mask, time_chunk(k) * kChunkT, L, B, b, lane));
+    __syncthreads();
 
     SmemPartials acc{reinterpret_cast<double*>(smem + Lay::ACC_OFF) + tid, CJ / 2};
 #pragma unroll
@@ -701,7 +720,9 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
     for (int k = 0; k < nch; ++k) {
         const int s = k % S;
         const int tc = time_chunk(k), t0 = tc * kChunkT;
-        const uint32_t valid = chunk_valid_bits(mask, t0, L, B, b, lane);
+        const uint32_t valid = vring[k & 3];
+        // this lane's row of the chunk whose loads go out at the end of this iteration
+        const bool row_next = k + kAhead < nch && chunk_row_ok(mask, time_chunk(k + kAhead) * kChunkT, L, B, b, lane);
         const uint32_t inrange = chunk_inrange_bits(t0, L);
         const float2 ck2 = ckpt_of(k + 2);
         DUT* dUp = dU + (size_t)t0 * u_tstride + (size_t)bd * 3 * d + j;
@@ -752,7 +773,7 @@ __global__ void __launch_bounds__(CJ / 2) sru_bwd_seq_kernel(
                 }
             }
         }
-        if (tid < 32 && k + kAhead < nch) issue(k + kAhead);
+        if (tid < 32 && k + kAhead < nch) issue(k + kAhead, chunk_vote(row_next));
         ck0 = ck1;
         ck1 = ck2;
     }
