@@ -809,6 +809,20 @@ int64_t fused_resident_pairs() {
 }  // namespace
 
 // =========================================================================
+// grid: two CTAs per SM (one for the widest rows), at most one per kNormRows
+// rows (the slices the workspace holds); returns the slices written
+template <int NV>
+unsigned norm_backward_params_reg(const float* dR, const __nv_bfloat16* Q, const float* A, float alpha, const float* g,
+                                  float* dQ, __nv_bfloat16* dA, float2* stats, float* part, int64_t M, int64_t dp,
+                                  cudaStream_t st) {
+    const unsigned per_sm = NV <= 4 ? 2u : 1u;
+    unsigned grid = (unsigned)sm_count() * per_sm;
+    const unsigned cap = blocks_for((size_t)M, sru::kNormRows);
+    if (grid > cap) grid = cap;
+    sru::sru_norm_backward_params_reg_kernel<NV><<<grid, sru::kRowWarps * 32, 0, st>>>(dR, Q, A, alpha, g, dQ, dA,
+                                                                                     stats, part, (int)M, (int)dp);
+    return grid;
+}
 template <int NV>
 void norm_backward_reg(const float* dR, const __nv_bfloat16* Q, const float* A, float alpha, const float* g, float* dQ,
                        __nv_bfloat16* dA, float2* stats, int64_t M, int64_t dp, cudaStream_t st) {
@@ -846,6 +860,27 @@ sru_status launch_softmax_rows(const float* S, __nv_bfloat16* P, int64_t L, int6
     else
         sru::sru_softmax_rows_kernel<<<blocks_for((size_t)rows, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(
             S, P, (int)L, (int)rows, scale, causal);
+    SRU_CUDA_TRY(cudaGetLastError());
+    return SRU_OK;
+}
+template <int NV>
+void softmax_backward_reg(const float* dP, const __nv_bfloat16* P, __nv_bfloat16* dS, int64_t L, int64_t rows,
+                          float scale, int causal, cudaStream_t st) {
+    sru::sru_softmax_backward_rows_reg_kernel<NV>
+        <<<blocks_for((size_t)rows, sru::kRowWarps), sru::kRowWarps * 32, 0, st>>>(dP, P, dS, (int)L, (int)rows,
+                                                                                  scale, causal);
+}
+sru_status launch_softmax_backward_rows(const float* dP, const __nv_bfloat16* P, __nv_bfloat16* dS, int64_t L,
+                                        int64_t rows, float scale, int causal, cudaStream_t st) {
+    const int64_t nv = (L + 127) / 128;
+    if (nv <= 1) softmax_backward_reg<1>(dP, P, dS, L, rows, scale, causal, st);
+    else if (nv <= 2) softmax_backward_reg<2>(dP, P, dS, L, rows, scale, causal, st);
+    else if (nv <= 4) softmax_backward_reg<4>(dP, P, dS, L, rows, scale, causal, st);
+    else if (nv <= 8) softmax_backward_reg<8>(dP, P, dS, L, rows, scale, causal, st);
+    else if (nv <= 16) softmax_backward_reg<16>(dP, P, dS, L, rows, scale, causal, st);
+    else
+        sru::sru_softmax_backward_rows_kernel<<<blocks_for((size_t)rows, sru::kRowWarps), sru::kRowWarps * 32, 0,
+                                                st>>>(dP, P, dS, (int)L, (int)rows, scale, causal);
     SRU_CUDA_TRY(cudaGetLastError());
     return SRU_OK;
 }
@@ -1521,16 +1556,30 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
     if (s != SRU_OK) return s;
     s = project_dW_split(dU, R, dWo, M, N, dp, split, w.split_bytes, st);
     if (s != SRU_OK) return s;
-    // through the norm (or the identity): dQ = dZ, dA = alpha dZ
-    s = launch_norm_backward(dR, Q, A, alpha, ln_gamma, dQ, dA, stats, M, dp, st);
-    if (s != SRU_OK) return s;
-    if (norm) {
-        const unsigned slices = (unsigned)((M + sru::kNormRows - 1) / sru::kNormRows);
-        if (slices > 65535u) return SRU_ERR_UNSUPPORTED;
-        const dim3 grid(blocks_for((size_t)dp, sru::kNormParamThreads), slices);
-        sru::sru_norm_param_partial_kernel<<<grid, sru::kNormParamThreads, 0, st>>>(dR, Q, A, alpha, stats, part,
-                                                                                   (int)M, (int)dp);
+    // through the norm (or the identity): dQ = dZ, dA = alpha dZ.  With the norm, the
+    // first stage of dgamma / dbeta (slices of kNormRows tokens) is taken inside the
+    // norm's backward where the row fits in registers.
+    const int64_t nv = (dp + 127) / 128;
+    unsigned slices = (unsigned)((M + sru::kNormRows - 1) / sru::kNormRows);
+    if (norm && nv <= 8) {
+        auto run = nv <= 1 ? norm_backward_params_reg<1>
+                   : nv <= 2 ? norm_backward_params_reg<2>
+                   : nv <= 4 ? norm_backward_params_reg<4>
+                             : norm_backward_params_reg<8>;
+        slices = run(dR, Q, A, alpha, ln_gamma, dQ, dA, stats, part, M, dp, st);
         SRU_CUDA_TRY(cudaGetLastError());
+    } else {
+        s = launch_norm_backward(dR, Q, A, alpha, ln_gamma, dQ, dA, stats, M, dp, st);
+        if (s != SRU_OK) return s;
+        if (norm) {
+            if (slices > 65535u) return SRU_ERR_UNSUPPORTED;
+            const dim3 grid(blocks_for((size_t)dp, sru::kNormParamThreads), slices);
+            sru::sru_norm_param_partial_kernel<<<grid, sru::kNormParamThreads, 0, st>>>(dR, Q, A, alpha, stats,
+                                                                                       part, (int)M, (int)dp);
+            SRU_CUDA_TRY(cudaGetLastError());
+        }
+    }
+    if (norm) {
         sru::sru_norm_param_reduce_kernel<<<blocks_for((size_t)(2 * dp), sru::kNormRedCols),
                                             sru::kNormRedCols * sru::kNormRedGroups, 0, st>>>(part, (int)slices,
                                                                                             (int)dp, dgamma, dbeta);
@@ -1564,9 +1613,8 @@ sru_status sru_attention_project_backward(const void* dU, const void* X, const v
         s = causal ? launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st)
                    : launch_tc_gemm_batched<false, false, sru::gemm::kOutF32, 1, 1>(ma, mb, S, L, L, dp, L, g, L * L, st);
         if (s != SRU_OK) return s;
-        sru::sru_softmax_backward_rows_kernel<<<blocks_for((size_t)(g * L), sru::kRowWarps), sru::kRowWarps * 32, 0,
-                                                st>>>(S, Pg, dS, (int)L, (int)(g * L), scale, causal ? 1 : 0);
-        SRU_CUDA_TRY(cudaGetLastError());
+        s = launch_softmax_backward_rows(S, Pg, dS, L, g * L, scale, causal ? 1 : 0, st);
+        if (s != SRU_OK) return s;
         // dV = P^T dA and dK = dS^T Q (bf16, into [dK | dV]): the first operand read
         // MN-major (element (s, t) of batch z at z L^2 + t L + s), the second too
         // (element (j, t) at (t B + b0 + z) d' + j)

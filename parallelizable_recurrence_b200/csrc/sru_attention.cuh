@@ -224,6 +224,66 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_softmax_backward_rows_kern
         drow[s] = __float2bfloat16_rn(s < n ? __bfloat162float(prow[s]) * (grow[s] - dot) * scale : 0.f);
 }
 
+// The same gradient with the row held in registers (rows of at most NV * 128,
+// read once with 16-byte loads of dP and 8-byte loads of P): lane l owns
+// entries 4l .. 4l + 3 of every 128.  When causal, dS is written only up to
+// the end of the row's 256-wide tile, as P is: the products that read dS
+// (dS K up to the end of each row tile, dS^T Q from each row tile's diagonal
+// on) never read further.
+template <int NV>
+__global__ void __launch_bounds__(kRowWarps * 32, NV <= 8 ? 2 : 1) sru_softmax_backward_rows_reg_kernel(
+    const float* __restrict__ dP, const __nv_bfloat16* __restrict__ P, __nv_bfloat16* __restrict__ dS, int L, int rows,
+    float scale, int causal) {
+    const int row = blockIdx.x * kRowWarps + threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (row >= rows) return;
+    const int t = row % L;
+    const float4* grow = reinterpret_cast<const float4*>(dP + (size_t)row * L);
+    const uint2* prow = reinterpret_cast<const uint2*>(P + (size_t)row * L);
+    uint2* drow = reinterpret_cast<uint2*>(dS + (size_t)row * L);
+    const int n = causal ? t + 1 : L;
+    const int end = causal ? min(L, (t / 256 + 1) * 256) : L;  // written: [0, end)
+    float4 gr[NV];
+    uint2 pr[NV];  // 4 bf16
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int s0 = k * 128 + lane * 4;
+        gr[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        pr[k] = make_uint2(0u, 0u);
+        if (s0 < n) {
+            gr[k] = grow[s0 / 4];
+            pr[k] = prow[s0 / 4];
+        }
+    }
+    // entry e of chunk k as fp32, 0 where invisible (s >= n)
+    auto pval = [&](int k, int e) {
+        const uint32_t w = e < 2 ? pr[k].x : pr[k].y;
+        const float v = __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+        return k * 128 + lane * 4 + e < n ? v : 0.f;
+    };
+    auto gval = [&](int k, int e) {
+        const float v = e == 0 ? gr[k].x : e == 1 ? gr[k].y : e == 2 ? gr[k].z : gr[k].w;
+        return k * 128 + lane * 4 + e < n ? v : 0.f;
+    };
+    float dot = 0.f;
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dot = fmaf(pval(k, e), gval(k, e), dot);
+    dot = warp_sum(dot);
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int s0 = k * 128 + lane * 4;
+        if (s0 >= end) continue;
+        // invisible entries have p = 0, so they come out as 0
+        float o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] = pval(k, e) * (gval(k, e) - dot) * scale;
+        __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(o[2], o[3]);
+        drow[s0 / 4] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+    }
+}
+
 // Gradient through R = Z (no norm) or R = layernorm(Z) gamma + beta, with
 // Z = Q + alpha A recomputed exactly as the forward did.  Row m:
 //   no norm:  dZ = dR
@@ -280,18 +340,35 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_kernel(
 }
 
 // The same gradient with the row held in registers (d' at most NV * 128, each
-// input read once): lane l owns features 4l .. 4l + 3 of every 128.
+// input read once): lane l owns features 4l .. 4l + 3 of every 128.  The
+// row's inputs are loaded first (NormRowIn), so that a caller walking several
+// rows can have the next row's loads in flight while this one is computed.
 template <int NV>
-__global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_reg_kernel(
-    const float* __restrict__ dR, const __nv_bfloat16* __restrict__ Q, const float* __restrict__ A, float alpha,
-    const float* __restrict__ gamma, float* __restrict__ dQ, __nv_bfloat16* __restrict__ dA,
-    float2* __restrict__ stats, int M, int dp) {
-    const int m = blockIdx.x * kRowWarps + threadIdx.x / 32, lane = threadIdx.x % 32;
-    if (m >= M) return;
-    const float4* dr = reinterpret_cast<const float4*>(dR + (size_t)m * dp);
-    float4* dq = reinterpret_cast<float4*>(dQ + (size_t)m * dp);
-    uint2* da = reinterpret_cast<uint2*>(dA + (size_t)m * dp);
-    float g[NV][4], z[NV][4];
+struct NormRowIn {
+    float4 r[NV];  // dR
+    float4 a[NV];  // A (with the norm)
+    uint2 q[NV];   // Q, 4 bf16 (with the norm)
+};
+template <int NV>
+__device__ __forceinline__ void load_norm_row(NormRowIn<NV>& in, const float* __restrict__ dR,
+                                              const __nv_bfloat16* __restrict__ Q, const float* __restrict__ A,
+                                              bool norm, int m, int dp, int lane) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int j0 = k * 128 + lane * 4;
+        if (j0 >= dp) continue;
+        in.r[k] = reinterpret_cast<const float4*>(dR + (size_t)m * dp)[j0 / 4];
+        if (norm) {
+            in.q[k] = reinterpret_cast<const uint2*>(Q + (size_t)m * dp)[j0 / 4];
+            in.a[k] = reinterpret_cast<const float4*>(A + (size_t)m * dp)[j0 / 4];
+        }
+    }
+}
+// Row m's inputs as fp32: g = dR, z = Q + alpha A (with the norm); returns the
+// lane's sum of z.  After this the NormRowIn may be reloaded.
+template <int NV>
+__device__ __forceinline__ float unpack_norm_row(const NormRowIn<NV>& in, float alpha, bool norm, int dp, int lane,
+                                                 float (&g)[NV][4], float (&z)[NV][4]) {
     float sum = 0.f;
 #pragma unroll
     for (int k = 0; k < NV; ++k) {
@@ -301,14 +378,14 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_reg_kernel(
             for (int e = 0; e < 4; ++e) g[k][e] = z[k][e] = 0.f;
             continue;
         }
-        const float4 r4 = dr[j0 / 4];
+        const float4 r4 = in.r[k];
         g[k][0] = r4.x;
         g[k][1] = r4.y;
         g[k][2] = r4.z;
         g[k][3] = r4.w;
-        if (gamma != nullptr) {
-            const uint2 qq = reinterpret_cast<const uint2*>(Q + (size_t)m * dp)[j0 / 4];
-            const float4 aa = reinterpret_cast<const float4*>(A + (size_t)m * dp)[j0 / 4];
+        if (norm) {
+            const uint2 qq = in.q[k];
+            const float4 aa = in.a[k];
             const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qq.x));
             const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qq.y));
             z[k][0] = fmaf(alpha, aa.x, q01.x);
@@ -318,6 +395,18 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_reg_kernel(
             sum += z[k][0] + z[k][1] + z[k][2] + z[k][3];
         }
     }
+    return sum;
+}
+// Row m's gradient from its unpacked inputs.  With PARAMS (gamma given) row
+// m's terms of the parameter gradients are added to the lane's running sums:
+// pg += dR * Zhat (dgamma), pb += dR (dbeta).
+template <int NV, bool PARAMS>
+__device__ __forceinline__ void finish_norm_row(float (&g)[NV][4], float (&z)[NV][4], float sum, float alpha,
+                                                const float* __restrict__ gamma, float* __restrict__ dQ,
+                                                __nv_bfloat16* __restrict__ dA, float2* __restrict__ stats, int m,
+                                                int dp, int lane, float (&pg)[NV][4], float (&pb)[NV][4]) {
+    float4* dq = reinterpret_cast<float4*>(dQ + (size_t)m * dp);
+    uint2* da = reinterpret_cast<uint2*>(dA + (size_t)m * dp);
     if (gamma != nullptr) {
         const float mean = warp_sum(sum) / (float)dp;
         float sq = 0.f;
@@ -338,7 +427,11 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_reg_kernel(
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 z[k][e] = (z[k][e] - mean) * rstd;  // Zhat from here on
-                g[k][e] *= gv[e];                   // dZhat = dR * gamma
+                if (PARAMS) {
+                    pg[k][e] = fmaf(g[k][e], z[k][e], pg[k][e]);
+                    pb[k][e] += g[k][e];
+                }
+                g[k][e] *= gv[e];  // dZhat = dR * gamma
                 s1 += g[k][e];
                 s2 = fmaf(g[k][e], z[k][e], s2);
             }
@@ -364,12 +457,27 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_reg_kernel(
     }
 }
 
+template <int NV>
+__global__ void __launch_bounds__(kRowWarps * 32) sru_norm_backward_reg_kernel(
+    const float* __restrict__ dR, const __nv_bfloat16* __restrict__ Q, const float* __restrict__ A, float alpha,
+    const float* __restrict__ gamma, float* __restrict__ dQ, __nv_bfloat16* __restrict__ dA,
+    float2* __restrict__ stats, int M, int dp) {
+    const int m = blockIdx.x * kRowWarps + threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (m >= M) return;
+    NormRowIn<NV> in;
+    load_norm_row<NV>(in, dR, Q, A, gamma != nullptr, m, dp, lane);
+    float g[NV][4], z[NV][4];
+    const float sum = unpack_norm_row<NV>(in, alpha, gamma != nullptr, dp, lane, g, z);
+    float pg[NV][4], pb[NV][4];  // not used without PARAMS
+    finish_norm_row<NV, false>(g, z, sum, alpha, gamma, dQ, dA, stats, m, dp, lane, pg, pb);
+}
+
 // The norm's parameter gradients, first stage: slice y of the rows (rows
 // [y * kNormRows, (y + 1) * kNormRows)) summed per feature j in fp32, in row
 // order, into part[y][0][j] (dgamma: dR * Zhat) and part[y][1][j] (dbeta: dR).
-// (Slices of 64 rows: the second stage then sums a few hundred slices, 32
-// thread groups per column, instead of a thousand on 8 groups.)
-constexpr int kNormRows = 64;
+// This kernel re-reads dR, Q and A; sru_norm_backward_params_reg_kernel
+// below does the same stage inside the norm's backward for d' <= 1024.
+constexpr int kNormRows = 32;
 constexpr int kNormParamThreads = 256;
 __global__ void __launch_bounds__(kNormParamThreads) sru_norm_param_partial_kernel(
     const float* __restrict__ dR, const __nv_bfloat16* __restrict__ Q, const float* __restrict__ A, float alpha,
@@ -387,6 +495,58 @@ __global__ void __launch_bounds__(kNormParamThreads) sru_norm_param_partial_kern
     }
     part[((size_t)blockIdx.y * 2 + 0) * dp + j] = sg;
     part[((size_t)blockIdx.y * 2 + 1) * dp + j] = sb;
+}
+
+// The norm's backward and the first stage of its parameter gradients in one
+// pass (gamma given, d' at most NV * 128), on a grid that stays resident:
+// warp w of CTA y takes rows (y + i * gridDim.x) * kRowWarps + w for i = 0,
+// 1, ... (so every warp has the same number of rows, give or take one), keeps
+// its sums of dR * Zhat and dR per feature in registers, and the warps' sums
+// are added in warp order into slice y: part[y][0][j] (dgamma) and
+// part[y][1][j] (dbeta).  For a given grid the order is fixed, so the result
+// is the same on every run.
+template <int NV>
+__global__ void __launch_bounds__(kRowWarps * 32, NV <= 4 ? 2 : 1) sru_norm_backward_params_reg_kernel(
+    const float* __restrict__ dR, const __nv_bfloat16* __restrict__ Q, const float* __restrict__ A, float alpha,
+    const float* __restrict__ gamma, float* __restrict__ dQ, __nv_bfloat16* __restrict__ dA,
+    float2* __restrict__ stats, float* __restrict__ part, int M, int dp) {
+    __shared__ float red[2][NV * 128];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    float pg[NV][4], pb[NV][4];
+#pragma unroll
+    for (int k = 0; k < NV; ++k)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pg[k][e] = pb[k][e] = 0.f;
+    const int stride = gridDim.x * kRowWarps;
+    // the next row's loads are issued as soon as this row's inputs are unpacked,
+    // so they are in flight while this row is computed
+    NormRowIn<NV> in;
+    int m = blockIdx.x * kRowWarps + warp;
+    if (m < M) load_norm_row<NV>(in, dR, Q, A, true, m, dp, lane);
+#pragma unroll 1
+    for (; m < M; m += stride) {
+        float g[NV][4], z[NV][4];
+        const float sum = unpack_norm_row<NV>(in, alpha, true, dp, lane, g, z);
+        if (m + stride < M) load_norm_row<NV>(in, dR, Q, A, true, m + stride, dp, lane);
+        finish_norm_row<NV, true>(g, z, sum, alpha, gamma, dQ, dA, stats, m, dp, lane, pg, pb);
+    }
+    for (int w = 0; w < kRowWarps; ++w) {
+        if (warp == w) {
+#pragma unroll
+            for (int k = 0; k < NV; ++k) {
+                const int j0 = k * 128 + lane * 4;
+                if (j0 >= dp) continue;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    red[0][j0 + e] = w == 0 ? pg[k][e] : red[0][j0 + e] + pg[k][e];
+                    red[1][j0 + e] = w == 0 ? pb[k][e] : red[1][j0 + e] + pb[k][e];
+                }
+            }
+        }
+        __syncthreads();
+    }
+    float* out = part + (size_t)blockIdx.x * 2 * dp;
+    for (int c = threadIdx.x; c < 2 * dp; c += kRowWarps * 32) out[c] = red[c / dp][c % dp];
 }
 
 // Second stage: column c of the slices' partial sums (c < d': dgamma, else

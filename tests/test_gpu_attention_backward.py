@@ -99,6 +99,9 @@ def _compare(out, ref):
     (2048, 5, 64, 16, 0.5, True, False),     # every batch row's probabilities kept by the forward (one group)
     (4096, 3, 64, 16, 0.5, True, True),      # long rows in groups of 2: the probabilities are recomputed
     (72, 3, 96, 40, 0.9, True, True),        # widths that are not multiples of a tile or a k-block
+    (48, 2, 64, 1024, 0.5, True, True),      # d' = 1024: the widest norm row held in registers
+    (48, 2, 64, 1152, 0.5, False, True),     # d' past that: the norm's row-loop kernels
+    (80, 5, 64, 200, 0.5, True, True),       # norm slices of 32 tokens ending mid-slice
 ])
 def test_attention_backward_matches_oracle(sru, L, B, d, dp, alpha, causal, ln):
     out, ref = _run(sru, L, B, d, dp, alpha, causal, ln, seed=L + B + d + dp)
