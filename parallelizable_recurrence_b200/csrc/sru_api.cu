@@ -319,9 +319,13 @@ sru_status launch_tc_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* ou
         const int64_t pairs = units < sm_count() / 2 ? units : sm_count() / 2;
         int tail_s = 0;
         const int64_t kblocks = (Kr + sru::gemm::BK - 1) / sru::gemm::BK;
-        if (tail_split && OUT == sru::gemm::kOutF32 && splits == 1 && tiles > pairs && tiles % pairs != 0 &&
-            kblocks >= 6) {
-            const int64_t F = tiles / pairs, Rt = tiles % pairs;
+        // the schedule (sru::gemm::pair_next) covers every tail tile only while the
+        // partial round holds at most two thirds of the pairs: past that the short
+        // pieces outnumber the pairs left to take two each, so no split
+        const int64_t Rt = tiles % pairs;
+        if (tail_split && OUT == sru::gemm::kOutF32 && splits == 1 && tiles > pairs && Rt != 0 &&
+            3 * Rt <= 2 * pairs && kblocks >= 6) {
+            const int64_t F = tiles / pairs;
             tail_s = (int)(2 * Rt <= pairs ? kblocks / 2 : kblocks / 3);
             const dim3 zgrid((unsigned)Rt, (unsigned)(sru::gemm::P_BM / sru::gemm::kZeroRows));
             sru::gemm::zero_tail_tiles_kernel<<<zgrid, 256, 0, st>>>(reinterpret_cast<float*>(out), (int)R, (int)C,
@@ -982,8 +986,11 @@ sru_status sru_project_backward(const void* dU, const void* X, const void* W, in
             CUtensorMap ma, mb;
             // A = dU (M x N) K-major; B(c = k, red = n) = W[n][k]: MN-major with ld = K
             if (!map_kmajor(&ma, dU, M, N, sru::gemm::P_CM) || !map_mnmajor(&mb, W, K, N, K)) return SRU_ERR_INVALID;
+            // written (not accumulated): the tiles of a last, partial round of CTA pairs are
+            // cut in two k-pieces, as for dW
             sru_status s = accumulate ? launch_tc_gemm<false, true, sru::gemm::kOutF32Acc>(ma, mb, dX, M, K, N, st)
-                                      : launch_tc_gemm<false, true, sru::gemm::kOutF32>(ma, mb, dX, M, K, N, st);
+                                      : launch_tc_gemm<false, true, sru::gemm::kOutF32>(ma, mb, dX, M, K, N, st, 1,
+                                                                                        -1, /*tail_split=*/true);
             if (s != SRU_OK) return s;
         }
     }

@@ -202,7 +202,9 @@ __device__ __forceinline__ PairUnit pair_unit(int u, int m_tiles, int n_tiles, i
 //   tile (P - R) + (p - R).
 // The host takes s = K/2 when 2R <= P (every piece its own pair) and s = K/3
 // otherwise (some pairs take two short pieces): the tail then costs half or
-// two thirds of a round instead of a whole one.
+// two thirds of a round instead of a whole one.  The second case covers all R
+// tail tiles only while R - (P - R) <= P - R, i.e. R <= 2P/3; the host splits
+// no tail past that.
 template <int CAUSAL>
 __device__ __forceinline__ bool pair_next(int i, int p, int P, int units, int m_tiles, int n_tiles, int splits,
                                           int kblocks, int kper, int tail_s, PairUnit& w) {

@@ -104,12 +104,13 @@ def test_project_large_k_sampled(sru):
     tl.assert_close_sum("dW sampled", tl.host_f64(dW)[rows, cols], ref, absref)
 
 
-@pytest.mark.parametrize("N,K", [(6144, 2048), (3072, 2048)])
+@pytest.mark.parametrize("N,K", [(6144, 2048), (3072, 2048), (4096, 2048)])
 def test_tail_split_dw_matches_oracle_and_is_deterministic(sru, N, K):
     """dW whose output tiles do not fill whole rounds of the 74 CTA pairs: the
     tiles of the last, partial round are cut in two k-pieces that add onto a
     zeroed region (192 tiles: pieces of K/3 and 2K/3, some pairs taking two short
-    pieces; 96 tiles: halves).  Entries of those tiles and of whole tiles match
+    pieces; 96 tiles: halves).  At 128 tiles the partial round holds 54 of the
+    74 pairs, more than two thirds, and no tail is split.  Entries of those tiles and of whole tiles match
     the oracle's plain sums, and with two addends per element the fp32 result is
     the same whichever piece lands first: repeated calls agree bit for bit."""
     rng = np.random.default_rng(5)
@@ -130,3 +131,31 @@ def test_tail_split_dw_matches_oracle_and_is_deterministic(sru, N, K):
     ref = oracle.project_dW_entries(dUb, Xb, rows, cols)
     absref = oracle.project_dW_entries(tl.abs_operand(dUb), tl.abs_operand(Xb), rows, cols)
     tl.assert_close_sum("dW sampled", got[rows, cols], ref, absref)
+
+
+@pytest.mark.parametrize("M,K", [(16384, 512), (15360, 512), (12288, 512)])
+def test_tail_split_dx_matches_oracle_and_is_deterministic(sru, M, K):
+    """dX written (not accumulated) whose output tiles do not fill whole rounds
+    of the 74 CTA pairs: 128 tiles (a partial round of 54 pairs, more than two
+    thirds: no split), 120 tiles (pieces of a third and two thirds of the
+    reduction) and 96 tiles (halves) of 256 x 256.  The pieces add onto a zeroed
+    region, two addends per element, so repeated calls agree bit for bit; sampled
+    entries, and every entry of the last row and column, match the oracle."""
+    rng = np.random.default_rng(11)
+    N = 1024                          # the reduction: 16 k-blocks
+    dUb, Wb = _bf16(rng, (M, N)), _bf16(rng, (N, K), 0.1)
+    dUd, Wd = tl.to_dev_bf16(dUb), tl.to_dev_bf16(Wb)
+    Xd = tl.to_dev_bf16(_bf16(rng, (M, K)))
+    outs = []
+    for _ in range(3):
+        dX = torch.full((M, K), float("nan"), device="cuda")
+        sru.sru_project_backward(dUd, Xd, Wd, dX=dX, accumulate=False)
+        outs.append(dX)
+    assert sru.sru_sync_status() == 0
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    got = tl.host_f64(outs[0])
+    rows = np.concatenate([rng.integers(0, M, 2048), np.full(K, M - 1), np.arange(M - 256, M)])
+    cols = np.concatenate([rng.integers(0, K, 2048), np.arange(K), np.full(256, K - 1)])
+    ref = oracle.project_dX_entries(dUb, Wb, rows, cols)
+    absref = oracle.project_dX_entries(tl.abs_operand(dUb), tl.abs_operand(Wb), rows, cols)
+    tl.assert_close_sum("dX sampled", got[rows, cols], ref, absref)
