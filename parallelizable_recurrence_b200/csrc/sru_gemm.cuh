@@ -196,15 +196,12 @@ __device__ __forceinline__ PairUnit pair_unit(int u, int m_tiles, int n_tiles, i
 // the R tiles of the last, partial round are cut in two k-pieces, [0, s) and
 // [s, K), that both add onto an output region zeroed beforehand (0 + a + b
 // rounds the same in either order, so the result is deterministic):
-//   pair p < R              the piece [s, K) of tail tile p
-//   R <= p < 2R             the piece [0, s) of tail tile p - R
-//   and, when 2R > P, pair p with p - R < 2R - P also the piece [0, s) of tail
-//   tile (P - R) + (p - R).
-// The host takes s = K/2 when 2R <= P (every piece its own pair) and s = K/3
-// otherwise (some pairs take two short pieces): the tail then costs half or
-// two thirds of a round instead of a whole one.  The second case covers all R
-// tail tiles only while R - (P - R) <= P - R, i.e. R <= 2P/3; the host splits
-// no tail past that.
+//   pair p < R              the long piece [s, K) of tail tile p
+//   pair p >= R             the short pieces [0, s) of tail tiles
+//                           (p - R) + j (P - R), j = 0, 1, ..., below R
+// so each of the P - R pairs past R takes at most q = ceil(R / (P - R)) short
+// pieces.  The host takes s = K / (q + 1): the tail then costs q / (q + 1) of
+// a round instead of a whole one (a half for q = 1, two thirds for q = 2).
 template <int CAUSAL>
 __device__ __forceinline__ bool pair_next(int i, int p, int P, int units, int m_tiles, int n_tiles, int splits,
                                           int kblocks, int kper, int tail_s, PairUnit& w) {
@@ -219,15 +216,14 @@ __device__ __forceinline__ bool pair_next(int i, int p, int P, int units, int m_
     bool large = false;
     if (i < F) {
         tile = p + i * P;
-    } else if (i == F) {
-        if (p < R) {
+    } else if (p < R) {
+        if (i == F) {
             tile = F * P + p;
             large = true;
-        } else if (p - R < R) {
-            tile = F * P + (p - R);
         }
-    } else if (i == F + 1) {
-        if (p >= R && p - R < 2 * R - P) tile = F * P + (P - R) + (p - R);
+    } else {
+        const int t = (p - R) + (i - F) * (P - R);  // short piece j = i - F
+        if (t < R) tile = F * P + t;
     }
     if (tile < 0) return false;
     w.z = 0;
