@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kRowWarps * 32) sru_softmax_backward_rows_kern
 // (dS K up to the end of each row tile, dS^T Q from each row tile's diagonal
 // on) never read further.
 template <int NV>
-__global__ void __launch_bounds__(kRowWarps * 32, NV <= 8 ? 2 : 1) sru_softmax_backward_rows_reg_kernel(
+__global__ void __launch_bounds__(kRowWarps * 32, NV <= 8 ? 3 : 1) sru_softmax_backward_rows_reg_kernel(
     const float* __restrict__ dP, const __nv_bfloat16* __restrict__ P, __nv_bfloat16* __restrict__ dS, int L, int rows,
     float scale, int causal) {
     const int row = blockIdx.x * kRowWarps + threadIdx.x / 32, lane = threadIdx.x % 32;
